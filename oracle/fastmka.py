@@ -1,0 +1,340 @@
+"""FastMKA layer, restated step by step in float64 NumPy -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+legs use this module; the CUDA path shares no code with it.
+
+Sources (both pages are titled "MKA: Memory-Keyed Attention for Efficient
+Long-Context Reasoning"; "notes" is the paper-notes page, "abstract" the
+abstract-and-tables page):
+
+* notes §1 (三级分层记忆 table): L1 local = the current tokens, L2 session = a
+  causal prefix summary M2[t] = Summary(X[:, 1:t, :]) that uses past tokens only,
+  L3 long-term = recall of R << T past blocks through a vectorised hash index.
+* notes §2 (动态路由门): lambda = softmax(MLP(q)), shape [B, S, 3], per token.
+* notes §3 (FastMKA): X_fused = sum_l lambda_l * L_l; K, V = X_fused W_k, X_fused W_v;
+  then one standard causal attention over the fused K/V.
+* notes §4 (Block-MKA): online max-shift, running max mu, old partial sums
+  rescaled by exp(mu_prev - mu_new).
+* abstract page: FastMKA is "broadcast-routed" -- lambda is shared by every
+  channel and head.
+
+Readings where the pages leave a step open (the workload specification fixes
+the parameters): L2 is the EMA M2[t] = a*M2[t-1] + (1-a)*X[t-1], M2[0] = 0;
+L3 uses fixed blocks of b rows, summary = block mean of X, hash = signs of an
+nbits-wide projection P (bit k set iff (v P)_k > 0, bit k = projection k),
+block j is eligible at t iff (j+1)*b <= t, the R nearest by Hamming distance
+are recalled with ties going to the lowest block index, and
+M3[t] = mean of the recalled summaries (0 when none is eligible).  The router
+MLP has no biases and uses the exact-erf GELU.  Query heads map to KV groups
+contiguously, g(h) = h // (Hq / Hkv).  There is no positional encoding and no
+output projection (the per-head outputs are concatenated).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+from scipy.special import erfc
+
+# A recalled-index mismatch at token t is excused only if one of the hash
+# projections that decide it (the token's own, or an eligible block's) is
+# closer to zero than this.
+EXCUSE_EPS = 1e-4
+
+
+# ----------------------------------------------------------------------------- router
+def gelu_erf(x: np.ndarray) -> np.ndarray:
+    """GELU(x) = x * Phi(x) = 0.5 x (1 + erf(x / sqrt(2))) = 0.5 x erfc(-x / sqrt(2)).
+
+    The erfc form avoids the cancellation of 1 + erf(.) for large negative x.
+    """
+    return 0.5 * x * erfc(-x / math.sqrt(2.0))
+
+
+def softmax_rows(z: np.ndarray) -> np.ndarray:
+    """Softmax over the last axis (max subtracted first)."""
+    m = z.max(axis=-1, keepdims=True)
+    e = np.exp(z - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def router(q: np.ndarray, w_r1: np.ndarray, w_r2: np.ndarray) -> np.ndarray:
+    """Routing gate lambda = softmax(MLP(q)) over the three memory sources.
+
+    notes §2: one weight per token and source, shared by all heads.  MLP(q) =
+    GELU(q W_r1) W_r2.  q: [..., dq] -> lambda: [..., 3].
+    """
+    h = q @ w_r1
+    z = gelu_erf(h) @ w_r2
+    return softmax_rows(z)
+
+
+# ----------------------------------------------------------------------------- L2
+def session_ema(X: np.ndarray, alpha: float, m_init: Optional[np.ndarray] = None):
+    """L2 session memory as the causal EMA M2[t] = a*M2[t-1] + (1-a)*X[t-1].
+
+    notes §1: M2[t] summarises X[:, 1:t, :] only (no leakage of token t).
+    X: [B, S, d].  M2[0] = m_init (zeros by default).  Returns (M2, m_next) where
+    m_next = M2[S], the state a following token would read.
+    """
+    B, S, d = X.shape
+    M2 = np.zeros((B, S, d))
+    m = np.zeros((B, d)) if m_init is None else np.array(m_init, dtype=np.float64, copy=True)
+    for t in range(S):
+        M2[:, t] = m
+        m = alpha * m + (1.0 - alpha) * X[:, t]
+    return M2, m
+
+
+# ----------------------------------------------------------------------------- L3
+def block_summaries(X: np.ndarray, b: int) -> np.ndarray:
+    """Summary of block j = mean of rows [j*b, (j+1)*b) (full blocks only).  X: [B, S, d]."""
+    B, S, d = X.shape
+    n = S // b
+    return X[:, : n * b].reshape(B, n, b, d).mean(axis=2)
+
+
+def hash_codes(V: np.ndarray, P: np.ndarray):
+    """Sign-random-projection code: bit k = [(V P)_k > 0], bit k of a uint32 is projection k.
+
+    Returns (codes uint32 [...], projections float64 [..., nbits]).
+    """
+    p = V @ P
+    nb = P.shape[1]
+    bits = (p > 0).astype(np.uint64)
+    place = np.left_shift(np.uint64(1), np.arange(nb, dtype=np.uint64))
+    codes = (bits * place).sum(axis=-1).astype(np.uint32)
+    return codes, p
+
+
+def hamming(a, b) -> np.ndarray:
+    """Number of differing bits."""
+    return np.bitwise_count(np.bitwise_xor(np.asarray(a, np.uint32), np.asarray(b, np.uint32))).astype(np.int64)
+
+
+def recall_select(code_t: int, summary_codes: np.ndarray, n_eligible: int, R: int) -> np.ndarray:
+    """Indices of the R nearest eligible blocks, ordered by (Hamming distance, block index)."""
+    if n_eligible <= 0:
+        return np.zeros(0, dtype=np.int64)
+    dist = hamming(code_t, summary_codes[:n_eligible])
+    order = np.lexsort((np.arange(n_eligible), dist))  # last key is primary: distance, then index
+    return order[:R].astype(np.int64)
+
+
+def longterm_recall(x_rows: np.ndarray, positions: np.ndarray, summaries: np.ndarray, P: np.ndarray,
+                    b: int, R: int, summary_proj: Optional[np.ndarray] = None):
+    """L3 long-term memory for the rows of ONE sequence.
+
+    x_rows [n, d] are the raw tokens at `positions` [n]; summaries [nblk, d] the
+    block means of the whole sequence.  Block j is eligible at t iff (j+1)*b <= t.
+    Returns (idx [n, R] with -1 padding, count [n], M3 [n, d], excuse [n], x_codes [n], x_proj [n, nb]).
+    """
+    n, d = x_rows.shape
+    s_codes, s_proj = hash_codes(summaries, P)
+    if summary_proj is not None:
+        s_proj = summary_proj
+    x_codes, x_proj = hash_codes(x_rows, P)
+    idx = np.full((n, R), -1, dtype=np.int64)
+    count = np.zeros(n, dtype=np.int64)
+    M3 = np.zeros((n, d))
+    excuse = np.zeros(n, dtype=bool)
+    near_zero_block = (np.abs(s_proj) < EXCUSE_EPS).any(axis=-1) if len(summaries) else np.zeros(0, bool)
+    for i, t in enumerate(positions):
+        n_elig = min(int(t) // b, len(summaries))
+        sel = recall_select(int(x_codes[i]), s_codes, n_elig, R)
+        idx[i, : len(sel)] = sel
+        count[i] = len(sel)
+        if len(sel):
+            M3[i] = summaries[sel].mean(axis=0)
+        excuse[i] = bool((np.abs(x_proj[i]) < EXCUSE_EPS).any() or near_zero_block[:n_elig].any())
+    return idx, count, M3, excuse, x_codes, x_proj
+
+
+# ----------------------------------------------------------------------------- fuse + K/V
+def fuse_sources(lam: np.ndarray, L1: np.ndarray, L2: np.ndarray, L3: np.ndarray) -> np.ndarray:
+    """notes §3: X_fused = sum_l lambda_l * L_l, lambda broadcast over channels."""
+    return lam[..., 0:1] * L1 + lam[..., 1:2] * L2 + lam[..., 2:3] * L3
+
+
+def kv_project(X_fused: np.ndarray, w_k: np.ndarray, w_v: np.ndarray):
+    """notes §3: K = X_fused W_k, V = X_fused W_v."""
+    return X_fused @ w_k, X_fused @ w_v
+
+
+# ----------------------------------------------------------------------------- attention
+def causal_gqa_attention(q_rows: np.ndarray, positions: np.ndarray, K: np.ndarray, V: np.ndarray,
+                         n_kv_heads: int, scale: float, row_chunk: int = 64) -> np.ndarray:
+    """One causal attention over the fused K/V of ONE sequence (notes §3), two-pass softmax.
+
+    O[t, h] = sum_{j <= t} softmax_j(scale * q[t,h] . K[j,g(h)]) V[j,g(h)], g(h) = h // (Hq/Hkv).
+    q_rows [n, Hq, dh] at `positions` [n]; K, V [S, Hkv, dh].  Returns [n, Hq, dh].
+    """
+    n, Hq, dh = q_rows.shape
+    G = Hq // n_kv_heads
+    out = np.zeros((n, Hq, dh))
+    for r0 in range(0, n, row_chunk):
+        pos = positions[r0:r0 + row_chunk]
+        tmax = int(pos.max()) + 1
+        mask = np.arange(tmax)[None, :] > pos[:, None]          # [rows, j]: future keys
+        for g in range(n_kv_heads):
+            qg = q_rows[r0:r0 + row_chunk, g * G:(g + 1) * G]  # [rows, G, dh]
+            s = np.einsum("rhd,jd->rhj", qg, K[:tmax, g]) * scale
+            s[np.broadcast_to(mask[:, None, :], s.shape)] = -np.inf
+            m = s.max(axis=-1, keepdims=True)                   # pass 1: row maximum
+            p = np.exp(s - m)                                   # pass 2: weights
+            out[r0:r0 + row_chunk, g * G:(g + 1) * G] = (
+                np.einsum("rhj,jd->rhd", p, V[:tmax, g]) / p.sum(axis=-1, keepdims=True))
+    return out
+
+
+def online_softmax_attend(s: np.ndarray, Vt: np.ndarray, tile: int) -> np.ndarray:
+    """notes §4: softmax(s) @ Vt with the online max-shift over tiles of `tile` keys.
+
+    Keeps a running maximum mu; on each new tile the old partial sum and output
+    are rescaled by exp(mu_prev - mu_new).  s: [n_keys]; Vt: [n_keys, dv].
+    """
+    mu = -np.inf
+    l = 0.0
+    o = np.zeros(Vt.shape[1])
+    for k0 in range(0, len(s), tile):
+        st = s[k0:k0 + tile]
+        mu_new = max(mu, float(st.max()))
+        corr = math.exp(mu - mu_new) if mu != -np.inf else 0.0
+        e = np.exp(st - mu_new)
+        l = l * corr + e.sum()
+        o = o * corr + e @ Vt[k0:k0 + tile]
+        mu = mu_new
+    return o / l
+
+
+# ----------------------------------------------------------------------------- whole layer
+@dataclasses.dataclass
+class Weights64:
+    w_q: np.ndarray
+    w_k: np.ndarray
+    w_v: np.ndarray
+    w_r1: np.ndarray
+    w_r2: np.ndarray
+    P: np.ndarray
+
+
+def weights_f64(w_q, w_k, w_v, w_r1, w_r2, P) -> Weights64:
+    f = lambda a: np.asarray(a, dtype=np.float64)
+    return Weights64(f(w_q), f(w_k), f(w_v), f(w_r1), f(w_r2), f(P))
+
+
+def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray] = None,
+                    lam_override: Optional[np.ndarray] = None, row_chunk: int = 8192,
+                    keep_d_space: bool = False) -> dict:
+    """The FastMKA layer forward over whole sequences, in page order.
+
+    X: [B, S, d] (any float dtype; widened to float64 a chunk of rows at a time).
+    cfg supplies n_q_heads, n_kv_heads, d_head, alpha, block, recall_r, scale.
+    Steps per sequence: q = X W_q; lambda = router(q); M2 = EMA(X); M3 = L3
+    recall; X_fused = lambda-weighted sum of (X, M2, M3); K, V projections;
+    causal GQA attention on the query rows `rows` (all rows when None).
+    Rows are processed in chunks only to bound memory; the EMA state is carried
+    across chunks, so every value is the one the unchunked recurrence gives.
+    """
+    B, S, d = X.shape
+    Hq, Hkv, dh = cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head
+    b, R = cfg.block, cfg.recall_r
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    nblk = S // b
+    out = {
+        "rows": rows,
+        "lam": np.zeros((B, S, 3)),
+        "idx": np.full((B, S, R), -1, np.int64),
+        "count": np.zeros((B, S), np.int64),
+        "excuse": np.zeros((B, S), bool),
+        "x_codes": np.zeros((B, S), np.uint32),
+        "x_proj": np.zeros((B, S, w.P.shape[1])),
+        "summary_codes": np.zeros((B, nblk), np.uint32),
+        "summary_proj": np.zeros((B, nblk, w.P.shape[1])),
+        "K": np.zeros((B, S, Hkv, dh)),
+        "V": np.zeros((B, S, Hkv, dh)),
+        "q": np.zeros((B, len(rows), Hq, dh)),
+        "O": np.zeros((B, len(rows), Hq * dh)),
+        "m2_next": np.zeros((B, d)),
+    }
+    if keep_d_space:
+        for k in ("M2", "M3", "X_fused"):
+            out[k] = np.zeros((B, S, d))
+    for bi in range(B):
+        # L3 block summaries need the whole sequence's full blocks.
+        summ = np.zeros((nblk, d))
+        for j0 in range(0, nblk, max(1, row_chunk // b)):
+            j1 = min(nblk, j0 + max(1, row_chunk // b))
+            summ[j0:j1] = block_summaries(np.asarray(X[bi:bi + 1, j0 * b:j1 * b], np.float64), b)[0]
+        s_codes, s_proj = hash_codes(summ, w.P)
+        out["summary_codes"][bi], out["summary_proj"][bi] = s_codes, s_proj
+        m2 = np.zeros((1, d))
+        for r0 in range(0, S, row_chunk):
+            r1 = min(S, r0 + row_chunk)
+            xc = np.asarray(X[bi:bi + 1, r0:r1], np.float64)          # [1, n, d]
+            qc = xc[0] @ w.w_q                                          # q = X W_q
+            lam = router(qc, w.w_r1, w.w_r2) if lam_override is None else np.broadcast_to(
+                np.asarray(lam_override, np.float64), (r1 - r0, 3))
+            M2, m2 = session_ema(xc, cfg.alpha, m2)
+            pos = np.arange(r0, r1)
+            idx, cnt, M3, exc, xcodes, xproj = longterm_recall(xc[0], pos, summ, w.P, b, R, s_proj)
+            Xf = fuse_sources(lam, xc[0], M2[0], M3)
+            Kc, Vc = kv_project(Xf, w.w_k, w.w_v)
+            out["lam"][bi, r0:r1] = lam
+            out["idx"][bi, r0:r1], out["count"][bi, r0:r1], out["excuse"][bi, r0:r1] = idx, cnt, exc
+            out["x_codes"][bi, r0:r1], out["x_proj"][bi, r0:r1] = xcodes, xproj
+            out["K"][bi, r0:r1] = Kc.reshape(-1, Hkv, dh)
+            out["V"][bi, r0:r1] = Vc.reshape(-1, Hkv, dh)
+            sel = (rows >= r0) & (rows < r1)
+            out["q"][bi, sel] = qc[rows[sel] - r0].reshape(-1, Hq, dh)
+            if keep_d_space:
+                out["M2"][bi, r0:r1], out["M3"][bi, r0:r1], out["X_fused"][bi, r0:r1] = M2[0], M3, Xf
+        out["m2_next"][bi] = m2[0]
+        O = causal_gqa_attention(out["q"][bi], rows, out["K"][bi], out["V"][bi], Hkv, cfg.scale)
+        out["O"][bi] = O.reshape(len(rows), Hq * dh)
+    return out
+
+
+def fastmka_decode(X: np.ndarray, w: Weights64, cfg) -> np.ndarray:
+    """Token-at-a-time FastMKA, carrying the decode state.  Returns O [B, S, Hq*dh].
+
+    State per sequence: the fused K/V cache, the EMA value M2 for the next
+    token, the running sum of the unfinished block, and the finished block
+    summaries with their codes.  Token t reads the state, appends its fused
+    K/V, attends over cache[0..t], then advances the EMA and, when it closes a
+    block ((t+1) % b == 0), finalises that block's summary and code.  A block is
+    therefore visible exactly from t = (j+1)*b on, the strictly-past rule.
+    """
+    B, S, d = X.shape
+    Hq, Hkv, dh = cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head
+    b, R = cfg.block, cfg.recall_r
+    O = np.zeros((B, S, Hq * dh))
+    for bi in range(B):
+        Kc = np.zeros((S, Hkv, dh))
+        Vc = np.zeros((S, Hkv, dh))
+        m2 = np.zeros(d)
+        block_sum = np.zeros(d)
+        summaries, codes = [], []
+        for t in range(S):
+            x = np.asarray(X[bi, t], np.float64)
+            q = x @ w.w_q
+            lam = router(q[None], w.w_r1, w.w_r2)[0]
+            code_t, _ = hash_codes(x[None], w.P)
+            s_arr = np.array(summaries).reshape(-1, d)
+            sel = recall_select(int(code_t[0]), np.array(codes, np.uint32), len(summaries), R)
+            M3 = s_arr[sel].mean(axis=0) if len(sel) else np.zeros(d)
+            xf = fuse_sources(lam[None], x[None], m2[None], M3[None])
+            k, v = kv_project(xf, w.w_k, w.w_v)
+            Kc[t], Vc[t] = k.reshape(Hkv, dh), v.reshape(Hkv, dh)
+            o = causal_gqa_attention(q.reshape(1, Hq, dh), np.array([t]), Kc[: t + 1], Vc[: t + 1], Hkv, cfg.scale)
+            O[bi, t] = o.reshape(-1)
+            m2 = cfg.alpha * m2 + (1.0 - cfg.alpha) * x
+            block_sum = block_sum + x
+            if (t + 1) % b == 0:
+                s_new = block_sum / b
+                summaries.append(s_new)
+                codes.append(int(hash_codes(s_new[None], w.P)[0][0]))
+                block_sum = np.zeros(d)
+    return O

@@ -1,0 +1,429 @@
+"""Pins for the CPU oracle: facts the pages and mathematics fix, checked without the oracle's own code path.
+
+Every pin is written as a `check_*` function that takes the oracle function
+under test, so the mutation tests at the bottom can plant plausible mistakes in
+copies of the oracle (on the CPU) and show that some pin fails for each.
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.stats
+import torch
+
+import oracle
+from oracle import fastmka as O
+from fastmka_inputs import CONFIGS, FastMKAConfig, make_inputs, to_f64
+
+RNG = np.random.default_rng(1234)
+
+
+def tiny_cfg(**kw) -> FastMKAConfig:
+    base = FastMKAConfig("pin", 2, 40, 12, 4, 2, 3, 5, 0.7, 4, 3, 4, "f32", 99)
+    return base.replace(**kw)
+
+
+def tiny_weights(cfg, rng):
+    d, dq, dkv, rh, nb = cfg.d_model, cfg.dq, cfg.dkv, cfg.router_hidden, cfg.hash_bits
+    return O.weights_f64(rng.standard_normal((d, dq)) / math.sqrt(d), rng.standard_normal((d, dkv)) / math.sqrt(d),
+                         rng.standard_normal((d, dkv)) / math.sqrt(d), rng.standard_normal((dq, rh)) / math.sqrt(dq),
+                         rng.standard_normal((rh, 3)) / math.sqrt(rh), rng.standard_normal((d, nb)))
+
+
+# ============================================================================ router (notes §2)
+def check_router_rows(router_fn):
+    q = RNG.standard_normal((50, 8))
+    lam = router_fn(q, RNG.standard_normal((8, 6)), RNG.standard_normal((6, 3)))
+    assert lam.shape == (50, 3)
+    assert np.all(lam > 0)
+    np.testing.assert_allclose(lam.sum(-1), 1.0, rtol=0, atol=1e-15)
+
+
+def check_router_closed_form(router_fn):
+    # W_r1 = W_r2 = I and h = 10 + [0, ln 2, ln 4]: GELU(h) = h exactly in float64
+    # (1 - Phi(10) ~ 7.6e-24), so lambda = softmax(h) = (1, 2, 4) / 7.
+    h = 10.0 + np.log(np.array([1.0, 2.0, 4.0]))
+    lam = router_fn(h[None], np.eye(3), np.eye(3))[0]
+    np.testing.assert_allclose(lam, np.array([1.0, 2.0, 4.0]) / 7.0, rtol=1e-14)
+    # A zero first layer gives GELU(0) = 0, hence equal gates.
+    lam0 = router_fn(RNG.standard_normal((4, 5)), np.zeros((5, 7)), RNG.standard_normal((7, 3)))
+    np.testing.assert_allclose(lam0, 1.0 / 3.0, rtol=1e-15)
+    # Only the second column of W_r2 sees positive inputs -> lambda_2 dominates.
+    lam1 = router_fn(np.full((1, 2), 20.0), np.eye(2), np.array([[0.0, 5.0, -5.0], [0.0, 5.0, -5.0]]))[0]
+    # GELU(20) = 20, z = (0, 200, -200): lambda = (e^-200, 1, e^-400) / (1 + e^-200 + e^-400).
+    np.testing.assert_allclose(lam1, [math.exp(-200), 1.0, math.exp(-400)], rtol=1e-13)
+    # h = (-1, 0, 1): GELU(h) = (-Phi(-1), 0, Phi(1)) with the textbook normal-table values.
+    lam2 = router_fn(np.array([[-1.0, 0.0, 1.0]]), np.eye(3), np.eye(3))[0]
+    e = [math.exp(-0.15865525393145707), 1.0, math.exp(0.8413447460685429)]
+    np.testing.assert_allclose(lam2, np.array(e) / sum(e), rtol=1e-14)
+
+
+def test_router_rows_sum_to_one():
+    check_router_rows(O.router)
+
+
+def test_router_closed_form():
+    check_router_closed_form(O.router)
+
+
+def test_gelu_is_x_times_normal_cdf():
+    x = np.linspace(-6, 6, 101)
+    np.testing.assert_allclose(O.gelu_erf(x), x * scipy.stats.norm.cdf(x), rtol=1e-13, atol=1e-300)
+    # Textbook: Phi(1) = 0.8413447460685429, Phi(-1) = 0.15865525393145707.
+    np.testing.assert_allclose(O.gelu_erf(np.array([1.0, -1.0])), [0.8413447460685429, -0.15865525393145707],
+                               rtol=1e-15)
+
+
+# ============================================================================ L2 session EMA
+def check_ema_closed_form(ema_fn):
+    for alpha in (0.0, 0.5, 0.9, 0.999):
+        X = RNG.standard_normal((2, 17, 3))
+        M2, m_next = ema_fn(X, alpha)
+        ref = np.zeros_like(X)
+        for t in range(X.shape[1]):
+            for k in range(t):
+                ref[:, t] += alpha ** k * (1 - alpha) * X[:, t - 1 - k]
+        np.testing.assert_allclose(M2, ref, rtol=1e-12, atol=1e-14)
+        nxt = sum(alpha ** k * (1 - alpha) * X[:, X.shape[1] - 1 - k] for k in range(X.shape[1]))
+        np.testing.assert_allclose(m_next, nxt, rtol=1e-12, atol=1e-14)
+    # alpha = 0: a pure one-step shift; M2[0] = 0.
+    X = RNG.standard_normal((1, 9, 4))
+    M2, _ = ema_fn(X, 0.0)
+    np.testing.assert_array_equal(M2[:, 1:], X[:, :-1])
+    np.testing.assert_array_equal(M2[:, 0], 0.0)
+
+
+def check_ema_carry(ema_fn):
+    # Splitting a sequence and carrying the state gives the unsplit result.
+    X = RNG.standard_normal((2, 30, 5))
+    full, m_full = ema_fn(X, 0.8)
+    a, m_a = ema_fn(X[:, :11], 0.8)
+    b, m_b = ema_fn(X[:, 11:], 0.8, m_a)
+    np.testing.assert_allclose(np.concatenate([a, b], 1), full, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(m_b, m_full, rtol=1e-14)
+
+
+def test_ema_closed_form():
+    check_ema_closed_form(O.session_ema)
+
+
+def test_ema_carry():
+    check_ema_carry(O.session_ema)
+
+
+# ============================================================================ L3 recall
+def brute_summaries(X1, b):
+    S, d = X1.shape
+    out = []
+    for j in range(S // b):
+        acc = np.zeros(d)
+        for r in range(j * b, (j + 1) * b):
+            acc += X1[r]
+        out.append(acc / b)
+    return np.array(out).reshape(-1, d)
+
+
+def brute_code(v, P):
+    code = 0
+    for k in range(P.shape[1]):
+        if float(sum(v[i] * P[i, k] for i in range(len(v)))) > 0:
+            code |= 1 << k
+    return code
+
+
+def check_recall_brute_force(recall_fn, b=4, R=3, nb=4, S=60, d=5, seed=7):
+    rng = np.random.default_rng(seed)
+    X1 = rng.standard_normal((S, d))
+    P = rng.standard_normal((d, nb))
+    summ = brute_summaries(X1, b)
+    idx, count, M3, excuse, xcodes, _ = recall_fn(X1, np.arange(S), summ, P, b, R)
+    scodes = [brute_code(s, P) for s in summ]
+    for t in range(S):
+        xc = brute_code(X1[t], P)
+        assert int(xcodes[t]) == xc
+        eligible = [j for j in range(len(summ)) if (j + 1) * b <= t]   # strictly past, full blocks
+        assert count[t] == min(R, len(eligible))
+        sel = [int(j) for j in idx[t, : count[t]]]
+        assert all(j == -1 for j in idx[t, count[t]:])
+        key = {j: (bin(xc ^ scodes[j]).count("1"), j) for j in eligible}
+        assert set(sel) <= set(eligible) and len(set(sel)) == len(sel)
+        # Every recalled block beats every block left out, in (distance, index) order.
+        for js in sel:
+            for ju in set(eligible) - set(sel):
+                assert key[js] < key[ju]
+        assert [key[j] for j in sel] == sorted(key[j] for j in sel)
+        ref = np.mean([summ[j] for j in sel], axis=0) if sel else np.zeros(d)
+        np.testing.assert_allclose(M3[t], ref, rtol=1e-14, atol=1e-15)
+
+
+def test_recall_brute_force_heavy_ties():
+    check_recall_brute_force(O.longterm_recall)                      # 4-bit codes: ties everywhere
+    check_recall_brute_force(O.longterm_recall, b=3, R=5, nb=7, S=50, seed=3)
+
+
+def test_recall_special_cases():
+    rng = np.random.default_rng(11)
+    X1 = rng.standard_normal((40, 6))
+    P = rng.standard_normal((6, 8))
+    b = 8
+    summ = O.block_summaries(X1[None], b)[0]
+    # M3 == 0 and no index for t < b.
+    idx, count, M3, *_ = O.longterm_recall(X1, np.arange(40), summ, P, b, 2)
+    assert np.all(count[:b] == 0) and np.all(M3[:b] == 0) and np.all(idx[:b] == -1)
+    # R >= number of eligible blocks: M3 is the mean of all eligible summaries, whatever the codes.
+    idx, count, M3, *_ = O.longterm_recall(X1, np.arange(40), summ, P, b, 100)
+    for t in range(40):
+        n = t // b
+        ref = summ[:n].mean(0) if n else np.zeros(6)
+        np.testing.assert_allclose(M3[t], ref, rtol=1e-14, atol=1e-15)
+    # b >= S: nothing is ever eligible.
+    summ_big = O.block_summaries(X1[None], 64)[0]
+    _, count, M3, *_ = O.longterm_recall(X1, np.arange(40), summ_big, P, 64, 2)
+    assert np.all(count == 0) and np.all(M3 == 0)
+
+
+def test_hash_bit_order_and_zero():
+    P = np.eye(5)
+    v = np.array([[1.0, -1.0, 0.0, 2.0, -0.5]])
+    codes, p = O.hash_codes(v, P)
+    assert int(codes[0]) == (1 << 0) | (1 << 3)        # p = 0 gives bit 0
+    assert O.hamming(0b1011, 0b0110) == 3
+
+
+# ============================================================================ attention
+def brute_causal_gqa(q, K, V, Hkv, scale):
+    """Explicit S x S masked score matrix per head."""
+    S, Hq, dh = q.shape
+    G = Hq // Hkv
+    out = np.zeros_like(q)
+    for h in range(Hq):
+        g = h // G
+        sc = np.full((S, S), -np.inf)
+        for t in range(S):
+            for j in range(t + 1):
+                sc[t, j] = scale * float(np.dot(q[t, h], K[j, g]))
+        w = np.exp(sc - sc.max(1, keepdims=True))
+        w /= w.sum(1, keepdims=True)
+        out[:, h] = w @ V[:, g]
+    return out
+
+
+def check_attention_brute(attn_fn, S=23, Hq=6, Hkv=2, dh=4):
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((S, Hq, dh)) * 2
+    K = rng.standard_normal((S, Hkv, dh))
+    V = rng.standard_normal((S, Hkv, dh))
+    got = attn_fn(q, np.arange(S), K, V, Hkv, 0.37, row_chunk=5)
+    np.testing.assert_allclose(got, brute_causal_gqa(q, K, V, Hkv, 0.37), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_brute_force():
+    check_attention_brute(O.causal_gqa_attention)
+    check_attention_brute(O.causal_gqa_attention, S=9, Hq=3, Hkv=3, dh=5)    # Hq = Hkv: plain MHA
+
+
+def test_attention_matches_torch_sdpa():
+    rng = np.random.default_rng(8)
+    S, Hq, Hkv, dh = 31, 8, 2, 16
+    q, K, V = rng.standard_normal((S, Hq, dh)), rng.standard_normal((S, Hkv, dh)), rng.standard_normal((S, Hkv, dh))
+    got = O.causal_gqa_attention(q, np.arange(S), K, V, Hkv, 1 / 4)
+    tq = torch.from_numpy(q).permute(1, 0, 2)[None]
+    tk = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)[None]
+    tv = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=0.25)
+    np.testing.assert_allclose(got, ref[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("tile", [1, 7, 64])
+def test_online_max_shift_equals_two_pass(tile):
+    rng = np.random.default_rng(tile)
+    for scale in (1.0, 30.0):                      # large scores force many max updates
+        s = rng.standard_normal(150) * scale + np.linspace(-20, 20, 150)
+        Vt = rng.standard_normal((150, 6))
+        w = np.exp(s - s.max())
+        np.testing.assert_allclose(O.online_softmax_attend(s, Vt, tile), (w / w.sum()) @ Vt, rtol=1e-12, atol=1e-14)
+
+
+# ============================================================================ whole layer
+def _run(cfg, X, w, **kw):
+    return O.fastmka_prefill(X, w, cfg, **kw)
+
+
+def test_layer_lambda_one_is_standard_causal_attention():
+    """lambda = (1,0,0) ("L1 only (=MHA)" in the abstract page's Table 9) is textbook causal GQA."""
+    cfg = tiny_cfg()
+    w = tiny_weights(cfg, np.random.default_rng(2))
+    X = np.random.default_rng(3).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    out = _run(cfg, X, w, lam_override=[1.0, 0.0, 0.0])
+    for bi in range(cfg.batch):
+        q = (X[bi] @ w.w_q).reshape(cfg.seq, cfg.n_q_heads, cfg.d_head)
+        K = (X[bi] @ w.w_k).reshape(cfg.seq, cfg.n_kv_heads, cfg.d_head)
+        V = (X[bi] @ w.w_v).reshape(cfg.seq, cfg.n_kv_heads, cfg.d_head)
+        ref = brute_causal_gqa(q, K, V, cfg.n_kv_heads, cfg.scale)
+        np.testing.assert_allclose(out["O"][bi].reshape(ref.shape), ref, rtol=1e-11, atol=1e-12)
+
+
+def test_layer_sources_enter_as_defined():
+    """lambda = e_2 or e_3 routes the EMA or the recalled mean alone into K/V."""
+    cfg = tiny_cfg()
+    w = tiny_weights(cfg, np.random.default_rng(4))
+    X = np.random.default_rng(5).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    o2 = _run(cfg, X, w, lam_override=[0.0, 1.0, 0.0], keep_d_space=True)
+    M2, _ = O.session_ema(X, cfg.alpha)
+    np.testing.assert_allclose(o2["K"].reshape(cfg.batch, cfg.seq, -1), M2 @ w.w_k, rtol=1e-12, atol=1e-13)
+    o3 = _run(cfg, X, w, lam_override=[0.0, 0.0, 1.0], keep_d_space=True)
+    np.testing.assert_allclose(o3["V"].reshape(cfg.batch, cfg.seq, -1), o3["M3"] @ w.w_v, rtol=1e-12, atol=1e-13)
+
+
+def test_layer_first_row_and_lambda_sum():
+    cfg = tiny_cfg()
+    w = tiny_weights(cfg, np.random.default_rng(6))
+    X = np.random.default_rng(7).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    out = _run(cfg, X, w)
+    np.testing.assert_allclose(out["lam"].sum(-1), 1.0, atol=1e-15)
+    G = cfg.n_q_heads // cfg.n_kv_heads
+    for bi in range(cfg.batch):
+        V0 = out["lam"][bi, 0, 0] * (X[bi, 0] @ w.w_v)       # M2[0] = M3[0] = 0
+        O0 = out["O"][bi, 0].reshape(cfg.n_q_heads, cfg.d_head)
+        for h in range(cfg.n_q_heads):
+            np.testing.assert_allclose(O0[h], V0.reshape(cfg.n_kv_heads, cfg.d_head)[h // G], rtol=1e-13)
+
+
+def test_layer_causality_under_future_perturbation():
+    cfg = tiny_cfg(seq=48)
+    w = tiny_weights(cfg, np.random.default_rng(8))
+    X = np.random.default_rng(9).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    base = _run(cfg, X, w)
+    for t0 in (0, 5, 17, 31, 46):
+        Xp = X.copy()
+        Xp[:, t0 + 1:] = np.random.default_rng(t0).standard_normal(Xp[:, t0 + 1:].shape) * 3
+        pert = _run(cfg, Xp, w)
+        np.testing.assert_allclose(pert["O"][:, : t0 + 1], base["O"][:, : t0 + 1], rtol=1e-12, atol=1e-13)
+        np.testing.assert_array_equal(pert["idx"][:, : t0 + 1], base["idx"][:, : t0 + 1])
+
+
+def test_decode_equals_prefill_rows():
+    cfg = tiny_cfg(seq=37)
+    w = tiny_weights(cfg, np.random.default_rng(10))
+    X = np.random.default_rng(11).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    pre = _run(cfg, X, w)
+    dec = O.fastmka_decode(X, w, cfg)
+    np.testing.assert_allclose(dec, pre["O"], rtol=1e-11, atol=1e-12)
+
+
+def test_chunked_rows_equal_unchunked():
+    cfg = tiny_cfg(seq=40)
+    w = tiny_weights(cfg, np.random.default_rng(12))
+    X = np.random.default_rng(13).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    a = _run(cfg, X, w)
+    b = _run(cfg, X, w, row_chunk=7, rows=np.array([0, 3, 8, 9, 39]))
+    np.testing.assert_allclose(b["O"], a["O"][:, [0, 3, 8, 9, 39]], rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(b["idx"], a["idx"])
+    np.testing.assert_allclose(b["K"], a["K"], rtol=1e-12, atol=1e-13)
+
+
+def test_tiny_workload_runs():
+    cfg = CONFIGS["tiny_f32"]
+    inp = make_inputs(cfg)
+    w = O.weights_f64(*(to_f64(t) for t in (inp.w_q, inp.w_k, inp.w_v, inp.w_r1, inp.w_r2, inp.hash_proj)))
+    out = _run(cfg, to_f64(inp.x), w)
+    assert np.isfinite(out["O"]).all()
+    np.testing.assert_allclose(out["lam"].sum(-1), 1.0, atol=1e-15)
+    assert out["count"][0, cfg.block] == 1 and out["count"][0, -1] == cfg.recall_r
+
+
+# ============================================================================ planted mistakes
+def _mut_ema_reads_current(X, alpha, m_init=None):
+    B, S, d = X.shape
+    M2 = np.zeros((B, S, d))
+    m = np.zeros((B, d)) if m_init is None else m_init.copy()
+    for t in range(S):
+        m = alpha * m + (1 - alpha) * X[:, t]       # leaks token t into its own summary
+        M2[:, t] = m
+    return M2, m
+
+
+def _mut_ema_swapped_weights(X, alpha, m_init=None):
+    return O.session_ema(X, 1.0 - alpha, m_init)
+
+
+def _mut_router_no_gelu(q, w_r1, w_r2):
+    return O.softmax_rows((q @ w_r1) @ w_r2)
+
+
+def _mut_router_softmax_axis(q, w_r1, w_r2):
+    z = O.gelu_erf(q @ w_r1) @ w_r2
+    e = np.exp(z - z.max(0, keepdims=True))
+    return e / e.sum(0, keepdims=True)
+
+
+def _mut_recall_factory(kind):
+    def select(code_t, summary_codes, n_eligible, R):
+        if kind == "eligible_off_by_one":
+            n_eligible = min(n_eligible + 1, len(summary_codes))
+        if n_eligible <= 0:
+            return np.zeros(0, np.int64)
+        dist = O.hamming(code_t, summary_codes[:n_eligible])
+        if kind == "tie_high_index":
+            order = np.lexsort((-np.arange(n_eligible), dist))
+        elif kind == "farthest":
+            order = np.lexsort((np.arange(n_eligible), -dist))
+        else:
+            order = np.lexsort((np.arange(n_eligible), dist))
+        return order[:R]
+    return select
+
+
+def _mut_attention_factory(kind):
+    def attn(q_rows, positions, K, V, n_kv_heads, scale, row_chunk=64):
+        n, Hq, dh = q_rows.shape
+        G = Hq // n_kv_heads
+        out = np.zeros((n, Hq, dh))
+        for i, t in enumerate(positions):
+            for h in range(Hq):
+                g = h % n_kv_heads if kind == "gqa_interleaved" else h // G
+                hi = t if kind == "exclusive_mask" and t > 0 else t + 1
+                s = K[:hi, g] @ q_rows[i, h] * scale
+                p = np.exp(s - s.max())
+                out[i, h] = p @ V[:hi, g] / p.sum()
+        return out
+    return attn
+
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    for bad in (_mut_ema_reads_current, _mut_ema_swapped_weights):
+        with pytest.raises(AssertionError):
+            check_ema_closed_form(bad)
+    for bad in (_mut_router_no_gelu, _mut_router_softmax_axis):
+        with pytest.raises(AssertionError):
+            check_router_rows(bad)
+            check_router_closed_form(bad)
+    for kind in ("eligible_off_by_one", "tie_high_index", "farthest"):
+        with monkeypatch.context() as m:
+            m.setattr(O, "recall_select", _mut_recall_factory(kind))
+            with pytest.raises(AssertionError):
+                check_recall_brute_force(O.longterm_recall)
+    for kind in ("exclusive_mask", "gqa_interleaved"):
+        with pytest.raises(AssertionError):
+            check_attention_brute(_mut_attention_factory(kind))
+    # The unplanted copy of the attention mutant passes, so the failures above are the mistakes'.
+    check_attention_brute(_mut_attention_factory("none"))
+
+
+# ============================================================================ regression snapshot
+def test_golden_snapshot_unchanged():
+    """tests/golden/tiny_f32_oracle.json (written by tests/golden/make_golden.py from the oracle) still holds."""
+    import importlib.util
+    import json
+    import os
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location("make_golden", os.path.join(here, "make_golden.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    with open(os.path.join(here, "tiny_f32_oracle.json")) as f:
+        stored = json.load(f)
+    now = mod.compute()
+    assert now["idx"] == stored["idx"] and now["x_codes"] == stored["x_codes"]
+    assert now["summary_codes"] == stored["summary_codes"]
+    for k in ("lam", "O_row_sums", "O_first8"):
+        np.testing.assert_allclose(np.array(now[k]), np.array(stored[k]), rtol=1e-12, atol=1e-13)
