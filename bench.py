@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""FastMKA layer benchmark on B200.
+
+Headline: prefill tokens/s of the Qwen2.5-7B-shaped FastMKA layer (batch 2 x
+seq 4096, bf16; every step runs the whole layer: projections, router, L2 EMA,
+L3 hash recall, route-fuse, causal GQA attention).  Also reported: decode
+us/token over a 131072-position fused cache (256 steps in one CUDA graph), the
+roofline fraction of the dominant kernel (measured live with CUDA events on the
+launching stream), the end-to-end rate through host buffers, and the CPU oracle.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs an independent replica
+of the workload (the layer shards by sequence with no exchange): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fastmka_inputs import CONFIGS, make_inputs, sample_rows, to_f64  # noqa: E402
+
+REASON_BITS = {  # nvidia-smi clocks_event_reasons bitmask
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+PREFILL_STAGES = ["projection_gemm", "router_tail", "token_codes", "block_sums", "block_codes", "ema_carry", "recall",
+                  "route_fuse", "attention", "state_tail"]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if not getattr(self, "out", ""):
+            return None
+        sm, mx, reasons, power = [], [], 0, []
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 5:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                power.append(float(f[3]))
+                reasons |= int(f[4], 16)
+            except ValueError:
+                continue
+        if not sm:
+            return None
+        loaded = [s for s, p in zip(sm, power) if p > 200.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "samples": len(sm),
+                "power_w_max": max(power), "reasons": [n for b, n in REASON_BITS.items() if reasons & b]}
+
+
+# ------------------------------------------------------------------ workload arithmetic
+def prefill_flops(cfg) -> dict:
+    T, d, dq, dkv, rh, nb = cfg.tokens, cfg.d_model, cfg.dq, cfg.dkv, cfg.router_hidden, cfg.hash_bits
+    causal_pairs = cfg.batch * cfg.seq * (cfg.seq + 1) / 2
+    return {
+        "projections": 2.0 * T * d * (dq + 2 * dkv + 2 * rh + nb),
+        "attention": 4.0 * cfg.d_head * cfg.n_q_heads * causal_pairs,  # QK^T and PV over j <= t only
+    }
+
+
+def decode_bytes_per_token(cfg, ctx: int, ntot: int) -> float:
+    w = ntot * cfg.d_model * 2                       # packed projection weights, bf16
+    cache = ctx * cfg.dkv * 2 * 2                    # K and V rows read by the attention
+    state = 2 * cfg.dkv * 4 * (cfg.recall_r + 4) + cfg.d_model * 8 * 2
+    return float(w + cache + state)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import route_kv_memory_b200 as mka
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = CONFIGS[args.workload]
+    inp = make_inputs(cfg)
+    weights = {k: v.to(dev) for k, v in inp.tensors().items() if k != "x"}
+    layer = mka.FastMKALayer(cfg, weights, dev)
+    x = inp.x[:, :cfg.seq].contiguous().to(dev)
+    out = torch.empty(cfg.batch, cfg.seq, cfg.dq, dtype=x.dtype, device=dev)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        layer.prefill(x, out)
+    torch.cuda.synchronize()
+    assert mka.mka_status() == 0
+
+    # ---- timed region: K prefill steps, L2 flushed before each, device time by CUDA events
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ms = []
+    mka.mka_profile_enable(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev0[i].record(stream)
+            layer.prefill(x, out)
+            ev1[i].record(stream)
+            stage_ms.append(mka.mka_profile_read())
+        torch.cuda.synchronize()
+    barrier(world)
+    mka.mka_profile_enable(False)
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    ms = statistics.mean(step_ms)
+    ms = max_over_ranks(ms, world)
+    launches_per_step = len(stage_ms[0])
+    stages = np.array(stage_ms).mean(axis=0)
+    value = world * cfg.tokens / (ms / 1e3)
+
+    peaks = load_peaks()
+    fl = prefill_flops(cfg)
+    attn_ms = float(stages[8])
+    attn_tflops = fl["attention"] / (attn_ms / 1e3) / 1e12
+    roofline = {"kernel": "attention (causal GQA, online max-shift)", "bound": "tensor",
+                "achieved": round(attn_tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
+                "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)",
+                "traffic": traffic_from_profiles("attention"), "avg_ms": round(attn_ms, 4),
+                "flops_per_launch": fl["attention"]}
+    layer_tflops = (fl["projections"] + fl["attention"]) / (ms / 1e3) / 1e12
+
+    # ---- end to end through host buffers (pinned): H2D of X, the layer, D2H of O, every step
+    x_host = inp.x[:, :cfg.seq].contiguous().pin_memory()
+    o_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(max(3, args.steps // 4))]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(len(e0))]
+    for i in range(2):
+        x.copy_(x_host, non_blocking=True)
+        layer.prefill(x, out)
+        o_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    for i in range(len(e0)):
+        flush.zero_()
+        e0[i].record(stream)
+        x.copy_(x_host, non_blocking=True)
+        layer.prefill(x, out)
+        o_host.copy_(out, non_blocking=True)
+        e1[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(e0, e1)), world)
+    e2e = {"value": world * cfg.tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+           "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "ms_per_step": round(e2e_ms, 4)}
+    del x_host, o_host
+
+    result = {
+        "metric": "FastMKA layer prefill tokens/s (decode us/token and roofline fraction alongside)",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) inputs, N(0,1/d_in) weights)",
+        "config": {"workload": f"{cfg.name}: Qwen2.5-7B-shaped FastMKA layer prefill, batch {cfg.batch} x seq "
+                               f"{cfg.seq}, d_model {cfg.d_model}, {cfg.n_q_heads}/{cfg.n_kv_heads} heads, d_h "
+                               f"{cfg.d_head}, router {cfg.dq}->{cfg.router_hidden}->3, alpha {cfg.alpha}, L3 block "
+                               f"{cfg.block}, R {cfg.recall_r}, nbits {cfg.hash_bits}, seed {cfg.seed}",
+                   "global_batch": cfg.batch * world, "seq_len": cfg.seq,
+                   "parallelism": f"replicas x{world} (independent sequences, no exchange)",
+                   "l2": "flushed (512 MB write) before every timed step"},
+        "roofline": roofline,
+        "layer_tflops": round(layer_tflops, 1),
+        "stage_ms": {n: round(float(v), 4) for n, v in zip(PREFILL_STAGES, stages)},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    del flush
+    if world == 1 and not args.no_decode:
+        result["decode"] = run_decode(args, cfg, inp, weights, dev, layer_pack=None)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, inp, budget_rows=args.cpu_rows)
+    return result
+
+
+def run_decode(args, cfg_prefill, inp_unused, weights_unused, dev, layer_pack=None):
+    """Decode us/token over a fused cache of `ctx` positions: 256 steps captured in one CUDA graph."""
+    import route_kv_memory_b200 as mka
+    out = {}
+    dcfg = CONFIGS["qwen7b_decode"]
+    dinp = make_inputs(dcfg, seq_total=max(args.decode_ctx) + dcfg.decode_new)
+    w = {k: v.to(dev) for k, v in dinp.tensors().items() if k != "x"}
+    peaks = load_peaks()
+    for ctx in args.decode_ctx:
+        n_new = dcfg.decode_new
+        lmax = ctx + n_new
+        c = dcfg.replace(seq=ctx, decode_new=0)
+        layer = mka.FastMKALayer(c, w, dev)
+        x = dinp.x[:, :ctx + n_new].contiguous().to(dev)
+        pre = torch.empty(1, ctx, dcfg.dq, dtype=x.dtype, device=dev)
+        state = layer.new_state(lmax)
+        layer.prefill(x[:, :ctx].contiguous(), pre, state=state, max_positions=lmax)
+        snapshot = state.clone()
+        xs = [x[:, t].contiguous() for t in range(ctx, ctx + n_new)]
+        outs = [torch.empty(1, dcfg.dq, dtype=x.dtype, device=dev) for _ in range(n_new)]
+        # per-stage times of one eager step (profiling off in the graph)
+        mka.mka_profile_enable(True)
+        layer.decode(state, lmax, xs[0], outs[0])
+        stages = mka.mka_profile_read()
+        mka.mka_profile_enable(False)
+        state.copy_(snapshot)
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            layer.decode(state, lmax, xs[0], outs[0], stream=s)  # creates the workspace outside capture
+            state.copy_(snapshot)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=s):
+                for t in range(n_new):
+                    layer.decode(state, lmax, xs[t], outs[t], stream=s)
+        torch.cuda.synchronize()
+        times = []
+        for rep in range(4):
+            state.copy_(snapshot)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            if rep > 0:
+                times.append(e0.elapsed_time(e1))
+        assert mka.mka_status() == 0
+        us = statistics.mean(times) * 1e3 / n_new
+        ntot = dcfg.dq + 2 * dcfg.dkv + 2 * dcfg.router_hidden + dcfg.hash_bits
+        byt = decode_bytes_per_token(dcfg, ctx + n_new // 2, ntot)
+        gbs = byt / (us * 1e-6) / 1e9
+        out[str(ctx)] = {"us_per_token": round(us, 2), "tokens": n_new, "launches_per_token": 4,
+                         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                                      "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                      "bytes_per_token": byt},
+                         "stage_us_one_step": {n: round(v * 1e3, 2) for n, v in
+                                               zip(["gemv", "token_update", "splitkv_attention", "merge"], stages)}}
+        del g, layer, x, pre, state, snapshot, xs, outs
+        torch.cuda.empty_cache()
+    return {"workload": "qwen7b_decode: Qwen2.5-7B-shaped decode, batch 1, 256 new tokens after a prefilled "
+                        "fused cache; block 256, R 8, nbits 32, alpha 0.99, seed 4", "by_context": out}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_baseline(cfg, inp, budget_rows=48):
+    """The oracle as it stands on this host's cores: all linear parts of the layer for every token, the
+    attention for a strided row sample, extrapolated to all rows by the causal pair count."""
+    import oracle
+    X = inp.x[:, :cfg.seq].float().numpy()
+    w = oracle.weights_f64(*(to_f64(t) for t in (inp.w_q, inp.w_k, inp.w_v, inp.w_r1, inp.w_r2, inp.hash_proj)))
+    rows = sample_rows(cfg.seq, cfg.block, max_rows=budget_rows)
+    t0 = time.perf_counter()
+    out = oracle.fastmka_prefill(X, w, cfg, rows=rows)
+    t_total = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    for bi in range(cfg.batch):
+        oracle.causal_gqa_attention(out["q"][bi], rows, out["K"][bi], out["V"][bi], cfg.n_kv_heads, cfg.scale)
+    t_attn = time.perf_counter() - t1
+    t_lin = max(t_total - t_attn, 0.0)
+    pairs_all = cfg.seq * (cfg.seq + 1) / 2
+    pairs_sample = float(np.sum(rows + 1))
+    t_full = t_lin + t_attn * pairs_all / pairs_sample
+    cores = len(os.sched_getaffinity(0))
+    return {"value": round(cfg.tokens / t_full, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"float64 NumPy oracle, {cfg.name}: projections/router/EMA/L3/fuse/K,V for all "
+                      f"{cfg.tokens} tokens ({t_lin:.1f} s) + attention for {len(rows)} strided query rows per "
+                      f"sequence ({t_attn:.1f} s), extrapolated by causal pair count to {t_full:.1f} s per layer",
+            "measured_s": round(t_total, 2)}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle, timed per step on a bounded sample of the same workload."""
+    if rank != 0:
+        return None
+    cfg = CONFIGS[args.workload]
+    inp = make_inputs(cfg)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(cfg, inp, budget_rows=max(8, args.cpu_rows // 4))
+        if i >= args.warmup:
+            vals.append(r)
+    v = statistics.mean(r["value"] for r in vals)
+    ms = statistics.mean(cfg.tokens / r["value"] * 1e3 for r in vals)
+    return {"impl": "reference", "metric": "FastMKA layer prefill tokens/s (decode us/token and roofline fraction "
+                                           "alongside)", "value": round(v, 2), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "global_batch": cfg.batch, "seq_len": cfg.seq,
+                       "parallelism": "CPU oracle, rank 0 only"},
+            "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "cores": vals[-1]["cores"], "kind": "oracle",
+                             "sample": vals[-1]["sample"]},
+            "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def traffic_from_profiles(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary (profiles/*.json), if one matches the current kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    return d.get(kernel)
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen7b_4k")
+    ap.add_argument("--decode-ctx", type=int, nargs="*", default=[131072])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=48)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

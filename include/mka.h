@@ -1,0 +1,206 @@
+/*
+ * mka.h -- C ABI of the B200 (sm_100a) FastMKA layer library, libmka.so.
+ *
+ * Route-Fused Memory-Keyed Attention ("MKA: Memory-Keyed Attention for
+ * Efficient Long-Context Reasoning"; "notes" = the paper-notes page, "abstract"
+ * = the abstract-and-tables page):
+ *   lambda  = softmax(MLP(q))                          notes §2 (routing gate)
+ *   L2: M2[t] = a*M2[t-1] + (1-a)*X[t-1], M2[0] = 0     notes §1 (session memory, causal)
+ *   L3: R nearest strictly-past block summaries by
+ *       sign-projection Hamming distance                notes §1 (long-term memory)
+ *   X_fused = l1*X + l2*M2 + l3*M3; K,V = X_fused W_k,v notes §3 (FastMKA)
+ *   O = one causal GQA attention over the fused K/V,
+ *       online max-shift softmax                        notes §3-§4
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers unless a parameter says "host".  They are
+ *     owned by the caller, contiguous, row-major and token-major ([B, S, ...]).
+ *     The library never allocates and never frees.
+ *   - Weights are [d_in, d_out] (y = x W).  Head-major columns: column h*d_head+i
+ *     of q / O is head h, channel i; query head h reads KV group
+ *     g(h) = h / (n_q_heads / n_kv_heads).
+ *   - `dtype` (MKA_F32 or MKA_BF16) is the element type of X, the weights, q,
+ *     K, V and O.  lambda, EMA states, summaries and projections are float32.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call is asynchronous on it.
+ *   - Return value: MKA_OK or a negative mka_status_t for errors found on the
+ *     host (arguments, sizes, alignment, launch failures).  Errors found by a
+ *     kernel (a bounded wait that ran out, an index out of range, a full decode
+ *     cache) are recorded in a device status word read by mka_status().  No
+ *     call traps or asserts on the device.  mka_last_error() gives a message.
+ *   - Alignment: every pointer must be 16-byte aligned.
+ *   - Supported shapes: d_head in {64, 128}; n_q_heads % n_kv_heads == 0;
+ *     d_model % 64 == 0; router_hidden % 8 == 0 and <= 1024; 1 <= hash_bits <= 32;
+ *     1 <= recall_r <= 64; block_size >= 1; 0 <= ema_alpha <= 1.
+ */
+#ifndef MKA_H
+#define MKA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MKA_API __attribute__((visibility("default")))
+#else
+#define MKA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MKA_OK = 0,
+  MKA_ERR_INVALID_ARG = -1,    /* null / misaligned pointer, bad size or parameter */
+  MKA_ERR_UNSUPPORTED = -2,    /* valid FastMKA shape this build does not implement */
+  MKA_ERR_CUDA = -3,           /* a CUDA runtime call or a kernel launch failed */
+  MKA_ERR_CAPACITY = -4,       /* decode cache full (device status) */
+  MKA_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait ran out (device status) */
+  MKA_ERR_DEVICE_BOUNDS = -6,  /* a kernel's bounds check failed (device status) */
+  MKA_ERR_WORKSPACE = -7       /* workspace / buffer smaller than the size query says */
+} mka_status_t;
+
+typedef enum { MKA_F32 = 0, MKA_BF16 = 1 } mka_dtype_t;
+
+typedef struct mka_config {
+  int32_t batch;         /* B */
+  int32_t seq;           /* S: rows per sequence of a prefill call */
+  int32_t d_model;       /* d */
+  int32_t n_q_heads;     /* Hq */
+  int32_t n_kv_heads;    /* Hkv */
+  int32_t d_head;        /* dh */
+  int32_t router_hidden; /* rh: router MLP d_q -> rh (GELU) -> 3 */
+  float ema_alpha;       /* a of the L2 EMA */
+  int32_t block_size;    /* b: L3 block length */
+  int32_t recall_r;      /* R: blocks recalled per token */
+  int32_t hash_bits;     /* nbits of the sign-projection code */
+  int32_t dtype;         /* mka_dtype_t */
+  float attn_scale;      /* <= 0 selects 1/sqrt(d_head) */
+} mka_config;
+
+/* Raw layer weights, all in cfg->dtype, all [d_in, d_out] row-major. */
+typedef struct mka_weights {
+  const void* w_q;       /* [d, Hq*dh] */
+  const void* w_k;       /* [d, Hkv*dh] */
+  const void* w_v;       /* [d, Hkv*dh] */
+  const void* w_r1;      /* [Hq*dh, rh] */
+  const void* w_r2;      /* [rh, 3] */
+  const void* hash_proj; /* [d, nbits]: the L3 sign-random-projection P */
+} mka_weights;
+
+/* ------------------------------------------------------------------ sizes */
+
+/* Bytes of the packed-weight buffer that mka_pack_weights fills (0 on a bad cfg). */
+MKA_API size_t mka_packed_weights_size(const mka_config* cfg);
+
+/* Bytes of scratch that mka_prefill_forward needs for cfg (0 on a bad cfg). */
+MKA_API size_t mka_workspace_size(const mka_config* cfg);
+
+/* Bytes of scratch that mka_router / mka_session_ema / mka_longterm_recall need. */
+MKA_API size_t mka_router_workspace_size(const mka_config* cfg);
+MKA_API size_t mka_session_ema_workspace_size(const mka_config* cfg);
+MKA_API size_t mka_longterm_recall_workspace_size(const mka_config* cfg);
+
+/* Bytes of a decode state holding up to max_positions tokens per sequence, and
+ * bytes of the scratch mka_decode_step needs. */
+MKA_API size_t mka_state_size(const mka_config* cfg, int32_t max_positions);
+MKA_API size_t mka_decode_workspace_size(const mka_config* cfg, int32_t max_positions);
+
+/* ------------------------------------------------------------------ set-up */
+
+/* Pack the raw weights into the layout the fused kernels read: the transposed
+ * concatenation [W_q | W_k | W_v | W_q W_r1 | P]^T (for bf16 the folded router
+ * matrix W_q W_r1 is stored as a bf16 hi/lo pair so that the router sees q at
+ * float32 accuracy), W_r2 in float32, and P^T in float64 for exact sign
+ * decisions.  The fold is exact in real arithmetic: (X W_q) W_r1 = X (W_q W_r1)
+ * (notes §2 applies the MLP to q = X W_q).  `packed` must hold
+ * mka_packed_weights_size(cfg) bytes.  Re-run after the weights change. */
+MKA_API int mka_pack_weights(const mka_config* cfg, const mka_weights* w, void* packed, size_t packed_bytes,
+                     void* stream);
+
+/* Initialise a decode state (device buffer of mka_state_size bytes): empty cache,
+ * M2 = 0, no finished block, position 0. */
+MKA_API int mka_state_init(const mka_config* cfg, int32_t max_positions, void* state, size_t state_bytes, void* stream);
+
+/* ------------------------------------------------------------------ the five steps */
+
+/* Routing gate, notes §2: lambda[t] = softmax(GELU(q[t] W_r1) W_r2), one triple per
+ * token shared by all heads.  q [B*S, Hq*dh] (dtype), w_r1 [Hq*dh, rh], w_r2 [rh, 3]
+ * (dtype) -> lambda [B*S, 3] float32.  No biases; GELU is x*Phi(x) (erf form).
+ * ws: mka_router_workspace_size(cfg) bytes. */
+MKA_API int mka_router(const mka_config* cfg, const void* q, const void* w_r1, const void* w_r2, float* lambda,
+               void* ws, size_t ws_bytes, void* stream);
+
+/* L2 session memory, notes §1: M2[t] = a*M2[t-1] + (1-a)*X[t-1] per sequence, with
+ * M2[0] = carry_in (zeros when NULL).  x [B, S, d] (dtype) -> m2 [B, S, d] float32.
+ * carry_out (nullable) [B, d] float32 receives M2[S], the state of the next token.
+ * ws: mka_session_ema_workspace_size(cfg) bytes. */
+MKA_API int mka_session_ema(const mka_config* cfg, const void* x, const float* carry_in, float* m2, float* carry_out,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* L3 long-term memory, notes §1: block j = rows [j*b, (j+1)*b) of a sequence, summary
+ * s_j = block mean of X; code(v) = bits [(v P)_k > 0] (bit k = projection k).  Block j
+ * is eligible at row t iff (j+1)*b <= t.  For every row, the R eligible blocks with the
+ * smallest (Hamming distance, j) are recalled.  Sign decisions are exact: a projection
+ * whose float32 value is within the float32 error bound of zero is recomputed in
+ * float64.  x [B, S, d], hash_proj [d, nbits] (dtype) ->
+ *   idx   [B, S, R] int32, sorted by (distance, j), -1 padded
+ *   count [B, S] int32 (nullable) = min(R, floor(t/b))
+ *   m3    [B, S, d] float32 (nullable) = mean of the recalled summaries, 0 if none.
+ * ws: mka_longterm_recall_workspace_size(cfg) bytes. */
+MKA_API int mka_longterm_recall(const mka_config* cfg, const void* x, const void* hash_proj, int32_t* idx, int32_t* count,
+                        float* m3, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer forward over B sequences of S rows (notes §1-§4):
+ * x [B, S, d] (dtype) -> out [B, S, Hq*dh] (dtype, heads concatenated, no output
+ * projection).  `packed` comes from mka_pack_weights.  Optional outputs (NULL to
+ * skip): lambda_out [B*S, 3] float32, recall_idx_out [B, S, R] int32.  When `state`
+ * is not NULL (mka_state_init'ed, max_positions >= S), the fused K/V rows, M2[S],
+ * the finished block summaries and the unfinished block's partial sums are left in
+ * it and its position is set to S, ready for mka_decode_step.
+ * ws: mka_workspace_size(cfg) bytes. */
+MKA_API int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x, void* out, float* lambda_out,
+                        int32_t* recall_idx_out, void* state, size_t state_bytes, int32_t max_positions,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* One decode step for the next token of each sequence (notes §3: the cache holds the
+ * fused routed K/V).  x_new [B, d] (dtype) -> out [B, Hq*dh] (dtype).  Runs the
+ * router, reads M2 and recalls from the finished blocks, appends the fused K/V row
+ * at the current position, attends over cache[0..pos] (split-KV with a max-shift
+ * merge), then advances M2, the block sums and the position.  The position lives
+ * in device memory, so a sequence of steps can be captured in a CUDA graph.  A
+ * step on a full cache records MKA_ERR_CAPACITY in the status word and changes
+ * nothing.  ws: mka_decode_workspace_size(cfg, max_positions) bytes. */
+MKA_API int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size_t state_bytes,
+                    int32_t max_positions, const void* x_new, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ status */
+
+/* Synchronises the current device and returns the device status word (MKA_OK or one
+ * of the device-side codes), then clears it. */
+MKA_API int mka_status(void);
+
+/* Message for the last host-side error of the calling thread ("" if none). */
+MKA_API const char* mka_last_error(void);
+
+/* Stage timing, for measurement.  While enabled, mka_prefill_forward and
+ * mka_decode_step record a CUDA event on their stream before each stage and
+ * after the last one.  mka_profile_read waits for the most recent call's last
+ * event, writes the device milliseconds of up to max_stages of its stages into
+ * the HOST array ms, and returns how many stages that call had.  Stages of a
+ * prefill: 0 projection GEMM, 1 router tail, 2 token codes, 3 block sums,
+ * 4 block codes, 5 EMA carries, 6 recall, 7 route-fuse, 8 attention
+ * (9 decode-state tail when a state is filled).  Stages of a decode step:
+ * 0 GEMV, 1 token update, 2 split-KV attention, 3 merge.  Not for use while
+ * capturing a CUDA graph.  Returns a negative mka_status_t on error. */
+MKA_API int mka_profile_enable(int enable);
+MKA_API int mka_profile_read(float* ms, int max_stages);
+
+/* Library version string. */
+MKA_API const char* mka_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MKA_H */

@@ -1,0 +1,583 @@
+// C ABI of libmka.so: argument checks, buffer layouts and launch sequences.
+// Declarations and the contract of every entry point are in include/mka.h.
+#include <math.h>
+#include <stdarg.h>
+#include <mutex>
+#include <stdio.h>
+#include <string.h>
+#include <string>
+
+#include "../../include/mka.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace mka;
+
+// Device status word: kernels record device-side errors here (never trap).
+__device__ int g_mka_status = 0;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                        \
+  do {                                                                                        \
+    cudaError_t e_ = (expr);                                                                  \
+    if (e_ != cudaSuccess) return fail(MKA_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+int* status_ptr() {
+  static std::mutex mu;
+  static int* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_mka_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = (int*)p;
+  }
+  return ptrs[dev];
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+inline size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+struct Dims {
+  int B, S, d, Hq, Hkv, dh, rh, blk, R, nb, bf16, elem;
+  int dq, dkv, width, nblk, T;
+  float alpha, scale;
+};
+
+int check_cfg(const mka_config* c, Dims* o) {
+  if (!c) return fail(MKA_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->batch < 1 || c->seq < 1) return fail(MKA_ERR_INVALID_ARG, "batch and seq must be >= 1");
+  if (c->d_model < 64 || c->d_model % 64) return fail(MKA_ERR_UNSUPPORTED, "d_model must be a positive multiple of 64");
+  if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads)
+    return fail(MKA_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+  if (c->d_head != 64 && c->d_head != 128) return fail(MKA_ERR_UNSUPPORTED, "d_head must be 64 or 128");
+  if (c->router_hidden < 8 || c->router_hidden % 8 || c->router_hidden > 1024)
+    return fail(MKA_ERR_UNSUPPORTED, "router_hidden must be a multiple of 8 in [8, 1024]");
+  if (!(c->ema_alpha >= 0.f && c->ema_alpha <= 1.f)) return fail(MKA_ERR_INVALID_ARG, "ema_alpha must be in [0, 1]");
+  if (c->block_size < 1) return fail(MKA_ERR_INVALID_ARG, "block_size must be >= 1");
+  if (c->recall_r < 1 || c->recall_r > 64) return fail(MKA_ERR_UNSUPPORTED, "recall_r must be in [1, 64]");
+  if (c->hash_bits < 1 || c->hash_bits > 32) return fail(MKA_ERR_UNSUPPORTED, "hash_bits must be in [1, 32]");
+  if (c->dtype != MKA_F32 && c->dtype != MKA_BF16) return fail(MKA_ERR_INVALID_ARG, "dtype must be MKA_F32 or MKA_BF16");
+  long long T = (long long)c->batch * c->seq;
+  if (T > (1LL << 30)) return fail(MKA_ERR_UNSUPPORTED, "batch * seq too large");
+  if ((c->seq + c->block_size - 1) / c->block_size > 65535) return fail(MKA_ERR_UNSUPPORTED, "seq / block_size > 65535");
+  Dims& d = *o;
+  d.B = c->batch;
+  d.S = c->seq;
+  d.d = c->d_model;
+  d.Hq = c->n_q_heads;
+  d.Hkv = c->n_kv_heads;
+  d.dh = c->d_head;
+  d.rh = c->router_hidden;
+  d.blk = c->block_size;
+  d.R = c->recall_r;
+  d.nb = c->hash_bits;
+  d.bf16 = c->dtype == MKA_BF16;
+  d.elem = d.bf16 ? 2 : 4;
+  d.dq = d.Hq * d.dh;
+  d.dkv = d.Hkv * d.dh;
+  d.width = 2 * d.dkv;
+  d.nblk = d.S / d.blk;
+  d.T = (int)T;
+  d.alpha = c->ema_alpha;
+  d.scale = c->attn_scale > 0.f ? c->attn_scale : 1.f / sqrtf((float)d.dh);
+  return MKA_OK;
+}
+
+// ---------------------------------------------------------------- packed weights
+struct PackLayout {
+  int Ntot, Npad, seg_q, seg_k, seg_v, seg_r, seg_rlo, seg_p, rh_segs;
+  size_t wcat, wr2, pT64, wqr32, wr1T, total;
+};
+PackLayout pack_layout(const Dims& d) {
+  PackLayout p;
+  p.rh_segs = d.bf16 ? 2 : 1;
+  p.seg_q = 0;
+  p.seg_k = d.dq;
+  p.seg_v = d.dq + d.dkv;
+  p.seg_r = d.dq + 2 * d.dkv;
+  p.seg_rlo = d.bf16 ? p.seg_r + d.rh : -1;
+  p.seg_p = p.seg_r + p.rh_segs * d.rh;
+  p.Ntot = p.seg_p + d.nb;
+  p.Npad = (p.Ntot + 127) / 128 * 128;
+  size_t o = 0;
+  p.wcat = o; o += al((size_t)p.Npad * d.d * d.elem);
+  p.wr2 = o; o += al((size_t)d.rh * 3 * 4);
+  p.pT64 = o; o += al((size_t)d.nb * d.d * 8);
+  p.wqr32 = o; o += al((size_t)d.rh * d.d * 4);
+  p.wr1T = o; o += al((size_t)d.rh * d.dq * d.elem);
+  p.total = o;
+  return p;
+}
+
+// ---------------------------------------------------------------- prefill workspace
+struct PrefillWs {
+  size_t q, xkv, h1, h2, proj, lam, tcode, eps, bsum, bend, carry, scode, idx, cnt, k, v, total;
+};
+PrefillWs prefill_ws(const Dims& d) {
+  PrefillWs w;
+  size_t T = d.T, o = 0;
+  w.q = o; o += al(T * d.dq * d.elem);
+  w.xkv = o; o += al(T * d.width * 4);
+  w.h1 = o; o += al(T * d.rh * 4);
+  w.h2 = o; o += d.bf16 ? al(T * d.rh * 4) : 0;
+  w.proj = o; o += al(T * d.nb * 4);
+  w.lam = o; o += al(T * 3 * 4);
+  w.tcode = o; o += al(T * 4);
+  w.eps = o; o += al(T * 4);
+  w.bsum = o; o += al((size_t)d.B * d.nblk * d.width * 4);
+  w.bend = o; o += al((size_t)d.B * d.nblk * d.width * 4);
+  w.carry = o; o += al((size_t)d.B * (d.nblk + 1) * d.width * 4);
+  w.scode = o; o += al((size_t)d.B * d.nblk * 4);
+  w.idx = o; o += al(T * d.R * 4);
+  w.cnt = o; o += al(T * 4);
+  w.k = o; o += al(T * d.dkv * d.elem);
+  w.v = o; o += al(T * d.dkv * d.elem);
+  w.total = o;
+  return w;
+}
+
+// ---------------------------------------------------------------- decode state
+struct StateLayout {
+  int Lmax, maxblk;
+  size_t pos, kc, vc, ema, blk_sum, blk_p, blk_eps, blk_x, summ, scode, total;
+};
+StateLayout state_layout(const Dims& d, int Lmax) {
+  StateLayout s;
+  s.Lmax = Lmax;
+  s.maxblk = Lmax / d.blk;
+  size_t o = 0, B = d.B;
+  s.pos = o; o += al(B * 4);
+  s.kc = o; o += al(B * Lmax * d.dkv * d.elem);
+  s.vc = o; o += al(B * Lmax * d.dkv * d.elem);
+  s.ema = o; o += al(B * d.width * 4);
+  s.blk_sum = o; o += al(B * d.width * 4);
+  s.blk_p = o; o += al(B * 32 * 4);
+  s.blk_eps = o; o += al(B * 4);
+  s.blk_x = o; o += al(B * d.d * 8);
+  s.summ = o; o += al(B * (size_t)s.maxblk * d.width * 4);
+  s.scode = o; o += al(B * (size_t)s.maxblk * 4);
+  s.total = o;
+  return s;
+}
+
+int decode_nsplit(const Dims& d, int Lmax) {
+  int sms = sm_count();
+  int ns;
+  if (d.bf16) ns = (sms + d.B * d.Hkv - 1) / (d.B * d.Hkv);
+  else ns = (2 * sms + d.B * d.Hq - 1) / (d.B * d.Hq);
+  int cap = (Lmax + 127) / 128;
+  if (ns > cap) ns = cap;
+  if (ns < 1) ns = 1;
+  if (ns > 512) ns = 512;
+  return ns;
+}
+
+struct DecodeWs {
+  int nsplit;
+  size_t y, qf, part, total;
+};
+DecodeWs decode_ws(const Dims& d, int Lmax) {
+  DecodeWs w;
+  PackLayout p = pack_layout(d);
+  w.nsplit = decode_nsplit(d, Lmax);
+  size_t o = 0, B = d.B;
+  w.y = o; o += al(B * p.Ntot * 4);
+  w.qf = o; o += al(B * d.dq * 4);
+  w.part = o; o += al(B * d.Hq * (size_t)w.nsplit * (d.dh + 2) * 4);
+  w.total = o;
+  return w;
+}
+
+inline char* P(void* base, size_t off) { return (char*)base + off; }
+
+// ---------------------------------------------------------------- stage timing
+constexpr int kMaxStages = 16;
+struct Profiler {
+  bool on = false;
+  bool created = false;
+  int n = 0;  // events recorded by the last call
+  cudaEvent_t ev[kMaxStages + 1];
+  cudaError_t mark(cudaStream_t s) {
+    if (!on || n > kMaxStages) return cudaSuccess;
+    return cudaEventRecord(ev[n++], s);
+  }
+};
+Profiler g_prof;
+
+inline void prof_begin() { g_prof.n = 0; }
+#define STAGE(s) CUDA_TRY(g_prof.mark(s))
+
+}  // namespace
+
+extern "C" {
+
+const char* mka_version(void) { return "fastmka-b200 0.1 (sm_100a)"; }
+
+int mka_profile_enable(int enable) {
+  if (enable && !g_prof.created) {
+    for (int i = 0; i <= kMaxStages; ++i) CUDA_TRY(cudaEventCreate(&g_prof.ev[i]));
+    g_prof.created = true;
+  }
+  g_prof.on = enable != 0;
+  g_prof.n = 0;
+  return MKA_OK;
+}
+
+int mka_profile_read(float* ms, int max_stages) {
+  if (!g_prof.created || g_prof.n < 2) return fail(MKA_ERR_INVALID_ARG, "no profiled call to read");
+  CUDA_TRY(cudaEventSynchronize(g_prof.ev[g_prof.n - 1]));
+  int stages = g_prof.n - 1;
+  for (int i = 0; i < stages && i < max_stages; ++i) CUDA_TRY(cudaEventElapsedTime(&ms[i], g_prof.ev[i], g_prof.ev[i + 1]));
+  return stages;
+}
+const char* mka_last_error(void) { return g_err.c_str(); }
+
+int mka_status(void) {
+  int* p = status_ptr();
+  if (!p) return fail(MKA_ERR_CUDA, "no CUDA device");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail(MKA_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
+  int v = 0;
+  e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(MKA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  int z = 0;
+  cudaMemcpy(p, &z, sizeof(int), cudaMemcpyHostToDevice);
+  return v;
+}
+
+size_t mka_packed_weights_size(const mka_config* cfg) {
+  Dims d;
+  if (check_cfg(cfg, &d) != MKA_OK) return 0;
+  return pack_layout(d).total;
+}
+
+size_t mka_workspace_size(const mka_config* cfg) {
+  Dims d;
+  if (check_cfg(cfg, &d) != MKA_OK) return 0;
+  return prefill_ws(d).total;
+}
+
+size_t mka_router_workspace_size(const mka_config* cfg) {
+  Dims d;
+  if (check_cfg(cfg, &d) != MKA_OK) return 0;
+  return al((size_t)d.rh * d.dq * d.elem) + al((size_t)d.rh * 3 * 4) + al((size_t)d.T * d.rh * 4);
+}
+
+static const int kEmaChunk = 64;
+
+size_t mka_session_ema_workspace_size(const mka_config* cfg) {
+  Dims d;
+  if (check_cfg(cfg, &d) != MKA_OK) return 0;
+  size_t nch = d.S / kEmaChunk;
+  return al((size_t)d.B * nch * d.d * 4) + al((size_t)d.B * (nch + 1) * d.d * 4);
+}
+
+size_t mka_longterm_recall_workspace_size(const mka_config* cfg) {
+  Dims d;
+  if (check_cfg(cfg, &d) != MKA_OK) return 0;
+  size_t T = d.T;
+  return al((size_t)d.nb * d.d * d.elem) + al((size_t)d.nb * d.d * 8) + al(T * d.nb * 4) + al(T * 4) + al(T * 4) +
+         al((size_t)d.B * d.nblk * d.d * 4) + al((size_t)d.B * d.nblk * 4) + al(T * 4);
+}
+
+size_t mka_state_size(const mka_config* cfg, int32_t max_positions) {
+  Dims d;
+  if (check_cfg(cfg, &d) != MKA_OK || max_positions < 1) return 0;
+  return state_layout(d, max_positions).total;
+}
+
+size_t mka_decode_workspace_size(const mka_config* cfg, int32_t max_positions) {
+  Dims d;
+  if (check_cfg(cfg, &d) != MKA_OK || max_positions < 1) return 0;
+  return decode_ws(d, max_positions).total;
+}
+
+int mka_pack_weights(const mka_config* cfg, const mka_weights* w, void* packed, size_t packed_bytes, void* stream) {
+  Dims d;
+  int rc = check_cfg(cfg, &d);
+  if (rc) return rc;
+  if (!w || !w->w_q || !w->w_k || !w->w_v || !w->w_r1 || !w->w_r2 || !w->hash_proj || !packed)
+    return fail(MKA_ERR_INVALID_ARG, "NULL weight or packed pointer");
+  if (!aligned16(w->w_q) || !aligned16(w->w_k) || !aligned16(w->w_v) || !aligned16(w->w_r1) || !aligned16(packed))
+    return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  PackLayout L = pack_layout(d);
+  if (packed_bytes < L.total) return fail(MKA_ERR_WORKSPACE, "packed buffer %zu < %zu bytes", packed_bytes, L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  char* wc = P(packed, L.wcat);
+  size_t row = (size_t)d.d * d.elem;
+  CUDA_TRY(cudaMemsetAsync(wc, 0, (size_t)L.Npad * row, s));
+  CUDA_TRY(transpose(w->w_q, d.d, d.dq, d.dq, wc + L.seg_q * row, d.d, d.elem, 0, s));
+  CUDA_TRY(transpose(w->w_k, d.d, d.dkv, d.dkv, wc + L.seg_k * row, d.d, d.elem, 0, s));
+  CUDA_TRY(transpose(w->w_v, d.d, d.dkv, d.dkv, wc + L.seg_v * row, d.d, d.elem, 0, s));
+  CUDA_TRY(transpose(w->hash_proj, d.d, d.nb, d.nb, wc + L.seg_p * row, d.d, d.elem, 0, s));
+  CUDA_TRY(transpose(w->hash_proj, d.d, d.nb, d.nb, P(packed, L.pT64), d.d, d.elem, 1, s));
+  CUDA_TRY(widen_f32(w->w_r2, d.rh * 3, d.bf16, (float*)P(packed, L.wr2), s));
+  // Router fold: (W_q W_r1)^T [rh, d] = W_r1^T [rh, dq] . W_q^T, float32 accumulation.
+  CUDA_TRY(transpose(w->w_r1, d.dq, d.rh, d.rh, P(packed, L.wr1T), d.dq, d.elem, 0, s));
+  Epilogue ep{};
+  ep.nseg = 1;
+  ep.seg[0] = OutSeg{0, d.d, P(packed, L.wqr32), d.d, 0};
+  CUDA_TRY(gemm_tn_ffma(P(packed, L.wr1T), d.dq, d.bf16, w->w_q, d.dq, d.bf16, d.rh, d.d, d.dq, ep, s));
+  if (d.bf16) {
+    CUDA_TRY(split_hi_lo((const float*)P(packed, L.wqr32), d.rh * d.d, wc + L.seg_r * row, wc + L.seg_rlo * row, s));
+  } else {
+    CUDA_TRY(cudaMemcpyAsync(wc + L.seg_r * row, P(packed, L.wqr32), (size_t)d.rh * d.d * 4, cudaMemcpyDeviceToDevice, s));
+  }
+  return MKA_OK;
+}
+
+int mka_state_init(const mka_config* cfg, int32_t max_positions, void* state, size_t state_bytes, void* stream) {
+  Dims d;
+  int rc = check_cfg(cfg, &d);
+  if (rc) return rc;
+  if (max_positions < 1) return fail(MKA_ERR_INVALID_ARG, "max_positions must be >= 1");
+  if (!state || !aligned16(state)) return fail(MKA_ERR_INVALID_ARG, "state must be a 16-byte aligned device pointer");
+  StateLayout L = state_layout(d, max_positions);
+  if (state_bytes < L.total) return fail(MKA_ERR_WORKSPACE, "state buffer %zu < %zu bytes", state_bytes, L.total);
+  CUDA_TRY(cudaMemsetAsync(state, 0, L.total, (cudaStream_t)stream));
+  return MKA_OK;
+}
+
+int mka_router(const mka_config* cfg, const void* q, const void* w_r1, const void* w_r2, float* lambda, void* ws,
+               size_t ws_bytes, void* stream) {
+  Dims d;
+  int rc = check_cfg(cfg, &d);
+  if (rc) return rc;
+  if (!q || !w_r1 || !w_r2 || !lambda || !ws) return fail(MKA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(q) || !aligned16(w_r1) || !aligned16(lambda) || !aligned16(ws))
+    return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  size_t need = mka_router_workspace_size(cfg);
+  if (ws_bytes < need) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w1T = (char*)ws;
+  float* wr2 = (float*)(w1T + al((size_t)d.rh * d.dq * d.elem));
+  float* h = (float*)((char*)wr2 + al((size_t)d.rh * 3 * 4));
+  CUDA_TRY(transpose(w_r1, d.dq, d.rh, d.rh, w1T, d.dq, d.elem, 0, s));
+  CUDA_TRY(widen_f32(w_r2, d.rh * 3, d.bf16, wr2, s));
+  Epilogue ep{};
+  ep.nseg = 1;
+  ep.seg[0] = OutSeg{0, d.rh, h, d.rh, 0};
+  if (d.bf16) CUDA_TRY(gemm_tn_bf16(q, d.dq, w1T, d.dq, d.T, d.rh, d.dq, ep, s));
+  else CUDA_TRY(gemm_tn_ffma(q, d.dq, 0, w1T, d.dq, 0, d.T, d.rh, d.dq, ep, s));
+  CUDA_TRY(router_tail(h, nullptr, d.rh, d.T, d.rh, wr2, lambda, s));
+  return MKA_OK;
+}
+
+int mka_session_ema(const mka_config* cfg, const void* x, const float* carry_in, float* m2, float* carry_out,
+                    void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  int rc = check_cfg(cfg, &d);
+  if (rc) return rc;
+  if (!x || !m2 || !ws) return fail(MKA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(x) || !aligned16(m2) || !aligned16(ws) || (carry_in && !aligned16(carry_in)) ||
+      (carry_out && !aligned16(carry_out)))
+    return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  size_t need = mka_session_ema_workspace_size(cfg);
+  if (ws_bytes < need) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  cudaStream_t s = (cudaStream_t)stream;
+  int nch = d.S / kEmaChunk;
+  float* bend = (float*)ws;
+  float* carry = (float*)((char*)ws + al((size_t)d.B * nch * d.d * 4));
+  double apb = pow((double)d.alpha, (double)kEmaChunk);
+  CUDA_TRY(block_reduce(x, d.bf16, d.d, d.d, d.B, d.S, nch, kEmaChunk, d.alpha, nullptr, 0, bend, s));
+  CUDA_TRY(ema_carry(bend, d.d, d.B, nch, (float)apb, carry_in, carry, s));
+  CUDA_TRY(ema_apply(x, d.bf16, d.d, d.B, d.S, nch, kEmaChunk, d.alpha, carry, m2, carry_out, s));
+  return MKA_OK;
+}
+
+int mka_longterm_recall(const mka_config* cfg, const void* x, const void* hash_proj, int32_t* idx, int32_t* count,
+                        float* m3, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  int rc = check_cfg(cfg, &d);
+  if (rc) return rc;
+  if (!x || !hash_proj || !idx || !ws) return fail(MKA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(x) || !aligned16(ws) || !aligned16(idx) || (m3 && !aligned16(m3)))
+    return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  size_t need = mka_longterm_recall_workspace_size(cfg);
+  if (ws_bytes < need) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  cudaStream_t s = (cudaStream_t)stream;
+  size_t T = d.T;
+  char* o = (char*)ws;
+  void* pT = o; o += al((size_t)d.nb * d.d * d.elem);
+  double* pT64 = (double*)o; o += al((size_t)d.nb * d.d * 8);
+  float* proj = (float*)o; o += al(T * d.nb * 4);
+  float* eps = (float*)o; o += al(T * 4);
+  uint32_t* tcode = (uint32_t*)o; o += al(T * 4);
+  float* bsum = (float*)o; o += al((size_t)d.B * d.nblk * d.d * 4);
+  uint32_t* scode = (uint32_t*)o; o += al((size_t)d.B * d.nblk * 4);
+  int* cnt = count ? count : (int*)o;
+  CUDA_TRY(transpose(hash_proj, d.d, d.nb, d.nb, pT, d.d, d.elem, 0, s));
+  CUDA_TRY(transpose(hash_proj, d.d, d.nb, d.nb, pT64, d.d, d.elem, 1, s));
+  Epilogue ep{};
+  ep.nseg = 1;
+  ep.seg[0] = OutSeg{0, d.nb, proj, d.nb, 0};
+  if (d.bf16) CUDA_TRY(gemm_tn_bf16(x, d.d, pT, d.d, d.T, d.nb, d.d, ep, s));
+  else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, pT, d.d, 0, d.T, d.nb, d.d, ep, s));
+  HashArgs ha{proj, d.nb, x, d.bf16, pT64, d.d, d.nb, d.d};
+  CUDA_TRY(token_codes(ha, d.T, tcode, eps, s));
+  CUDA_TRY(summary_codes(ha, d.B, d.S, d.nblk, d.blk, eps, scode, d.nblk, s));
+  CUDA_TRY(recall_select(tcode, scode, d.nblk, d.B, d.S, d.nblk, d.blk, d.R, idx, cnt, s));
+  if (m3) {
+    CUDA_TRY(block_reduce(x, d.bf16, d.d, d.d, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, (long long)d.nblk * d.d, nullptr, s));
+    CUDA_TRY(gather_mean(idx, cnt, d.R, bsum, d.nblk, d.d, d.blk, d.B, d.S, m3, s));
+  }
+  return MKA_OK;
+}
+
+int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x, void* out, float* lambda_out,
+                        int32_t* recall_idx_out, void* state, size_t state_bytes, int32_t max_positions, void* ws,
+                        size_t ws_bytes, void* stream) {
+  Dims d;
+  int rc = check_cfg(cfg, &d);
+  if (rc) return rc;
+  if (!packed || !x || !out || !ws) return fail(MKA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(out) || !aligned16(ws) ||
+      (lambda_out && !aligned16(lambda_out)) || (recall_idx_out && !aligned16(recall_idx_out)) ||
+      (state && !aligned16(state)))
+    return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  PrefillWs W = prefill_ws(d);
+  if (ws_bytes < W.total) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, W.total);
+  StateLayout SL{};
+  if (state) {
+    if (max_positions < d.S) return fail(MKA_ERR_CAPACITY, "max_positions %d < seq %d", max_positions, d.S);
+    SL = state_layout(d, max_positions);
+    if (state_bytes < SL.total) return fail(MKA_ERR_WORKSPACE, "state buffer %zu < %zu bytes", state_bytes, SL.total);
+  }
+  PackLayout PL = pack_layout(d);
+  cudaStream_t s = (cudaStream_t)stream;
+  void* q = P(ws, W.q);
+  float* xkv = (float*)P(ws, W.xkv);
+  float* h1 = (float*)P(ws, W.h1);
+  float* h2 = d.bf16 ? (float*)P(ws, W.h2) : nullptr;
+  float* proj = (float*)P(ws, W.proj);
+  float* lam = lambda_out ? lambda_out : (float*)P(ws, W.lam);
+  uint32_t* tcode = (uint32_t*)P(ws, W.tcode);
+  float* eps = (float*)P(ws, W.eps);
+  float* bsum = state ? (float*)P(state, SL.summ) : (float*)P(ws, W.bsum);
+  long long bsum_bstride = (long long)(state ? SL.maxblk : d.nblk) * d.width;
+  float* bend = (float*)P(ws, W.bend);
+  float* carry = (float*)P(ws, W.carry);
+  uint32_t* scode = state ? (uint32_t*)P(state, SL.scode) : (uint32_t*)P(ws, W.scode);
+  int code_bstride = state ? SL.maxblk : d.nblk;
+  int* idx = recall_idx_out ? recall_idx_out : (int*)P(ws, W.idx);
+  int* cnt = (int*)P(ws, W.cnt);
+  void* kbuf = state ? P(state, SL.kc) : P(ws, W.k);
+  void* vbuf = state ? P(state, SL.vc) : P(ws, W.v);
+  long long kv_bstride = (long long)(state ? max_positions : d.S) * d.dkv;
+  const void* wcat = P((void*)packed, PL.wcat);
+
+  prof_begin();
+  STAGE(s);
+  // 1. projections: q | XW_k | XW_v | X(W_q W_r1) | XP
+  Epilogue ep{};
+  int ns = 0;
+  ep.seg[ns++] = OutSeg{PL.seg_q, PL.seg_k, q, d.dq, d.bf16};
+  ep.seg[ns++] = OutSeg{PL.seg_k, PL.seg_r, xkv, d.width, 0};
+  ep.seg[ns++] = OutSeg{PL.seg_r, PL.seg_r + d.rh, h1, d.rh, 0};
+  if (d.bf16) ep.seg[ns++] = OutSeg{PL.seg_rlo, PL.seg_rlo + d.rh, h2, d.rh, 0};
+  ep.seg[ns++] = OutSeg{PL.seg_p, PL.Ntot, proj, d.nb, 0};
+  ep.nseg = ns;
+  if (d.bf16) CUDA_TRY(gemm_tn_bf16(x, d.d, wcat, d.d, d.T, PL.Ntot, d.d, ep, s));
+  else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, wcat, d.d, 0, d.T, PL.Ntot, d.d, ep, s));
+  STAGE(s);
+  // 2. router tail
+  CUDA_TRY(router_tail(h1, h2, d.rh, d.T, d.rh, (const float*)P((void*)packed, PL.wr2), lam, s));
+  STAGE(s);
+  // 3. L3 codes, 4. block sums / EMA end states, carries, recall
+  HashArgs ha{proj, d.nb, x, d.bf16, (const double*)P((void*)packed, PL.pT64), d.d, d.nb, d.d};
+  CUDA_TRY(token_codes(ha, d.T, tcode, eps, s));
+  STAGE(s);
+  CUDA_TRY(block_reduce(xkv, 0, d.width, d.width, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, bsum_bstride, bend, s));
+  STAGE(s);
+  CUDA_TRY(summary_codes(ha, d.B, d.S, d.nblk, d.blk, eps, scode, code_bstride, s));
+  STAGE(s);
+  CUDA_TRY(ema_carry(bend, d.width, d.B, d.nblk, (float)pow((double)d.alpha, (double)d.blk), nullptr, carry, s));
+  STAGE(s);
+  CUDA_TRY(recall_select(tcode, scode, code_bstride, d.B, d.S, d.nblk, d.blk, d.R, idx, cnt, s));
+  STAGE(s);
+  // 5. route-fuse -> K, V
+  FuseArgs fa{};
+  fa.xkv = xkv; fa.ld = d.width; fa.width = d.width; fa.lam = lam; fa.idx = idx; fa.count = cnt; fa.R = d.R;
+  fa.bsum = bsum; fa.bsum_bstride = bsum_bstride; fa.carry = carry;
+  fa.B = d.B; fa.S = d.S; fa.nblk = d.nblk; fa.blk = d.blk; fa.dkv = d.dkv; fa.alpha = d.alpha;
+  fa.k_out = kbuf; fa.v_out = vbuf; fa.kv_bstride = kv_bstride; fa.out_bf16 = d.bf16;
+  fa.state_ema = state ? (float*)P(state, SL.ema) : nullptr;
+  CUDA_TRY(fuse_kv(fa, s));
+  STAGE(s);
+  // 6. causal GQA attention over the fused K/V
+  AttnArgs aa{};
+  aa.q = q; aa.q_bstride = (long long)d.S * d.dq; aa.q_ld = d.dq;
+  aa.k = kbuf; aa.v = vbuf; aa.kv_bstride = kv_bstride; aa.kv_ld = d.dkv;
+  aa.o = out; aa.o_bstride = (long long)d.S * d.dq; aa.o_ld = d.dq;
+  aa.B = d.B; aa.S = d.S; aa.Hq = d.Hq; aa.Hkv = d.Hkv; aa.dh = d.dh; aa.scale = d.scale;
+  CUDA_TRY(attention_prefill(aa, d.bf16, s));
+  STAGE(s);
+  if (state) {
+    CUDA_TRY(prefill_tail_state(xkv, d.width, d.width, proj, d.nb, d.nb, eps, x, d.bf16, d.d, d.B, d.S, d.blk,
+                                (float*)P(state, SL.blk_sum), (float*)P(state, SL.blk_p), (float*)P(state, SL.blk_eps),
+                                (double*)P(state, SL.blk_x), (int*)P(state, SL.pos), s));
+    STAGE(s);
+  }
+  return MKA_OK;
+}
+
+int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size_t state_bytes, int32_t max_positions,
+                    const void* x_new, void* out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  int rc = check_cfg(cfg, &d);
+  if (rc) return rc;
+  if (!packed || !state || !x_new || !out || !ws) return fail(MKA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(packed) || !aligned16(state) || !aligned16(x_new) || !aligned16(out) || !aligned16(ws))
+    return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (max_positions < 1) return fail(MKA_ERR_INVALID_ARG, "max_positions must be >= 1");
+  if (d.B > 8) return fail(MKA_ERR_UNSUPPORTED, "decode batch must be <= 8");
+  if (d.bf16 && d.Hq / d.Hkv > 16) return fail(MKA_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads must be <= 16 for decode");
+  StateLayout SL = state_layout(d, max_positions);
+  if (state_bytes < SL.total) return fail(MKA_ERR_WORKSPACE, "state buffer %zu < %zu bytes", state_bytes, SL.total);
+  DecodeWs W = decode_ws(d, max_positions);
+  if (ws_bytes < W.total) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, W.total);
+  PackLayout PL = pack_layout(d);
+  DecodeArgs a{};
+  a.wcatT = P((void*)packed, PL.wcat); a.Ntot = PL.Ntot; a.d = d.d; a.x_bf16 = d.bf16;
+  a.w_r2 = (const float*)P((void*)packed, PL.wr2); a.pT64 = (const double*)P((void*)packed, PL.pT64);
+  a.dq = d.dq; a.dkv = d.dkv; a.rh = d.rh; a.nb = d.nb; a.rh_segs = PL.rh_segs;
+  a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.dh = d.dh; a.blk = d.blk; a.R = d.R; a.Lmax = max_positions;
+  a.maxblk = SL.maxblk; a.alpha = d.alpha; a.scale = d.scale;
+  a.x_new = x_new; a.out = out;
+  a.pos = (int*)P(state, SL.pos); a.kcache = P(state, SL.kc); a.vcache = P(state, SL.vc);
+  a.ema = (float*)P(state, SL.ema); a.blk_sum = (float*)P(state, SL.blk_sum); a.blk_p = (float*)P(state, SL.blk_p);
+  a.blk_eps = (float*)P(state, SL.blk_eps); a.blk_x = (double*)P(state, SL.blk_x);
+  a.summ = (float*)P(state, SL.summ); a.scode = (uint32_t*)P(state, SL.scode);
+  a.y = (float*)P(ws, W.y); a.qf = (float*)P(ws, W.qf); a.part = (float*)P(ws, W.part); a.nsplit = W.nsplit;
+  a.status = status_ptr();
+  prof_begin();
+  a.prof = g_prof.on ? g_prof.ev : nullptr;
+  CUDA_TRY(decode_step(a, (cudaStream_t)stream));
+  if (g_prof.on) g_prof.n = 5;
+  return MKA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,303 @@
+// Dense projections of the FastMKA layer: X [T, d] times the packed weight
+// matrix [W_q | W_k | W_v | W_q W_r1 | P]^T (notes §2-§3 of the MKA paper:
+// q = X W_q feeds the router and the attention, K/V come from X_fused W_k,v,
+// which is linear in X's projections).  Both operands are K-major ("TN").
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mka {
+
+// ---------------------------------------------------------------- epilogue store
+__device__ __forceinline__ void ep_store1(const Epilogue& ep, int m, int n, float v) {
+#pragma unroll
+  for (int s = 0; s < kMaxSegs; ++s) {
+    if (s >= ep.nseg) break;
+    const OutSeg& g = ep.seg[s];
+    if (n >= g.n_begin && n < g.n_end) {
+      size_t off = (size_t)m * g.ld + (n - g.n_begin);
+      if (g.is_bf16) ((bf16*)g.ptr)[off] = __float2bfloat16_rn(v);
+      else ((float*)g.ptr)[off] = v;
+      return;
+    }
+  }
+}
+
+// Stores columns n and n+1 of row m (n+1 may fall in the next segment or past N).
+__device__ __forceinline__ void ep_store2(const Epilogue& ep, int m, int n, float v0, float v1, int M, int N) {
+  if (m >= M) return;
+#pragma unroll
+  for (int s = 0; s < kMaxSegs; ++s) {
+    if (s >= ep.nseg) break;
+    const OutSeg& g = ep.seg[s];
+    if (n >= g.n_begin && n < g.n_end) {
+      size_t off = (size_t)m * g.ld + (n - g.n_begin);
+      if (n + 1 < g.n_end && (off & 1) == 0) {
+        if (g.is_bf16) *(__nv_bfloat162*)((bf16*)g.ptr + off) = __floats2bfloat162_rn(v0, v1);
+        else *(float2*)((float*)g.ptr + off) = make_float2(v0, v1);
+        return;
+      }
+      if (g.is_bf16) ((bf16*)g.ptr)[off] = __float2bfloat16_rn(v0);
+      else ((float*)g.ptr)[off] = v0;
+      if (n + 1 < N) ep_store1(ep, m, n + 1, v1);
+      return;
+    }
+  }
+  if (n + 1 < N) ep_store1(ep, m, n + 1, v1);
+}
+
+// ---------------------------------------------------------------- bf16 tensor-core GEMM (mma.sync)
+namespace tc {
+constexpr int BM = 128, BN = 128, BK = 64, STAGES = 3, NT = 256;
+constexpr int SMEM = STAGES * (BM + BN) * BK * 2;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N> __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+__device__ __forceinline__ void ldsm_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Tile rows are BK = 64 bf16 = 128 B = 8 chunks of 16 B; chunk c of row r lives at c ^ (r & 7).
+__device__ __forceinline__ int swz(int r, int c) { return r * BK + ((c ^ (r & 7)) << 3); }
+
+__global__ void __launch_bounds__(NT) gemm_tn_bf16_kernel(const bf16* __restrict__ A, int lda,
+                                                          const bf16* __restrict__ B, int ldb, int M, int N, int K,
+                                                          Epilogue ep) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  bf16* sA = (bf16*)smem_raw;
+  bf16* sB = sA + STAGES * BM * BK;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int wm = warp >> 2, wn = warp & 3;  // 2 x 4 warps, warp tile 64 x 32
+  const int KT = (K + BK - 1) / BK;
+
+  auto load_stage = [&](int stage, int kt) {
+    bf16* a = sA + stage * BM * BK;
+    bf16* b = sB + stage * BN * BK;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int c = tid + i * NT, r = c >> 3, ch = c & 7;
+      int gk = kt * BK + ch * 8;
+      int gm = m0 + r;
+      bool ok = gm < M && gk < K;
+      cp_async16(smem_u32(a + swz(r, ch)), ok ? (const void*)(A + (size_t)gm * lda + gk) : (const void*)A, ok ? 16 : 0);
+      int gn = n0 + r;
+      ok = gn < N && gk < K;
+      cp_async16(smem_u32(b + swz(r, ch)), ok ? (const void*)(B + (size_t)gn * ldb + gk) : (const void*)B, ok ? 16 : 0);
+    }
+  };
+
+  float acc[4][4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[i][j][k] = 0.f;
+
+#pragma unroll
+  for (int s = 0; s < STAGES - 1; ++s) {
+    if (s < KT) load_stage(s, s);
+    cp_commit();
+  }
+  for (int kt = 0; kt < KT; ++kt) {
+    cp_wait<STAGES - 2>();
+    __syncthreads();
+    int nk = kt + STAGES - 1;
+    if (nk < KT) load_stage(nk % STAGES, nk);
+    cp_commit();
+    const bf16* a = sA + (kt % STAGES) * BM * BK;
+    const bf16* b = sB + (kt % STAGES) * BN * BK;
+#pragma unroll
+    for (int kk = 0; kk < BK / 16; ++kk) {
+      uint32_t af[4][4], bfr[4][2];
+#pragma unroll
+      for (int mi = 0; mi < 4; ++mi) {
+        int r = wm * 64 + mi * 16 + (lane & 15);
+        int ch = kk * 2 + (lane >> 4);
+        ldsm_x4(af[mi][0], af[mi][1], af[mi][2], af[mi][3], smem_u32(a + swz(r, ch)));
+      }
+#pragma unroll
+      for (int nj = 0; nj < 2; ++nj) {
+        int r = wn * 32 + nj * 16 + ((lane >> 4) << 3) + (lane & 7);
+        int ch = kk * 2 + ((lane >> 3) & 1);
+        ldsm_x4(bfr[2 * nj][0], bfr[2 * nj][1], bfr[2 * nj + 1][0], bfr[2 * nj + 1][1], smem_u32(b + swz(r, ch)));
+      }
+#pragma unroll
+      for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) mma_bf16(acc[mi][ni], af[mi], bfr[ni]);
+    }
+  }
+  cp_wait<0>();
+
+#pragma unroll
+  for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni) {
+      int m = m0 + wm * 64 + mi * 16 + (lane >> 2);
+      int n = n0 + wn * 32 + ni * 8 + (lane & 3) * 2;
+      if (n < N) {
+        ep_store2(ep, m, n, acc[mi][ni][0], acc[mi][ni][1], M, N);
+        ep_store2(ep, m + 8, n, acc[mi][ni][2], acc[mi][ni][3], M, N);
+      }
+    }
+}
+}  // namespace tc
+
+cudaError_t gemm_tn_bf16(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
+                         cudaStream_t s) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  cudaError_t e = set_max_smem(tc::gemm_tn_bf16_kernel, tc::SMEM, s);
+  if (e != cudaSuccess) return e;
+  dim3 grid((N + tc::BN - 1) / tc::BN, (M + tc::BM - 1) / tc::BM);
+  tc::gemm_tn_bf16_kernel<<<grid, tc::NT, tc::SMEM, s>>>((const bf16*)A, lda, (const bf16*)B, ldb, M, N, K, ep);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- FFMA GEMM (float32 workloads, weight folding)
+namespace ff {
+constexpr int BM = 64, BN = 64, BK = 16, NT = 256;
+
+template <typename TA, typename TB>
+__global__ void __launch_bounds__(NT) gemm_tn_ffma_kernel(const TA* __restrict__ A, int lda, const TB* __restrict__ B,
+                                                          int ldb, int M, int N, int K, Epilogue ep) {
+  __shared__ float As[BK][BM + 4];
+  __shared__ float Bs[BK][BN + 4];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += BK) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int e = tid + i * NT, r = e >> 4, kk = e & 15;
+      int gm = m0 + r, gn = n0 + r, gk = k0 + kk;
+      As[kk][r] = (gm < M && gk < K) ? to_f<TA>(A[(size_t)gm * lda + gk]) : 0.f;
+      Bs[kk][r] = (gn < N && gk < K) ? to_f<TB>(B[(size_t)gn * ldb + gk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; j += 2) {
+      int m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
+      if (n < N) ep_store2(ep, m, n, acc[i][j], acc[i][j + 1], M, N);
+    }
+}
+}  // namespace ff
+
+cudaError_t gemm_tn_ffma(const void* A, int lda, int a_bf16, const void* B, int ldb, int b_bf16, int M, int N, int K,
+                         const Epilogue& ep, cudaStream_t s) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  dim3 grid((N + ff::BN - 1) / ff::BN, (M + ff::BM - 1) / ff::BM);
+  if (a_bf16 && b_bf16)
+    ff::gemm_tn_ffma_kernel<bf16, bf16><<<grid, ff::NT, 0, s>>>((const bf16*)A, lda, (const bf16*)B, ldb, M, N, K, ep);
+  else if (!a_bf16 && !b_bf16)
+    ff::gemm_tn_ffma_kernel<float, float><<<grid, ff::NT, 0, s>>>((const float*)A, lda, (const float*)B, ldb, M, N, K, ep);
+  else if (a_bf16)
+    ff::gemm_tn_ffma_kernel<bf16, float><<<grid, ff::NT, 0, s>>>((const bf16*)A, lda, (const float*)B, ldb, M, N, K, ep);
+  else
+    ff::gemm_tn_ffma_kernel<float, bf16><<<grid, ff::NT, 0, s>>>((const float*)A, lda, (const bf16*)B, ldb, M, N, K, ep);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- small packing kernels
+template <typename Tin, typename Tout>
+__global__ void transpose_kernel(const Tin* __restrict__ in, int rows, int cols, int ld_in, Tout* __restrict__ out,
+                                 int ld_out) {
+  __shared__ float tile[32][33];
+  int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = to_f<Tin>(in[(size_t)r * ld_in + c]);
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) out[(size_t)c * ld_out + r] = (Tout)tile[threadIdx.x][i];
+  }
+}
+template <typename Tin>
+__global__ void transpose_bf16_out_kernel(const Tin* __restrict__ in, int rows, int cols, int ld_in,
+                                          bf16* __restrict__ out, int ld_out) {
+  __shared__ float tile[32][33];
+  int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = to_f<Tin>(in[(size_t)r * ld_in + c]);
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) out[(size_t)c * ld_out + r] = __float2bfloat16_rn(tile[threadIdx.x][i]);
+  }
+}
+
+cudaError_t transpose(const void* in, int rows, int cols, int ld_in, void* out, int ld_out, int elem, int to_f64,
+                      cudaStream_t s) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32), block(32, 8);
+  if (to_f64) {
+    if (elem == 2) transpose_kernel<bf16, double><<<grid, block, 0, s>>>((const bf16*)in, rows, cols, ld_in, (double*)out, ld_out);
+    else transpose_kernel<float, double><<<grid, block, 0, s>>>((const float*)in, rows, cols, ld_in, (double*)out, ld_out);
+  } else if (elem == 2) {
+    transpose_bf16_out_kernel<bf16><<<grid, block, 0, s>>>((const bf16*)in, rows, cols, ld_in, (bf16*)out, ld_out);
+  } else {
+    transpose_kernel<float, float><<<grid, block, 0, s>>>((const float*)in, rows, cols, ld_in, (float*)out, ld_out);
+  }
+  return cudaGetLastError();
+}
+
+__global__ void split_hi_lo_kernel(const float* __restrict__ w, int n, bf16* __restrict__ hi, bf16* __restrict__ lo) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    float v = w[i];
+    bf16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+cudaError_t split_hi_lo(const float* w, int n, void* hi, void* lo, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  split_hi_lo_kernel<<<(n + 255) / 256, 256, 0, s>>>(w, n, (bf16*)hi, (bf16*)lo);
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void widen_kernel(const T* __restrict__ in, int n, float* __restrict__ out) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = to_f<T>(in[i]);
+}
+cudaError_t widen_f32(const void* in, int n, int in_bf16, float* out, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  if (in_bf16) widen_kernel<bf16><<<(n + 255) / 256, 256, 0, s>>>((const bf16*)in, n, out);
+  else widen_kernel<float><<<(n + 255) / 256, 256, 0, s>>>((const float*)in, n, out);
+  return cudaGetLastError();
+}
+
+}  // namespace mka

@@ -1,0 +1,123 @@
+// Internal launch interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mka {
+
+// One column range of a GEMM output and where it is stored.
+struct OutSeg {
+  int n_begin, n_end;  // [n_begin, n_end) of the GEMM's N
+  void* ptr;           // element (m, n) goes to ptr[m * ld + (n - n_begin)]
+  int ld;
+  int is_bf16;         // 1: bf16 store, 0: float32 store
+};
+constexpr int kMaxSegs = 6;
+struct Epilogue {
+  int nseg;
+  OutSeg seg[kMaxSegs];
+};
+
+// C[M, N] = A[M, K] * B[N, K]^T (both operands K-major), float32 accumulation.
+// bf16 operands on tensor cores; `f32` variants use CUDA-core FFMA (no TF32).
+cudaError_t gemm_tn_bf16(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
+                         cudaStream_t s);
+cudaError_t gemm_tn_ffma(const void* A, int lda, int a_bf16, const void* B, int ldb, int b_bf16, int M, int N, int K,
+                         const Epilogue& ep, cudaStream_t s);
+
+// out[c, r] = in[r, c] for in [rows, cols] (row stride ld_in), out row stride ld_out.
+// elem: 2 (bf16), 4 (f32).  to_f64 widens to float64 output instead.
+cudaError_t transpose(const void* in, int rows, int cols, int ld_in, void* out, int ld_out, int elem, int to_f64,
+                      cudaStream_t s);
+// Split float32 w into bf16 hi = rn(w) and lo = rn(w - hi).
+cudaError_t split_hi_lo(const float* w, int n, void* hi, void* lo, cudaStream_t s);
+// Copy/widen [n] elements of type (bf16|f32) to float32.
+cudaError_t widen_f32(const void* in, int n, int in_bf16, float* out, cudaStream_t s);
+
+// ---------------------------------------------------------------- memory / routing kernels
+struct HashArgs {
+  const float* proj;     // [T, ldp] float32 token projections (column k = bit k)
+  int ldp;
+  const void* x;         // [T, d] token rows (dtype) for exact refinement
+  int x_bf16;
+  const double* pT64;    // [nb, d] float64 P^T
+  int d, nb, K;          // K: length of the dot products that produced proj
+};
+
+cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, float* lam,
+                        cudaStream_t s);
+cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, float* eps, cudaStream_t s);
+cudaError_t summary_codes(const HashArgs& a, int B, int S, int nblk, int blk, const float* eps, uint32_t* codes,
+                          int code_bstride, cudaStream_t s);
+// Per full block j of each sequence: bsum = sum of its rows, bend = EMA end state from a zero carry.
+// x: [B*S, ld] (bf16 or float32), first `width` columns.  bsum[b*bsum_bstride + j*width + c].
+cudaError_t block_reduce(const void* x, int x_bf16, int ld, int width, int B, int S, int nblk, int blk, float alpha,
+                         float* bsum, long long bsum_bstride, float* bend, cudaStream_t s);
+cudaError_t ema_carry(const float* bend, int width, int B, int nblk, float alpha_pow_b, const float* carry_in,
+                      float* carry, cudaStream_t s);
+cudaError_t recall_select(const uint32_t* tok_codes, const uint32_t* blk_codes, int blk_codes_bstride, int B, int S,
+                          int nblk, int blk, int R, int* idx, int* count, cudaStream_t s);
+
+struct FuseArgs {
+  const float* xkv; int ld;       // [B*S, ld] float32 projected rows (K part then V part)
+  int width;                      // 2*dkv
+  const float* lam;               // [B*S, 3]
+  const int* idx; const int* count; int R;
+  const float* bsum; long long bsum_bstride;  // [B][nblk][width] block SUMS
+  const float* carry;             // [B][nblk+1][width] EMA value at each block start
+  int B, S, nblk, blk, dkv;
+  float alpha;
+  void* k_out; void* v_out; long long kv_bstride; int out_bf16;  // [B][.. rows][dkv]
+  float* state_ema;               // [B][width] <- M2[S] (nullable)
+};
+cudaError_t fuse_kv(const FuseArgs& a, cudaStream_t s);
+
+// Standalone d-space pieces.
+cudaError_t ema_apply(const void* x, int x_bf16, int width, int B, int S, int nblk, int blk, float alpha,
+                      const float* carry, float* m2, float* carry_out, cudaStream_t s);
+cudaError_t gather_mean(const int* idx, const int* count, int R, const float* bsum, int nblk, int width, int blk,
+                        int B, int S, float* m3, cudaStream_t s);
+
+// State tail after a prefill: the unfinished block's sums.
+cudaError_t prefill_tail_state(const float* xkv, int ld, int width, const float* proj, int ldp, int nb,
+                               const float* eps, const void* x, int x_bf16, int d, int B, int S, int blk,
+                               float* blk_sum, float* blk_p, float* blk_eps, double* blk_x, int* pos,
+                               cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+struct AttnArgs {
+  const void* q; long long q_bstride; int q_ld;      // q[b][t][h*dh + i]: b*q_bstride + t*q_ld + h*dh + i
+  const void* k; const void* v; long long kv_bstride; int kv_ld;  // k[b][j][g*dh + i]
+  void* o; long long o_bstride; int o_ld;
+  int B, S, Hq, Hkv, dh;
+  float scale;
+};
+cudaError_t attention_prefill(const AttnArgs& a, int bf16, cudaStream_t s);
+
+// ---------------------------------------------------------------- decode
+struct DecodeArgs {
+  // packed weights
+  const void* wcatT; int Ntot; int d; int x_bf16;
+  const float* w_r2; const double* pT64;
+  // layout of the fused projection row
+  int dq, dkv, rh, nb, rh_segs;  // rh_segs: 2 for bf16 (hi+lo), 1 for f32
+  int B, Hq, Hkv, dh, blk, R, Lmax, maxblk;
+  float alpha, scale;
+  const void* x_new;             // [B, d]
+  void* out;                     // [B, dq]
+  // state
+  int* pos; void* kcache; void* vcache; float* ema; float* blk_sum; float* blk_p; float* blk_eps; double* blk_x;
+  float* summ; uint32_t* scode;
+  // scratch
+  float* y;                      // [B, Ntot] projection row
+  float* qf;                     // [B, dq] float32 query
+  float* part;                   // split-KV partials
+  int nsplit;
+  int* status;
+  cudaEvent_t* prof;             // 5 events around the 4 stages, or NULL
+};
+cudaError_t decode_step(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace mka

@@ -1,0 +1,502 @@
+// Router tail, L2 session EMA, L3 long-term recall and the route-fuse of the
+// FastMKA layer ("MKA: Memory-Keyed Attention for Efficient Long-Context
+// Reasoning", paper-notes page §1-§3).  All bandwidth-bound: float4 row
+// streaming, warp-level reductions, per-block parallel scans.
+//
+// Projected space: K = X_fused W_k = l1 (X W_k) + l2 (M2 W_k) + l3 (M3 W_k), and
+// both M2 (an EMA) and M3 (a mean of block means) commute with the projection,
+// so the session and long-term memories run on the 2*dkv projected columns of
+// each token instead of its d_model columns.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mka {
+
+// ---------------------------------------------------------------- router tail
+// lambda = softmax(GELU(h) W_r2) per token (notes §2); h = h1 (+ h2) when the
+// first layer was applied as a bf16 hi/lo pair.
+__global__ void router_tail_kernel(const float* __restrict__ h1, const float* __restrict__ h2, int ldh, int T, int rh,
+                                   const float* __restrict__ w_r2, float* __restrict__ lam) {
+  extern __shared__ float sw[];
+  for (int i = threadIdx.x; i < rh * 3; i += blockDim.x) sw[i] = w_r2[i];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= T) return;
+  float z0 = 0.f, z1 = 0.f, z2 = 0.f;
+  const float* a = h1 + (size_t)t * ldh;
+  const float* b = h2 ? h2 + (size_t)t * ldh : nullptr;
+  for (int j = lane; j < rh; j += 32) {
+    float h = a[j];
+    if (b) h += b[j];
+    float g = gelu_erf(h);
+    z0 = fmaf(g, sw[j * 3 + 0], z0);
+    z1 = fmaf(g, sw[j * 3 + 1], z1);
+    z2 = fmaf(g, sw[j * 3 + 2], z2);
+  }
+  z0 = warp_sum(z0);
+  z1 = warp_sum(z1);
+  z2 = warp_sum(z2);
+  if (lane == 0) {
+    float m = fmaxf(z0, fmaxf(z1, z2));
+    float e0 = expf(z0 - m), e1 = expf(z1 - m), e2 = expf(z2 - m);
+    float inv = 1.f / (e0 + e1 + e2);
+    lam[(size_t)t * 3 + 0] = e0 * inv;
+    lam[(size_t)t * 3 + 1] = e1 * inv;
+    lam[(size_t)t * 3 + 2] = e2 * inv;
+  }
+}
+
+cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, float* lam,
+                        cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  router_tail_kernel<<<(T + 7) / 8, 256, rh * 3 * sizeof(float), s>>>(h1, h2, ldh, T, rh, w_r2, lam);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- L3 sign codes
+// The float32 projection p = x . P_k carries a rounding error far below
+// eps = K * 2^-20 * rms_k(p) (K * 2^-23 * |partial sum| is the worst-case
+// sequential bound; rms_k(p) estimates the partial sums' scale).  Signs of
+// projections within eps of zero are decided again from an exact float64 dot
+// product, so every code bit equals the sign of the exact projection.
+template <typename T>
+__device__ __forceinline__ double dot_row_f64(const T* __restrict__ x, const double* __restrict__ p, int d, int lane) {
+  double acc = 0.0;
+  for (int i = lane; i < d; i += 32) acc = fma(to_d<T>(x[i]), p[i], acc);
+  return warp_sum_d(acc);
+}
+
+template <typename T>
+__global__ void token_codes_kernel(HashArgs a, int T_, uint32_t* __restrict__ codes, float* __restrict__ eps) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T_) return;
+  float p = lane < a.nb ? a.proj[(size_t)t * a.ldp + lane] : 0.f;
+  float rms = sqrtf(warp_sum(p * p) / (float)a.nb);
+  float e = (float)a.K * 0x1p-20f * rms;
+  bool bit = p > 0.f;
+  unsigned doubt = __ballot_sync(0xffffffffu, lane < a.nb && fabsf(p) <= e);
+  const T* xr = (const T*)a.x + (size_t)t * a.d;
+  while (doubt) {
+    int k = __ffs(doubt) - 1;
+    doubt &= doubt - 1;
+    double v = dot_row_f64<T>(xr, a.pT64 + (size_t)k * a.d, a.d, lane);
+    if (lane == k) bit = v > 0.0;
+  }
+  unsigned code = __ballot_sync(0xffffffffu, bit && lane < a.nb);
+  if (lane == 0) {
+    codes[t] = code;
+    if (eps) eps[t] = e;
+  }
+}
+
+cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, float* eps, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  if (a.x_bf16) token_codes_kernel<bf16><<<(T + 7) / 8, 256, 0, s>>>(a, T, codes, eps);
+  else token_codes_kernel<float><<<(T + 7) / 8, 256, 0, s>>>(a, T, codes, eps);
+  return cudaGetLastError();
+}
+
+// Block code: bits of sum_t p_t over the block (the sign of the block mean's
+// projection).  The float32 sum's error is below 2 * sum_t eps_t; in doubt, the
+// exact float64 block sum of X in d_model space is formed and projected.
+template <typename T>
+__global__ void summary_codes_kernel(HashArgs a, int S, int nblk, int blk, const float* __restrict__ eps,
+                                     uint32_t* __restrict__ codes, int code_bstride) {
+  extern __shared__ double sx[];  // [d]
+  __shared__ float sp[8][32];
+  __shared__ float se[8];
+  __shared__ unsigned s_doubt, s_code;
+  const int bi = blockIdx.y, j = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t t0 = (size_t)bi * S + (size_t)j * blk;
+  float acc = 0.f, eacc = 0.f;
+  for (int r = warp; r < blk; r += 8) {
+    if (lane < a.nb) acc += a.proj[(t0 + r) * a.ldp + lane];
+    if (lane == 0) eacc += eps[t0 + r];
+  }
+  sp[warp][lane] = acc;
+  if (lane == 0) se[warp] = eacc;
+  __syncthreads();
+  if (warp == 0) {
+    float tot = 0.f, et = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      tot += sp[w][lane];
+      et += se[w];
+    }
+    et *= 2.f;
+    unsigned doubt = __ballot_sync(0xffffffffu, lane < a.nb && fabsf(tot) <= et);
+    unsigned code = __ballot_sync(0xffffffffu, lane < a.nb && tot > 0.f);
+    if (lane == 0) {
+      s_doubt = doubt;
+      s_code = code & ~doubt;
+    }
+  }
+  __syncthreads();
+  unsigned doubt = s_doubt;
+  if (doubt) {
+    const T* x = (const T*)a.x;
+    for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
+      double s = 0.0;
+      for (int r = 0; r < blk; ++r) s += to_d<T>(x[(t0 + r) * a.d + i]);
+      sx[i] = s;
+    }
+    __syncthreads();
+    for (int k = warp; k < a.nb; k += 8) {
+      if (!((doubt >> k) & 1u)) continue;
+      double v = 0.0;
+      for (int i = lane; i < a.d; i += 32) v = fma(sx[i], a.pT64[(size_t)k * a.d + i], v);
+      v = warp_sum_d(v);
+      if (lane == 0 && v > 0.0) atomicOr(&s_code, 1u << k);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) codes[(size_t)bi * code_bstride + j] = s_code;
+}
+
+cudaError_t summary_codes(const HashArgs& a, int B, int S, int nblk, int blk, const float* eps, uint32_t* codes,
+                          int code_bstride, cudaStream_t s) {
+  if (B <= 0 || nblk <= 0) return cudaSuccess;
+  dim3 grid(nblk, B);
+  size_t sm = (size_t)a.d * sizeof(double);
+  if (a.x_bf16) {
+    set_max_smem(summary_codes_kernel<bf16>, sm, s);
+    summary_codes_kernel<bf16><<<grid, 256, sm, s>>>(a, S, nblk, blk, eps, codes, code_bstride);
+  } else {
+    set_max_smem(summary_codes_kernel<float>, sm, s);
+    summary_codes_kernel<float><<<grid, 256, sm, s>>>(a, S, nblk, blk, eps, codes, code_bstride);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- block sums + EMA end states
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+  static __device__ __forceinline__ float4 load(const float* p) { return *(const float4*)p; }
+};
+template <> struct Vec4<bf16> {
+  static __device__ __forceinline__ float4 load(const bf16* p) {
+    uint2 u = *(const uint2*)p;
+    __nv_bfloat162 a = *(__nv_bfloat162*)&u.x, b = *(__nv_bfloat162*)&u.y;
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+};
+__device__ __forceinline__ float4 f4_fma(float a, float4 x, float4 y) {
+  return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
+}
+__device__ __forceinline__ float4 f4_add(float4 x, float4 y) { return make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w); }
+__device__ __forceinline__ float4 f4_scale(float a, float4 x) { return make_float4(a * x.x, a * x.y, a * x.z, a * x.w); }
+// One EMA step m <- a*m + (1-a)*x.
+__device__ __forceinline__ float4 ema_step(float al, float om, float4 m, float4 x) {
+  return make_float4(fmaf(al, m.x, om * x.x), fmaf(al, m.y, om * x.y), fmaf(al, m.z, om * x.z), fmaf(al, m.w, om * x.w));
+}
+
+constexpr int kRG = 4;  // row groups per block in block_reduce
+
+template <typename T>
+__global__ void __launch_bounds__(256) block_reduce_kernel(const T* __restrict__ x, int ld, int width, int S, int nblk,
+                                                            int blk, float alpha, float* __restrict__ bsum,
+                                                            long long bsum_bstride, float* __restrict__ bend) {
+  __shared__ float4 ssum[kRG][64], send[kRG][64];
+  const int bi = blockIdx.z, j = blockIdx.y;
+  const int cl = threadIdx.x & 63, rg = threadIdx.x >> 6;
+  const int c = (blockIdx.x * 64 + cl) * 4;
+  const int per = (blk + kRG - 1) / kRG;
+  const int ra = min(rg * per, blk), rb = min(ra + per, blk);
+  const float om = 1.f - alpha;
+  float4 s = make_float4(0, 0, 0, 0), e = s;
+  if (c < width) {
+    const T* p = x + ((size_t)bi * S + (size_t)j * blk) * ld + c;
+#pragma unroll 4
+    for (int r = ra; r < rb; ++r) {
+      float4 v = Vec4<T>::load(p + (size_t)r * ld);
+      s = f4_add(s, v);
+      e = ema_step(alpha, om, e, v);
+    }
+  }
+  ssum[rg][cl] = s;
+  send[rg][cl] = e;
+  __syncthreads();
+  if (rg == 0 && c < width) {
+    float4 S4 = ssum[0][cl], E4 = send[0][cl];
+    for (int g = 1; g < kRG; ++g) {
+      int ga = min(g * per, blk), gb = min(ga + per, blk);
+      float ap = 1.f;
+      for (int i = ga; i < gb; ++i) ap *= alpha;  // a^(rows of group g)
+      S4 = f4_add(S4, ssum[g][cl]);
+      E4 = f4_add(f4_scale(ap, E4), send[g][cl]);
+    }
+    if (bsum) *(float4*)(bsum + (size_t)bi * bsum_bstride + (size_t)j * width + c) = S4;
+    if (bend) *(float4*)(bend + ((size_t)bi * nblk + j) * width + c) = E4;
+  }
+}
+
+cudaError_t block_reduce(const void* x, int x_bf16, int ld, int width, int B, int S, int nblk, int blk, float alpha,
+                         float* bsum, long long bsum_bstride, float* bend, cudaStream_t s) {
+  if (B <= 0 || nblk <= 0) return cudaSuccess;
+  dim3 grid((width / 4 + 63) / 64, nblk, B);
+  if (x_bf16)
+    block_reduce_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)x, ld, width, S, nblk, blk, alpha, bsum, bsum_bstride, bend);
+  else
+    block_reduce_kernel<float><<<grid, 256, 0, s>>>((const float*)x, ld, width, S, nblk, blk, alpha, bsum, bsum_bstride, bend);
+  return cudaGetLastError();
+}
+
+// carry[b][0] = carry_in (or 0); carry[b][j+1] = a^b * carry[b][j] + bend[b][j].
+__global__ void ema_carry_kernel(const float* __restrict__ bend, int width, int B, int nblk, float apb,
+                                 const float* __restrict__ carry_in, float* __restrict__ carry) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * width) return;
+  int bi = i / width, c = i % width;
+  float cur = carry_in ? carry_in[i] : 0.f;
+  float* out = carry + (size_t)bi * (nblk + 1) * width + c;
+  const float* e = bend + (size_t)bi * nblk * width + c;
+  out[0] = cur;
+#pragma unroll 8
+  for (int j = 0; j < nblk; ++j) {
+    cur = fmaf(apb, cur, e[(size_t)j * width]);
+    out[(size_t)(j + 1) * width] = cur;
+  }
+}
+
+cudaError_t ema_carry(const float* bend, int width, int B, int nblk, float alpha_pow_b, const float* carry_in,
+                      float* carry, cudaStream_t s) {
+  int n = B * width;
+  if (n <= 0) return cudaSuccess;
+  ema_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(bend, width, B, nblk, alpha_pow_b, carry_in, carry);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- top-R recall
+// One warp per token.  Distances take at most 33 values, so the (distance,
+// index) order is built by counting: a histogram gives each distance's first
+// output slot, and a pass in index order places equal-distance blocks by rank
+// (__match_any_sync groups the lanes that share a distance).  Deterministic, no
+// sort, every output position written exactly once.
+__global__ void __launch_bounds__(256) recall_kernel(const uint32_t* __restrict__ tok, const uint32_t* __restrict__ blkc,
+                                                     int bstride, int B, int S, int nblk, int blk, int R,
+                                                     int* __restrict__ idx, int* __restrict__ count) {
+  __shared__ int base[8][34];
+  __shared__ int run[8][34];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long tg = (long long)blockIdx.x * 8 + w;
+  if (tg >= (long long)B * S) return;
+  const int bi = (int)(tg / S), t = (int)(tg % S);
+  const int n = min(t / blk, nblk);
+  const int cnt = min(R, n);
+  const uint32_t code = tok[tg];
+  const uint32_t* bc = blkc + (size_t)bi * bstride;
+  int* out = idx + tg * R;
+  for (int i = lane; i < 34; i += 32) {
+    base[w][i] = 0;
+    run[w][i] = 0;
+  }
+  __syncwarp();
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    int j = j0 + lane;
+    if (j < n) atomicAdd(&base[w][__popc(code ^ bc[j])], 1);
+  }
+  __syncwarp();
+  if (lane == 0) {
+    int acc = 0;
+    for (int dd = 0; dd < 34; ++dd) {
+      int h = base[w][dd];
+      base[w][dd] = acc;
+      acc += h;
+    }
+  }
+  __syncwarp();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    int j = j0 + lane;
+    bool valid = j < n;
+    int dist = valid ? __popc(code ^ bc[j]) : 64 + lane;
+    unsigned grp = __match_any_sync(0xffffffffu, dist);
+    int rank = __popc(grp & lt);
+    int pos = valid ? base[w][dist] + run[w][dist] + rank : R;
+    __syncwarp();
+    if (valid && pos < R) out[pos] = j;
+    if (valid && rank == 0) run[w][dist] += __popc(grp);
+    __syncwarp();
+  }
+  for (int p = cnt + lane; p < R; p += 32) out[p] = -1;
+  if (lane == 0 && count) count[tg] = cnt;
+}
+
+cudaError_t recall_select(const uint32_t* tok_codes, const uint32_t* blk_codes, int blk_codes_bstride, int B, int S,
+                          int nblk, int blk, int R, int* idx, int* count, cudaStream_t s) {
+  long long T = (long long)B * S;
+  if (T <= 0) return cudaSuccess;
+  recall_kernel<<<(unsigned)((T + 7) / 8), 256, 0, s>>>(tok_codes, blk_codes, blk_codes_bstride, B, S, nblk, blk, R, idx,
+                                                        count);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- route-fuse -> K, V
+// notes §3: X_fused = l1*X + l2*M2 + l3*M3, applied to the projected columns.
+// One CTA per (sequence, block, 256 columns); rows of the block run in order
+// (the EMA recurrence), starting from the block's carried EMA value.
+template <typename OutT>
+__device__ __forceinline__ void store4(OutT* p, float4 v);
+template <> __device__ __forceinline__ void store4<float>(float* p, float4 v) { *(float4*)p = v; }
+template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *(uint32_t*)&a;
+  u.y = *(uint32_t*)&b;
+  *(uint2*)p = u;
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(64) fuse_kernel(FuseArgs a) {
+  extern __shared__ float sm[];
+  float* slam = sm;                                   // [blk*3]
+  int* sidx = (int*)(slam + a.blk * 3);               // [blk*R]
+  int* scnt = sidx + a.blk * a.R;                     // [blk]
+  const int bi = blockIdx.z, j = blockIdx.y;
+  const int r0 = j * a.blk, r1 = min(r0 + a.blk, a.S), nr = r1 - r0;
+  const size_t tg0 = (size_t)bi * a.S + r0;
+  for (int i = threadIdx.x; i < nr * 3; i += blockDim.x) slam[i] = a.lam[tg0 * 3 + i];
+  for (int i = threadIdx.x; i < nr * a.R; i += blockDim.x) sidx[i] = a.idx[tg0 * a.R + i];
+  for (int i = threadIdx.x; i < nr; i += blockDim.x) scnt[i] = a.count[tg0 + i];
+  __syncthreads();
+  const int c = (blockIdx.x * 64 + threadIdx.x) * 4;
+  if (c >= a.width) return;
+  const float om = 1.f - a.alpha;
+  float4 m2 = *(const float4*)(a.carry + ((size_t)bi * (a.nblk + 1) + j) * a.width + c);
+  const float* bs = a.bsum + (size_t)bi * a.bsum_bstride + c;
+  const bool is_k = c < a.dkv;
+  OutT* dst = (OutT*)(is_k ? a.k_out : a.v_out) + (size_t)bi * a.kv_bstride + (size_t)r0 * a.dkv + (is_k ? c : c - a.dkv);
+  const float* xp = a.xkv + tg0 * a.ld + c;
+  const float invb = 1.f / (float)a.blk;
+  for (int r = 0; r < nr; ++r) {
+    float4 x = *(const float4*)(xp + (size_t)r * a.ld);
+    int cnt = scnt[r];
+    float4 m3 = make_float4(0, 0, 0, 0);
+    for (int q = 0; q < cnt; ++q) m3 = f4_add(m3, *(const float4*)(bs + (size_t)sidx[r * a.R + q] * a.width));
+    float s3 = cnt ? invb / (float)cnt : 0.f;
+    float l0 = slam[r * 3], l1 = slam[r * 3 + 1], l2 = slam[r * 3 + 2];
+    float4 o = f4_fma(l0, x, f4_fma(l1, m2, f4_scale(l2 * s3, m3)));
+    store4<OutT>(dst + (size_t)r * a.dkv, o);
+    m2 = ema_step(a.alpha, om, m2, x);
+  }
+  if (r1 == a.S && a.state_ema) *(float4*)(a.state_ema + (size_t)bi * a.width + c) = m2;
+}
+
+cudaError_t fuse_kv(const FuseArgs& a, cudaStream_t s) {
+  if (a.B <= 0 || a.S <= 0) return cudaSuccess;
+  int nb_all = (a.S + a.blk - 1) / a.blk;
+  dim3 grid((a.width / 4 + 63) / 64, nb_all, a.B);
+  size_t sm = (size_t)a.blk * (3 * sizeof(float) + (a.R + 1) * sizeof(int));
+  if (a.out_bf16) {
+    set_max_smem(fuse_kernel<bf16>, sm, s);
+    fuse_kernel<bf16><<<grid, 64, sm, s>>>(a);
+  } else {
+    set_max_smem(fuse_kernel<float>, sm, s);
+    fuse_kernel<float><<<grid, 64, sm, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- standalone d-space pieces
+template <typename T>
+__global__ void __launch_bounds__(64) ema_apply_kernel(const T* __restrict__ x, int width, int S, int nblk, int blk,
+                                                        float alpha, const float* __restrict__ carry,
+                                                        float* __restrict__ m2, float* __restrict__ carry_out) {
+  const int bi = blockIdx.z, j = blockIdx.y;
+  const int c = (blockIdx.x * 64 + threadIdx.x) * 4;
+  if (c >= width) return;
+  const int r0 = j * blk, r1 = min(r0 + blk, S);
+  const float om = 1.f - alpha;
+  float4 m = *(const float4*)(carry + ((size_t)bi * (nblk + 1) + j) * width + c);
+  const size_t base = ((size_t)bi * S + r0) * width + c;
+  for (int r = 0; r < r1 - r0; ++r) {
+    *(float4*)(m2 + base + (size_t)r * width) = m;
+    m = ema_step(alpha, om, m, Vec4<T>::load(x + base + (size_t)r * width));
+  }
+  if (r1 == S && carry_out) *(float4*)(carry_out + (size_t)bi * width + c) = m;
+}
+
+cudaError_t ema_apply(const void* x, int x_bf16, int width, int B, int S, int nblk, int blk, float alpha,
+                      const float* carry, float* m2, float* carry_out, cudaStream_t s) {
+  if (B <= 0 || S <= 0) return cudaSuccess;
+  dim3 grid((width / 4 + 63) / 64, (S + blk - 1) / blk, B);
+  if (x_bf16) ema_apply_kernel<bf16><<<grid, 64, 0, s>>>((const bf16*)x, width, S, nblk, blk, alpha, carry, m2, carry_out);
+  else ema_apply_kernel<float><<<grid, 64, 0, s>>>((const float*)x, width, S, nblk, blk, alpha, carry, m2, carry_out);
+  return cudaGetLastError();
+}
+
+// m3[t] = (1 / (count * blk)) * sum_q bsum[idx[t][q]]  (mean of the recalled block means).
+__global__ void gather_mean_kernel(const int* __restrict__ idx, const int* __restrict__ count, int R,
+                                   const float* __restrict__ bsum, int nblk, int width, int blk, int S,
+                                   float* __restrict__ m3) {
+  const size_t tg = blockIdx.x;
+  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  if (c >= width) return;
+  const int bi = (int)(tg / S);
+  const int cnt = count[tg];
+  const float* bs = bsum + (size_t)bi * nblk * width + c;
+  float4 acc = make_float4(0, 0, 0, 0);
+  for (int q = 0; q < cnt; ++q) acc = f4_add(acc, *(const float4*)(bs + (size_t)idx[tg * R + q] * width));
+  float sc = cnt ? 1.f / ((float)cnt * (float)blk) : 0.f;
+  *(float4*)(m3 + tg * width + c) = f4_scale(sc, acc);
+}
+
+cudaError_t gather_mean(const int* idx, const int* count, int R, const float* bsum, int nblk, int width, int blk,
+                        int B, int S, float* m3, cudaStream_t s) {
+  if (B <= 0 || S <= 0) return cudaSuccess;
+  dim3 grid(B * S, (width / 4 + 127) / 128);
+  gather_mean_kernel<<<grid, 128, 0, s>>>(idx, count, R, bsum, nblk, width, blk, S, m3);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- decode state after a prefill
+template <typename T>
+__global__ void prefill_tail_kernel(const float* __restrict__ xkv, int ld, int width, const float* __restrict__ proj,
+                                    int ldp, int nb, const float* __restrict__ eps, const T* __restrict__ x, int d,
+                                    int S, int blk, float* blk_sum, float* blk_p, float* blk_eps, double* blk_x,
+                                    int* pos) {
+  const int bi = blockIdx.x;
+  const int r0 = (S / blk) * blk;  // first row of the unfinished block
+  const size_t t0 = (size_t)bi * S;
+  for (int c = threadIdx.x; c < width; c += blockDim.x) {
+    float s = 0.f;
+    for (int r = r0; r < S; ++r) s += xkv[(t0 + r) * ld + c];
+    blk_sum[(size_t)bi * width + c] = s;
+  }
+  for (int k = threadIdx.x; k < nb; k += blockDim.x) {
+    float s = 0.f;
+    for (int r = r0; r < S; ++r) s += proj[(t0 + r) * ldp + k];
+    blk_p[(size_t)bi * 32 + k] = s;
+  }
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    double s = 0.0;
+    for (int r = r0; r < S; ++r) s += to_d<T>(x[(t0 + r) * d + i]);
+    blk_x[(size_t)bi * d + i] = s;
+  }
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int r = r0; r < S; ++r) s += eps[t0 + r];
+    blk_eps[bi] = s;
+    pos[bi] = S;
+  }
+}
+
+cudaError_t prefill_tail_state(const float* xkv, int ld, int width, const float* proj, int ldp, int nb,
+                               const float* eps, const void* x, int x_bf16, int d, int B, int S, int blk,
+                               float* blk_sum, float* blk_p, float* blk_eps, double* blk_x, int* pos,
+                               cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  if (x_bf16)
+    prefill_tail_kernel<bf16><<<B, 256, 0, s>>>(xkv, ld, width, proj, ldp, nb, eps, (const bf16*)x, d, S, blk, blk_sum,
+                                                blk_p, blk_eps, blk_x, pos);
+  else
+    prefill_tail_kernel<float><<<B, 256, 0, s>>>(xkv, ld, width, proj, ldp, nb, eps, (const float*)x, d, S, blk,
+                                                 blk_sum, blk_p, blk_eps, blk_x, pos);
+  return cudaGetLastError();
+}
+
+}  // namespace mka

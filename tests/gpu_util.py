@@ -1,0 +1,96 @@
+"""Helpers for the GPU parity tests: run the CUDA path through the C ABI and
+compare it with the CPU oracle on the same seeded inputs.
+
+Tolerances (stated once, used by every parity test):
+  lambda          max relative error <= 1e-3
+  recall indices  bit-exact; a mismatch is excused only at tokens where a hash
+                  projection that decides it has |p| < 1e-4 (counted, reported)
+  float32 outputs max-abs error <= 1e-4
+  bf16 outputs    relative L2 error <= 1e-2 and max-abs error <= 3e-2
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from fastmka_inputs import FastMKAConfig, FastMKAInputs, make_inputs, to_f64
+
+LAMBDA_RTOL = 1e-3
+F32_ATOL = 1e-4
+BF16_REL_L2 = 1e-2
+BF16_ATOL = 3e-2
+
+
+def oracle_weights(inp: FastMKAInputs):
+    return oracle.weights_f64(*(to_f64(t) for t in (inp.w_q, inp.w_k, inp.w_v, inp.w_r1, inp.w_r2, inp.hash_proj)))
+
+
+def oracle_prefill(cfg: FastMKAConfig, inp: FastMKAInputs, rows=None, seq=None):
+    S = cfg.seq if seq is None else seq
+    X = inp.x[:, :S].float().numpy()
+    return oracle.fastmka_prefill(X, oracle_weights(inp), cfg.replace(seq=S), rows=rows)
+
+
+def gpu_weights(inp: FastMKAInputs, device="cuda"):
+    return {k: v.to(device) for k, v in inp.tensors().items() if k != "x"}
+
+
+def gpu_prefill(cfg: FastMKAConfig, inp: FastMKAInputs, seq=None, with_state=0, device="cuda"):
+    """Runs mka_prefill_forward; returns (O, lambda, idx, layer, state)."""
+    import route_kv_memory_b200 as mka
+    S = cfg.seq if seq is None else seq
+    c = cfg.replace(seq=S)
+    layer = mka.FastMKALayer(c, gpu_weights(inp, device), device)
+    x = inp.x[:, :S].contiguous().to(device)
+    out = torch.empty(cfg.batch, S, cfg.dq, dtype=x.dtype, device=device)
+    lam = torch.empty(cfg.batch * S, 3, dtype=torch.float32, device=device)
+    idx = torch.empty(cfg.batch, S, cfg.recall_r, dtype=torch.int32, device=device)
+    state = layer.new_state(with_state) if with_state else None
+    layer.prefill(x, out, lam, idx, state, with_state)
+    torch.cuda.synchronize()
+    assert mka.mka_status() == 0
+    return out, lam, idx, layer, state
+
+
+def check_lambda(lam_gpu: torch.Tensor, lam_ref: np.ndarray):
+    g = lam_gpu.detach().cpu().double().numpy().reshape(lam_ref.shape)
+    rel = np.abs(g - lam_ref) / np.abs(lam_ref)
+    assert rel.max() <= LAMBDA_RTOL, f"lambda max rel err {rel.max():.3e}"
+    return float(rel.max())
+
+
+def check_recall(idx_gpu: torch.Tensor, out_ref: dict, rows=None):
+    """Bit-exact recalled indices; returns (unexcused, excused) mismatching tokens."""
+    g = idx_gpu.detach().cpu().numpy().astype(np.int64).reshape(out_ref["idx"].shape)
+    ref = out_ref["idx"]
+    if rows is not None:
+        g, ref = g[:, rows], ref[:, rows]
+        exc = out_ref["excuse"][:, rows]
+    else:
+        exc = out_ref["excuse"]
+    bad = (g != ref).any(axis=-1)
+    unexcused = int((bad & ~exc).sum())
+    excused = int((bad & exc).sum())
+    assert unexcused == 0, f"{unexcused} tokens recall different blocks (excused: {excused})"
+    return unexcused, excused
+
+
+def out_errors(o_gpu: np.ndarray, o_ref: np.ndarray):
+    diff = o_gpu - o_ref
+    max_abs = float(np.abs(diff).max())
+    rel_l2 = float(np.linalg.norm(diff) / np.linalg.norm(o_ref))
+    return max_abs, rel_l2
+
+
+def check_out(o_gpu: torch.Tensor, o_ref: np.ndarray, dtype: str, rows=None):
+    g = o_gpu.detach().float().cpu().double().numpy()
+    if rows is not None:
+        g = g[:, rows]
+    g = g.reshape(o_ref.shape)
+    max_abs, rel_l2 = out_errors(g, o_ref)
+    if dtype == "f32":
+        assert max_abs <= F32_ATOL, f"f32 max-abs {max_abs:.3e}"
+    else:
+        assert rel_l2 <= BF16_REL_L2 and max_abs <= BF16_ATOL, f"bf16 rel-L2 {rel_l2:.3e} max-abs {max_abs:.3e}"
+    return max_abs, rel_l2

@@ -1,0 +1,217 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fastmka_inputs import CONFIGS, FastMKAConfig, make_inputs, sample_rows, to_f64
+from gpu_util import (check_lambda, check_out, check_recall, gpu_prefill, gpu_weights, oracle_prefill,
+                      oracle_weights, out_errors, F32_ATOL)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mka():
+    import route_kv_memory_b200 as m
+    return m
+
+
+def small(name, dtype, **kw):
+    base = dict(batch=1, seq=256, d_model=256, n_q_heads=4, n_kv_heads=2, d_head=64, router_hidden=64, alpha=0.9,
+                block=32, recall_r=2, hash_bits=16, dtype=dtype, seed=100)
+    base.update(kw)
+    return FastMKAConfig(name, **base)
+
+
+# ------------------------------------------------------------------ whole layer
+def test_tiny_f32_layer():
+    cfg = CONFIGS["tiny_f32"]
+    inp = make_inputs(cfg)
+    ref = oracle_prefill(cfg, inp)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    check_recall(idx, ref)
+    max_abs, _ = check_out(out, ref["O"], "f32")
+    print(f"tiny_f32: O max-abs {max_abs:.2e}")
+
+
+EDGE = [
+    small("f32_s1", "f32", seq=1),
+    small("f32_s31", "f32", seq=31),
+    small("f32_s33", "f32", seq=33, seed=5),
+    small("f32_ragged", "f32", seq=250, batch=3, seed=6),
+    small("f32_alpha0", "f32", alpha=0.0, seed=7),
+    small("f32_alpha_half", "f32", alpha=0.5, seed=8),
+    small("f32_alpha_999", "f32", alpha=0.999, seed=9),
+    small("f32_mha_dh128", "f32", n_q_heads=2, n_kv_heads=2, d_head=128, seed=10),
+    small("f32_block_ge_seq", "f32", seq=100, block=128, seed=11),
+    small("f32_big_r", "f32", seq=200, block=8, recall_r=40, hash_bits=5, seed=12),
+    small("bf16_ragged_dh64", "bf16", seq=300, block=64, seed=13),
+    small("bf16_g8_dh128", "bf16", seq=1000, n_q_heads=8, n_kv_heads=1, d_head=128, router_hidden=256, block=128,
+          recall_r=8, hash_bits=32, seed=14),
+    small("bf16_b2_s129", "bf16", batch=2, seq=129, n_q_heads=4, n_kv_heads=4, d_head=128, seed=15),
+    small("bf16_s1", "bf16", seq=1, d_head=128, seed=16),
+]
+
+
+@pytest.mark.parametrize("cfg", EDGE, ids=[c.name for c in EDGE])
+def test_layer_edge_cases(cfg):
+    inp = make_inputs(cfg)
+    ref = oracle_prefill(cfg, inp)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    check_recall(idx, ref)
+    check_out(out, ref["O"], cfg.dtype)
+
+
+def test_qwen7b_4k_layer():
+    """Qwen2.5-7B-shaped layer, batch 2 x 4096, bf16: lambda and recall on every row, O on a row sample."""
+    cfg = CONFIGS["qwen7b_4k"]
+    inp = make_inputs(cfg)
+    rows = sample_rows(cfg.seq, cfg.block, max_rows=192)
+    ref = oracle_prefill(cfg, inp, rows=rows)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    lam_err = check_lambda(lam, ref["lam"])
+    unexc, exc = check_recall(idx, ref)
+    max_abs, rel = check_out(out, ref["O"], "bf16", rows=rows)
+    print(f"qwen7b_4k: lambda rel {lam_err:.2e}, recall excused {exc}, O rel-L2 {rel:.2e} max-abs {max_abs:.2e}")
+
+
+def test_deterministic(mka):
+    cfg = small("det", "bf16", seq=700, d_head=128, n_q_heads=8, n_kv_heads=2, block=64, seed=21)
+    inp = make_inputs(cfg)
+    a, la, ia, *_ = gpu_prefill(cfg, inp)
+    b, lb, ib, *_ = gpu_prefill(cfg, inp)
+    assert torch.equal(a, b) and torch.equal(la, lb) and torch.equal(ia, ib)
+
+
+# ------------------------------------------------------------------ entry points one by one
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_router_entry(mka, dtype):
+    cfg = small("router", dtype, batch=2, seq=100, n_q_heads=8, d_head=64, router_hidden=256, seed=31)
+    inp = make_inputs(cfg)
+    g = torch.Generator().manual_seed(77)
+    q = torch.randn(cfg.batch * cfg.seq, cfg.dq, generator=g).to(inp.w_r1.dtype)
+    c = mka.make_config(cfg)
+    lam = torch.empty(cfg.batch * cfg.seq, 3, device="cuda")
+    ws = mka.buffer(mka.mka_router_workspace_size(c))
+    mka.mka_router(c, q.cuda(), inp.w_r1.cuda(), inp.w_r2.cuda(), lam, ws)
+    ref = oracle.router(to_f64(q), to_f64(inp.w_r1), to_f64(inp.w_r2))
+    check_lambda(lam, ref)
+
+
+@pytest.mark.parametrize("dtype,carry", [("f32", False), ("f32", True), ("bf16", True)])
+def test_session_ema_entry(mka, dtype, carry):
+    cfg = small("ema", dtype, batch=2, seq=333, alpha=0.97, seed=41)
+    inp = make_inputs(cfg)
+    c = mka.make_config(cfg)
+    x = inp.x.cuda()
+    cin = torch.randn(cfg.batch, cfg.d_model, generator=torch.Generator().manual_seed(3)) if carry else None
+    m2 = torch.empty(cfg.batch, cfg.seq, cfg.d_model, device="cuda")
+    cout = torch.empty(cfg.batch, cfg.d_model, device="cuda")
+    ws = mka.buffer(mka.mka_session_ema_workspace_size(c))
+    mka.mka_session_ema(c, x, None if cin is None else cin.cuda(), m2, cout, ws)
+    M2, m_next = oracle.session_ema(to_f64(inp.x), cfg.alpha, None if cin is None else cin.double().numpy())
+    assert np.abs(m2.cpu().double().numpy() - M2).max() <= F32_ATOL
+    assert np.abs(cout.cpu().double().numpy() - m_next).max() <= F32_ATOL
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_longterm_recall_entry(mka, dtype):
+    cfg = small("l3", dtype, batch=2, seq=300, block=16, recall_r=5, hash_bits=12, seed=51)
+    inp = make_inputs(cfg)
+    c = mka.make_config(cfg)
+    idx = torch.empty(cfg.batch, cfg.seq, cfg.recall_r, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(cfg.batch, cfg.seq, dtype=torch.int32, device="cuda")
+    m3 = torch.empty(cfg.batch, cfg.seq, cfg.d_model, device="cuda")
+    ws = mka.buffer(mka.mka_longterm_recall_workspace_size(c))
+    mka.mka_longterm_recall(c, inp.x.cuda(), inp.hash_proj.cuda(), idx, cnt, m3, ws)
+    X = to_f64(inp.x)
+    P = to_f64(inp.hash_proj)
+    for bi in range(cfg.batch):
+        summ = oracle.block_summaries(X[bi:bi + 1], cfg.block)[0]
+        ridx, rcnt, rM3, exc, *_ = oracle.longterm_recall(X[bi], np.arange(cfg.seq), summ, P, cfg.block, cfg.recall_r)
+        g = idx[bi].cpu().numpy()
+        bad = (g != ridx).any(-1)
+        assert int((bad & ~exc).sum()) == 0
+        assert np.array_equal(cnt[bi].cpu().numpy(), rcnt)
+        ok = ~bad
+        assert np.abs(m3[bi].cpu().double().numpy()[ok] - rM3[ok]).max() <= F32_ATOL
+
+
+# ------------------------------------------------------------------ decode
+def decode_run(cfg, inp, ctx, n_new, lmax):
+    """Prefill ctx rows into a state, then decode n_new rows one at a time; returns [B, n_new, dq]."""
+    import route_kv_memory_b200 as mka
+    layer = mka.FastMKALayer(cfg.replace(seq=max(ctx, 1)), gpu_weights(inp))
+    x = inp.x.cuda()
+    if ctx > 0:
+        out = torch.empty(cfg.batch, ctx, cfg.dq, dtype=x.dtype, device="cuda")
+        state = layer.new_state(lmax)
+        layer.prefill(x[:, :ctx].contiguous(), out, state=state, max_positions=lmax)
+    else:
+        state = layer.new_state(lmax)
+    outs = []
+    for t in range(ctx, ctx + n_new):
+        o = torch.empty(cfg.batch, cfg.dq, dtype=x.dtype, device="cuda")
+        layer.decode(state, lmax, x[:, t].contiguous(), o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert mka.mka_status() == 0
+    return torch.stack(outs, 1)
+
+
+@pytest.mark.parametrize("ctx", [0, 100, 200])
+def test_decode_tiny_f32(ctx):
+    cfg = CONFIGS["tiny_f32"]
+    inp = make_inputs(cfg)
+    n_new = cfg.seq - ctx
+    got = decode_run(cfg, inp, ctx, n_new, 300)
+    ref = oracle_prefill(cfg, inp, rows=np.arange(ctx, cfg.seq))
+    check_out(got, ref["O"], "f32")
+
+
+def test_decode_matches_oracle_recurrence_f32():
+    cfg = small("dec", "f32", batch=2, seq=70, block=8, recall_r=3, hash_bits=6, seed=61)
+    inp = make_inputs(cfg)
+    got = decode_run(cfg, inp, 0, cfg.seq, 80)
+    ref = oracle.fastmka_decode(to_f64(inp.x), oracle_weights(inp), cfg)
+    check_out(got, ref, "f32")
+
+
+def test_decode_bf16_small():
+    cfg = small("decbf", "bf16", batch=2, seq=1100, d_head=128, n_q_heads=8, n_kv_heads=2, router_hidden=128,
+                block=64, recall_r=4, hash_bits=32, seed=62)
+    inp = make_inputs(cfg)
+    ctx = 1000
+    got = decode_run(cfg, inp, ctx, cfg.seq - ctx, 1200)
+    ref = oracle_prefill(cfg, inp, rows=np.arange(ctx, cfg.seq))
+    check_out(got, ref["O"], "bf16")
+
+
+def test_decode_qwen_shape_4k():
+    """Qwen decode shapes (28/4 heads, d 3584, block 256, R 8): 4096-token prefix, 24 decoded tokens."""
+    cfg = CONFIGS["qwen7b_decode"].replace(seq=4096 + 24, decode_new=0)
+    inp = make_inputs(cfg)
+    ctx = 4096
+    got = decode_run(cfg, inp, ctx, 24, 4096 + 64)
+    ref = oracle_prefill(cfg, inp, rows=np.arange(ctx, ctx + 24))
+    max_abs, rel = check_out(got, ref["O"], "bf16")
+    print(f"decode qwen 4k: rel-L2 {rel:.2e} max-abs {max_abs:.2e}")
+
+
+def test_decode_capacity_is_a_device_status(mka):
+    cfg = CONFIGS["tiny_f32"].replace(seq=64)
+    inp = make_inputs(cfg, seq_total=65)
+    layer = mka.FastMKALayer(cfg, gpu_weights(inp))
+    x = inp.x.cuda()
+    state = layer.new_state(64)
+    out = torch.empty(1, 64, cfg.dq, device="cuda")
+    layer.prefill(x[:, :64].contiguous(), out, state=state, max_positions=64)
+    o = torch.empty(1, cfg.dq, device="cuda")
+    layer.decode(state, 64, x[:, 64].contiguous(), o)
+    assert mka.mka_status() == mka.MKA_ERR_CAPACITY
+    assert mka.mka_status() == 0
