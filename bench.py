@@ -344,13 +344,20 @@ def run_reference(args, rank, world):
 
 
 def traffic_from_profiles(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary (profiles/*.json), if one matches the current kernel."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary profiles/traffic.txt,
+    or None when the kernel's source changed after the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        d = json.load(f)
-    return d.get(kernel)
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    with open(os.path.join(ROOT, d["source"]), "rb") as f:
+        if hashlib.sha1(f.read()).hexdigest() != d["source_sha1"]:
+            return None
+    return d["dram_bytes_per_launch"]
 
 
 # ------------------------------------------------------------------ distributed plumbing
