@@ -174,6 +174,33 @@ MKA_API int mka_prefill_forward(const mka_config* cfg, const void* packed, const
 MKA_API int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size_t state_bytes,
                     int32_t max_positions, const void* x_new, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ without caller scratch */
+
+/* Bytes of the library's built-in scratch used by mka_session_ema_noalloc. */
+#define MKA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* mka_session_ema for callers that cannot allocate device memory (no counterpart
+ * in the paper; it exists for the library's users).  Some host programs cannot
+ * hand the library a scratch buffer: for example a plugin running inside a host
+ * application whose memory manager owns every device allocation and does not let
+ * plugins call cudaMalloc, or a caller whose device memory is fully reserved up
+ * front.  This call computes exactly what mka_session_ema computes, with the same
+ * kernels, but takes its scratch from a fixed MKA_NOALLOC_SCRATCH_BYTES (16 MiB)
+ * array inside the library's device image, held by every GPU that loads the
+ * library until the process exits.  It allocates nothing and frees nothing.
+ *   - Limit: shapes whose mka_session_ema_workspace_size(cfg) exceeds 16 MiB
+ *     (about B * (2*floor(S/64) + 1) * d * 4 bytes) are rejected with
+ *     MKA_ERR_WORKSPACE and a message naming both sizes; use mka_session_ema.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current (cudaGetSymbolAddress) and caches it; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, and each call overwrites what the previous
+ *     one left there before reading it.  Calls that overlap on the GPU (on two
+ *     streams or from two host threads) race on it: serialise them.
+ * Arguments, layouts and errors are those of mka_session_ema. */
+MKA_API int mka_session_ema_noalloc(const mka_config* cfg, const void* x, const float* carry_in, float* m2,
+                                    float* carry_out, void* stream);
+
 /* ------------------------------------------------------------------ status */
 
 /* Synchronises the current device and returns the device status word (MKA_OK or one

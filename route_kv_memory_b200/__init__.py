@@ -38,6 +38,7 @@ EXPORTED = [
     "mka_longterm_recall_workspace_size", "mka_state_size", "mka_decode_workspace_size", "mka_pack_weights",
     "mka_state_init", "mka_router", "mka_session_ema", "mka_longterm_recall", "mka_prefill_forward",
     "mka_decode_step", "mka_status", "mka_last_error", "mka_version", "mka_profile_enable", "mka_profile_read",
+    "mka_session_ema_noalloc",
 ]
 
 
@@ -75,6 +76,7 @@ _SIGS = {
     "mka_last_error": (ctypes.c_char_p, []),
     "mka_version": (ctypes.c_char_p, []),
     "mka_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+    "mka_session_ema_noalloc": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _vp]),
     "mka_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -170,6 +172,12 @@ def mka_router(c: mka_config, q, w_r1, w_r2, lam, ws, stream=None) -> None:
 def mka_session_ema(c: mka_config, x, carry_in, m2, carry_out, ws, stream=None) -> None:
     _check(_lib.mka_session_ema(ctypes.byref(c), _ptr(x), _ptr(carry_in), _ptr(m2), _ptr(carry_out), _ptr(ws),
                                 ws.numel() * ws.element_size(), _stream(stream)), "mka_session_ema")
+
+
+def mka_session_ema_noalloc(c: mka_config, x, carry_in, m2, carry_out, stream=None) -> None:
+    """mka_session_ema without a caller scratch buffer (uses the library's fixed 16 MiB device array)."""
+    _check(_lib.mka_session_ema_noalloc(ctypes.byref(c), _ptr(x), _ptr(carry_in), _ptr(m2), _ptr(carry_out),
+                                        _stream(stream)), "mka_session_ema_noalloc")
 
 
 def mka_longterm_recall(c: mka_config, x, hash_proj, idx, count, m3, ws, stream=None) -> None:

@@ -232,6 +232,11 @@ inline void prof_begin() { g_prof.n = 0; }
 
 }  // namespace
 
+int mka::set_last_error(int code, const char* msg) {
+  g_err = msg;
+  return code;
+}
+
 extern "C" {
 
 const char* mka_version(void) { return "fastmka-b200 0.1 (sm_100a)"; }

@@ -7,6 +7,9 @@
 
 namespace mka {
 
+// Records `msg` as the calling thread's mka_last_error() text; returns `code`.
+int set_last_error(int code, const char* msg);
+
 // One column range of a GEMM output and where it is stored.
 struct OutSeg {
   int n_begin, n_end;  // [n_begin, n_end) of the GEMM's N
