@@ -134,7 +134,7 @@ PackLayout pack_layout(const Dims& d) {
 
 // ---------------------------------------------------------------- prefill workspace
 struct PrefillWs {
-  size_t q, xkv, h1, h2, proj, lam, tcode, eps, bsum, bend, carry, scode, idx, cnt, k, v, total;
+  size_t q, xkv, h1, h2, proj, lam, tcode, xsum, bsum, bend, gend, carry, scode, idx, cnt, k, v, total;
 };
 PrefillWs prefill_ws(const Dims& d) {
   PrefillWs w;
@@ -146,9 +146,10 @@ PrefillWs prefill_ws(const Dims& d) {
   w.proj = o; o += al(T * d.nb * 4);
   w.lam = o; o += al(T * 3 * 4);
   w.tcode = o; o += al(T * 4);
-  w.eps = o; o += al(T * 4);
+  w.xsum = o; o += al((size_t)d.B * d.nblk * d.d * 8);
   w.bsum = o; o += al((size_t)d.B * d.nblk * d.width * 4);
   w.bend = o; o += al((size_t)d.B * d.nblk * d.width * 4);
+  w.gend = o; o += al((size_t)d.B * d.nblk * 8 * d.width * 4);
   w.carry = o; o += al((size_t)d.B * (d.nblk + 1) * d.width * 4);
   w.scode = o; o += al((size_t)d.B * d.nblk * 4);
   w.idx = o; o += al(T * d.R * 4);
@@ -162,7 +163,7 @@ PrefillWs prefill_ws(const Dims& d) {
 // ---------------------------------------------------------------- decode state
 struct StateLayout {
   int Lmax, maxblk;
-  size_t pos, kc, vc, ema, blk_sum, blk_p, blk_eps, blk_x, summ, scode, total;
+  size_t pos, kc, vc, ema, blk_sum, blk_x, summ, scode, total;
 };
 StateLayout state_layout(const Dims& d, int Lmax) {
   StateLayout s;
@@ -174,8 +175,6 @@ StateLayout state_layout(const Dims& d, int Lmax) {
   s.vc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.ema = o; o += al(B * d.width * 4);
   s.blk_sum = o; o += al(B * d.width * 4);
-  s.blk_p = o; o += al(B * 32 * 4);
-  s.blk_eps = o; o += al(B * 4);
   s.blk_x = o; o += al(B * d.d * 8);
   s.summ = o; o += al(B * (size_t)s.maxblk * d.width * 4);
   s.scode = o; o += al(B * (size_t)s.maxblk * 4);
@@ -304,8 +303,9 @@ size_t mka_longterm_recall_workspace_size(const mka_config* cfg) {
   Dims d;
   if (check_cfg(cfg, &d) != MKA_OK) return 0;
   size_t T = d.T;
-  return al((size_t)d.nb * d.d * d.elem) + al((size_t)d.nb * d.d * 8) + al(T * d.nb * 4) + al(T * 4) + al(T * 4) +
-         al((size_t)d.B * d.nblk * d.d * 4) + al((size_t)d.B * d.nblk * 4) + al(T * 4);
+  return al((size_t)d.nb * d.d * d.elem) + al((size_t)d.nb * d.d * 8) + al(T * d.nb * 4) + al(T * 4) +
+         al((size_t)d.B * d.nblk * d.d * 8) + al((size_t)d.B * d.nblk * d.d * 4) + al((size_t)d.B * d.nblk * 4) +
+         al(T * 4);
 }
 
 size_t mka_state_size(const mka_config* cfg, int32_t max_positions) {
@@ -407,7 +407,7 @@ int mka_session_ema(const mka_config* cfg, const void* x, const float* carry_in,
   float* bend = (float*)ws;
   float* carry = (float*)((char*)ws + al((size_t)d.B * nch * d.d * 4));
   double apb = pow((double)d.alpha, (double)kEmaChunk);
-  CUDA_TRY(block_reduce(x, d.bf16, d.d, d.d, d.B, d.S, nch, kEmaChunk, d.alpha, nullptr, 0, bend, s));
+  CUDA_TRY(block_reduce(x, d.bf16, d.d, d.d, d.B, d.S, nch, kEmaChunk, d.alpha, nullptr, 0, bend, nullptr, s));
   CUDA_TRY(ema_carry(bend, d.d, d.B, nch, (float)apb, carry_in, carry, s));
   CUDA_TRY(ema_apply(x, d.bf16, d.d, d.B, d.S, nch, kEmaChunk, d.alpha, carry, m2, carry_out, s));
   return MKA_OK;
@@ -429,8 +429,8 @@ int mka_longterm_recall(const mka_config* cfg, const void* x, const void* hash_p
   void* pT = o; o += al((size_t)d.nb * d.d * d.elem);
   double* pT64 = (double*)o; o += al((size_t)d.nb * d.d * 8);
   float* proj = (float*)o; o += al(T * d.nb * 4);
-  float* eps = (float*)o; o += al(T * 4);
   uint32_t* tcode = (uint32_t*)o; o += al(T * 4);
+  double* xsum = (double*)o; o += al((size_t)d.B * d.nblk * d.d * 8);
   float* bsum = (float*)o; o += al((size_t)d.B * d.nblk * d.d * 4);
   uint32_t* scode = (uint32_t*)o; o += al((size_t)d.B * d.nblk * 4);
   int* cnt = count ? count : (int*)o;
@@ -442,11 +442,12 @@ int mka_longterm_recall(const mka_config* cfg, const void* x, const void* hash_p
   if (d.bf16) CUDA_TRY(gemm_tn_bf16(x, d.d, pT, d.d, d.T, d.nb, d.d, ep, s));
   else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, pT, d.d, 0, d.T, d.nb, d.d, ep, s));
   HashArgs ha{proj, d.nb, x, d.bf16, pT64, d.d, d.nb, d.d};
-  CUDA_TRY(token_codes(ha, d.T, tcode, eps, s));
-  CUDA_TRY(summary_codes(ha, d.B, d.S, d.nblk, d.blk, eps, scode, d.nblk, s));
+  CUDA_TRY(token_codes(ha, d.T, tcode, s));
+  CUDA_TRY(summary_codes(x, d.bf16, d.d, d.B, d.S, d.nblk, d.blk, pT64, d.nb, xsum, scode, d.nblk, s));
   CUDA_TRY(recall_select(tcode, scode, d.nblk, d.B, d.S, d.nblk, d.blk, d.R, idx, cnt, s));
   if (m3) {
-    CUDA_TRY(block_reduce(x, d.bf16, d.d, d.d, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, (long long)d.nblk * d.d, nullptr, s));
+    CUDA_TRY(block_reduce(x, d.bf16, d.d, d.d, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, (long long)d.nblk * d.d, nullptr,
+                          nullptr, s));
     CUDA_TRY(gather_mean(idx, cnt, d.R, bsum, d.nblk, d.d, d.blk, d.B, d.S, m3, s));
   }
   return MKA_OK;
@@ -480,10 +481,11 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   float* proj = (float*)P(ws, W.proj);
   float* lam = lambda_out ? lambda_out : (float*)P(ws, W.lam);
   uint32_t* tcode = (uint32_t*)P(ws, W.tcode);
-  float* eps = (float*)P(ws, W.eps);
+  double* xsum = (double*)P(ws, W.xsum);
   float* bsum = state ? (float*)P(state, SL.summ) : (float*)P(ws, W.bsum);
   long long bsum_bstride = (long long)(state ? SL.maxblk : d.nblk) * d.width;
   float* bend = (float*)P(ws, W.bend);
+  float* gend = (float*)P(ws, W.gend);
   float* carry = (float*)P(ws, W.carry);
   uint32_t* scode = state ? (uint32_t*)P(state, SL.scode) : (uint32_t*)P(ws, W.scode);
   int code_bstride = state ? SL.maxblk : d.nblk;
@@ -513,11 +515,11 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   STAGE(s);
   // 3. L3 codes, 4. block sums / EMA end states, carries, recall
   HashArgs ha{proj, d.nb, x, d.bf16, (const double*)P((void*)packed, PL.pT64), d.d, d.nb, d.d};
-  CUDA_TRY(token_codes(ha, d.T, tcode, eps, s));
+  CUDA_TRY(token_codes(ha, d.T, tcode, s));
   STAGE(s);
-  CUDA_TRY(block_reduce(xkv, 0, d.width, d.width, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, bsum_bstride, bend, s));
+  CUDA_TRY(block_reduce(xkv, 0, d.width, d.width, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, bsum_bstride, bend, gend, s));
   STAGE(s);
-  CUDA_TRY(summary_codes(ha, d.B, d.S, d.nblk, d.blk, eps, scode, code_bstride, s));
+  CUDA_TRY(summary_codes(x, d.bf16, d.d, d.B, d.S, d.nblk, d.blk, ha.pT64, d.nb, xsum, scode, code_bstride, s));
   STAGE(s);
   CUDA_TRY(ema_carry(bend, d.width, d.B, d.nblk, (float)pow((double)d.alpha, (double)d.blk), nullptr, carry, s));
   STAGE(s);
@@ -526,7 +528,7 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   // 5. route-fuse -> K, V
   FuseArgs fa{};
   fa.xkv = xkv; fa.ld = d.width; fa.width = d.width; fa.lam = lam; fa.idx = idx; fa.count = cnt; fa.R = d.R;
-  fa.bsum = bsum; fa.bsum_bstride = bsum_bstride; fa.carry = carry;
+  fa.bsum = bsum; fa.bsum_bstride = bsum_bstride; fa.carry = carry; fa.gend = gend;
   fa.B = d.B; fa.S = d.S; fa.nblk = d.nblk; fa.blk = d.blk; fa.dkv = d.dkv; fa.alpha = d.alpha;
   fa.k_out = kbuf; fa.v_out = vbuf; fa.kv_bstride = kv_bstride; fa.out_bf16 = d.bf16;
   fa.state_ema = state ? (float*)P(state, SL.ema) : nullptr;
@@ -541,8 +543,7 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   CUDA_TRY(attention_prefill(aa, d.bf16, s));
   STAGE(s);
   if (state) {
-    CUDA_TRY(prefill_tail_state(xkv, d.width, d.width, proj, d.nb, d.nb, eps, x, d.bf16, d.d, d.B, d.S, d.blk,
-                                (float*)P(state, SL.blk_sum), (float*)P(state, SL.blk_p), (float*)P(state, SL.blk_eps),
+    CUDA_TRY(prefill_tail_state(xkv, d.width, d.width, x, d.bf16, d.d, d.B, d.S, d.blk, (float*)P(state, SL.blk_sum),
                                 (double*)P(state, SL.blk_x), (int*)P(state, SL.pos), s));
     STAGE(s);
   }
@@ -573,8 +574,7 @@ int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size
   a.maxblk = SL.maxblk; a.alpha = d.alpha; a.scale = d.scale;
   a.x_new = x_new; a.out = out;
   a.pos = (int*)P(state, SL.pos); a.kcache = P(state, SL.kc); a.vcache = P(state, SL.vc);
-  a.ema = (float*)P(state, SL.ema); a.blk_sum = (float*)P(state, SL.blk_sum); a.blk_p = (float*)P(state, SL.blk_p);
-  a.blk_eps = (float*)P(state, SL.blk_eps); a.blk_x = (double*)P(state, SL.blk_x);
+  a.ema = (float*)P(state, SL.ema); a.blk_sum = (float*)P(state, SL.blk_sum); a.blk_x = (double*)P(state, SL.blk_x);
   a.summ = (float*)P(state, SL.summ); a.scode = (uint32_t*)P(state, SL.scode);
   a.y = (float*)P(ws, W.y); a.qf = (float*)P(ws, W.qf); a.part = (float*)P(ws, W.part); a.nsplit = W.nsplit;
   a.status = status_ptr();

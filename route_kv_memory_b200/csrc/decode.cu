@@ -71,9 +71,8 @@ __global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
   __shared__ int s_idx[64];
   __shared__ int s_cnt, s_pos, s_skip;
   __shared__ unsigned s_code;
-  __shared__ float s_eps;
   __shared__ int s_base[34], s_run[34];
-  __shared__ unsigned s_scode, s_sdoubt;
+  __shared__ unsigned s_scode;
   const int bi = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   const float* y = a.y + (size_t)bi * a.Ntot;
@@ -130,10 +129,7 @@ __global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
       if (lane == k) bit = acc > 0.0;
     }
     unsigned code = __ballot_sync(0xffffffffu, bit && lane < a.nb);
-    if (lane == 0) {
-      s_code = code;
-      s_eps = e;
-    }
+    if (lane == 0) s_code = code;
   }
   __syncthreads();
   if (tid == 0) {
@@ -210,33 +206,22 @@ __global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
       bsum[c] += xv;
     }
     for (int i = tid; i < a.d; i += blockDim.x) a.blk_x[(size_t)bi * a.d + i] += to_d<T>(xn[i]);
-    if (tid < a.nb) a.blk_p[(size_t)bi * 32 + tid] += p[tid];
-    if (tid == 0) a.blk_eps[bi] += s_eps;
     // query for the attention, rounded to the layer dtype as the prefill path stores it
     for (int c = tid; c < a.dq; c += blockDim.x) a.qf[(size_t)bi * a.dq + c] = to_f<T>(from_f<T>(q[c]));
   }
   __syncthreads();
-  // finish a block: summary = block sum, code = signs of sum_t p_t (exact in doubt)
+  // finish a block: summary = its projected-row sum; code = signs of its exact float64
+  // d_model-space sum projected in float64 (the same decision as the prefill path)
   if ((pos + 1) % a.blk == 0 && pos / a.blk < a.maxblk) {
     const int j = pos / a.blk;
     float* bsum = a.blk_sum + (size_t)bi * width;
     float* summ = a.summ + ((size_t)bi * a.maxblk + j) * width;
-    if (warp == 0) {
-      float sp = lane < a.nb ? a.blk_p[(size_t)bi * 32 + lane] : 0.f;
-      float et = 2.f * a.blk_eps[bi];
-      unsigned doubt = __ballot_sync(0xffffffffu, lane < a.nb && fabsf(sp) <= et);
-      unsigned code = __ballot_sync(0xffffffffu, lane < a.nb && sp > 0.f);
-      if (lane == 0) {
-        s_sdoubt = doubt;
-        s_scode = code & ~doubt;
-      }
-    }
+    if (tid == 0) s_scode = 0u;
     __syncthreads();
-    const unsigned doubt = s_sdoubt;
+    const double* bx = a.blk_x + (size_t)bi * a.d;
     for (int k = warp; k < a.nb; k += nw) {
-      if (!((doubt >> k) & 1u)) continue;
       double v = 0.0;
-      for (int i = lane; i < a.d; i += 32) v = fma(a.blk_x[(size_t)bi * a.d + i], a.pT64[(size_t)k * a.d + i], v);
+      for (int i = lane; i < a.d; i += 32) v = fma(bx[i], a.pT64[(size_t)k * a.d + i], v);
       v = warp_sum_d(v);
       if (lane == 0 && v > 0.0) atomicOr(&s_scode, 1u << k);
     }
@@ -246,11 +231,7 @@ __global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
     }
     __syncthreads();
     for (int i = tid; i < a.d; i += blockDim.x) a.blk_x[(size_t)bi * a.d + i] = 0.0;
-    if (tid < 32) a.blk_p[(size_t)bi * 32 + tid] = 0.f;
-    if (tid == 0) {
-      a.blk_eps[bi] = 0.f;
-      a.scode[(size_t)bi * a.maxblk + j] = s_scode;
-    }
+    if (tid == 0) a.scode[(size_t)bi * a.maxblk + j] = s_scode;
   }
   if (tid == 0) a.pos[bi] = pos + 1;
 }

@@ -51,13 +51,17 @@ struct HashArgs {
 
 cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, float* lam,
                         cudaStream_t s);
-cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, float* eps, cudaStream_t s);
-cudaError_t summary_codes(const HashArgs& a, int B, int S, int nblk, int blk, const float* eps, uint32_t* codes,
-                          int code_bstride, cudaStream_t s);
-// Per full block j of each sequence: bsum = sum of its rows, bend = EMA end state from a zero carry.
-// x: [B*S, ld] (bf16 or float32), first `width` columns.  bsum[b*bsum_bstride + j*width + c].
+cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, cudaStream_t s);
+// Codes of the full blocks: exact float64 block sums of x in d_model space (xsum scratch [B][nblk][d]),
+// projected in float64.  codes[b*code_bstride + j].
+cudaError_t summary_codes(const void* x, int x_bf16, int d, int B, int S, int nblk, int blk, const double* pT64,
+                          int nb, double* xsum, uint32_t* codes, int code_bstride, cudaStream_t s);
+// Per full block j of each sequence: bsum = sum of its rows, bend = EMA end state from a zero carry,
+// gend = the zero-carry EMA end state of each of its 8 row groups (all three nullable).
+// x: [B*S, ld] (bf16 or float32), first `width` columns.  bsum[b*bsum_bstride + j*width + c],
+// bend[(b*nblk + j)*width + c], gend[((b*nblk + j)*8 + g)*width + c].
 cudaError_t block_reduce(const void* x, int x_bf16, int ld, int width, int B, int S, int nblk, int blk, float alpha,
-                         float* bsum, long long bsum_bstride, float* bend, cudaStream_t s);
+                         float* bsum, long long bsum_bstride, float* bend, float* gend, cudaStream_t s);
 cudaError_t ema_carry(const float* bend, int width, int B, int nblk, float alpha_pow_b, const float* carry_in,
                       float* carry, cudaStream_t s);
 cudaError_t recall_select(const uint32_t* tok_codes, const uint32_t* blk_codes, int blk_codes_bstride, int B, int S,
@@ -70,6 +74,7 @@ struct FuseArgs {
   const int* idx; const int* count; int R;
   const float* bsum; long long bsum_bstride;  // [B][nblk][width] block SUMS
   const float* carry;             // [B][nblk+1][width] EMA value at each block start
+  const float* gend;              // [B][nblk][8][width] zero-carry EMA end state of each row group
   int B, S, nblk, blk, dkv;
   float alpha;
   void* k_out; void* v_out; long long kv_bstride; int out_bf16;  // [B][.. rows][dkv]
@@ -84,10 +89,8 @@ cudaError_t gather_mean(const int* idx, const int* count, int R, const float* bs
                         int B, int S, float* m3, cudaStream_t s);
 
 // State tail after a prefill: the unfinished block's sums.
-cudaError_t prefill_tail_state(const float* xkv, int ld, int width, const float* proj, int ldp, int nb,
-                               const float* eps, const void* x, int x_bf16, int d, int B, int S, int blk,
-                               float* blk_sum, float* blk_p, float* blk_eps, double* blk_x, int* pos,
-                               cudaStream_t s);
+cudaError_t prefill_tail_state(const float* xkv, int ld, int width, const void* x, int x_bf16, int d, int B, int S,
+                               int blk, float* blk_sum, double* blk_x, int* pos, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
 struct AttnArgs {
@@ -111,7 +114,7 @@ struct DecodeArgs {
   const void* x_new;             // [B, d]
   void* out;                     // [B, dq]
   // state
-  int* pos; void* kcache; void* vcache; float* ema; float* blk_sum; float* blk_p; float* blk_eps; double* blk_x;
+  int* pos; void* kcache; void* vcache; float* ema; float* blk_sum; double* blk_x;
   float* summ; uint32_t* scode;
   // scratch
   float* y;                      // [B, Ntot] projection row

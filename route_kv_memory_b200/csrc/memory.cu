@@ -54,6 +54,18 @@ cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh
   return cudaGetLastError();
 }
 
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+  static __device__ __forceinline__ float4 load(const float* p) { return *(const float4*)p; }
+};
+template <> struct Vec4<bf16> {
+  static __device__ __forceinline__ float4 load(const bf16* p) {
+    uint2 u = *(const uint2*)p;
+    __nv_bfloat162 a = *(__nv_bfloat162*)&u.x, b = *(__nv_bfloat162*)&u.y;
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+};
 // ---------------------------------------------------------------- L3 sign codes
 // The float32 projection p = x . P_k carries a rounding error far below
 // eps = K * 2^-20 * rms_k(p) (K * 2^-23 * |partial sum| is the worst-case
@@ -68,7 +80,7 @@ __device__ __forceinline__ double dot_row_f64(const T* __restrict__ x, const dou
 }
 
 template <typename T>
-__global__ void token_codes_kernel(HashArgs a, int T_, uint32_t* __restrict__ codes, float* __restrict__ eps) {
+__global__ void token_codes_kernel(HashArgs a, int T_, uint32_t* __restrict__ codes) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T_) return;
@@ -85,105 +97,83 @@ __global__ void token_codes_kernel(HashArgs a, int T_, uint32_t* __restrict__ co
     if (lane == k) bit = v > 0.0;
   }
   unsigned code = __ballot_sync(0xffffffffu, bit && lane < a.nb);
-  if (lane == 0) {
-    codes[t] = code;
-    if (eps) eps[t] = e;
-  }
+  if (lane == 0) codes[t] = code;
 }
 
-cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, float* eps, cudaStream_t s) {
+cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  if (a.x_bf16) token_codes_kernel<bf16><<<(T + 7) / 8, 256, 0, s>>>(a, T, codes, eps);
-  else token_codes_kernel<float><<<(T + 7) / 8, 256, 0, s>>>(a, T, codes, eps);
+  if (a.x_bf16) token_codes_kernel<bf16><<<(T + 7) / 8, 256, 0, s>>>(a, T, codes);
+  else token_codes_kernel<float><<<(T + 7) / 8, 256, 0, s>>>(a, T, codes);
   return cudaGetLastError();
 }
 
-// Block code: bits of sum_t p_t over the block (the sign of the block mean's
-// projection).  The float32 sum's error is below 2 * sum_t eps_t; in doubt, the
-// exact float64 block sum of X in d_model space is formed and projected.
+// Block codes.  The code of block j is the sign pattern of (sum of its rows) P,
+// the same signs as (block mean) P.  The block sums are formed exactly in
+// float64 in d_model space (sums of at most a few hundred bf16 or float32
+// values), then projected in float64: no float32 rounding enters the decision.
 template <typename T>
-__global__ void summary_codes_kernel(HashArgs a, int S, int nblk, int blk, const float* __restrict__ eps,
-                                     uint32_t* __restrict__ codes, int code_bstride) {
-  extern __shared__ double sx[];  // [d]
-  __shared__ float sp[8][32];
-  __shared__ float se[8];
-  __shared__ unsigned s_doubt, s_code;
+__global__ void __launch_bounds__(256) block_xsum_kernel(const T* __restrict__ x, int d, int S, int blk,
+                                                          int nblk, double* __restrict__ xsum) {
+  __shared__ double sacc[4][64][4];
+  const int bi = blockIdx.z, j = blockIdx.y;
+  const int cl = threadIdx.x & 63, rg = threadIdx.x >> 6;
+  const int c = (blockIdx.x * 64 + cl) * 4;
+  const int per = (blk + 3) / 4;
+  const int ra = min(rg * per, blk), rb = min(ra + per, blk);
+  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+  if (c < d) {
+    const T* p = x + ((size_t)bi * S + (size_t)j * blk) * d + c;
+#pragma unroll 4
+    for (int r = ra; r < rb; ++r) {
+      float4 v = Vec4<T>::load(p + (size_t)r * d);
+      a0 += v.x;
+      a1 += v.y;
+      a2 += v.z;
+      a3 += v.w;
+    }
+  }
+  sacc[rg][cl][0] = a0;
+  sacc[rg][cl][1] = a1;
+  sacc[rg][cl][2] = a2;
+  sacc[rg][cl][3] = a3;
+  __syncthreads();
+  if (rg == 0 && c < d) {
+    double* o = xsum + ((size_t)bi * nblk + j) * d + c;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = sacc[0][cl][e] + sacc[1][cl][e] + sacc[2][cl][e] + sacc[3][cl][e];
+  }
+}
+
+__global__ void __launch_bounds__(256) summary_codes_kernel(const double* __restrict__ xsum,
+                                                            const double* __restrict__ pT64, int d, int nb, int nblk,
+                                                            uint32_t* __restrict__ codes, int code_bstride) {
+  __shared__ unsigned s_code;
   const int bi = blockIdx.y, j = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t t0 = (size_t)bi * S + (size_t)j * blk;
-  float acc = 0.f, eacc = 0.f;
-  for (int r = warp; r < blk; r += 8) {
-    if (lane < a.nb) acc += a.proj[(t0 + r) * a.ldp + lane];
-    if (lane == 0) eacc += eps[t0 + r];
-  }
-  sp[warp][lane] = acc;
-  if (lane == 0) se[warp] = eacc;
+  if (threadIdx.x == 0) s_code = 0u;
   __syncthreads();
-  if (warp == 0) {
-    float tot = 0.f, et = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      tot += sp[w][lane];
-      et += se[w];
-    }
-    et *= 2.f;
-    unsigned doubt = __ballot_sync(0xffffffffu, lane < a.nb && fabsf(tot) <= et);
-    unsigned code = __ballot_sync(0xffffffffu, lane < a.nb && tot > 0.f);
-    if (lane == 0) {
-      s_doubt = doubt;
-      s_code = code & ~doubt;
-    }
+  const double* v = xsum + ((size_t)bi * nblk + j) * d;
+  for (int k = warp; k < nb; k += 8) {
+    double acc = 0.0;
+    for (int i = lane; i < d; i += 32) acc = fma(v[i], pT64[(size_t)k * d + i], acc);
+    acc = warp_sum_d(acc);
+    if (lane == 0 && acc > 0.0) atomicOr(&s_code, 1u << k);
   }
   __syncthreads();
-  unsigned doubt = s_doubt;
-  if (doubt) {
-    const T* x = (const T*)a.x;
-    for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
-      double s = 0.0;
-      for (int r = 0; r < blk; ++r) s += to_d<T>(x[(t0 + r) * a.d + i]);
-      sx[i] = s;
-    }
-    __syncthreads();
-    for (int k = warp; k < a.nb; k += 8) {
-      if (!((doubt >> k) & 1u)) continue;
-      double v = 0.0;
-      for (int i = lane; i < a.d; i += 32) v = fma(sx[i], a.pT64[(size_t)k * a.d + i], v);
-      v = warp_sum_d(v);
-      if (lane == 0 && v > 0.0) atomicOr(&s_code, 1u << k);
-    }
-    __syncthreads();
-  }
   if (threadIdx.x == 0) codes[(size_t)bi * code_bstride + j] = s_code;
 }
 
-cudaError_t summary_codes(const HashArgs& a, int B, int S, int nblk, int blk, const float* eps, uint32_t* codes,
-                          int code_bstride, cudaStream_t s) {
+cudaError_t summary_codes(const void* x, int x_bf16, int d, int B, int S, int nblk, int blk, const double* pT64,
+                          int nb, double* xsum, uint32_t* codes, int code_bstride, cudaStream_t s) {
   if (B <= 0 || nblk <= 0) return cudaSuccess;
-  dim3 grid(nblk, B);
-  size_t sm = (size_t)a.d * sizeof(double);
-  if (a.x_bf16) {
-    set_max_smem(summary_codes_kernel<bf16>, sm, s);
-    summary_codes_kernel<bf16><<<grid, 256, sm, s>>>(a, S, nblk, blk, eps, codes, code_bstride);
-  } else {
-    set_max_smem(summary_codes_kernel<float>, sm, s);
-    summary_codes_kernel<float><<<grid, 256, sm, s>>>(a, S, nblk, blk, eps, codes, code_bstride);
-  }
+  dim3 g1((d / 4 + 63) / 64, nblk, B);
+  if (x_bf16) block_xsum_kernel<bf16><<<g1, 256, 0, s>>>((const bf16*)x, d, S, blk, nblk, xsum);
+  else block_xsum_kernel<float><<<g1, 256, 0, s>>>((const float*)x, d, S, blk, nblk, xsum);
+  summary_codes_kernel<<<dim3(nblk, B), 256, 0, s>>>(xsum, pT64, d, nb, nblk, codes, code_bstride);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- block sums + EMA end states
-template <typename T> struct Vec4;
-template <> struct Vec4<float> {
-  static __device__ __forceinline__ float4 load(const float* p) { return *(const float4*)p; }
-};
-template <> struct Vec4<bf16> {
-  static __device__ __forceinline__ float4 load(const bf16* p) {
-    uint2 u = *(const uint2*)p;
-    __nv_bfloat162 a = *(__nv_bfloat162*)&u.x, b = *(__nv_bfloat162*)&u.y;
-    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-    return make_float4(fa.x, fa.y, fb.x, fb.y);
-  }
-};
 __device__ __forceinline__ float4 f4_fma(float a, float4 x, float4 y) {
   return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
 }
@@ -194,18 +184,26 @@ __device__ __forceinline__ float4 ema_step(float al, float om, float4 m, float4 
   return make_float4(fmaf(al, m.x, om * x.x), fmaf(al, m.y, om * x.y), fmaf(al, m.z, om * x.z), fmaf(al, m.w, om * x.w));
 }
 
-constexpr int kRG = 4;  // row groups per block in block_reduce
+constexpr int kRG = 8;  // row groups per block in block_reduce and fuse_kv
+
+// Rows [ra, rb) of row group g of a block of `blk` rows.
+__device__ __forceinline__ void group_rows(int g, int blk, int& ra, int& rb) {
+  const int per = (blk + kRG - 1) / kRG;
+  ra = min(g * per, blk);
+  rb = min(ra + per, blk);
+}
 
 template <typename T>
-__global__ void __launch_bounds__(256) block_reduce_kernel(const T* __restrict__ x, int ld, int width, int S, int nblk,
+__global__ void __launch_bounds__(512) block_reduce_kernel(const T* __restrict__ x, int ld, int width, int S, int nblk,
                                                             int blk, float alpha, float* __restrict__ bsum,
-                                                            long long bsum_bstride, float* __restrict__ bend) {
+                                                            long long bsum_bstride, float* __restrict__ bend,
+                                                            float* __restrict__ gend) {
   __shared__ float4 ssum[kRG][64], send[kRG][64];
   const int bi = blockIdx.z, j = blockIdx.y;
   const int cl = threadIdx.x & 63, rg = threadIdx.x >> 6;
   const int c = (blockIdx.x * 64 + cl) * 4;
-  const int per = (blk + kRG - 1) / kRG;
-  const int ra = min(rg * per, blk), rb = min(ra + per, blk);
+  int ra, rb;
+  group_rows(rg, blk, ra, rb);
   const float om = 1.f - alpha;
   float4 s = make_float4(0, 0, 0, 0), e = s;
   if (c < width) {
@@ -216,6 +214,7 @@ __global__ void __launch_bounds__(256) block_reduce_kernel(const T* __restrict__
       s = f4_add(s, v);
       e = ema_step(alpha, om, e, v);
     }
+    if (gend) *(float4*)(gend + (((size_t)bi * nblk + j) * kRG + rg) * width + c) = e;
   }
   ssum[rg][cl] = s;
   send[rg][cl] = e;
@@ -223,7 +222,8 @@ __global__ void __launch_bounds__(256) block_reduce_kernel(const T* __restrict__
   if (rg == 0 && c < width) {
     float4 S4 = ssum[0][cl], E4 = send[0][cl];
     for (int g = 1; g < kRG; ++g) {
-      int ga = min(g * per, blk), gb = min(ga + per, blk);
+      int ga, gb;
+      group_rows(g, blk, ga, gb);
       float ap = 1.f;
       for (int i = ga; i < gb; ++i) ap *= alpha;  // a^(rows of group g)
       S4 = f4_add(S4, ssum[g][cl]);
@@ -235,13 +235,15 @@ __global__ void __launch_bounds__(256) block_reduce_kernel(const T* __restrict__
 }
 
 cudaError_t block_reduce(const void* x, int x_bf16, int ld, int width, int B, int S, int nblk, int blk, float alpha,
-                         float* bsum, long long bsum_bstride, float* bend, cudaStream_t s) {
+                         float* bsum, long long bsum_bstride, float* bend, float* gend, cudaStream_t s) {
   if (B <= 0 || nblk <= 0) return cudaSuccess;
   dim3 grid((width / 4 + 63) / 64, nblk, B);
   if (x_bf16)
-    block_reduce_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)x, ld, width, S, nblk, blk, alpha, bsum, bsum_bstride, bend);
+    block_reduce_kernel<bf16><<<grid, 64 * kRG, 0, s>>>((const bf16*)x, ld, width, S, nblk, blk, alpha, bsum,
+                                                         bsum_bstride, bend, gend);
   else
-    block_reduce_kernel<float><<<grid, 256, 0, s>>>((const float*)x, ld, width, S, nblk, blk, alpha, bsum, bsum_bstride, bend);
+    block_reduce_kernel<float><<<grid, 64 * kRG, 0, s>>>((const float*)x, ld, width, S, nblk, blk, alpha, bsum,
+                                                          bsum_bstride, bend, gend);
   return cudaGetLastError();
 }
 
@@ -351,7 +353,7 @@ template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
 }
 
 template <typename OutT>
-__global__ void __launch_bounds__(64) fuse_kernel(FuseArgs a) {
+__global__ void __launch_bounds__(64 * kRG) fuse_kernel(FuseArgs a) {
   extern __shared__ float sm[];
   float* slam = sm;                                   // [blk*3]
   int* sidx = (int*)(slam + a.blk * 3);               // [blk*R]
@@ -363,16 +365,34 @@ __global__ void __launch_bounds__(64) fuse_kernel(FuseArgs a) {
   for (int i = threadIdx.x; i < nr * a.R; i += blockDim.x) sidx[i] = a.idx[tg0 * a.R + i];
   for (int i = threadIdx.x; i < nr; i += blockDim.x) scnt[i] = a.count[tg0 + i];
   __syncthreads();
-  const int c = (blockIdx.x * 64 + threadIdx.x) * 4;
+  const int cl = threadIdx.x & 63, rg = threadIdx.x >> 6;
+  const int c = (blockIdx.x * 64 + cl) * 4;
   if (c >= a.width) return;
   const float om = 1.f - a.alpha;
+  // EMA value at the first row of this thread's row group: the block's carry advanced
+  // over the preceding groups (their zero-carry end states come from block_reduce).
   float4 m2 = *(const float4*)(a.carry + ((size_t)bi * (a.nblk + 1) + j) * a.width + c);
+  int ra, rb;
+  if (j < a.nblk) {
+    group_rows(rg, a.blk, ra, rb);
+    for (int g = 0; g < rg; ++g) {
+      int ga, gb;
+      group_rows(g, a.blk, ga, gb);
+      float ap = 1.f;
+      for (int i = ga; i < gb; ++i) ap *= a.alpha;
+      float4 ge = *(const float4*)(a.gend + (((size_t)bi * a.nblk + j) * kRG + g) * a.width + c);
+      m2 = f4_add(f4_scale(ap, m2), ge);
+    }
+  } else {  // the unfinished last block: one group walks all its rows
+    ra = 0;
+    rb = rg == 0 ? nr : 0;
+  }
   const float* bs = a.bsum + (size_t)bi * a.bsum_bstride + c;
   const bool is_k = c < a.dkv;
   OutT* dst = (OutT*)(is_k ? a.k_out : a.v_out) + (size_t)bi * a.kv_bstride + (size_t)r0 * a.dkv + (is_k ? c : c - a.dkv);
   const float* xp = a.xkv + tg0 * a.ld + c;
   const float invb = 1.f / (float)a.blk;
-  for (int r = 0; r < nr; ++r) {
+  for (int r = ra; r < rb; ++r) {
     float4 x = *(const float4*)(xp + (size_t)r * a.ld);
     int cnt = scnt[r];
     float4 m3 = make_float4(0, 0, 0, 0);
@@ -383,7 +403,7 @@ __global__ void __launch_bounds__(64) fuse_kernel(FuseArgs a) {
     store4<OutT>(dst + (size_t)r * a.dkv, o);
     m2 = ema_step(a.alpha, om, m2, x);
   }
-  if (r1 == a.S && a.state_ema) *(float4*)(a.state_ema + (size_t)bi * a.width + c) = m2;
+  if (r1 == a.S && rb == nr && rb > ra && a.state_ema) *(float4*)(a.state_ema + (size_t)bi * a.width + c) = m2;
 }
 
 cudaError_t fuse_kv(const FuseArgs& a, cudaStream_t s) {
@@ -392,11 +412,13 @@ cudaError_t fuse_kv(const FuseArgs& a, cudaStream_t s) {
   dim3 grid((a.width / 4 + 63) / 64, nb_all, a.B);
   size_t sm = (size_t)a.blk * (3 * sizeof(float) + (a.R + 1) * sizeof(int));
   if (a.out_bf16) {
-    set_max_smem(fuse_kernel<bf16>, sm, s);
-    fuse_kernel<bf16><<<grid, 64, sm, s>>>(a);
+    cudaError_t e = set_max_smem(fuse_kernel<bf16>, sm, s);
+    if (e != cudaSuccess) return e;
+    fuse_kernel<bf16><<<grid, 64 * kRG, sm, s>>>(a);
   } else {
-    set_max_smem(fuse_kernel<float>, sm, s);
-    fuse_kernel<float><<<grid, 64, sm, s>>>(a);
+    cudaError_t e = set_max_smem(fuse_kernel<float>, sm, s);
+    if (e != cudaSuccess) return e;
+    fuse_kernel<float><<<grid, 64 * kRG, sm, s>>>(a);
   }
   return cudaGetLastError();
 }
@@ -454,11 +476,11 @@ cudaError_t gather_mean(const int* idx, const int* count, int R, const float* bs
 }
 
 // ---------------------------------------------------------------- decode state after a prefill
+// The unfinished last block of each sequence: its projected-row sums and its exact float64
+// d_model-space sum (from which decode forms the block's code once the block is complete).
 template <typename T>
-__global__ void prefill_tail_kernel(const float* __restrict__ xkv, int ld, int width, const float* __restrict__ proj,
-                                    int ldp, int nb, const float* __restrict__ eps, const T* __restrict__ x, int d,
-                                    int S, int blk, float* blk_sum, float* blk_p, float* blk_eps, double* blk_x,
-                                    int* pos) {
+__global__ void prefill_tail_kernel(const float* __restrict__ xkv, int ld, int width, const T* __restrict__ x, int d,
+                                    int S, int blk, float* blk_sum, double* blk_x, int* pos) {
   const int bi = blockIdx.x;
   const int r0 = (S / blk) * blk;  // first row of the unfinished block
   const size_t t0 = (size_t)bi * S;
@@ -467,35 +489,21 @@ __global__ void prefill_tail_kernel(const float* __restrict__ xkv, int ld, int w
     for (int r = r0; r < S; ++r) s += xkv[(t0 + r) * ld + c];
     blk_sum[(size_t)bi * width + c] = s;
   }
-  for (int k = threadIdx.x; k < nb; k += blockDim.x) {
-    float s = 0.f;
-    for (int r = r0; r < S; ++r) s += proj[(t0 + r) * ldp + k];
-    blk_p[(size_t)bi * 32 + k] = s;
-  }
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
     double s = 0.0;
     for (int r = r0; r < S; ++r) s += to_d<T>(x[(t0 + r) * d + i]);
     blk_x[(size_t)bi * d + i] = s;
   }
-  if (threadIdx.x == 0) {
-    float s = 0.f;
-    for (int r = r0; r < S; ++r) s += eps[t0 + r];
-    blk_eps[bi] = s;
-    pos[bi] = S;
-  }
+  if (threadIdx.x == 0) pos[bi] = S;
 }
 
-cudaError_t prefill_tail_state(const float* xkv, int ld, int width, const float* proj, int ldp, int nb,
-                               const float* eps, const void* x, int x_bf16, int d, int B, int S, int blk,
-                               float* blk_sum, float* blk_p, float* blk_eps, double* blk_x, int* pos,
-                               cudaStream_t s) {
+cudaError_t prefill_tail_state(const float* xkv, int ld, int width, const void* x, int x_bf16, int d, int B, int S,
+                               int blk, float* blk_sum, double* blk_x, int* pos, cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
   if (x_bf16)
-    prefill_tail_kernel<bf16><<<B, 256, 0, s>>>(xkv, ld, width, proj, ldp, nb, eps, (const bf16*)x, d, S, blk, blk_sum,
-                                                blk_p, blk_eps, blk_x, pos);
+    prefill_tail_kernel<bf16><<<B, 256, 0, s>>>(xkv, ld, width, (const bf16*)x, d, S, blk, blk_sum, blk_x, pos);
   else
-    prefill_tail_kernel<float><<<B, 256, 0, s>>>(xkv, ld, width, proj, ldp, nb, eps, (const float*)x, d, S, blk,
-                                                 blk_sum, blk_p, blk_eps, blk_x, pos);
+    prefill_tail_kernel<float><<<B, 256, 0, s>>>(xkv, ld, width, (const float*)x, d, S, blk, blk_sum, blk_x, pos);
   return cudaGetLastError();
 }
 
