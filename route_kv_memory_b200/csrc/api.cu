@@ -385,7 +385,7 @@ int mka_router(const mka_config* cfg, const void* q, const void* w_r1, const voi
   Epilogue ep{};
   ep.nseg = 1;
   ep.seg[0] = OutSeg{0, d.rh, h, d.rh, 0};
-  if (d.bf16) CUDA_TRY(gemm_tn_bf16(q, d.dq, w1T, d.dq, d.T, d.rh, d.dq, ep, s));
+  if (d.bf16) CUDA_TRY(gemm_tn_bf16_tc(q, d.dq, w1T, d.dq, d.T, d.rh, d.dq, ep, status_ptr(), s));
   else CUDA_TRY(gemm_tn_ffma(q, d.dq, 0, w1T, d.dq, 0, d.T, d.rh, d.dq, ep, s));
   CUDA_TRY(router_tail(h, nullptr, d.rh, d.T, d.rh, wr2, lambda, s));
   return MKA_OK;
@@ -439,7 +439,7 @@ int mka_longterm_recall(const mka_config* cfg, const void* x, const void* hash_p
   Epilogue ep{};
   ep.nseg = 1;
   ep.seg[0] = OutSeg{0, d.nb, proj, d.nb, 0};
-  if (d.bf16) CUDA_TRY(gemm_tn_bf16(x, d.d, pT, d.d, d.T, d.nb, d.d, ep, s));
+  if (d.bf16) CUDA_TRY(gemm_tn_bf16_tc(x, d.d, pT, d.d, d.T, d.nb, d.d, ep, status_ptr(), s));
   else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, pT, d.d, 0, d.T, d.nb, d.d, ep, s));
   HashArgs ha{proj, d.nb, x, d.bf16, pT64, d.d, d.nb, d.d};
   CUDA_TRY(token_codes(ha, d.T, tcode, s));
@@ -507,7 +507,7 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   if (d.bf16) ep.seg[ns++] = OutSeg{PL.seg_rlo, PL.seg_rlo + d.rh, h2, d.rh, 0};
   ep.seg[ns++] = OutSeg{PL.seg_p, PL.Ntot, proj, d.nb, 0};
   ep.nseg = ns;
-  if (d.bf16) CUDA_TRY(gemm_tn_bf16(x, d.d, wcat, d.d, d.T, PL.Ntot, d.d, ep, s));
+  if (d.bf16) CUDA_TRY(gemm_tn_bf16_tc(x, d.d, wcat, d.d, d.T, PL.Ntot, d.d, ep, status_ptr(), s));
   else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, wcat, d.d, 0, d.T, PL.Ntot, d.d, ep, s));
   STAGE(s);
   // 2. router tail

@@ -1,7 +1,7 @@
-// Dense projections of the FastMKA layer: X [T, d] times the packed weight
-// matrix [W_q | W_k | W_v | W_q W_r1 | P]^T (notes §2-§3 of the MKA paper:
-// q = X W_q feeds the router and the attention, K/V come from X_fused W_k,v,
-// which is linear in X's projections).  Both operands are K-major ("TN").
+// CUDA-core pieces of the dense projections: the float32 FFMA GEMM (float32
+// workloads, where tensor-core TF32 would break the float32 tolerance, and the
+// one-time fold W_q W_r1), the shared epilogue store, and weight packing
+// (transposes, bf16 hi/lo split).  The bf16 GEMM runs on tcgen05 (tc_gemm.cu).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,127 +43,6 @@ __device__ __forceinline__ void ep_store2(const Epilogue& ep, int m, int n, floa
     }
   }
   if (n + 1 < N) ep_store1(ep, m, n + 1, v1);
-}
-
-// ---------------------------------------------------------------- bf16 tensor-core GEMM (mma.sync)
-namespace tc {
-constexpr int BM = 128, BN = 128, BK = 64, STAGES = 3, NT = 256;
-constexpr int SMEM = STAGES * (BM + BN) * BK * 2;
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N> __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
-__device__ __forceinline__ void ldsm_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, const uint32_t* b) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// Tile rows are BK = 64 bf16 = 128 B = 8 chunks of 16 B; chunk c of row r lives at c ^ (r & 7).
-__device__ __forceinline__ int swz(int r, int c) { return r * BK + ((c ^ (r & 7)) << 3); }
-
-__global__ void __launch_bounds__(NT) gemm_tn_bf16_kernel(const bf16* __restrict__ A, int lda,
-                                                          const bf16* __restrict__ B, int ldb, int M, int N, int K,
-                                                          Epilogue ep) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  bf16* sA = (bf16*)smem_raw;
-  bf16* sB = sA + STAGES * BM * BK;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-  const int wm = warp >> 2, wn = warp & 3;  // 2 x 4 warps, warp tile 64 x 32
-  const int KT = (K + BK - 1) / BK;
-
-  auto load_stage = [&](int stage, int kt) {
-    bf16* a = sA + stage * BM * BK;
-    bf16* b = sB + stage * BN * BK;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int c = tid + i * NT, r = c >> 3, ch = c & 7;
-      int gk = kt * BK + ch * 8;
-      int gm = m0 + r;
-      bool ok = gm < M && gk < K;
-      cp_async16(smem_u32(a + swz(r, ch)), ok ? (const void*)(A + (size_t)gm * lda + gk) : (const void*)A, ok ? 16 : 0);
-      int gn = n0 + r;
-      ok = gn < N && gk < K;
-      cp_async16(smem_u32(b + swz(r, ch)), ok ? (const void*)(B + (size_t)gn * ldb + gk) : (const void*)B, ok ? 16 : 0);
-    }
-  };
-
-  float acc[4][4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[i][j][k] = 0.f;
-
-#pragma unroll
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (s < KT) load_stage(s, s);
-    cp_commit();
-  }
-  for (int kt = 0; kt < KT; ++kt) {
-    cp_wait<STAGES - 2>();
-    __syncthreads();
-    int nk = kt + STAGES - 1;
-    if (nk < KT) load_stage(nk % STAGES, nk);
-    cp_commit();
-    const bf16* a = sA + (kt % STAGES) * BM * BK;
-    const bf16* b = sB + (kt % STAGES) * BN * BK;
-#pragma unroll
-    for (int kk = 0; kk < BK / 16; ++kk) {
-      uint32_t af[4][4], bfr[4][2];
-#pragma unroll
-      for (int mi = 0; mi < 4; ++mi) {
-        int r = wm * 64 + mi * 16 + (lane & 15);
-        int ch = kk * 2 + (lane >> 4);
-        ldsm_x4(af[mi][0], af[mi][1], af[mi][2], af[mi][3], smem_u32(a + swz(r, ch)));
-      }
-#pragma unroll
-      for (int nj = 0; nj < 2; ++nj) {
-        int r = wn * 32 + nj * 16 + ((lane >> 4) << 3) + (lane & 7);
-        int ch = kk * 2 + ((lane >> 3) & 1);
-        ldsm_x4(bfr[2 * nj][0], bfr[2 * nj][1], bfr[2 * nj + 1][0], bfr[2 * nj + 1][1], smem_u32(b + swz(r, ch)));
-      }
-#pragma unroll
-      for (int mi = 0; mi < 4; ++mi)
-#pragma unroll
-        for (int ni = 0; ni < 4; ++ni) mma_bf16(acc[mi][ni], af[mi], bfr[ni]);
-    }
-  }
-  cp_wait<0>();
-
-#pragma unroll
-  for (int mi = 0; mi < 4; ++mi)
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni) {
-      int m = m0 + wm * 64 + mi * 16 + (lane >> 2);
-      int n = n0 + wn * 32 + ni * 8 + (lane & 3) * 2;
-      if (n < N) {
-        ep_store2(ep, m, n, acc[mi][ni][0], acc[mi][ni][1], M, N);
-        ep_store2(ep, m + 8, n, acc[mi][ni][2], acc[mi][ni][3], M, N);
-      }
-    }
-}
-}  // namespace tc
-
-cudaError_t gemm_tn_bf16(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
-                         cudaStream_t s) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
-  cudaError_t e = set_max_smem(tc::gemm_tn_bf16_kernel, tc::SMEM, s);
-  if (e != cudaSuccess) return e;
-  dim3 grid((N + tc::BN - 1) / tc::BN, (M + tc::BM - 1) / tc::BM);
-  tc::gemm_tn_bf16_kernel<<<grid, tc::NT, tc::SMEM, s>>>((const bf16*)A, lda, (const bf16*)B, ldb, M, N, K, ep);
-  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- FFMA GEMM (float32 workloads, weight folding)

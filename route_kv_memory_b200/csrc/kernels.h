@@ -25,8 +25,10 @@ struct Epilogue {
 
 // C[M, N] = A[M, K] * B[N, K]^T (both operands K-major), float32 accumulation.
 // bf16 operands on tensor cores; `f32` variants use CUDA-core FFMA (no TF32).
-cudaError_t gemm_tn_bf16(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
-                         cudaStream_t s);
+// The bf16 path is the persistent tcgen05 kernel of tc_gemm.cu (K, lda, ldb multiples of 8;
+// A and B 16-byte aligned); a bounded wait that runs out records MKA_ERR_DEVICE_TIMEOUT in *status.
+cudaError_t gemm_tn_bf16_tc(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
+                            int* status, cudaStream_t s);
 cudaError_t gemm_tn_ffma(const void* A, int lda, int a_bf16, const void* B, int ldb, int b_bf16, int M, int N, int K,
                          const Epilogue& ep, cudaStream_t s);
 

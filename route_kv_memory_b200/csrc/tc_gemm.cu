@@ -1,0 +1,277 @@
+// Tensor-core (tcgen05) GEMM for the layer's dense projections:
+// C[M, N] = A[M, K] * B[N, K]^T with bf16 operands and a float32 accumulator
+// (MKA paper notes §2-§3: q = X W_q, X W_k, X W_v, the folded router layer
+// X (W_q W_r1), and the L3 projection X P all share the A operand X, so they run
+// as one GEMM over the packed weight matrix).
+//
+// Persistent kernel, one CTA per SM, 192 threads:
+//   warp 0      TMA producer: A and B tiles (128x64 and 256x64, 128-B swizzle)
+//               into a 4-stage shared-memory ring
+//   warp 1      MMA issuer: 4 x tcgen05.mma (128x256x16) per stage into one of
+//               two TMEM accumulators (2 x 256 columns); tcgen05.commit frees the
+//               stage and, after the last k-block, hands the accumulator over
+//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time (each thread owns one
+//               output row), convert and store per output segment, then
+//               release the accumulator.  The epilogue of tile i overlaps the
+//               main loop of tile i+1.
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace mka {
+namespace tcg {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int NTHREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+__device__ __forceinline__ void store1(const Epilogue& ep, int m, int n, float v) {
+#pragma unroll
+  for (int s = 0; s < kMaxSegs; ++s) {
+    if (s >= ep.nseg) break;
+    const OutSeg& g = ep.seg[s];
+    if (n >= g.n_begin && n < g.n_end) {
+      size_t off = (size_t)m * g.ld + (n - g.n_begin);
+      if (g.is_bf16) ((bf16*)g.ptr)[off] = __float2bfloat16_rn(v);
+      else ((float*)g.ptr)[off] = v;
+      return;
+    }
+  }
+}
+
+// Columns n .. n+31 of row m.
+__device__ __forceinline__ void store_chunk(const Epilogue& ep, int m, int n, const uint32_t (&r)[32], int N) {
+#pragma unroll
+  for (int s = 0; s < kMaxSegs; ++s) {
+    if (s >= ep.nseg) break;
+    const OutSeg& g = ep.seg[s];
+    if (n >= g.n_begin && n + 32 <= g.n_end && n + 32 <= N) {
+      const size_t off = (size_t)m * g.ld + (n - g.n_begin);
+      if (g.is_bf16) {
+        bf16* p = (bf16*)g.ptr + off;
+        if ((off & 7) == 0) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            uint32_t* w = (uint32_t*)&u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * e]), __uint_as_float(r[v * 8 + 2 * e + 1]));
+              w[e] = *(uint32_t*)&h;
+            }
+            *(uint4*)(p + v * 8) = u;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) p[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+        }
+      } else {
+        float* p = (float*)g.ptr + off;
+        if ((off & 3) == 0) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            *(float4*)(p + v * 4) = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) p[i] = __uint_as_float(r[i]);
+        }
+      }
+      return;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (n + i < N) store1(ep, m, n + i, __uint_as_float(r[i]));
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
+                   Epilogue ep, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  volatile int* abort = (volatile int*)(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  const int nM = (M + BM - 1) / BM, nN = (N + BN - 1) / BN, ntiles = nM * nN;
+  const int kblocks = (K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int it = 0;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
+        for (int k = 0; k < kblocks; ++k, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1, abort, status)) goto producer_done;
+          uint8_t* st = smem + s * STAGE_BYTES;
+          mbar_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_2d(st, &tmA, &full[s], k * BK, m0);
+          tma_load_2d(st + A_BYTES, &tmB, &full[s], k * BK, n0);
+        }
+      }
+    producer_done:
+      // On an abort, let the copies already issued land before the CTA unwinds:
+      // for each stage, wait (100 ms at most) for its most recent load.
+      if (*abort) {
+        for (int s = 0; s < STAGES; ++s) {
+          if (it - 1 < s) continue;
+          const int last = s + ((it - 1 - s) / STAGES) * STAGES;
+          const unsigned long long t0 = globaltimer();
+          while (!mbar_try_wait(&full[s], (last / STAGES) & 1) && globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int it = 0, tl = 0;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
+        const int acc = tl & 1;
+        const uint32_t aph = (tl >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1, abort, status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tbase + acc * BN;
+        bool ok = true;
+        for (int k = 0; k < kblocks; ++k, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&full[s], ph, abort, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* st = smem + s * STAGE_BYTES;
+          const uint64_t a_desc = sdesc_kmajor_sw128(st);
+          const uint64_t b_desc = sdesc_kmajor_sw128(st + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_ss(d_tmem, a_desc + (uint64_t)(kk * 2), b_desc + (uint64_t)(kk * 2), IDESC, (k | kk) != 0);
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+      if (*abort) {  // let the MMAs already issued finish before the TMEM is released
+        umma_commit(drain);
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    int tl = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
+      const int acc = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], aph, abort, status)) break;
+      tc_fence_after();
+      const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
+      const int m = m0 + q * 32 + lane;
+      for (int c = 0; c < BN; c += 32) {
+        if (n0 + c >= N) break;
+        uint32_t r[32];
+        tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + acc * BN + c, r);
+        tmem_ld_wait();
+        if (m < M) store_chunk(ep, m, n0 + c, r, N);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  }
+  return fn;
+}
+
+}  // namespace tcg
+
+// bf16 [rows, cols] row-major (row stride ld elements) as a 2-D TMA tensor with a
+// box of box_rows x 64 columns and 128-byte swizzle; out-of-range reads give zeros.
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows) {
+  auto fn = tcg::encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t gemm_tn_bf16_tc(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
+                            int* status, cudaStream_t s) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  if ((K % 8) || (lda % 8) || (ldb % 8) || ((uintptr_t)A & 15) || ((uintptr_t)B & 15)) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  cudaError_t e = make_tmap_bf16(&ta, A, M, K, lda, tcg::BM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16(&tb, B, N, K, ldb, tcg::BN);
+  if (e != cudaSuccess) return e;
+  e = set_max_smem(tcg::gemm_tc_kernel, tcg::SMEM_BYTES, s);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ntiles = ((M + tcg::BM - 1) / tcg::BM) * ((N + tcg::BN - 1) / tcg::BN);
+  const int grid = ntiles < sms ? ntiles : sms;
+  tcg::gemm_tc_kernel<<<grid, tcg::NTHREADS, tcg::SMEM_BYTES, s>>>(ta, tb, M, N, K, ep, status);
+  return cudaGetLastError();
+}
+
+}  // namespace mka
