@@ -540,7 +540,8 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   aa.k = kbuf; aa.v = vbuf; aa.kv_bstride = kv_bstride; aa.kv_ld = d.dkv;
   aa.o = out; aa.o_bstride = (long long)d.S * d.dq; aa.o_ld = d.dq;
   aa.B = d.B; aa.S = d.S; aa.Hq = d.Hq; aa.Hkv = d.Hkv; aa.dh = d.dh; aa.scale = d.scale;
-  CUDA_TRY(attention_prefill(aa, d.bf16, s));
+  if (d.bf16) CUDA_TRY(attention_prefill_tc(aa, status_ptr(), s));
+  else CUDA_TRY(attention_prefill(aa, 0, s));
   STAGE(s);
   if (state) {
     CUDA_TRY(prefill_tail_state(xkv, d.width, d.width, x, d.bf16, d.d, d.B, d.S, d.blk, (float*)P(state, SL.blk_sum),

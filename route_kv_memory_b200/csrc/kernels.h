@@ -103,6 +103,8 @@ struct AttnArgs {
   float scale;
 };
 cudaError_t attention_prefill(const AttnArgs& a, int bf16, cudaStream_t s);
+// bf16 path on tcgen05 (tc_attention.cu): persistent, TMA-fed, S and P in TMEM.
+cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode
 struct DecodeArgs {
