@@ -171,7 +171,7 @@ def run_ours(args, rank, world, local_rank):
                 "achieved": round(attn_tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
                 "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)",
-                "traffic": traffic_from_profiles("attention"), "avg_ms": round(attn_ms, 4),
+                "traffic": traffic_from_profiles("attention_tc"), "avg_ms": round(attn_ms, 4),
                 "flops_per_launch": fl["attention"]}
     layer_tflops = (fl["projections"] + fl["attention"]) / (ms / 1e3) / 1e12
 

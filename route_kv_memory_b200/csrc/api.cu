@@ -109,7 +109,7 @@ int check_cfg(const mka_config* c, Dims* o) {
 // ---------------------------------------------------------------- packed weights
 struct PackLayout {
   int Ntot, Npad, seg_q, seg_k, seg_v, seg_r, seg_rlo, seg_p, rh_segs;
-  size_t wcat, wr2, pT64, wqr32, wr1T, total;
+  size_t wcat, wr2, pT64, p64, wqr32, wr1T, total;
 };
 PackLayout pack_layout(const Dims& d) {
   PackLayout p;
@@ -126,6 +126,7 @@ PackLayout pack_layout(const Dims& d) {
   p.wcat = o; o += al((size_t)p.Npad * d.d * d.elem);
   p.wr2 = o; o += al((size_t)d.rh * 3 * 4);
   p.pT64 = o; o += al((size_t)d.nb * d.d * 8);
+  p.p64 = o; o += al((size_t)d.d * 32 * 8);
   p.wqr32 = o; o += al((size_t)d.rh * d.d * 4);
   p.wr1T = o; o += al((size_t)d.rh * d.dq * d.elem);
   p.total = o;
@@ -146,7 +147,7 @@ PrefillWs prefill_ws(const Dims& d) {
   w.proj = o; o += al(T * d.nb * 4);
   w.lam = o; o += al(T * 3 * 4);
   w.tcode = o; o += al(T * 4);
-  w.xsum = o; o += al((size_t)d.B * d.nblk * d.d * 8);
+  w.xsum = o; o += al(summary_codes_scratch(d.d, d.B, d.nblk));
   w.bsum = o; o += al((size_t)d.B * d.nblk * d.width * 4);
   w.bend = o; o += al((size_t)d.B * d.nblk * d.width * 4);
   w.gend = o; o += al((size_t)d.B * d.nblk * 8 * d.width * 4);
@@ -303,9 +304,9 @@ size_t mka_longterm_recall_workspace_size(const mka_config* cfg) {
   Dims d;
   if (check_cfg(cfg, &d) != MKA_OK) return 0;
   size_t T = d.T;
-  return al((size_t)d.nb * d.d * d.elem) + al((size_t)d.nb * d.d * 8) + al(T * d.nb * 4) + al(T * 4) +
-         al((size_t)d.B * d.nblk * d.d * 8) + al((size_t)d.B * d.nblk * d.d * 4) + al((size_t)d.B * d.nblk * 4) +
-         al(T * 4);
+  return al((size_t)d.nb * d.d * d.elem) + al((size_t)d.nb * d.d * 8) + al((size_t)d.d * 32 * 8) + al(T * d.nb * 4) +
+         al(T * 4) + al(summary_codes_scratch(d.d, d.B, d.nblk)) + al((size_t)d.B * d.nblk * d.d * 4) +
+         al((size_t)d.B * d.nblk * 4) + al(T * 4);
 }
 
 size_t mka_state_size(const mka_config* cfg, int32_t max_positions) {
@@ -339,6 +340,7 @@ int mka_pack_weights(const mka_config* cfg, const mka_weights* w, void* packed, 
   CUDA_TRY(transpose(w->w_v, d.d, d.dkv, d.dkv, wc + L.seg_v * row, d.d, d.elem, 0, s));
   CUDA_TRY(transpose(w->hash_proj, d.d, d.nb, d.nb, wc + L.seg_p * row, d.d, d.elem, 0, s));
   CUDA_TRY(transpose(w->hash_proj, d.d, d.nb, d.nb, P(packed, L.pT64), d.d, d.elem, 1, s));
+  CUDA_TRY(widen_pad32_f64(w->hash_proj, d.d, d.nb, d.bf16, (double*)P(packed, L.p64), s));
   CUDA_TRY(widen_f32(w->w_r2, d.rh * 3, d.bf16, (float*)P(packed, L.wr2), s));
   // Router fold: (W_q W_r1)^T [rh, d] = W_r1^T [rh, dq] . W_q^T, float32 accumulation.
   CUDA_TRY(transpose(w->w_r1, d.dq, d.rh, d.rh, P(packed, L.wr1T), d.dq, d.elem, 0, s));
@@ -428,14 +430,16 @@ int mka_longterm_recall(const mka_config* cfg, const void* x, const void* hash_p
   char* o = (char*)ws;
   void* pT = o; o += al((size_t)d.nb * d.d * d.elem);
   double* pT64 = (double*)o; o += al((size_t)d.nb * d.d * 8);
+  double* p64 = (double*)o; o += al((size_t)d.d * 32 * 8);
   float* proj = (float*)o; o += al(T * d.nb * 4);
   uint32_t* tcode = (uint32_t*)o; o += al(T * 4);
-  double* xsum = (double*)o; o += al((size_t)d.B * d.nblk * d.d * 8);
+  double* xsum = (double*)o; o += al(summary_codes_scratch(d.d, d.B, d.nblk));
   float* bsum = (float*)o; o += al((size_t)d.B * d.nblk * d.d * 4);
   uint32_t* scode = (uint32_t*)o; o += al((size_t)d.B * d.nblk * 4);
   int* cnt = count ? count : (int*)o;
   CUDA_TRY(transpose(hash_proj, d.d, d.nb, d.nb, pT, d.d, d.elem, 0, s));
   CUDA_TRY(transpose(hash_proj, d.d, d.nb, d.nb, pT64, d.d, d.elem, 1, s));
+  CUDA_TRY(widen_pad32_f64(hash_proj, d.d, d.nb, d.bf16, p64, s));
   Epilogue ep{};
   ep.nseg = 1;
   ep.seg[0] = OutSeg{0, d.nb, proj, d.nb, 0};
@@ -443,7 +447,7 @@ int mka_longterm_recall(const mka_config* cfg, const void* x, const void* hash_p
   else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, pT, d.d, 0, d.T, d.nb, d.d, ep, s));
   HashArgs ha{proj, d.nb, x, d.bf16, pT64, d.d, d.nb, d.d};
   CUDA_TRY(token_codes(ha, d.T, tcode, s));
-  CUDA_TRY(summary_codes(x, d.bf16, d.d, d.B, d.S, d.nblk, d.blk, pT64, d.nb, xsum, scode, d.nblk, s));
+  CUDA_TRY(summary_codes(x, d.bf16, d.d, d.B, d.S, d.nblk, d.blk, p64, d.nb, xsum, scode, d.nblk, s));
   CUDA_TRY(recall_select(tcode, scode, d.nblk, d.B, d.S, d.nblk, d.blk, d.R, idx, cnt, s));
   if (m3) {
     CUDA_TRY(block_reduce(x, d.bf16, d.d, d.d, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, (long long)d.nblk * d.d, nullptr,
@@ -519,7 +523,8 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   STAGE(s);
   CUDA_TRY(block_reduce(xkv, 0, d.width, d.width, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, bsum_bstride, bend, gend, s));
   STAGE(s);
-  CUDA_TRY(summary_codes(x, d.bf16, d.d, d.B, d.S, d.nblk, d.blk, ha.pT64, d.nb, xsum, scode, code_bstride, s));
+  CUDA_TRY(summary_codes(x, d.bf16, d.d, d.B, d.S, d.nblk, d.blk, (const double*)P((void*)packed, PL.p64), d.nb, xsum,
+                         scode, code_bstride, s));
   STAGE(s);
   CUDA_TRY(ema_carry(bend, d.width, d.B, d.nblk, (float)pow((double)d.alpha, (double)d.blk), nullptr, carry, s));
   STAGE(s);

@@ -168,6 +168,21 @@ cudaError_t split_hi_lo(const float* w, int n, void* hi, void* lo, cudaStream_t 
 }
 
 template <typename T>
+__global__ void widen_pad32_kernel(const T* __restrict__ in, int rows, int cols, double* __restrict__ out) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows * 32) return;
+  int r = i >> 5, c = i & 31;
+  out[i] = c < cols ? (double)to_f<T>(in[(size_t)r * cols + c]) : 0.0;
+}
+cudaError_t widen_pad32_f64(const void* in, int rows, int cols, int in_bf16, double* out, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  int n = rows * 32;
+  if (in_bf16) widen_pad32_kernel<bf16><<<(n + 255) / 256, 256, 0, s>>>((const bf16*)in, rows, cols, out);
+  else widen_pad32_kernel<float><<<(n + 255) / 256, 256, 0, s>>>((const float*)in, rows, cols, out);
+  return cudaGetLastError();
+}
+
+template <typename T>
 __global__ void widen_kernel(const T* __restrict__ in, int n, float* __restrict__ out) {
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = to_f<T>(in[i]);

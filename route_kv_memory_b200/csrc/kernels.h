@@ -54,10 +54,14 @@ struct HashArgs {
 cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, float* lam,
                         cudaStream_t s);
 cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, cudaStream_t s);
-// Codes of the full blocks: exact float64 block sums of x in d_model space (xsum scratch [B][nblk][d]),
-// projected in float64.  codes[b*code_bstride + j].
-cudaError_t summary_codes(const void* x, int x_bf16, int d, int B, int S, int nblk, int blk, const double* pT64,
-                          int nb, double* xsum, uint32_t* codes, int code_bstride, cudaStream_t s);
+// Codes of the full blocks from exact float64 block sums of x in d_model space projected in float64.
+// P64: [d][32] float64 (P row-major, padded to 32 columns).  part: summary_codes_scratch() bytes.
+// codes[b*code_bstride + j].
+size_t summary_codes_scratch(int d, int B, int nblk);
+cudaError_t summary_codes(const void* x, int x_bf16, int d, int B, int S, int nblk, int blk, const double* P64,
+                          int nb, double* part, uint32_t* codes, int code_bstride, cudaStream_t s);
+// out[r][0..31] = in[r][0..cols) widened to float64, zero padded (in: [rows, cols] bf16 or float32).
+cudaError_t widen_pad32_f64(const void* in, int rows, int cols, int in_bf16, double* out, cudaStream_t s);
 // Per full block j of each sequence: bsum = sum of its rows, bend = EMA end state from a zero carry,
 // gend = the zero-carry EMA end state of each of its 8 row groups (all three nullable).
 // x: [B*S, ld] (bf16 or float32), first `width` columns.  bsum[b*bsum_bstride + j*width + c],

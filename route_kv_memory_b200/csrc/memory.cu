@@ -67,16 +67,26 @@ template <> struct Vec4<bf16> {
   }
 };
 // ---------------------------------------------------------------- L3 sign codes
-// The float32 projection p = x . P_k carries a rounding error far below
-// eps = K * 2^-20 * rms_k(p) (K * 2^-23 * |partial sum| is the worst-case
-// sequential bound; rms_k(p) estimates the partial sums' scale).  Signs of
-// projections within eps of zero are decided again from an exact float64 dot
-// product, so every code bit equals the sign of the exact projection.
+// The float32 projection p = x . P_k (a tensor-core or FFMA dot product of
+// length K) carries a rounding error below about K/16 * 2^-23 * |partial sum|
+// per step-accumulation, i.e. under K * 2^-23 * rms_k(p) for partial sums of a
+// few standard deviations (rms_k(p) estimates that scale).  Signs of
+// projections within eps = K * 2^-21 * rms_k(p) of zero (a 4x margin) are
+// decided again from an exact float64 dot product, so every code bit equals
+// the sign of the exact projection.
 template <typename T>
 __device__ __forceinline__ double dot_row_f64(const T* __restrict__ x, const double* __restrict__ p, int d, int lane) {
-  double acc = 0.0;
-  for (int i = lane; i < d; i += 32) acc = fma(to_d<T>(x[i]), p[i], acc);
-  return warp_sum_d(acc);
+  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+  int i = lane * 4;
+  for (; i + 3 < d; i += 128) {  // d is a multiple of 64: each lane takes 4 consecutive elements
+    float4 v = Vec4<T>::load(x + i);
+    const double2 p01 = *(const double2*)(p + i), p23 = *(const double2*)(p + i + 2);
+    a0 = fma((double)v.x, p01.x, a0);
+    a1 = fma((double)v.y, p01.y, a1);
+    a2 = fma((double)v.z, p23.x, a2);
+    a3 = fma((double)v.w, p23.y, a3);
+  }
+  return warp_sum_d((a0 + a1) + (a2 + a3));
 }
 
 template <typename T>
@@ -86,7 +96,7 @@ __global__ void token_codes_kernel(HashArgs a, int T_, uint32_t* __restrict__ co
   if (t >= T_) return;
   float p = lane < a.nb ? a.proj[(size_t)t * a.ldp + lane] : 0.f;
   float rms = sqrtf(warp_sum(p * p) / (float)a.nb);
-  float e = (float)a.K * 0x1p-20f * rms;
+  float e = (float)a.K * 0x1p-21f * rms;
   bool bit = p > 0.f;
   unsigned doubt = __ballot_sync(0xffffffffu, lane < a.nb && fabsf(p) <= e);
   const T* xr = (const T*)a.x + (size_t)t * a.d;
@@ -108,68 +118,103 @@ cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, cudaStream_t 
 }
 
 // Block codes.  The code of block j is the sign pattern of (sum of its rows) P,
-// the same signs as (block mean) P.  The block sums are formed exactly in
-// float64 in d_model space (sums of at most a few hundred bf16 or float32
-// values), then projected in float64: no float32 rounding enters the decision.
+// the same signs as (block mean) P.  Both are formed in float64 from the exact
+// inputs: the block's column sums in d_model space (sums of at most a few
+// hundred bf16 or float32 values), then dot products with P.  No float32
+// rounding enters the decision.
+//
+// Pass 1: CTA (64-column chunk c, sequence b, group of blocks).  For each block it
+// sums the block's rows over the chunk (16 row groups x 16 four-column threads),
+// then 32 x 8 threads form the 64-long partial dot products with P's chunk.
+// Pass 2: per block and bit, the partials are summed over the chunks in order.
+constexpr int kXChunk = 64;
+
 template <typename T>
-__global__ void __launch_bounds__(256) block_xsum_kernel(const T* __restrict__ x, int d, int S, int blk,
-                                                          int nblk, double* __restrict__ xsum) {
-  __shared__ double sacc[4][64][4];
-  const int bi = blockIdx.z, j = blockIdx.y;
-  const int cl = threadIdx.x & 63, rg = threadIdx.x >> 6;
-  const int c = (blockIdx.x * 64 + cl) * 4;
-  const int per = (blk + 3) / 4;
+__global__ void __launch_bounds__(256) block_proj_partial_kernel(const T* __restrict__ x, int d, int S, int blk,
+                                                                  int nblk, int blocks_per_group,
+                                                                  const double* __restrict__ P64, int nb,
+                                                                  double* __restrict__ part) {
+  __shared__ double Ps[kXChunk][33];
+  __shared__ double xs[16][kXChunk];
+  __shared__ double xt[kXChunk];
+  const int chunk = blockIdx.x, nchunk = gridDim.x, bi = blockIdx.y;
+  const int c0 = chunk * kXChunk;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kXChunk * 32; i += 256) {
+    int c = i >> 5, k = i & 31;
+    Ps[c][k] = (k < nb && c0 + c < d) ? P64[(size_t)(c0 + c) * 32 + k] : 0.0;
+  }
+  const int cq = tid & 15, rg = tid >> 4;
+  const int col = c0 + cq * 4;
+  const int per = (blk + 15) / 16;
   const int ra = min(rg * per, blk), rb = min(ra + per, blk);
-  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-  if (c < d) {
-    const T* p = x + ((size_t)bi * S + (size_t)j * blk) * d + c;
+  const int j0 = blockIdx.z * blocks_per_group, j1 = min(nblk, j0 + blocks_per_group);
+  const int k = tid >> 3, sub = tid & 7;
+  for (int j = j0; j < j1; ++j) {
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    if (col < d) {
+      const T* p = x + ((size_t)bi * S + (size_t)j * blk) * d + col;
 #pragma unroll 4
-    for (int r = ra; r < rb; ++r) {
-      float4 v = Vec4<T>::load(p + (size_t)r * d);
-      a0 += v.x;
-      a1 += v.y;
-      a2 += v.z;
-      a3 += v.w;
+      for (int r = ra; r < rb; ++r) {
+        float4 v = Vec4<T>::load(p + (size_t)r * d);
+        a0 += v.x;
+        a1 += v.y;
+        a2 += v.z;
+        a3 += v.w;
+      }
     }
-  }
-  sacc[rg][cl][0] = a0;
-  sacc[rg][cl][1] = a1;
-  sacc[rg][cl][2] = a2;
-  sacc[rg][cl][3] = a3;
-  __syncthreads();
-  if (rg == 0 && c < d) {
-    double* o = xsum + ((size_t)bi * nblk + j) * d + c;
+    xs[rg][cq * 4 + 0] = a0;
+    xs[rg][cq * 4 + 1] = a1;
+    xs[rg][cq * 4 + 2] = a2;
+    xs[rg][cq * 4 + 3] = a3;
+    __syncthreads();
+    if (tid < kXChunk) {
+      double t = 0.0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] = sacc[0][cl][e] + sacc[1][cl][e] + sacc[2][cl][e] + sacc[3][cl][e];
+      for (int g = 0; g < 16; ++g) t += xs[g][tid];
+      xt[tid] = t;
+    }
+    __syncthreads();
+    double v = 0.0;
+#pragma unroll
+    for (int c = sub; c < kXChunk; c += 8) v = fma(xt[c], Ps[c][k], v);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    if (sub == 0) part[(((size_t)bi * nblk + j) * nchunk + chunk) * 32 + k] = v;
+    __syncthreads();
   }
 }
 
-__global__ void __launch_bounds__(256) summary_codes_kernel(const double* __restrict__ xsum,
-                                                            const double* __restrict__ pT64, int d, int nb, int nblk,
-                                                            uint32_t* __restrict__ codes, int code_bstride) {
-  __shared__ unsigned s_code;
-  const int bi = blockIdx.y, j = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) s_code = 0u;
-  __syncthreads();
-  const double* v = xsum + ((size_t)bi * nblk + j) * d;
-  for (int k = warp; k < nb; k += 8) {
-    double acc = 0.0;
-    for (int i = lane; i < d; i += 32) acc = fma(v[i], pT64[(size_t)k * d + i], acc);
-    acc = warp_sum_d(acc);
-    if (lane == 0 && acc > 0.0) atomicOr(&s_code, 1u << k);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) codes[(size_t)bi * code_bstride + j] = s_code;
+__global__ void block_codes_kernel(const double* __restrict__ part, int nchunk, int nb, int nblk,
+                                   uint32_t* __restrict__ codes, int code_bstride) {
+  const int j = blockIdx.x, bi = blockIdx.y, lane = threadIdx.x;
+  const double* p = part + ((size_t)bi * nblk + j) * nchunk * 32 + lane;
+  double v = 0.0;
+  for (int c = 0; c < nchunk; ++c) v += p[(size_t)c * 32];
+  unsigned code = __ballot_sync(0xffffffffu, lane < nb && v > 0.0);
+  if (lane == 0) codes[(size_t)bi * code_bstride + j] = code;
 }
 
-cudaError_t summary_codes(const void* x, int x_bf16, int d, int B, int S, int nblk, int blk, const double* pT64,
-                          int nb, double* xsum, uint32_t* codes, int code_bstride, cudaStream_t s) {
+size_t summary_codes_scratch(int d, int B, int nblk) {
+  return (size_t)B * nblk * ((d + kXChunk - 1) / kXChunk) * 32 * sizeof(double);
+}
+
+cudaError_t summary_codes(const void* x, int x_bf16, int d, int B, int S, int nblk, int blk, const double* P64,
+                          int nb, double* part, uint32_t* codes, int code_bstride, cudaStream_t s) {
   if (B <= 0 || nblk <= 0) return cudaSuccess;
-  dim3 g1((d / 4 + 63) / 64, nblk, B);
-  if (x_bf16) block_xsum_kernel<bf16><<<g1, 256, 0, s>>>((const bf16*)x, d, S, blk, nblk, xsum);
-  else block_xsum_kernel<float><<<g1, 256, 0, s>>>((const float*)x, d, S, blk, nblk, xsum);
-  summary_codes_kernel<<<dim3(nblk, B), 256, 0, s>>>(xsum, pT64, d, nb, nblk, codes, code_bstride);
+  const int nchunk = (d + kXChunk - 1) / kXChunk;
+  // enough CTAs to stream X at full bandwidth: about 4 waves over the SMs
+  int groups = (4 * 148 + nchunk * B - 1) / (nchunk * B);
+  groups = groups < 1 ? 1 : (groups > nblk ? nblk : groups);
+  const int bpg = (nblk + groups - 1) / groups;
+  groups = (nblk + bpg - 1) / bpg;
+  dim3 g1(nchunk, B, groups);
+  if (x_bf16)
+    block_proj_partial_kernel<bf16><<<g1, 256, 0, s>>>((const bf16*)x, d, S, blk, nblk, bpg, P64, nb, part);
+  else
+    block_proj_partial_kernel<float><<<g1, 256, 0, s>>>((const float*)x, d, S, blk, nblk, bpg, P64, nb, part);
+  block_codes_kernel<<<dim3(nblk, B), 32, 0, s>>>(part, nchunk, nb, nblk, codes, code_bstride);
   return cudaGetLastError();
 }
 
