@@ -223,6 +223,13 @@ MKA_API const char* mka_last_error(void);
 MKA_API int mka_profile_enable(int enable);
 MKA_API int mka_profile_read(float* ms, int max_stages);
 
+/* Self-test of the device-side wait limit used by the tcgen05 kernels (not part of the
+ * layer; the paper has no counterpart).  Launches one CTA that waits on an mbarrier
+ * nothing arrives at, with a limit of limit_us microseconds (1 .. 1e6).  The wait gives
+ * up, records MKA_ERR_DEVICE_TIMEOUT in the status word (read it with mka_status) and
+ * the kernel returns.  *result (device int) is set to 0, or to 1 if the wait completed. */
+MKA_API int mka_selftest_wait_timeout(int limit_us, int* result, void* stream);
+
 /* Library version string. */
 MKA_API const char* mka_version(void);
 

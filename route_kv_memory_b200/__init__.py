@@ -38,7 +38,7 @@ EXPORTED = [
     "mka_longterm_recall_workspace_size", "mka_state_size", "mka_decode_workspace_size", "mka_pack_weights",
     "mka_state_init", "mka_router", "mka_session_ema", "mka_longterm_recall", "mka_prefill_forward",
     "mka_decode_step", "mka_status", "mka_last_error", "mka_version", "mka_profile_enable", "mka_profile_read",
-    "mka_session_ema_noalloc",
+    "mka_session_ema_noalloc", "mka_selftest_wait_timeout",
 ]
 
 
@@ -77,6 +77,7 @@ _SIGS = {
     "mka_version": (ctypes.c_char_p, []),
     "mka_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "mka_session_ema_noalloc": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _vp]),
+    "mka_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int, _vp, _vp]),
     "mka_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -215,6 +216,10 @@ def mka_profile_read(max_stages: int = 16) -> list:
     if n < 0:
         raise MKAError(n, "mka_profile_read")
     return [buf[i] for i in range(min(n, max_stages))]
+
+
+def mka_selftest_wait_timeout(limit_us: int, result: torch.Tensor, stream=None) -> None:
+    _check(_lib.mka_selftest_wait_timeout(limit_us, _ptr(result), _stream(stream)), "mka_selftest_wait_timeout")
 
 
 def mka_version() -> str:

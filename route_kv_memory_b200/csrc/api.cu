@@ -241,6 +241,14 @@ extern "C" {
 
 const char* mka_version(void) { return "fastmka-b200 0.1 (sm_100a)"; }
 
+int mka_selftest_wait_timeout(int limit_us, int* result, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000 || !result) return fail(MKA_ERR_INVALID_ARG, "limit_us in [1, 1e6] and result");
+  int* st = status_ptr();
+  if (!st) return fail(MKA_ERR_CUDA, "no CUDA device");
+  CUDA_TRY(selftest_wait_timeout(limit_us, st, result, (cudaStream_t)stream));
+  return MKA_OK;
+}
+
 int mka_profile_enable(int enable) {
   if (enable && !g_prof.created) {
     for (int i = 0; i <= kMaxStages; ++i) CUDA_TRY(cudaEventCreate(&g_prof.ev[i]));

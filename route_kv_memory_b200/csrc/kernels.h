@@ -134,4 +134,7 @@ struct DecodeArgs {
 };
 cudaError_t decode_step(const DecodeArgs& a, cudaStream_t s);
 
+// Waits `limit_us` on an mbarrier nothing arrives at; *result = 1 if the wait (wrongly) completed.
+cudaError_t selftest_wait_timeout(int limit_us, int* status, int* result, cudaStream_t s);
+
 }  // namespace mka

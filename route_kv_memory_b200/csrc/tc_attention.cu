@@ -2,19 +2,22 @@
 // attention over the fused K/V; §4: online max-shift, partial sums rescaled by
 // exp(mu_old - mu_new) when the running maximum grows).
 //
-// Persistent CTAs walk work items (sequence b, query head h, 128-row query tile i)
-// longest first.  Per item the CTA streams the 128-key tiles j <= i of KV group
-// g(h) = h / (Hq / Hkv):
-//   warp 0      TMA: the Q tile once, then K_j and V_j into a 2-stage ring
-//   warp 1      MMA: S_j = Q K_j^T into one of two TMEM score buffers, then
-//               O += P_j V_j with P_j read from TMEM (A operand) and V_j from
-//               shared memory as an MN-major B operand
-//   warps 2-5   softmax, one query row per thread: scale, causal mask, running
-//               maximum, P = exp2(s - m) packed to bf16 into TMEM over S_j; O is
-//               rescaled (TMEM load, scale, store) only when the running maximum
-//               of some row in the warp grew by more than 2^8, so the stale
-//               maximum bounds P by 256; at the end O / l goes to global memory.
-// TMEM: O in columns [0, 128), S/P buffers at [128, 256) and [256, 384).
+// Persistent CTAs walk work items (sequence b, query head h, pair p of 128-row
+// query tiles 2p and 2p+1) longest first.  Per item the CTA streams the 128-key
+// tiles j <= 2p+1 of KV group g(h) = h / (Hq / Hkv), shared by both query tiles:
+//   warp 0      TMA: both Q tiles once, then K_j and V_j into a 2-stage ring
+//   warp 1      MMA, ping-pong between the two query tiles t = 0, 1:
+//               S_t = Q_t K_j^T into TMEM, O_t += P_t V_j with P_t read from
+//               TMEM (A operand) and V_j from shared memory (MN-major B operand);
+//               while one softmax warpgroup works on S_0 the tensor pipe runs
+//               the other tile's P V and next S
+//   warps 2-5   softmax warpgroup of tile 0, warps 6-9 of tile 1, one query row
+//               per thread: running maximum over the row, P = 2^(s*scale*log2e - m)
+//               packed to bf16 into TMEM over S_t; O_t is rescaled (TMEM load,
+//               scale, store) only when a row's maximum grew by more than 2^8, so
+//               the stale maximum bounds P by 256; at the end O_t / l goes to
+//               global memory.
+// TMEM columns: O_0 [0,128), O_1 [128,256), S_0/P_0 [256,384), S_1/P_1 [384,512).
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
@@ -29,28 +32,26 @@ namespace tca {
 using namespace sm100;
 
 constexpr int BQ = 128, BKV = 128;
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t O_COL = 0, S_COL0 = 128;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
 template <int DH>
 struct Cfg {
-  static constexpr int Q_BYTES = BQ * DH * 2;
+  static constexpr int Q_BYTES = BQ * DH * 2;    // one query tile
   static constexpr int K_BYTES = BKV * DH * 2;
-  static constexpr int V_BYTES = BKV * DH * 2;
-  static constexpr int KV_BYTES = K_BYTES + V_BYTES;
-  static constexpr int HALF = 128 * 64 * 2;  // one 128-row x 64-column swizzled box
-  static constexpr int SMEM = Q_BYTES + 2 * KV_BYTES + 1024 + 256;
+  static constexpr int KV_BYTES = 2 * K_BYTES;   // K then V
+  static constexpr int HALF = 128 * 64 * 2;      // one 128-row x 64-column swizzled box
+  static constexpr int SMEM = 2 * Q_BYTES + 2 * KV_BYTES + 1024 + 256;
 };
 
 struct Work {
-  int b, h, qt;
+  int b, h, pair;
 };
-__device__ __forceinline__ Work work_item(int w, int B, int Hq, int nqt) {
+__device__ __forceinline__ Work work_item(int w, int B, int Hq, int npairs) {
   Work r;
   const int per = B * Hq;
-  r.qt = nqt - 1 - w / per;  // longest rows first
+  r.pair = npairs - 1 - w / per;  // longest rows first
   const int rem = w % per;
   r.h = rem % Hq;
   r.b = rem / Hq;
@@ -69,6 +70,12 @@ __device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(const void* tile) {
   return d;
 }
 
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -79,20 +86,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr uint32_t IDESC_O = idesc_bf16_f32_bmn(BQ, DH);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + C::Q_BYTES;  // stage st: K at st*KV_BYTES, V at st*KV_BYTES + K_BYTES
-  uint64_t* bars = (uint64_t*)(smem + C::Q_BYTES + 2 * C::KV_BYTES);
+  uint8_t* sQ = smem;                      // tile t at t * Q_BYTES
+  uint8_t* sKV = smem + 2 * C::Q_BYTES;    // stage st: K at st*KV_BYTES, V at + K_BYTES
+  uint64_t* bars = (uint64_t*)(smem + 2 * C::Q_BYTES + 2 * C::KV_BYTES);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;   // [2]
+  uint64_t* kv_full = bars + 2;   // [2] stages
   uint64_t* kv_empty = bars + 4;  // [2]
-  uint64_t* s_full = bars + 6;    // [2]
+  uint64_t* s_full = bars + 6;    // [2] query tiles
   uint64_t* p_full = bars + 8;    // [2]
-  uint64_t* pv_done = bars + 10;
-  uint64_t* o_full = bars + 11;
-  uint64_t* o_empty = bars + 12;
-  uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
+  uint64_t* pv_done = bars + 10;  // [2]
+  uint64_t* o_full = bars + 12;   // [2]
+  uint64_t* o_empty = bars + 14;  // [2]
+  uint64_t* drain = bars + 16;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 17);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -104,10 +111,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 4);
     }
-    mbar_init(pv_done, 1);
-    mbar_init(o_full, 1);
-    mbar_init(o_empty, 4);
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -117,11 +124,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  // TMEM column of O_t and of S_t / P_t
+#define O_COL(t) (128u * (uint32_t)(t))
+#define S_COL(t) (256u + 128u * (uint32_t)(t))
 
   const int nqt = (a.S + BQ - 1) / BQ;
-  const int nwork = a.B * a.Hq * nqt;
+  const int npairs = (nqt + 1) / 2;
+  const int nwork = a.B * a.Hq * npairs;
   const int G = a.Hq / a.Hkv;
-  const long long q_rows_per_b = a.q_bstride / a.q_ld;    // rows of the 2-D q view per sequence
+  const long long q_rows_per_b = a.q_bstride / a.q_ld;
   const long long kv_rows_per_b = a.kv_bstride / a.kv_ld;
 
   if (warp == 0) {
@@ -132,13 +143,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tma_prefetch_desc(&tmV);
       int wi = 0, kvit = 0;
       for (int w = blockIdx.x; w < nwork; w += gridDim.x, ++wi) {
-        const Work it = work_item(w, a.B, a.Hq, nqt);
+        const Work it = work_item(w, a.B, a.Hq, npairs);
         const int g = it.h / G;
         if (!mbar_wait(q_empty, (wi & 1) ^ 1, abort, status)) break;
-        mbar_expect_tx(q_full, C::Q_BYTES);
-        const int qy = (int)(it.b * q_rows_per_b) + it.qt * BQ;
-        for (int hb = 0; hb < NH; ++hb) tma_load_2d(sQ + hb * C::HALF, &tmQ, q_full, it.h * DH + hb * 64, qy);
-        const int nkv = it.qt + 1;
+        mbar_expect_tx(q_full, 2 * C::Q_BYTES);
+        for (int t = 0; t < 2; ++t) {
+          const int qy = (int)(it.b * q_rows_per_b) + (2 * it.pair + t) * BQ;
+          for (int hb = 0; hb < NH; ++hb)
+            tma_load_2d(sQ + t * C::Q_BYTES + hb * C::HALF, &tmQ, q_full, it.h * DH + hb * 64, qy);
+        }
+        const int nkv = 2 * it.pair + 2;
         bool ok = true;
         for (int j = 0; j < nkv; ++j, ++kvit) {
           const int st = kvit & 1;
@@ -165,60 +179,70 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int wi = 0, kvit = 0;
-      for (int w = blockIdx.x; w < nwork; w += gridDim.x, ++wi) {
-        const Work it = work_item(w, a.B, a.Hq, nqt);
-        const int nkv = it.qt + 1;
-        if (!mbar_wait(q_full, wi & 1, abort, status)) break;
-        tc_fence_after();
-        const uint64_t qd = sdesc_kmajor_sw128(sQ);
-        bool ok = true;
-        // S_0
-        auto issue_s = [&](int kv_index) -> bool {
-          const int st = kv_index & 1;
-          if (!mbar_wait(&kv_full[st], (kv_index >> 1) & 1, abort, status)) return false;
-          tc_fence_after();
-          const uint64_t kd = sdesc_kmajor_sw128(sKV + st * C::KV_BYTES);
-          const uint32_t d_tmem = tbase + S_COL0 + (kv_index & 1) * 128;
+      int wi = 0, kvit = 0, pc[2] = {0, 0};
+      bool ok = true;
+      const uint64_t qd0 = sdesc_kmajor_sw128(sQ), qd1 = sdesc_kmajor_sw128(sQ + C::Q_BYTES);
+      auto issue_s = [&](int t, int st) {
+        const uint64_t kd = sdesc_kmajor_sw128(sKV + st * C::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            const uint64_t off = (uint64_t)((kk >> 2) * (C::HALF >> 4) + (kk & 3) * 2);
-            umma_bf16_ss(d_tmem, qd + off, kd + off, IDESC_S, kk != 0);
-          }
-          umma_commit(&s_full[kv_index & 1]);
-          return true;
-        };
-        if (!issue_s(kvit)) break;
-        for (int j = 0; j < nkv; ++j) {
-          const int cur = kvit + j;
-          if (j + 1 < nkv) {
-            if (!issue_s(cur + 1)) {
-              ok = false;
-              break;
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint64_t off = (uint64_t)((kk >> 2) * (C::HALF >> 4) + (kk & 3) * 2);
+          umma_bf16_ss(tbase + S_COL(t), (t ? qd1 : qd0) + off, kd + off, IDESC_S, kk != 0);
+        }
+        umma_commit(&s_full[t]);
+      };
+      auto issue_pv = [&](int t, int st, int j) {
+        const uint64_t vd = sdesc_mnmajor_sw128(sKV + st * C::KV_BYTES + C::K_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          umma_bf16_ts(tbase + O_COL(t), tbase + S_COL(t) + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
+                       (j | kk) != 0);
+        umma_commit(&pv_done[t]);
+      };
+      for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x, ++wi) {
+        const Work it = work_item(w, a.B, a.Hq, npairs);
+        const int n0 = 2 * it.pair + 1, n1 = 2 * it.pair + 2;
+        if (!mbar_wait(q_full, wi & 1, abort, status)) break;
+        if (!mbar_wait(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
+        tc_fence_after();
+        issue_s(0, kvit & 1);
+        issue_s(1, kvit & 1);
+        for (int j = 0; j < n1; ++j) {
+          const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
+          bool next_ready = false;
+          if (j < n0) {
+            if (!mbar_wait(&p_full[0], pc[0] & 1, abort, status)) { ok = false; break; }
+            if (j == 0 && !mbar_wait(&o_empty[0], (wi & 1) ^ 1, abort, status)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(0, st, j);
+            ++pc[0];
+            if (j + 1 == n0) umma_commit(&o_full[0]);
+            if (j + 1 < n0) {
+              if (!mbar_wait(&kv_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
+              tc_fence_after();
+              next_ready = true;
+              issue_s(0, nst);
             }
           }
-          if (j + 1 == nkv) umma_commit(q_empty);  // last use of Q by this item
-          if (!mbar_wait(&p_full[cur & 1], (cur >> 1) & 1, abort, status)) {
-            ok = false;
-            break;
-          }
-          if (j == 0 && !mbar_wait(o_empty, (wi & 1) ^ 1, abort, status)) {
-            ok = false;
-            break;
-          }
+          if (!mbar_wait(&p_full[1], pc[1] & 1, abort, status)) { ok = false; break; }
+          if (j == 0 && !mbar_wait(&o_empty[1], (wi & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
-          const int st = cur & 1;
-          const uint64_t vd = sdesc_mnmajor_sw128(sKV + st * C::KV_BYTES + C::K_BYTES);
-          const uint32_t p_tmem = tbase + S_COL0 + (cur & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk)
-            umma_bf16_ts(tbase + O_COL, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), IDESC_O, (j | kk) != 0);
-          umma_commit(pv_done);
+          issue_pv(1, st, j);
+          ++pc[1];
           umma_commit(&kv_empty[st]);
+          if (j + 1 < n1) {
+            if (!next_ready) {
+              if (!mbar_wait(&kv_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
+              tc_fence_after();
+            }
+            issue_s(1, nst);
+          } else {
+            umma_commit(&o_full[1]);
+          }
         }
         if (!ok) break;
-        kvit += nkv;
-        umma_commit(o_full);
+        umma_commit(q_empty);
+        kvit += n1;
       }
       if (*abort) {
         umma_commit(drain);
@@ -228,104 +252,106 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue
+    // ------------------------------------------------------------ softmax + epilogue, tile t
+    const int t = (warp - 2) >> 2;           // 0 for warps 2-5, 1 for warps 6-9
     const int q4 = warp & 3;                 // TMEM lane quadrant
     const int r = q4 * 32 + lane;            // row within the query tile
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t s_tmem = tbase + lane_off + S_COL(t);
+    const uint32_t o_tmem = tbase + lane_off + O_COL(t);
     const float sl2 = a.scale * 1.4426950408889634f;
     int wi = 0, sit = 0;
     for (int w = blockIdx.x; w < nwork; w += gridDim.x, ++wi) {
-      const Work it = work_item(w, a.B, a.Hq, nqt);
-      const int nkv = it.qt + 1;
-      const int row = it.qt * BQ + r;
+      const Work it = work_item(w, a.B, a.Hq, npairs);
+      const int qt = 2 * it.pair + t;
+      const int nkv = qt + 1;
+      const int row = qt * BQ + r;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv; ++j, ++sit) {
-        const int buf = sit & 1;
-        if (!mbar_wait(&s_full[buf], (sit >> 1) & 1, abort, status)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait(&s_full[t], sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t s_tmem = tbase + lane_off + S_COL0 + buf * 128;
-        uint32_t sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(s_tmem + c * 32, *(uint32_t(*)[32])(sv + c * 32));
-        tmem_ld_wait();
         const bool diag = (j == nkv - 1);
-        const int key0 = j * BKV;
+        const int lim = row - j * BKV;  // keys c > lim are in the future of this row
+        // pass 1: row maximum of the raw scores
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float v = __uint_as_float(sv[c]) * sl2;
-          if (diag && key0 + c > row) v = -INFINITY;
-          sv[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+        for (int c = 0; c < BKV; c += 64) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(s_tmem + c, v0);
+          tmem_ld32(s_tmem + c + 32, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float f0 = (diag && c + e > lim) ? -INFINITY : __uint_as_float(v0[e]);
+            const float f1 = (diag && c + 32 + e > lim) ? -INFINITY : __uint_as_float(v1[e]);
+            mx = fmaxf(mx, fmaxf(f0, f1));
+          }
         }
-        // lazy rescale: move the reference maximum only when it is exceeded by > 2^8
+        mx *= sl2;
+        // lazy rescale: move the reference maximum only when it is exceeded by more than 2^8
         const bool need = mx > m_ref + RESCALE_THRESHOLD;
         float corr = 1.f;
         if (need) {
-          corr = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
+          corr = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
           m_ref = mx;
           l *= corr;
         }
-        const unsigned vote = __ballot_sync(0xffffffffu, need && j > 0);
-        if (vote) {  // rescale O rows of this warp once PV_{j-1} has landed
-          if (!mbar_wait(pv_done, (sit - 1) & 1, abort, status)) {
-            ok = false;
-            break;
-          }
+        if (__ballot_sync(0xffffffffu, need && j > 0)) {  // rescale O rows once PV_{j-1} has landed
+          if (!mbar_wait(&pv_done[t], (sit - 1) & 1, abort, status)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < DH; c += 32) {
             uint32_t ov[32];
-            tmem_ld32(tbase + lane_off + O_COL + c, ov);
+            tmem_ld32(o_tmem + c, ov);
             tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
             uint32_t lo[16], hi[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              lo[e] = ov[e];
-              hi[e] = ov[16 + e];
+              lo[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+              hi[e] = __float_as_uint(__uint_as_float(ov[16 + e]) * corr);
             }
-            tmem_st16(tbase + lane_off + O_COL + c, lo);
-            tmem_st16(tbase + lane_off + O_COL + c + 16, hi);
+            tmem_st16(o_tmem + c, lo);
+            tmem_st16(o_tmem + c + 16, hi);
           }
         }
-        // P = exp2(s - m_ref), packed bf16 pairs, written over the first 64 columns of S
-        const float mr = m_ref;
+        // pass 2: P = 2^(s*sl2 - m_ref) as bf16 pairs over the first 64 columns of S
+        const float nm = -m_ref;
         float lsum = 0.f;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c = 0; c < BKV; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(s_tmem + c, v);
+          tmem_ld_wait();
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = exp2f(__uint_as_float(sv[c4 * 32 + 2 * e]) - mr);
-            const float p1 = exp2f(__uint_as_float(sv[c4 * 32 + 2 * e + 1]) - mr);
+            float p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sl2, nm));
+            float p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sl2, nm));
+            if (diag && c + 2 * e > lim) p0 = 0.f;
+            if (diag && c + 2 * e + 1 > lim) p1 = 0.f;
             lsum += p0 + p1;
             __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
             pk[e] = *(uint32_t*)&hb;
           }
-          tmem_st16(s_tmem + c4 * 16, pk);
+          tmem_st16(s_tmem + c / 2, pk);
         }
         l += lsum;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[buf]);
+        if (lane == 0) mbar_arrive(&p_full[t]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 -> global
-      if (!mbar_wait(o_full, wi & 1, abort, status)) break;
+      // epilogue: O_t / l -> bf16 -> global
+      if (!mbar_wait(&o_full[t], wi & 1, abort, status)) break;
       tc_fence_after();
       const float inv = 1.f / l;
       bf16* orow = (bf16*)a.o + (size_t)it.b * a.o_bstride + (size_t)row * a.o_ld + (size_t)it.h * DH;
 #pragma unroll
       for (int c = 0; c < DH; c += 32) {
         uint32_t ov[32];
-        tmem_ld32(tbase + lane_off + O_COL + c, ov);
+        tmem_ld32(o_tmem + c, ov);
         tmem_ld_wait();
         if (row < a.S) {
 #pragma unroll
@@ -344,7 +370,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_empty);
+      if (lane == 0) mbar_arrive(&o_empty[t]);
     }
   }
   tc_fence_before();
@@ -353,6 +379,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
   }
+#undef O_COL
+#undef S_COL
 }
 
 }  // namespace tca
@@ -375,7 +403,8 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int nwork = a.B * a.Hq * ((a.S + tca::BQ - 1) / tca::BQ);
+  const int nqt = (a.S + tca::BQ - 1) / tca::BQ;
+  const int nwork = a.B * a.Hq * ((nqt + 1) / 2);
   const int grid = nwork < sms ? nwork : sms;
   if (a.dh == 128) {
     e = set_max_smem(tca::attn_tc_kernel<128>, tca::Cfg<128>::SMEM, s);

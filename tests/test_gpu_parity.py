@@ -215,3 +215,16 @@ def test_decode_capacity_is_a_device_status(mka):
     layer.decode(state, 64, x[:, 64].contiguous(), o)
     assert mka.mka_status() == mka.MKA_ERR_CAPACITY
     assert mka.mka_status() == 0
+
+
+def test_bounded_wait_reports_timeout(mka):
+    """A device wait that nothing satisfies gives up after its limit, records the timeout and returns."""
+    result = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    mka.mka_status()  # clear
+    mka.mka_selftest_wait_timeout(20000, result)  # 20 ms
+    assert mka.mka_status() == mka.MKA_ERR_DEVICE_TIMEOUT
+    assert int(result.item()) == 0
+    assert mka.mka_status() == 0
+    # the context is still usable
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum().item()) == 8.0
