@@ -164,7 +164,7 @@ PrefillWs prefill_ws(const Dims& d) {
 // ---------------------------------------------------------------- decode state
 struct StateLayout {
   int Lmax, maxblk;
-  size_t pos, kc, vc, ema, blk_sum, blk_x, summ, scode, total;
+  size_t pos, sync, kc, vc, ema, blk_sum, blk_x, summ, scode, total;
 };
 StateLayout state_layout(const Dims& d, int Lmax) {
   StateLayout s;
@@ -172,6 +172,7 @@ StateLayout state_layout(const Dims& d, int Lmax) {
   s.maxblk = Lmax / d.blk;
   size_t o = 0, B = d.B;
   s.pos = o; o += al(B * 4);
+  s.sync = o; o += al(2 * 4);
   s.kc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.vc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.ema = o; o += al(B * d.width * 4);
@@ -186,7 +187,8 @@ StateLayout state_layout(const Dims& d, int Lmax) {
 int decode_nsplit(const Dims& d, int Lmax) {
   int sms = sm_count();
   int ns;
-  if (d.bf16) ns = (sms + d.B * d.Hkv - 1) / (d.B * d.Hkv);
+  // fused bf16 launch: one attention unit per CTA not busy with the token update (32 of them)
+  if (d.bf16) ns = (2 * sms - 32) / (d.B * d.Hkv);
   else ns = (2 * sms + d.B * d.Hq - 1) / (d.B * d.Hq);
   int cap = (Lmax + 127) / 128;
   if (ns > cap) ns = cap;
@@ -591,6 +593,7 @@ int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size
   a.ema = (float*)P(state, SL.ema); a.blk_sum = (float*)P(state, SL.blk_sum); a.blk_x = (double*)P(state, SL.blk_x);
   a.summ = (float*)P(state, SL.summ); a.scode = (uint32_t*)P(state, SL.scode);
   a.y = (float*)P(ws, W.y); a.qf = (float*)P(ws, W.qf); a.part = (float*)P(ws, W.part); a.nsplit = W.nsplit;
+  a.sync = (unsigned*)P(state, SL.sync);
   a.status = status_ptr();
   prof_begin();
   a.prof = g_prof.on ? g_prof.ev : nullptr;

@@ -7,6 +7,7 @@
 //   4. merge     max-shift combination of the partials
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace mka {
 
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(const T* __restrict__ W, int 
 
 // ---------------------------------------------------------------- 2. per-token state update
 template <typename T>
-__global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
+__device__ void token_update(const DecodeArgs& a, const int bi) {
   __shared__ float s_red[32][4];
   __shared__ float s_lam[3];
   __shared__ int s_idx[64];
@@ -73,7 +74,6 @@ __global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
   __shared__ unsigned s_code;
   __shared__ int s_base[34], s_run[34];
   __shared__ unsigned s_scode;
-  const int bi = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   const float* y = a.y + (size_t)bi * a.Ntot;
   const int width = 2 * a.dkv;
@@ -236,6 +236,11 @@ __global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
   if (tid == 0) a.pos[bi] = pos + 1;
 }
 
+template <typename T>
+__global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
+  token_update<T>(a, blockIdx.x);
+}
+
 // ---------------------------------------------------------------- 3. split-KV attention, bf16 tensor cores
 namespace dk {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -263,25 +268,25 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *(uint32_t*)&v;
 }
-constexpr int TP = 32;  // positions per warp tile
+constexpr int TP = 16;  // positions per warp tile
 constexpr int NWD = 4;  // warps per CTA
 template <int DH> __device__ __forceinline__ int swz(int r, int c) { return r * DH + ((c ^ (r & 7)) << 3); }
 
-// Grid (nsplit, Hkv, B).  The G = Hq/Hkv query heads of a KV group are the rows
-// of one 16-row MMA tile (rows >= G are zero).  Each warp owns a 32-position
-// tile per step; the CTA streams its split through a 2-stage cp.async ring.
+// One split of one KV group: positions [split * chunk, ...) of cache[0, L).  The
+// G = Hq/Hkv query heads of the group are the rows of one 16-row MMA tile (rows
+// >= G are zero); q is read from qsrc (row stride qstride) and rounded to bf16.
+// Each warp owns a 32-position tile per step; the CTA (NWD warps) streams its
+// split through a 2-stage cp.async ring in smem_raw (2 * 2 * NWD * TP * DH bf16).
 template <int DH>
-__global__ void __launch_bounds__(NWD * 32) decode_attn_kernel(DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
+__device__ void attn_unit(const DecodeArgs& a, const int split, const int g, const int bi, const int L,
+                          const float* qsrc, const int qstride, uint8_t* smem_raw) {
   constexpr int CH = DH / 8;
   constexpr int TILE = TP * DH;  // elements of one K (or V) warp tile
   bf16* sK = (bf16*)smem_raw;                // [2][NWD][TP][DH]
   bf16* sV = sK + 2 * NWD * TILE;            // [2][NWD][TP][DH]
   __shared__ float s_m[NWD][16], s_l[NWD][16];
-  const int split = blockIdx.x, g = blockIdx.y, bi = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.Hq / a.Hkv;
-  const int L = a.pos[bi];  // cache length after the append
   const int step = NWD * TP;
   int chunk = (L + a.nsplit - 1) / a.nsplit;
   chunk = (chunk + step - 1) / step * step;
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(NWD * 32) decode_attn_kernel(DecodeArgs a) {
   // query fragments (rows = heads g*G .. g*G+G-1)
   uint32_t qf[DH / 16][4];
   {
-    const float* qb = a.qf + (size_t)bi * a.dq + (size_t)g * G * DH;
+    const float* qb = qsrc + (size_t)bi * qstride + (size_t)g * G * DH;
     int r0 = lane >> 2, r1 = r0 + 8;
 #pragma unroll
     for (int kk = 0; kk < DH / 16; ++kk) {
@@ -420,9 +425,9 @@ __global__ void __launch_bounds__(NWD * 32) decode_attn_kernel(DecodeArgs a) {
     s_l[warp][(lane >> 2) + 8] = l_r[1];
   }
   __syncthreads();
-  float* so = (float*)smem_raw;  // reuse the ring: [16][DH] merged output (after all loads finished)
-  for (int i = tid; i < 16 * DH; i += NWD * 32) so[i] = 0.f;
-  __syncthreads();
+  // Each warp parks its weighted rows in the (now idle) ring, then one pass sums the
+  // warps in a fixed order: deterministic, one barrier.
+  float* so = (float*)smem_raw;  // [NWD][16][DH]
   float M[2], Lsum[2], wgt[2];
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -435,26 +440,28 @@ __global__ void __launch_bounds__(NWD * 32) decode_attn_kernel(DecodeArgs a) {
     Lsum[r] = ls;
     wgt[r] = m_r[r] == -INFINITY ? 0.f : exp2f(m_r[r] - mm);
   }
-  for (int w = 0; w < NWD; ++w) {
-    if (warp == w) {
+  {
+    float* mine = so + (size_t)warp * 16 * DH;
 #pragma unroll
-      for (int i = 0; i < DH / 8; ++i) {
-        int c = i * 8 + (lane & 3) * 2;
-        int r0 = lane >> 2;
-        so[r0 * DH + c] += o[i][0] * wgt[0];
-        so[r0 * DH + c + 1] += o[i][1] * wgt[0];
-        so[(r0 + 8) * DH + c] += o[i][2] * wgt[1];
-        so[(r0 + 8) * DH + c + 1] += o[i][3] * wgt[1];
-      }
+    for (int i = 0; i < DH / 8; ++i) {
+      int c = i * 8 + (lane & 3) * 2;
+      int r0 = lane >> 2;
+      mine[r0 * DH + c] = o[i][0] * wgt[0];
+      mine[r0 * DH + c + 1] = o[i][1] * wgt[0];
+      mine[(r0 + 8) * DH + c] = o[i][2] * wgt[1];
+      mine[(r0 + 8) * DH + c + 1] = o[i][3] * wgt[1];
     }
-    __syncthreads();
   }
+  __syncthreads();
   // partial record per (b, head, split): [m (log2 units), l, o[DH] (unnormalised)]
   const int rec = DH + 2;
   for (int i = tid; i < G * DH; i += NWD * 32) {
     int r = i / DH, c = i % DH;
     int hq = g * G + r;
-    a.part[(((size_t)bi * a.Hq + hq) * a.nsplit + split) * rec + 2 + c] = so[r * DH + c];
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < NWD; ++w) v += so[((size_t)w * 16 + r) * DH + c];
+    a.part[(((size_t)bi * a.Hq + hq) * a.nsplit + split) * rec + 2 + c] = v;
   }
   if (warp == 0 && (lane & 3) == 0) {
 #pragma unroll
@@ -467,6 +474,12 @@ __global__ void __launch_bounds__(NWD * 32) decode_attn_kernel(DecodeArgs a) {
       }
     }
   }
+  __syncthreads();  // the next unit of this CTA reuses the shared memory
+}
+template <int DH>
+__global__ void __launch_bounds__(NWD * 32) decode_attn_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  attn_unit<DH>(a, blockIdx.x, blockIdx.y, blockIdx.z, a.pos[blockIdx.z], a.qf, a.dq, smem_raw);
 }
 }  // namespace dk
 
@@ -556,6 +569,415 @@ __global__ void decode_merge_kernel(DecodeArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- token update, parallel form
+// Per-token decisions, recomputed by every CTA of the fused launch (deterministic, cheap):
+// lambda (router), the code of x_new (exact sign decisions), and the recalled blocks.
+struct TokenDecision {
+  float lam[3];
+  int cnt;
+  int idx[64];
+};
+
+template <typename T>
+__device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, TokenDecision* td) {
+  __shared__ float s_red[32][3];
+  __shared__ unsigned s_code;
+  __shared__ int s_base[34], s_run[34];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const float* y = a.y + (size_t)bi * a.Ntot;
+  const float* h = y + a.dq + 2 * a.dkv;
+  const float* p = h + a.rh * a.rh_segs;
+  const T* xn = (const T*)a.x_new + (size_t)bi * a.d;
+  float z0 = 0.f, z1 = 0.f, z2 = 0.f;
+  for (int j = tid; j < a.rh; j += blockDim.x) {
+    float hv = h[j];
+    if (a.rh_segs == 2) hv += h[a.rh + j];
+    const float gv = gelu_erf(hv);
+    z0 = fmaf(gv, a.w_r2[j * 3], z0);
+    z1 = fmaf(gv, a.w_r2[j * 3 + 1], z1);
+    z2 = fmaf(gv, a.w_r2[j * 3 + 2], z2);
+  }
+  z0 = warp_sum(z0);
+  z1 = warp_sum(z1);
+  z2 = warp_sum(z2);
+  if (lane == 0) {
+    s_red[warp][0] = z0;
+    s_red[warp][1] = z1;
+    s_red[warp][2] = z2;
+  }
+  if (warp == 0) {  // code of x_new, same decision rule as the prefill path
+    const float pv = lane < a.nb ? p[lane] : 0.f;
+    const float rms = sqrtf(warp_sum(pv * pv) / (float)a.nb);
+    const float e = (float)a.d * 0x1p-21f * rms;
+    bool bit = pv > 0.f;
+    unsigned doubt = __ballot_sync(0xffffffffu, lane < a.nb && fabsf(pv) <= e);
+    while (doubt) {
+      const int k = __ffs(doubt) - 1;
+      doubt &= doubt - 1;
+      double acc = 0.0;
+      for (int i = lane; i < a.d; i += 32) acc = fma(to_d<T>(xn[i]), a.pT64[(size_t)k * a.d + i], acc);
+      acc = warp_sum_d(acc);
+      if (lane == k) bit = acc > 0.0;
+    }
+    const unsigned code = __ballot_sync(0xffffffffu, bit && lane < a.nb);
+    if (lane == 0) s_code = code;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float t0 = 0.f, t1 = 0.f, t2 = 0.f;
+    for (int w = 0; w < nw; ++w) {
+      t0 += s_red[w][0];
+      t1 += s_red[w][1];
+      t2 += s_red[w][2];
+    }
+    const float m = fmaxf(t0, fmaxf(t1, t2));
+    const float e0 = expf(t0 - m), e1 = expf(t1 - m), e2 = expf(t2 - m);
+    const float inv = 1.f / (e0 + e1 + e2);
+    td->lam[0] = e0 * inv;
+    td->lam[1] = e1 * inv;
+    td->lam[2] = e2 * inv;
+  }
+  // recall among the finished blocks: counting select by (distance, index)
+  const int n_elig = min(pos / a.blk, a.maxblk);
+  const uint32_t* bc = a.scode + (size_t)bi * a.maxblk;
+  if (warp == 0) {
+    const uint32_t code = s_code;
+    for (int i = lane; i < 34; i += 32) {
+      s_base[i] = 0;
+      s_run[i] = 0;
+    }
+    __syncwarp();
+    for (int j0 = 0; j0 < n_elig; j0 += 32) {
+      const int j = j0 + lane;
+      if (j < n_elig) atomicAdd(&s_base[__popc(code ^ bc[j])], 1);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      int acc = 0;
+      for (int dd = 0; dd < 34; ++dd) {
+        const int hh = s_base[dd];
+        s_base[dd] = acc;
+        acc += hh;
+      }
+      td->cnt = min(a.R, n_elig);
+    }
+    __syncwarp();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < n_elig; j0 += 32) {
+      const int j = j0 + lane;
+      const bool valid = j < n_elig;
+      const int dist = valid ? __popc(code ^ bc[j]) : 64 + lane;
+      const unsigned grp = __match_any_sync(0xffffffffu, dist);
+      const int rank = __popc(grp & lt);
+      const int ps = valid ? s_base[dist] + s_run[dist] + rank : a.R;
+      __syncwarp();
+      if (valid && ps < a.R) td->idx[ps] = j;
+      if (valid && rank == 0) s_run[dist] += __popc(grp);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+}
+
+// This CTA's share of the token's state update: fused K/V columns [c0, c1) appended at
+// `pos`, their EMA values and block sums, and d_model-space block sums [i0, i1).  A token
+// at the start of a block (pos % b == 0) starts the block sums from zero.
+template <typename T>
+__device__ void token_slice(const DecodeArgs& a, const int bi, const int pos, const TokenDecision* td, const int c0,
+                            const int c1, const int i0, const int i1) {
+  const int width = 2 * a.dkv;
+  const float* xkv = a.y + (size_t)bi * a.Ntot + a.dq;
+  const T* xn = (const T*)a.x_new + (size_t)bi * a.d;
+  const bool fresh = (pos % a.blk) == 0;
+  const float l0 = td->lam[0], l1 = td->lam[1], l2 = td->lam[2];
+  const int cnt = td->cnt;
+  const float s3 = cnt ? 1.f / ((float)cnt * (float)a.blk) : 0.f;
+  const float* summ = a.summ + (size_t)bi * a.maxblk * width;
+  float* ema = a.ema + (size_t)bi * width;
+  float* bsum = a.blk_sum + (size_t)bi * width;
+  for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
+    const float xv = xkv[c];
+    const float m2 = ema[c];
+    float m3 = 0.f;
+    for (int r = 0; r < cnt; ++r) m3 += summ[(size_t)td->idx[r] * width + c];
+    const float o = fmaf(l0, xv, fmaf(l1, m2, l2 * s3 * m3));
+    T* dst = (T*)(c < a.dkv ? a.kcache : a.vcache) + ((size_t)bi * a.Lmax + pos) * a.dkv + (c < a.dkv ? c : c - a.dkv);
+    *dst = from_f<T>(o);
+    ema[c] = fmaf(a.alpha, m2, (1.f - a.alpha) * xv);
+    bsum[c] = (fresh ? 0.f : bsum[c]) + xv;
+  }
+  double* bx = a.blk_x + (size_t)bi * a.d;
+  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) bx[i] = (fresh ? 0.0 : bx[i]) + to_d<T>(xn[i]);
+}
+
+// ---------------------------------------------------------------- fused decode step (bf16)
+// One cooperative launch, two CTAs per SM, NWD warps each:
+//   A  the projection row y = x_new [W_q | W_k | W_v | W_q W_r1 | P] for every sequence:
+//      each CTA streams its share of the packed weight rows (TMA bulk copies into a
+//      2-stage shared-memory ring) and forms the dot products from shared memory
+//   -- grid barrier --
+//   B  CTA b < B: the token update of sequence b (router, L3 recall, fuse, append the
+//      fused K/V row at position pos, EMA / block update, pos + 1); every other CTA:
+//      split-KV attention of the new queries over the old cache rows [0, pos)
+//   -- grid barrier --
+//   C  per (sequence, query head): merge the split partials and the new row's own
+//      term (its score against the appended K row, weight on the appended V row)
+// The two barriers are counters in the decode state, each wait bounded by a time
+// limit that records MKA_ERR_DEVICE_TIMEOUT.  All CTAs are co-resident
+// (cooperative launch), so the barrier cannot deadlock on scheduling.
+constexpr int kFusedRing = 2 * 2 * dk::NWD * dk::TP * 128 * 2;  // 64 KB: GEMV chunks, then K/V tiles
+static_assert(kFusedRing >= dk::NWD * 16 * 128 * 4, "attention merge scratch must fit the ring");
+
+__device__ bool grid_sync(unsigned* count, unsigned* gen, unsigned nblocks, int* status) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_ok = 1;
+    const unsigned g = *(volatile unsigned*)gen;
+    __threadfence();
+    if (atomicAdd(count, 1u) == nblocks - 1) {
+      atomicExch(count, 0u);
+      __threadfence();
+      atomicAdd(gen, 1u);
+    } else {
+      const unsigned long long t0 = sm100::globaltimer();
+      while (*(volatile unsigned*)gen == g) {
+        if (sm100::globaltimer() - t0 > sm100::kWaitLimitNs) {
+          set_status(status, kStatusTimeout);
+          s_ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   sm100::smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(sm100::smem_u32(bar))
+               : "memory");
+}
+
+// Block-wide sum / max of one value per thread (blockDim.x <= 1024).
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float u = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, u) : v + u;
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = red[0];
+  for (int w = 1; w < nw; ++w) t = is_max ? fmaxf(t, red[w]) : t + red[w];
+  return t;
+}
+
+constexpr int kMaxSplits = 512;
+
+// Combines the split partials (m in log2 units, l, unnormalised o) of (sequence bi, query
+// head hq) and, when the step appended a row at pos_old, that row's own term.
+template <int DH>
+__device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, const int pos_old) {
+  __shared__ float s_w[kMaxSplits];
+  __shared__ float red[32];
+  const int tid = threadIdx.x;
+  const int rec = DH + 2;
+  const int g = hq / (a.Hq / a.Hkv);
+  const float* pr = a.part + ((size_t)bi * a.Hq + hq) * a.nsplit * rec;
+  const bool has_new = pos_old < a.Lmax;
+  const bf16* kn = (const bf16*)a.kcache + ((size_t)bi * a.Lmax + pos_old) * a.dkv + (size_t)g * DH;
+  const bf16* vn = (const bf16*)a.vcache + ((size_t)bi * a.Lmax + pos_old) * a.dkv + (size_t)g * DH;
+  const float* q = a.y + (size_t)bi * a.Ntot + (size_t)hq * DH;
+  float s = 0.f;
+  if (has_new)
+    for (int c = tid; c < DH; c += blockDim.x)
+      s = fmaf(__bfloat162float(__float2bfloat16_rn(q[c])), __bfloat162float(kn[c]), s);
+  const float snew = block_reduce(s, false, red) * a.scale * 1.4426950408889634f;
+  float mloc = has_new ? snew : -INFINITY;
+  for (int sp = tid; sp < a.nsplit; sp += blockDim.x) {
+    const float m = pr[(size_t)sp * rec];
+    s_w[sp] = m;
+    mloc = fmaxf(mloc, m);
+  }
+  const float M = block_reduce(mloc, true, red);
+  float lloc = 0.f;
+  for (int sp = tid; sp < a.nsplit; sp += blockDim.x) {
+    const float m = s_w[sp];
+    const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+    s_w[sp] = w;
+    lloc += w * pr[(size_t)sp * rec + 1];
+  }
+  const float wn = has_new ? exp2f(snew - M) : 0.f;
+  const float Ls = block_reduce(lloc, false, red) + wn;  // also orders the s_w writes before the reads below
+  const float inv = 1.f / Ls;
+  for (int c = tid; c < DH; c += blockDim.x) {
+    float a0 = has_new ? wn * __bfloat162float(vn[c]) : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int sp = 0;
+    for (; sp + 3 < a.nsplit; sp += 4) {
+      a0 = fmaf(pr[(size_t)sp * rec + 2 + c], s_w[sp], a0);
+      a1 = fmaf(pr[(size_t)(sp + 1) * rec + 2 + c], s_w[sp + 1], a1);
+      a2 = fmaf(pr[(size_t)(sp + 2) * rec + 2 + c], s_w[sp + 2], a2);
+      a3 = fmaf(pr[(size_t)(sp + 3) * rec + 2 + c], s_w[sp + 3], a3);
+    }
+    for (; sp < a.nsplit; ++sp) a0 = fmaf(pr[(size_t)sp * rec + 2 + c], s_w[sp], a0);
+    ((bf16*)a.out)[(size_t)bi * a.dq + (size_t)hq * DH + c] = __float2bfloat16_rn(((a0 + a1) + (a2 + a3)) * inv);
+  }
+  __syncthreads();
+}
+
+template <int DH>
+__global__ void __launch_bounds__(dk::NWD * 32, 2) decode_fused_kernel(DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* ring = smem;
+  bf16* sx = (bf16*)(smem + kFusedRing);
+  uint64_t* gbar = (uint64_t*)(smem + kFusedRing + (((size_t)a.B * a.d * 2 + 15) & ~(size_t)15));
+  __shared__ int s_pos[kMaxDecodeBatch];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int NW = dk::NWD;
+  const unsigned nblk = gridDim.x;
+  if (tid < a.B) s_pos[tid] = a.pos[tid];  // positions before this step changes them
+  if (tid == 0) {
+    sm100::mbar_init(&gbar[0], 1);
+    sm100::mbar_init(&gbar[1], 1);
+    sm100::fence_barrier_init();
+  }
+  for (int i = tid; i < a.B * a.d / 8; i += blockDim.x) ((uint4*)sx)[i] = ((const uint4*)a.x_new)[i];
+  __syncthreads();
+
+  // ---- A: projection row, this CTA's share of the packed weight rows
+  {
+    const int rpc = (a.Ntot + (int)nblk - 1) / (int)nblk;
+    const int r0 = blockIdx.x * rpc, r1 = min(a.Ntot, r0 + rpc);
+    const size_t row_bytes = (size_t)a.d * 2;
+    const int CR = (int)((kFusedRing / 2) / row_bytes);  // rows per ring stage
+    const int nrows = max(0, r1 - r0);
+    const int nch = (nrows + CR - 1) / CR;
+    const bf16* W = (const bf16*)a.wcatT;
+    auto issue = [&](int c) {
+      if (tid == 0) {
+        const int ra = r0 + c * CR, rb = min(r1, ra + CR);
+        uint8_t* dst = ring + (size_t)(c & 1) * CR * row_bytes;
+        sm100::mbar_expect_tx(&gbar[c & 1], (uint32_t)((rb - ra) * row_bytes));
+        for (int r = ra; r < rb; ++r)
+          bulk_copy(dst + (size_t)(r - ra) * row_bytes, W + (size_t)r * a.d, (uint32_t)row_bytes, &gbar[c & 1]);
+      }
+    };
+    volatile int abort_flag = 0;
+    if (nch > 0) issue(0);
+    for (int c = 0; c < nch; ++c) {
+      if (c + 1 < nch) issue(c + 1);
+      if (!sm100::mbar_wait(&gbar[c & 1], (c >> 1) & 1, &abort_flag, a.status)) return;
+      const int ra = r0 + c * CR, rb = min(r1, ra + CR);
+      const bf16* wst = (const bf16*)(ring + (size_t)(c & 1) * CR * row_bytes);
+      for (int r = ra + warp; r < rb; r += NW) {
+        const bf16* wr = wst + (size_t)(r - ra) * a.d;
+        float acc[kMaxDecodeBatch];
+#pragma unroll
+        for (int b = 0; b < kMaxDecodeBatch; ++b) acc[b] = 0.f;
+        for (int i = lane * 8; i < a.d; i += 256) {
+          const uint4 wu = *(const uint4*)(wr + i);
+          const __nv_bfloat162* wh = (const __nv_bfloat162*)&wu;
+          float wf[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(wh[e]);
+            wf[2 * e] = f.x;
+            wf[2 * e + 1] = f.y;
+          }
+#pragma unroll
+          for (int b = 0; b < kMaxDecodeBatch; ++b) {
+            if (b < a.B) {
+              const uint4 xu = *(const uint4*)(sx + (size_t)b * a.d + i);
+              const __nv_bfloat162* xh = (const __nv_bfloat162*)&xu;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(xh[e]);
+                acc[b] = fmaf(wf[2 * e], f.x, acc[b]);
+                acc[b] = fmaf(wf[2 * e + 1], f.y, acc[b]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kMaxDecodeBatch; ++b) {
+          if (b < a.B) {
+            const float v = warp_sum(acc[b]);
+            if (lane == 0) a.y[(size_t)b * a.Ntot + r] = v;
+          }
+        }
+      }
+      __syncthreads();  // stage (c & 1) is free for chunk c + 2
+    }
+  }
+  if (!grid_sync(a.sync, a.sync + 1, nblk, a.status)) return;
+
+  // ---- B: split-KV attention over the old rows (units handed out from CTA ntok on), and the
+  // token update, split over the first ntok CTAs
+  {
+    const int ntok = min((int)nblk, 32);
+    const int units = a.B * a.Hkv * a.nsplit;
+    for (int u = ((int)blockIdx.x - ntok + (int)nblk) % (int)nblk; u < units; u += nblk) {
+      const int split = u % a.nsplit, g = (u / a.nsplit) % a.Hkv, bi = u / (a.nsplit * a.Hkv);
+      dk::attn_unit<DH>(a, split, g, bi, min(s_pos[bi], a.Lmax), a.y, a.Ntot, ring);
+    }
+    if ((int)blockIdx.x < ntok) {
+      __shared__ TokenDecision td;
+      const int width = 2 * a.dkv;
+      const int cpc = (width + ntok - 1) / ntok;  // fused columns per CTA
+      const int dpc = (a.d + ntok - 1) / ntok;    // d_model elements per CTA
+      for (int bi = 0; bi < a.B; ++bi) {
+        const int pos = s_pos[bi];
+        if (pos < 0 || pos >= a.Lmax) {
+          if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, kStatusCapacity);
+          continue;
+        }
+        const int c0 = min(width, (int)blockIdx.x * cpc), c1 = min(width, c0 + cpc);
+        const int i0 = min(a.d, (int)blockIdx.x * dpc), i1 = min(a.d, i0 + dpc);
+        token_decide<bf16>(a, bi, pos, &td);
+        token_slice<bf16>(a, bi, pos, &td, c0, c1, i0, i1);
+        __syncthreads();
+      }
+      if (blockIdx.x == 0 && threadIdx.x < a.B && s_pos[threadIdx.x] < a.Lmax)
+        a.pos[threadIdx.x] = s_pos[threadIdx.x] + 1;
+    }
+  }
+  if (!grid_sync(a.sync, a.sync + 1, nblk, a.status)) return;
+
+  // ---- C: merge, and finish a block completed by this token: its projected sum becomes
+  // the summary, its code the signs of the exact float64 d_model-space sum projected on P
+  for (int u = blockIdx.x; u < a.B * a.Hq; u += nblk) merge_unit<DH>(a, u / a.Hq, u % a.Hq, s_pos[u / a.Hq]);
+  {
+    const int width = 2 * a.dkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int bi = 0; bi < a.B; ++bi) {
+      const int pos = s_pos[bi];
+      if (pos < 0 || pos >= a.Lmax || (pos + 1) % a.blk != 0 || pos / a.blk >= a.maxblk) continue;
+      const int j = pos / a.blk;
+      const float* bsum = a.blk_sum + (size_t)bi * width;
+      float* summ = a.summ + ((size_t)bi * a.maxblk + j) * width;
+      for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < width; c += nblk * blockDim.x) summ[c] = bsum[c];
+      // bit k on CTA (nblk - 1 - k), one warp per bit
+      const int k = (int)nblk - 1 - (int)blockIdx.x;
+      if (k >= 0 && k < a.nb && warp == 0) {
+        const double* bx = a.blk_x + (size_t)bi * a.d;
+        double v = 0.0;
+        for (int i = lane; i < a.d; i += 32) v = fma(bx[i], a.pT64[(size_t)k * a.d + i], v);
+        v = warp_sum_d(v);
+        if (lane == 0 && v > 0.0) atomicOr(a.scode + (size_t)bi * a.maxblk + j, 1u << k);
+      }
+    }
+  }
+}
+
+size_t decode_fused_smem(int B, int d) { return kFusedRing + (((size_t)B * d * 2 + 15) & ~(size_t)15) + 64; }
+
 cudaError_t decode_step(const DecodeArgs& a, cudaStream_t s) {
   if (a.B <= 0) return cudaSuccess;
   if (a.B > kMaxDecodeBatch) return cudaErrorInvalidValue;
@@ -565,25 +987,33 @@ cudaError_t decode_step(const DecodeArgs& a, cudaStream_t s) {
   if (a.prof) cudaEventRecord(a.prof[i], s);
   MARK(0);
   if (a.x_bf16) {
-    e = set_max_smem(gemv_kernel<bf16>, smx, s);
+    const size_t sm = decode_fused_smem(a.B, a.d);
+    if (sm > 227 * 1024) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    e = a.dh == 128 ? set_max_smem(decode_fused_kernel<128>, sm, s) : set_max_smem(decode_fused_kernel<64>, sm, s);
     if (e != cudaSuccess) return e;
-    gemv_kernel<bf16><<<(a.Ntot + 7) / 8, 256, smx, s>>>((const bf16*)a.wcatT, a.Ntot, a.d, (const bf16*)a.x_new, a.B, a.y);
+    cudaLaunchConfig_t cfg = {};
+    int occ = 1;
+    if (a.dh == 128) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_fused_kernel<128>, dk::NWD * 32, sm);
+    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_fused_kernel<64>, dk::NWD * 32, sm);
+    if (occ < 1) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3((occ >= 2 ? 2 : 1) * sms);  // co-resident CTAs (two per SM when they fit)
+    cfg.blockDim = dim3(dk::NWD * 32);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (a.dh == 128) e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<128>, a);
+    else e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<64>, a);
+    if (e != cudaSuccess) return e;
     MARK(1);
-    token_kernel<bf16><<<a.B, 1024, 0, s>>>(a);
     MARK(2);
-    size_t sm = (size_t)2 * 2 * dk::NWD * dk::TP * a.dh * sizeof(bf16);
-    dim3 grid(a.nsplit, a.Hkv, a.B);
-    if (a.dh == 128) {
-      e = set_max_smem(dk::decode_attn_kernel<128>, sm, s);
-      if (e != cudaSuccess) return e;
-      dk::decode_attn_kernel<128><<<grid, dk::NWD * 32, sm, s>>>(a);
-    } else {
-      e = set_max_smem(dk::decode_attn_kernel<64>, sm, s);
-      if (e != cudaSuccess) return e;
-      dk::decode_attn_kernel<64><<<grid, dk::NWD * 32, sm, s>>>(a);
-    }
     MARK(3);
-    decode_merge_kernel<bf16><<<dim3(a.Hq, a.B), 128, 0, s>>>(a);
     MARK(4);
   } else {
     e = set_max_smem(gemv_kernel<float>, smx, s);

@@ -129,9 +129,12 @@ struct DecodeArgs {
   float* qf;                     // [B, dq] float32 query
   float* part;                   // split-KV partials
   int nsplit;
+  unsigned* sync;                // 2 words in the decode state: grid-barrier count and generation
   int* status;
   cudaEvent_t* prof;             // 5 events around the 4 stages, or NULL
 };
+// bf16: one cooperative launch of decode_fused_kernel over all SMs (nsplit = (SMs - B) / (B * Hkv)
+// attention units); float32: GEMV, token update, split-KV attention and merge as four launches.
 cudaError_t decode_step(const DecodeArgs& a, cudaStream_t s);
 
 // Waits `limit_us` on an mbarrier nothing arrives at; *result = 1 if the wait (wrongly) completed.
