@@ -89,24 +89,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sQ = smem;                      // tile t at t * Q_BYTES
   uint8_t* sKV = smem + 2 * C::Q_BYTES;    // stage st: K at st*KV_BYTES, V at + K_BYTES
   uint64_t* bars = (uint64_t*)(smem + 2 * C::Q_BYTES + 2 * C::KV_BYTES);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;   // [2] stages
-  uint64_t* kv_empty = bars + 4;  // [2]
-  uint64_t* s_full = bars + 6;    // [2] query tiles
-  uint64_t* p_full = bars + 8;    // [2]
-  uint64_t* pv_done = bars + 10;  // [2]
-  uint64_t* o_full = bars + 12;   // [2]
-  uint64_t* o_empty = bars + 14;  // [2]
-  uint64_t* drain = bars + 16;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 17);
+  uint64_t* q_full = bars + 0;    // [2] query tiles
+  uint64_t* q_empty = bars + 2;   // [2]
+  uint64_t* kv_full = bars + 4;   // [2] stages
+  uint64_t* kv_empty = bars + 6;  // [2]
+  uint64_t* s_full = bars + 8;    // [2] query tiles
+  uint64_t* p_full = bars + 10;   // [2]
+  uint64_t* pv_done = bars + 12;  // [2]
+  uint64_t* o_full = bars + 14;   // [2]
+  uint64_t* o_empty = bars + 16;  // [2]
+  uint64_t* drain = bars + 18;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 19);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
@@ -145,13 +145,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int w = blockIdx.x; w < nwork; w += gridDim.x, ++wi) {
         const Work it = work_item(w, a.B, a.Hq, npairs);
         const int g = it.h / G;
-        if (!mbar_wait(q_empty, (wi & 1) ^ 1, abort, status)) break;
-        mbar_expect_tx(q_full, 2 * C::Q_BYTES);
-        for (int t = 0; t < 2; ++t) {
+        bool qok = true;
+        for (int t = 0; t < 2; ++t) {  // each tile as soon as the previous item's last S_t has read it
+          if (!mbar_wait(&q_empty[t], (wi & 1) ^ 1, abort, status)) {
+            qok = false;
+            break;
+          }
+          mbar_expect_tx(&q_full[t], C::Q_BYTES);
           const int qy = (int)(it.b * q_rows_per_b) + (2 * it.pair + t) * BQ;
           for (int hb = 0; hb < NH; ++hb)
-            tma_load_2d(sQ + t * C::Q_BYTES + hb * C::HALF, &tmQ, q_full, it.h * DH + hb * 64, qy);
+            tma_load_2d(sQ + t * C::Q_BYTES + hb * C::HALF, &tmQ, &q_full[t], it.h * DH + hb * 64, qy);
         }
+        if (!qok) break;
         const int nkv = 2 * it.pair + 2;
         bool ok = true;
         for (int j = 0; j < nkv; ++j, ++kvit) {
@@ -202,10 +207,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x, ++wi) {
         const Work it = work_item(w, a.B, a.Hq, npairs);
         const int n0 = 2 * it.pair + 1, n1 = 2 * it.pair + 2;
-        if (!mbar_wait(q_full, wi & 1, abort, status)) break;
+        if (!mbar_wait(&q_full[0], wi & 1, abort, status)) break;
         if (!mbar_wait(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
         tc_fence_after();
         issue_s(0, kvit & 1);
+        if (n0 == 1) umma_commit(&q_empty[0]);  // Q_0's last use
+        if (!mbar_wait(&q_full[1], wi & 1, abort, status)) break;
+        tc_fence_after();
         issue_s(1, kvit & 1);
         for (int j = 0; j < n1; ++j) {
           const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
@@ -222,6 +230,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               tc_fence_after();
               next_ready = true;
               issue_s(0, nst);
+              if (j + 2 == n0) umma_commit(&q_empty[0]);  // Q_0's last use
             }
           }
           if (!mbar_wait(&p_full[1], pc[1] & 1, abort, status)) { ok = false; break; }
@@ -236,12 +245,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               tc_fence_after();
             }
             issue_s(1, nst);
+            if (j + 2 == n1) umma_commit(&q_empty[1]);  // Q_1's last use
           } else {
             umma_commit(&o_full[1]);
           }
         }
         if (!ok) break;
-        umma_commit(q_empty);
         kvit += n1;
       }
       if (*abort) {
@@ -273,20 +282,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         const bool diag = (j == nkv - 1);
         const int lim = row - j * BKV;  // keys c > lim are in the future of this row
-        // pass 1: row maximum of the raw scores
+        // pass 1: row maximum of the raw scores (four TMEM loads behind one wait)
         float mx = -INFINITY;
+        {
+          uint32_t v[4][32];
 #pragma unroll
-        for (int c = 0; c < BKV; c += 64) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(s_tmem + c, v0);
-          tmem_ld32(s_tmem + c + 32, v1);
+          for (int c = 0; c < 4; ++c) tmem_ld32(s_tmem + c * 32, v[c]);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float f0 = (diag && c + e > lim) ? -INFINITY : __uint_as_float(v0[e]);
-            const float f1 = (diag && c + 32 + e > lim) ? -INFINITY : __uint_as_float(v1[e]);
-            mx = fmaxf(mx, fmaxf(f0, f1));
-          }
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float f = (diag && c * 32 + e > lim) ? -INFINITY : __uint_as_float(v[c][e]);
+              mx = fmaxf(mx, f);
+            }
         }
         mx *= sl2;
         // lazy rescale: move the reference maximum only when it is exceeded by more than 2^8
@@ -315,26 +324,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_st16(o_tmem + c + 16, hi);
           }
         }
-        // pass 2: P = 2^(s*sl2 - m_ref) as bf16 pairs over the first 64 columns of S
+        // pass 2: P = 2^(s*sl2 - m_ref) as bf16 pairs over the first 64 columns of S; the
+        // TMEM load of chunk c+1 is in flight while chunk c is exponentiated
         const float nm = -m_ref;
         float lsum = 0.f;
+        uint32_t vb[2][32];
+        tmem_ld32(s_tmem, vb[0]);
 #pragma unroll
-        for (int c = 0; c < BKV; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(s_tmem + c, v);
+        for (int c = 0; c < 4; ++c) {
           tmem_ld_wait();
+          if (c + 1 < 4) tmem_ld32(s_tmem + (c + 1) * 32, vb[(c + 1) & 1]);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sl2, nm));
-            float p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sl2, nm));
-            if (diag && c + 2 * e > lim) p0 = 0.f;
-            if (diag && c + 2 * e + 1 > lim) p1 = 0.f;
+            float p0 = ex2(fmaf(__uint_as_float(vb[c & 1][2 * e]), sl2, nm));
+            float p1 = ex2(fmaf(__uint_as_float(vb[c & 1][2 * e + 1]), sl2, nm));
+            if (diag && c * 32 + 2 * e > lim) p0 = 0.f;
+            if (diag && c * 32 + 2 * e + 1 > lim) p1 = 0.f;
             lsum += p0 + p1;
             __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
             pk[e] = *(uint32_t*)&hb;
           }
-          tmem_st16(s_tmem + c / 2, pk);
+          tmem_st16(s_tmem + c * 16, pk);
         }
         l += lsum;
         tmem_st_wait();
