@@ -3,7 +3,7 @@
 // exp(mu_old - mu_new) when the running maximum grows).
 //
 // Persistent CTAs walk work items (sequence b, query head h, pair p of 128-row
-// query tiles 2p and 2p+1) longest first.  Per item the CTA streams the 128-key
+// query tiles 2p and 2p+1) longest first, dealt to the CTAs in snake order.  Per item the CTA streams the 128-key
 // tiles j <= 2p+1 of KV group g(h) = h / (Hq / Hkv), shared by both query tiles:
 //   warp 0      TMA: both Q tiles once, then K_j and V_j into a 2-stage ring
 //   warp 1      MMA, ping-pong between the two query tiles t = 0, 1:
@@ -56,6 +56,14 @@ __device__ __forceinline__ Work work_item(int w, int B, int Hq, int npairs) {
   r.h = rem % Hq;
   r.b = rem / Hq;
   return r;
+}
+
+// Work item of round r for this CTA: items are sorted longest first and dealt in a
+// snake order (CTA order reversed every other round), which balances the causal
+// work across CTAs far better than plain round-robin.  -1 past the end.
+__device__ __forceinline__ int snake_item(int r, int grid, int cta, int nwork) {
+  const int w = r * grid + ((r & 1) ? grid - 1 - cta : cta);
+  return w < nwork ? w : -1;
 }
 
 // MN-major (V) descriptor: 8-key groups of 128-B rows 1024 B apart (stride byte
@@ -141,8 +149,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      int wi = 0, kvit = 0;
-      for (int w = blockIdx.x; w < nwork; w += gridDim.x, ++wi) {
+      int kvit = 0;
+      for (int rr = 0; rr * (int)gridDim.x < nwork; ++rr) {
+        const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
+        if (w < 0) break;
+        const int wi = rr;  // items this CTA has started before this one
         const Work it = work_item(w, a.B, a.Hq, npairs);
         const int g = it.h / G;
         bool qok = true;
@@ -184,7 +195,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int wi = 0, kvit = 0, pc[2] = {0, 0};
+      int kvit = 0, pc[2] = {0, 0};
       bool ok = true;
       const uint64_t qd0 = sdesc_kmajor_sw128(sQ), qd1 = sdesc_kmajor_sw128(sQ + C::Q_BYTES);
       auto issue_s = [&](int t, int st) {
@@ -204,7 +215,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                        (j | kk) != 0);
         umma_commit(&pv_done[t]);
       };
-      for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x, ++wi) {
+      for (int rr = 0; rr * (int)gridDim.x < nwork && ok; ++rr) {
+        const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
+        if (w < 0) break;
+        const int wi = rr;  // items this CTA has started before this one
         const Work it = work_item(w, a.B, a.Hq, npairs);
         const int n0 = 2 * it.pair + 1, n1 = 2 * it.pair + 2;
         if (!mbar_wait(&q_full[0], wi & 1, abort, status)) break;
@@ -269,8 +283,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t s_tmem = tbase + lane_off + S_COL(t);
     const uint32_t o_tmem = tbase + lane_off + O_COL(t);
     const float sl2 = a.scale * 1.4426950408889634f;
-    int wi = 0, sit = 0;
-    for (int w = blockIdx.x; w < nwork; w += gridDim.x, ++wi) {
+    int sit = 0;
+    for (int rr = 0; rr * (int)gridDim.x < nwork; ++rr) {
+      const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
+      if (w < 0) break;
+      const int wi = rr;
       const Work it = work_item(w, a.B, a.Hq, npairs);
       const int qt = 2 * it.pair + t;
       const int nkv = qt + 1;
