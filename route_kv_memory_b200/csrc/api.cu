@@ -109,6 +109,7 @@ int check_cfg(const mka_config* c, Dims* o) {
 // ---------------------------------------------------------------- packed weights
 struct PackLayout {
   int Ntot, Npad, seg_q, seg_k, seg_v, seg_r, seg_rlo, seg_p, rh_segs;
+  int router_fused;  // bf16 with 256-aligned router rows: hi/lo interleaved per 128 units, GELU.W_r2 in the GEMM epilogue
   size_t wcat, wr2, pT64, p64, wqr32, wr1T, total;
 };
 PackLayout pack_layout(const Dims& d) {
@@ -122,6 +123,7 @@ PackLayout pack_layout(const Dims& d) {
   p.seg_p = p.seg_r + p.rh_segs * d.rh;
   p.Ntot = p.seg_p + d.nb;
   p.Npad = (p.Ntot + 127) / 128 * 128;
+  p.router_fused = d.bf16 && (p.seg_r % 256 == 0) && (d.rh % 128 == 0);
   size_t o = 0;
   p.wcat = o; o += al((size_t)p.Npad * d.d * d.elem);
   p.wr2 = o; o += al((size_t)d.rh * 3 * 4);
@@ -358,7 +360,9 @@ int mka_pack_weights(const mka_config* cfg, const mka_weights* w, void* packed, 
   ep.nseg = 1;
   ep.seg[0] = OutSeg{0, d.d, P(packed, L.wqr32), d.d, 0};
   CUDA_TRY(gemm_tn_ffma(P(packed, L.wr1T), d.dq, d.bf16, w->w_q, d.dq, d.bf16, d.rh, d.d, d.dq, ep, s));
-  if (d.bf16) {
+  if (d.bf16 && L.router_fused) {
+    CUDA_TRY(split_hi_lo_interleaved((const float*)P(packed, L.wqr32), d.rh, d.d, wc + L.seg_r * row, s));
+  } else if (d.bf16) {
     CUDA_TRY(split_hi_lo((const float*)P(packed, L.wqr32), d.rh * d.d, wc + L.seg_r * row, wc + L.seg_rlo * row, s));
   } else {
     CUDA_TRY(cudaMemcpyAsync(wc + L.seg_r * row, P(packed, L.wqr32), (size_t)d.rh * d.d * 4, cudaMemcpyDeviceToDevice, s));
@@ -521,11 +525,18 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   if (d.bf16) ep.seg[ns++] = OutSeg{PL.seg_rlo, PL.seg_rlo + d.rh, h2, d.rh, 0};
   ep.seg[ns++] = OutSeg{PL.seg_p, PL.Ntot, proj, d.nb, 0};
   ep.nseg = ns;
+  if (PL.router_fused) {  // hidden layer reduced in the epilogue; h1 holds the partials
+    ep.r_begin = PL.seg_r;
+    ep.r_end = PL.seg_r + 2 * d.rh;
+    ep.w_r2 = (const float*)P((void*)packed, PL.wr2);
+    ep.zpart = h1;
+  }
   if (d.bf16) CUDA_TRY(gemm_tn_bf16_tc(x, d.d, wcat, d.d, d.T, PL.Ntot, d.d, ep, status_ptr(), s));
   else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, wcat, d.d, 0, d.T, PL.Ntot, d.d, ep, s));
   STAGE(s);
   // 2. router tail
-  CUDA_TRY(router_tail(h1, h2, d.rh, d.T, d.rh, (const float*)P((void*)packed, PL.wr2), lam, s));
+  if (PL.router_fused) CUDA_TRY(router_softmax(h1, d.rh / 128, d.T, lam, s));
+  else CUDA_TRY(router_tail(h1, h2, d.rh, d.T, d.rh, (const float*)P((void*)packed, PL.wr2), lam, s));
   STAGE(s);
   // 3. L3 codes, 4. block sums / EMA end states, carries, recall
   HashArgs ha{proj, d.nb, x, d.bf16, (const double*)P((void*)packed, PL.pT64), d.d, d.nb, d.d};
@@ -585,7 +596,7 @@ int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size
   DecodeArgs a{};
   a.wcatT = P((void*)packed, PL.wcat); a.Ntot = PL.Ntot; a.d = d.d; a.x_bf16 = d.bf16;
   a.w_r2 = (const float*)P((void*)packed, PL.wr2); a.pT64 = (const double*)P((void*)packed, PL.pT64);
-  a.dq = d.dq; a.dkv = d.dkv; a.rh = d.rh; a.nb = d.nb; a.rh_segs = PL.rh_segs;
+  a.dq = d.dq; a.dkv = d.dkv; a.rh = d.rh; a.nb = d.nb; a.rh_segs = PL.rh_segs; a.r_inter = PL.router_fused;
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.dh = d.dh; a.blk = d.blk; a.R = d.R; a.Lmax = max_positions;
   a.maxblk = SL.maxblk; a.alpha = d.alpha; a.scale = d.scale;
   a.x_new = x_new; a.out = out;

@@ -98,8 +98,9 @@ __device__ void token_update(const DecodeArgs& a, const int bi) {
   // router (notes §2): z = GELU(h) W_r2, lambda = softmax(z)
   float z0 = 0.f, z1 = 0.f, z2 = 0.f;
   for (int j = tid; j < a.rh; j += blockDim.x) {
-    float hv = h[j];
-    if (a.rh_segs == 2) hv += h[a.rh + j];
+    float hv;
+    if (a.r_inter) hv = h[(j >> 7) * 256 + (j & 127)] + h[(j >> 7) * 256 + 128 + (j & 127)];
+    else hv = a.rh_segs == 2 ? h[j] + h[a.rh + j] : h[j];
     float gv = gelu_erf(hv);
     z0 = fmaf(gv, a.w_r2[j * 3], z0);
     z1 = fmaf(gv, a.w_r2[j * 3 + 1], z1);
@@ -590,8 +591,9 @@ __device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, T
   const T* xn = (const T*)a.x_new + (size_t)bi * a.d;
   float z0 = 0.f, z1 = 0.f, z2 = 0.f;
   for (int j = tid; j < a.rh; j += blockDim.x) {
-    float hv = h[j];
-    if (a.rh_segs == 2) hv += h[a.rh + j];
+    float hv;
+    if (a.r_inter) hv = h[(j >> 7) * 256 + (j & 127)] + h[(j >> 7) * 256 + 128 + (j & 127)];
+    else hv = a.rh_segs == 2 ? h[j] + h[a.rh + j] : h[j];
     const float gv = gelu_erf(hv);
     z0 = fmaf(gv, a.w_r2[j * 3], z0);
     z1 = fmaf(gv, a.w_r2[j * 3 + 1], z1);

@@ -167,6 +167,23 @@ cudaError_t split_hi_lo(const float* w, int n, void* hi, void* lo, cudaStream_t 
   return cudaGetLastError();
 }
 
+__global__ void split_hi_lo_interleaved_kernel(const float* __restrict__ w, int rh, int d, bf16* __restrict__ dst) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (size_t)rh * d) return;
+  const int u = (int)(i / d), col = (int)(i % d);
+  const float v = w[i];
+  const bf16 h = __float2bfloat16_rn(v);
+  const size_t row_hi = (size_t)(u / 128) * 256 + (u % 128);
+  dst[row_hi * d + col] = h;
+  dst[(row_hi + 128) * d + col] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+cudaError_t split_hi_lo_interleaved(const float* w, int rh, int d, void* dst, cudaStream_t s) {
+  const size_t n = (size_t)rh * d;
+  if (n == 0) return cudaSuccess;
+  split_hi_lo_interleaved_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w, rh, d, (bf16*)dst);
+  return cudaGetLastError();
+}
+
 template <typename T>
 __global__ void widen_pad32_kernel(const T* __restrict__ in, int rows, int cols, double* __restrict__ out) {
   int i = blockIdx.x * blockDim.x + threadIdx.x;

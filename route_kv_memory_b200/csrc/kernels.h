@@ -21,6 +21,13 @@ constexpr int kMaxSegs = 6;
 struct Epilogue {
   int nseg;
   OutSeg seg[kMaxSegs];
+  // Router columns [r_begin, r_end) of the bf16 projection GEMM (0, 0: none): tiles of 256
+  // columns holding the hi then lo halves of 128 hidden units of X (W_q W_r1).  The
+  // epilogue writes zpart[(r * M + m) * 4 + k] = sum_u GELU(hi_u + lo_u) W_r2[u][k] for
+  // the r-th such tile, instead of storing the hidden layer.
+  int r_begin, r_end;
+  const float* w_r2;
+  float* zpart;
 };
 
 // C[M, N] = A[M, K] * B[N, K]^T (both operands K-major), float32 accumulation.
@@ -53,6 +60,11 @@ struct HashArgs {
 
 cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, float* lam,
                         cudaStream_t s);
+// lambda = softmax(sum_r zpart[r][t][0..2]) for the router partials of the fused GEMM epilogue.
+cudaError_t router_softmax(const float* zpart, int nparts, int T, float* lam, cudaStream_t s);
+// Writes the bf16 hi/lo split of w [rh, d] float32 into the rows of the packed matrix so that every
+// 256-row group holds the hi then the lo rows of 128 consecutive hidden units (rh % 128 == 0).
+cudaError_t split_hi_lo_interleaved(const float* w, int rh, int d, void* dst, cudaStream_t s);
 cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, cudaStream_t s);
 // Codes of the full blocks from exact float64 block sums of x in d_model space projected in float64.
 // P64: [d][32] float64 (P row-major, padded to 32 columns).  part: summary_codes_scratch() bytes.
@@ -117,6 +129,7 @@ struct DecodeArgs {
   const float* w_r2; const double* pT64;
   // layout of the fused projection row
   int dq, dkv, rh, nb, rh_segs;  // rh_segs: 2 for bf16 (hi+lo), 1 for f32
+  int r_inter;                   // hi/lo rows interleaved per 128 hidden units (else [hi | lo])
   int B, Hq, Hkv, dh, blk, R, Lmax, maxblk;
   float alpha, scale;
   const void* x_new;             // [B, d]

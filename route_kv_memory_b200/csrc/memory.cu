@@ -66,6 +66,30 @@ template <> struct Vec4<bf16> {
     return make_float4(fa.x, fa.y, fb.x, fb.y);
   }
 };
+__global__ void router_softmax_kernel(const float* __restrict__ zpart, int nparts, int T, float* __restrict__ lam) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  float z0 = 0.f, z1 = 0.f, z2 = 0.f;
+  for (int r = 0; r < nparts; ++r) {
+    const float4 v = *(const float4*)(zpart + ((size_t)r * T + t) * 4);
+    z0 += v.x;
+    z1 += v.y;
+    z2 += v.z;
+  }
+  const float m = fmaxf(z0, fmaxf(z1, z2));
+  const float e0 = expf(z0 - m), e1 = expf(z1 - m), e2 = expf(z2 - m);
+  const float inv = 1.f / (e0 + e1 + e2);
+  lam[(size_t)t * 3 + 0] = e0 * inv;
+  lam[(size_t)t * 3 + 1] = e1 * inv;
+  lam[(size_t)t * 3 + 2] = e2 * inv;
+}
+
+cudaError_t router_softmax(const float* zpart, int nparts, int T, float* lam, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  router_softmax_kernel<<<(T + 255) / 256, 256, 0, s>>>(zpart, nparts, T, lam);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- L3 sign codes
 // The float32 projection p = x . P_k (a tensor-core or FFMA dot product of
 // length K) carries a rounding error below about K/16 * 2^-23 * |partial sum|
@@ -292,28 +316,53 @@ cudaError_t block_reduce(const void* x, int x_bf16, int ld, int width, int B, in
   return cudaGetLastError();
 }
 
-// carry[b][0] = carry_in (or 0); carry[b][j+1] = a^b * carry[b][j] + bend[b][j].
-__global__ void ema_carry_kernel(const float* __restrict__ bend, int width, int B, int nblk, float apb,
-                                 const float* __restrict__ carry_in, float* __restrict__ carry) {
-  int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= B * width) return;
-  int bi = i / width, c = i % width;
-  float cur = carry_in ? carry_in[i] : 0.f;
-  float* out = carry + (size_t)bi * (nblk + 1) * width + c;
+// carry[b][0] = carry_in (or 0); carry[b][j+1] = A * carry[b][j] + bend[b][j], A = a^blk.
+// CTA = (32 columns, sequence b), 32 warps: warp w scans blocks [w*cpw, (w+1)*cpw) from a
+// zero carry (lanes = columns, coalesced), the 32 chunk end states are chained in order
+// (A^len * c + end), then every warp rescans its chunk from its true carry-in.
+__global__ void __launch_bounds__(1024) ema_carry_kernel(const float* __restrict__ bend, int width, int nblk,
+                                                          float apb, const float* __restrict__ carry_in,
+                                                          float* __restrict__ carry) {
+  __shared__ float sA[32][33], sL[32][33], sC[33][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int bi = blockIdx.y, c = blockIdx.x * 32 + lane;
+  const int cpw = (nblk + 31) / 32;
+  const int j0 = min(nblk, w * cpw), j1 = min(nblk, j0 + cpw);
+  const bool ok = c < width;
   const float* e = bend + (size_t)bi * nblk * width + c;
-  out[0] = cur;
-#pragma unroll 8
-  for (int j = 0; j < nblk; ++j) {
-    cur = fmaf(apb, cur, e[(size_t)j * width]);
-    out[(size_t)(j + 1) * width] = cur;
+  float L = 0.f, A = 1.f;
+  if (ok)
+    for (int j = j0; j < j1; ++j) {
+      L = fmaf(apb, L, e[(size_t)j * width]);
+      A *= apb;
+    }
+  sA[w][lane] = A;
+  sL[w][lane] = L;
+  __syncthreads();
+  if (w == 0) {
+    float cur = (ok && carry_in) ? carry_in[(size_t)bi * width + c] : 0.f;
+    for (int k = 0; k < 32; ++k) {
+      sC[k][lane] = cur;
+      cur = fmaf(sA[k][lane], cur, sL[k][lane]);
+    }
+    sC[32][lane] = cur;
   }
+  __syncthreads();
+  if (!ok) return;
+  float* out = carry + (size_t)bi * (nblk + 1) * width + c;
+  float cur = sC[w][lane];
+  for (int j = j0; j < j1; ++j) {
+    out[(size_t)j * width] = cur;
+    cur = fmaf(apb, cur, e[(size_t)j * width]);
+  }
+  if (w == 31) out[(size_t)nblk * width] = sC[32][lane];
 }
 
 cudaError_t ema_carry(const float* bend, int width, int B, int nblk, float alpha_pow_b, const float* carry_in,
                       float* carry, cudaStream_t s) {
-  int n = B * width;
-  if (n <= 0) return cudaSuccess;
-  ema_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(bend, width, B, nblk, alpha_pow_b, carry_in, carry);
+  if (B <= 0 || width <= 0) return cudaSuccess;
+  dim3 grid((width + 31) / 32, B);
+  ema_carry_kernel<<<grid, 1024, 0, s>>>(bend, width, nblk, alpha_pow_b, carry_in, carry);
   return cudaGetLastError();
 }
 

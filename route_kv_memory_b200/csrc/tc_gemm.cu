@@ -205,12 +205,36 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
       const int m = m0 + q * 32 + lane;
-      for (int c = 0; c < BN; c += 32) {
-        if (n0 + c >= N) break;
-        uint32_t r[32];
-        tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + acc * BN + c, r);
-        tmem_ld_wait();
-        if (m < M) store_chunk(ep, m, n0 + c, r, N);
+      const uint32_t trow = tbase + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if (n0 >= ep.r_begin && n0 < ep.r_end) {
+        // router tile: hidden units u0 .. u0+127, hi in columns [0,128), lo in [128,256)
+        const int rt = (n0 - ep.r_begin) / BN;
+        const int u0 = rt * 128;
+        float z0 = 0.f, z1 = 0.f, z2 = 0.f;
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t hi[32], lo[32];
+          tmem_ld32(trow + c, hi);
+          tmem_ld32(trow + 128 + c, lo);
+          tmem_ld_wait();
+#pragma unroll 8
+          for (int i = 0; i < 32; ++i) {
+            const float h = __uint_as_float(hi[i]) + __uint_as_float(lo[i]);
+            const float g = gelu_erf(h);
+            const float* w = ep.w_r2 + (size_t)(u0 + c + i) * 3;
+            z0 = fmaf(g, w[0], z0);
+            z1 = fmaf(g, w[1], z1);
+            z2 = fmaf(g, w[2], z2);
+          }
+        }
+        if (m < M) *(float4*)(ep.zpart + ((size_t)rt * M + m) * 4) = make_float4(z0, z1, z2, 0.f);
+      } else {
+        for (int c = 0; c < BN; c += 32) {
+          if (n0 + c >= N) break;
+          uint32_t r[32];
+          tmem_ld32(trow + c, r);
+          tmem_ld_wait();
+          if (m < M) store_chunk(ep, m, n0 + c, r, N);
+        }
       }
       tc_fence_before();
       __syncwarp();
