@@ -385,6 +385,7 @@ def main():
     ap.add_argument("--workload", default="qwen7b_4k")
     ap.add_argument("--decode-ctx", type=int, nargs="*", default=[131072])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true", help="run only the decode measurement (no prefill line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=48)
     args = ap.parse_args()
@@ -402,6 +403,13 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
+        if args.decode_only:
+            torch.cuda.set_device(local_rank)
+            dev = torch.device("cuda", local_rank)
+            res = {"decode": run_decode(args, None, None, None, dev)}
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         res = run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(res), flush=True)

@@ -299,20 +299,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         const bool diag = (j == nkv - 1);
         const int lim = row - j * BKV;  // keys c > lim are in the future of this row
-        // pass 1: row maximum of the raw scores (four TMEM loads behind one wait)
+        // pass 1: row maximum of the raw scores (four TMEM loads behind one wait); only the
+        // diagonal tile needs the causal mask (a warp-uniform branch)
         float mx = -INFINITY;
         {
           uint32_t v[4][32];
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld32(s_tmem + c * 32, v[c]);
           tmem_ld_wait();
+          if (diag) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float f = (diag && c * 32 + e > lim) ? -INFINITY : __uint_as_float(v[c][e]);
-              mx = fmaxf(mx, f);
-            }
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(v[c][e]));
+          } else {
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(v[c][e]));
+            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          }
         }
         mx *= sl2;
         // lazy rescale: move the reference maximum only when it is exceeded by more than 2^8
@@ -333,9 +341,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_ld_wait();
             uint32_t lo[16], hi[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              lo[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-              hi[e] = __float_as_uint(__uint_as_float(ov[16 + e]) * corr);
+            for (int e = 0; e < 16; e += 2) {
+              const float2 c2 = make_float2(corr, corr);
+              const float2 a2 = __fmul2_rn(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), c2);
+              const float2 b2 = __fmul2_rn(make_float2(__uint_as_float(ov[16 + e]), __uint_as_float(ov[17 + e])), c2);
+              lo[e] = __float_as_uint(a2.x);
+              lo[e + 1] = __float_as_uint(a2.y);
+              hi[e] = __float_as_uint(b2.x);
+              hi[e + 1] = __float_as_uint(b2.y);
             }
             tmem_st16(o_tmem + c, lo);
             tmem_st16(o_tmem + c + 16, hi);
@@ -344,7 +357,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // pass 2: P = 2^(s*sl2 - m_ref) as bf16 pairs over the first 64 columns of S; the
         // TMEM load of chunk c+1 is in flight while chunk c is exponentiated
         const float nm = -m_ref;
-        float lsum = 0.f;
+        const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(nm, nm);
+        float2 lsum2 = make_float2(0.f, 0.f);
         uint32_t vb[2][32];
         tmem_ld32(s_tmem, vb[0]);
 #pragma unroll
@@ -354,16 +368,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float p0 = ex2(fmaf(__uint_as_float(vb[c & 1][2 * e]), sl2, nm));
-            float p1 = ex2(fmaf(__uint_as_float(vb[c & 1][2 * e + 1]), sl2, nm));
-            if (diag && c * 32 + 2 * e > lim) p0 = 0.f;
-            if (diag && c * 32 + 2 * e + 1 > lim) p1 = 0.f;
-            lsum += p0 + p1;
+            // packed FP32x2: one FFMA2 scales and shifts both scores, one FADD2 accumulates
+            const float2 x2 = __ffma2_rn(make_float2(__uint_as_float(vb[c & 1][2 * e]), __uint_as_float(vb[c & 1][2 * e + 1])),
+                                         sl2v, nmv);
+            float p0 = ex2(x2.x), p1 = ex2(x2.y);
+            if (diag) {
+              if (c * 32 + 2 * e > lim) p0 = 0.f;
+              if (c * 32 + 2 * e + 1 > lim) p1 = 0.f;
+            }
+            lsum2 = __fadd2_rn(lsum2, make_float2(p0, p1));
             __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
             pk[e] = *(uint32_t*)&hb;
           }
           tmem_st16(s_tmem + c * 16, pk);
         }
+        const float lsum = lsum2.x + lsum2.y;
         l += lsum;
         tmem_st_wait();
         tc_fence_before();
