@@ -78,6 +78,12 @@ __device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(const void* tile) {
   return d;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -299,8 +305,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         const bool diag = (j == nkv - 1);
         const int lim = row - j * BKV;  // keys c > lim are in the future of this row
-        // pass 1: row maximum of the raw scores (four TMEM loads behind one wait); only the
-        // diagonal tile needs the causal mask (a warp-uniform branch)
+        // pass 1: row maximum of the raw scores (four TMEM loads behind one wait; 3-input
+        // max); only the diagonal tile needs the causal mask (a warp-uniform branch)
         float mx = -INFINITY;
         {
           uint32_t v[4][32];
@@ -318,8 +324,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
-              for (int e = 0; e < 32; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(v[c][e]));
-            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+              for (int e = 0; e < 32; e += 8) {
+                m4[0] = max3(m4[0], __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]));
+                m4[1] = max3(m4[1], __uint_as_float(v[c][e + 2]), __uint_as_float(v[c][e + 3]));
+                m4[2] = max3(m4[2], __uint_as_float(v[c][e + 4]), __uint_as_float(v[c][e + 5]));
+                m4[3] = max3(m4[3], __uint_as_float(v[c][e + 6]), __uint_as_float(v[c][e + 7]));
+              }
+            mx = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
           }
         }
         mx *= sl2;
@@ -330,29 +341,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           corr = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
           m_ref = mx;
           l *= corr;
-        }
-        if (__ballot_sync(0xffffffffu, need && j > 0)) {  // rescale O rows once PV_{j-1} has landed
-          if (!mbar_wait(&pv_done[t], (sit - 1) & 1, abort, status)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < DH; c += 32) {
-            uint32_t ov[32];
-            tmem_ld32(o_tmem + c, ov);
-            tmem_ld_wait();
-            uint32_t lo[16], hi[16];
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const float2 c2 = make_float2(corr, corr);
-              const float2 a2 = __fmul2_rn(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), c2);
-              const float2 b2 = __fmul2_rn(make_float2(__uint_as_float(ov[16 + e]), __uint_as_float(ov[17 + e])), c2);
-              lo[e] = __float_as_uint(a2.x);
-              lo[e + 1] = __float_as_uint(a2.y);
-              hi[e] = __float_as_uint(b2.x);
-              hi[e + 1] = __float_as_uint(b2.y);
-            }
-            tmem_st16(o_tmem + c, lo);
-            tmem_st16(o_tmem + c + 16, hi);
-          }
         }
         // pass 2: P = 2^(s*sl2 - m_ref) as bf16 pairs over the first 64 columns of S; the
         // TMEM load of chunk c+1 is in flight while chunk c is exponentiated
@@ -384,6 +372,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         const float lsum = lsum2.x + lsum2.y;
         l += lsum;
+        // rescale the O rows (rare with the lazy threshold).  S_j landing means PV_{j-1},
+        // issued before QK_j, has completed, so the wait below returns at once.  PV_j is
+        // issued only after p_full, so it accumulates onto the rescaled rows.
+        if (__ballot_sync(0xffffffffu, need && j > 0)) {
+          if (!mbar_wait(&pv_done[t], (sit - 1) & 1, abort, status)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < DH; c += 32) {
+            uint32_t ov[32];
+            tmem_ld32(o_tmem + c, ov);
+            tmem_ld_wait();
+            const float2 c2 = make_float2(corr, corr);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), c2);
+              ov[e] = __float_as_uint(o2.x);
+              ov[e + 1] = __float_as_uint(o2.y);
+            }
+            tmem_st16(o_tmem + c, *reinterpret_cast<const uint32_t(*)[16]>(&ov[0]));
+            tmem_st16(o_tmem + c + 16, *reinterpret_cast<const uint32_t(*)[16]>(&ov[16]));
+          }
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
