@@ -234,6 +234,39 @@ Profiler g_prof;
 inline void prof_begin() { g_prof.n = 0; }
 #define STAGE(s) CUDA_TRY(g_prof.mark(s))
 
+// ---------------------------------------------------------------- concurrent branches
+// Library-owned streams of the current device for the independent memory kernels of a
+// prefill (they are small enough at a few thousand tokens that running them one after
+// another costs mostly launch and ramp time).  Work is forked from the caller's stream
+// with an event and joined back with events before the call's later kernels, so the
+// caller's stream orders everything and stream capture sees one fork/join graph.  The
+// events are shared, so the enqueue sequence holds aux_mutex().
+struct AuxStreams {
+  cudaStream_t st[2];
+  cudaEvent_t fork, join[3];
+};
+std::mutex& aux_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+// Called with aux_mutex() held.  nullptr when the streams cannot be made.
+AuxStreams* aux_streams() {
+  static AuxStreams per_dev[64];
+  static bool made[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  AuxStreams& a = per_dev[dev];
+  if (!made[dev]) {
+    for (int i = 0; i < 2; ++i)
+      if (cudaStreamCreateWithFlags(&a.st[i], cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    for (int i = 0; i < 3; ++i)
+      if (cudaEventCreateWithFlags(&a.join[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    made[dev] = true;
+  }
+  return &a;
+}
+
 }  // namespace
 
 int mka::set_last_error(int code, const char* msg) {
@@ -534,20 +567,61 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   if (d.bf16) CUDA_TRY(gemm_tn_bf16_tc(x, d.d, wcat, d.d, d.T, PL.Ntot, d.d, ep, status_ptr(), s));
   else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, wcat, d.d, 0, d.T, PL.Ntot, d.d, ep, s));
   STAGE(s);
-  // 2. router tail
-  if (PL.router_fused) CUDA_TRY(router_softmax(h1, d.rh / 128, d.T, lam, s));
-  else CUDA_TRY(router_tail(h1, h2, d.rh, d.T, d.rh, (const float*)P((void*)packed, PL.wr2), lam, s));
-  STAGE(s);
-  // 3. L3 codes, 4. block sums / EMA end states, carries, recall
+  // 2-4: router tail, L3 codes, block sums / EMA end states, carries.  With stage timing on
+  // they run one after another on the caller's stream (so each stage has its own time);
+  // otherwise as three concurrent branches joined before the recall.
   HashArgs ha{proj, d.nb, x, d.bf16, (const double*)P((void*)packed, PL.pT64), d.d, d.nb, d.d};
-  CUDA_TRY(token_codes(ha, d.T, tcode, s));
-  STAGE(s);
-  CUDA_TRY(block_reduce(xkv, 0, d.width, d.width, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, bsum_bstride, bend, gend, s));
-  STAGE(s);
-  CUDA_TRY(summary_codes(x, d.bf16, d.d, d.B, d.S, d.nblk, d.blk, (const double*)P((void*)packed, PL.p64), d.nb, xsum,
-                         scode, code_bstride, s));
-  STAGE(s);
-  CUDA_TRY(ema_carry(bend, d.width, d.B, d.nblk, (float)pow((double)d.alpha, (double)d.blk), nullptr, carry, s));
+  const double* p64 = (const double*)P((void*)packed, PL.p64);
+  auto k_router = [&](cudaStream_t st) {
+    return PL.router_fused ? router_softmax(h1, d.rh / 128, d.T, lam, st)
+                           : router_tail(h1, h2, d.rh, d.T, d.rh, (const float*)P((void*)packed, PL.wr2), lam, st);
+  };
+  auto k_tcode = [&](cudaStream_t st) { return token_codes(ha, d.T, tcode, st); };
+  auto k_bsum = [&](cudaStream_t st) {
+    return block_reduce(xkv, 0, d.width, d.width, d.B, d.S, d.nblk, d.blk, d.alpha, bsum, bsum_bstride, bend, gend, st);
+  };
+  auto k_scode = [&](cudaStream_t st) {
+    return summary_codes(x, d.bf16, d.d, d.B, d.S, d.nblk, d.blk, p64, d.nb, xsum, scode, code_bstride, st);
+  };
+  auto k_carry = [&](cudaStream_t st) {
+    return ema_carry(bend, d.width, d.B, d.nblk, (float)pow((double)d.alpha, (double)d.blk), nullptr, carry, st);
+  };
+  auto k_tail = [&](cudaStream_t st) {
+    return prefill_tail_state(xkv, d.width, d.width, x, d.bf16, d.d, d.B, d.S, d.blk, (float*)P(state, SL.blk_sum),
+                              (double*)P(state, SL.blk_x), (int*)P(state, SL.pos), st);
+  };
+  std::unique_lock<std::mutex> aux_lock(aux_mutex(), std::defer_lock);
+  AuxStreams* ax = nullptr;
+  if (!g_prof.on) {
+    aux_lock.lock();
+    ax = aux_streams();
+  }
+  if (ax) {
+    CUDA_TRY(cudaEventRecord(ax->fork, s));
+    CUDA_TRY(cudaStreamWaitEvent(ax->st[0], ax->fork, 0));
+    CUDA_TRY(cudaStreamWaitEvent(ax->st[1], ax->fork, 0));
+    CUDA_TRY(k_scode(ax->st[0]));
+    CUDA_TRY(cudaEventRecord(ax->join[0], ax->st[0]));
+    if (state) CUDA_TRY(k_tail(ax->st[0]));  // reads x and xkv only; joined at the end
+    CUDA_TRY(cudaEventRecord(ax->join[2], ax->st[0]));
+    CUDA_TRY(k_router(ax->st[1]));
+    CUDA_TRY(k_tcode(ax->st[1]));
+    CUDA_TRY(cudaEventRecord(ax->join[1], ax->st[1]));
+    CUDA_TRY(k_bsum(s));
+    CUDA_TRY(k_carry(s));
+    CUDA_TRY(cudaStreamWaitEvent(s, ax->join[0], 0));
+    CUDA_TRY(cudaStreamWaitEvent(s, ax->join[1], 0));
+  } else {
+    CUDA_TRY(k_router(s));
+    STAGE(s);
+    CUDA_TRY(k_tcode(s));
+    STAGE(s);
+    CUDA_TRY(k_bsum(s));
+    STAGE(s);
+    CUDA_TRY(k_scode(s));
+    STAGE(s);
+    CUDA_TRY(k_carry(s));
+  }
   STAGE(s);
   CUDA_TRY(recall_select(tcode, scode, code_bstride, d.B, d.S, d.nblk, d.blk, d.R, idx, cnt, s));
   STAGE(s);
@@ -569,9 +643,10 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   if (d.bf16) CUDA_TRY(attention_prefill_tc(aa, status_ptr(), s));
   else CUDA_TRY(attention_prefill(aa, 0, s));
   STAGE(s);
-  if (state) {
-    CUDA_TRY(prefill_tail_state(xkv, d.width, d.width, x, d.bf16, d.d, d.B, d.S, d.blk, (float*)P(state, SL.blk_sum),
-                                (double*)P(state, SL.blk_x), (int*)P(state, SL.pos), s));
+  if (ax) {
+    CUDA_TRY(cudaStreamWaitEvent(s, ax->join[2], 0));
+  } else if (state) {
+    CUDA_TRY(k_tail(s));
     STAGE(s);
   }
   return MKA_OK;

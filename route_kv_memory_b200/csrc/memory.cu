@@ -152,6 +152,10 @@ cudaError_t token_codes(const HashArgs& a, int T, uint32_t* codes, cudaStream_t 
 // then 32 x 8 threads form the 64-long partial dot products with P's chunk.
 // Pass 2: per block and bit, the partials are summed over the chunks in order.
 constexpr int kXChunk = 64;
+#ifndef MKA_BP_UNROLL
+#define MKA_BP_UNROLL 4
+#endif
+constexpr int kBpUnroll = MKA_BP_UNROLL;
 
 template <typename T>
 __global__ void __launch_bounds__(256) block_proj_partial_kernel(const T* __restrict__ x, int d, int S, int blk,
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(256) block_proj_partial_kernel(const T* __rest
     double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
     if (col < d) {
       const T* p = x + ((size_t)bi * S + (size_t)j * blk) * d + col;
-#pragma unroll 4
+#pragma unroll kBpUnroll
       for (int r = ra; r < rb; ++r) {
         float4 v = Vec4<T>::load(p + (size_t)r * d);
         a0 += v.x;
@@ -228,8 +232,11 @@ cudaError_t summary_codes(const void* x, int x_bf16, int d, int B, int S, int nb
                           int nb, double* part, uint32_t* codes, int code_bstride, cudaStream_t s) {
   if (B <= 0 || nblk <= 0) return cudaSuccess;
   const int nchunk = (d + kXChunk - 1) / kXChunk;
-  // enough CTAs to stream X at full bandwidth: about 4 waves over the SMs
-  int groups = (4 * 148 + nchunk * B - 1) / (nchunk * B);
+  // enough CTAs to stream X at full bandwidth: about MKA_BP_WAVES waves over the SMs
+#ifndef MKA_BP_WAVES
+#define MKA_BP_WAVES 16
+#endif
+  int groups = (MKA_BP_WAVES * 148 + nchunk * B - 1) / (nchunk * B);
   groups = groups < 1 ? 1 : (groups > nblk ? nblk : groups);
   const int bpg = (nblk + groups - 1) / groups;
   groups = (nblk + bpg - 1) / bpg;

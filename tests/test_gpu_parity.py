@@ -88,6 +88,23 @@ def test_deterministic(mka):
     assert torch.equal(a, b) and torch.equal(la, lb) and torch.equal(ia, ib)
 
 
+def test_concurrent_branches_match_sequential(mka):
+    """With stage timing off the prefill runs its independent memory kernels as concurrent
+    branches; with it on, one after another.  Both orders give identical bytes, state included."""
+    cfg = CONFIGS["qwen7b_4k"].replace(seq=1000)
+    inp = make_inputs(cfg)
+    runs = []
+    for prof in (False, True):
+        mka.mka_profile_enable(prof)
+        try:
+            out, lam, idx, _, state = gpu_prefill(cfg, inp, with_state=cfg.seq + 24)
+        finally:
+            mka.mka_profile_enable(False)
+        runs.append((out, lam, idx, state))
+    for u, v in zip(*runs):
+        assert torch.equal(u, v)
+
+
 # ------------------------------------------------------------------ entry points one by one
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_router_entry(mka, dtype):
