@@ -120,6 +120,10 @@ def decode_bytes_per_token(cfg, ctx: int, ntot: int) -> float:
     return float(w + cache + state)
 
 
+def model_name(cfg) -> str:
+    return "Llama-3.1-8B" if cfg.name.startswith("llama") else "Qwen2.5-7B"
+
+
 def prefill_kernels(cfg) -> int:
     """Kernel launches of one prefill call: projection GEMM, router softmax, token codes, block
     sums, block sums of X and block codes (two), EMA carries, recall, fuse, attention."""
@@ -189,36 +193,62 @@ def run_ours(args, rank, world, local_rank):
                 "flops_per_launch": fl["attention"]}
     layer_tflops = (fl["projections"] + fl["attention"]) / (ms / 1e3) / 1e12
 
-    # ---- end to end through host buffers (pinned): H2D of X, the layer, D2H of O, every step
+    # ---- end to end through host buffers (pinned): every step copies its X in (H2D), runs the
+    # layer and copies its O out (D2H), all inside the timed region.  Steps are pipelined the way
+    # a serving loop streams batches: three streams and double-buffered device X / O, so the
+    # copy-in of step i+1 and the copy-out of step i-1 (separate copy engines, full-duplex PCIe)
+    # overlap the layer of step i.  L2 is flushed before every layer call, as in the timed loop.
+    n_e2e = max(4, args.steps // 4)
     x_host = inp.x[:, :cfg.seq].contiguous().pin_memory()
-    o_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(max(3, args.steps // 4))]
-    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(len(e0))]
-    for i in range(2):
-        x.copy_(x_host, non_blocking=True)
-        layer.prefill(x, out)
-        o_host.copy_(out, non_blocking=True)
-    torch.cuda.synchronize()
-    for i in range(len(e0)):
-        flush.zero_()
-        e0[i].record(stream)
-        x.copy_(x_host, non_blocking=True)
-        layer.prefill(x, out)
-        o_host.copy_(out, non_blocking=True)
-        e1[i].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(e0, e1)), world)
+    o_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    xb, ob = [x, torch.empty_like(x)], [out, torch.empty_like(out)]
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def e2e_run(n, timed):
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_cmp = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record(s_in)
+        for i in range(n):
+            k = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[i - 2])   # layer i-2 has read xb[k]
+                xb[k].copy_(x_host, non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[i])
+                if i >= 2:
+                    s_cmp.wait_event(ev_out[i - 2])  # ob[k] copied out
+                flush.zero_()
+                layer.prefill(xb[k], ob[k], stream=s_cmp)
+                ev_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                o_host[k].copy_(ob[k], non_blocking=True)
+                ev_out[i].record(s_out)
+        t1.record(s_out)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n
+
+    e2e_run(3, False)
+    e2e_ms = max_over_ranks(e2e_run(n_e2e, True), world)
     e2e = {"value": world * cfg.tokens / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-           "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "ms_per_step": round(e2e_ms, 4)}
-    del x_host, o_host
+           "d2h_bytes_per_step": o_host[0].numel() * o_host[0].element_size(), "ms_per_step": round(e2e_ms, 4),
+           "steps": n_e2e,
+           "how": "pinned host X -> device, layer, device O -> pinned host, every step; steps pipelined over "
+                  "copy-in / compute / copy-out streams with double-buffered device X and O"}
+    del x_host, o_host, xb, ob
 
     result = {
         "metric": "FastMKA layer prefill tokens/s (decode us/token and roofline fraction alongside)",
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) inputs, N(0,1/d_in) weights)",
-        "config": {"workload": f"{cfg.name}: Qwen2.5-7B-shaped FastMKA layer prefill, batch {cfg.batch} x seq "
+        "config": {"workload": f"{cfg.name}: {model_name(cfg)}-shaped FastMKA layer prefill, batch {cfg.batch} x seq "
                                f"{cfg.seq}, d_model {cfg.d_model}, {cfg.n_q_heads}/{cfg.n_kv_heads} heads, d_h "
                                f"{cfg.d_head}, router {cfg.dq}->{cfg.router_hidden}->3, alpha {cfg.alpha}, L3 block "
                                f"{cfg.block}, R {cfg.recall_r}, nbits {cfg.hash_bits}, seed {cfg.seed}",
@@ -260,7 +290,10 @@ def run_decode(args, cfg_prefill, inp_unused, weights_unused, dev, layer_pack=No
         snapshot = state.clone()
         xs = [x[:, t].contiguous() for t in range(ctx, ctx + n_new)]
         outs = [torch.empty(1, dcfg.dq, dtype=x.dtype, device=dev) for _ in range(n_new)]
-        # per-stage times of one eager step (profiling off in the graph)
+        # per-stage times of one eager step (profiling off in the graph), after one warm-up step
+        # (the first decode call of a process pays one-time launch set-up)
+        layer.decode(state, lmax, xs[0], outs[0])
+        state.copy_(snapshot)
         mka.mka_profile_enable(True)
         layer.decode(state, lmax, xs[0], outs[0])
         stages = mka.mka_profile_read()
