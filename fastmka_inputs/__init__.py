@@ -49,6 +49,8 @@ class FastMKAConfig:
     seed: int
     attn_scale: Optional[float] = None  # None -> 1/sqrt(d_head)
     decode_new: int = 0  # tokens decoded one at a time after a prefix of `seq`
+    route_mode: str = "soft"  # routing gate variant: "soft", "fixed", "top1", "top2"
+    tiers: int = 7  # active memory tiers: bit 0 L1, bit 1 L2, bit 2 L3
 
     @property
     def dq(self) -> int:

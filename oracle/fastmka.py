@@ -60,15 +60,73 @@ def softmax_rows(z: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=-1, keepdims=True)
 
 
-def router(q: np.ndarray, w_r1: np.ndarray, w_r2: np.ndarray) -> np.ndarray:
+def router_logits(q: np.ndarray, w_r1: np.ndarray, w_r2: np.ndarray) -> np.ndarray:
+    """Router logits z = MLP(q) = GELU(q W_r1) W_r2 (notes §2).  q: [..., dq] -> z: [..., 3]."""
+    h = q @ w_r1
+    return gelu_erf(h) @ w_r2
+
+
+ROUTE_MODES = ("soft", "fixed", "top1", "top2")
+
+
+def route_gate(z: np.ndarray, mode: str = "soft", tiers: int = 7) -> np.ndarray:
+    """Routing weights over the three memory sources from the logits z.
+
+    notes §2: the published gate is lambda = softmax(z).  The abstract page's
+    ablations (Table 9: L1+L2 only, L1+L3 only, L1 only; Table 10: fixed 1/3,
+    hard top-2, hard top-1 routing) are read with the same logits: a removed
+    tier is left out of the gate and gets 0; "fixed" puts equal weight on the
+    active tiers; "top1" puts all weight on the largest active logit; "top2"
+    takes the softmax over the two largest active logits and 0 elsewhere.  Ties
+    go to the lower tier index.  tiers: bit 0 L1, bit 1 L2, bit 2 L3.
+    z: [..., 3] -> lambda: [..., 3].
+    """
+    z = np.asarray(z, np.float64)
+    act = np.array([(tiers >> i) & 1 for i in range(3)], bool)
+    if not act.any() or mode not in ROUTE_MODES:
+        raise ValueError("need at least one tier and a known mode")
+    lam = np.zeros(z.shape)
+    zz = np.where(act, z, -np.inf)
+    if mode == "soft":
+        e = np.where(act, np.exp(zz - zz.max(axis=-1, keepdims=True)), 0.0)
+        return e / e.sum(axis=-1, keepdims=True)
+    if mode == "fixed":
+        lam[..., act] = 1.0 / act.sum()
+        return lam
+    order = np.argsort(-zz, axis=-1, kind="stable")  # largest first, lower index first on ties
+    i1 = order[..., :1]
+    if mode == "top1" or act.sum() == 1:
+        np.put_along_axis(lam, i1, 1.0, axis=-1)
+        return lam
+    i2 = order[..., 1:2]
+    z1, z2 = np.take_along_axis(z, i1, axis=-1), np.take_along_axis(z, i2, axis=-1)
+    e = np.exp(z2 - z1)
+    np.put_along_axis(lam, i1, 1.0 / (1.0 + e), axis=-1)
+    np.put_along_axis(lam, i2, e / (1.0 + e), axis=-1)
+    return lam
+
+
+def route_margin(z: np.ndarray, mode: str = "soft", tiers: int = 7) -> np.ndarray:
+    """The logit gap a hard gate decides on: largest minus second largest active
+    logit for "top1", second minus third for "top2" (inf where nothing is
+    decided, and for the soft and fixed gates).  z: [..., 3] -> [...]."""
+    z = np.asarray(z, np.float64)
+    act = np.array([(tiers >> i) & 1 for i in range(3)], bool)
+    k = {"top1": 1, "top2": 2}.get(mode)
+    if k is None or act.sum() <= k:
+        return np.full(z.shape[:-1], np.inf)
+    zs = -np.sort(-np.where(act, z, -np.inf), axis=-1)
+    return zs[..., k - 1] - zs[..., k]
+
+
+def router(q: np.ndarray, w_r1: np.ndarray, w_r2: np.ndarray, mode: str = "soft", tiers: int = 7) -> np.ndarray:
     """Routing gate lambda = softmax(MLP(q)) over the three memory sources.
 
     notes §2: one weight per token and source, shared by all heads.  MLP(q) =
-    GELU(q W_r1) W_r2.  q: [..., dq] -> lambda: [..., 3].
+    GELU(q W_r1) W_r2.  q: [..., dq] -> lambda: [..., 3].  mode / tiers select
+    the ablation gates of route_gate (the defaults give the published gate).
     """
-    h = q @ w_r1
-    z = gelu_erf(h) @ w_r2
-    return softmax_rows(z)
+    return route_gate(router_logits(q, w_r1, w_r2), mode, tiers)
 
 
 # ----------------------------------------------------------------------------- L2
@@ -258,6 +316,7 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
         "q": np.zeros((B, len(rows), Hq, dh)),
         "O": np.zeros((B, len(rows), Hq * dh)),
         "m2_next": np.zeros((B, d)),
+        "route_margin": np.zeros((B, S)),
     }
     if keep_d_space:
         for k in ("M2", "M3", "X_fused"):
@@ -275,8 +334,11 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
             r1 = min(S, r0 + row_chunk)
             xc = np.asarray(X[bi:bi + 1, r0:r1], np.float64)          # [1, n, d]
             qc = xc[0] @ w.w_q                                          # q = X W_q
-            lam = router(qc, w.w_r1, w.w_r2) if lam_override is None else np.broadcast_to(
+            mode, tiers = getattr(cfg, "route_mode", "soft"), getattr(cfg, "tiers", 7)
+            z = router_logits(qc, w.w_r1, w.w_r2)
+            lam = route_gate(z, mode, tiers) if lam_override is None else np.broadcast_to(
                 np.asarray(lam_override, np.float64), (r1 - r0, 3))
+            out["route_margin"][bi, r0:r1] = route_margin(z, mode, tiers)
             M2, m2 = session_ema(xc, cfg.alpha, m2)
             pos = np.arange(r0, r1)
             idx, cnt, M3, exc, xcodes, xproj = longterm_recall(xc[0], pos, summ, w.P, b, R, s_proj)
@@ -320,7 +382,7 @@ def fastmka_decode(X: np.ndarray, w: Weights64, cfg) -> np.ndarray:
         for t in range(S):
             x = np.asarray(X[bi, t], np.float64)
             q = x @ w.w_q
-            lam = router(q[None], w.w_r1, w.w_r2)[0]
+            lam = router(q[None], w.w_r1, w.w_r2, getattr(cfg, "route_mode", "soft"), getattr(cfg, "tiers", 7))[0]
             code_t, _ = hash_codes(x[None], w.P)
             s_arr = np.array(summaries).reshape(-1, d)
             sel = recall_select(int(code_t[0]), np.array(codes, np.uint32), len(summaries), R)

@@ -8,6 +8,7 @@ import math
 
 import numpy as np
 import pytest
+import scipy.special
 import scipy.stats
 import torch
 
@@ -408,6 +409,117 @@ def test_planted_mistakes_are_caught(monkeypatch):
             check_attention_brute(_mut_attention_factory(kind))
     # The unplanted copy of the attention mutant passes, so the failures above are the mistakes'.
     check_attention_brute(_mut_attention_factory("none"))
+
+
+# ============================================================================ routing and tier variants
+# abstract page, Tables 9 (tiers) and 10 (routing); gates read as in oracle.route_gate.
+_ZL = np.log(np.array([[1.0, 2.0, 4.0]]))  # softmax gives (1, 2, 4) / 7
+ROUTE_CLOSED_FORMS = [
+    ("soft", 7, [1 / 7, 2 / 7, 4 / 7]), ("fixed", 7, [1 / 3] * 3), ("top1", 7, [0, 0, 1]), ("top2", 7, [0, 1 / 3, 2 / 3]),
+    ("soft", 3, [1 / 3, 2 / 3, 0]), ("fixed", 3, [0.5, 0.5, 0]), ("top1", 3, [0, 1, 0]), ("top2", 3, [1 / 3, 2 / 3, 0]),
+    ("soft", 5, [1 / 5, 0, 4 / 5]), ("fixed", 5, [0.5, 0, 0.5]), ("top1", 5, [0, 0, 1]), ("top2", 5, [1 / 5, 0, 4 / 5]),
+    ("soft", 1, [1, 0, 0]), ("fixed", 1, [1, 0, 0]), ("top1", 1, [1, 0, 0]), ("top2", 1, [1, 0, 0]),
+]
+
+
+def check_route_closed_forms(gate):
+    for mode, tiers, want in ROUTE_CLOSED_FORMS:
+        np.testing.assert_allclose(gate(_ZL, mode, tiers)[0], want, rtol=1e-14, atol=1e-15, err_msg=f"{mode} {tiers}")
+    # ties go to the lower tier index
+    np.testing.assert_array_equal(gate(np.array([[1.0, 1.0, 0.0]]), "top1", 7)[0], [1, 0, 0])
+    np.testing.assert_array_equal(gate(np.array([[0.0, 2.0, 2.0]]), "top1", 7)[0], [0, 1, 0])
+    np.testing.assert_allclose(gate(np.array([[0.0, 3.0, 3.0]]), "top2", 7)[0], [0, 0.5, 0.5], rtol=1e-15)
+    e = math.exp(-3.0)
+    np.testing.assert_allclose(gate(np.array([[3.0, 0.0, 0.0]]), "top2", 7)[0], [1 / (1 + e), e / (1 + e), 0],
+                               rtol=1e-15)
+
+
+def test_route_gate_closed_forms():
+    check_route_closed_forms(O.route_gate)
+
+
+def test_route_gate_soft_is_softmax_and_rows_sum_to_one():
+    z = RNG.standard_normal((200, 3)) * 4
+    np.testing.assert_allclose(O.route_gate(z), scipy.special.softmax(z, axis=1), rtol=1e-13)
+    for mode in O.ROUTE_MODES:
+        for tiers in range(1, 8):
+            lam = O.route_gate(z, mode, tiers)
+            np.testing.assert_allclose(lam.sum(-1), 1.0, atol=1e-15)
+            for i in range(3):
+                if not (tiers >> i) & 1:
+                    assert (lam[:, i] == 0).all()
+            if mode in ("top1", "top2"):
+                k = 1 if mode == "top1" else min(2, bin(tiers).count("1"))
+                assert ((lam > 0).sum(-1) <= k).all()
+
+
+def test_route_margin():
+    np.testing.assert_allclose(O.route_margin(_ZL, "top1"), [math.log(2.0)], rtol=1e-15)
+    np.testing.assert_allclose(O.route_margin(_ZL, "top2"), [math.log(2.0)], rtol=1e-15)
+    np.testing.assert_allclose(O.route_margin(_ZL, "top1", 5), [math.log(4.0)], rtol=1e-15)
+    assert np.isinf(O.route_margin(_ZL, "soft")).all() and np.isinf(O.route_margin(_ZL, "top2", 3)).all()
+
+
+def test_layer_l1_only_tier_is_standard_causal_attention():
+    """tiers = L1 only ("L1 only (=MHA)", Table 9) through the configuration is textbook causal GQA."""
+    cfg = tiny_cfg(tiers=1)
+    w = tiny_weights(cfg, np.random.default_rng(21))
+    X = np.random.default_rng(22).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    out = _run(cfg, X, w)
+    assert (out["lam"] == np.array([1.0, 0.0, 0.0])).all()
+    for bi in range(cfg.batch):
+        q = (X[bi] @ w.w_q).reshape(cfg.seq, cfg.n_q_heads, cfg.d_head)
+        K = (X[bi] @ w.w_k).reshape(cfg.seq, cfg.n_kv_heads, cfg.d_head)
+        V = (X[bi] @ w.w_v).reshape(cfg.seq, cfg.n_kv_heads, cfg.d_head)
+        ref = brute_causal_gqa(q, K, V, cfg.n_kv_heads, cfg.scale)
+        np.testing.assert_allclose(out["O"][bi].reshape(ref.shape), ref, rtol=1e-11, atol=1e-12)
+
+
+def test_layer_fixed_and_hard_routing():
+    """Fixed routing equals lambda = 1/3 everywhere; hard top-1 picks each token's largest logit."""
+    cfg = tiny_cfg()
+    w = tiny_weights(cfg, np.random.default_rng(23))
+    X = np.random.default_rng(24).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    fixed = _run(cfg.replace(route_mode="fixed"), X, w)
+    ref = _run(cfg, X, w, lam_override=[1 / 3, 1 / 3, 1 / 3])
+    np.testing.assert_allclose(fixed["O"], ref["O"], rtol=1e-13, atol=1e-14)
+    top1 = _run(cfg.replace(route_mode="top1"), X, w)
+    soft = _run(cfg, X, w)
+    np.testing.assert_array_equal(top1["lam"].argmax(-1), soft["lam"].argmax(-1))
+    assert ((top1["lam"] == 0) | (top1["lam"] == 1)).all()
+    # the published layer is the soft gate
+    np.testing.assert_allclose(soft["lam"], O.softmax_rows(O.router_logits(
+        (X.reshape(-1, cfg.d_model) @ w.w_q), w.w_r1, w.w_r2)).reshape(soft["lam"].shape), rtol=1e-13)
+
+
+def test_decode_equals_prefill_rows_for_variants():
+    for kw in (dict(route_mode="top2"), dict(tiers=5), dict(route_mode="fixed", tiers=3)):
+        cfg = tiny_cfg(seq=29, **kw)
+        w = tiny_weights(cfg, np.random.default_rng(25))
+        X = np.random.default_rng(26).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+        np.testing.assert_allclose(O.fastmka_decode(X, w, cfg), _run(cfg, X, w)["O"], rtol=1e-11, atol=1e-12)
+
+
+def _mut_route_top2_unnormalised(z, mode="soft", tiers=7):
+    lam = O.route_gate(z, "soft", tiers)
+    if mode == "top2":
+        lam = np.where(lam == lam.min(-1, keepdims=True), 0.0, lam)
+    return lam if mode in ("soft", "top2") else O.route_gate(z, mode, tiers)
+
+
+def _mut_route_tie_high_index(z, mode="soft", tiers=7):
+    if mode != "top1":
+        return O.route_gate(z, mode, tiers)
+    zz = np.where(np.array([(tiers >> i) & 1 for i in range(3)], bool), z, -np.inf)
+    lam = np.zeros(np.shape(z))
+    np.put_along_axis(lam, (2 - np.argmax(zz[..., ::-1], axis=-1))[..., None], 1.0, axis=-1)
+    return lam
+
+
+def test_planted_routing_mistakes_are_caught():
+    for bad in (_mut_route_top2_unnormalised, _mut_route_tie_high_index):
+        with pytest.raises(AssertionError):
+            check_route_closed_forms(bad)
 
 
 # ============================================================================ regression snapshot
