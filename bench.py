@@ -120,6 +120,11 @@ def decode_bytes_per_token(cfg, ctx: int, ntot: int) -> float:
     return float(w + cache + state)
 
 
+def workload_cfg(args, name):
+    """The named workload with the routing gate / memory tiers the command line selects."""
+    return CONFIGS[name].replace(route_mode=args.route, tiers=args.tiers)
+
+
 def model_name(cfg) -> str:
     return "Llama-3.1-8B" if cfg.name.startswith("llama") else "Qwen2.5-7B"
 
@@ -135,7 +140,7 @@ def run_ours(args, rank, world, local_rank):
     import route_kv_memory_b200 as mka
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    cfg = CONFIGS[args.workload]
+    cfg = workload_cfg(args, args.workload)
     inp = make_inputs(cfg)
     weights = {k: v.to(dev) for k, v in inp.tensors().items() if k != "x"}
     layer = mka.FastMKALayer(cfg, weights, dev)
@@ -251,7 +256,9 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"{cfg.name}: {model_name(cfg)}-shaped FastMKA layer prefill, batch {cfg.batch} x seq "
                                f"{cfg.seq}, d_model {cfg.d_model}, {cfg.n_q_heads}/{cfg.n_kv_heads} heads, d_h "
                                f"{cfg.d_head}, router {cfg.dq}->{cfg.router_hidden}->3, alpha {cfg.alpha}, L3 block "
-                               f"{cfg.block}, R {cfg.recall_r}, nbits {cfg.hash_bits}, seed {cfg.seed}",
+                               f"{cfg.block}, R {cfg.recall_r}, nbits {cfg.hash_bits}, seed {cfg.seed}"
+                               + ("" if (cfg.route_mode, cfg.tiers) == ("soft", 7) else
+                                  f"; routing {cfg.route_mode}, tiers mask {cfg.tiers}"),
                    "global_batch": cfg.batch * world, "seq_len": cfg.seq,
                    "parallelism": f"replicas x{world} (independent sequences, no exchange)",
                    "l2": "flushed (512 MB write) before every timed step"},
@@ -274,7 +281,7 @@ def run_decode(args, cfg_prefill, inp_unused, weights_unused, dev, layer_pack=No
     """Decode us/token over a fused cache of `ctx` positions: 256 steps captured in one CUDA graph."""
     import route_kv_memory_b200 as mka
     out = {}
-    dcfg = CONFIGS["qwen7b_decode"]
+    dcfg = workload_cfg(args, "qwen7b_decode")
     dinp = make_inputs(dcfg, seq_total=max(args.decode_ctx) + dcfg.decode_new)
     w = {k: v.to(dev) for k, v in dinp.tensors().items() if k != "x"}
     peaks = load_peaks()
@@ -372,7 +379,7 @@ def run_reference(args, rank, world):
     """--impl reference: the CPU oracle, timed per step on a bounded sample of the same workload."""
     if rank != 0:
         return None
-    cfg = CONFIGS[args.workload]
+    cfg = workload_cfg(args, args.workload)
     inp = make_inputs(cfg)
     vals = []
     for i in range(args.warmup + args.steps):
@@ -430,6 +437,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen7b_4k")
+    ap.add_argument("--route", default="soft", choices=["soft", "fixed", "top1", "top2"],
+                    help="routing gate variant (the published layer is soft)")
+    ap.add_argument("--tiers", type=int, default=7, help="memory tier mask: 1 L1, 2 L2, 4 L3 (7 = all)")
     ap.add_argument("--decode-ctx", type=int, nargs="*", default=[131072])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode measurement (no prefill line)")

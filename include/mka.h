@@ -62,6 +62,22 @@ typedef enum {
 
 typedef enum { MKA_F32 = 0, MKA_BF16 = 1 } mka_dtype_t;
 
+/* Routing gate variants (abstract-and-tables page, Table 10).  From the router logits z
+ * (notes §2, z = GELU(q W_r1) W_r2) over the active tiers:
+ *   SOFT   lambda = softmax(z) (the layer as published);
+ *   FIXED  equal weights, 1 / (number of active tiers);
+ *   TOP1   all weight on the largest logit (ties to the lower tier index);
+ *   TOP2   softmax over the two largest logits, 0 for the third.
+ * Inactive tiers always get weight 0. */
+typedef enum { MKA_ROUTE_SOFT = 0, MKA_ROUTE_FIXED = 1, MKA_ROUTE_TOP1 = 2, MKA_ROUTE_TOP2 = 3 } mka_route_t;
+
+/* Memory tiers taking part (abstract-and-tables page, Table 9): a bit mask of L1 (the token),
+ * L2 (session EMA) and L3 (recalled blocks).  0 selects all three.  With L3 off the prefill
+ * skips the L3 codes and recall (recall_idx_out, if given, is filled with -1). */
+#define MKA_TIER_L1 1
+#define MKA_TIER_L2 2
+#define MKA_TIER_L3 4
+
 typedef struct mka_config {
   int32_t batch;         /* B */
   int32_t seq;           /* S: rows per sequence of a prefill call */
@@ -76,6 +92,8 @@ typedef struct mka_config {
   int32_t hash_bits;     /* nbits of the sign-projection code */
   int32_t dtype;         /* mka_dtype_t */
   float attn_scale;      /* <= 0 selects 1/sqrt(d_head) */
+  int32_t route_mode;    /* mka_route_t; MKA_ROUTE_SOFT for the published layer */
+  int32_t tiers;         /* MKA_TIER_* mask; 0 = all three */
 } mka_config;
 
 /* Raw layer weights, all in cfg->dtype, all [d_in, d_out] row-major. */

@@ -11,10 +11,11 @@ Pins (see ``tests/test_oracle_pins.py``) tie every function to facts the pages
 and mathematics fix: router rows sum to one, the EMA closed form, the
 strictly-past recall rule checked by brute force, lambda=(1,0,0) reducing to
 textbook causal attention, the online max-shift equalling the two-pass softmax,
-causality under future perturbation, and decode == prefill rows.
+causality under future perturbation, decode == prefill rows, and closed forms of
+the routing-gate variants (fixed, hard top-1 / top-2, removed tiers).
 """
 from .fastmka import (  # noqa: F401
-    gelu_erf, softmax_rows, router, session_ema, block_summaries, hash_codes, hamming,
+    gelu_erf, softmax_rows, router, router_logits, route_gate, route_margin, ROUTE_MODES, session_ema, block_summaries, hash_codes, hamming,
     recall_select, longterm_recall, fuse_sources, kv_project, causal_gqa_attention,
     online_softmax_attend, fastmka_prefill, fastmka_decode, Weights64, weights_f64,
     EXCUSE_EPS,

@@ -32,6 +32,9 @@ MKA_ERR_DEVICE_BOUNDS = -6
 MKA_ERR_WORKSPACE = -7
 MKA_F32 = 0
 MKA_BF16 = 1
+# routing gate variants (mka_route_t) and memory tiers (MKA_TIER_*)
+ROUTE_MODES = {"soft": 0, "fixed": 1, "top1": 2, "top2": 3}
+MKA_TIER_L1, MKA_TIER_L2, MKA_TIER_L3 = 1, 2, 4
 
 EXPORTED = [
     "mka_packed_weights_size", "mka_workspace_size", "mka_router_workspace_size", "mka_session_ema_workspace_size",
@@ -48,7 +51,7 @@ class mka_config(ctypes.Structure):
         ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("d_head", ctypes.c_int32),
         ("router_hidden", ctypes.c_int32), ("ema_alpha", ctypes.c_float), ("block_size", ctypes.c_int32),
         ("recall_r", ctypes.c_int32), ("hash_bits", ctypes.c_int32), ("dtype", ctypes.c_int32),
-        ("attn_scale", ctypes.c_float),
+        ("attn_scale", ctypes.c_float), ("route_mode", ctypes.c_int32), ("tiers", ctypes.c_int32),
     ]
 
 
@@ -118,7 +121,8 @@ def make_config(cfg, seq: Optional[int] = None, batch: Optional[int] = None) -> 
         n_q_heads=cfg.n_q_heads, n_kv_heads=cfg.n_kv_heads, d_head=cfg.d_head, router_hidden=cfg.router_hidden,
         ema_alpha=cfg.alpha, block_size=cfg.block, recall_r=cfg.recall_r, hash_bits=cfg.hash_bits,
         dtype=MKA_F32 if cfg.dtype == "f32" else MKA_BF16,
-        attn_scale=cfg.attn_scale if cfg.attn_scale is not None else 0.0)
+        attn_scale=cfg.attn_scale if cfg.attn_scale is not None else 0.0,
+        route_mode=ROUTE_MODES[getattr(cfg, "route_mode", "soft")], tiers=getattr(cfg, "tiers", 7))
 
 
 # ------------------------------------------------------------------ sizes

@@ -64,6 +64,7 @@ struct Dims {
   int B, S, d, Hq, Hkv, dh, rh, blk, R, nb, bf16, elem;
   int dq, dkv, width, nblk, T;
   float alpha, scale;
+  int route, tiers;  // routing gate variant; active tiers (MKA_TIER_* mask, never 0)
 };
 
 int check_cfg(const mka_config* c, Dims* o) {
@@ -80,6 +81,10 @@ int check_cfg(const mka_config* c, Dims* o) {
   if (c->recall_r < 1 || c->recall_r > 64) return fail(MKA_ERR_UNSUPPORTED, "recall_r must be in [1, 64]");
   if (c->hash_bits < 1 || c->hash_bits > 32) return fail(MKA_ERR_UNSUPPORTED, "hash_bits must be in [1, 32]");
   if (c->dtype != MKA_F32 && c->dtype != MKA_BF16) return fail(MKA_ERR_INVALID_ARG, "dtype must be MKA_F32 or MKA_BF16");
+  if (c->route_mode < MKA_ROUTE_SOFT || c->route_mode > MKA_ROUTE_TOP2)
+    return fail(MKA_ERR_INVALID_ARG, "route_mode must be one of MKA_ROUTE_*");
+  if (c->tiers & ~(MKA_TIER_L1 | MKA_TIER_L2 | MKA_TIER_L3))
+    return fail(MKA_ERR_INVALID_ARG, "tiers must be a mask of MKA_TIER_L1 | MKA_TIER_L2 | MKA_TIER_L3");
   long long T = (long long)c->batch * c->seq;
   if (T > (1LL << 30)) return fail(MKA_ERR_UNSUPPORTED, "batch * seq too large");
   if ((c->seq + c->block_size - 1) / c->block_size > 65535) return fail(MKA_ERR_UNSUPPORTED, "seq / block_size > 65535");
@@ -102,6 +107,8 @@ int check_cfg(const mka_config* c, Dims* o) {
   d.nblk = d.S / d.blk;
   d.T = (int)T;
   d.alpha = c->ema_alpha;
+  d.route = c->route_mode;
+  d.tiers = c->tiers ? c->tiers : (MKA_TIER_L1 | MKA_TIER_L2 | MKA_TIER_L3);
   d.scale = c->attn_scale > 0.f ? c->attn_scale : 1.f / sqrtf((float)d.dh);
   return MKA_OK;
 }
@@ -436,7 +443,7 @@ int mka_router(const mka_config* cfg, const void* q, const void* w_r1, const voi
   ep.seg[0] = OutSeg{0, d.rh, h, d.rh, 0};
   if (d.bf16) CUDA_TRY(gemm_tn_bf16_tc(q, d.dq, w1T, d.dq, d.T, d.rh, d.dq, ep, status_ptr(), s));
   else CUDA_TRY(gemm_tn_ffma(q, d.dq, 0, w1T, d.dq, 0, d.T, d.rh, d.dq, ep, s));
-  CUDA_TRY(router_tail(h, nullptr, d.rh, d.T, d.rh, wr2, lambda, s));
+  CUDA_TRY(router_tail(h, nullptr, d.rh, d.T, d.rh, wr2, d.route, d.tiers, lambda, s));
   return MKA_OK;
 }
 
@@ -573,8 +580,9 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   HashArgs ha{proj, d.nb, x, d.bf16, (const double*)P((void*)packed, PL.pT64), d.d, d.nb, d.d};
   const double* p64 = (const double*)P((void*)packed, PL.p64);
   auto k_router = [&](cudaStream_t st) {
-    return PL.router_fused ? router_softmax(h1, d.rh / 128, d.T, lam, st)
-                           : router_tail(h1, h2, d.rh, d.T, d.rh, (const float*)P((void*)packed, PL.wr2), lam, st);
+    return PL.router_fused
+               ? router_softmax(h1, d.rh / 128, d.T, d.route, d.tiers, lam, st)
+               : router_tail(h1, h2, d.rh, d.T, d.rh, (const float*)P((void*)packed, PL.wr2), d.route, d.tiers, lam, st);
   };
   auto k_tcode = [&](cudaStream_t st) { return token_codes(ha, d.T, tcode, st); };
   auto k_bsum = [&](cudaStream_t st) {
@@ -596,16 +604,18 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
     aux_lock.lock();
     ax = aux_streams();
   }
+  // With L3 off (MKA_TIER_L3 not set) its weight is 0: no codes and no recall, count 0 for every token.
+  const bool l3 = (d.tiers & MKA_TIER_L3) != 0;
   if (ax) {
     CUDA_TRY(cudaEventRecord(ax->fork, s));
     CUDA_TRY(cudaStreamWaitEvent(ax->st[0], ax->fork, 0));
     CUDA_TRY(cudaStreamWaitEvent(ax->st[1], ax->fork, 0));
-    CUDA_TRY(k_scode(ax->st[0]));
+    if (l3) CUDA_TRY(k_scode(ax->st[0]));
     CUDA_TRY(cudaEventRecord(ax->join[0], ax->st[0]));
     if (state) CUDA_TRY(k_tail(ax->st[0]));  // reads x and xkv only; joined at the end
     CUDA_TRY(cudaEventRecord(ax->join[2], ax->st[0]));
     CUDA_TRY(k_router(ax->st[1]));
-    CUDA_TRY(k_tcode(ax->st[1]));
+    if (l3) CUDA_TRY(k_tcode(ax->st[1]));
     CUDA_TRY(cudaEventRecord(ax->join[1], ax->st[1]));
     CUDA_TRY(k_bsum(s));
     CUDA_TRY(k_carry(s));
@@ -614,16 +624,21 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   } else {
     CUDA_TRY(k_router(s));
     STAGE(s);
-    CUDA_TRY(k_tcode(s));
+    if (l3) CUDA_TRY(k_tcode(s));
     STAGE(s);
     CUDA_TRY(k_bsum(s));
     STAGE(s);
-    CUDA_TRY(k_scode(s));
+    if (l3) CUDA_TRY(k_scode(s));
     STAGE(s);
     CUDA_TRY(k_carry(s));
   }
   STAGE(s);
-  CUDA_TRY(recall_select(tcode, scode, code_bstride, d.B, d.S, d.nblk, d.blk, d.R, idx, cnt, s));
+  if (l3) {
+    CUDA_TRY(recall_select(tcode, scode, code_bstride, d.B, d.S, d.nblk, d.blk, d.R, idx, cnt, s));
+  } else {
+    CUDA_TRY(cudaMemsetAsync(cnt, 0, (size_t)d.T * sizeof(int), s));
+    if (recall_idx_out) CUDA_TRY(cudaMemsetAsync(idx, 0xff, (size_t)d.T * d.R * sizeof(int), s));
+  }
   STAGE(s);
   // 5. route-fuse -> K, V
   FuseArgs fa{};
@@ -673,7 +688,7 @@ int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size
   a.w_r2 = (const float*)P((void*)packed, PL.wr2); a.pT64 = (const double*)P((void*)packed, PL.pT64);
   a.dq = d.dq; a.dkv = d.dkv; a.rh = d.rh; a.nb = d.nb; a.rh_segs = PL.rh_segs; a.r_inter = PL.router_fused;
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.dh = d.dh; a.blk = d.blk; a.R = d.R; a.Lmax = max_positions;
-  a.maxblk = SL.maxblk; a.alpha = d.alpha; a.scale = d.scale;
+  a.maxblk = SL.maxblk; a.alpha = d.alpha; a.scale = d.scale; a.route_mode = d.route; a.tiers = d.tiers;
   a.x_new = x_new; a.out = out;
   a.pos = (int*)P(state, SL.pos); a.kcache = P(state, SL.kc); a.vcache = P(state, SL.vc);
   a.ema = (float*)P(state, SL.ema); a.blk_sum = (float*)P(state, SL.blk_sum); a.blk_x = (double*)P(state, SL.blk_x);

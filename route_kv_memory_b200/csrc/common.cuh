@@ -48,6 +48,53 @@ __device__ __forceinline__ float warp_max(float v) {
 // GELU(x) = x * Phi(x), Phi(x) = 0.5 * erfc(-x / sqrt(2)).
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * erfcf(-x * 0.70710678118654752f); }
 
+// Routing gate over the three memory sources from the router logits (notes §2), with the
+// routing variant and the active tiers of the layer configuration (abstract page, Tables 9
+// and 10).  mode: 0 soft = softmax over the active tiers; 1 fixed = equal weights over them;
+// 2 top-1 = all weight on the largest active logit; 3 top-2 = softmax over the two largest
+// active logits.  Ties go to the lower tier index.  tiers: bit 0 L1, bit 1 L2, bit 2 L3
+// (never 0 here).  Inactive tiers get 0.
+__device__ __forceinline__ void route_gate(float z0, float z1, float z2, int mode, int tiers, float* l) {
+  const float z[3] = {z0, z1, z2};
+  int i1 = -1, i2 = -1, n = 0;  // the two largest active logits, in (value desc, index asc) order
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    if (!((tiers >> i) & 1)) continue;
+    ++n;
+    if (i1 < 0 || z[i] > z[i1]) {
+      i2 = i1;
+      i1 = i;
+    } else if (i2 < 0 || z[i] > z[i2]) {
+      i2 = i;
+    }
+  }
+  l[0] = l[1] = l[2] = 0.f;
+  if (mode == 1) {
+    const float w = 1.f / (float)n;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      if ((tiers >> i) & 1) l[i] = w;
+  } else if (mode == 2 || (mode == 3 && i2 < 0)) {
+    l[i1] = 1.f;
+  } else if (mode == 3) {
+    const float e = expf(z[i2] - z[i1]);
+    const float inv = 1.f / (1.f + e);
+    l[i1] = inv;
+    l[i2] = e * inv;
+  } else {
+    const float m = z[i1];
+    float e[3], sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      e[i] = ((tiers >> i) & 1) ? expf(z[i] - m) : 0.f;
+      sum += e[i];
+    }
+    const float inv = 1.f / sum;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) l[i] = e[i] * inv;
+  }
+}
+
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Raise a kernel's dynamic shared memory limit.  Skipped while `s` is being

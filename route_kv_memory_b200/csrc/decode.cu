@@ -95,7 +95,7 @@ __device__ void token_update(const DecodeArgs& a, const int bi) {
   if (s_skip) return;
   const int pos = s_pos;
 
-  // router (notes §2): z = GELU(h) W_r2, lambda = softmax(z)
+  // router (notes §2): z = GELU(h) W_r2, lambda = route_gate(z) (softmax for the published layer)
   float z0 = 0.f, z1 = 0.f, z2 = 0.f;
   for (int j = tid; j < a.rh; j += blockDim.x) {
     float hv;
@@ -140,12 +140,7 @@ __device__ void token_update(const DecodeArgs& a, const int bi) {
       t1 += s_red[w][1];
       t2 += s_red[w][2];
     }
-    float m = fmaxf(t0, fmaxf(t1, t2));
-    float e0 = expf(t0 - m), e1 = expf(t1 - m), e2 = expf(t2 - m);
-    float inv = 1.f / (e0 + e1 + e2);
-    s_lam[0] = e0 * inv;
-    s_lam[1] = e1 * inv;
-    s_lam[2] = e2 * inv;
+    route_gate(t0, t1, t2, a.route_mode, a.tiers, s_lam);
   }
   // L3 recall over the finished blocks (notes §1): counting select, warp 0
   const int n_elig = min(pos / a.blk, a.maxblk);
@@ -632,12 +627,7 @@ __device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, T
       t1 += s_red[w][1];
       t2 += s_red[w][2];
     }
-    const float m = fmaxf(t0, fmaxf(t1, t2));
-    const float e0 = expf(t0 - m), e1 = expf(t1 - m), e2 = expf(t2 - m);
-    const float inv = 1.f / (e0 + e1 + e2);
-    td->lam[0] = e0 * inv;
-    td->lam[1] = e1 * inv;
-    td->lam[2] = e2 * inv;
+    route_gate(t0, t1, t2, a.route_mode, a.tiers, td->lam);
   }
   // recall among the finished blocks: counting select by (distance, index)
   const int n_elig = min(pos / a.blk, a.maxblk);

@@ -58,10 +58,11 @@ struct HashArgs {
   int d, nb, K;          // K: length of the dot products that produced proj
 };
 
-cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, float* lam,
-                        cudaStream_t s);
-// lambda = softmax(sum_r zpart[r][t][0..2]) for the router partials of the fused GEMM epilogue.
-cudaError_t router_softmax(const float* zpart, int nparts, int T, float* lam, cudaStream_t s);
+// lambda = route_gate(GELU(h1 + h2) . w_r2) per token (mode, tiers: see route_gate in common.cuh).
+cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, int mode,
+                        int tiers, float* lam, cudaStream_t s);
+// lambda = route_gate(sum_r zpart[r][t][0..2]) for the router partials of the fused GEMM epilogue.
+cudaError_t router_softmax(const float* zpart, int nparts, int T, int mode, int tiers, float* lam, cudaStream_t s);
 // Writes the bf16 hi/lo split of w [rh, d] float32 into the rows of the packed matrix so that every
 // 256-row group holds the hi then the lo rows of 128 consecutive hidden units (rh % 128 == 0).
 cudaError_t split_hi_lo_interleaved(const float* w, int rh, int d, void* dst, cudaStream_t s);
@@ -132,6 +133,7 @@ struct DecodeArgs {
   int r_inter;                   // hi/lo rows interleaved per 128 hidden units (else [hi | lo])
   int B, Hq, Hkv, dh, blk, R, Lmax, maxblk;
   float alpha, scale;
+  int route_mode, tiers;         // routing gate variant and active tiers (route_gate)
   const void* x_new;             // [B, d]
   void* out;                     // [B, dq]
   // state

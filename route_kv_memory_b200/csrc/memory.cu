@@ -16,7 +16,7 @@ namespace mka {
 // lambda = softmax(GELU(h) W_r2) per token (notes §2); h = h1 (+ h2) when the
 // first layer was applied as a bf16 hi/lo pair.
 __global__ void router_tail_kernel(const float* __restrict__ h1, const float* __restrict__ h2, int ldh, int T, int rh,
-                                   const float* __restrict__ w_r2, float* __restrict__ lam) {
+                                   const float* __restrict__ w_r2, int mode, int tiers, float* __restrict__ lam) {
   extern __shared__ float sw[];
   for (int i = threadIdx.x; i < rh * 3; i += blockDim.x) sw[i] = w_r2[i];
   __syncthreads();
@@ -38,19 +38,18 @@ __global__ void router_tail_kernel(const float* __restrict__ h1, const float* __
   z1 = warp_sum(z1);
   z2 = warp_sum(z2);
   if (lane == 0) {
-    float m = fmaxf(z0, fmaxf(z1, z2));
-    float e0 = expf(z0 - m), e1 = expf(z1 - m), e2 = expf(z2 - m);
-    float inv = 1.f / (e0 + e1 + e2);
-    lam[(size_t)t * 3 + 0] = e0 * inv;
-    lam[(size_t)t * 3 + 1] = e1 * inv;
-    lam[(size_t)t * 3 + 2] = e2 * inv;
+    float l[3];
+    route_gate(z0, z1, z2, mode, tiers, l);
+    lam[(size_t)t * 3 + 0] = l[0];
+    lam[(size_t)t * 3 + 1] = l[1];
+    lam[(size_t)t * 3 + 2] = l[2];
   }
 }
 
-cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, float* lam,
-                        cudaStream_t s) {
+cudaError_t router_tail(const float* h1, const float* h2, int ldh, int T, int rh, const float* w_r2, int mode,
+                        int tiers, float* lam, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  router_tail_kernel<<<(T + 7) / 8, 256, rh * 3 * sizeof(float), s>>>(h1, h2, ldh, T, rh, w_r2, lam);
+  router_tail_kernel<<<(T + 7) / 8, 256, rh * 3 * sizeof(float), s>>>(h1, h2, ldh, T, rh, w_r2, mode, tiers, lam);
   return cudaGetLastError();
 }
 
@@ -66,7 +65,8 @@ template <> struct Vec4<bf16> {
     return make_float4(fa.x, fa.y, fb.x, fb.y);
   }
 };
-__global__ void router_softmax_kernel(const float* __restrict__ zpart, int nparts, int T, float* __restrict__ lam) {
+__global__ void router_softmax_kernel(const float* __restrict__ zpart, int nparts, int T, int mode, int tiers,
+                                      float* __restrict__ lam) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
   float z0 = 0.f, z1 = 0.f, z2 = 0.f;
@@ -76,17 +76,16 @@ __global__ void router_softmax_kernel(const float* __restrict__ zpart, int npart
     z1 += v.y;
     z2 += v.z;
   }
-  const float m = fmaxf(z0, fmaxf(z1, z2));
-  const float e0 = expf(z0 - m), e1 = expf(z1 - m), e2 = expf(z2 - m);
-  const float inv = 1.f / (e0 + e1 + e2);
-  lam[(size_t)t * 3 + 0] = e0 * inv;
-  lam[(size_t)t * 3 + 1] = e1 * inv;
-  lam[(size_t)t * 3 + 2] = e2 * inv;
+  float l[3];
+  route_gate(z0, z1, z2, mode, tiers, l);
+  lam[(size_t)t * 3 + 0] = l[0];
+  lam[(size_t)t * 3 + 1] = l[1];
+  lam[(size_t)t * 3 + 2] = l[2];
 }
 
-cudaError_t router_softmax(const float* zpart, int nparts, int T, float* lam, cudaStream_t s) {
+cudaError_t router_softmax(const float* zpart, int nparts, int T, int mode, int tiers, float* lam, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  router_softmax_kernel<<<(T + 255) / 256, 256, 0, s>>>(zpart, nparts, T, lam);
+  router_softmax_kernel<<<(T + 255) / 256, 256, 0, s>>>(zpart, nparts, T, mode, tiers, lam);
   return cudaGetLastError();
 }
 

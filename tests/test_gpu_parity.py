@@ -105,6 +105,53 @@ def test_concurrent_branches_match_sequential(mka):
         assert torch.equal(u, v)
 
 
+# ------------------------------------------------------------------ routing and tier variants
+ROUTE_VARIANTS = [("fixed", 7), ("top1", 7), ("top2", 7), ("soft", 3), ("soft", 5), ("soft", 1), ("top2", 5),
+                  ("top1", 3)]
+MARGIN_MIN = 1e-4  # hard gates: every token's deciding logit gap in the oracle clears this
+
+
+def margin_safe_inputs(cfg, seeds=range(31, 60)):
+    """The first seed whose hard-gate decisions (oracle logits, float64) are all far from a tie, so both
+    sides take every top-1 / top-2 decision the same way; soft and fixed gates take the first seed."""
+    for seed in seeds:
+        c = cfg.replace(seed=seed)
+        inp = make_inputs(c)
+        w = oracle_weights(inp)
+        X = inp.x[:, :c.seq].double().numpy().reshape(-1, c.d_model)
+        margin = oracle.route_margin(oracle.router_logits(X @ w.w_q, w.w_r1, w.w_r2), c.route_mode, c.tiers)
+        if margin.min() > MARGIN_MIN:
+            return c, inp
+    raise AssertionError("no seed with every routing decision clear of a tie")
+
+
+@pytest.mark.parametrize("mode,tiers", ROUTE_VARIANTS, ids=[f"{m}-{t}" for m, t in ROUTE_VARIANTS])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_routing_variants(mode, tiers, dtype):
+    kw = dict(seq=600, d_head=128, n_q_heads=8, n_kv_heads=2, router_hidden=128, block=64, recall_r=4,
+              hash_bits=32) if dtype == "bf16" else {}
+    cfg, inp = margin_safe_inputs(small("route", dtype, route_mode=mode, tiers=tiers, **kw))
+    ref = oracle_prefill(cfg, inp)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    if tiers & 4:
+        check_recall(idx, ref)
+    else:
+        assert (idx.cpu() == -1).all()
+    check_out(out, ref["O"], dtype)
+
+
+@pytest.mark.parametrize("mode,tiers", [("top2", 7), ("soft", 3), ("fixed", 5)])
+def test_routing_variants_decode(mode, tiers):
+    base = small("decroute", "bf16", batch=2, seq=700, d_head=128, n_q_heads=8, n_kv_heads=2, router_hidden=128,
+                 block=64, recall_r=4, hash_bits=32, route_mode=mode, tiers=tiers)
+    cfg, inp = margin_safe_inputs(base)
+    ctx = 640
+    got = decode_run(cfg, inp, ctx, cfg.seq - ctx, 720)
+    ref = oracle_prefill(cfg, inp, rows=np.arange(ctx, cfg.seq))
+    check_out(got, ref["O"], "bf16")
+
+
 # ------------------------------------------------------------------ entry points one by one
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_router_entry(mka, dtype):
