@@ -400,3 +400,74 @@ def fastmka_decode(X: np.ndarray, w: Weights64, cfg) -> np.ndarray:
                 codes.append(int(hash_codes(s_new[None], w.P)[0][0]))
                 block_sum = np.zeros(d)
     return O
+
+
+# ----------------------------------------------------------------------------- full MKA (three paths)
+def recalled_block_attention(q_rows: np.ndarray, idx: np.ndarray, count: np.ndarray, K: np.ndarray,
+                             V: np.ndarray, b: int, n_kv_heads: int, scale: float) -> np.ndarray:
+    """a_3 of full MKA for ONE sequence: each query row attends to every token of its recalled blocks.
+
+    notes §1 / §2: L3 recalls R past blocks and a_3 = softmax(q k_3^T) v_3 over them.  Read here as
+    the keys and values of the recalled blocks' tokens (block j = rows [j*b, (j+1)*b), all strictly
+    past, so no mask); 0 where nothing is recalled.  q_rows [n, Hq, dh]; idx [n, R] (-1 padded),
+    count [n]; K, V [S, Hkv, dh].  Returns [n, Hq, dh].
+    """
+    n, Hq, dh = q_rows.shape
+    G = Hq // n_kv_heads
+    out = np.zeros((n, Hq, dh))
+    for i in range(n):
+        c = int(count[i])
+        if c == 0:
+            continue
+        tok = (idx[i, :c, None] * b + np.arange(b)[None, :]).reshape(-1)
+        for h in range(Hq):
+            g = h // G
+            s = K[tok, g] @ q_rows[i, h] * scale
+            p = np.exp(s - s.max())
+            out[i, h] = (p @ V[tok, g]) / p.sum()
+    return out
+
+
+def mka_full_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray] = None,
+                     lam_override: Optional[np.ndarray] = None) -> dict:
+    """Full MKA over whole sequences: three attention outputs mixed by the gate (notes §2).
+
+    O_h = sum_l lambda_l * a_l with a_l = softmax(q_h k_l^T) v_l:
+      a_1  causal attention over the tokens themselves, k_1, v_1 = X W_k, X W_v (L1);
+      a_2  attention over the L2 session summary of position t, one key, so weight 1 and
+           a_2 = M2[t] W_v (M2 the causal EMA, M2[0] = 0);
+      a_3  attention over the tokens of the blocks L3 recalls for t (recalled_block_attention).
+    lambda is the routing gate (route_gate with cfg's mode and tiers) unless lam_override.
+    The abstract page's Table 11 contrasts this three-path form with FastMKA.
+    """
+    B, S, d = X.shape
+    Hq, Hkv, dh = cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head
+    b, R = cfg.block, cfg.recall_r
+    G = Hq // Hkv
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = {"rows": rows, "lam": np.zeros((B, S, 3)), "idx": np.zeros((B, S, R), np.int64),
+           "count": np.zeros((B, S), np.int64), "excuse": np.zeros((B, S), bool),
+           "O": np.zeros((B, len(rows), Hq * dh)), "route_margin": np.zeros((B, S))}
+    mode, tiers = getattr(cfg, "route_mode", "soft"), getattr(cfg, "tiers", 7)
+    for bi in range(B):
+        Xb = np.asarray(X[bi], np.float64)
+        q = Xb @ w.w_q
+        z = router_logits(q, w.w_r1, w.w_r2)
+        lam = route_gate(z, mode, tiers) if lam_override is None else np.broadcast_to(
+            np.asarray(lam_override, np.float64), (S, 3))
+        K1 = (Xb @ w.w_k).reshape(S, Hkv, dh)
+        V1 = (Xb @ w.w_v).reshape(S, Hkv, dh)
+        M2, _ = session_ema(Xb[None], cfg.alpha)
+        V2 = (M2[0] @ w.w_v).reshape(S, Hkv, dh)
+        summ = block_summaries(Xb[None], b)[0]
+        idx, cnt, _, exc, _, _ = longterm_recall(Xb, np.arange(S), summ, w.P, b, R)
+        qr = q[rows].reshape(len(rows), Hq, dh)
+        a1 = causal_gqa_attention(qr, rows, K1, V1, Hkv, cfg.scale)
+        a2 = V2[rows][:, np.arange(Hq) // G]
+        a3 = recalled_block_attention(qr, idx[rows], cnt[rows], K1, V1, b, Hkv, cfg.scale)
+        lr = lam[rows]
+        O = lr[:, 0, None, None] * a1 + lr[:, 1, None, None] * a2 + lr[:, 2, None, None] * a3
+        out["O"][bi] = O.reshape(len(rows), Hq * dh)
+        out["lam"][bi], out["idx"][bi], out["count"][bi], out["excuse"][bi] = lam, idx, cnt, exc
+        out["route_margin"][bi] = route_margin(z, mode, tiers)
+    return out

@@ -522,6 +522,137 @@ def test_planted_routing_mistakes_are_caught():
             check_route_closed_forms(bad)
 
 
+# ============================================================================ full MKA (three paths)
+def brute_masked_gqa(q, K, V, Hkv, scale, allowed):
+    """Softmax attention with an explicit boolean key mask allowed[t, j]; rows with no key give 0."""
+    S, Hq, dh = q.shape
+    G = Hq // Hkv
+    out = np.zeros_like(q)
+    for h in range(Hq):
+        g = h // G
+        for t in range(S):
+            keys = [j for j in range(K.shape[0]) if allowed[t, j]]
+            if not keys:
+                continue
+            sc = np.array([scale * float(np.dot(q[t, h], K[j, g])) for j in keys])
+            wts = np.exp(sc - sc.max())
+            out[t, h] = (wts / wts.sum()) @ V[keys, g]
+    return out
+
+
+def _mka_setup(seed, **kw):
+    cfg = tiny_cfg(**kw)
+    w = tiny_weights(cfg, np.random.default_rng(seed))
+    X = np.random.default_rng(seed + 1).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    return cfg, w, X
+
+
+def _heads(cfg, X, w, bi):
+    q = (X[bi] @ w.w_q).reshape(cfg.seq, cfg.n_q_heads, cfg.d_head)
+    K = (X[bi] @ w.w_k).reshape(cfg.seq, cfg.n_kv_heads, cfg.d_head)
+    V = (X[bi] @ w.w_v).reshape(cfg.seq, cfg.n_kv_heads, cfg.d_head)
+    return q, K, V
+
+
+def check_mka_l1_path(fn):
+    cfg, w, X = _mka_setup(30)
+    out = fn(X, w, cfg, lam_override=[1.0, 0.0, 0.0])
+    for bi in range(cfg.batch):
+        q, K, V = _heads(cfg, X, w, bi)
+        ref = brute_causal_gqa(q, K, V, cfg.n_kv_heads, cfg.scale)
+        np.testing.assert_allclose(out["O"][bi].reshape(ref.shape), ref, rtol=1e-11, atol=1e-12)
+
+
+def check_mka_l2_path(fn):
+    """lambda = e_2: O[t, h] = (M2[t] W_v)[g(h)], M2 from the closed form sum_k a^k (1-a) X[t-1-k]."""
+    cfg, w, X = _mka_setup(32)
+    out = fn(X, w, cfg, lam_override=[0.0, 1.0, 0.0])
+    a, G = cfg.alpha, cfg.n_q_heads // cfg.n_kv_heads
+    for bi in range(cfg.batch):
+        for t in range(cfg.seq):
+            m2 = sum(a ** k * (1 - a) * X[bi, t - 1 - k] for k in range(t)) if t else np.zeros(cfg.d_model)
+            v2 = (m2 @ w.w_v).reshape(cfg.n_kv_heads, cfg.d_head)
+            want = v2[np.arange(cfg.n_q_heads) // G].reshape(-1)
+            np.testing.assert_allclose(out["O"][bi, t], want, rtol=1e-11, atol=1e-12)
+
+
+def check_mka_l3_path_recall_all(fn):
+    """R >= every eligible block: a_3 attends to the whole prefix of full blocks [0, floor(t/b)*b)."""
+    cfg, w, X = _mka_setup(34, recall_r=20)
+    out = fn(X, w, cfg, lam_override=[0.0, 0.0, 1.0])
+    S, b = cfg.seq, cfg.block
+    allowed = np.arange(S)[None, :] < (np.arange(S) // b * b)[:, None]
+    for bi in range(cfg.batch):
+        q, K, V = _heads(cfg, X, w, bi)
+        ref = brute_masked_gqa(q, K, V, cfg.n_kv_heads, cfg.scale, allowed)
+        np.testing.assert_allclose(out["O"][bi].reshape(ref.shape), ref, rtol=1e-11, atol=1e-12)
+
+
+def test_mka_l1_path_is_textbook_causal_attention():
+    check_mka_l1_path(O.mka_full_prefill)
+
+
+def test_mka_l2_path_is_the_ema_value():
+    check_mka_l2_path(O.mka_full_prefill)
+
+
+def test_mka_l3_path_with_every_block_recalled():
+    check_mka_l3_path_recall_all(O.mka_full_prefill)
+
+
+def test_mka_l3_path_matches_a_dense_block_mask():
+    """Small R: the recalled blocks (pinned by the brute-force recall tests) as a dense key mask."""
+    cfg, w, X = _mka_setup(36, recall_r=2)
+    out = O.mka_full_prefill(X, w, cfg, lam_override=[0.0, 0.0, 1.0])
+    S, b = cfg.seq, cfg.block
+    for bi in range(cfg.batch):
+        allowed = np.zeros((S, S), bool)
+        for t in range(S):
+            for j in out["idx"][bi, t, :out["count"][bi, t]]:
+                allowed[t, j * b:(j + 1) * b] = True
+        assert (allowed.sum(1) == out["count"][bi] * b).all()
+        q, K, V = _heads(cfg, X, w, bi)
+        ref = brute_masked_gqa(q, K, V, cfg.n_kv_heads, cfg.scale, allowed)
+        np.testing.assert_allclose(out["O"][bi].reshape(ref.shape), ref, rtol=1e-11, atol=1e-12)
+
+
+def test_mka_mixes_paths_linearly():
+    cfg, w, X = _mka_setup(38)
+    lam = np.array([0.2, 0.5, 0.3])
+    mixed = O.mka_full_prefill(X, w, cfg, lam_override=lam)["O"]
+    parts = [O.mka_full_prefill(X, w, cfg, lam_override=np.eye(3)[i])["O"] for i in range(3)]
+    np.testing.assert_allclose(mixed, sum(l * p for l, p in zip(lam, parts)), rtol=1e-12, atol=1e-13)
+
+
+def _mut_mka_a3_current_block(X, w, cfg, rows=None, lam_override=None):
+    """Planted mistake: the L3 path also sees the current, unfinished block."""
+    cfg2 = cfg.replace(block=cfg.block)
+    out = O.mka_full_prefill(X, w, cfg2, rows, lam_override)
+    S, b = cfg.seq, cfg.block
+    for bi in range(cfg.batch):
+        q, K, V = _heads(cfg, X, w, bi)
+        allowed = np.arange(S)[None, :] < np.minimum(S, (np.arange(S) // b + 1) * b)[:, None]
+        allowed &= np.arange(S)[None, :] <= np.arange(S)[:, None]
+        extra = brute_masked_gqa(q, K, V, cfg.n_kv_heads, cfg.scale, allowed)
+        lam = np.asarray(lam_override if lam_override is not None else [0, 0, 1], float)
+        out["O"][bi] = out["O"][bi] * (1 - lam[2]) + lam[2] * extra.reshape(S, -1)
+    return out
+
+
+def _mut_mka_a2_leaks_current(X, w, cfg, rows=None, lam_override=None):
+    """Planted mistake: the L2 summary at t already contains x_t."""
+    Xs = np.concatenate([X[:, 1:], X[:, -1:]], axis=1)
+    return O.mka_full_prefill(Xs, w, cfg, rows, lam_override) if lam_override is not None and \
+        lam_override[1] == 1.0 else O.mka_full_prefill(X, w, cfg, rows, lam_override)
+
+
+def test_planted_mka_mistakes_are_caught():
+    with pytest.raises(AssertionError):
+        check_mka_l3_path_recall_all(_mut_mka_a3_current_block)
+    with pytest.raises(AssertionError):
+        check_mka_l2_path(_mut_mka_a2_leaks_current)
+
+
 # ============================================================================ regression snapshot
 def test_golden_snapshot_unchanged():
     """tests/golden/tiny_f32_oracle.json (written by tests/golden/make_golden.py from the oracle) still holds."""
