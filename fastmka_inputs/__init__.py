@@ -51,6 +51,7 @@ class FastMKAConfig:
     decode_new: int = 0  # tokens decoded one at a time after a prefix of `seq`
     route_mode: str = "soft"  # routing gate variant: "soft", "fixed", "top1", "top2"
     tiers: int = 7  # active memory tiers: bit 0 L1, bit 1 L2, bit 2 L3
+    attention_paths: int = 1  # 1: FastMKA (fused K/V, one attention); 3: full MKA (three attention paths)
 
     @property
     def dq(self) -> int:

@@ -94,6 +94,12 @@ typedef struct mka_config {
   float attn_scale;      /* <= 0 selects 1/sqrt(d_head) */
   int32_t route_mode;    /* mka_route_t; MKA_ROUTE_SOFT for the published layer */
   int32_t tiers;         /* MKA_TIER_* mask; 0 = all three */
+  int32_t attention_paths; /* 1 (or 0): FastMKA, fused K/V and one attention (notes §3);
+                              3: full MKA, three attention outputs mixed by the gate (notes §2):
+                              causal over the tokens, the L2 summary value, attention over the
+                              recalled L3 blocks' tokens.  3 is implemented for bf16 prefill with
+                              block_size a multiple of 128 and no decode state; otherwise
+                              MKA_ERR_UNSUPPORTED */
 } mka_config;
 
 /* Raw layer weights, all in cfg->dtype, all [d_in, d_out] row-major. */

@@ -52,6 +52,7 @@ class mka_config(ctypes.Structure):
         ("router_hidden", ctypes.c_int32), ("ema_alpha", ctypes.c_float), ("block_size", ctypes.c_int32),
         ("recall_r", ctypes.c_int32), ("hash_bits", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("attn_scale", ctypes.c_float), ("route_mode", ctypes.c_int32), ("tiers", ctypes.c_int32),
+        ("attention_paths", ctypes.c_int32),
     ]
 
 
@@ -122,7 +123,8 @@ def make_config(cfg, seq: Optional[int] = None, batch: Optional[int] = None) -> 
         ema_alpha=cfg.alpha, block_size=cfg.block, recall_r=cfg.recall_r, hash_bits=cfg.hash_bits,
         dtype=MKA_F32 if cfg.dtype == "f32" else MKA_BF16,
         attn_scale=cfg.attn_scale if cfg.attn_scale is not None else 0.0,
-        route_mode=ROUTE_MODES[getattr(cfg, "route_mode", "soft")], tiers=getattr(cfg, "tiers", 7))
+        route_mode=ROUTE_MODES[getattr(cfg, "route_mode", "soft")], tiers=getattr(cfg, "tiers", 7),
+        attention_paths=getattr(cfg, "attention_paths", 1))
 
 
 # ------------------------------------------------------------------ sizes

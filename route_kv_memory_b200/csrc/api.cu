@@ -65,6 +65,7 @@ struct Dims {
   int dq, dkv, width, nblk, T;
   float alpha, scale;
   int route, tiers;  // routing gate variant; active tiers (MKA_TIER_* mask, never 0)
+  int paths;         // 1 FastMKA, 3 full MKA
 };
 
 int check_cfg(const mka_config* c, Dims* o) {
@@ -85,6 +86,10 @@ int check_cfg(const mka_config* c, Dims* o) {
     return fail(MKA_ERR_INVALID_ARG, "route_mode must be one of MKA_ROUTE_*");
   if (c->tiers & ~(MKA_TIER_L1 | MKA_TIER_L2 | MKA_TIER_L3))
     return fail(MKA_ERR_INVALID_ARG, "tiers must be a mask of MKA_TIER_L1 | MKA_TIER_L2 | MKA_TIER_L3");
+  if (c->attention_paths != 0 && c->attention_paths != 1 && c->attention_paths != 3)
+    return fail(MKA_ERR_INVALID_ARG, "attention_paths must be 1 (FastMKA) or 3 (full MKA)");
+  if (c->attention_paths == 3 && (c->dtype != MKA_BF16 || c->block_size % 128))
+    return fail(MKA_ERR_UNSUPPORTED, "full MKA needs bf16 and a block_size that is a multiple of 128");
   long long T = (long long)c->batch * c->seq;
   if (T > (1LL << 30)) return fail(MKA_ERR_UNSUPPORTED, "batch * seq too large");
   if ((c->seq + c->block_size - 1) / c->block_size > 65535) return fail(MKA_ERR_UNSUPPORTED, "seq / block_size > 65535");
@@ -108,6 +113,7 @@ int check_cfg(const mka_config* c, Dims* o) {
   d.T = (int)T;
   d.alpha = c->ema_alpha;
   d.route = c->route_mode;
+  d.paths = c->attention_paths == 3 ? 3 : 1;
   d.tiers = c->tiers ? c->tiers : (MKA_TIER_L1 | MKA_TIER_L2 | MKA_TIER_L3);
   d.scale = c->attn_scale > 0.f ? c->attn_scale : 1.f / sqrtf((float)d.dh);
   return MKA_OK;
@@ -144,7 +150,7 @@ PackLayout pack_layout(const Dims& d) {
 
 // ---------------------------------------------------------------- prefill workspace
 struct PrefillWs {
-  size_t q, xkv, h1, h2, proj, lam, tcode, xsum, bsum, bend, gend, carry, scode, idx, cnt, k, v, total;
+  size_t q, xkv, h1, h2, proj, lam, tcode, xsum, bsum, bend, gend, carry, scode, idx, cnt, k, v, v2, total;
 };
 PrefillWs prefill_ws(const Dims& d) {
   PrefillWs w;
@@ -166,6 +172,7 @@ PrefillWs prefill_ws(const Dims& d) {
   w.cnt = o; o += al(T * 4);
   w.k = o; o += al(T * d.dkv * d.elem);
   w.v = o; o += al(T * d.dkv * d.elem);
+  w.v2 = o; o += d.paths == 3 ? al(T * d.dkv * 4) : 0;  // full MKA: the L2 path's value M2 W_v
   w.total = o;
   return w;
 }
@@ -525,6 +532,7 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   PrefillWs W = prefill_ws(d);
   if (ws_bytes < W.total) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, W.total);
   StateLayout SL{};
+  if (state && d.paths == 3) return fail(MKA_ERR_UNSUPPORTED, "full MKA has no decode state");
   if (state) {
     if (max_positions < d.S) return fail(MKA_ERR_CAPACITY, "max_positions %d < seq %d", max_positions, d.S);
     SL = state_layout(d, max_positions);
@@ -647,6 +655,7 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   fa.B = d.B; fa.S = d.S; fa.nblk = d.nblk; fa.blk = d.blk; fa.dkv = d.dkv; fa.alpha = d.alpha;
   fa.k_out = kbuf; fa.v_out = vbuf; fa.kv_bstride = kv_bstride; fa.out_bf16 = d.bf16;
   fa.state_ema = state ? (float*)P(state, SL.ema) : nullptr;
+  if (d.paths == 3) fa.v2_out = (float*)P(ws, W.v2);  // K, V <- the tokens' own; v2 <- M2 W_v
   CUDA_TRY(fuse_kv(fa, s));
   STAGE(s);
   // 6. causal GQA attention over the fused K/V
@@ -657,6 +666,11 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   aa.B = d.B; aa.S = d.S; aa.Hq = d.Hq; aa.Hkv = d.Hkv; aa.dh = d.dh; aa.scale = d.scale;
   if (d.bf16) CUDA_TRY(attention_prefill_tc(aa, status_ptr(), s));
   else CUDA_TRY(attention_prefill(aa, 0, s));
+  if (d.paths == 3) {  // full MKA: the recalled-block path, mixed with the causal one and the L2 value
+    AttnArgs a3 = aa;
+    a3.ridx = idx; a3.rcnt = cnt; a3.R = d.R; a3.blk = d.blk; a3.lam = lam; a3.v2 = (const float*)P(ws, W.v2);
+    CUDA_TRY(attention_prefill_tc(a3, status_ptr(), s));
+  }
   STAGE(s);
   if (ax) {
     CUDA_TRY(cudaStreamWaitEvent(s, ax->join[2], 0));
@@ -676,6 +690,7 @@ int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size
   if (!aligned16(packed) || !aligned16(state) || !aligned16(x_new) || !aligned16(out) || !aligned16(ws))
     return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if (max_positions < 1) return fail(MKA_ERR_INVALID_ARG, "max_positions must be >= 1");
+  if (d.paths == 3) return fail(MKA_ERR_UNSUPPORTED, "full MKA has no decode step");
   if (d.B > 8) return fail(MKA_ERR_UNSUPPORTED, "decode batch must be <= 8");
   if (d.bf16 && d.Hq / d.Hkv > 16) return fail(MKA_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads must be <= 16 for decode");
   StateLayout SL = state_layout(d, max_positions);

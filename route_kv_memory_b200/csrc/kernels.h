@@ -98,6 +98,9 @@ struct FuseArgs {
   float alpha;
   void* k_out; void* v_out; long long kv_bstride; int out_bf16;  // [B][.. rows][dkv]
   float* state_ema;               // [B][width] <- M2[S] (nullable)
+  // Full MKA (three paths) instead of the fused K/V: k_out, v_out <- the tokens' own XW_k, XW_v
+  // and v2_out [B*S][dkv] float32 <- the L2 path's value M2 W_v (its EMA of XW_v); no recall gather.
+  float* v2_out = nullptr;
 };
 cudaError_t fuse_kv(const FuseArgs& a, cudaStream_t s);
 
@@ -118,9 +121,16 @@ struct AttnArgs {
   void* o; long long o_bstride; int o_ld;
   int B, S, Hq, Hkv, dh;
   float scale;
+  // Recalled-block attention of full MKA (set ridx to select it): row t attends to the keys of
+  // its recalled L3 blocks only (ridx [B*S][R], rcnt [B*S]; block length blk, a multiple of 128),
+  // and the output row becomes lam0 * o (the causal pass, read back) + lam1 * v2 + lam2 * that.
+  const int* ridx = nullptr; const int* rcnt = nullptr; int R = 0, blk = 0;
+  const float* lam = nullptr;     // [B*S][3]
+  const float* v2 = nullptr;      // [B*S][Hkv*dh] float32: the L2 path's value M2 W_v
 };
 cudaError_t attention_prefill(const AttnArgs& a, int bf16, cudaStream_t s);
-// bf16 path on tcgen05 (tc_attention.cu): persistent, TMA-fed, S and P in TMEM.
+// bf16 path on tcgen05 (tc_attention.cu): persistent, TMA-fed, S and P in TMEM; causal, or the
+// recalled-block pass of full MKA when a.ridx is set.
 cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode

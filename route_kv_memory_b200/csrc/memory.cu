@@ -492,6 +492,17 @@ __global__ void __launch_bounds__(64 * kRG) fuse_kernel(FuseArgs a) {
   OutT* dst = (OutT*)(is_k ? a.k_out : a.v_out) + (size_t)bi * a.kv_bstride + (size_t)r0 * a.dkv + (is_k ? c : c - a.dkv);
   const float* xp = a.xkv + tg0 * a.ld + c;
   const float invb = 1.f / (float)a.blk;
+  if (a.v2_out) {  // full MKA: raw K/V of the tokens and the L2 value, no fusion
+    float* v2 = is_k ? nullptr : a.v2_out + tg0 * a.dkv + (c - a.dkv);
+    for (int r = ra; r < rb; ++r) {
+      const float4 x = *(const float4*)(xp + (size_t)r * a.ld);
+      store4<OutT>(dst + (size_t)r * a.dkv, x);
+      if (v2) *(float4*)(v2 + (size_t)r * a.dkv) = m2;
+      m2 = ema_step(a.alpha, om, m2, x);
+    }
+    if (r1 == a.S && rb == nr && rb > ra && a.state_ema) *(float4*)(a.state_ema + (size_t)bi * a.width + c) = m2;
+    return;
+  }
   for (int r = ra; r < rb; ++r) {
     float4 x = *(const float4*)(xp + (size_t)r * a.ld);
     int cnt = scnt[r];

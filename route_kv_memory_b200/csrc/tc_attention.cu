@@ -90,7 +90,11 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-template <int DH>
+// RC selects the recalled-block pass of full MKA: tile t of a pair runs only the key tiles
+// before its query block's L3 block (n_t = (qt / m) * m for L3 blocks of m key tiles, possibly
+// 0), a row keeps a key tile only if that tile's block is among the row's recalled blocks, and
+// the epilogue writes lam0 * (causal output already in a.o) + lam1 * v2 + lam2 * this pass.
+template <int DH, bool RC>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, AttnArgs a, int* status) {
@@ -148,6 +152,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int G = a.Hq / a.Hkv;
   const long long q_rows_per_b = a.q_bstride / a.q_ld;
   const long long kv_rows_per_b = a.kv_bstride / a.kv_ld;
+  const int mt = RC ? a.blk / BKV : 1;  // key tiles per L3 block
+  // key tiles query tile qt runs: causal up to its own tile, or the tiles of strictly past L3 blocks
+  auto ntiles = [&](int qt) { return RC ? (qt / mt) * mt : qt + 1; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ loader
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_2d(sQ + t * C::Q_BYTES + hb * C::HALF, &tmQ, &q_full[t], it.h * DH + hb * 64, qy);
         }
         if (!qok) break;
-        const int nkv = 2 * it.pair + 2;
+        const int nkv = ntiles(2 * it.pair + 1);
         bool ok = true;
         for (int j = 0; j < nkv; ++j, ++kvit) {
           const int st = kvit & 1;
@@ -226,15 +233,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (w < 0) break;
         const int wi = rr;  // items this CTA has started before this one
         const Work it = work_item(w, a.B, a.Hq, npairs);
-        const int n0 = 2 * it.pair + 1, n1 = 2 * it.pair + 2;
+        const int n0 = ntiles(2 * it.pair), n1 = ntiles(2 * it.pair + 1);  // n0 <= n1
         if (!mbar_wait(&q_full[0], wi & 1, abort, status)) break;
-        if (!mbar_wait(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
+        if (n1 > 0 && !mbar_wait(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
         tc_fence_after();
-        issue_s(0, kvit & 1);
-        if (n0 == 1) umma_commit(&q_empty[0]);  // Q_0's last use
+        if (n0 > 0) issue_s(0, kvit & 1);
+        if (n0 <= 1) umma_commit(&q_empty[0]);  // Q_0's last use (or none)
+        if (n0 == 0) umma_commit(&o_full[0]);   // no key tile: the epilogue adds nothing from TMEM
         if (!mbar_wait(&q_full[1], wi & 1, abort, status)) break;
         tc_fence_after();
-        issue_s(1, kvit & 1);
+        if (n1 > 0) issue_s(1, kvit & 1);
+        if (n1 <= 1) umma_commit(&q_empty[1]);
+        if (n1 == 0) umma_commit(&o_full[1]);
         for (int j = 0; j < n1; ++j) {
           const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
           bool next_ready = false;
@@ -296,14 +306,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int wi = rr;
       const Work it = work_item(w, a.B, a.Hq, npairs);
       const int qt = 2 * it.pair + t;
-      const int nkv = qt + 1;
+      const int nkv = ntiles(qt);
       const int row = qt * BQ + r;
+      // recalled-block pass: this row's recalled L3 blocks
+      const size_t tok = (size_t)it.b * a.S + (row < a.S ? row : 0);
+      const int my_cnt = (RC && row < a.S) ? a.rcnt[tok] : 0;
+      const int* my_idx = RC ? a.ridx + tok * a.R : nullptr;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv; ++j, ++sit) {
         if (!mbar_wait(&s_full[t], sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
-        const bool diag = (j == nkv - 1);
+        const bool diag = !RC && (j == nkv - 1);
+        bool keep = true;  // RC: this key tile belongs to one of the row's recalled blocks
+        if (RC) {
+          keep = false;
+          for (int q = 0; q < my_cnt; ++q) keep |= (__ldg(my_idx + q) == j / mt);
+        }
         const int lim = row - j * BKV;  // keys c > lim are in the future of this row
         // pass 1: row maximum of the raw scores (four TMEM loads behind one wait; 3-input
         // max); only the diagonal tile needs the causal mask (a warp-uniform branch)
@@ -334,6 +353,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         mx *= sl2;
+        if (RC && !keep) mx = -INFINITY;
         // lazy rescale: move the reference maximum only when it is exceeded by more than 2^8
         const bool need = mx > m_ref + RESCALE_THRESHOLD;
         float corr = 1.f;
@@ -363,6 +383,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (diag) {
               if (c * 32 + 2 * e > lim) p0 = 0.f;
               if (c * 32 + 2 * e + 1 > lim) p1 = 0.f;
+            }
+            if (RC && !keep) {
+              p0 = 0.f;
+              p1 = 0.f;
             }
             lsum2 = __fadd2_rn(lsum2, make_float2(p0, p1));
             __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
@@ -403,8 +427,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // epilogue: O_t / l -> bf16 -> global
       if (!mbar_wait(&o_full[t], wi & 1, abort, status)) break;
       tc_fence_after();
-      const float inv = 1.f / l;
+      // RC: a row with no kept key (l == 0) adds nothing, and TMEM may then hold a stale tile
+      const bool has_o = !RC || l > 0.f;
+      const float inv = has_o ? 1.f / l : 0.f;
       bf16* orow = (bf16*)a.o + (size_t)it.b * a.o_bstride + (size_t)row * a.o_ld + (size_t)it.h * DH;
+      float lam0 = 1.f, lam1 = 0.f, lam2 = 0.f;
+      const float* v2row = nullptr;
+      if (RC && row < a.S) {
+        lam0 = a.lam[tok * 3];
+        lam1 = a.lam[tok * 3 + 1];
+        lam2 = a.lam[tok * 3 + 2];
+        v2row = a.v2 + tok * (size_t)(a.Hkv * DH) + (size_t)(it.h / G) * DH;
+      }
 #pragma unroll
       for (int c = 0; c < DH; c += 32) {
         uint32_t ov[32];
@@ -415,11 +449,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int v = 0; v < 4; ++v) {
             uint4 u;
             uint32_t* wv = (uint32_t*)&u;
+            if (RC) {  // lam0 * causal output (in a.o) + lam1 * v2 + lam2 * recalled-block output
+              const uint4 o1 = *(const uint4*)(orow + c + v * 8);
+              const uint32_t* o1w = (const uint32_t*)&o1;
+              const float4 va = *(const float4*)(v2row + c + v * 8), vb = *(const float4*)(v2row + c + v * 8 + 4);
+              const float v2e[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(ov[v * 8 + 2 * e]) * inv,
-                                                        __uint_as_float(ov[v * 8 + 2 * e + 1]) * inv);
-              wv[e] = *(uint32_t*)&hb;
+              for (int e = 0; e < 4; ++e) {
+                const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&o1w[e]);
+                const float x0 = has_o ? __uint_as_float(ov[v * 8 + 2 * e]) * inv : 0.f;
+                const float x1 = has_o ? __uint_as_float(ov[v * 8 + 2 * e + 1]) * inv : 0.f;
+                __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(lam0, f1.x, fmaf(lam1, v2e[2 * e], lam2 * x0)),
+                                                          fmaf(lam0, f1.y, fmaf(lam1, v2e[2 * e + 1], lam2 * x1)));
+                wv[e] = *(uint32_t*)&hb;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(ov[v * 8 + 2 * e]) * inv,
+                                                          __uint_as_float(ov[v * 8 + 2 * e + 1]) * inv);
+                wv[e] = *(uint32_t*)&hb;
+              }
             }
             *(uint4*)(orow + c + v * 8) = u;
           }
@@ -463,14 +513,28 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
   const int nqt = (a.S + tca::BQ - 1) / tca::BQ;
   const int nwork = a.B * a.Hq * ((nqt + 1) / 2);
   const int grid = nwork < sms ? nwork : sms;
+  if (a.ridx && (!a.rcnt || !a.lam || !a.v2 || a.R < 1 || a.blk < tca::BKV || a.blk % tca::BKV))
+    return cudaErrorInvalidValue;
   if (a.dh == 128) {
-    e = set_max_smem(tca::attn_tc_kernel<128>, tca::Cfg<128>::SMEM, s);
-    if (e != cudaSuccess) return e;
-    tca::attn_tc_kernel<128><<<grid, tca::NTHREADS, tca::Cfg<128>::SMEM, s>>>(tq, tk, tv, a, status);
+    if (a.ridx) {
+      e = set_max_smem(tca::attn_tc_kernel<128, true>, tca::Cfg<128>::SMEM, s);
+      if (e != cudaSuccess) return e;
+      tca::attn_tc_kernel<128, true><<<grid, tca::NTHREADS, tca::Cfg<128>::SMEM, s>>>(tq, tk, tv, a, status);
+    } else {
+      e = set_max_smem(tca::attn_tc_kernel<128, false>, tca::Cfg<128>::SMEM, s);
+      if (e != cudaSuccess) return e;
+      tca::attn_tc_kernel<128, false><<<grid, tca::NTHREADS, tca::Cfg<128>::SMEM, s>>>(tq, tk, tv, a, status);
+    }
   } else {
-    e = set_max_smem(tca::attn_tc_kernel<64>, tca::Cfg<64>::SMEM, s);
-    if (e != cudaSuccess) return e;
-    tca::attn_tc_kernel<64><<<grid, tca::NTHREADS, tca::Cfg<64>::SMEM, s>>>(tq, tk, tv, a, status);
+    if (a.ridx) {
+      e = set_max_smem(tca::attn_tc_kernel<64, true>, tca::Cfg<64>::SMEM, s);
+      if (e != cudaSuccess) return e;
+      tca::attn_tc_kernel<64, true><<<grid, tca::NTHREADS, tca::Cfg<64>::SMEM, s>>>(tq, tk, tv, a, status);
+    } else {
+      e = set_max_smem(tca::attn_tc_kernel<64, false>, tca::Cfg<64>::SMEM, s);
+      if (e != cudaSuccess) return e;
+      tca::attn_tc_kernel<64, false><<<grid, tca::NTHREADS, tca::Cfg<64>::SMEM, s>>>(tq, tk, tv, a, status);
+    }
   }
   return cudaGetLastError();
 }

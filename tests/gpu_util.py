@@ -29,6 +29,8 @@ def oracle_weights(inp: FastMKAInputs):
 def oracle_prefill(cfg: FastMKAConfig, inp: FastMKAInputs, rows=None, seq=None):
     S = cfg.seq if seq is None else seq
     X = inp.x[:, :S].float().numpy()
+    if getattr(cfg, "attention_paths", 1) == 3:
+        return oracle.mka_full_prefill(X, oracle_weights(inp), cfg.replace(seq=S), rows=rows)
     return oracle.fastmka_prefill(X, oracle_weights(inp), cfg.replace(seq=S), rows=rows)
 
 

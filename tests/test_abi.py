@@ -73,6 +73,7 @@ def test_sizes(mka):
 @pytest.mark.parametrize("field,value", [
     ("d_head", 96), ("n_kv_heads", 5), ("hash_bits", 33), ("recall_r", 0), ("router_hidden", 12), ("d_model", 100),
     ("dtype", 7), ("block_size", 0), ("batch", 0), ("route_mode", 4), ("route_mode", -1), ("tiers", 8),
+    ("attention_paths", 2), ("attention_paths", 4),
 ])
 def test_bad_configs_size_zero(mka, field, value):
     c = qwen_cfg(mka, **{field: value})
@@ -84,11 +85,18 @@ def test_routing_fields_follow_attn_scale(mka):
     """The routing fields were appended to mka_config; the earlier fields keep their offsets, and a
     zero-initialised tiers field selects all three tiers (the published layer)."""
     fields = [f[0] for f in mka.mka_config._fields_]
-    assert fields[-3:] == ["attn_scale", "route_mode", "tiers"]
-    assert ctypes.sizeof(mka.mka_config) == 15 * 4
+    assert fields[-4:] == ["attn_scale", "route_mode", "tiers", "attention_paths"]
+    assert ctypes.sizeof(mka.mka_config) == 16 * 4
     for mode in range(4):
         for tiers in range(8):
             assert mka.mka_workspace_size(qwen_cfg(mka, route_mode=mode, tiers=tiers)) > 0
+
+
+def test_full_mka_limits(mka):
+    """Three attention paths: bf16 prefill with block_size % 128 == 0; no decode state."""
+    assert mka.mka_workspace_size(qwen_cfg(mka, attention_paths=3)) > mka.mka_workspace_size(qwen_cfg(mka))
+    assert mka.mka_workspace_size(qwen_cfg(mka, attention_paths=3, block_size=64)) == 0
+    assert mka.mka_workspace_size(qwen_cfg(mka, attention_paths=3, dtype=mka.MKA_F32)) == 0
 
 
 def test_host_side_errors_before_any_device_call(mka):

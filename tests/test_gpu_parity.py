@@ -152,6 +152,53 @@ def test_routing_variants_decode(mode, tiers):
     check_out(got, ref["O"], "bf16")
 
 
+# ------------------------------------------------------------------ full MKA (three attention paths)
+MKA_CASES = [
+    small("mka_b128", "bf16", seq=600, d_head=128, n_q_heads=8, n_kv_heads=2, router_hidden=128, block=128,
+          recall_r=2, hash_bits=32, seed=71, attention_paths=3),
+    small("mka_b256_pairs", "bf16", batch=2, seq=900, d_head=128, n_q_heads=4, n_kv_heads=1, block=256, recall_r=3,
+          hash_bits=32, seed=72, attention_paths=3),
+    small("mka_ragged_all_recalled", "bf16", seq=333, d_head=128, block=128, recall_r=8, seed=73, attention_paths=3),
+    small("mka_dh64", "bf16", seq=520, d_head=64, n_q_heads=6, n_kv_heads=2, block=128, recall_r=3, seed=74,
+          attention_paths=3),
+    small("mka_no_l3", "bf16", seq=400, d_head=128, block=128, recall_r=2, seed=75, attention_paths=3, tiers=3),
+]
+
+
+@pytest.mark.parametrize("cfg", MKA_CASES, ids=[c.name for c in MKA_CASES])
+def test_full_mka_layer(cfg):
+    inp = make_inputs(cfg)
+    ref = oracle_prefill(cfg, inp)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    if cfg.tiers & 4:
+        check_recall(idx, ref)
+    check_out(out, ref["O"], "bf16")
+
+
+def test_full_mka_top2_routing():
+    cfg, inp = margin_safe_inputs(small("mka_top2", "bf16", seq=500, d_head=128, n_q_heads=8, n_kv_heads=2,
+                                        router_hidden=128, block=128, recall_r=2, hash_bits=32,
+                                        route_mode="top2", attention_paths=3))
+    ref = oracle_prefill(cfg, inp)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    check_out(out, ref["O"], "bf16")
+
+
+def test_full_mka_qwen7b_4k_rows():
+    """Full MKA at the Qwen 2 x 4096 layer shape: lambda and recall on every row, O on a row sample."""
+    cfg = CONFIGS["qwen7b_4k"].replace(attention_paths=3)
+    inp = make_inputs(cfg)
+    rows = sample_rows(cfg.seq, cfg.block, max_rows=48)
+    ref = oracle_prefill(cfg, inp, rows=rows)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    check_recall(idx, ref)
+    max_abs, rel = check_out(out, ref["O"], "bf16", rows=rows)
+    print(f"full MKA qwen7b_4k: O rel-L2 {rel:.2e} max-abs {max_abs:.2e}")
+
+
 # ------------------------------------------------------------------ entry points one by one
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_router_entry(mka, dtype):
