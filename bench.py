@@ -107,10 +107,13 @@ class ClockSampler:
 def prefill_flops(cfg) -> dict:
     T, d, dq, dkv, rh, nb = cfg.tokens, cfg.d_model, cfg.dq, cfg.dkv, cfg.router_hidden, cfg.hash_bits
     causal_pairs = cfg.batch * cfg.seq * (cfg.seq + 1) / 2
-    return {
-        "projections": 2.0 * T * d * (dq + 2 * dkv + 2 * rh + nb),
-        "attention": 4.0 * cfg.d_head * cfg.n_q_heads * causal_pairs,  # QK^T and PV over j <= t only
-    }
+    attn = 4.0 * cfg.d_head * cfg.n_q_heads * causal_pairs  # QK^T and PV over j <= t only
+    if getattr(cfg, "attention_paths", 1) == 3 and cfg.tiers & 4:
+        # full MKA's recalled-block path: row t attends to min(R, t // b) blocks of b keys
+        t = np.arange(cfg.seq)
+        keys = np.minimum(cfg.recall_r, t // cfg.block) * cfg.block
+        attn += 4.0 * cfg.d_head * cfg.n_q_heads * cfg.batch * float(keys.sum())
+    return {"projections": 2.0 * T * d * (dq + 2 * dkv + 2 * rh + nb), "attention": attn}
 
 
 def decode_bytes_per_token(cfg, ctx: int, ntot: int) -> float:
@@ -122,7 +125,8 @@ def decode_bytes_per_token(cfg, ctx: int, ntot: int) -> float:
 
 def workload_cfg(args, name):
     """The named workload with the routing gate / memory tiers the command line selects."""
-    return CONFIGS[name].replace(route_mode=args.route, tiers=args.tiers)
+    return CONFIGS[name].replace(route_mode=args.route, tiers=args.tiers,
+                                 attention_paths=getattr(args, "paths", 1))
 
 
 def model_name(cfg) -> str:
@@ -190,7 +194,8 @@ def run_ours(args, rank, world, local_rank):
     fl = prefill_flops(cfg)
     attn_ms = float(stages[8])
     attn_tflops = fl["attention"] / (attn_ms / 1e3) / 1e12
-    roofline = {"kernel": "attention (causal GQA, online max-shift)", "bound": "tensor",
+    roofline = {"kernel": "attention (causal GQA, online max-shift)" if cfg.attention_paths == 1 else
+                "attention (full MKA: causal pass + recalled-block pass)", "bound": "tensor",
                 "achieved": round(attn_tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
                 "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)",
@@ -258,7 +263,8 @@ def run_ours(args, rank, world, local_rank):
                                f"{cfg.d_head}, router {cfg.dq}->{cfg.router_hidden}->3, alpha {cfg.alpha}, L3 block "
                                f"{cfg.block}, R {cfg.recall_r}, nbits {cfg.hash_bits}, seed {cfg.seed}"
                                + ("" if (cfg.route_mode, cfg.tiers) == ("soft", 7) else
-                                  f"; routing {cfg.route_mode}, tiers mask {cfg.tiers}"),
+                                  f"; routing {cfg.route_mode}, tiers mask {cfg.tiers}")
+                               + ("; full MKA, three attention paths" if cfg.attention_paths == 3 else ""),
                    "global_batch": cfg.batch * world, "seq_len": cfg.seq,
                    "parallelism": f"replicas x{world} (independent sequences, no exchange)",
                    "l2": "flushed (512 MB write) before every timed step"},
@@ -270,7 +276,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
     }
     del flush
-    if world == 1 and not args.no_decode:
+    if world == 1 and not args.no_decode and args.paths == 1:  # full MKA has no decode step
         result["decode"] = run_decode(args, cfg, inp, weights, dev, layer_pack=None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, inp, budget_rows=args.cpu_rows)
@@ -440,6 +446,8 @@ def main():
     ap.add_argument("--route", default="soft", choices=["soft", "fixed", "top1", "top2"],
                     help="routing gate variant (the published layer is soft)")
     ap.add_argument("--tiers", type=int, default=7, help="memory tier mask: 1 L1, 2 L2, 4 L3 (7 = all)")
+    ap.add_argument("--paths", type=int, default=1, choices=[1, 3],
+                    help="1: FastMKA (the layer measured); 3: full MKA, three attention paths (prefill only)")
     ap.add_argument("--decode-ctx", type=int, nargs="*", default=[131072])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode measurement (no prefill line)")

@@ -98,8 +98,8 @@ typedef struct mka_config {
                               3: full MKA, three attention outputs mixed by the gate (notes §2):
                               causal over the tokens, the L2 summary value, attention over the
                               recalled L3 blocks' tokens.  3 is implemented for bf16 prefill with
-                              block_size a multiple of 128 and no decode state; otherwise
-                              MKA_ERR_UNSUPPORTED */
+                              block_size a multiple of 128, recall_r <= 16 and no decode state;
+                              otherwise MKA_ERR_UNSUPPORTED */
 } mka_config;
 
 /* Raw layer weights, all in cfg->dtype, all [d_in, d_out] row-major. */

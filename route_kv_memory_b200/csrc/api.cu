@@ -88,8 +88,8 @@ int check_cfg(const mka_config* c, Dims* o) {
     return fail(MKA_ERR_INVALID_ARG, "tiers must be a mask of MKA_TIER_L1 | MKA_TIER_L2 | MKA_TIER_L3");
   if (c->attention_paths != 0 && c->attention_paths != 1 && c->attention_paths != 3)
     return fail(MKA_ERR_INVALID_ARG, "attention_paths must be 1 (FastMKA) or 3 (full MKA)");
-  if (c->attention_paths == 3 && (c->dtype != MKA_BF16 || c->block_size % 128))
-    return fail(MKA_ERR_UNSUPPORTED, "full MKA needs bf16 and a block_size that is a multiple of 128");
+  if (c->attention_paths == 3 && (c->dtype != MKA_BF16 || c->block_size % 128 || c->recall_r > 16))
+    return fail(MKA_ERR_UNSUPPORTED, "full MKA needs bf16, a block_size that is a multiple of 128 and recall_r <= 16");
   long long T = (long long)c->batch * c->seq;
   if (T > (1LL << 30)) return fail(MKA_ERR_UNSUPPORTED, "batch * seq too large");
   if ((c->seq + c->block_size - 1) / c->block_size > 65535) return fail(MKA_ERR_UNSUPPORTED, "seq / block_size > 65535");

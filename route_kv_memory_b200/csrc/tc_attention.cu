@@ -43,7 +43,10 @@ struct Cfg {
   static constexpr int KV_BYTES = 2 * K_BYTES;   // K then V
   static constexpr int HALF = 128 * 64 * 2;      // one 128-row x 64-column swizzled box
   static constexpr int SMEM = 2 * Q_BYTES + 2 * KV_BYTES + 1024 + 256;
+  // recalled-block pass: each softmax row's recalled block indices, staged per item
+  static constexpr int REC_BYTES = 2 * BQ * 16 * 4;
 };
+constexpr int MAX_RECALL_RC = 16;  // recall_r the recalled-block pass stages in shared memory
 
 struct Work {
   int b, h, pair;
@@ -118,6 +121,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* o_empty = bars + 16;  // [2]
   uint64_t* drain = bars + 18;
   uint32_t* tmem_slot = (uint32_t*)(bars + 19);
+  int* srec = (int*)(smem + 2 * C::Q_BYTES + 2 * C::KV_BYTES + 256);  // RC only: [2][BQ][MAX_RECALL_RC]
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -239,12 +243,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         if (n0 > 0) issue_s(0, kvit & 1);
         if (n0 <= 1) umma_commit(&q_empty[0]);  // Q_0's last use (or none)
-        if (n0 == 0) umma_commit(&o_full[0]);   // no key tile: the epilogue adds nothing from TMEM
+        // No key tile: the epilogue adds nothing from TMEM, but o_full still moves one phase per
+        // item, and only after the previous item's epilogue released O_t: without that wait two
+        // items in a row could commit two phases before the softmax warps wait for the first,
+        // which then reads as the wrong parity and never completes.
+        if (n0 == 0) {
+          if (!mbar_wait(&o_empty[0], (wi & 1) ^ 1, abort, status)) break;
+          umma_commit(&o_full[0]);
+        }
         if (!mbar_wait(&q_full[1], wi & 1, abort, status)) break;
         tc_fence_after();
         if (n1 > 0) issue_s(1, kvit & 1);
         if (n1 <= 1) umma_commit(&q_empty[1]);
-        if (n1 == 0) umma_commit(&o_full[1]);
+        if (n1 == 0) {
+          if (!mbar_wait(&o_empty[1], (wi & 1) ^ 1, abort, status)) break;
+          umma_commit(&o_full[1]);
+        }
         for (int j = 0; j < n1; ++j) {
           const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
           bool next_ready = false;
@@ -309,9 +323,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int nkv = ntiles(qt);
       const int row = qt * BQ + r;
       // recalled-block pass: this row's recalled L3 blocks
-      const size_t tok = (size_t)it.b * a.S + (row < a.S ? row : 0);
-      const int my_cnt = (RC && row < a.S) ? a.rcnt[tok] : 0;
-      const int* my_idx = RC ? a.ridx + tok * a.R : nullptr;
+      int my_cnt = 0;
+      if (RC) {  // stage this row's recalled blocks in shared memory (keeps them out of registers)
+        const size_t tok = (size_t)it.b * a.S + row;
+        my_cnt = row < a.S ? a.rcnt[tok] : 0;
+        for (int q = 0; q < my_cnt; ++q) srec[(t * BQ + r) * MAX_RECALL_RC + q] = a.ridx[tok * a.R + q];
+        if (row < a.S) {  // the epilogue's inputs (causal output, L2 value) into L2 while the tiles run
+          const char* o1 = (const char*)((const bf16*)a.o + (size_t)it.b * a.o_bstride + (size_t)row * a.o_ld +
+                                         (size_t)it.h * DH);
+          const char* v2 = (const char*)(a.v2 + tok * (size_t)(a.Hkv * DH) + (size_t)(it.h / G) * DH);
+#pragma unroll
+          for (int k = 0; k < DH * 2; k += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(o1 + k));
+#pragma unroll
+          for (int k = 0; k < DH * 4; k += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(v2 + k));
+        }
+      }
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv; ++j, ++sit) {
@@ -321,7 +347,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool keep = true;  // RC: this key tile belongs to one of the row's recalled blocks
         if (RC) {
           keep = false;
-          for (int q = 0; q < my_cnt; ++q) keep |= (__ldg(my_idx + q) == j / mt);
+          const int* rec = srec + (t * BQ + r) * MAX_RECALL_RC;
+          for (int q = 0; q < my_cnt; ++q) keep |= (rec[q] == j / mt);
         }
         const int lim = row - j * BKV;  // keys c > lim are in the future of this row
         // pass 1: row maximum of the raw scores (four TMEM loads behind one wait; 3-input
@@ -357,8 +384,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // lazy rescale: move the reference maximum only when it is exceeded by more than 2^8
         const bool need = mx > m_ref + RESCALE_THRESHOLD;
         float corr = 1.f;
+        bool rescale = false;  // O and l hold earlier tiles only once a key has been kept
         if (need) {
-          corr = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
+          rescale = m_ref != -INFINITY;
+          corr = rescale ? ex2(m_ref - mx) : 0.f;
           m_ref = mx;
           l *= corr;
         }
@@ -399,7 +428,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // rescale the O rows (rare with the lazy threshold).  S_j landing means PV_{j-1},
         // issued before QK_j, has completed, so the wait below returns at once.  PV_j is
         // issued only after p_full, so it accumulates onto the rescaled rows.
-        if (__ballot_sync(0xffffffffu, need && j > 0)) {
+        if (__ballot_sync(0xffffffffu, rescale)) {
           if (!mbar_wait(&pv_done[t], (sit - 1) & 1, abort, status)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -434,6 +463,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float lam0 = 1.f, lam1 = 0.f, lam2 = 0.f;
       const float* v2row = nullptr;
       if (RC && row < a.S) {
+        const size_t tok = (size_t)it.b * a.S + row;
         lam0 = a.lam[tok * 3];
         lam1 = a.lam[tok * 3 + 1];
         lam2 = a.lam[tok * 3 + 2];
@@ -445,33 +475,51 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld32(o_tmem + c, ov);
         tmem_ld_wait();
         if (row < a.S) {
+          if (RC) {
+            // lam0 * causal output + lam1 * L2 value + lam2 * recalled-block output, 16 columns at a
+            // time with that half's loads issued together (the stores would otherwise order them)
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 u;
-            uint32_t* wv = (uint32_t*)&u;
-            if (RC) {  // lam0 * causal output (in a.o) + lam1 * v2 + lam2 * recalled-block output
-              const uint4 o1 = *(const uint4*)(orow + c + v * 8);
-              const uint32_t* o1w = (const uint32_t*)&o1;
-              const float4 va = *(const float4*)(v2row + c + v * 8), vb = *(const float4*)(v2row + c + v * 8 + 4);
-              const float v2e[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+            for (int hh = 0; hh < 2; ++hh) {
+              const int c0 = c + hh * 16;
+              uint4 o1[2];
+              float4 v2c[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&o1w[e]);
-                const float x0 = has_o ? __uint_as_float(ov[v * 8 + 2 * e]) * inv : 0.f;
-                const float x1 = has_o ? __uint_as_float(ov[v * 8 + 2 * e + 1]) * inv : 0.f;
-                __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(lam0, f1.x, fmaf(lam1, v2e[2 * e], lam2 * x0)),
-                                                          fmaf(lam0, f1.y, fmaf(lam1, v2e[2 * e + 1], lam2 * x1)));
-                wv[e] = *(uint32_t*)&hb;
+              for (int v = 0; v < 2; ++v) o1[v] = *(const uint4*)(orow + c0 + v * 8);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) v2c[v] = *(const float4*)(v2row + c0 + v * 4);
+#pragma unroll
+              for (int v = 0; v < 2; ++v) {
+                uint4 u;
+                uint32_t* wv = (uint32_t*)&u;
+                const uint32_t* o1w = (const uint32_t*)&o1[v];
+                const float v2e[8] = {v2c[2 * v].x, v2c[2 * v].y, v2c[2 * v].z, v2c[2 * v].w,
+                                      v2c[2 * v + 1].x, v2c[2 * v + 1].y, v2c[2 * v + 1].z, v2c[2 * v + 1].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int k = hh * 16 + v * 8 + 2 * e;
+                  const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&o1w[e]);
+                  const float x0 = has_o ? __uint_as_float(ov[k]) * inv : 0.f;
+                  const float x1 = has_o ? __uint_as_float(ov[k + 1]) * inv : 0.f;
+                  __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(lam0, f1.x, fmaf(lam1, v2e[2 * e], lam2 * x0)),
+                                                            fmaf(lam0, f1.y, fmaf(lam1, v2e[2 * e + 1], lam2 * x1)));
+                  wv[e] = *(uint32_t*)&hb;
+                }
+                *(uint4*)(orow + c0 + v * 8) = u;
               }
-            } else {
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 u;
+              uint32_t* wv = (uint32_t*)&u;
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(ov[v * 8 + 2 * e]) * inv,
                                                           __uint_as_float(ov[v * 8 + 2 * e + 1]) * inv);
                 wv[e] = *(uint32_t*)&hb;
               }
+              *(uint4*)(orow + c + v * 8) = u;
             }
-            *(uint4*)(orow + c + v * 8) = u;
           }
         }
       }
@@ -513,13 +561,15 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
   const int nqt = (a.S + tca::BQ - 1) / tca::BQ;
   const int nwork = a.B * a.Hq * ((nqt + 1) / 2);
   const int grid = nwork < sms ? nwork : sms;
-  if (a.ridx && (!a.rcnt || !a.lam || !a.v2 || a.R < 1 || a.blk < tca::BKV || a.blk % tca::BKV))
+  if (a.ridx && (!a.rcnt || !a.lam || !a.v2 || a.R < 1 || a.R > tca::MAX_RECALL_RC || a.blk < tca::BKV ||
+                 a.blk % tca::BKV))
     return cudaErrorInvalidValue;
   if (a.dh == 128) {
     if (a.ridx) {
-      e = set_max_smem(tca::attn_tc_kernel<128, true>, tca::Cfg<128>::SMEM, s);
+      constexpr int sm = tca::Cfg<128>::SMEM + tca::Cfg<128>::REC_BYTES;
+      e = set_max_smem(tca::attn_tc_kernel<128, true>, sm, s);
       if (e != cudaSuccess) return e;
-      tca::attn_tc_kernel<128, true><<<grid, tca::NTHREADS, tca::Cfg<128>::SMEM, s>>>(tq, tk, tv, a, status);
+      tca::attn_tc_kernel<128, true><<<grid, tca::NTHREADS, sm, s>>>(tq, tk, tv, a, status);
     } else {
       e = set_max_smem(tca::attn_tc_kernel<128, false>, tca::Cfg<128>::SMEM, s);
       if (e != cudaSuccess) return e;
@@ -527,9 +577,10 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
     }
   } else {
     if (a.ridx) {
-      e = set_max_smem(tca::attn_tc_kernel<64, true>, tca::Cfg<64>::SMEM, s);
+      constexpr int sm = tca::Cfg<64>::SMEM + tca::Cfg<64>::REC_BYTES;
+      e = set_max_smem(tca::attn_tc_kernel<64, true>, sm, s);
       if (e != cudaSuccess) return e;
-      tca::attn_tc_kernel<64, true><<<grid, tca::NTHREADS, tca::Cfg<64>::SMEM, s>>>(tq, tk, tv, a, status);
+      tca::attn_tc_kernel<64, true><<<grid, tca::NTHREADS, sm, s>>>(tq, tk, tv, a, status);
     } else {
       e = set_max_smem(tca::attn_tc_kernel<64, false>, tca::Cfg<64>::SMEM, s);
       if (e != cudaSuccess) return e;
