@@ -4,7 +4,8 @@
 // X (W_q W_r1), and the L3 projection X P all share the A operand X, so they run
 // as one GEMM over the packed weight matrix).
 //
-// Persistent kernel, one CTA per SM, 192 threads:
+// Persistent kernel, one CTA per SM, 192 threads (the CTA-pair variant below is the one
+// launched; this single-CTA form is the fallback where 2-CTA clusters cannot be placed):
 //   warp 0      TMA producer: A and B tiles (128x64 and 256x64, 128-B swizzle)
 //               into a 4-stage shared-memory ring
 //   warp 1      MMA issuer: 4 x tcgen05.mma (128x256x16) per stage into one of
@@ -91,6 +92,42 @@ __device__ __forceinline__ void store_chunk(const Epilogue& ep, int m, int n, co
 #pragma unroll
   for (int i = 0; i < 32; ++i)
     if (n + i < N) store1(ep, m, n + i, __uint_as_float(r[i]));
+}
+
+// One thread's output row of a finished 128 x 256 accumulator tile (TMEM row `trow`):
+// either the router's hidden units (hi in columns [0,128), lo in [128,256)) reduced
+// through GELU . W_r2 to 3 partials, or the columns stored per output segment.
+__device__ __forceinline__ void epilogue_tile(const Epilogue& ep, uint32_t trow, int m, int n0, int M, int N) {
+  if (n0 >= ep.r_begin && n0 < ep.r_end) {
+    // router tile: hidden units u0 .. u0+127, hi in columns [0,128), lo in [128,256)
+    const int rt = (n0 - ep.r_begin) / BN;
+    const int u0 = rt * 128;
+    float z0 = 0.f, z1 = 0.f, z2 = 0.f;
+    for (int c = 0; c < 128; c += 32) {
+      uint32_t hi[32], lo[32];
+      tmem_ld32(trow + c, hi);
+      tmem_ld32(trow + 128 + c, lo);
+      tmem_ld_wait();
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        const float h = __uint_as_float(hi[i]) + __uint_as_float(lo[i]);
+        const float g = gelu_erf(h);
+        const float* w = ep.w_r2 + (size_t)(u0 + c + i) * 3;
+        z0 = fmaf(g, w[0], z0);
+        z1 = fmaf(g, w[1], z1);
+        z2 = fmaf(g, w[2], z2);
+      }
+    }
+    if (m < M) *(float4*)(ep.zpart + ((size_t)rt * M + m) * 4) = make_float4(z0, z1, z2, 0.f);
+  } else {
+    for (int c = 0; c < BN; c += 32) {
+      if (n0 + c >= N) break;
+      uint32_t r[32];
+      tmem_ld32(trow + c, r);
+      tmem_ld_wait();
+      if (m < M) store_chunk(ep, m, n0 + c, r, N);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -206,36 +243,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
       const int m = m0 + q * 32 + lane;
       const uint32_t trow = tbase + ((uint32_t)(q * 32) << 16) + acc * BN;
-      if (n0 >= ep.r_begin && n0 < ep.r_end) {
-        // router tile: hidden units u0 .. u0+127, hi in columns [0,128), lo in [128,256)
-        const int rt = (n0 - ep.r_begin) / BN;
-        const int u0 = rt * 128;
-        float z0 = 0.f, z1 = 0.f, z2 = 0.f;
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t hi[32], lo[32];
-          tmem_ld32(trow + c, hi);
-          tmem_ld32(trow + 128 + c, lo);
-          tmem_ld_wait();
-#pragma unroll 8
-          for (int i = 0; i < 32; ++i) {
-            const float h = __uint_as_float(hi[i]) + __uint_as_float(lo[i]);
-            const float g = gelu_erf(h);
-            const float* w = ep.w_r2 + (size_t)(u0 + c + i) * 3;
-            z0 = fmaf(g, w[0], z0);
-            z1 = fmaf(g, w[1], z1);
-            z2 = fmaf(g, w[2], z2);
-          }
-        }
-        if (m < M) *(float4*)(ep.zpart + ((size_t)rt * M + m) * 4) = make_float4(z0, z1, z2, 0.f);
-      } else {
-        for (int c = 0; c < BN; c += 32) {
-          if (n0 + c >= N) break;
-          uint32_t r[32];
-          tmem_ld32(trow + c, r);
-          tmem_ld_wait();
-          if (m < M) store_chunk(ep, m, n0 + c, r, N);
-        }
-      }
+      epilogue_tile(ep, trow, m, n0, M, N);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -246,6 +254,148 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- CTA-pair variant
+// Same GEMM on 256 x 256 output tiles computed by a pair of CTAs (a cluster of 2) with
+// tcgen05.mma.cta_group::2: each CTA stages its own 128 rows of A and 128 of the tile's 256
+// rows of B (32 KB per k-block instead of 48 KB), so the operand stream per SM is two thirds
+// of the single-CTA kernel's and six stages fit.  Rank 0 sets the transaction count of both
+// CTAs' loads on its full barrier and issues the MMAs; their commits release both CTAs'
+// stages and accumulators (multicast); both CTAs' epilogue warps release rank 0's
+// accumulator barrier.  Each CTA's TMEM holds its 128 output rows x 256 columns.
+constexpr int PAIR_BM = 256, HALF_ROWS = 128, PAIR_STAGES = 6;
+constexpr int PAIR_STAGE_BYTES = 2 * HALF_ROWS * BK * 2;  // A rows + B rows of this CTA
+constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * PAIR_STAGE_BYTES + 1024 + 256;
+constexpr uint32_t PAIR_IDESC = idesc_bf16_f32(PAIR_BM, BN);
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                    int K, Epilogue ep, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + PAIR_STAGES * PAIR_STAGE_BYTES);  // rank 0's copy is used
+  uint64_t* empty = full + PAIR_STAGES;
+  uint64_t* tfull = empty + PAIR_STAGES;
+  uint64_t* tempty = tfull + 2;  // rank 0's copy is used
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  volatile int* abort = (volatile int*)(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(&full[s], 1);   // rank 0's expect_tx arrival; both CTAs' bytes
+      mbar_init(&empty[s], 1);  // the pair's MMA commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc2(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised and TMEM allocated before any use
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  const int nM = (M + PAIR_BM - 1) / PAIR_BM, nN = (N + BN - 1) / BN, ntiles = nM * nN;
+  const int kblocks = (K + BK - 1) / BK;
+  const int pair = (int)cluster_id_x(), npairs = (int)cluster_count_x();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int it = 0;
+      for (int tile = pair; tile < ntiles; tile += npairs) {
+        const int ma = (tile / nN) * PAIR_BM + (int)rank * HALF_ROWS;  // this CTA's A rows
+        const int nb = (tile % nN) * BN + (int)rank * HALF_ROWS;       // this CTA's B rows
+        for (int k = 0; k < kblocks; ++k, ++it) {
+          const int s = it % PAIR_STAGES;
+          const uint32_t ph = (it / PAIR_STAGES) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1, abort, status)) goto producer_done;
+          uint8_t* st = smem + s * PAIR_STAGE_BYTES;
+          if (rank == 0) mbar_expect_tx(&full[s], 2 * PAIR_STAGE_BYTES);
+          tma_load_2d_pair(st, &tmA, &full[s], k * BK, ma);
+          tma_load_2d_pair(st + HALF_ROWS * BK * 2, &tmB, &full[s], k * BK, nb);
+        }
+      }
+    producer_done:
+      // Wait (bounded) until the pair's MMAs have released every stage this CTA filled: rank 0
+      // reads this CTA's shared memory until then.
+      for (int s = 0; s < PAIR_STAGES; ++s) {
+        if (it - 1 < s) continue;
+        const int last = s + ((it - 1 - s) / PAIR_STAGES) * PAIR_STAGES;
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(&empty[s], (last / PAIR_STAGES) & 1) && globaltimer() - t0 < 200000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      int it = 0, tl = 0;
+      for (int tile = pair; tile < ntiles; tile += npairs, ++tl) {
+        const int acc = tl & 1;
+        const uint32_t aph = (tl >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1, abort, status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tbase + acc * BN;
+        bool ok = true;
+        for (int k = 0; k < kblocks; ++k, ++it) {
+          const int s = it % PAIR_STAGES;
+          const uint32_t ph = (it / PAIR_STAGES) & 1;
+          if (!mbar_wait(&full[s], ph, abort, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* st = smem + s * PAIR_STAGE_BYTES;
+          const uint64_t a_desc = sdesc_kmajor_sw128(st);
+          const uint64_t b_desc = sdesc_kmajor_sw128(st + HALF_ROWS * BK * 2);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma2_bf16_ss(d_tmem, a_desc + (uint64_t)(kk * 2), b_desc + (uint64_t)(kk * 2), PAIR_IDESC,
+                          (k | kk) != 0);
+          umma2_commit_mc(&empty[s], 0x3);
+        }
+        if (!ok) break;
+        umma2_commit_mc(&tfull[acc], 0x3);
+      }
+      if (*abort) {  // let the MMAs already issued finish before the TMEM is released
+        umma2_commit_mc(drain, 0x1);
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    int tl = 0;
+    for (int tile = pair; tile < ntiles; tile += npairs, ++tl) {
+      const int acc = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], aph, abort, status)) break;
+      tc_fence_after();
+      const int n0 = (tile % nN) * BN;
+      const int m = (tile / nN) * PAIR_BM + (int)rank * HALF_ROWS + q * 32 + lane;
+      const uint32_t trow = tbase + ((uint32_t)(q * 32) << 16) + acc * BN;
+      epilogue_tile(ep, trow, m, n0, M, N);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_rank0(&tempty[acc]);
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // neither CTA frees TMEM or leaves while the pair's MMAs may still run
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc2(tbase, TMEM_COLS);
   }
 }
 
@@ -285,16 +435,40 @@ cudaError_t gemm_tn_bf16_tc(const void* A, int lda, const void* B, int ldb, int 
   CUtensorMap ta, tb;
   cudaError_t e = make_tmap_bf16(&ta, A, M, K, lda, tcg::BM);
   if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // CTA pairs: 256 x 256 tiles, two SMs per tile, grid of whole pairs
+  {
+    e = make_tmap_bf16(&tb, B, N, K, ldb, tcg::HALF_ROWS);
+    if (e != cudaSuccess) return e;
+    e = set_max_smem(tcg::gemm_tc2_kernel, tcg::PAIR_SMEM_BYTES, s);
+    if (e != cudaSuccess) return e;
+    const int ntiles = ((M + tcg::PAIR_BM - 1) / tcg::PAIR_BM) * ((N + tcg::BN - 1) / tcg::BN);
+    int pairs = sms / 2;
+    if (ntiles < pairs) pairs = ntiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(tcg::NTHREADS);
+    cfg.dynamicSmemBytes = tcg::PAIR_SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, tcg::gemm_tc2_kernel, ta, tb, M, N, K, ep, status);
+    if (e == cudaSuccess) return cudaSuccess;
+    cudaGetLastError();  // a device or partition that cannot place 2-CTA clusters: one CTA per tile
+  }
   e = make_tmap_bf16(&tb, B, N, K, ldb, tcg::BN);
   if (e != cudaSuccess) return e;
   e = set_max_smem(tcg::gemm_tc_kernel, tcg::SMEM_BYTES, s);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int ntiles = ((M + tcg::BM - 1) / tcg::BM) * ((N + tcg::BN - 1) / tcg::BN);
-  const int grid = ntiles < sms ? ntiles : sms;
-  tcg::gemm_tc_kernel<<<grid, tcg::NTHREADS, tcg::SMEM_BYTES, s>>>(ta, tb, M, N, K, ep, status);
+  const int ntiles1 = ((M + tcg::BM - 1) / tcg::BM) * ((N + tcg::BN - 1) / tcg::BN);
+  tcg::gemm_tc_kernel<<<ntiles1 < sms ? ntiles1 : sms, tcg::NTHREADS, tcg::SMEM_BYTES, s>>>(ta, tb, M, N, K, ep, status);
   return cudaGetLastError();
 }
 
