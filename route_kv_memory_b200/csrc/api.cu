@@ -257,7 +257,7 @@ inline void prof_begin() { g_prof.n = 0; }
 // events are shared, so the enqueue sequence holds aux_mutex().
 struct AuxStreams {
   cudaStream_t st[2];
-  cudaEvent_t fork, join[3];
+  cudaEvent_t fork_pre, fork, join[3];
 };
 std::mutex& aux_mutex() {
   static std::mutex mu;
@@ -274,6 +274,7 @@ AuxStreams* aux_streams() {
     for (int i = 0; i < 2; ++i)
       if (cudaStreamCreateWithFlags(&a.st[i], cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     if (cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&a.fork_pre, cudaEventDisableTiming) != cudaSuccess) return nullptr;
     for (int i = 0; i < 3; ++i)
       if (cudaEventCreateWithFlags(&a.join[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
     made[dev] = true;
@@ -562,29 +563,11 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   long long kv_bstride = (long long)(state ? max_positions : d.S) * d.dkv;
   const void* wcat = P((void*)packed, PL.wcat);
 
-  prof_begin();
-  STAGE(s);
-  // 1. projections: q | XW_k | XW_v | X(W_q W_r1) | XP
-  Epilogue ep{};
-  int ns = 0;
-  ep.seg[ns++] = OutSeg{PL.seg_q, PL.seg_k, q, d.dq, d.bf16};
-  ep.seg[ns++] = OutSeg{PL.seg_k, PL.seg_r, xkv, d.width, 0};
-  ep.seg[ns++] = OutSeg{PL.seg_r, PL.seg_r + d.rh, h1, d.rh, 0};
-  if (d.bf16) ep.seg[ns++] = OutSeg{PL.seg_rlo, PL.seg_rlo + d.rh, h2, d.rh, 0};
-  ep.seg[ns++] = OutSeg{PL.seg_p, PL.Ntot, proj, d.nb, 0};
-  ep.nseg = ns;
-  if (PL.router_fused) {  // hidden layer reduced in the epilogue; h1 holds the partials
-    ep.r_begin = PL.seg_r;
-    ep.r_end = PL.seg_r + 2 * d.rh;
-    ep.w_r2 = (const float*)P((void*)packed, PL.wr2);
-    ep.zpart = h1;
-  }
-  if (d.bf16) CUDA_TRY(gemm_tn_bf16_tc(x, d.d, wcat, d.d, d.T, PL.Ntot, d.d, ep, status_ptr(), s));
-  else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, wcat, d.d, 0, d.T, PL.Ntot, d.d, ep, s));
-  STAGE(s);
   // 2-4: router tail, L3 codes, block sums / EMA end states, carries.  With stage timing on
   // they run one after another on the caller's stream (so each stage has its own time);
-  // otherwise as three concurrent branches joined before the recall.
+  // otherwise as concurrent branches joined before the recall: the block codes (which read X
+  // only) start before the projection GEMM and share the SMs with it, the router tail and
+  // the token codes, and the block sums and carries, follow the GEMM.
   HashArgs ha{proj, d.nb, x, d.bf16, (const double*)P((void*)packed, PL.pT64), d.d, d.nb, d.d};
   const double* p64 = (const double*)P((void*)packed, PL.p64);
   auto k_router = [&](cudaStream_t st) {
@@ -614,12 +597,36 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   }
   // With L3 off (MKA_TIER_L3 not set) its weight is 0: no codes and no recall, count 0 for every token.
   const bool l3 = (d.tiers & MKA_TIER_L3) != 0;
+  prof_begin();
+  if (ax && l3) {  // the L3 block codes read X only: they run beside the projection GEMM
+    CUDA_TRY(cudaEventRecord(ax->fork_pre, s));
+    CUDA_TRY(cudaStreamWaitEvent(ax->st[0], ax->fork_pre, 0));
+    CUDA_TRY(k_scode(ax->st[0]));
+  }
+  STAGE(s);
+  // 1. projections: q | XW_k | XW_v | X(W_q W_r1) | XP
+  Epilogue ep{};
+  int ns = 0;
+  ep.seg[ns++] = OutSeg{PL.seg_q, PL.seg_k, q, d.dq, d.bf16};
+  ep.seg[ns++] = OutSeg{PL.seg_k, PL.seg_r, xkv, d.width, 0};
+  ep.seg[ns++] = OutSeg{PL.seg_r, PL.seg_r + d.rh, h1, d.rh, 0};
+  if (d.bf16) ep.seg[ns++] = OutSeg{PL.seg_rlo, PL.seg_rlo + d.rh, h2, d.rh, 0};
+  ep.seg[ns++] = OutSeg{PL.seg_p, PL.Ntot, proj, d.nb, 0};
+  ep.nseg = ns;
+  if (PL.router_fused) {  // hidden layer reduced in the epilogue; h1 holds the partials
+    ep.r_begin = PL.seg_r;
+    ep.r_end = PL.seg_r + 2 * d.rh;
+    ep.w_r2 = (const float*)P((void*)packed, PL.wr2);
+    ep.zpart = h1;
+  }
+  if (d.bf16) CUDA_TRY(gemm_tn_bf16_tc(x, d.d, wcat, d.d, d.T, PL.Ntot, d.d, ep, status_ptr(), s));
+  else CUDA_TRY(gemm_tn_ffma(x, d.d, 0, wcat, d.d, 0, d.T, PL.Ntot, d.d, ep, s));
+  STAGE(s);
   if (ax) {
     CUDA_TRY(cudaEventRecord(ax->fork, s));
     CUDA_TRY(cudaStreamWaitEvent(ax->st[0], ax->fork, 0));
     CUDA_TRY(cudaStreamWaitEvent(ax->st[1], ax->fork, 0));
-    if (l3) CUDA_TRY(k_scode(ax->st[0]));
-    CUDA_TRY(cudaEventRecord(ax->join[0], ax->st[0]));
+    CUDA_TRY(cudaEventRecord(ax->join[0], ax->st[0]));  // the block codes, started before the GEMM
     if (state) CUDA_TRY(k_tail(ax->st[0]));  // reads x and xkv only; joined at the end
     CUDA_TRY(cudaEventRecord(ax->join[2], ax->st[0]));
     CUDA_TRY(k_router(ax->st[1]));
