@@ -52,6 +52,7 @@ class FastMKAConfig:
     route_mode: str = "soft"  # routing gate variant: "soft", "fixed", "top1", "top2"
     tiers: int = 7  # active memory tiers: bit 0 L1, bit 1 L2, bit 2 L3
     attention_paths: int = 1  # 1: FastMKA (fused K/V, one attention); 3: full MKA (three attention paths)
+    block_sparse: int = 0  # 1: Block-MKA's block-sparse attention (own block + recalled blocks)
 
     @property
     def dq(self) -> int:

@@ -18,6 +18,6 @@ from .fastmka import (  # noqa: F401
     gelu_erf, softmax_rows, router, router_logits, route_gate, route_margin, ROUTE_MODES, session_ema, block_summaries, hash_codes, hamming,
     recall_select, longterm_recall, fuse_sources, kv_project, causal_gqa_attention,
     online_softmax_attend, fastmka_prefill, fastmka_decode, Weights64, weights_f64,
-    recalled_block_attention, mka_full_prefill,
+    recalled_block_attention, mka_full_prefill, block_sparse_gqa_attention,
     EXCUSE_EPS,
 )

@@ -247,6 +247,31 @@ def causal_gqa_attention(q_rows: np.ndarray, positions: np.ndarray, K: np.ndarra
     return out
 
 
+def block_sparse_gqa_attention(q_rows: np.ndarray, positions: np.ndarray, K: np.ndarray, V: np.ndarray,
+                               idx: np.ndarray, count: np.ndarray, b: int, n_kv_heads: int,
+                               scale: float) -> np.ndarray:
+    """Block-MKA's block-sparse attention for ONE sequence (notes §4 / §5).
+
+    Query t attends, in one softmax, to the keys j <= t of its own block (j // b == t // b) and
+    to every key of the blocks L3 recalled for t (idx[i, :count[i]], all strictly past).
+    q_rows [n, Hq, dh] at `positions`; idx [n, R], count [n] for the same rows; K, V [S, Hkv, dh].
+    """
+    n, Hq, dh = q_rows.shape
+    G = Hq // n_kv_heads
+    out = np.zeros((n, Hq, dh))
+    for i, t in enumerate(positions):
+        t = int(t)
+        own = np.arange((t // b) * b, t + 1)
+        rec = (idx[i, :int(count[i]), None] * b + np.arange(b)[None, :]).reshape(-1)
+        keys = np.concatenate([rec, own])
+        for h in range(Hq):
+            g = h // G
+            s = K[keys, g] @ q_rows[i, h] * scale
+            p = np.exp(s - s.max())
+            out[i, h] = (p @ V[keys, g]) / p.sum()
+    return out
+
+
 def online_softmax_attend(s: np.ndarray, Vt: np.ndarray, tile: int) -> np.ndarray:
     """notes §4: softmax(s) @ Vt with the online max-shift over tiles of `tile` keys.
 
@@ -292,7 +317,8 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
     cfg supplies n_q_heads, n_kv_heads, d_head, alpha, block, recall_r, scale.
     Steps per sequence: q = X W_q; lambda = router(q); M2 = EMA(X); M3 = L3
     recall; X_fused = lambda-weighted sum of (X, M2, M3); K, V projections;
-    causal GQA attention on the query rows `rows` (all rows when None).
+    causal GQA attention on the query rows `rows` (all rows when None); with cfg.block_sparse the
+    attention is Block-MKA's block-sparse one (block_sparse_gqa_attention).
     Rows are processed in chunks only to bound memory; the EMA state is carried
     across chunks, so every value is the one the unchunked recurrence gives.
     """
@@ -354,7 +380,11 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
             if keep_d_space:
                 out["M2"][bi, r0:r1], out["M3"][bi, r0:r1], out["X_fused"][bi, r0:r1] = M2[0], M3, Xf
         out["m2_next"][bi] = m2[0]
-        O = causal_gqa_attention(out["q"][bi], rows, out["K"][bi], out["V"][bi], Hkv, cfg.scale)
+        if getattr(cfg, "block_sparse", 0):
+            O = block_sparse_gqa_attention(out["q"][bi], rows, out["K"][bi], out["V"][bi], out["idx"][bi, rows],
+                                           out["count"][bi, rows], b, Hkv, cfg.scale)
+        else:
+            O = causal_gqa_attention(out["q"][bi], rows, out["K"][bi], out["V"][bi], Hkv, cfg.scale)
         out["O"][bi] = O.reshape(len(rows), Hq * dh)
     return out
 

@@ -653,6 +653,65 @@ def test_planted_mka_mistakes_are_caught():
         check_mka_l2_path(_mut_mka_a2_leaks_current)
 
 
+# ============================================================================ Block-MKA block-sparse attention
+def check_block_sparse_recall_all(fn):
+    """R covering every eligible block: the block-sparse attention is the full causal one."""
+    cfg = tiny_cfg(recall_r=20, seq=41)
+    w = tiny_weights(cfg, np.random.default_rng(40))
+    X = np.random.default_rng(41).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    causal = O.fastmka_prefill(X, w, cfg)
+    sparse = fn(X, w, cfg.replace(block_sparse=1))
+    np.testing.assert_allclose(sparse["O"], causal["O"], rtol=1e-11, atol=1e-12)
+
+
+def check_block_sparse_dense_mask(fn):
+    """Small R: own block up to t plus the recalled blocks, as an explicit key mask."""
+    cfg = tiny_cfg(recall_r=2, seq=43, block_sparse=1)
+    w = tiny_weights(cfg, np.random.default_rng(42))
+    X = np.random.default_rng(43).standard_normal((cfg.batch, cfg.seq, cfg.d_model))
+    out = fn(X, w, cfg)
+    S, b = cfg.seq, cfg.block
+    for bi in range(cfg.batch):
+        allowed = np.zeros((S, S), bool)
+        for t in range(S):
+            allowed[t, (t // b) * b:t + 1] = True
+            for j in out["idx"][bi, t, :out["count"][bi, t]]:
+                allowed[t, j * b:(j + 1) * b] = True
+        q = out["q"][bi]
+        ref = brute_masked_gqa(q, out["K"][bi], out["V"][bi], cfg.n_kv_heads, cfg.scale, allowed)
+        np.testing.assert_allclose(out["O"][bi].reshape(ref.shape), ref, rtol=1e-11, atol=1e-12)
+
+
+def test_block_sparse_with_every_block_recalled_is_causal_attention():
+    check_block_sparse_recall_all(O.fastmka_prefill)
+
+
+def test_block_sparse_matches_a_dense_mask():
+    check_block_sparse_dense_mask(O.fastmka_prefill)
+
+
+def _mut_block_sparse_own_block_unmasked(X, w, cfg, **kw):
+    """Planted mistake: the own block is attended whole, future keys included."""
+    out = O.fastmka_prefill(X, w, cfg.replace(block_sparse=0), **kw)
+    if not getattr(cfg, "block_sparse", 0):
+        return out
+    S, b = cfg.seq, cfg.block
+    for bi in range(cfg.batch):
+        allowed = np.zeros((S, S), bool)
+        for t in range(S):
+            allowed[t, (t // b) * b:min(S, (t // b + 1) * b)] = True
+            for j in out["idx"][bi, t, :out["count"][bi, t]]:
+                allowed[t, j * b:(j + 1) * b] = True
+        ref = brute_masked_gqa(out["q"][bi], out["K"][bi], out["V"][bi], cfg.n_kv_heads, cfg.scale, allowed)
+        out["O"][bi] = ref.reshape(S, -1)
+    return out
+
+
+def test_planted_block_sparse_mistake_is_caught():
+    with pytest.raises(AssertionError):
+        check_block_sparse_dense_mask(_mut_block_sparse_own_block_unmasked)
+
+
 # ============================================================================ regression snapshot
 def test_golden_snapshot_unchanged():
     """tests/golden/tiny_f32_oracle.json (written by tests/golden/make_golden.py from the oracle) still holds."""
