@@ -381,8 +381,10 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
                 out["M2"][bi, r0:r1], out["M3"][bi, r0:r1], out["X_fused"][bi, r0:r1] = M2[0], M3, Xf
         out["m2_next"][bi] = m2[0]
         if getattr(cfg, "block_sparse", 0):
+            # without the L3 tier there is no recall: a token keeps its own block only
+            cnt = out["count"][bi, rows] if getattr(cfg, "tiers", 7) & 4 else np.zeros(len(rows), np.int64)
             O = block_sparse_gqa_attention(out["q"][bi], rows, out["K"][bi], out["V"][bi], out["idx"][bi, rows],
-                                           out["count"][bi, rows], b, Hkv, cfg.scale)
+                                           cnt, b, Hkv, cfg.scale)
         else:
             O = causal_gqa_attention(out["q"][bi], rows, out["K"][bi], out["V"][bi], Hkv, cfg.scale)
         out["O"][bi] = O.reshape(len(rows), Hq * dh)
