@@ -108,6 +108,11 @@ def prefill_flops(cfg) -> dict:
     T, d, dq, dkv, rh, nb = cfg.tokens, cfg.d_model, cfg.dq, cfg.dkv, cfg.router_hidden, cfg.hash_bits
     causal_pairs = cfg.batch * cfg.seq * (cfg.seq + 1) / 2
     attn = 4.0 * cfg.d_head * cfg.n_q_heads * causal_pairs  # QK^T and PV over j <= t only
+    if getattr(cfg, "block_sparse", 0):
+        # Block-MKA: row t attends to keys <= t of its own block and to min(R, t // b) recalled blocks
+        t = np.arange(cfg.seq)
+        keys = t % cfg.block + 1 + (np.minimum(cfg.recall_r, t // cfg.block) * cfg.block if cfg.tiers & 4 else 0)
+        attn = 4.0 * cfg.d_head * cfg.n_q_heads * cfg.batch * float(keys.sum())
     if getattr(cfg, "attention_paths", 1) == 3 and cfg.tiers & 4:
         # full MKA's recalled-block path: row t attends to min(R, t // b) blocks of b keys
         t = np.arange(cfg.seq)
@@ -126,7 +131,8 @@ def decode_bytes_per_token(cfg, ctx: int, ntot: int) -> float:
 def workload_cfg(args, name):
     """The named workload with the routing gate / memory tiers the command line selects."""
     return CONFIGS[name].replace(route_mode=args.route, tiers=args.tiers,
-                                 attention_paths=getattr(args, "paths", 1))
+                                 attention_paths=getattr(args, "paths", 1),
+                                 block_sparse=int(getattr(args, "block_sparse", False)))
 
 
 def model_name(cfg) -> str:
@@ -194,7 +200,8 @@ def run_ours(args, rank, world, local_rank):
     fl = prefill_flops(cfg)
     attn_ms = float(stages[8])
     attn_tflops = fl["attention"] / (attn_ms / 1e3) / 1e12
-    roofline = {"kernel": "attention (causal GQA, online max-shift)" if cfg.attention_paths == 1 else
+    roofline = {"kernel": ("attention (Block-MKA block-sparse: own block + recalled blocks)" if cfg.block_sparse else
+                           "attention (causal GQA, online max-shift)") if cfg.attention_paths == 1 else
                 "attention (full MKA: causal pass + recalled-block pass)", "bound": "tensor",
                 "achieved": round(attn_tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
@@ -264,7 +271,8 @@ def run_ours(args, rank, world, local_rank):
                                f"{cfg.block}, R {cfg.recall_r}, nbits {cfg.hash_bits}, seed {cfg.seed}"
                                + ("" if (cfg.route_mode, cfg.tiers) == ("soft", 7) else
                                   f"; routing {cfg.route_mode}, tiers mask {cfg.tiers}")
-                               + ("; full MKA, three attention paths" if cfg.attention_paths == 3 else ""),
+                               + ("; full MKA, three attention paths" if cfg.attention_paths == 3 else "")
+                               + ("; Block-MKA block-sparse attention" if cfg.block_sparse else ""),
                    "global_batch": cfg.batch * world, "seq_len": cfg.seq,
                    "parallelism": f"replicas x{world} (independent sequences, no exchange)",
                    "l2": "flushed (512 MB write) before every timed step"},
@@ -276,7 +284,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
     }
     del flush
-    if world == 1 and not args.no_decode and args.paths == 1:  # full MKA has no decode step
+    if world == 1 and not args.no_decode and args.paths == 1 and not args.block_sparse:  # prefill-only variants
         result["decode"] = run_decode(args, cfg, inp, weights, dev, layer_pack=None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, inp, budget_rows=args.cpu_rows)
@@ -448,6 +456,8 @@ def main():
     ap.add_argument("--tiers", type=int, default=7, help="memory tier mask: 1 L1, 2 L2, 4 L3 (7 = all)")
     ap.add_argument("--paths", type=int, default=1, choices=[1, 3],
                     help="1: FastMKA (the layer measured); 3: full MKA, three attention paths (prefill only)")
+    ap.add_argument("--block-sparse", action="store_true",
+                    help="Block-MKA block-sparse attention: own block + recalled blocks (prefill only)")
     ap.add_argument("--decode-ctx", type=int, nargs="*", default=[131072])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode measurement (no prefill line)")

@@ -100,6 +100,11 @@ typedef struct mka_config {
                               recalled L3 blocks' tokens.  3 is implemented for bf16 prefill with
                               block_size a multiple of 128, recall_r <= 16 and no decode state;
                               otherwise MKA_ERR_UNSUPPORTED */
+  int32_t block_sparse;  /* 0: one full causal attention (notes §3).  1: Block-MKA's block-sparse
+                            attention (notes §4-5): token t attends, in one softmax, to the keys <= t
+                            of its own L3 block and to every key of its recalled blocks.  With
+                            attention_paths 1 only; bf16 prefill, block_size a multiple of 128,
+                            recall_r <= 16, no decode state; otherwise MKA_ERR_UNSUPPORTED */
 } mka_config;
 
 /* Raw layer weights, all in cfg->dtype, all [d_in, d_out] row-major. */
@@ -182,7 +187,8 @@ MKA_API int mka_longterm_recall(const mka_config* cfg, const void* x, const void
  * is not NULL (mka_state_init'ed, max_positions >= S), the fused K/V rows, M2[S],
  * the finished block summaries and the unfinished block's partial sums are left in
  * it and its position is set to S, ready for mka_decode_step.
- * ws: mka_workspace_size(cfg) bytes. */
+ * ws: mka_workspace_size(cfg) bytes, 16-byte aligned (32-byte aligned for full MKA and
+ * block-sparse attention, whose partial results are written 32 bytes at a time). */
 MKA_API int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x, void* out, float* lambda_out,
                         int32_t* recall_idx_out, void* state, size_t state_bytes, int32_t max_positions,
                         void* ws, size_t ws_bytes, void* stream);

@@ -52,7 +52,7 @@ class mka_config(ctypes.Structure):
         ("router_hidden", ctypes.c_int32), ("ema_alpha", ctypes.c_float), ("block_size", ctypes.c_int32),
         ("recall_r", ctypes.c_int32), ("hash_bits", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("attn_scale", ctypes.c_float), ("route_mode", ctypes.c_int32), ("tiers", ctypes.c_int32),
-        ("attention_paths", ctypes.c_int32),
+        ("attention_paths", ctypes.c_int32), ("block_sparse", ctypes.c_int32),
     ]
 
 
@@ -124,7 +124,7 @@ def make_config(cfg, seq: Optional[int] = None, batch: Optional[int] = None) -> 
         dtype=MKA_F32 if cfg.dtype == "f32" else MKA_BF16,
         attn_scale=cfg.attn_scale if cfg.attn_scale is not None else 0.0,
         route_mode=ROUTE_MODES[getattr(cfg, "route_mode", "soft")], tiers=getattr(cfg, "tiers", 7),
-        attention_paths=getattr(cfg, "attention_paths", 1))
+        attention_paths=getattr(cfg, "attention_paths", 1), block_sparse=getattr(cfg, "block_sparse", 0))
 
 
 # ------------------------------------------------------------------ sizes

@@ -66,6 +66,7 @@ struct Dims {
   float alpha, scale;
   int route, tiers;  // routing gate variant; active tiers (MKA_TIER_* mask, never 0)
   int paths;         // 1 FastMKA, 3 full MKA
+  int block_sparse;  // Block-MKA's block-sparse attention
 };
 
 int check_cfg(const mka_config* c, Dims* o) {
@@ -90,6 +91,10 @@ int check_cfg(const mka_config* c, Dims* o) {
     return fail(MKA_ERR_INVALID_ARG, "attention_paths must be 1 (FastMKA) or 3 (full MKA)");
   if (c->attention_paths == 3 && (c->dtype != MKA_BF16 || c->block_size % 128 || c->recall_r > 16))
     return fail(MKA_ERR_UNSUPPORTED, "full MKA needs bf16, a block_size that is a multiple of 128 and recall_r <= 16");
+  if (c->block_sparse != 0 && c->block_sparse != 1) return fail(MKA_ERR_INVALID_ARG, "block_sparse must be 0 or 1");
+  if (c->block_sparse && (c->attention_paths == 3 || c->dtype != MKA_BF16 || c->block_size % 128 || c->recall_r > 16))
+    return fail(MKA_ERR_UNSUPPORTED,
+                "block-sparse attention needs FastMKA, bf16, a block_size that is a multiple of 128 and recall_r <= 16");
   long long T = (long long)c->batch * c->seq;
   if (T > (1LL << 30)) return fail(MKA_ERR_UNSUPPORTED, "batch * seq too large");
   if ((c->seq + c->block_size - 1) / c->block_size > 65535) return fail(MKA_ERR_UNSUPPORTED, "seq / block_size > 65535");
@@ -114,6 +119,7 @@ int check_cfg(const mka_config* c, Dims* o) {
   d.alpha = c->ema_alpha;
   d.route = c->route_mode;
   d.paths = c->attention_paths == 3 ? 3 : 1;
+  d.block_sparse = c->block_sparse;
   d.tiers = c->tiers ? c->tiers : (MKA_TIER_L1 | MKA_TIER_L2 | MKA_TIER_L3);
   d.scale = c->attn_scale > 0.f ? c->attn_scale : 1.f / sqrtf((float)d.dh);
   return MKA_OK;
@@ -150,8 +156,15 @@ PackLayout pack_layout(const Dims& d) {
 
 // ---------------------------------------------------------------- prefill workspace
 struct PrefillWs {
-  size_t q, xkv, h1, h2, proj, lam, tcode, xsum, bsum, bend, gend, carry, scode, idx, cnt, k, v, v2, total;
+  size_t q, xkv, h1, h2, proj, lam, tcode, xsum, bsum, bend, gend, carry, scode, idx, cnt, k, v, v2;
+  size_t g_nrec, g_recoff, g_cursor, g_pairoff, g_pairbj, g_list, part_o, part_lse, total;
 };
+// Block-gathered attention (Block-MKA block-sparse, full MKA's recalled-block path): every L3
+// block, the last partial one included, has a token list; each token keeps one partial result
+// per attended block: R recalled, plus its own block for Block-MKA.
+static int gathered_blocks(const Dims& d) { return (d.S + d.blk - 1) / d.blk; }
+static int gathered_slots(const Dims& d) { return d.R + (d.block_sparse ? 1 : 0); }
+static int gathered_tpt(const Dims& d) { return 128 / gathered_rows_per_token(d.Hq / d.Hkv); }
 PrefillWs prefill_ws(const Dims& d) {
   PrefillWs w;
   size_t T = d.T, o = 0;
@@ -173,6 +186,16 @@ PrefillWs prefill_ws(const Dims& d) {
   w.k = o; o += al(T * d.dkv * d.elem);
   w.v = o; o += al(T * d.dkv * d.elem);
   w.v2 = o; o += d.paths == 3 ? al(T * d.dkv * 4) : 0;  // full MKA: the L2 path's value M2 W_v
+  const bool ga = d.paths == 3 || d.block_sparse;
+  const size_t nbj = ga ? (size_t)d.B * gathered_blocks(d) : 0, ns = ga ? gathered_slots(d) : 0;
+  w.g_nrec = o; o += al(nbj * 4);
+  w.g_recoff = o; o += al(nbj * 4);
+  w.g_cursor = o; o += al(nbj * 4);
+  w.g_pairoff = o; o += ga ? al((nbj + 1) * 4) : 0;
+  w.g_pairbj = o; o += ga ? al(gathered_max_pairs(T, d.R, d.block_sparse, gathered_tpt(d), nbj) * 4) : 0;
+  w.g_list = o; o += ga ? al(T * d.R * 4) : 0;
+  w.part_o = o; o += al(T * ns * d.dq * 2);
+  w.part_lse = o; o += al(T * ns * d.Hq * 4);
   w.total = o;
   return w;
 }
@@ -530,10 +553,13 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
       (lambda_out && !aligned16(lambda_out)) || (recall_idx_out && !aligned16(recall_idx_out)) ||
       (state && !aligned16(state)))
     return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((d.paths == 3 || d.block_sparse) && ((uintptr_t)ws & 31))  // 32-byte stores into its partial results
+    return fail(MKA_ERR_INVALID_ARG, "full MKA and block-sparse attention need a 32-byte aligned workspace");
   PrefillWs W = prefill_ws(d);
   if (ws_bytes < W.total) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, W.total);
   StateLayout SL{};
-  if (state && d.paths == 3) return fail(MKA_ERR_UNSUPPORTED, "full MKA has no decode state");
+  if (state && (d.paths == 3 || d.block_sparse))
+    return fail(MKA_ERR_UNSUPPORTED, "full MKA and block-sparse attention have no decode state");
   if (state) {
     if (max_positions < d.S) return fail(MKA_ERR_CAPACITY, "max_positions %d < seq %d", max_positions, d.S);
     SL = state_layout(d, max_positions);
@@ -665,18 +691,42 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   if (d.paths == 3) fa.v2_out = (float*)P(ws, W.v2);  // K, V <- the tokens' own; v2 <- M2 W_v
   CUDA_TRY(fuse_kv(fa, s));
   STAGE(s);
-  // 6. causal GQA attention over the fused K/V
+  // 6. causal GQA attention over the fused K/V (Block-MKA: none; its own-block part is gathered)
   AttnArgs aa{};
   aa.q = q; aa.q_bstride = (long long)d.S * d.dq; aa.q_ld = d.dq;
   aa.k = kbuf; aa.v = vbuf; aa.kv_bstride = kv_bstride; aa.kv_ld = d.dkv;
   aa.o = out; aa.o_bstride = (long long)d.S * d.dq; aa.o_ld = d.dq;
   aa.B = d.B; aa.S = d.S; aa.Hq = d.Hq; aa.Hkv = d.Hkv; aa.dh = d.dh; aa.scale = d.scale;
-  if (d.bf16) CUDA_TRY(attention_prefill_tc(aa, status_ptr(), s));
-  else CUDA_TRY(attention_prefill(aa, 0, s));
-  if (d.paths == 3) {  // full MKA: the recalled-block path, mixed with the causal one and the L2 value
-    AttnArgs a3 = aa;
-    a3.ridx = idx; a3.rcnt = cnt; a3.R = d.R; a3.blk = d.blk; a3.lam = lam; a3.v2 = (const float*)P(ws, W.v2);
-    CUDA_TRY(attention_prefill_tc(a3, status_ptr(), s));
+  if (!d.block_sparse) {
+    if (d.bf16) CUDA_TRY(attention_prefill_tc(aa, status_ptr(), s));
+    else CUDA_TRY(attention_prefill(aa, 0, s));
+  }
+  if (d.block_sparse || d.paths == 3) {
+    // Block-MKA: each token's own block (causal) and recalled blocks; full MKA: the recalled
+    // blocks' tokens, then mixed with the causal output and the L2 value.  Rows are gathered
+    // per block, attended on the tensor cores, and their per-block results merged.
+    const int own = d.block_sparse, nball = gathered_blocks(d), ns = gathered_slots(d);
+    int* nrec = (int*)P(ws, W.g_nrec);
+    int* recoff = (int*)P(ws, W.g_recoff);
+    int* pairoff = (int*)P(ws, W.g_pairoff);
+    int* list = (int*)P(ws, W.g_list);
+    int* pairbj = (int*)P(ws, W.g_pairbj);
+    CUDA_TRY(block_lists(idx, cnt, d.B, d.S, d.R, d.blk, nball, own, own, gathered_tpt(d), nrec, recoff,
+                         (int*)P(ws, W.g_cursor), pairoff, pairbj, list, s));
+    AttnArgs ag = aa;
+    ag.g_nrec = nrec; ag.g_recoff = recoff; ag.g_list = list; ag.g_pairoff = pairoff; ag.g_pairbj = pairbj;
+    ag.g_own = own; ag.nblk = nball; ag.blk = d.blk; ag.nslot = ns;
+    ag.part_o = P(ws, W.part_o); ag.part_lse = (float*)P(ws, W.part_lse);
+    CUDA_TRY(attention_prefill_tc(ag, status_ptr(), s));
+    MergeArgs mg{};
+    mg.part_o = ag.part_o; mg.part_lse = ag.part_lse; mg.nslot = ns; mg.cnt = cnt; mg.own = own;
+    mg.B = d.B; mg.S = d.S; mg.Hq = d.Hq; mg.Hkv = d.Hkv; mg.dh = d.dh;
+    mg.o = out; mg.o_bstride = (long long)d.S * d.dq; mg.o_ld = d.dq;
+    if (d.paths == 3) {
+      mg.lam = lam;
+      mg.v2 = (const float*)P(ws, W.v2);
+    }
+    CUDA_TRY(merge_partials(mg, s));
   }
   STAGE(s);
   if (ax) {
@@ -697,7 +747,8 @@ int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size
   if (!aligned16(packed) || !aligned16(state) || !aligned16(x_new) || !aligned16(out) || !aligned16(ws))
     return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if (max_positions < 1) return fail(MKA_ERR_INVALID_ARG, "max_positions must be >= 1");
-  if (d.paths == 3) return fail(MKA_ERR_UNSUPPORTED, "full MKA has no decode step");
+  if (d.paths == 3 || d.block_sparse)
+    return fail(MKA_ERR_UNSUPPORTED, "full MKA and block-sparse attention have no decode step");
   if (d.B > 8) return fail(MKA_ERR_UNSUPPORTED, "decode batch must be <= 8");
   if (d.bf16 && d.Hq / d.Hkv > 16) return fail(MKA_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads must be <= 16 for decode");
   StateLayout SL = state_layout(d, max_positions);

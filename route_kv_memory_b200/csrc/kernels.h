@@ -121,17 +121,53 @@ struct AttnArgs {
   void* o; long long o_bstride; int o_ld;
   int B, S, Hq, Hkv, dh;
   float scale;
-  // Recalled-block attention of full MKA (set ridx to select it): row t attends to the keys of
-  // its recalled L3 blocks only (ridx [B*S][R], rcnt [B*S]; block length blk, a multiple of 128),
-  // and the output row becomes lam0 * o (the causal pass, read back) + lam1 * v2 + lam2 * that.
-  const int* ridx = nullptr; const int* rcnt = nullptr; int R = 0, blk = 0;
-  const float* lam = nullptr;     // [B*S][3]
-  const float* v2 = nullptr;      // [B*S][Hkv*dh] float32: the L2 path's value M2 W_v
+  // Block-gathered attention (set g_pairoff to select it; bf16, tcgen05 only).  The rows of a
+  // work item are (token, query head) pairs that all attend to the keys of one L3 block j of
+  // sequence b: the tokens of block j's list (its own tokens first when g_own, under the causal
+  // mask, then the tokens that recalled it), each with the G = Hq / Hkv query heads of one KV
+  // group.  No o is written: each row leaves its partial softmax result, O / l in bf16 and the
+  // log2 normaliser m + log2(l), in slot `slot` of its token, for merge_partials to combine.
+  const int* g_nrec = nullptr;     // [B*nblk] tokens that recalled block (b, j)
+  const int* g_recoff = nullptr;   // [B*nblk] where their entries start in g_list
+  const int* g_list = nullptr;     // entries (t << 5) | slot, t the position in the sequence
+  const int* g_pairoff = nullptr;  // [B*nblk + 1] first tile pair of each block; [B*nblk] = all pairs
+  const int* g_pairbj = nullptr;   // [all pairs] the block (b * nblk + j) of each tile pair
+  int g_own = 0, nblk = 0, blk = 0, nslot = 0;
+  void* part_o = nullptr;          // [B*S][nslot][Hq*dh] bf16
+  float* part_lse = nullptr;       // [B*S][nslot][Hq]
 };
 cudaError_t attention_prefill(const AttnArgs& a, int bf16, cudaStream_t s);
-// bf16 path on tcgen05 (tc_attention.cu): persistent, TMA-fed, S and P in TMEM; causal, or the
-// recalled-block pass of full MKA when a.ridx is set.
+// bf16 path on tcgen05 (tc_attention.cu): persistent, TMA-fed, S and P in TMEM; causal, or
+// block-gathered when a.g_pairoff is set.
 cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s);
+
+// ---------------------------------------------------------------- block-gathered attention (block_sparse.cu)
+// Query-tile rows one token takes in the block-gathered attention: its G = Hq / Hkv heads, or an
+// aligned 8-row slot for 4 < G <= 8 (one 3-D TMA box per token and 64-column half).
+__host__ __device__ inline int gathered_rows_per_token(int G) { return G > 4 && G <= 8 ? 8 : G; }
+// Tile pairs the block-gathered attention can run at most (block_lists' pairbj capacity).
+inline size_t gathered_max_pairs(long long T, int R, int own, int tpt, long long nbj) {
+  return (size_t)((T * (R + own)) / (2 * tpt) + nbj + 1);
+}
+// Lists, per L3 block (b, j), the tokens whose recall picked it, and the tile pairs the gathered
+// attention runs for it (own tokens of the block first when own).  Entry slot = r + slot_base for
+// recall rank r.  Scratch from the caller: nrec, recoff, cursor [B*nblk], pairoff [B*nblk + 1],
+// list [B*S*R], pairbj [gathered_max_pairs()].  tpt: tokens per 128-row query tile
+// (128 / gathered_rows_per_token(Hq / Hkv)).
+cudaError_t block_lists(const int* idx, const int* cnt, int B, int S, int R, int blk, int nblk, int own,
+                        int slot_base, int tpt, int* nrec, int* recoff, int* cursor, int* pairoff, int* pairbj,
+                        int* list, cudaStream_t s);
+struct MergeArgs {
+  const void* part_o; const float* part_lse; int nslot;
+  const int* cnt; int own;          // partial slots of token t: [0, cnt[t] + own)
+  int B, S, Hq, Hkv, dh;
+  void* o; long long o_bstride; int o_ld;   // bf16 output rows
+  // full MKA (lam set): o = lam0 * o (read back) + lam1 * v2 + lam2 * merged; else o = merged
+  const float* lam = nullptr; const float* v2 = nullptr;  // [B*S][3], [B*S][Hkv*dh]
+};
+// Combines each row's partial softmax results: w_s = 2^(lse_s - max lse), o = sum w_s O_s / sum w_s
+// (0 when the row has no slot).
+cudaError_t merge_partials(const MergeArgs& m, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode
 struct DecodeArgs {

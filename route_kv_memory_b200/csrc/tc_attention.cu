@@ -18,6 +18,13 @@
 //               the stale maximum bounds P by 256; at the end O_t / l goes to
 //               global memory.
 // TMEM columns: O_0 [0,128), O_1 [128,256), S_0/P_0 [256,384), S_1/P_1 [384,512).
+//
+// MODE 1 (block-gathered, for Block-MKA's block-sparse attention and full MKA's recalled-block
+// path): an item is a pair of 128-row tiles of (token, head) rows that all read the keys of one
+// L3 block (block_sparse.cu lists them).  The loader warp gathers the query rows four at a time
+// with TMA (tile::gather4) into the same swizzled tile layout; each row keeps its own softmax
+// over the block's key tiles (the causal mask only for the block's own tokens) and leaves O / l
+// in bf16 with its log2 normaliser for the merge.
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
@@ -26,6 +33,8 @@
 namespace mka {
 
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows);
+cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, int d0, int d1, int d2, long long s1, long long s2,
+                              int box1);
 
 namespace tca {
 
@@ -35,6 +44,7 @@ constexpr int BQ = 128, BKV = 128;
 constexpr int NTHREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+constexpr int kNoMask = 0x7fffffff;
 
 template <int DH>
 struct Cfg {
@@ -43,10 +53,8 @@ struct Cfg {
   static constexpr int KV_BYTES = 2 * K_BYTES;   // K then V
   static constexpr int HALF = 128 * 64 * 2;      // one 128-row x 64-column swizzled box
   static constexpr int SMEM = 2 * Q_BYTES + 2 * KV_BYTES + 1024 + 256;
-  // recalled-block pass: each softmax row's recalled block indices, staged per item
-  static constexpr int REC_BYTES = 2 * BQ * 16 * 4;
+  static constexpr int GATHER_BYTES = 2 * BQ * 4;  // MODE 1: the loader's token lists of both tiles
 };
-constexpr int MAX_RECALL_RC = 16;  // recall_r the recalled-block pass stages in shared memory
 
 struct Work {
   int b, h, pair;
@@ -67,6 +75,34 @@ __device__ __forceinline__ Work work_item(int w, int B, int Hq, int npairs) {
 __device__ __forceinline__ int snake_item(int r, int grid, int cta, int nwork) {
   const int w = r * grid + ((r & 1) ? grid - 1 - cta : cta);
   return w < nwork ? w : -1;
+}
+
+// MODE 1 work item: tile pair p of the row list of block j of sequence b, KV group g.
+struct GWork {
+  int b, g, j, p, own, entries, recbase;
+};
+__device__ __forceinline__ GWork gwork_item(int w, const AttnArgs& a) {
+  GWork r;
+  const int P = w / a.Hkv;
+  r.g = w - P * a.Hkv;
+  const int lo = a.g_pairbj[P];
+  r.p = P - a.g_pairoff[lo];
+  r.b = lo / a.nblk;
+  r.j = lo - r.b * a.nblk;
+  r.own = a.g_own ? min(a.blk, a.S - r.j * a.blk) : 0;
+  r.entries = r.own + a.g_nrec[lo];
+  r.recbase = a.g_recoff[lo];
+  return r;
+}
+// Token (position in the sequence) and partial slot of entry e of the item's list; -1 past the end.
+__device__ __forceinline__ int gwork_token(const AttnArgs& a, const GWork& it, int e, int* slot) {
+  *slot = 0;
+  if (e >= it.entries) return -1;
+  if (e < it.own) return it.j * a.blk + e;
+  const int v = a.g_list[it.recbase + e - it.own];
+  *slot = v & 31;
+  const int t = v >> 5;
+  return t < a.S ? t : -1;
 }
 
 // MN-major (V) descriptor: 8-key groups of 128-B rows 1024 B apart (stride byte
@@ -93,11 +129,8 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// RC selects the recalled-block pass of full MKA: tile t of a pair runs only the key tiles
-// before its query block's L3 block (n_t = (qt / m) * m for L3 blocks of m key tiles, possibly
-// 0), a row keeps a key tile only if that tile's block is among the row's recalled blocks, and
-// the epilogue writes lam0 * (causal output already in a.o) + lam1 * v2 + lam2 * this pass.
-template <int DH, bool RC>
+// MODE 0: causal attention; MODE 1: block-gathered rows (see the top of the file).
+template <int DH, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, AttnArgs a, int* status) {
@@ -121,10 +154,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* o_empty = bars + 16;  // [2]
   uint64_t* drain = bars + 18;
   uint32_t* tmem_slot = (uint32_t*)(bars + 19);
-  int* srec = (int*)(smem + 2 * C::Q_BYTES + 2 * C::KV_BYTES + 256);  // RC only: [2][BQ][MAX_RECALL_RC]
+  int* stok = (int*)(smem + 2 * C::Q_BYTES + 2 * C::KV_BYTES + 256);  // MODE 1: loader's tokens, [2][BQ]
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  constexpr bool GA = MODE == 1;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
@@ -152,17 +186,122 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int nqt = (a.S + BQ - 1) / BQ;
   const int npairs = (nqt + 1) / 2;
-  const int nwork = a.B * a.Hq * npairs;
+  const int nbj = a.B * a.nblk;
+  const int nwork = GA ? a.Hkv * a.g_pairoff[nbj] : a.B * a.Hq * npairs;
   const int G = a.Hq / a.Hkv;
+  const int RPT = gathered_rows_per_token(G);  // MODE 1: tile rows per token (its G heads first)
+  const int tpt = BQ / RPT;                    // MODE 1: tokens per query tile
   const long long q_rows_per_b = a.q_bstride / a.q_ld;
   const long long kv_rows_per_b = a.kv_bstride / a.kv_ld;
-  const int mt = RC ? a.blk / BKV : 1;  // key tiles per L3 block
-  // key tiles query tile qt runs: causal up to its own tile, or the tiles of strictly past L3 blocks
-  auto ntiles = [&](int qt) { return RC ? (qt / mt) * mt : qt + 1; };
+  const int mt = GA ? a.blk / BKV : 1;  // MODE 1: key tiles per L3 block
+  // Key tiles of the two query tiles of an item (n0 <= n1).  Causal: tile qt runs tiles 0..qt.
+  // MODE 1: local tile t holds list tile 2p + 1 - t, so tile 1 always exists and tile 0 may be
+  // empty (0 key tiles); both read the same mt key tiles of block j.
+  auto item_tiles = [&](int w, int& n0, int& n1) {
+    if constexpr (GA) {
+      const GWork it = gwork_item(w, a);
+      n0 = (2 * it.p + 1) * tpt < it.entries ? mt : 0;
+      n1 = mt;
+    } else {
+      const Work it = work_item(w, a.B, a.Hq, npairs);
+      n0 = 2 * it.pair + 1;
+      n1 = 2 * it.pair + 2;
+    }
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ loader
-    if (lane == 0) {
+    if constexpr (GA) {
+      // The warp looks up the tile's tokens, then every lane gathers four query rows per 64-column
+      // half with one TMA (tmQ views q as [B*S*Hq rows][dh]); lane 0 then issues the block's K/V.
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
+      int kvit = 0;
+      for (int rr = 0; rr * (int)gridDim.x < nwork; ++rr) {
+        const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
+        if (w < 0) break;
+        const int wi = rr;
+        const GWork it = gwork_item(w, a);
+        // the block's K/V first: its stages free up earlier than the query tiles
+        bool ok = true;
+        if (lane == 0) {
+          for (int jj = 0; jj < mt; ++jj, ++kvit) {
+            const int st = kvit & 1;
+            if (!mbar_wait(&kv_empty[st], ((kvit >> 1) & 1) ^ 1, abort, status)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(&kv_full[st], C::KV_BYTES);
+            uint8_t* kdst = sKV + st * C::KV_BYTES;
+            const int ky = (int)(it.b * kv_rows_per_b) + it.j * a.blk + jj * BKV;
+            for (int hb = 0; hb < NH; ++hb) {
+              tma_load_2d(kdst + hb * C::HALF, &tmK, &kv_full[st], it.g * DH + hb * 64, ky);
+              tma_load_2d(kdst + C::K_BYTES + hb * C::HALF, &tmV, &kv_full[st], it.g * DH + hb * 64, ky);
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        bool qok = true;
+        for (int t = 0; t < 2; ++t) {
+          const int lt = 2 * it.p + 1 - t;
+          const bool full = lt * tpt < it.entries;
+          int tok = -1;  // token of slot `lane` (8-row slots) or of entry `lane` (gather4)
+          if (full && lane < tpt) {
+            int slot;
+            tok = gwork_token(a, it, lt * tpt + lane, &slot);
+          }
+          if (RPT != 8 && full)
+            for (int k = lane; k < tpt; k += 32) {
+              int slot;
+              stok[t * BQ + k] = k == lane ? tok : gwork_token(a, it, lt * tpt + k, &slot);
+            }
+          const bool ok_t = mbar_wait(&q_empty[t], (wi & 1) ^ 1, abort, status);
+          if (!__all_sync(0xffffffffu, ok_t)) {
+            qok = false;
+            break;
+          }
+          if (full) {
+            if (lane == 0) mbar_expect_tx(&q_full[t], C::Q_BYTES);
+            __syncwarp();
+            uint8_t* dst_t = sQ + t * C::Q_BYTES;
+            if (RPT == 8) {
+              // one box of the token's 8 heads from g * G (tmQ: [B*S][Hq][dh]) per 64-column half
+              if (lane < tpt) {
+                const int z = it.b * a.S + (tok >= 0 ? tok : 0);
+#pragma unroll
+                for (int hb = 0; hb < NH; ++hb)
+                  tma_load_3d(dst_t + hb * C::HALF + lane * 1024, &tmQ, &q_full[t], hb * 64, it.g * G, z);
+              }
+            } else {
+              // four rows per lane and half (tmQ: [B*S*Hq][dh], one-row boxes)
+              const int row0 = it.b * a.S * a.Hq;  // a valid row for the padding rows
+              int rows[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int r = 4 * lane + u, k = r / G;
+                const int tk = k < tpt ? stok[t * BQ + k] : -1;
+                rows[u] = tk >= 0 ? (it.b * a.S + tk) * a.Hq + it.g * G + (r - k * G) : row0;
+              }
+#pragma unroll
+              for (int hb = 0; hb < NH; ++hb)
+                tma_gather4_2d(dst_t + hb * C::HALF + 4 * lane * 128, &tmQ, &q_full[t], hb * 64, rows[0], rows[1],
+                               rows[2], rows[3]);
+            }
+          } else if (lane == 0) {
+            mbar_arrive(&q_full[t]);  // empty tile: nothing to load
+          }
+          __syncwarp();
+        }
+      }
+      if (lane == 0 && *abort) {  // let issued copies land (bounded) before unwinding
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 50000000ull) {
+        }
+      }
+    } else if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -185,7 +324,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_2d(sQ + t * C::Q_BYTES + hb * C::HALF, &tmQ, &q_full[t], it.h * DH + hb * 64, qy);
         }
         if (!qok) break;
-        const int nkv = ntiles(2 * it.pair + 1);
+        const int nkv = 2 * it.pair + 2;
         bool ok = true;
         for (int j = 0; j < nkv; ++j, ++kvit) {
           const int st = kvit & 1;
@@ -232,12 +371,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                        (j | kk) != 0);
         umma_commit(&pv_done[t]);
       };
+      int nx0 = 0, nx1 = 0;  // tiles of the next item, looked up while this one runs
+      {
+        const int w0 = snake_item(0, gridDim.x, blockIdx.x, nwork);
+        if (w0 >= 0) item_tiles(w0, nx0, nx1);
+      }
       for (int rr = 0; rr * (int)gridDim.x < nwork && ok; ++rr) {
         const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
         if (w < 0) break;
         const int wi = rr;  // items this CTA has started before this one
-        const Work it = work_item(w, a.B, a.Hq, npairs);
-        const int n0 = ntiles(2 * it.pair), n1 = ntiles(2 * it.pair + 1);  // n0 <= n1
+        const int n0 = nx0, n1 = nx1;  // n0 <= n1, n1 >= 1
         if (!mbar_wait(&q_full[0], wi & 1, abort, status)) break;
         if (n1 > 0 && !mbar_wait(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
         tc_fence_after();
@@ -258,6 +401,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (n1 == 0) {
           if (!mbar_wait(&o_empty[1], (wi & 1) ^ 1, abort, status)) break;
           umma_commit(&o_full[1]);
+        }
+        {  // the next item's tile counts, looked up while these S MMAs and the softmax run
+          const int wn = snake_item(rr + 1, gridDim.x, blockIdx.x, nwork);
+          if (wn >= 0) item_tiles(wn, nx0, nx1);
         }
         for (int j = 0; j < n1; ++j) {
           const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
@@ -318,39 +465,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
       if (w < 0) break;
       const int wi = rr;
-      const Work it = work_item(w, a.B, a.Hq, npairs);
-      const int qt = 2 * it.pair + t;
-      const int nkv = ntiles(qt);
-      const int row = qt * BQ + r;
-      // recalled-block pass: this row's recalled L3 blocks
-      int my_cnt = 0;
-      if (RC) {  // stage this row's recalled blocks in shared memory (keeps them out of registers)
-        const size_t tok = (size_t)it.b * a.S + row;
-        my_cnt = row < a.S ? a.rcnt[tok] : 0;
-        for (int q = 0; q < my_cnt; ++q) srec[(t * BQ + r) * MAX_RECALL_RC + q] = a.ridx[tok * a.R + q];
-        if (row < a.S) {  // the epilogue's inputs (causal output, L2 value) into L2 while the tiles run
-          const char* o1 = (const char*)((const bf16*)a.o + (size_t)it.b * a.o_bstride + (size_t)row * a.o_ld +
-                                         (size_t)it.h * DH);
-          const char* v2 = (const char*)(a.v2 + tok * (size_t)(a.Hkv * DH) + (size_t)(it.h / G) * DH);
-#pragma unroll
-          for (int k = 0; k < DH * 2; k += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(o1 + k));
-#pragma unroll
-          for (int k = 0; k < DH * 4; k += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(v2 + k));
-        }
+      // This row: causal, position `row` of query head h of sequence b; MODE 1, the token of
+      // entry e of the item's list (-1 for a padding row), query head h of KV group g.
+      int b, h, row, nkv, slot = 0, key0 = 0;
+      int row_lim;  // keys after this position are masked (kNoMask: none)
+      bool masked;  // warp-uniform: the causal mask applies to some row of the warp
+      if constexpr (GA) {
+        const GWork it = gwork_item(w, a);
+        const int lt = 2 * it.p + 1 - t, k = r / RPT, hh = r - k * RPT;
+        b = it.b;
+        h = it.g * G + hh;
+        nkv = lt * tpt < it.entries ? mt : 0;
+        row = k < tpt && hh < G ? gwork_token(a, it, lt * tpt + k, &slot) : -1;
+        key0 = it.j * a.blk;  // keys of the block's tiles start here
+        row_lim = row >= 0 && row / a.blk == it.j ? row : kNoMask;  // the block's own tokens only
+        masked = __any_sync(0xffffffffu, row_lim != kNoMask);
+      } else {
+        const Work it = work_item(w, a.B, a.Hq, npairs);
+        const int qt = 2 * it.pair + t;
+        b = it.b;
+        h = it.h;
+        nkv = qt + 1;
+        row = qt * BQ + r;
+        row_lim = row;
+        masked = false;
       }
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv; ++j, ++sit) {
         if (!mbar_wait(&s_full[t], sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
-        const bool diag = !RC && (j == nkv - 1);
-        bool keep = true;  // RC: this key tile belongs to one of the row's recalled blocks
-        if (RC) {
-          keep = false;
-          const int* rec = srec + (t * BQ + r) * MAX_RECALL_RC;
-          for (int q = 0; q < my_cnt; ++q) keep |= (rec[q] == j / mt);
-        }
-        const int lim = row - j * BKV;  // keys c > lim are in the future of this row
+        const bool diag = GA ? masked : (j == nkv - 1);
+        // keys c > lim of this tile are in the future of this row
+        const int lim = row_lim == kNoMask ? kNoMask : row_lim - (key0 + j * BKV);
         // pass 1: row maximum of the raw scores (four TMEM loads behind one wait; 3-input
         // max); only the diagonal tile needs the causal mask (a warp-uniform branch)
         float mx = -INFINITY;
@@ -380,7 +527,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         mx *= sl2;
-        if (RC && !keep) mx = -INFINITY;
         // lazy rescale: move the reference maximum only when it is exceeded by more than 2^8
         const bool need = mx > m_ref + RESCALE_THRESHOLD;
         float corr = 1.f;
@@ -412,10 +558,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (diag) {
               if (c * 32 + 2 * e > lim) p0 = 0.f;
               if (c * 32 + 2 * e + 1 > lim) p1 = 0.f;
-            }
-            if (RC && !keep) {
-              p0 = 0.f;
-              p1 = 0.f;
             }
             lsum2 = __fadd2_rn(lsum2, make_float2(p0, p1));
             __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
@@ -456,69 +598,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // epilogue: O_t / l -> bf16 -> global
       if (!mbar_wait(&o_full[t], wi & 1, abort, status)) break;
       tc_fence_after();
-      // RC: a row with no kept key (l == 0) adds nothing, and TMEM may then hold a stale tile
-      const bool has_o = !RC || l > 0.f;
-      const float inv = has_o ? 1.f / l : 0.f;
-      bf16* orow = (bf16*)a.o + (size_t)it.b * a.o_bstride + (size_t)row * a.o_ld + (size_t)it.h * DH;
-      float lam0 = 1.f, lam1 = 0.f, lam2 = 0.f;
-      const float* v2row = nullptr;
-      if (RC && row < a.S) {
-        const size_t tok = (size_t)it.b * a.S + row;
-        lam0 = a.lam[tok * 3];
-        lam1 = a.lam[tok * 3 + 1];
-        lam2 = a.lam[tok * 3 + 2];
-        v2row = a.v2 + tok * (size_t)(a.Hkv * DH) + (size_t)(it.h / G) * DH;
+      const float inv = 1.f / l;
+      // causal: row `row` of the output; MODE 1: slot `slot` of the token's partial results
+      bf16* orow;
+      bool store;
+      if constexpr (GA) {
+        store = row >= 0;
+        const size_t ps = ((size_t)b * a.S + (store ? row : 0)) * a.nslot + slot;
+        orow = (bf16*)a.part_o + ps * (size_t)(a.Hq * DH) + (size_t)h * DH;
+        if (store) a.part_lse[ps * a.Hq + h] = m_ref + __log2f(l);
+      } else {
+        store = row < a.S;
+        orow = (bf16*)a.o + (size_t)b * a.o_bstride + (size_t)row * a.o_ld + (size_t)h * DH;
       }
 #pragma unroll
-      for (int c = 0; c < DH; c += 32) {
-        uint32_t ov[32];
-        tmem_ld32(o_tmem + c, ov);
+      for (int c = 0; c < DH; c += 64) {  // two TMEM loads behind one wait
+        uint32_t ov[2][32];
+        tmem_ld32(o_tmem + c, ov[0]);
+        tmem_ld32(o_tmem + c + 32, ov[1]);
         tmem_ld_wait();
-        if (row < a.S) {
-          if (RC) {
-            // lam0 * causal output + lam1 * L2 value + lam2 * recalled-block output, 16 columns at a
-            // time with that half's loads issued together (the stores would otherwise order them)
+        if (store) {
+          // 16 columns (one full 32-byte sector) per store into the workspace's partials; 8 into o
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int c0 = c + hh * 16;
-              uint4 o1[2];
-              float4 v2c[4];
+          for (int v = 0; v < 4; ++v) {
+            uint32_t wv[8];
 #pragma unroll
-              for (int v = 0; v < 2; ++v) o1[v] = *(const uint4*)(orow + c0 + v * 8);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) v2c[v] = *(const float4*)(v2row + c0 + v * 4);
-#pragma unroll
-              for (int v = 0; v < 2; ++v) {
-                uint4 u;
-                uint32_t* wv = (uint32_t*)&u;
-                const uint32_t* o1w = (const uint32_t*)&o1[v];
-                const float v2e[8] = {v2c[2 * v].x, v2c[2 * v].y, v2c[2 * v].z, v2c[2 * v].w,
-                                      v2c[2 * v + 1].x, v2c[2 * v + 1].y, v2c[2 * v + 1].z, v2c[2 * v + 1].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int k = hh * 16 + v * 8 + 2 * e;
-                  const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&o1w[e]);
-                  const float x0 = has_o ? __uint_as_float(ov[k]) * inv : 0.f;
-                  const float x1 = has_o ? __uint_as_float(ov[k + 1]) * inv : 0.f;
-                  __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(lam0, f1.x, fmaf(lam1, v2e[2 * e], lam2 * x0)),
-                                                            fmaf(lam0, f1.y, fmaf(lam1, v2e[2 * e + 1], lam2 * x1)));
-                  wv[e] = *(uint32_t*)&hb;
-                }
-                *(uint4*)(orow + c0 + v * 8) = u;
-              }
+            for (int e = 0; e < 8; ++e) {
+              __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(ov[v >> 1][(v & 1) * 16 + 2 * e]) * inv,
+                                                        __uint_as_float(ov[v >> 1][(v & 1) * 16 + 2 * e + 1]) * inv);
+              wv[e] = *(uint32_t*)&hb;
             }
-          } else {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 u;
-              uint32_t* wv = (uint32_t*)&u;
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(ov[v * 8 + 2 * e]) * inv,
-                                                          __uint_as_float(ov[v * 8 + 2 * e + 1]) * inv);
-                wv[e] = *(uint32_t*)&hb;
-              }
-              *(uint4*)(orow + c + v * 8) = u;
+            if constexpr (GA) {
+              st_global_v8(orow + c + v * 16, wv);
+            } else {
+              *(uint4*)(orow + c + v * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+              *(uint4*)(orow + c + v * 16 + 8) = make_uint4(wv[4], wv[5], wv[6], wv[7]);
             }
           }
         }
@@ -540,6 +654,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace tca
 
+template <int DH, int MODE>
+cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
+                        int* status, int grid, cudaStream_t s) {
+  constexpr int sm = tca::Cfg<DH>::SMEM + (MODE ? tca::Cfg<DH>::GATHER_BYTES : 0);
+  cudaError_t e = set_max_smem(tca::attn_tc_kernel<DH, MODE>, sm, s);
+  if (e != cudaSuccess) return e;
+  tca::attn_tc_kernel<DH, MODE><<<grid, tca::NTHREADS, sm, s>>>(tq, tk, tv, a, status);
+  return cudaGetLastError();
+}
+
 cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s) {
   if (a.B <= 0 || a.S <= 0) return cudaSuccess;
   if ((a.dh != 64 && a.dh != 128) || (a.q_ld % 8) || (a.kv_ld % 8) || (a.o_ld % 8) || (a.q_bstride % a.q_ld) ||
@@ -548,8 +672,18 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
   const long long q_rows = (long long)a.B * (a.q_bstride / a.q_ld);
   const long long kv_rows = (long long)a.B * (a.kv_bstride / a.kv_ld);
   if (q_rows >= (1LL << 31) || kv_rows >= (1LL << 31)) return cudaErrorInvalidValue;
+  const bool ga = a.g_pairoff != nullptr;
+  // MODE 1 gathers query rows from q viewed as [B*S*Hq][dh], one-row boxes (q must be dense)
+  if (ga && (a.q_ld != a.Hq * a.dh || a.q_bstride != (long long)a.S * a.q_ld ||
+             (long long)a.B * a.S * a.Hq >= (1LL << 31)))
+    return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
-  cudaError_t e = make_tmap_bf16(&tq, a.q, (int)q_rows, a.Hq * a.dh, a.q_ld, tca::BQ);
+  cudaError_t e;
+  if (!ga) e = make_tmap_bf16(&tq, a.q, (int)q_rows, a.Hq * a.dh, a.q_ld, tca::BQ);
+  else if (gathered_rows_per_token(a.Hq / a.Hkv) == 8)  // [B*S][Hq][dh], boxes of 8 heads
+    e = make_tmap_bf16_3d(&tq, a.q, a.dh, a.Hq, a.B * a.S, a.dh, a.q_ld, 8);
+  else  // [B*S*Hq][dh], one-row boxes for tile::gather4
+    e = make_tmap_bf16(&tq, a.q, a.B * a.S * a.Hq, a.dh, a.dh, 1);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&tk, a.k, (int)kv_rows, a.Hkv * a.dh, a.kv_ld, tca::BKV);
   if (e != cudaSuccess) return e;
@@ -558,36 +692,17 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (ga && (((uintptr_t)a.part_o & 31) || !a.g_nrec || !a.g_pairbj || !a.g_recoff || !a.g_list || !a.part_o || !a.part_lse || a.nblk < 1 || a.nslot < 1 ||
+             a.blk < tca::BKV || a.blk % tca::BKV || a.Hq % a.Hkv || a.Hq / a.Hkv > tca::BQ ||
+             (long long)a.nblk * a.blk < a.S))
+    return cudaErrorInvalidValue;
+  // MODE 1: the item count is on the device (block_lists); idle CTAs leave at once
   const int nqt = (a.S + tca::BQ - 1) / tca::BQ;
   const int nwork = a.B * a.Hq * ((nqt + 1) / 2);
-  const int grid = nwork < sms ? nwork : sms;
-  if (a.ridx && (!a.rcnt || !a.lam || !a.v2 || a.R < 1 || a.R > tca::MAX_RECALL_RC || a.blk < tca::BKV ||
-                 a.blk % tca::BKV))
-    return cudaErrorInvalidValue;
-  if (a.dh == 128) {
-    if (a.ridx) {
-      constexpr int sm = tca::Cfg<128>::SMEM + tca::Cfg<128>::REC_BYTES;
-      e = set_max_smem(tca::attn_tc_kernel<128, true>, sm, s);
-      if (e != cudaSuccess) return e;
-      tca::attn_tc_kernel<128, true><<<grid, tca::NTHREADS, sm, s>>>(tq, tk, tv, a, status);
-    } else {
-      e = set_max_smem(tca::attn_tc_kernel<128, false>, tca::Cfg<128>::SMEM, s);
-      if (e != cudaSuccess) return e;
-      tca::attn_tc_kernel<128, false><<<grid, tca::NTHREADS, tca::Cfg<128>::SMEM, s>>>(tq, tk, tv, a, status);
-    }
-  } else {
-    if (a.ridx) {
-      constexpr int sm = tca::Cfg<64>::SMEM + tca::Cfg<64>::REC_BYTES;
-      e = set_max_smem(tca::attn_tc_kernel<64, true>, sm, s);
-      if (e != cudaSuccess) return e;
-      tca::attn_tc_kernel<64, true><<<grid, tca::NTHREADS, sm, s>>>(tq, tk, tv, a, status);
-    } else {
-      e = set_max_smem(tca::attn_tc_kernel<64, false>, tca::Cfg<64>::SMEM, s);
-      if (e != cudaSuccess) return e;
-      tca::attn_tc_kernel<64, false><<<grid, tca::NTHREADS, tca::Cfg<64>::SMEM, s>>>(tq, tk, tv, a, status);
-    }
-  }
-  return cudaGetLastError();
+  const int grid = ga ? sms : (nwork < sms ? nwork : sms);
+  if (a.dh == 128)
+    return ga ? launch_attn<128, 1>(tq, tk, tv, a, status, grid, s) : launch_attn<128, 0>(tq, tk, tv, a, status, grid, s);
+  return ga ? launch_attn<64, 1>(tq, tk, tv, a, status, grid, s) : launch_attn<64, 0>(tq, tk, tv, a, status, grid, s);
 }
 
 }  // namespace mka

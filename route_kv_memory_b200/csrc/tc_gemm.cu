@@ -428,6 +428,21 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int col
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 3-D bf16 tensor [d2][d1][d0] (d0 contiguous, strides s1, s2 elements), box {64, box1, 1}, 128B swizzle.
+cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, int d0, int d1, int d2, long long s1, long long s2,
+                              int box1) {
+  auto fn = tcg::encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t gdim[3] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2};
+  cuuint64_t gstride[2] = {(cuuint64_t)s1 * 2, (cuuint64_t)s2 * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t gemm_tn_bf16_tc(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
                             int* status, cudaStream_t s) {
   if (M <= 0 || N <= 0) return cudaSuccess;

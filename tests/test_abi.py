@@ -73,7 +73,7 @@ def test_sizes(mka):
 @pytest.mark.parametrize("field,value", [
     ("d_head", 96), ("n_kv_heads", 5), ("hash_bits", 33), ("recall_r", 0), ("router_hidden", 12), ("d_model", 100),
     ("dtype", 7), ("block_size", 0), ("batch", 0), ("route_mode", 4), ("route_mode", -1), ("tiers", 8),
-    ("attention_paths", 2), ("attention_paths", 4),
+    ("attention_paths", 2), ("attention_paths", 4), ("block_sparse", 2),
 ])
 def test_bad_configs_size_zero(mka, field, value):
     c = qwen_cfg(mka, **{field: value})
@@ -85,8 +85,8 @@ def test_routing_fields_follow_attn_scale(mka):
     """The routing fields were appended to mka_config; the earlier fields keep their offsets, and a
     zero-initialised tiers field selects all three tiers (the published layer)."""
     fields = [f[0] for f in mka.mka_config._fields_]
-    assert fields[-4:] == ["attn_scale", "route_mode", "tiers", "attention_paths"]
-    assert ctypes.sizeof(mka.mka_config) == 16 * 4
+    assert fields[-5:] == ["attn_scale", "route_mode", "tiers", "attention_paths", "block_sparse"]
+    assert ctypes.sizeof(mka.mka_config) == 17 * 4
     for mode in range(4):
         for tiers in range(8):
             assert mka.mka_workspace_size(qwen_cfg(mka, route_mode=mode, tiers=tiers)) > 0
@@ -97,6 +97,8 @@ def test_full_mka_limits(mka):
     assert mka.mka_workspace_size(qwen_cfg(mka, attention_paths=3)) > mka.mka_workspace_size(qwen_cfg(mka))
     assert mka.mka_workspace_size(qwen_cfg(mka, attention_paths=3, block_size=64)) == 0
     assert mka.mka_workspace_size(qwen_cfg(mka, attention_paths=3, dtype=mka.MKA_F32)) == 0
+    assert mka.mka_workspace_size(qwen_cfg(mka, block_sparse=1)) > 0
+    assert mka.mka_workspace_size(qwen_cfg(mka, block_sparse=1, attention_paths=3)) == 0
 
 
 def test_host_side_errors_before_any_device_call(mka):
@@ -116,6 +118,11 @@ def test_host_side_errors_before_any_device_call(mka):
     assert lib.mka_session_ema(ctypes.byref(c), a, None, a, None, a, 16, None) == mka.MKA_ERR_WORKSPACE
     assert lib.mka_decode_step(ctypes.byref(qwen_cfg(mka, batch=9)), a, a, 1 << 40, 16, a, a, a, 1 << 40,
                                None) == mka.MKA_ERR_UNSUPPORTED
+    # the gathered attention (block-sparse, full MKA) writes its partials 32 bytes at a time
+    for kw in ({"block_sparse": 1}, {"attention_paths": 3}):
+        assert lib.mka_prefill_forward(ctypes.byref(qwen_cfg(mka, **kw)), a, a, a, None, None, None, 0, 0,
+                                       ctypes.c_void_p(0x1010), 1 << 40, None) == mka.MKA_ERR_INVALID_ARG
+        assert b"32-byte" in lib.mka_last_error()
 
 
 def test_product_path_has_no_fallback():

@@ -162,6 +162,8 @@ MKA_CASES = [
     small("mka_dh64", "bf16", seq=520, d_head=64, n_q_heads=6, n_kv_heads=2, block=128, recall_r=3, seed=74,
           attention_paths=3),
     small("mka_no_l3", "bf16", seq=400, d_head=128, block=128, recall_r=2, seed=75, attention_paths=3, tiers=3),
+    small("mka_g7_boxes", "bf16", seq=700, d_head=128, n_q_heads=14, n_kv_heads=2, block=128, recall_r=4, seed=76,
+          attention_paths=3),
 ]
 
 
@@ -197,6 +199,47 @@ def test_full_mka_qwen7b_4k_rows():
     check_recall(idx, ref)
     max_abs, rel = check_out(out, ref["O"], "bf16", rows=rows)
     print(f"full MKA qwen7b_4k: O rel-L2 {rel:.2e} max-abs {max_abs:.2e}")
+
+
+# ------------------------------------------------------------------ Block-MKA block-sparse attention
+BS_CASES = [
+    small("bs_b128", "bf16", seq=700, d_head=128, n_q_heads=8, n_kv_heads=2, router_hidden=128, block=128,
+          recall_r=2, hash_bits=32, seed=81, block_sparse=1),
+    small("bs_b256_pairs", "bf16", batch=2, seq=900, d_head=128, n_q_heads=4, n_kv_heads=1, block=256, recall_r=2,
+          hash_bits=32, seed=82, block_sparse=1),
+    small("bs_all_recalled", "bf16", seq=520, d_head=128, block=128, recall_r=8, seed=83, block_sparse=1),
+    small("bs_dh64_no_l3", "bf16", seq=400, d_head=64, n_q_heads=6, n_kv_heads=2, block=128, recall_r=3, seed=84,
+          block_sparse=1, tiers=3),
+    # 4 < G <= 8: each token's query heads come in as one 8-row TMA box (G = 7 and G = 5, the last
+    # group's box running past the last head)
+    small("bs_g7_boxes", "bf16", batch=2, seq=650, d_head=128, n_q_heads=14, n_kv_heads=2, block=128, recall_r=3,
+          hash_bits=32, seed=85, block_sparse=1),
+    small("bs_g5_dh64_b256", "bf16", seq=800, d_head=64, n_q_heads=10, n_kv_heads=2, block=256, recall_r=2,
+          seed=86, block_sparse=1),
+]
+
+
+@pytest.mark.parametrize("cfg", BS_CASES, ids=[c.name for c in BS_CASES])
+def test_block_sparse_layer(cfg):
+    inp = make_inputs(cfg)
+    ref = oracle_prefill(cfg, inp)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    if cfg.tiers & 4:
+        check_recall(idx, ref)
+    check_out(out, ref["O"], "bf16")
+
+
+def test_block_sparse_qwen7b_4k_rows():
+    cfg = CONFIGS["qwen7b_4k"].replace(block_sparse=1)
+    inp = make_inputs(cfg)
+    rows = sample_rows(cfg.seq, cfg.block, max_rows=48)
+    ref = oracle_prefill(cfg, inp, rows=rows)
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    check_recall(idx, ref)
+    max_abs, rel = check_out(out, ref["O"], "bf16", rows=rows)
+    print(f"block-sparse qwen7b_4k: O rel-L2 {rel:.2e} max-abs {max_abs:.2e}")
 
 
 # ------------------------------------------------------------------ entry points one by one
