@@ -219,12 +219,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
       }
+      // An item's block and the tokens of its two tiles are looked up while the previous item's
+      // copies are in flight: lane k < tpt holds the token of slot k (8-row slots), and the
+      // tokens of all tpt entries go to stok (gather4).
+      GWork it;
+      int tk[2] = {-1, -1};
+      auto lookup = [&](int w) {
+        it = gwork_item(w, a);
+        for (int t = 0; t < 2; ++t) {
+          const int e0 = (2 * it.p + 1 - t) * tpt;
+          tk[t] = -1;
+          if (e0 >= it.entries) continue;
+          int slot;
+          if (lane < tpt) tk[t] = gwork_token(a, it, e0 + lane, &slot);
+          if (RPT != 8)
+            for (int k = lane; k < tpt; k += 32)
+              stok[t * BQ + k] = k == lane ? tk[t] : gwork_token(a, it, e0 + k, &slot);
+        }
+      };
       int kvit = 0;
+      int w = snake_item(0, gridDim.x, blockIdx.x, nwork);
+      if (w >= 0) lookup(w);
       for (int rr = 0; rr * (int)gridDim.x < nwork; ++rr) {
-        const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
         if (w < 0) break;
         const int wi = rr;
-        const GWork it = gwork_item(w, a);
         // the block's K/V first: its stages free up earlier than the query tiles
         bool ok = true;
         if (lane == 0) {
@@ -246,18 +264,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         bool qok = true;
         for (int t = 0; t < 2; ++t) {
-          const int lt = 2 * it.p + 1 - t;
-          const bool full = lt * tpt < it.entries;
-          int tok = -1;  // token of slot `lane` (8-row slots) or of entry `lane` (gather4)
-          if (full && lane < tpt) {
-            int slot;
-            tok = gwork_token(a, it, lt * tpt + lane, &slot);
-          }
-          if (RPT != 8 && full)
-            for (int k = lane; k < tpt; k += 32) {
-              int slot;
-              stok[t * BQ + k] = k == lane ? tok : gwork_token(a, it, lt * tpt + k, &slot);
-            }
+          const bool full = (2 * it.p + 1 - t) * tpt < it.entries;
+          const int tok = tk[t];
           const bool ok_t = mbar_wait(&q_empty[t], (wi & 1) ^ 1, abort, status);
           if (!__all_sync(0xffffffffu, ok_t)) {
             qok = false;
@@ -282,8 +290,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 const int r = 4 * lane + u, k = r / G;
-                const int tk = k < tpt ? stok[t * BQ + k] : -1;
-                rows[u] = tk >= 0 ? (it.b * a.S + tk) * a.Hq + it.g * G + (r - k * G) : row0;
+                const int tr = k < tpt ? stok[t * BQ + k] : -1;
+                rows[u] = tr >= 0 ? (it.b * a.S + tr) * a.Hq + it.g * G + (r - k * G) : row0;
               }
 #pragma unroll
               for (int hb = 0; hb < NH; ++hb)
@@ -295,6 +303,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           __syncwarp();
         }
+        if (!qok) break;
+        w = snake_item(rr + 1, gridDim.x, blockIdx.x, nwork);
+        if (w >= 0) lookup(w);
       }
       if (lane == 0 && *abort) {  // let issued copies land (bounded) before unwinding
         const unsigned long long t0 = globaltimer();
