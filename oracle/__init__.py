@@ -21,3 +21,7 @@ from .fastmka import (  # noqa: F401
     recalled_block_attention, mka_full_prefill, block_sparse_gqa_attention,
     EXCUSE_EPS,
 )
+from .backward import (  # noqa: F401
+    fastmka_backward, causal_gqa_attention_backward, session_ema_backward, longterm_recall_backward,
+    route_gate_backward, gelu_erf_grad,
+)

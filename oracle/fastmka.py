@@ -310,7 +310,7 @@ def weights_f64(w_q, w_k, w_v, w_r1, w_r2, P) -> Weights64:
 
 def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray] = None,
                     lam_override: Optional[np.ndarray] = None, row_chunk: int = 8192,
-                    keep_d_space: bool = False) -> dict:
+                    keep_d_space: bool = False, recall_fixed: Optional[tuple] = None) -> dict:
     """The FastMKA layer forward over whole sequences, in page order.
 
     X: [B, S, d] (any float dtype; widened to float64 a chunk of rows at a time).
@@ -321,6 +321,8 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
     attention is Block-MKA's block-sparse one (block_sparse_gqa_attention).
     Rows are processed in chunks only to bound memory; the EMA state is carried
     across chunks, so every value is the one the unchunked recurrence gives.
+    recall_fixed = (idx [B,S,R], count [B,S]) replaces the hash selection by the given recalled
+    blocks (M3 is still their mean): the discrete recall held fixed, as a gradient treats it.
     """
     B, S, d = X.shape
     Hq, Hkv, dh = cfg.n_q_heads, cfg.n_kv_heads, cfg.d_head
@@ -368,6 +370,11 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
             M2, m2 = session_ema(xc, cfg.alpha, m2)
             pos = np.arange(r0, r1)
             idx, cnt, M3, exc, xcodes, xproj = longterm_recall(xc[0], pos, summ, w.P, b, R, s_proj)
+            if recall_fixed is not None:
+                idx = np.asarray(recall_fixed[0][bi, r0:r1], np.int64)
+                cnt = np.asarray(recall_fixed[1][bi, r0:r1], np.int64)
+                M3 = np.array([summ[idx[i, :cnt[i]]].mean(axis=0) if cnt[i] else np.zeros(d)
+                               for i in range(r1 - r0)]).reshape(r1 - r0, d)
             Xf = fuse_sources(lam, xc[0], M2[0], M3)
             Kc, Vc = kv_project(Xf, w.w_k, w.w_v)
             out["lam"][bi, r0:r1] = lam
