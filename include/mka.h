@@ -193,6 +193,31 @@ MKA_API int mka_prefill_forward(const mka_config* cfg, const void* packed, const
                         int32_t* recall_idx_out, void* state, size_t state_bytes, int32_t max_positions,
                         void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- training (layer backward)
+ * Gradients of L = sum(dout * out) of the FastMKA prefill forward with respect to x and the trained
+ * weights W_q, W_k, W_v, W_r1, W_r2 (notes §1-§4 differentiated step by step).  The L3 recall is a
+ * discrete selection and is held fixed (straight-through): gradients reach x through the recalled
+ * block means, not through the choice of blocks; the hash projection P is not trained.  The
+ * routing gate passes gradient through its softmax (soft: over the active tiers; hard top-2: over
+ * its two chosen logits); fixed and hard top-1 weights pass none.
+ * Supported: bf16 FastMKA (attention_paths 1, block_sparse 0), router_hidden % 32 == 0 and <= 512;
+ * otherwise MKA_ERR_UNSUPPORTED (mka_train_workspace_size returns 0).
+ * Workspace: mka_train_workspace_size(cfg) bytes, 32-byte aligned, shared by the two calls below. */
+MKA_API size_t mka_train_workspace_size(const mka_config* cfg);
+/* The prefill forward (as mka_prefill_forward without optional outputs or state) that also keeps
+ * the attention's per-row softmax normaliser and leaves in ws every activation the backward reads.
+ * x [B, S, d] bf16 -> out [B, S, Hq*dh] bf16. */
+MKA_API int mka_prefill_forward_train(const mka_config* cfg, const void* packed, const void* x, void* out, void* ws,
+                                      size_t ws_bytes, void* stream);
+/* The layer backward.  Must follow mka_prefill_forward_train of the same cfg, x and packed weights
+ * on the same stream with ws untouched in between; out is that call's output.  dout [B, S, Hq*dh]
+ * bf16 -> dx [B, S, d] bf16 and float32 dw_q [d, dq], dw_k [d, dkv], dw_v [d, dkv], dw_r1 [dq, rh],
+ * dw_r2 [rh, 3] (overwritten, the weights' layouts of mka_weights); dlambda_out [B*S, 3] float32
+ * (nullable) <- dL/dlambda.  All device pointers, 16-byte aligned. */
+MKA_API int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* x, const void* out,
+                                 const void* dout, void* dx, float* dw_q, float* dw_k, float* dw_v, float* dw_r1,
+                                 float* dw_r2, float* dlambda_out, void* ws, size_t ws_bytes, void* stream);
+
 /* One decode step for the next token of each sequence (notes §3: the cache holds the
  * fused routed K/V).  x_new [B, d] (dtype) -> out [B, Hq*dh] (dtype).  Runs the
  * router, reads M2 and recalls from the finished blocks, appends the fused K/V row

@@ -41,7 +41,8 @@ EXPORTED = [
     "mka_longterm_recall_workspace_size", "mka_state_size", "mka_decode_workspace_size", "mka_pack_weights",
     "mka_state_init", "mka_router", "mka_session_ema", "mka_longterm_recall", "mka_prefill_forward",
     "mka_decode_step", "mka_status", "mka_last_error", "mka_version", "mka_profile_enable", "mka_profile_read",
-    "mka_session_ema_noalloc", "mka_selftest_wait_timeout",
+    "mka_session_ema_noalloc", "mka_selftest_wait_timeout", "mka_train_workspace_size", "mka_prefill_forward_train",
+    "mka_prefill_backward",
 ]
 
 
@@ -76,6 +77,10 @@ _SIGS = {
     "mka_longterm_recall": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mka_prefill_forward": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i32, _vp, _sz, _vp]),
     "mka_decode_step": (ctypes.c_int, [_cfgp, _vp, _vp, _sz, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "mka_train_workspace_size": (_sz, [_cfgp]),
+    "mka_prefill_forward_train": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mka_prefill_backward": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                            _vp]),
     "mka_status": (ctypes.c_int, []),
     "mka_last_error": (ctypes.c_char_p, []),
     "mka_version": (ctypes.c_char_p, []),
@@ -201,6 +206,23 @@ def mka_prefill_forward(c: mka_config, packed, x, out, lambda_out, recall_idx_ou
                                     ws.numel() * ws.element_size(), _stream(stream)), "mka_prefill_forward")
 
 
+def mka_train_workspace_size(c: mka_config) -> int:
+    return _lib.mka_train_workspace_size(ctypes.byref(c))
+
+
+def mka_prefill_forward_train(c: mka_config, packed, x, out, ws, stream=None) -> None:
+    _check(_lib.mka_prefill_forward_train(ctypes.byref(c), _ptr(packed), _ptr(x), _ptr(out), _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream)), "mka_prefill_forward_train")
+
+
+def mka_prefill_backward(c: mka_config, packed, x, out, dout, dx, dw_q, dw_k, dw_v, dw_r1, dw_r2, dlambda_out, ws,
+                         stream=None) -> None:
+    _check(_lib.mka_prefill_backward(ctypes.byref(c), _ptr(packed), _ptr(x), _ptr(out), _ptr(dout), _ptr(dx),
+                                     _ptr(dw_q), _ptr(dw_k), _ptr(dw_v), _ptr(dw_r1), _ptr(dw_r2), _ptr(dlambda_out),
+                                     _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "mka_prefill_backward")
+
+
 def mka_decode_step(c: mka_config, packed, state, max_positions: int, x_new, out, ws, stream=None) -> None:
     _check(_lib.mka_decode_step(ctypes.byref(c), _ptr(packed), _ptr(state), state.numel() * state.element_size(),
                                 max_positions, _ptr(x_new), _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
@@ -264,6 +286,27 @@ class FastMKALayer:
         mka_prefill_forward(c, self.packed, x, out, lambda_out, recall_idx_out, state, max_positions,
                             self.workspace(c), stream)
         return out
+
+    def train_workspace(self, c: mka_config) -> torch.Tensor:
+        key = ("train", c.batch, c.seq)
+        if key not in self._ws:
+            self._ws[key] = buffer(mka_train_workspace_size(c), self.device)
+        return self._ws[key]
+
+    def forward_train(self, x: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+        """The prefill forward, keeping in this layer's training workspace what backward() reads."""
+        c = make_config(self.cfg, seq=x.shape[1], batch=x.shape[0])
+        mka_prefill_forward_train(c, self.packed, x, out, self.train_workspace(c), stream)
+        return out
+
+    def backward(self, x: torch.Tensor, out: torch.Tensor, dout: torch.Tensor, grads: dict, dlambda_out=None,
+                 stream=None) -> dict:
+        """Gradients of sum(dout * out) after forward_train(x, out) on the same stream: grads holds
+        dx (like x) and float32 dw_q, dw_k, dw_v, dw_r1, dw_r2 in the weights' shapes."""
+        c = make_config(self.cfg, seq=x.shape[1], batch=x.shape[0])
+        mka_prefill_backward(c, self.packed, x, out, dout, grads["dx"], grads["dw_q"], grads["dw_k"], grads["dw_v"],
+                             grads["dw_r1"], grads["dw_r2"], dlambda_out, self.train_workspace(c), stream)
+        return grads
 
     def new_state(self, max_positions: int, batch: Optional[int] = None, stream=None) -> torch.Tensor:
         c = make_config(self.cfg, batch=batch)

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmka.so")
-SOURCES = ["api.cu", "gemm.cu", "memory.cu", "attention.cu", "decode.cu", "noalloc.cu", "tc_gemm.cu", "tc_attention.cu", "block_sparse.cu", "selftest.cu"]
+SOURCES = ["api.cu", "gemm.cu", "memory.cu", "attention.cu", "decode.cu", "noalloc.cu", "tc_gemm.cu", "tc_attention.cu", "block_sparse.cu", "tc_attention_bwd.cu", "backward.cu", "selftest.cu"]
 HEADERS = ["common.cuh", "kernels.h", "sm100.cuh"]
 
 NVCC_FLAGS = [

@@ -542,9 +542,11 @@ int mka_longterm_recall(const mka_config* cfg, const void* x, const void* hash_p
   return MKA_OK;
 }
 
-int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x, void* out, float* lambda_out,
-                        int32_t* recall_idx_out, void* state, size_t state_bytes, int32_t max_positions, void* ws,
-                        size_t ws_bytes, void* stream) {
+// The prefill forward; lse (nullable) receives the attention's per-row log2 normaliser,
+// [B*Hq][S rounded up to 128], for the backward.
+static int prefill_forward(const mka_config* cfg, const void* packed, const void* x, void* out, float* lambda_out,
+                           int32_t* recall_idx_out, void* state, size_t state_bytes, int32_t max_positions, void* ws,
+                           size_t ws_bytes, void* stream, float* lse) {
   Dims d;
   int rc = check_cfg(cfg, &d);
   if (rc) return rc;
@@ -697,6 +699,10 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   aa.k = kbuf; aa.v = vbuf; aa.kv_bstride = kv_bstride; aa.kv_ld = d.dkv;
   aa.o = out; aa.o_bstride = (long long)d.S * d.dq; aa.o_ld = d.dq;
   aa.B = d.B; aa.S = d.S; aa.Hq = d.Hq; aa.Hkv = d.Hkv; aa.dh = d.dh; aa.scale = d.scale;
+  if (lse) {
+    aa.lse = lse;
+    aa.lse_ld = (d.S + 127) / 128 * 128;
+  }
   if (!d.block_sparse) {
     if (d.bf16) CUDA_TRY(attention_prefill_tc(aa, status_ptr(), s));
     else CUDA_TRY(attention_prefill(aa, 0, s));
@@ -734,6 +740,224 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
   } else if (state) {
     CUDA_TRY(k_tail(s));
     STAGE(s);
+  }
+  return MKA_OK;
+}
+
+int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x, void* out, float* lambda_out,
+                        int32_t* recall_idx_out, void* state, size_t state_bytes, int32_t max_positions, void* ws,
+                        size_t ws_bytes, void* stream) {
+  return prefill_forward(cfg, packed, x, out, lambda_out, recall_idx_out, state, state_bytes, max_positions, ws,
+                         ws_bytes, stream, nullptr);
+}
+
+// ---------------------------------------------------------------- training: forward + backward
+// The training workspace is the prefill workspace (whose activations the backward reads: q, the
+// projected sources, lambda, the EMA carries, the block sums, the recall, the fused K/V) followed
+// by the attention normalisers the training forward writes and the backward's own scratch.
+struct TrainWs {
+  PrefillWs fw;
+  int Spad, Tp, ncat, nball;
+  size_t lse, dsum, dq, dy, ema, m3, hrec, dlam, dh, dqr, gsum, rsum, cs, acat, wcatT, wr1, xT, acatT, qT, dhT;
+  size_t nrec, recoff, cursor, pairoff, pairbj, list, total;
+};
+static TrainWs train_ws(const Dims& d) {
+  TrainWs w;
+  w.fw = prefill_ws(d);
+  const size_t T = d.T, W = d.width;
+  w.Spad = (d.S + 127) / 128 * 128;
+  w.Tp = (int)((T + 7) / 8 * 8);  // K of the weight-gradient products, padded with zero columns
+  w.ncat = d.dq + 2 * d.dkv;      // [dq | U] columns
+  w.nball = (d.S + d.blk - 1) / d.blk;
+  const size_t nbj = (size_t)d.B * d.nblk;
+  size_t o = w.fw.total;
+  w.lse = o; o += al((size_t)d.B * d.Hq * w.Spad * 4);
+  w.dsum = o; o += al((size_t)d.B * d.Hq * w.Spad * 4);
+  w.dq = o; o += al(T * d.dq * 4);
+  w.dy = o; o += al(T * W * 4);
+  w.ema = o; o += al(T * W * 4);
+  w.m3 = o; o += al(T * W * 4);
+  w.hrec = o; o += al(T * 2 * d.rh * 4);
+  w.dlam = o; o += al(T * 3 * 4);
+  w.dh = o; o += al(T * d.rh * 2);
+  w.dqr = o; o += al(T * d.dq * 4);
+  w.gsum = o; o += al(nbj * W * 4);
+  w.rsum = o; o += al((size_t)d.B * w.nball * W * 4);
+  w.cs = o; o += al((size_t)d.B * (w.nball + 1) * W * 4);
+  w.acat = o; o += al(T * w.ncat * 2);
+  w.wcatT = o; o += al((size_t)d.d * w.ncat * 2);
+  w.wr1 = o; o += al((size_t)d.dq * d.rh * 2);
+  w.xT = o; o += al((size_t)d.d * w.Tp * 2);
+  w.acatT = o; o += al((size_t)w.ncat * w.Tp * 2);
+  w.qT = o; o += al((size_t)d.dq * w.Tp * 2);
+  w.dhT = o; o += al((size_t)d.rh * w.Tp * 2);
+  w.nrec = o; o += al(nbj * 4);
+  w.recoff = o; o += al(nbj * 4);
+  w.cursor = o; o += al(nbj * 4);
+  w.pairoff = o; o += al((nbj + 1) * 4);
+  w.pairbj = o; o += al(gathered_max_pairs(T, d.R, 0, 128, nbj) * 4);
+  w.list = o; o += al(T * d.R * 4);
+  w.total = o;
+  return w;
+}
+
+static int check_train(const mka_config* cfg, Dims* d) {
+  int rc = check_cfg(cfg, d);
+  if (rc) return rc;
+  if (!d->bf16 || d->paths != 1 || d->block_sparse)
+    return fail(MKA_ERR_UNSUPPORTED, "the layer backward needs bf16 FastMKA (attention_paths 1, no block_sparse)");
+  if (d->rh % 32 || d->rh > 512) return fail(MKA_ERR_UNSUPPORTED, "the layer backward needs router_hidden % 32 == 0, <= 512");
+  return MKA_OK;
+}
+
+size_t mka_train_workspace_size(const mka_config* cfg) {
+  Dims d;
+  if (check_cfg(cfg, &d) != MKA_OK || !d.bf16 || d.paths != 1 || d.block_sparse || d.rh % 32 || d.rh > 512) return 0;
+  return train_ws(d).total;
+}
+
+int mka_prefill_forward_train(const mka_config* cfg, const void* packed, const void* x, void* out, void* ws,
+                              size_t ws_bytes, void* stream) {
+  Dims d;
+  int rc = check_train(cfg, &d);
+  if (rc) return rc;
+  if (!ws) return fail(MKA_ERR_INVALID_ARG, "NULL pointer");
+  if ((uintptr_t)ws & 31) return fail(MKA_ERR_INVALID_ARG, "the training workspace must be 32-byte aligned");
+  TrainWs W = train_ws(d);
+  if (ws_bytes < W.total) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, W.total);
+  // rows past S of the last query tile keep a defined normaliser (the backward masks them)
+  CUDA_TRY(cudaMemsetAsync(P(ws, W.lse), 0, (size_t)d.B * d.Hq * W.Spad * 4, (cudaStream_t)stream));
+  return prefill_forward(cfg, packed, x, out, nullptr, nullptr, nullptr, 0, 0, ws, ws_bytes, stream,
+                         (float*)P(ws, W.lse));
+}
+
+int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* x, const void* out, const void* dout,
+                         void* dx, float* dw_q, float* dw_k, float* dw_v, float* dw_r1, float* dw_r2,
+                         float* dlambda_out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  int rc = check_train(cfg, &d);
+  if (rc) return rc;
+  if (!packed || !x || !out || !dout || !dx || !dw_q || !dw_k || !dw_v || !dw_r1 || !dw_r2 || !ws)
+    return fail(MKA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(packed) || !aligned16(x) || !aligned16(out) || !aligned16(dout) || !aligned16(dx) ||
+      !aligned16(dw_q) || !aligned16(dw_k) || !aligned16(dw_v) || !aligned16(dw_r1) || !aligned16(dw_r2) ||
+      (dlambda_out && !aligned16(dlambda_out)))
+    return fail(MKA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((uintptr_t)ws & 31) return fail(MKA_ERR_INVALID_ARG, "the training workspace must be 32-byte aligned");
+  TrainWs W = train_ws(d);
+  if (ws_bytes < W.total) return fail(MKA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, W.total);
+  PackLayout PL = pack_layout(d);
+  cudaStream_t s = (cudaStream_t)stream;
+  const PrefillWs& F = W.fw;
+  const size_t T = d.T;
+  const int wd = d.width;  // 2 dkv: [dK | dV], [X W_k | X W_v]
+  const bf16* wcat = (const bf16*)P((void*)packed, PL.wcat);
+  float* lse = (float*)P(ws, W.lse);
+  float* dsum = (float*)P(ws, W.dsum);
+  float* dq = (float*)P(ws, W.dq);
+  float* dy = (float*)P(ws, W.dy);
+  float* ema = (float*)P(ws, W.ema);
+  float* m3 = (float*)P(ws, W.m3);
+  float* hrec = (float*)P(ws, W.hrec);
+  float* dlam = dlambda_out ? dlambda_out : (float*)P(ws, W.dlam);
+  void* dh = P(ws, W.dh);
+  float* dqr = (float*)P(ws, W.dqr);
+  void* acat = P(ws, W.acat);
+  void* wcatT = P(ws, W.wcatT);
+  void* wr1 = P(ws, W.wr1);
+  const float* lam = (const float*)P(ws, F.lam);
+  const int* idx = (const int*)P(ws, F.idx);
+  const int* cnt = (const int*)P(ws, F.cnt);
+
+  // weights in the orientation of the backward products: [W_q | W_k | W_v] as [d][dq + 2 dkv], W_r1 as [dq][rh]
+  CUDA_TRY(transpose(wcat, W.ncat, d.d, d.d, wcatT, W.ncat, 2, 0, s));
+  CUDA_TRY(transpose(P((void*)packed, PL.wr1T), d.rh, d.dq, d.dq, wr1, d.rh, 2, 0, s));
+  // attention: D = rowsum(dO * O), then dQ and [dK | dV]
+  CUDA_TRY(cudaMemsetAsync(dsum, 0, (size_t)d.B * d.Hq * W.Spad * 4, s));
+  CUDA_TRY(attention_dsum(dout, out, d.B, d.S, d.Hq, d.dh, W.Spad, dsum, s));
+  AttnBwdArgs ab{};
+  ab.q = P(ws, F.q); ab.k = P(ws, F.k); ab.v = P(ws, F.v); ab.dout = dout;
+  ab.lse = lse; ab.dsum = dsum; ab.lse_ld = W.Spad;
+  ab.dq = dq; ab.dkv = dy;
+  ab.B = d.B; ab.S = d.S; ab.Hq = d.Hq; ab.Hkv = d.Hkv; ab.dh = d.dh; ab.scale = d.scale;
+  CUDA_TRY(attention_backward_tc(ab, status_ptr(), s));
+  // the router's pre-activation h = X (W_q W_r1) from its packed hi / lo rows
+  {
+    Epilogue ep{};
+    ep.nseg = 1;
+    ep.seg[0] = OutSeg{0, 2 * d.rh, hrec, 2 * d.rh, 0};
+    CUDA_TRY(gemm_tn_bf16_tc(x, d.d, wcat + (size_t)PL.seg_r * d.d, d.d, (int)T, 2 * d.rh, d.d, ep, status_ptr(), s));
+  }
+  // the L2 and L3 values of the projected sources, as the forward fused them
+  const float* xkv = (const float*)P(ws, F.xkv);
+  CUDA_TRY(ema_apply(xkv, 0, wd, d.B, d.S, d.nblk, d.blk, d.alpha, (const float*)P(ws, F.carry), ema, nullptr, s));
+  CUDA_TRY(gather_mean(idx, cnt, d.R, (const float*)P(ws, F.bsum), d.nblk, wd, d.blk, d.B, d.S, m3, s));
+  // gate and router MLP
+  CUDA_TRY(cudaMemsetAsync(dw_r2, 0, (size_t)d.rh * 3 * sizeof(float), s));
+  RouterBwdArgs rb{};
+  rb.dy = dy; rb.width = wd; rb.xkv = xkv; rb.ld_xkv = wd; rb.ema = ema; rb.m3 = m3;
+  rb.lam = lam; rb.dlam = dlam; rb.hrec = hrec; rb.rh = d.rh; rb.r_inter = PL.router_fused;
+  rb.w_r2 = (const float*)P((void*)packed, PL.wr2); rb.dh = dh; rb.dw_r2 = dw_r2;
+  rb.B = d.B; rb.S = d.S; rb.route_mode = d.route; rb.tiers = d.tiers;
+  CUDA_TRY(router_backward(rb, s));
+  // dq = dq (attention) + dh W_r1^T, into the first dq columns of [dq | U] (bf16)
+  {
+    Epilogue ep{};
+    ep.nseg = 1;
+    ep.seg[0] = OutSeg{0, d.dq, dqr, d.dq, 0};
+    CUDA_TRY(gemm_tn_bf16_tc(dh, d.rh, wr1, d.rh, (int)T, d.dq, d.rh, ep, status_ptr(), s));
+  }
+  CUDA_TRY(add_to_bf16(dq, dqr, (long long)T, d.dq, acat, W.ncat, s));
+  // U = lam1 dY + EMA^T(lam2 dY) + M^T(lam3 dY), into the last 2 dkv columns
+  {
+    int* nrec = (int*)P(ws, W.nrec);
+    int* recoff = (int*)P(ws, W.recoff);
+    int* list = (int*)P(ws, W.list);
+    if (d.nblk > 0)
+      CUDA_TRY(block_lists(idx, cnt, d.B, d.S, d.R, d.blk, d.nblk, 0, 0, 128, nrec, recoff, (int*)P(ws, W.cursor),
+                           (int*)P(ws, W.pairoff), (int*)P(ws, W.pairbj), list, s));
+    MemAdjArgs ma{};
+    ma.dy = dy; ma.width = wd; ma.lam = lam; ma.cnt = cnt; ma.nrec = nrec; ma.recoff = recoff; ma.list = list;
+    ma.B = d.B; ma.S = d.S; ma.nblk = d.nblk; ma.blk = d.blk; ma.alpha = d.alpha;
+    ma.gsum = (float*)P(ws, W.gsum); ma.rsum = (float*)P(ws, W.rsum); ma.cs = (float*)P(ws, W.cs);
+    ma.u = (bf16*)acat + d.dq; ma.ldu = W.ncat;
+    CUDA_TRY(memory_adjoint(ma, s));
+  }
+  // dX = [dq | U] [W_q | W_k | W_v]^T
+  {
+    Epilogue ep{};
+    ep.nseg = 1;
+    ep.seg[0] = OutSeg{0, d.d, dx, d.d, 1};
+    CUDA_TRY(gemm_tn_bf16_tc(acat, W.ncat, wcatT, W.ncat, (int)T, d.d, W.ncat, ep, status_ptr(), s));
+  }
+  // weight gradients: [dW_q | dW_k | dW_v] = X^T [dq | U], dW_r1 = q^T dh, with the token axis as K
+  void* xT = P(ws, W.xT);
+  void* acatT = P(ws, W.acatT);
+  void* qT = P(ws, W.qT);
+  void* dhT = P(ws, W.dhT);
+  if ((size_t)W.Tp != T) {  // zero K padding
+    CUDA_TRY(cudaMemsetAsync(xT, 0, (size_t)d.d * W.Tp * 2, s));
+    CUDA_TRY(cudaMemsetAsync(acatT, 0, (size_t)W.ncat * W.Tp * 2, s));
+    CUDA_TRY(cudaMemsetAsync(qT, 0, (size_t)d.dq * W.Tp * 2, s));
+    CUDA_TRY(cudaMemsetAsync(dhT, 0, (size_t)d.rh * W.Tp * 2, s));
+  }
+  CUDA_TRY(transpose(x, (int)T, d.d, d.d, xT, W.Tp, 2, 0, s));
+  CUDA_TRY(transpose(acat, (int)T, W.ncat, W.ncat, acatT, W.Tp, 2, 0, s));
+  CUDA_TRY(transpose(P(ws, F.q), (int)T, d.dq, d.dq, qT, W.Tp, 2, 0, s));
+  CUDA_TRY(transpose(dh, (int)T, d.rh, d.rh, dhT, W.Tp, 2, 0, s));
+  {
+    Epilogue ep{};
+    ep.nseg = 3;
+    ep.seg[0] = OutSeg{0, d.dq, dw_q, d.dq, 0};
+    ep.seg[1] = OutSeg{d.dq, d.dq + d.dkv, dw_k, d.dkv, 0};
+    ep.seg[2] = OutSeg{d.dq + d.dkv, W.ncat, dw_v, d.dkv, 0};
+    CUDA_TRY(gemm_tn_bf16_tc(xT, W.Tp, acatT, W.Tp, d.d, W.ncat, W.Tp, ep, status_ptr(), s));
+  }
+  {
+    Epilogue ep{};
+    ep.nseg = 1;
+    ep.seg[0] = OutSeg{0, d.rh, dw_r1, d.rh, 0};
+    CUDA_TRY(gemm_tn_bf16_tc(qT, W.Tp, dhT, W.Tp, d.dq, d.rh, W.Tp, ep, status_ptr(), s));
   }
   return MKA_OK;
 }

@@ -121,6 +121,9 @@ struct AttnArgs {
   void* o; long long o_bstride; int o_ld;
   int B, S, Hq, Hkv, dh;
   float scale;
+  // causal mode, when set: each row's softmax normaliser in log2 units, m + log2(l) with the
+  // scores taken as scale * log2(e) * q.k, at lse[(b * Hq + h) * lse_ld + t] (for the backward)
+  float* lse = nullptr; int lse_ld = 0;
   // Block-gathered attention (set g_pairoff to select it; bf16, tcgen05 only).  The rows of a
   // work item are (token, query head) pairs that all attend to the keys of one L3 block j of
   // sequence b: the tokens of block j's list (its own tokens first when g_own, under the causal
@@ -168,6 +171,49 @@ struct MergeArgs {
 // Combines each row's partial softmax results: w_s = 2^(lse_s - max lse), o = sum w_s O_s / sum w_s
 // (0 when the row has no slot).
 cudaError_t merge_partials(const MergeArgs& m, cudaStream_t s);
+
+// ---------------------------------------------------------------- layer backward
+// Causal GQA attention backward on tcgen05 (tc_attention_bwd.cu); every tensor dense, token-major.
+struct AttnBwdArgs {
+  const void* q; const void* k; const void* v; const void* dout;  // bf16 [B][S][Hq*dh], [B][S][Hkv*dh], dO like q
+  const float* lse; const float* dsum; int lse_ld;  // [B*Hq][lse_ld >= S rounded up to 128]: forward lse, rowsum(dO*O)
+  float* dq;   // [B][S][Hq*dh] float32, 32-byte aligned
+  float* dkv;  // [B][S][2*Hkv*dh] float32: dK then dV per row, 32-byte aligned
+  int B, S, Hq, Hkv, dh;
+  float scale;
+};
+cudaError_t attention_backward_tc(const AttnBwdArgs& a, int* status, cudaStream_t s);
+// dsum[(b * Hq + h) * ld + t] = sum_i dO * O over head h of token t (bf16 inputs).
+cudaError_t attention_dsum(const void* dout, const void* o, int B, int S, int Hq, int dh, int ld, float* dsum,
+                           cudaStream_t s);
+// Gate and router-MLP backward (backward.cu).
+struct RouterBwdArgs {
+  const float* dy; int width;        // [B*S][width] dK | dV
+  const float* xkv; int ld_xkv;      // the three projected sources: X [W_k | W_v] rows (stride ld_xkv),
+  const float* ema; const float* m3; //   their EMA and their recalled mean ([B*S][width])
+  const float* lam; float* dlam;     // [B*S][3]; dlam (nullable) <- dL/dlam
+  const float* hrec; int rh;         // [B*S][2 rh] router pre-activation as hi and lo parts
+  int r_inter;                       // 1: hi, lo interleaved per 128 hidden units; 0: all hi then all lo
+  const float* w_r2;                 // [rh][3]
+  void* dh;                          // [B*S][rh] bf16 <- dL/dh
+  float* dw_r2;                      // [rh][3] += GELU(h)^T dz (zero it first)
+  int B, S, route_mode, tiers;
+};
+cudaError_t router_backward(const RouterBwdArgs& a, cudaStream_t s);
+// U = lam1 dY + EMA^T(lam2 dY) + M^T(lam3 dY) in the projected space (backward.cu).
+struct MemAdjArgs {
+  const float* dy; int width; const float* lam; const int* cnt;
+  const int* nrec; const int* recoff; const int* list;  // recall lists of the full blocks (block_lists, own 0)
+  int B, S, nblk, blk;
+  float alpha;
+  float* gsum;  // [B][nblk][width] scratch
+  float* rsum;  // [B][ceil(S/blk)][width] scratch
+  float* cs;    // [B][ceil(S/blk)+1][width] scratch
+  void* u; int ldu;  // bf16 rows of U (stride ldu)
+};
+cudaError_t memory_adjoint(const MemAdjArgs& a, cudaStream_t s);
+// out[r][0:n] = bf16(x[r] + y[r]) for float32 rows of n (out row stride ldo).
+cudaError_t add_to_bf16(const float* x, const float* y, long long rows, int n, void* out, int ldo, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode
 struct DecodeArgs {

@@ -105,29 +105,12 @@ __device__ __forceinline__ int gwork_token(const AttnArgs& a, const GWork& it, i
   return t < a.S ? t : -1;
 }
 
-// MN-major (V) descriptor: 8-key groups of 128-B rows 1024 B apart (stride byte
-// offset), 64-column halves of the head dimension 16 KB apart (leading byte offset).
-__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(const void* tile) {
-  const uint64_t addr = smem_u32(tile);
-  uint64_t d = (addr >> 4) & 0x3FFFull;
-  d |= (uint64_t)(16384 >> 4) << 16;
-  d |= (uint64_t)(1024 >> 4) << 32;
-  d |= 1ull << 46;
-  d |= 2ull << 61;
-  return d;
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // MODE 0: causal attention; MODE 1: block-gathered rows (see the top of the file).
 template <int DH, int MODE>
@@ -621,6 +604,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       } else {
         store = row < a.S;
         orow = (bf16*)a.o + (size_t)b * a.o_bstride + (size_t)row * a.o_ld + (size_t)h * DH;
+        if (a.lse && store) a.lse[((size_t)b * a.Hq + h) * a.lse_ld + row] = m_ref + __log2f(l);
       }
 #pragma unroll
       for (int c = 0; c < DH; c += 64) {  // two TMEM loads behind one wait

@@ -1,0 +1,597 @@
+// Backward of the causal GQA attention on tcgen05 tensor cores (the layer's attention, MKA paper
+// notes §3; its online max-shift, §4, leaves each row's normaliser lse = m + log2(l), which the
+// forward keeps).  With P = 2^(s * scale * log2e - lse) recomputed from the scores and
+// D = rowsum(dO * O):
+//   dS = P * (dO V^T - D),  dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO,
+// dK and dV summed over the G = Hq / Hkv query heads of a KV group.  Two kernels, no atomics:
+//
+//   attn_bwd_dq_kernel    per (sequence, query head, 128-row query tile), streaming the key
+//                         tiles j <= its own: S = Q K_j^T and dP = dO V_j^T into TMEM, four warps
+//                         turn them into scale * dS (bf16, written over S), then dQ += dS K_j
+//                         with dS read from TMEM and K_j as an MN-major operand.
+//   attn_bwd_dkdv_kernel  per (sequence, KV group, 128-key tile), K and V staying in shared
+//                         memory while the query tiles t >= its own of all G heads stream through
+//                         a 2-stage ring (Q, dO and their lse and D rows): S^T = K Q^T and
+//                         dP^T = V dO^T into TMEM, four warps write P^T and scale * dS^T (bf16)
+//                         over them, then dV += P^T dO and dK += dS^T Q accumulate in TMEM.
+// Warp 0 loads (TMA), warp 1 issues the MMAs, warps 2-5 compute, one TMEM lane (row) each.
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace mka {
+
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows);
+
+namespace tcb {
+
+using namespace sm100;
+
+constexpr int BT = 128;  // rows of every tile (query and key)
+constexpr int NTHREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+
+template <int DH>
+struct Cfg {
+  static constexpr int NH = DH / 64;             // 64-column boxes per row
+  static constexpr int TILE = BT * DH * 2;       // one 128-row bf16 tile
+  static constexpr int HALF = BT * 64 * 2;       // one 128-row x 64-column swizzled box
+  static constexpr int VEC = BT * 4;             // 128 floats (lse or D of a query tile)
+  static constexpr int STAGE = 2 * TILE + 1024;  // dK/dV ring stage: Q, dO, lse, D (1024-aligned)
+  static constexpr int SMEM_DQ = 2 * TILE + 2 * 2 * TILE + 1024 + 256;
+  static constexpr int SMEM_DKDV = 2 * TILE + 2 * STAGE + 1024 + 256;
+};
+
+__device__ __forceinline__ int snake(int r, int grid, int cta, int nwork) {
+  const int w = r * grid + ((r & 1) ? grid - 1 - cta : cta);
+  return w < nwork ? w : -1;
+}
+
+// Offset of K-step kk (16 elements of the K dimension) in a K-major 128B-swizzled tile descriptor.
+__device__ __forceinline__ uint64_t kstep(int kk, int half_bytes) {
+  return (uint64_t)((kk >> 2) * (half_bytes >> 4) + (kk & 3) * 2);
+}
+
+// scale * dS (or P) for 32 columns, packed as bf16 pairs.
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *(uint32_t*)&h;
+}
+
+// ============================================================================ dQ
+template <int DH>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       AttnBwdArgs a, int* status) {
+  using C = Cfg<DH>;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(BT, BT);
+  constexpr uint32_t IDESC_D = idesc_bf16_f32_bmn(BT, DH);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sdO = smem + C::TILE;
+  uint8_t* sKV = smem + 2 * C::TILE;  // stage st: K at st * 2 TILE, V at + TILE
+  uint64_t* bars = (uint64_t*)(smem + 6 * C::TILE);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;   // [2]
+  uint64_t* kv_empty = bars + 4;  // [2]
+  uint64_t* s_full = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* dq_full = bars + 8;
+  uint64_t* dq_empty = bars + 9;
+  uint64_t* drain = bars + 10;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 11);
+  volatile int* abort = (volatile int*)(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 4);
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  constexpr uint32_t S_COL = 0, P_COL = 128, Q_COL = 256;  // S (then scale*dS), dP, dQ
+
+  const int nqt = (a.S + BT - 1) / BT;
+  const int nwork = a.B * a.Hq * nqt;
+  const int G = a.Hq / a.Hkv;
+  // item w: query tile qt (longest first), head h, sequence b
+  auto item = [&](int w, int& b, int& h, int& qt) {
+    const int per = a.B * a.Hq;
+    qt = nqt - 1 - w / per;
+    const int rem = w % per;
+    h = rem % a.Hq;
+    b = rem / a.Hq;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmdO);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int kvit = 0;
+      bool ok = true;
+      for (int rr = 0; ok; ++rr) {
+        const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
+        if (w < 0) break;
+        int b, h, qt;
+        item(w, b, h, qt);
+        if (!mbar_wait(q_empty, (rr & 1) ^ 1, abort, status)) break;
+        mbar_expect_tx(q_full, 2 * C::TILE);
+        for (int hb = 0; hb < C::NH; ++hb) {
+          tma_load_2d(sQ + hb * C::HALF, &tmQ, q_full, h * DH + hb * 64, b * a.S + qt * BT);
+          tma_load_2d(sdO + hb * C::HALF, &tmdO, q_full, h * DH + hb * 64, b * a.S + qt * BT);
+        }
+        for (int j = 0; j <= qt; ++j, ++kvit) {
+          const int st = kvit & 1;
+          if (!mbar_wait(&kv_empty[st], ((kvit >> 1) & 1) ^ 1, abort, status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&kv_full[st], 2 * C::TILE);
+          uint8_t* dst = sKV + st * 2 * C::TILE;
+          for (int hb = 0; hb < C::NH; ++hb) {
+            tma_load_2d(dst + hb * C::HALF, &tmK, &kv_full[st], (h / G) * DH + hb * 64, b * a.S + j * BT);
+            tma_load_2d(dst + C::TILE + hb * C::HALF, &tmV, &kv_full[st], (h / G) * DH + hb * 64, b * a.S + j * BT);
+          }
+        }
+      }
+      if (*abort) {
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 50000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint64_t qd = sdesc_kmajor_sw128(sQ), dod = sdesc_kmajor_sw128(sdO);
+      int kvit = 0, pc = 0;
+      bool ok = true;
+      // dQ += scale*dS K_j for the key tile in ring slot `st`, dS read from TMEM over S
+      auto issue_dq = [&](int st, bool acc) {
+        const uint64_t kd = sdesc_mnmajor_sw128(sKV + st * 2 * C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk)
+          umma_bf16_ts(tbase + Q_COL, tbase + S_COL + kk * 8, kd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+                       (acc || kk) ? 1u : 0u);
+      };
+      for (int rr = 0; ok; ++rr) {
+        const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
+        if (w < 0) break;
+        int b, h, qt;
+        item(w, b, h, qt);
+        const int n = qt + 1;
+        if (!mbar_wait(q_full, rr & 1, abort, status)) break;
+        for (int j = 0; j < n; ++j) {
+          const int cur = kvit + j, st = cur & 1;
+          if (!mbar_wait(&kv_full[st], (cur >> 1) & 1, abort, status)) { ok = false; break; }
+          if (j > 0) {  // finish key tile j-1 before S_j overwrites its dS
+            if (!mbar_wait(p_full, pc & 1, abort, status)) { ok = false; break; }
+            ++pc;
+            if (j == 1 && !mbar_wait(dq_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
+            tc_fence_after();
+            issue_dq((cur - 1) & 1, j > 1);
+            umma_commit(&kv_empty[(cur - 1) & 1]);
+          }
+          tc_fence_after();
+          const uint64_t kd = sdesc_kmajor_sw128(sKV + st * 2 * C::TILE);
+          const uint64_t vd = sdesc_kmajor_sw128(sKV + st * 2 * C::TILE + C::TILE);
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk)
+            umma_bf16_ss(tbase + S_COL, qd + kstep(kk, C::HALF), kd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk)
+            umma_bf16_ss(tbase + P_COL, dod + kstep(kk, C::HALF), vd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+          umma_commit(s_full);
+          if (j == n - 1) umma_commit(q_empty);
+        }
+        if (!ok) break;
+        if (!mbar_wait(p_full, pc & 1, abort, status)) break;
+        ++pc;
+        if (n == 1 && !mbar_wait(dq_empty, (rr & 1) ^ 1, abort, status)) break;
+        tc_fence_after();
+        issue_dq((kvit + n - 1) & 1, n > 1);
+        umma_commit(&kv_empty[(kvit + n - 1) & 1]);
+        umma_commit(dq_full);
+        kvit += n;
+      }
+      if (*abort) {
+        umma_commit(drain);
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else {
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t s_tmem = tbase + lane_off + S_COL, p_tmem = tbase + lane_off + P_COL;
+    const uint32_t q_tmem = tbase + lane_off + Q_COL;
+    const float sl2 = a.scale * 1.4426950408889634f;
+    int sit = 0;
+    for (int rr = 0;; ++rr) {
+      const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
+      if (w < 0) break;
+      int b, h, qt;
+      item(w, b, h, qt);
+      const int n = qt + 1, row = qt * BT + r;
+      const bool valid = row < a.S;
+      const size_t li = ((size_t)b * a.Hq + h) * a.lse_ld + (valid ? row : 0);
+      const float lse2 = valid ? a.lse[li] : 0.f, drow = valid ? a.dsum[li] : 0.f;
+      bool ok = true;
+      for (int j = 0; j < n; ++j, ++sit) {
+        if (!mbar_wait(s_full, sit & 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        const int lim = valid ? row - j * BT : -1;  // keys c > lim are masked (all, for a padding row)
+        const bool diag = j == n - 1 || !valid;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32], pv[32], pk[16];
+          tmem_ld32(s_tmem + c * 32, sv);
+          tmem_ld32(p_tmem + c * 32, pv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int k0 = c * 32 + 2 * e;
+            float p0 = ex2(__uint_as_float(sv[2 * e]) * sl2 - lse2);
+            float p1 = ex2(__uint_as_float(sv[2 * e + 1]) * sl2 - lse2);
+            if (diag) {
+              p0 = k0 <= lim ? p0 : 0.f;
+              p1 = k0 + 1 <= lim ? p1 : 0.f;
+            }
+            pk[e] = pack2(a.scale * p0 * (__uint_as_float(pv[2 * e]) - drow),
+                          a.scale * p1 * (__uint_as_float(pv[2 * e + 1]) - drow));
+          }
+          tmem_st16(s_tmem + c * 16, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      if (!mbar_wait(dq_full, rr & 1, abort, status)) break;
+      tc_fence_after();
+      float* dst = a.dq + ((size_t)b * a.S + (valid ? row : 0)) * (size_t)(a.Hq * DH) + (size_t)h * DH;
+#pragma unroll
+      for (int c = 0; c < DH; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(q_tmem + c, v);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t u[8] = {v[8 * e], v[8 * e + 1], v[8 * e + 2], v[8 * e + 3],
+                                   v[8 * e + 4], v[8 * e + 5], v[8 * e + 6], v[8 * e + 7]};
+            st_global_v8(dst + c + 8 * e, u);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_empty);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TMEM_COLS);
+  }
+}
+
+// ============================================================================ dK, dV
+template <int DH>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                         const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         AttnBwdArgs a, int* status) {
+  using C = Cfg<DH>;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(BT, BT);
+  constexpr uint32_t IDESC_D = idesc_bf16_f32_bmn(BT, DH);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + C::TILE;
+  uint8_t* sQD = smem + 2 * C::TILE;  // stage st at st * STAGE: Q, dO, lse[128], D[128]
+  uint64_t* bars = (uint64_t*)(smem + 2 * C::TILE + 2 * C::STAGE);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* qd_full = bars + 2;   // [2]
+  uint64_t* qd_empty = bars + 4;  // [2]
+  uint64_t* s_full = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* acc_full = bars + 8;
+  uint64_t* acc_empty = bars + 9;
+  uint64_t* drain = bars + 10;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 11);
+  volatile int* abort = (volatile int*)(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qd_full[i], 1);
+      mbar_init(&qd_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  constexpr uint32_t S_COL = 0, P_COL = 128, V_COL = 256, K_COL = 256 + DH;  // S^T/P^T, dP^T/dS^T, dV, dK
+
+  const int nqt = (a.S + BT - 1) / BT;
+  const int nwork = a.B * a.Hkv * nqt;
+  const int G = a.Hq / a.Hkv;
+  // item w: key tile kt (longest first: the most query tiles), KV group g, sequence b; its steps
+  // run the G heads (outer) over the query tiles kt..nqt-1 (inner)
+  auto item = [&](int w, int& b, int& g, int& kt) {
+    const int per = a.B * a.Hkv;
+    kt = w / per;
+    const int rem = w % per;
+    g = rem % a.Hkv;
+    b = rem / a.Hkv;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmdO);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int qdit = 0;
+      bool ok = true;
+      for (int rr = 0; ok; ++rr) {
+        const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
+        if (w < 0) break;
+        int b, g, kt;
+        item(w, b, g, kt);
+        if (!mbar_wait(kv_empty, (rr & 1) ^ 1, abort, status)) break;
+        mbar_expect_tx(kv_full, 2 * C::TILE);
+        for (int hb = 0; hb < C::NH; ++hb) {
+          tma_load_2d(sK + hb * C::HALF, &tmK, kv_full, g * DH + hb * 64, b * a.S + kt * BT);
+          tma_load_2d(sV + hb * C::HALF, &tmV, kv_full, g * DH + hb * 64, b * a.S + kt * BT);
+        }
+        const int nq = nqt - kt;
+        for (int s = 0; s < G * nq; ++s, ++qdit) {
+          const int h = g * G + s / nq, qt = kt + s % nq, st = qdit & 1;
+          if (!mbar_wait(&qd_empty[st], ((qdit >> 1) & 1) ^ 1, abort, status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&qd_full[st], 2 * C::TILE + 2 * C::VEC);
+          uint8_t* dst = sQD + st * C::STAGE;
+          for (int hb = 0; hb < C::NH; ++hb) {
+            tma_load_2d(dst + hb * C::HALF, &tmQ, &qd_full[st], h * DH + hb * 64, b * a.S + qt * BT);
+            tma_load_2d(dst + C::TILE + hb * C::HALF, &tmdO, &qd_full[st], h * DH + hb * 64, b * a.S + qt * BT);
+          }
+          const size_t li = ((size_t)b * a.Hq + h) * a.lse_ld + (size_t)qt * BT;
+          bulk_load(dst + 2 * C::TILE, a.lse + li, C::VEC, &qd_full[st]);
+          bulk_load(dst + 2 * C::TILE + C::VEC, a.dsum + li, C::VEC, &qd_full[st]);
+        }
+      }
+      if (*abort) {
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 50000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint64_t kd = sdesc_kmajor_sw128(sK), vd = sdesc_kmajor_sw128(sV);
+      int qdit = 0, pc = 0;
+      bool ok = true;
+      // dV += P^T dO and dK += scale*dS^T Q for the query stage `st` (P^T, dS^T read from TMEM)
+      auto issue_acc = [&](int st, bool acc) {
+        const uint64_t dq = sdesc_mnmajor_sw128(sQD + st * C::STAGE);
+        const uint64_t dd = sdesc_mnmajor_sw128(sQD + st * C::STAGE + C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk)
+          umma_bf16_ts(tbase + V_COL, tbase + S_COL + kk * 8, dd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+                       (acc || kk) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk)
+          umma_bf16_ts(tbase + K_COL, tbase + P_COL + kk * 8, dq + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+                       (acc || kk) ? 1u : 0u);
+      };
+      for (int rr = 0; ok; ++rr) {
+        const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
+        if (w < 0) break;
+        int b, g, kt;
+        item(w, b, g, kt);
+        const int n = G * (nqt - kt);
+        if (!mbar_wait(kv_full, rr & 1, abort, status)) break;
+        for (int s = 0; s < n; ++s) {
+          const int cur = qdit + s, st = cur & 1;
+          if (!mbar_wait(&qd_full[st], (cur >> 1) & 1, abort, status)) { ok = false; break; }
+          if (s > 0) {  // finish step s-1 before S^T_s overwrites its P^T
+            if (!mbar_wait(p_full, pc & 1, abort, status)) { ok = false; break; }
+            ++pc;
+            if (s == 1 && !mbar_wait(acc_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
+            tc_fence_after();
+            issue_acc((cur - 1) & 1, s > 1);
+            umma_commit(&qd_empty[(cur - 1) & 1]);
+          }
+          tc_fence_after();
+          const uint64_t qd = sdesc_kmajor_sw128(sQD + st * C::STAGE);
+          const uint64_t dod = sdesc_kmajor_sw128(sQD + st * C::STAGE + C::TILE);
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk)
+            umma_bf16_ss(tbase + S_COL, kd + kstep(kk, C::HALF), qd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk)
+            umma_bf16_ss(tbase + P_COL, vd + kstep(kk, C::HALF), dod + kstep(kk, C::HALF), IDESC_S, kk != 0);
+          umma_commit(s_full);
+        }
+        if (!ok) break;
+        if (!mbar_wait(p_full, pc & 1, abort, status)) break;
+        ++pc;
+        if (n == 1 && !mbar_wait(acc_empty, (rr & 1) ^ 1, abort, status)) break;
+        tc_fence_after();
+        issue_acc((qdit + n - 1) & 1, n > 1);
+        umma_commit(&qd_empty[(qdit + n - 1) & 1]);
+        umma_commit(kv_empty);
+        umma_commit(acc_full);
+        qdit += n;
+      }
+      if (*abort) {
+        umma_commit(drain);
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else {
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;  // key row of the tile
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t s_tmem = tbase + lane_off + S_COL, p_tmem = tbase + lane_off + P_COL;
+    const float sl2 = a.scale * 1.4426950408889634f;
+    int sit = 0;
+    for (int rr = 0;; ++rr) {
+      const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
+      if (w < 0) break;
+      int b, g, kt;
+      item(w, b, g, kt);
+      const int nq = nqt - kt, n = G * nq, key = kt * BT + r;
+      bool ok = true;
+      for (int s = 0; s < n; ++s, ++sit) {
+        const int qt = kt + s % nq, st = sit & 1;
+        // the stage's lse and D rows: landed with its Q and dO (the stage is not refilled before
+        // this step's dV / dK MMAs, which wait for this warp)
+        if (!mbar_wait(&qd_full[st], (sit >> 1) & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait(s_full, sit & 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        const float* lse2 = (const float*)(sQD + st * C::STAGE + 2 * C::TILE);
+        const float* dsum = lse2 + BT;
+        // query column c is used iff it is a real row at or after this key: q0 + c < S, q0 + c >= key
+        const int q0 = qt * BT, cmax = a.S - q0, cmin = key - q0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32], pv[32], pp[16], pd[16];
+          tmem_ld32(s_tmem + c * 32, sv);
+          tmem_ld32(p_tmem + c * 32, pv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = c * 32 + 2 * e;
+            float p0 = ex2(__uint_as_float(sv[2 * e]) * sl2 - lse2[c0]);
+            float p1 = ex2(__uint_as_float(sv[2 * e + 1]) * sl2 - lse2[c0 + 1]);
+            const bool u0 = c0 < cmax && c0 >= cmin, u1 = c0 + 1 < cmax && c0 + 1 >= cmin;
+            p0 = u0 ? p0 : 0.f;
+            p1 = u1 ? p1 : 0.f;
+            pp[e] = pack2(p0, p1);
+            pd[e] = pack2(u0 ? a.scale * p0 * (__uint_as_float(pv[2 * e]) - dsum[c0]) : 0.f,
+                          u1 ? a.scale * p1 * (__uint_as_float(pv[2 * e + 1]) - dsum[c0 + 1]) : 0.f);
+          }
+          tmem_st16(s_tmem + c * 16, pp);
+          tmem_st16(p_tmem + c * 16, pd);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      if (!mbar_wait(acc_full, rr & 1, abort, status)) break;
+      tc_fence_after();
+      const bool valid = key < a.S;
+      const int wkv = 2 * a.Hkv * DH;
+      float* dst = a.dkv + ((size_t)b * a.S + (valid ? key : 0)) * (size_t)wkv + (size_t)g * DH;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {  // dK to columns [0, dkv), dV to [dkv, 2 dkv)
+        const uint32_t src = tbase + lane_off + (part ? V_COL : K_COL);
+        float* d = dst + (part ? a.Hkv * DH : 0);
+#pragma unroll
+        for (int c = 0; c < DH; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(src + c, v);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t u[8] = {v[8 * e], v[8 * e + 1], v[8 * e + 2], v[8 * e + 3],
+                                     v[8 * e + 4], v[8 * e + 5], v[8 * e + 6], v[8 * e + 7]};
+              st_global_v8(d + c + 8 * e, u);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TMEM_COLS);
+  }
+}
+
+}  // namespace tcb
+
+template <int DH>
+static cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const AttnBwdArgs& a, int* status, int sms, cudaStream_t s) {
+  using C = tcb::Cfg<DH>;
+  const int nqt = (a.S + tcb::BT - 1) / tcb::BT;
+  cudaError_t e = set_max_smem(tcb::attn_bwd_dkdv_kernel<DH>, C::SMEM_DKDV, s);
+  if (e != cudaSuccess) return e;
+  const int nkv = a.B * a.Hkv * nqt, nq = a.B * a.Hq * nqt;
+  tcb::attn_bwd_dkdv_kernel<DH><<<nkv < sms ? nkv : sms, tcb::NTHREADS, C::SMEM_DKDV, s>>>(tq, tdo, tk, tv, a, status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = set_max_smem(tcb::attn_bwd_dq_kernel<DH>, C::SMEM_DQ, s)) != cudaSuccess) return e;
+  tcb::attn_bwd_dq_kernel<DH><<<nq < sms ? nq : sms, tcb::NTHREADS, C::SMEM_DQ, s>>>(tq, tdo, tk, tv, a, status);
+  return cudaGetLastError();
+}
+
+cudaError_t attention_backward_tc(const AttnBwdArgs& a, int* status, cudaStream_t s) {
+  if (a.B <= 0 || a.S <= 0) return cudaSuccess;
+  if ((a.dh != 64 && a.dh != 128) || a.Hq % a.Hkv || a.lse_ld < (a.S + tcb::BT - 1) / tcb::BT * tcb::BT ||
+      ((uintptr_t)a.dq & 31) || ((uintptr_t)a.dkv & 31) || ((uintptr_t)a.lse & 15) || ((uintptr_t)a.dsum & 15) ||
+      (long long)a.B * a.S >= (1LL << 31))
+    return cudaErrorInvalidValue;
+  CUtensorMap tq, tdo, tk, tv;
+  const int rows = a.B * a.S;
+  cudaError_t e = make_tmap_bf16(&tq, a.q, rows, a.Hq * a.dh, a.Hq * a.dh, tcb::BT);
+  if (e == cudaSuccess) e = make_tmap_bf16(&tdo, a.dout, rows, a.Hq * a.dh, a.Hq * a.dh, tcb::BT);
+  if (e == cudaSuccess) e = make_tmap_bf16(&tk, a.k, rows, a.Hkv * a.dh, a.Hkv * a.dh, tcb::BT);
+  if (e == cudaSuccess) e = make_tmap_bf16(&tv, a.v, rows, a.Hkv * a.dh, a.Hkv * a.dh, tcb::BT);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return a.dh == 128 ? launch_bwd<128>(tq, tdo, tk, tv, a, status, sms, s)
+                     : launch_bwd<64>(tq, tdo, tk, tv, a, status, sms, s);
+}
+
+}  // namespace mka

@@ -101,6 +101,24 @@ def test_full_mka_limits(mka):
     assert mka.mka_workspace_size(qwen_cfg(mka, block_sparse=1, attention_paths=3)) == 0
 
 
+def test_training_limits(mka):
+    """The layer backward: bf16 FastMKA only, router_hidden % 32 == 0 and <= 512."""
+    assert mka.mka_train_workspace_size(qwen_cfg(mka)) > mka.mka_workspace_size(qwen_cfg(mka))
+    for kw in ({"dtype": mka.MKA_F32}, {"attention_paths": 3}, {"block_sparse": 1}, {"router_hidden": 48},
+               {"router_hidden": 1024}):
+        assert mka.mka_train_workspace_size(qwen_cfg(mka, **kw)) == 0, kw
+    lib, a = mka._lib, ctypes.c_void_p(0x1000)
+    c = qwen_cfg(mka, dtype=mka.MKA_F32)
+    assert lib.mka_prefill_forward_train(ctypes.byref(c), a, a, a, a, 1 << 40, None) == mka.MKA_ERR_UNSUPPORTED
+    c = qwen_cfg(mka)
+    assert lib.mka_prefill_forward_train(ctypes.byref(c), a, a, a, ctypes.c_void_p(0x1010), 1 << 40,
+                                         None) == mka.MKA_ERR_INVALID_ARG
+    assert lib.mka_prefill_backward(ctypes.byref(c), a, a, a, a, a, a, a, a, a, a, None, a, 16,
+                                    None) == mka.MKA_ERR_WORKSPACE
+    assert lib.mka_prefill_backward(ctypes.byref(c), a, a, a, None, a, a, a, a, a, a, None, a, 1 << 40,
+                                    None) == mka.MKA_ERR_INVALID_ARG
+
+
 def test_host_side_errors_before_any_device_call(mka):
     lib = mka._lib
     c = qwen_cfg(mka)
