@@ -291,6 +291,139 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+BACKWARD_STAGES = ["weight_transposes", "dsum", "attention_bwd", "router_preact_gemm", "router_bwd", "dq_gemm",
+                   "memory_adjoint", "dx_gemm", "act_transposes", "weight_grad_gemms"]
+
+
+def train_flops(cfg) -> dict:
+    """Algorithmic FLOPs of one training step (forward + backward).  Attention backward: the five
+    products of the textbook backward over the causal pairs (S and dP recomputed once, dV, dK, dQ),
+    10 dh Hq per pair; projections: dX and the weight gradients are two more GEMMs of the forward's
+    size, plus the router's hidden layer recomputed and its two backward products."""
+    fw = prefill_flops(cfg)
+    pairs = cfg.batch * cfg.seq * (cfg.seq + 1) / 2
+    T, d, dq, dkv, rh = cfg.tokens, cfg.d_model, cfg.dq, cfg.dkv, cfg.router_hidden
+    return {"forward": fw["projections"] + fw["attention"],
+            "attention_bwd": 10.0 * cfg.d_head * cfg.n_q_heads * pairs,
+            "projections_bwd": 2.0 * T * d * (dq + 2 * dkv) * 2 + 2.0 * T * d * 2 * rh + 2.0 * T * dq * rh * 2}
+
+
+def run_train(args, rank, world, local_rank):
+    """Training step of the layer: mka_prefill_forward_train then mka_prefill_backward with a fixed
+    synthetic output gradient; tokens/s of the whole step, roofline on the attention backward."""
+    import route_kv_memory_b200 as mka
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = workload_cfg(args, args.workload)
+    inp = make_inputs(cfg)
+    weights = {k: v.to(dev) for k, v in inp.tensors().items() if k != "x"}
+    layer = mka.FastMKALayer(cfg, weights, dev)
+    x = inp.x[:, :cfg.seq].contiguous().to(dev)
+    out = torch.empty(cfg.batch, cfg.seq, cfg.dq, dtype=x.dtype, device=dev)
+    g = torch.Generator().manual_seed(cfg.seed + 1000)
+    dout_host = torch.randn(cfg.batch, cfg.seq, cfg.dq, generator=g).to(torch.bfloat16)
+    dout = dout_host.to(dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = {"dx": torch.empty_like(x), "dw_q": torch.empty(cfg.d_model, cfg.dq, **f32),
+             "dw_k": torch.empty(cfg.d_model, cfg.dkv, **f32), "dw_v": torch.empty(cfg.d_model, cfg.dkv, **f32),
+             "dw_r1": torch.empty(cfg.dq, cfg.router_hidden, **f32), "dw_r2": torch.empty(cfg.router_hidden, 3, **f32)}
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward_train(x, out)
+        layer.backward(x, out, dout, grads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert mka.mka_status() == 0
+    fw_ms, bw_ms = [], []
+    mka.mka_profile_enable(True)
+    for i in range(min(args.steps, 10)):
+        flush.zero_()
+        layer.forward_train(x, out)
+        fw_ms.append(mka.mka_profile_read())
+        layer.backward(x, out, dout, grads)
+        bw_ms.append(mka.mka_profile_read(len(BACKWARD_STAGES)))
+    mka.mka_profile_enable(False)
+    torch.cuda.synchronize()
+    fw_st, bw_st = np.array(fw_ms).mean(axis=0), np.array(bw_ms).mean(axis=0)
+
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev0[i].record(stream)
+            step()
+            ev1[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(ev0, ev1)), world)
+    assert mka.mka_status() == 0
+
+    # end to end: X and dO from pinned host memory, dX back, every step (sequential)
+    x_host, dx_host = inp.x[:, :cfg.seq].contiguous().pin_memory(), torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    dout_pin = dout_host.pin_memory()
+    n_e2e = max(4, args.steps // 4)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(n_e2e):
+        x.copy_(x_host, non_blocking=True)
+        dout.copy_(dout_pin, non_blocking=True)
+        flush.zero_()
+        step()
+        dx_host.copy_(grads["dx"], non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1) / n_e2e, world)
+
+    peaks = load_peaks()
+    fl = train_flops(cfg)
+    ab_ms = float(bw_st[BACKWARD_STAGES.index("attention_bwd")])
+    ab_tf = fl["attention_bwd"] / (ab_ms / 1e3) / 1e12
+    return {
+        "metric": "FastMKA layer training step (forward + backward) tokens/s",
+        "value": round(world * cfg.tokens / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs and output gradient, N(0,1/d_in) weights)",
+        "config": {"workload": f"{cfg.name}: {model_name(cfg)}-shaped FastMKA layer training step (forward keeping "
+                               f"activations + backward to dX and dW_q, dW_k, dW_v, dW_r1, dW_r2), batch "
+                               f"{cfg.batch} x seq {cfg.seq}; recall held fixed (straight-through)",
+                   "global_batch": cfg.batch * world, "seq_len": cfg.seq,
+                   "parallelism": f"replicas x{world} (independent sequences, no exchange)",
+                   "l2": "flushed (512 MB write) before every timed step"},
+        "roofline": {"kernel": "attention backward (dK/dV and dQ kernels)", "bound": "tensor",
+                     "achieved": round(ab_tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(ab_tf / peaks["bf16_tflops"], 4),
+                     "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)", "traffic": None,
+                     "avg_ms": round(ab_ms, 4), "flops_per_launch": fl["attention_bwd"]},
+        "layer_tflops": round(sum(fl.values()) / (ms / 1e3) / 1e12, 1),
+        "forward_stage_ms": {n: round(float(v), 4) for n, v in zip(PREFILL_STAGES, fw_st)},
+        "backward_stage_ms": {n: round(float(v), 4) for n, v in zip(BACKWARD_STAGES, bw_st)},
+        "e2e": {"value": round(world * cfg.tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * x_host.numel() * x_host.element_size(),
+                "d2h_bytes_per_step": dx_host.numel() * dx_host.element_size(), "ms_per_step": round(e2e_ms, 4),
+                "how": "pinned host X and dO -> device, training step, device dX -> pinned host, sequential"},
+        "gpu_launches": train_kernels() * args.steps,
+        "clocks": clk.summary(),
+    }
+
+
+def train_kernels() -> int:
+    """Kernel launches of one training step: the 10 of the prefill, then the backward's weight
+    transposes (2), D, the two attention-backward kernels, the router pre-activation GEMM, the EMA
+    and recalled-mean recomputes (2), the router backward, the dq GEMM and its combine (2), the
+    recall lists (3), the memory adjoint (4), the dX GEMM, the activation transposes (4) and the
+    two weight-gradient GEMMs."""
+    return 10 + 2 + 1 + 2 + 1 + 2 + 1 + 2 + 3 + 4 + 1 + 4 + 2
+
+
 def run_decode(args, cfg_prefill, inp_unused, weights_unused, dev, layer_pack=None):
     """Decode us/token over a fused cache of `ctx` positions: 256 steps captured in one CUDA graph."""
     import route_kv_memory_b200 as mka
@@ -458,6 +591,8 @@ def main():
                     help="1: FastMKA (the layer measured); 3: full MKA, three attention paths (prefill only)")
     ap.add_argument("--block-sparse", action="store_true",
                     help="Block-MKA block-sparse attention: own block + recalled blocks (prefill only)")
+    ap.add_argument("--train", action="store_true",
+                    help="time the layer training step (forward keeping activations + backward) instead of prefill")
     ap.add_argument("--decode-ctx", type=int, nargs="*", default=[131072])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode measurement (no prefill line)")
@@ -485,7 +620,7 @@ def main():
             if rank == 0:
                 print(json.dumps(res), flush=True)
             return
-        res = run_ours(args, rank, world, local_rank)
+        res = run_train(args, rank, world, local_rank) if args.train else run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

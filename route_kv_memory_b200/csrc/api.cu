@@ -795,7 +795,7 @@ static TrainWs train_ws(const Dims& d) {
   w.recoff = o; o += al(nbj * 4);
   w.cursor = o; o += al(nbj * 4);
   w.pairoff = o; o += al((nbj + 1) * 4);
-  w.pairbj = o; o += al(gathered_max_pairs(T, d.R, 0, 128, nbj) * 4);
+  w.pairbj = o; o += al(gathered_max_pairs(T, d.R, 0, 32, nbj) * 4);
   w.list = o; o += al(T * d.R * 4);
   w.total = o;
   return w;
@@ -869,18 +869,23 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
   const int* idx = (const int*)P(ws, F.idx);
   const int* cnt = (const int*)P(ws, F.cnt);
 
+  prof_begin();
+  STAGE(s);
   // weights in the orientation of the backward products: [W_q | W_k | W_v] as [d][dq + 2 dkv], W_r1 as [dq][rh]
   CUDA_TRY(transpose(wcat, W.ncat, d.d, d.d, wcatT, W.ncat, 2, 0, s));
   CUDA_TRY(transpose(P((void*)packed, PL.wr1T), d.rh, d.dq, d.dq, wr1, d.rh, 2, 0, s));
+  STAGE(s);
   // attention: D = rowsum(dO * O), then dQ and [dK | dV]
   CUDA_TRY(cudaMemsetAsync(dsum, 0, (size_t)d.B * d.Hq * W.Spad * 4, s));
   CUDA_TRY(attention_dsum(dout, out, d.B, d.S, d.Hq, d.dh, W.Spad, dsum, s));
+  STAGE(s);
   AttnBwdArgs ab{};
   ab.q = P(ws, F.q); ab.k = P(ws, F.k); ab.v = P(ws, F.v); ab.dout = dout;
   ab.lse = lse; ab.dsum = dsum; ab.lse_ld = W.Spad;
   ab.dq = dq; ab.dkv = dy;
   ab.B = d.B; ab.S = d.S; ab.Hq = d.Hq; ab.Hkv = d.Hkv; ab.dh = d.dh; ab.scale = d.scale;
   CUDA_TRY(attention_backward_tc(ab, status_ptr(), s));
+  STAGE(s);
   // the router's pre-activation h = X (W_q W_r1) from its packed hi / lo rows
   {
     Epilogue ep{};
@@ -888,6 +893,7 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
     ep.seg[0] = OutSeg{0, 2 * d.rh, hrec, 2 * d.rh, 0};
     CUDA_TRY(gemm_tn_bf16_tc(x, d.d, wcat + (size_t)PL.seg_r * d.d, d.d, (int)T, 2 * d.rh, d.d, ep, status_ptr(), s));
   }
+  STAGE(s);
   // the L2 and L3 values of the projected sources, as the forward fused them
   const float* xkv = (const float*)P(ws, F.xkv);
   CUDA_TRY(ema_apply(xkv, 0, wd, d.B, d.S, d.nblk, d.blk, d.alpha, (const float*)P(ws, F.carry), ema, nullptr, s));
@@ -900,6 +906,7 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
   rb.w_r2 = (const float*)P((void*)packed, PL.wr2); rb.dh = dh; rb.dw_r2 = dw_r2;
   rb.B = d.B; rb.S = d.S; rb.route_mode = d.route; rb.tiers = d.tiers;
   CUDA_TRY(router_backward(rb, s));
+  STAGE(s);
   // dq = dq (attention) + dh W_r1^T, into the first dq columns of [dq | U] (bf16)
   {
     Epilogue ep{};
@@ -908,21 +915,24 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
     CUDA_TRY(gemm_tn_bf16_tc(dh, d.rh, wr1, d.rh, (int)T, d.dq, d.rh, ep, status_ptr(), s));
   }
   CUDA_TRY(add_to_bf16(dq, dqr, (long long)T, d.dq, acat, W.ncat, s));
+  STAGE(s);
   // U = lam1 dY + EMA^T(lam2 dY) + M^T(lam3 dY), into the last 2 dkv columns
   {
     int* nrec = (int*)P(ws, W.nrec);
     int* recoff = (int*)P(ws, W.recoff);
     int* list = (int*)P(ws, W.list);
     if (d.nblk > 0)
-      CUDA_TRY(block_lists(idx, cnt, d.B, d.S, d.R, d.blk, d.nblk, 0, 0, 128, nrec, recoff, (int*)P(ws, W.cursor),
+      CUDA_TRY(block_lists(idx, cnt, d.B, d.S, d.R, d.blk, d.nblk, 0, 0, 32, nrec, recoff, (int*)P(ws, W.cursor),
                            (int*)P(ws, W.pairoff), (int*)P(ws, W.pairbj), list, s));
     MemAdjArgs ma{};
     ma.dy = dy; ma.width = wd; ma.lam = lam; ma.cnt = cnt; ma.nrec = nrec; ma.recoff = recoff; ma.list = list;
+    ma.pairoff = (const int*)P(ws, W.pairoff); ma.pairbj = (const int*)P(ws, W.pairbj);
     ma.B = d.B; ma.S = d.S; ma.nblk = d.nblk; ma.blk = d.blk; ma.alpha = d.alpha;
     ma.gsum = (float*)P(ws, W.gsum); ma.rsum = (float*)P(ws, W.rsum); ma.cs = (float*)P(ws, W.cs);
     ma.u = (bf16*)acat + d.dq; ma.ldu = W.ncat;
     CUDA_TRY(memory_adjoint(ma, s));
   }
+  STAGE(s);
   // dX = [dq | U] [W_q | W_k | W_v]^T
   {
     Epilogue ep{};
@@ -930,6 +940,7 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
     ep.seg[0] = OutSeg{0, d.d, dx, d.d, 1};
     CUDA_TRY(gemm_tn_bf16_tc(acat, W.ncat, wcatT, W.ncat, (int)T, d.d, W.ncat, ep, status_ptr(), s));
   }
+  STAGE(s);
   // weight gradients: [dW_q | dW_k | dW_v] = X^T [dq | U], dW_r1 = q^T dh, with the token axis as K
   void* xT = P(ws, W.xT);
   void* acatT = P(ws, W.acatT);
@@ -945,6 +956,7 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
   CUDA_TRY(transpose(acat, (int)T, W.ncat, W.ncat, acatT, W.Tp, 2, 0, s));
   CUDA_TRY(transpose(P(ws, F.q), (int)T, d.dq, d.dq, qT, W.Tp, 2, 0, s));
   CUDA_TRY(transpose(dh, (int)T, d.rh, d.rh, dhT, W.Tp, 2, 0, s));
+  STAGE(s);
   {
     Epilogue ep{};
     ep.nseg = 3;
@@ -959,6 +971,7 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
     ep.seg[0] = OutSeg{0, d.rh, dw_r1, d.rh, 0};
     CUDA_TRY(gemm_tn_bf16_tc(qT, W.Tp, dhT, W.Tp, d.dq, d.rh, W.Tp, ep, status_ptr(), s));
   }
+  STAGE(s);
   return MKA_OK;
 }
 

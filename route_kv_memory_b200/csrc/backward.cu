@@ -126,27 +126,43 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(RouterBwdArgs a) {
   }
 }
 
-// G[b][j] = sum over the tokens t of block j's recall list of lam3[t] dY[t] / count[t]; one CTA per
-// block and 256 columns.
-__global__ void __launch_bounds__(64) recall_grad_kernel(const float* __restrict__ dy, int width,
-                                                         const float* __restrict__ lam, const int* __restrict__ cnt,
-                                                         const int* __restrict__ nrec, const int* __restrict__ recoff,
-                                                         const int* __restrict__ list, int S, int nblk,
-                                                         float* __restrict__ gsum) {
-  const int bj = blockIdx.x, c = (blockIdx.y * 64 + threadIdx.x) * 4;
-  if (c >= width) return;
-  const int b = bj / nblk, n = nrec[bj], base = recoff[bj];
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i = 0; i < n; ++i) {
-    const size_t tok = (size_t)b * S + (list[base + i] >> 5);
-    const float w = lam[tok * 3 + 2] / (float)cnt[tok];
-    const float4 g = *(const float4*)(dy + tok * width + c);
-    acc.x = fmaf(w, g.x, acc.x);
-    acc.y = fmaf(w, g.y, acc.y);
-    acc.z = fmaf(w, g.z, acc.z);
-    acc.w = fmaf(w, g.w, acc.w);
+// G[b][j] += sum over one 64-entry chunk of block j's recall list of lam3[t] dY[t] / count[t]
+// (chunk -> block from block_lists' pair table, built with 32 tokens per tile); persistent CTAs,
+// the chunk's tokens and weights staged in shared memory, then independent row loads.
+constexpr int kChunk = 64;
+__global__ void __launch_bounds__(256) recall_grad_kernel(const float* __restrict__ dy, int width,
+                                                          const float* __restrict__ lam, const int* __restrict__ cnt,
+                                                          const int* __restrict__ nrec, const int* __restrict__ recoff,
+                                                          const int* __restrict__ list, const int* __restrict__ pairoff,
+                                                          const int* __restrict__ pairbj, int nbj, int S, int nblk,
+                                                          float* __restrict__ gsum) {
+  __shared__ int stok[kChunk];
+  __shared__ float swt[kChunk];
+  const int nchunks = pairoff[nbj];
+  for (int w = blockIdx.x; w < nchunks; w += gridDim.x) {
+    const int bj = pairbj[w], b = bj / nblk;
+    const int e0 = (w - pairoff[bj]) * kChunk, m = min(kChunk, nrec[bj] - e0);
+    __syncthreads();  // the previous chunk's readers are done with stok / swt
+    if (threadIdx.x < m) {
+      const size_t tok = (size_t)b * S + (list[recoff[bj] + e0 + threadIdx.x] >> 5);
+      stok[threadIdx.x] = (int)tok;
+      swt[threadIdx.x] = lam[tok * 3 + 2] / (float)cnt[tok];
+    }
+    __syncthreads();
+    for (int c = threadIdx.x * 4; c < width; c += blockDim.x * 4) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+      for (int i = 0; i < m; ++i) {
+        const float wt = swt[i];
+        const float4 g = *(const float4*)(dy + (size_t)stok[i] * width + c);
+        acc.x = fmaf(wt, g.x, acc.x);
+        acc.y = fmaf(wt, g.y, acc.y);
+        acc.z = fmaf(wt, g.z, acc.z);
+        acc.w = fmaf(wt, g.w, acc.w);
+      }
+      atomicAdd((float4*)(gsum + (size_t)bj * width + c), acc);
+    }
   }
-  *(float4*)(gsum + (size_t)bj * width + c) = acc;
 }
 
 // EMA adjoint, pass 1: per block of blk rows, rsum = sum_{t in block} a^(t - start) lam2[t] dY[t]
@@ -261,8 +277,12 @@ cudaError_t memory_adjoint(const MemAdjArgs& a, cudaStream_t s) {
   const unsigned gx = (unsigned)((a.width / 4 + 63) / 64);
   cudaError_t e;
   if (a.nblk > 0) {
-    recall_grad_kernel<<<dim3(a.B * a.nblk, gx), 64, 0, s>>>(a.dy, a.width, a.lam, a.cnt, a.nrec, a.recoff, a.list,
-                                                             a.S, a.nblk, a.gsum);
+    if ((e = cudaMemsetAsync(a.gsum, 0, (size_t)a.B * a.nblk * a.width * sizeof(float), s)) != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    recall_grad_kernel<<<sms * 4, 256, 0, s>>>(a.dy, a.width, a.lam, a.cnt, a.nrec, a.recoff, a.list, a.pairoff,
+                                                a.pairbj, a.B * a.nblk, a.S, a.nblk, a.gsum);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   ema_adj_block_kernel<<<dim3(gx, nball, a.B), 64, 0, s>>>(a.dy, a.width, a.lam, a.S, nball, a.blk, a.alpha, a.rsum);

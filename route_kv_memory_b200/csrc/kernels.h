@@ -203,7 +203,8 @@ cudaError_t router_backward(const RouterBwdArgs& a, cudaStream_t s);
 // U = lam1 dY + EMA^T(lam2 dY) + M^T(lam3 dY) in the projected space (backward.cu).
 struct MemAdjArgs {
   const float* dy; int width; const float* lam; const int* cnt;
-  const int* nrec; const int* recoff; const int* list;  // recall lists of the full blocks (block_lists, own 0)
+  const int* nrec; const int* recoff; const int* list;  // recall lists of the full blocks (block_lists, own 0,
+  const int* pairoff; const int* pairbj;                //   32 tokens per tile: a "pair" is a 64-entry chunk)
   int B, S, nblk, blk;
   float alpha;
   float* gsum;  // [B][nblk][width] scratch

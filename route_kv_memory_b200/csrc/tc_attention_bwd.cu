@@ -14,7 +14,10 @@
 //                         a 2-stage ring (Q, dO and their lse and D rows): S^T = K Q^T and
 //                         dP^T = V dO^T into TMEM, four warps write P^T and scale * dS^T (bf16)
 //                         over them, then dV += P^T dO and dK += dS^T Q accumulate in TMEM.
-// Warp 0 loads (TMA), warp 1 issues the MMAs, warps 2-5 compute, one TMEM lane (row) each.
+// Warp 0 loads (TMA), warp 1 issues the MMAs, warps 2-9 compute: two warps per TMEM lane quadrant,
+// each taking 64 of a row's 128 columns; a warp packs its bf16 results into the first 32 columns of
+// its own 64-column range (so neither half overwrites what the other still reads), and the MMAs
+// read K-step kk (16 columns) at packed column kk * 8 + (kk >= 4 ? 32 : 0).
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
@@ -29,7 +32,11 @@ namespace tcb {
 using namespace sm100;
 
 constexpr int BT = 128;  // rows of every tile (query and key)
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 320;
+constexpr int NCOMPUTE = 8;  // compute warps
+
+// TMEM column (32-bit) of K-step kk of a packed bf16 A operand written by the two column halves.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (uint32_t)(kk * 8 + (kk >= 4 ? 32 : 0)); }
 constexpr uint32_t TMEM_COLS = 512;
 
 template <int DH>
@@ -94,9 +101,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, NCOMPUTE);
     mbar_init(dq_full, 1);
-    mbar_init(dq_empty, 4);
+    mbar_init(dq_empty, NCOMPUTE);
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -169,7 +176,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint64_t kd = sdesc_mnmajor_sw128(sKV + st * 2 * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_ts(tbase + Q_COL, tbase + S_COL + kk * 8, kd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+          umma_bf16_ts(tbase + Q_COL, tbase + S_COL + packed_col(kk), kd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
                        (acc || kk) ? 1u : 0u);
       };
       for (int rr = 0; ok; ++rr) {
@@ -220,11 +227,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else {
-    const int q4 = warp & 3;
+    const int q4 = warp & 3, half = (warp - 2) >> 2;  // lane quadrant; columns [64 half, 64 half + 64)
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t s_tmem = tbase + lane_off + S_COL, p_tmem = tbase + lane_off + P_COL;
-    const uint32_t q_tmem = tbase + lane_off + Q_COL;
+    const uint32_t q_tmem = tbase + lane_off + Q_COL + half * (DH / 2);
     const float sl2 = a.scale * 1.4426950408889634f;
     int sit = 0;
     for (int rr = 0;; ++rr) {
@@ -243,7 +250,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int lim = valid ? row - j * BT : -1;  // keys c > lim are masked (all, for a padding row)
         const bool diag = j == n - 1 || !valid;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
           uint32_t sv[32], pv[32], pk[16];
           tmem_ld32(s_tmem + c * 32, sv);
           tmem_ld32(p_tmem + c * 32, pv);
@@ -260,7 +268,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pk[e] = pack2(a.scale * p0 * (__uint_as_float(pv[2 * e]) - drow),
                           a.scale * p1 * (__uint_as_float(pv[2 * e + 1]) - drow));
           }
-          tmem_st16(s_tmem + c * 16, pk);
+          tmem_st16(s_tmem + 64 * half + cc * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -270,9 +278,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!ok) break;
       if (!mbar_wait(dq_full, rr & 1, abort, status)) break;
       tc_fence_after();
-      float* dst = a.dq + ((size_t)b * a.S + (valid ? row : 0)) * (size_t)(a.Hq * DH) + (size_t)h * DH;
+      float* dst = a.dq + ((size_t)b * a.S + (valid ? row : 0)) * (size_t)(a.Hq * DH) + (size_t)h * DH +
+                   half * (DH / 2);
 #pragma unroll
-      for (int c = 0; c < DH; c += 32) {
+      for (int c = 0; c < DH / 2; c += 32) {
         uint32_t v[32];
         tmem_ld32(q_tmem + c, v);
         tmem_ld_wait();
@@ -333,9 +342,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&qd_empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, NCOMPUTE);
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, NCOMPUTE);
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -414,11 +423,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint64_t dd = sdesc_mnmajor_sw128(sQD + st * C::STAGE + C::TILE);
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_ts(tbase + V_COL, tbase + S_COL + kk * 8, dd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+          umma_bf16_ts(tbase + V_COL, tbase + S_COL + packed_col(kk), dd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
                        (acc || kk) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_ts(tbase + K_COL, tbase + P_COL + kk * 8, dq + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+          umma_bf16_ts(tbase + K_COL, tbase + P_COL + packed_col(kk), dq + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
                        (acc || kk) ? 1u : 0u);
       };
       for (int rr = 0; ok; ++rr) {
@@ -469,7 +478,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
   } else {
-    const int q4 = warp & 3;
+    const int q4 = warp & 3, half = (warp - 2) >> 2;  // lane quadrant; query columns [64 half, 64 half + 64)
     const int r = q4 * 32 + lane;  // key row of the tile
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t s_tmem = tbase + lane_off + S_COL, p_tmem = tbase + lane_off + P_COL;
@@ -494,7 +503,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // query column c is used iff it is a real row at or after this key: q0 + c < S, q0 + c >= key
         const int q0 = qt * BT, cmax = a.S - q0, cmin = key - q0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
           uint32_t sv[32], pv[32], pp[16], pd[16];
           tmem_ld32(s_tmem + c * 32, sv);
           tmem_ld32(p_tmem + c * 32, pv);
@@ -511,8 +521,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pd[e] = pack2(u0 ? a.scale * p0 * (__uint_as_float(pv[2 * e]) - dsum[c0]) : 0.f,
                           u1 ? a.scale * p1 * (__uint_as_float(pv[2 * e + 1]) - dsum[c0 + 1]) : 0.f);
           }
-          tmem_st16(s_tmem + c * 16, pp);
-          tmem_st16(p_tmem + c * 16, pd);
+          tmem_st16(s_tmem + 64 * half + cc * 16, pp);
+          tmem_st16(p_tmem + 64 * half + cc * 16, pd);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -525,10 +535,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const bool valid = key < a.S;
       const int wkv = 2 * a.Hkv * DH;
       float* dst = a.dkv + ((size_t)b * a.S + (valid ? key : 0)) * (size_t)wkv + (size_t)g * DH;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {  // dK to columns [0, dkv), dV to [dkv, 2 dkv)
-        const uint32_t src = tbase + lane_off + (part ? V_COL : K_COL);
-        float* d = dst + (part ? a.Hkv * DH : 0);
+      {  // the first warpgroup writes dK (columns [0, dkv)), the second dV ([dkv, 2 dkv))
+        const uint32_t src = tbase + lane_off + (half ? V_COL : K_COL);
+        float* d = dst + (half ? a.Hkv * DH : 0);
 #pragma unroll
         for (int c = 0; c < DH; c += 32) {
           uint32_t v[32];
