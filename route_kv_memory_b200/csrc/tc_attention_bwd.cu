@@ -243,30 +243,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const bool valid = row < a.S;
       const size_t li = ((size_t)b * a.Hq + h) * a.lse_ld + (valid ? row : 0);
       const float lse2 = valid ? a.lse[li] : 0.f, drow = valid ? a.dsum[li] : 0.f;
+      const float2 sl2v = make_float2(sl2, sl2), nlse2v = make_float2(-lse2, -lse2);
+      const float2 ndrowv = make_float2(-drow, -drow), scalev = make_float2(a.scale, a.scale);
       bool ok = true;
       for (int j = 0; j < n; ++j, ++sit) {
         if (!mbar_wait(s_full, sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
         const int lim = valid ? row - j * BT : -1;  // keys c > lim are masked (all, for a padding row)
-        const bool diag = j == n - 1 || !valid;
+        const bool diag = __any_sync(0xffffffffu, j == n - 1 || !valid);  // warp-uniform
+        // the second chunk's TMEM loads are in flight while the first is processed
+        uint32_t sv[2][32], pv[2][32];
+        tmem_ld32(s_tmem + 64 * half, sv[0]);
+        tmem_ld32(p_tmem + 64 * half, pv[0]);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = 2 * half + cc;
-          uint32_t sv[32], pv[32], pk[16];
-          tmem_ld32(s_tmem + c * 32, sv);
-          tmem_ld32(p_tmem + c * 32, pv);
           tmem_ld_wait();
+          if (cc == 0) {
+            tmem_ld32(s_tmem + 64 * half + 32, sv[1]);
+            tmem_ld32(p_tmem + 64 * half + 32, pv[1]);
+          }
+          uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int k0 = c * 32 + 2 * e;
-            float p0 = ex2(__uint_as_float(sv[2 * e]) * sl2 - lse2);
-            float p1 = ex2(__uint_as_float(sv[2 * e + 1]) * sl2 - lse2);
+            const float2 x2 = __ffma2_rn(make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1])),
+                                         sl2v, nlse2v);
+            float p0 = ex2(x2.x), p1 = ex2(x2.y);
             if (diag) {
+              const int k0 = c * 32 + 2 * e;
               p0 = k0 <= lim ? p0 : 0.f;
               p1 = k0 + 1 <= lim ? p1 : 0.f;
             }
-            pk[e] = pack2(a.scale * p0 * (__uint_as_float(pv[2 * e]) - drow),
-                          a.scale * p1 * (__uint_as_float(pv[2 * e + 1]) - drow));
+            const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(pv[cc][2 * e]), __uint_as_float(pv[cc][2 * e + 1])),
+                                         ndrowv);
+            const float2 r2 = __fmul2_rn(__fmul2_rn(make_float2(p0, p1), scalev), d2);
+            pk[e] = pack2(r2.x, r2.y);
           }
           tmem_st16(s_tmem + 64 * half + cc * 16, pk);
         }
@@ -502,24 +513,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float* dsum = lse2 + BT;
         // query column c is used iff it is a real row at or after this key: q0 + c < S, q0 + c >= key
         const int q0 = qt * BT, cmax = a.S - q0, cmin = key - q0;
+        const bool masked = __any_sync(0xffffffffu, cmin > 64 * half || cmax < 64 * half + 64);  // warp-uniform
+        const float2 sl2v = make_float2(sl2, sl2), scalev = make_float2(a.scale, a.scale);
+        // the second chunk's TMEM loads are in flight while the first is processed
+        uint32_t sv[2][32], pv[2][32];
+        tmem_ld32(s_tmem + 64 * half, sv[0]);
+        tmem_ld32(p_tmem + 64 * half, pv[0]);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = 2 * half + cc;
-          uint32_t sv[32], pv[32], pp[16], pd[16];
-          tmem_ld32(s_tmem + c * 32, sv);
-          tmem_ld32(p_tmem + c * 32, pv);
           tmem_ld_wait();
+          if (cc == 0) {
+            tmem_ld32(s_tmem + 64 * half + 32, sv[1]);
+            tmem_ld32(p_tmem + 64 * half + 32, pv[1]);
+          }
+          uint32_t pp[16], pd[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = c * 32 + 2 * e;
-            float p0 = ex2(__uint_as_float(sv[2 * e]) * sl2 - lse2[c0]);
-            float p1 = ex2(__uint_as_float(sv[2 * e + 1]) * sl2 - lse2[c0 + 1]);
-            const bool u0 = c0 < cmax && c0 >= cmin, u1 = c0 + 1 < cmax && c0 + 1 >= cmin;
-            p0 = u0 ? p0 : 0.f;
-            p1 = u1 ? p1 : 0.f;
-            pp[e] = pack2(p0, p1);
-            pd[e] = pack2(u0 ? a.scale * p0 * (__uint_as_float(pv[2 * e]) - dsum[c0]) : 0.f,
-                          u1 ? a.scale * p1 * (__uint_as_float(pv[2 * e + 1]) - dsum[c0 + 1]) : 0.f);
+          for (int e4 = 0; e4 < 8; ++e4) {  // lse and D of four query columns per shared-memory load
+            const float4 l4 = *(const float4*)(lse2 + c * 32 + 4 * e4);
+            const float4 d4 = *(const float4*)(dsum + c * 32 + 4 * e4);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int e = 2 * e4 + k, c0 = c * 32 + 2 * e;
+              const float2 nl = k ? make_float2(-l4.z, -l4.w) : make_float2(-l4.x, -l4.y);
+              const float2 nd = k ? make_float2(-d4.z, -d4.w) : make_float2(-d4.x, -d4.y);
+              const float2 x2 = __ffma2_rn(make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1])),
+                                           sl2v, nl);
+              float p0 = ex2(x2.x), p1 = ex2(x2.y);
+              if (masked) {
+                p0 = (c0 < cmax && c0 >= cmin) ? p0 : 0.f;
+                p1 = (c0 + 1 < cmax && c0 + 1 >= cmin) ? p1 : 0.f;
+              }
+              pp[e] = pack2(p0, p1);
+              const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(pv[cc][2 * e]), __uint_as_float(pv[cc][2 * e + 1])),
+                                           nd);
+              const float2 r2 = __fmul2_rn(__fmul2_rn(make_float2(p0, p1), scalev), d2);
+              pd[e] = pack2(r2.x, r2.y);
+            }
           }
           tmem_st16(s_tmem + 64 * half + cc * 16, pp);
           tmem_st16(p_tmem + 64 * half + cc * 16, pd);
