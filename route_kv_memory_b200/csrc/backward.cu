@@ -26,28 +26,33 @@ __device__ __forceinline__ float warp_sum32(float v) {
   return v;
 }
 
-// D[(b * Hq + h) * ld + t] = sum_i dO[b, t, h, i] * O[b, t, h, i]; one thread per (token, head).
-__global__ void attn_dsum_kernel(const bf16* __restrict__ dout, const bf16* __restrict__ o, int B, int S, int Hq,
-                                 int dh, int ld, float* __restrict__ dsum) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (long long)B * S * Hq) return;
-  const int h = (int)(i % Hq);
-  const long long tok = i / Hq;
-  const uint4* a = (const uint4*)(dout + tok * (size_t)(Hq * dh) + (size_t)h * dh);
-  const uint4* c = (const uint4*)(o + tok * (size_t)(Hq * dh) + (size_t)h * dh);
-  float acc = 0.f;
-  for (int k = 0; k < dh / 8; ++k) {
-    const uint4 x = a[k], y = c[k];
-    const __nv_bfloat162* x2 = (const __nv_bfloat162*)&x;
-    const __nv_bfloat162* y2 = (const __nv_bfloat162*)&y;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 fx = __bfloat1622float2(x2[e]), fy = __bfloat1622float2(y2[e]);
-      acc = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, acc));
-    }
-  }
+// D[(b * Hq + h) * ld + t] = sum_i dO[b, t, h, i] * O[b, t, h, i]; one warp per token row, 16 lanes
+// per head (dh / 8 16-byte pieces each), the head's sum by shuffles within its 16 lanes.
+__global__ void __launch_bounds__(256) attn_dsum_kernel(const bf16* __restrict__ dout, const bf16* __restrict__ o,
+                                                        int B, int S, int Hq, int dh, int ld, float* __restrict__ dsum) {
+  const int lane = threadIdx.x & 31;
+  const long long tok = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (tok >= (long long)B * S) return;
+  const int row = Hq * dh, per = dh / 8;  // 16-byte pieces per head (8 or 16)
+  const uint4* a = (const uint4*)(dout + tok * (size_t)row);
+  const uint4* c = (const uint4*)(o + tok * (size_t)row);
   const int b = (int)(tok / S), t = (int)(tok % S);
-  dsum[((size_t)b * Hq + h) * ld + t] = acc;
+  for (int p0 = 0; p0 < row / 8; p0 += 32) {  // 32 pieces (512 bytes) per step: 2 or 4 heads
+    float acc = 0.f;
+    if (p0 + lane < row / 8) {
+      const uint4 x = a[p0 + lane], y = c[p0 + lane];
+      const __nv_bfloat162* x2 = (const __nv_bfloat162*)&x;
+      const __nv_bfloat162* y2 = (const __nv_bfloat162*)&y;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fx = __bfloat1622float2(x2[e]), fy = __bfloat1622float2(y2[e]);
+        acc = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, acc));
+      }
+    }
+    for (int o2 = per / 2; o2 > 0; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
+    const int piece = p0 + lane;
+    if (lane % per == 0 && piece < row / 8) dsum[((size_t)b * Hq + piece / per) * ld + t] = acc;
+  }
 }
 
 // dL/dz of the routing gate (route_gate in common.cuh) from lam and dL/dlam: where lam is a softmax
@@ -116,14 +121,20 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(RouterBwdArgs a) {
       gw[k][2] = fmaf(g, dz[2], gw[k][2]);
     }
   }
+  // the CTA's warps add into shared memory first: one atomic per weight and CTA
+  __shared__ float red[kMaxRhPerLane * 32 * 3];
+  for (int i = threadIdx.x; i < a.rh * 3; i += blockDim.x) red[i] = 0.f;
+  __syncthreads();
 #pragma unroll
   for (int k = 0; k < kMaxRhPerLane; ++k) {
     if (k >= nu) break;
     const int u = lane + 32 * k;
-    atomicAdd(&a.dw_r2[u * 3], gw[k][0]);
-    atomicAdd(&a.dw_r2[u * 3 + 1], gw[k][1]);
-    atomicAdd(&a.dw_r2[u * 3 + 2], gw[k][2]);
+    atomicAdd(&red[u * 3], gw[k][0]);
+    atomicAdd(&red[u * 3 + 1], gw[k][1]);
+    atomicAdd(&red[u * 3 + 2], gw[k][2]);
   }
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.rh * 3; i += blockDim.x) atomicAdd(&a.dw_r2[i], red[i]);
 }
 
 // G[b][j] += sum over one 64-entry chunk of block j's recall list of lam3[t] dY[t] / count[t]
@@ -254,8 +265,9 @@ cudaError_t attention_dsum(const void* dout, const void* o, int B, int S, int Hq
   const long long n = (long long)B * S * Hq;
   if (n <= 0) return cudaSuccess;
   if (dh % 8) return cudaErrorInvalidValue;
-  attn_dsum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>((const bf16*)dout, (const bf16*)o, B, S, Hq, dh, ld,
-                                                                  dsum);
+  const long long warps = (long long)B * S;
+  attn_dsum_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>((const bf16*)dout, (const bf16*)o, B, S, Hq,
+                                                                          dh, ld, dsum);
   return cudaGetLastError();
 }
 

@@ -121,6 +121,31 @@ __global__ void transpose_kernel(const Tin* __restrict__ in, int rows, int cols,
     if (r < rows && c < cols) out[(size_t)c * ld_out + r] = (Tout)tile[threadIdx.x][i];
   }
 }
+// bf16 -> bf16 transpose of 64 x 64 tiles with 16-byte loads and stores (rows, cols, ld_in, ld_out
+// multiples of 8, both pointers 16-byte aligned); 256 threads.
+__global__ void __launch_bounds__(256) transpose_bf16_v8_kernel(const bf16* __restrict__ in, int rows, int cols,
+                                                                int ld_in, bf16* __restrict__ out, int ld_out) {
+  __shared__ bf16 tile[64][64 + 8];
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {  // 512 vectors of 8 elements
+    const int v = threadIdx.x + 256 * k, r = v >> 3, c = (v & 7) * 8;
+    if (r0 + r < rows && c0 + c < cols)
+      *(uint4*)&tile[r][c] = *(const uint4*)(in + (size_t)(r0 + r) * ld_in + c0 + c);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int v = threadIdx.x + 256 * k, oc = v >> 3, orow = (v & 7) * 8;  // out row c0 + oc, columns r0 + orow..+7
+    if (c0 + oc < cols && r0 + orow < rows) {
+      uint4 u;
+      bf16* e = (bf16*)&u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) e[i] = tile[orow + i][oc];
+      *(uint4*)(out + (size_t)(c0 + oc) * ld_out + r0 + orow) = u;
+    }
+  }
+}
 template <typename Tin>
 __global__ void transpose_bf16_out_kernel(const Tin* __restrict__ in, int rows, int cols, int ld_in,
                                           bf16* __restrict__ out, int ld_out) {
@@ -144,6 +169,10 @@ cudaError_t transpose(const void* in, int rows, int cols, int ld_in, void* out, 
   if (to_f64) {
     if (elem == 2) transpose_kernel<bf16, double><<<grid, block, 0, s>>>((const bf16*)in, rows, cols, ld_in, (double*)out, ld_out);
     else transpose_kernel<float, double><<<grid, block, 0, s>>>((const float*)in, rows, cols, ld_in, (double*)out, ld_out);
+  } else if (elem == 2 && rows % 8 == 0 && cols % 8 == 0 && ld_in % 8 == 0 && ld_out % 8 == 0 &&
+             ((uintptr_t)in & 15) == 0 && ((uintptr_t)out & 15) == 0) {
+    transpose_bf16_v8_kernel<<<dim3((cols + 63) / 64, (rows + 63) / 64), 256, 0, s>>>((const bf16*)in, rows, cols,
+                                                                                      ld_in, (bf16*)out, ld_out);
   } else if (elem == 2) {
     transpose_bf16_out_kernel<bf16><<<grid, block, 0, s>>>((const bf16*)in, rows, cols, ld_in, (bf16*)out, ld_out);
   } else {
