@@ -401,7 +401,8 @@ def run_train(args, rank, world, local_rank):
         "roofline": {"kernel": "attention backward (dK/dV and dQ kernels)", "bound": "tensor",
                      "achieved": round(ab_tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(ab_tf / peaks["bf16_tflops"], 4),
-                     "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)", "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)",
+                     "traffic": traffic_from_profiles("attention_bwd"),
                      "avg_ms": round(ab_ms, 4), "flops_per_launch": fl["attention_bwd"]},
         "layer_tflops": round(sum(fl.values()) / (ms / 1e3) / 1e12, 1),
         "forward_stage_ms": {n: round(float(v), 4) for n, v in zip(PREFILL_STAGES, fw_st)},
