@@ -157,7 +157,7 @@ PackLayout pack_layout(const Dims& d) {
 // ---------------------------------------------------------------- prefill workspace
 struct PrefillWs {
   size_t q, xkv, h1, h2, proj, lam, tcode, xsum, bsum, bend, gend, carry, scode, idx, cnt, k, v, v2;
-  size_t g_nrec, g_recoff, g_cursor, g_pairoff, g_pairbj, g_list, part_o, part_lse, total;
+  size_t g_nrec, g_recoff, g_cursor, g_pairoff, g_pairbj, g_list, g_ptok, g_pinfo, part_o, part_lse, total;
 };
 // Block-gathered attention (Block-MKA block-sparse, full MKA's recalled-block path): every L3
 // block, the last partial one included, has a token list; each token keeps one partial result
@@ -194,6 +194,9 @@ PrefillWs prefill_ws(const Dims& d) {
   w.g_pairoff = o; o += ga ? al((nbj + 1) * 4) : 0;
   w.g_pairbj = o; o += ga ? al(gathered_max_pairs(T, d.R, d.block_sparse, gathered_tpt(d), nbj) * 4) : 0;
   w.g_list = o; o += ga ? al(T * d.R * 4) : 0;
+  const size_t maxp = ga ? gathered_max_pairs(T, d.R, d.block_sparse, gathered_tpt(d), nbj) : 0;
+  w.g_ptok = o; o += al(maxp * 2 * (ga ? gathered_tpt(d) : 0) * 4);
+  w.g_pinfo = o; o += al(maxp * 4);
   w.part_o = o; o += al(T * ns * d.dq * 2);
   w.part_lse = o; o += al(T * ns * d.Hq * 4);
   w.total = o;
@@ -717,10 +720,12 @@ static int prefill_forward(const mka_config* cfg, const void* packed, const void
     int* pairoff = (int*)P(ws, W.g_pairoff);
     int* list = (int*)P(ws, W.g_list);
     int* pairbj = (int*)P(ws, W.g_pairbj);
+    int* ptok = (int*)P(ws, W.g_ptok);
+    int* pinfo = (int*)P(ws, W.g_pinfo);
     CUDA_TRY(block_lists(idx, cnt, d.B, d.S, d.R, d.blk, nball, own, own, gathered_tpt(d), nrec, recoff,
-                         (int*)P(ws, W.g_cursor), pairoff, pairbj, list, s));
+                         (int*)P(ws, W.g_cursor), pairoff, pairbj, list, ptok, pinfo, s));
     AttnArgs ag = aa;
-    ag.g_nrec = nrec; ag.g_recoff = recoff; ag.g_list = list; ag.g_pairoff = pairoff; ag.g_pairbj = pairbj;
+    ag.g_pairoff = pairoff; ag.g_pinfo = pinfo; ag.g_ptok = ptok;
     ag.g_own = own; ag.nblk = nball; ag.blk = d.blk; ag.nslot = ns;
     ag.part_o = P(ws, W.part_o); ag.part_lse = (float*)P(ws, W.part_lse);
     CUDA_TRY(attention_prefill_tc(ag, status_ptr(), s));
@@ -923,7 +928,7 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
     int* list = (int*)P(ws, W.list);
     if (d.nblk > 0)
       CUDA_TRY(block_lists(idx, cnt, d.B, d.S, d.R, d.blk, d.nblk, 0, 0, 32, nrec, recoff, (int*)P(ws, W.cursor),
-                           (int*)P(ws, W.pairoff), (int*)P(ws, W.pairbj), list, s));
+                           (int*)P(ws, W.pairoff), (int*)P(ws, W.pairbj), list, nullptr, nullptr, s));
     MemAdjArgs ma{};
     ma.dy = dy; ma.width = wd; ma.lam = lam; ma.cnt = cnt; ma.nrec = nrec; ma.recoff = recoff; ma.list = list;
     ma.pairoff = (const int*)P(ws, W.pairoff); ma.pairbj = (const int*)P(ws, W.pairbj);

@@ -127,6 +127,25 @@ __global__ void __launch_bounds__(kListThreads) block_fill_kernel(const int* __r
   }
 }
 
+// Per tile pair P (persistent CTAs over the pairs): its block with a flag for a second tile, and its
+// 2 tpt list entries, the block's own tokens first (own), then the recalling tokens' entries.
+__global__ void __launch_bounds__(256) pair_tokens_kernel(const int* __restrict__ nrec, const int* __restrict__ recoff,
+                                                          const int* __restrict__ list, const int* __restrict__ pairoff,
+                                                          const int* __restrict__ pairbj, int nbj, int nblk, int blk,
+                                                          int S, int own, int tpt, int* __restrict__ ptok,
+                                                          int* __restrict__ pinfo) {
+  const int npairs = pairoff[nbj];
+  for (int P = blockIdx.x; P < npairs; P += gridDim.x) {
+    const int bj = pairbj[P], j = bj % nblk, p = P - pairoff[bj];
+    const int nown = own ? min(blk, S - j * blk) : 0, entries = nown + nrec[bj], e0 = 2 * p * tpt;
+    for (int i = threadIdx.x; i < 2 * tpt; i += blockDim.x) {
+      const int e = e0 + i;
+      ptok[(size_t)P * 2 * tpt + i] = e >= entries ? -1 : e < nown ? ((j * blk + e) << 5) : list[recoff[bj] + e - nown];
+    }
+    if (threadIdx.x == 0) pinfo[P] = bj | ((e0 + tpt < entries) ? (1 << 30) : 0);
+  }
+}
+
 __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -195,7 +214,7 @@ __global__ void __launch_bounds__(512) merge_kernel(MergeArgs m) {
 
 cudaError_t block_lists(const int* idx, const int* cnt, int B, int S, int R, int blk, int nblk, int own,
                         int slot_base, int tpt, int* nrec, int* recoff, int* cursor, int* pairoff, int* pairbj,
-                        int* list, cudaStream_t s) {
+                        int* list, int* ptok, int* pinfo, cudaStream_t s) {
   if (B <= 0 || S <= 0) return cudaSuccess;
   if (R < 1 || R + slot_base > 31 || blk <= 0 || nblk <= 0 || tpt <= 0 || S >= (1 << 26))
     return cudaErrorInvalidValue;
@@ -209,6 +228,13 @@ cudaError_t block_lists(const int* idx, const int* cnt, int B, int S, int R, int
   block_scan_kernel<<<1, 1024, 0, s>>>(nrec, B * nblk, nblk, blk, S, own, tpt, recoff, pairoff, cursor, pairbj);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   block_fill_kernel<<<dim3(gx, B), kListThreads, 0, s>>>(idx, cnt, S, R, nblk, slot_base, recoff, cursor, list);
+  if ((e = cudaGetLastError()) != cudaSuccess || !ptok) return e;
+  if (B * nblk >= (1 << 30)) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  pair_tokens_kernel<<<sms * 4, 256, 0, s>>>(nrec, recoff, list, pairoff, pairbj, B * nblk, nblk, blk, S, own, tpt,
+                                              ptok, pinfo);
   return cudaGetLastError();
 }
 

@@ -130,11 +130,9 @@ struct AttnArgs {
   // mask, then the tokens that recalled it), each with the G = Hq / Hkv query heads of one KV
   // group.  No o is written: each row leaves its partial softmax result, O / l in bf16 and the
   // log2 normaliser m + log2(l), in slot `slot` of its token, for merge_partials to combine.
-  const int* g_nrec = nullptr;     // [B*nblk] tokens that recalled block (b, j)
-  const int* g_recoff = nullptr;   // [B*nblk] where their entries start in g_list
-  const int* g_list = nullptr;     // entries (t << 5) | slot, t the position in the sequence
   const int* g_pairoff = nullptr;  // [B*nblk + 1] first tile pair of each block; [B*nblk] = all pairs
-  const int* g_pairbj = nullptr;   // [all pairs] the block (b * nblk + j) of each tile pair
+  const int* g_pinfo = nullptr;    // [all pairs] b * nblk + j of the pair's block, bit 30: second tile exists
+  const int* g_ptok = nullptr;     // [all pairs][2 tpt] the pair's list entries (t << 5) | slot, -1 past the end
   int g_own = 0, nblk = 0, blk = 0, nslot = 0;
   void* part_o = nullptr;          // [B*S][nslot][Hq*dh] bf16
   float* part_lse = nullptr;       // [B*S][nslot][Hq]
@@ -157,9 +155,11 @@ inline size_t gathered_max_pairs(long long T, int R, int own, int tpt, long long
 // recall rank r.  Scratch from the caller: nrec, recoff, cursor [B*nblk], pairoff [B*nblk + 1],
 // list [B*S*R], pairbj [gathered_max_pairs()].  tpt: tokens per 128-row query tile
 // (128 / gathered_rows_per_token(Hq / Hkv)).
+// ptok, pinfo (nullable, [max pairs][2 tpt] and [max pairs]): per tile pair its list entries, own
+// tokens as (t << 5) | 0, -1 past the end, and its block with bit 30 set when its second tile exists.
 cudaError_t block_lists(const int* idx, const int* cnt, int B, int S, int R, int blk, int nblk, int own,
                         int slot_base, int tpt, int* nrec, int* recoff, int* cursor, int* pairoff, int* pairbj,
-                        int* list, cudaStream_t s);
+                        int* list, int* ptok, int* pinfo, cudaStream_t s);
 struct MergeArgs {
   const void* part_o; const float* part_lse; int nslot;
   const int* cnt; int own;          // partial slots of token t: [0, cnt[t] + own)

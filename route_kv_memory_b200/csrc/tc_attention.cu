@@ -77,32 +77,32 @@ __device__ __forceinline__ int snake_item(int r, int grid, int cta, int nwork) {
   return w < nwork ? w : -1;
 }
 
-// MODE 1 work item: tile pair p of the row list of block j of sequence b, KV group g.
+// MODE 1 work item: tile pair P (of the row list of block j of sequence b) for KV group g.
+// g_pinfo[P] = b * nblk + j, bit 30 set when the pair's second list tile exists; g_ptok[P] holds the
+// pair's 2 tpt list entries ((t << 5) | slot, -1 past the end), written when the lists are built.
 struct GWork {
-  int b, g, j, p, own, entries, recbase;
+  int b, g, j, P, t1;
 };
 __device__ __forceinline__ GWork gwork_item(int w, const AttnArgs& a) {
   GWork r;
-  const int P = w / a.Hkv;
-  r.g = w - P * a.Hkv;
-  const int lo = a.g_pairbj[P];
-  r.p = P - a.g_pairoff[lo];
-  r.b = lo / a.nblk;
-  r.j = lo - r.b * a.nblk;
-  r.own = a.g_own ? min(a.blk, a.S - r.j * a.blk) : 0;
-  r.entries = r.own + a.g_nrec[lo];
-  r.recbase = a.g_recoff[lo];
+  r.P = w / a.Hkv;
+  r.g = w - r.P * a.Hkv;
+  const int info = a.g_pinfo[r.P];
+  const int bj = info & 0x3fffffff;
+  r.t1 = (info >> 30) & 1;
+  r.b = bj / a.nblk;
+  r.j = bj - r.b * a.nblk;
   return r;
 }
-// Token (position in the sequence) and partial slot of entry e of the item's list; -1 past the end.
-__device__ __forceinline__ int gwork_token(const AttnArgs& a, const GWork& it, int e, int* slot) {
-  *slot = 0;
-  if (e >= it.entries) return -1;
-  if (e < it.own) return it.j * a.blk + e;
-  const int v = a.g_list[it.recbase + e - it.own];
-  *slot = v & 31;
+// List entry k of local tile t (t = 0: the pair's second list tile, t = 1: its first); -1 if none.
+__device__ __forceinline__ int gwork_entry(const AttnArgs& a, int P, int t, int k, int tpt) {
+  return a.g_ptok[(size_t)P * 2 * tpt + (1 - t) * tpt + k];
+}
+// Token (position in the sequence) of an entry, -1 for none; its partial slot in *slot.
+__device__ __forceinline__ int entry_token(int v, int S, int* slot) {
+  *slot = v >= 0 ? (v & 31) : 0;
   const int t = v >> 5;
-  return t < a.S ? t : -1;
+  return v >= 0 && t < S ? t : -1;
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -182,8 +182,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // empty (0 key tiles); both read the same mt key tiles of block j.
   auto item_tiles = [&](int w, int& n0, int& n1) {
     if constexpr (GA) {
-      const GWork it = gwork_item(w, a);
-      n0 = (2 * it.p + 1) * tpt < it.entries ? mt : 0;
+      n0 = (a.g_pinfo[w / a.Hkv] >> 30) & 1 ? mt : 0;
       n1 = mt;
     } else {
       const Work it = work_item(w, a.B, a.Hq, npairs);
@@ -210,14 +209,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       auto lookup = [&](int w) {
         it = gwork_item(w, a);
         for (int t = 0; t < 2; ++t) {
-          const int e0 = (2 * it.p + 1 - t) * tpt;
-          tk[t] = -1;
-          if (e0 >= it.entries) continue;
           int slot;
-          if (lane < tpt) tk[t] = gwork_token(a, it, e0 + lane, &slot);
-          if (RPT != 8)
+          tk[t] = lane < tpt ? entry_token(gwork_entry(a, it.P, t, lane, tpt), a.S, &slot) : -1;
+          if (RPT != 8 && (t == 1 || it.t1))
             for (int k = lane; k < tpt; k += 32)
-              stok[t * BQ + k] = k == lane ? tk[t] : gwork_token(a, it, e0 + k, &slot);
+              stok[t * BQ + k] = k == lane ? tk[t] : entry_token(gwork_entry(a, it.P, t, k, tpt), a.S, &slot);
         }
       };
       int kvit = 0;
@@ -247,7 +243,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         bool qok = true;
         for (int t = 0; t < 2; ++t) {
-          const bool full = (2 * it.p + 1 - t) * tpt < it.entries;
+          const bool full = t == 1 || it.t1;
           const int tok = tk[t];
           const bool ok_t = mbar_wait(&q_empty[t], (wi & 1) ^ 1, abort, status);
           if (!__all_sync(0xffffffffu, ok_t)) {
@@ -466,11 +462,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       bool masked;  // warp-uniform: the causal mask applies to some row of the warp
       if constexpr (GA) {
         const GWork it = gwork_item(w, a);
-        const int lt = 2 * it.p + 1 - t, k = r / RPT, hh = r - k * RPT;
+        const int k = r / RPT, hh = r - k * RPT;
         b = it.b;
         h = it.g * G + hh;
-        nkv = lt * tpt < it.entries ? mt : 0;
-        row = k < tpt && hh < G ? gwork_token(a, it, lt * tpt + k, &slot) : -1;
+        nkv = t == 1 || it.t1 ? mt : 0;
+        row = k < tpt && hh < G ? entry_token(gwork_entry(a, it.P, t, k, tpt), a.S, &slot) : -1;
         key0 = it.j * a.blk;  // keys of the block's tiles start here
         row_lim = row >= 0 && row / a.blk == it.j ? row : kNoMask;  // the block's own tokens only
         masked = __any_sync(0xffffffffu, row_lim != kNoMask);
@@ -687,7 +683,7 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (ga && (((uintptr_t)a.part_o & 31) || !a.g_nrec || !a.g_pairbj || !a.g_recoff || !a.g_list || !a.part_o || !a.part_lse || a.nblk < 1 || a.nslot < 1 ||
+  if (ga && (((uintptr_t)a.part_o & 31) || !a.g_pinfo || !a.g_ptok || !a.part_o || !a.part_lse || a.nblk < 1 || a.nslot < 1 ||
              a.blk < tca::BKV || a.blk % tca::BKV || a.Hq % a.Hkv || a.Hq / a.Hkv > tca::BQ ||
              (long long)a.nblk * a.blk < a.S))
     return cudaErrorInvalidValue;
