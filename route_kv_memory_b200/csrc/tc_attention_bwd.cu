@@ -90,7 +90,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* dq_full = bars + 8;
   uint64_t* dq_empty = bars + 9;
   uint64_t* drain = bars + 10;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 11);
+  uint64_t* s_free = bars + 11;   // the compute warps hold S in registers: its columns are free
+  uint64_t* dp_full = bars + 12;  // dP has landed
+  uint32_t* tmem_slot = (uint32_t*)(bars + 13);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -104,6 +106,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(p_full, NCOMPUTE);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, NCOMPUTE);
+    mbar_init(s_free, NCOMPUTE);
+    mbar_init(dp_full, 1);
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -169,16 +173,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint64_t qd = sdesc_kmajor_sw128(sQ), dod = sdesc_kmajor_sw128(sdO);
-      int kvit = 0, pc = 0;
-      bool ok = true;
-      // dQ += scale*dS K_j for the key tile in ring slot `st`, dS read from TMEM over S
+      int kvit = 0, pc = 0, sf = 0;
+      bool ok = true, first = true;
+      // S = Q K^T for the key tile in ring slot `st`
+      auto issue_s = [&](int st) {
+        const uint64_t kd = sdesc_kmajor_sw128(sKV + st * 2 * C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          umma_bf16_ss(tbase + S_COL, qd + kstep(kk, C::HALF), kd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+        umma_commit(s_full);
+      };
+      // dP = dO V^T
+      auto issue_dp = [&](int st) {
+        const uint64_t vd = sdesc_kmajor_sw128(sKV + st * 2 * C::TILE + C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          umma_bf16_ss(tbase + P_COL, dod + kstep(kk, C::HALF), vd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+        umma_commit(dp_full);
+      };
+      // dQ += scale*dS K_j, dS packed over the dP columns
       auto issue_dq = [&](int st, bool acc) {
         const uint64_t kd = sdesc_mnmajor_sw128(sKV + st * 2 * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_ts(tbase + Q_COL, tbase + S_COL + packed_col(kk), kd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+          umma_bf16_ts(tbase + Q_COL, tbase + P_COL + packed_col(kk), kd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
                        (acc || kk) ? 1u : 0u);
       };
+      // S(j+1) goes in as soon as the compute warps hold S(j) in registers, so their exponentials
+      // of tile j+1 run under dQ(j) and dP(j+1); dP(j+1) follows dQ(j), which reads dS(j) over dP.
       for (int rr = 0; ok; ++rr) {
         const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
         if (w < 0) break;
@@ -186,36 +208,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         item(w, b, h, qt);
         const int n = qt + 1;
         if (!mbar_wait(q_full, rr & 1, abort, status)) break;
+        if (!mbar_wait(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
+        if (!first) {
+          if (!mbar_wait(s_free, sf & 1, abort, status)) break;
+          ++sf;
+        }
+        first = false;
+        tc_fence_after();
+        issue_s(kvit & 1);
+        issue_dp(kvit & 1);
+        if (n == 1) umma_commit(q_empty);
         for (int j = 0; j < n; ++j) {
-          const int cur = kvit + j, st = cur & 1;
-          if (!mbar_wait(&kv_full[st], (cur >> 1) & 1, abort, status)) { ok = false; break; }
-          if (j > 0) {  // finish key tile j-1 before S_j overwrites its dS
-            if (!mbar_wait(p_full, pc & 1, abort, status)) { ok = false; break; }
-            ++pc;
-            if (j == 1 && !mbar_wait(dq_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
+          const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
+          if (j + 1 < n) {
+            if (!mbar_wait(&kv_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
+            if (!mbar_wait(s_free, sf & 1, abort, status)) { ok = false; break; }
+            ++sf;
             tc_fence_after();
-            issue_dq((cur - 1) & 1, j > 1);
-            umma_commit(&kv_empty[(cur - 1) & 1]);
+            issue_s(nst);
           }
+          if (!mbar_wait(p_full, pc & 1, abort, status)) { ok = false; break; }
+          ++pc;
+          if (j == 0 && !mbar_wait(dq_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t kd = sdesc_kmajor_sw128(sKV + st * 2 * C::TILE);
-          const uint64_t vd = sdesc_kmajor_sw128(sKV + st * 2 * C::TILE + C::TILE);
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk)
-            umma_bf16_ss(tbase + S_COL, qd + kstep(kk, C::HALF), kd + kstep(kk, C::HALF), IDESC_S, kk != 0);
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk)
-            umma_bf16_ss(tbase + P_COL, dod + kstep(kk, C::HALF), vd + kstep(kk, C::HALF), IDESC_S, kk != 0);
-          umma_commit(s_full);
-          if (j == n - 1) umma_commit(q_empty);
+          issue_dq(st, j > 0);
+          umma_commit(&kv_empty[st]);
+          if (j + 1 < n) {
+            issue_dp(nst);
+            if (j + 2 == n) umma_commit(q_empty);  // Q and dO's last use
+          }
         }
         if (!ok) break;
-        if (!mbar_wait(p_full, pc & 1, abort, status)) break;
-        ++pc;
-        if (n == 1 && !mbar_wait(dq_empty, (rr & 1) ^ 1, abort, status)) break;
-        tc_fence_after();
-        issue_dq((kvit + n - 1) & 1, n > 1);
-        umma_commit(&kv_empty[(kvit + n - 1) & 1]);
         umma_commit(dq_full);
         kvit += n;
       }
@@ -251,19 +274,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         const int lim = valid ? row - j * BT : -1;  // keys c > lim are masked (all, for a padding row)
         const bool diag = __any_sync(0xffffffffu, j == n - 1 || !valid);  // warp-uniform
-        // the second chunk's TMEM loads are in flight while the first is processed
-        uint32_t sv[2][32], pv[2][32];
+        // phase 1: this half's 64 scores into registers (S's columns are then free for S(j+1)),
+        // P = 2^(s sl2 - lse) in float32
+        uint32_t sv[2][32];
         tmem_ld32(s_tmem + 64 * half, sv[0]);
-        tmem_ld32(p_tmem + 64 * half, pv[0]);
+        tmem_ld32(s_tmem + 64 * half + 32, sv[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = 2 * half + cc;
-          tmem_ld_wait();
-          if (cc == 0) {
-            tmem_ld32(s_tmem + 64 * half + 32, sv[1]);
-            tmem_ld32(p_tmem + 64 * half + 32, pv[1]);
-          }
-          uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float2 x2 = __ffma2_rn(make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1])),
@@ -274,12 +296,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               p0 = k0 <= lim ? p0 : 0.f;
               p1 = k0 + 1 <= lim ? p1 : 0.f;
             }
+            sv[cc][2 * e] = __float_as_uint(p0);
+            sv[cc][2 * e + 1] = __float_as_uint(p1);
+          }
+        }
+        // phase 2: dS = scale P (dP - D), packed over the first 32 of this half's dP columns
+        if (!mbar_wait(dp_full, sit & 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t pv[2][32];
+        tmem_ld32(p_tmem + 64 * half, pv[0]);
+        tmem_ld32(p_tmem + 64 * half + 32, pv[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
             const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(pv[cc][2 * e]), __uint_as_float(pv[cc][2 * e + 1])),
                                          ndrowv);
-            const float2 r2 = __fmul2_rn(__fmul2_rn(make_float2(p0, p1), scalev), d2);
+            const float2 r2 = __fmul2_rn(
+                __fmul2_rn(make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1])), scalev), d2);
             pk[e] = pack2(r2.x, r2.y);
           }
-          tmem_st16(s_tmem + 64 * half + cc * 16, pk);
+          tmem_st16(p_tmem + 64 * half + cc * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -342,7 +381,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* acc_full = bars + 8;
   uint64_t* acc_empty = bars + 9;
   uint64_t* drain = bars + 10;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 11);
+  uint64_t* s_free = bars + 11;   // the compute warps hold S^T in registers: its columns are free
+  uint64_t* dp_full = bars + 12;  // dP^T has landed
+  uint32_t* tmem_slot = (uint32_t*)(bars + 13);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -356,6 +397,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(p_full, NCOMPUTE);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, NCOMPUTE);
+    mbar_init(s_free, NCOMPUTE);
+    mbar_init(dp_full, 1);
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -426,21 +469,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint64_t kd = sdesc_kmajor_sw128(sK), vd = sdesc_kmajor_sw128(sV);
-      int qdit = 0, pc = 0;
-      bool ok = true;
-      // dV += P^T dO and dK += scale*dS^T Q for the query stage `st` (P^T, dS^T read from TMEM)
+      int qdit = 0, pc = 0, sf = 0;
+      bool ok = true, first = true;
+      // S^T = K Q^T for the query stage `st`
+      auto issue_s = [&](int st) {
+        const uint64_t qd = sdesc_kmajor_sw128(sQD + st * C::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          umma_bf16_ss(tbase + S_COL, kd + kstep(kk, C::HALF), qd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+        umma_commit(s_full);
+      };
+      // dP^T = V dO^T
+      auto issue_dp = [&](int st) {
+        const uint64_t dod = sdesc_kmajor_sw128(sQD + st * C::STAGE + C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          umma_bf16_ss(tbase + P_COL, vd + kstep(kk, C::HALF), dod + kstep(kk, C::HALF), IDESC_S, kk != 0);
+        umma_commit(dp_full);
+      };
+      // dV += P^T dO and dK += scale*dS^T Q; the compute warps pack P^T and dS^T over the dP^T
+      // columns: K-step kk (16 queries) of P^T at 64 (kk / 4) + 32 ((kk / 2) % 2) + 8 (kk % 2), of dS^T 16 further
       auto issue_acc = [&](int st, bool acc) {
         const uint64_t dq = sdesc_mnmajor_sw128(sQD + st * C::STAGE);
         const uint64_t dd = sdesc_mnmajor_sw128(sQD + st * C::STAGE + C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_ts(tbase + V_COL, tbase + S_COL + packed_col(kk), dd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+        for (int kk = 0; kk < BT / 16; ++kk) {
+          const uint32_t pcol = P_COL + 64 * (kk >> 2) + 32 * ((kk >> 1) & 1) + 8 * (kk & 1);
+          umma_bf16_ts(tbase + V_COL, tbase + pcol, dd + (uint64_t)(kk * (2048 >> 4)), IDESC_D, (acc || kk) ? 1u : 0u);
+          umma_bf16_ts(tbase + K_COL, tbase + pcol + 16, dq + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
                        (acc || kk) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_ts(tbase + K_COL, tbase + P_COL + packed_col(kk), dq + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
-                       (acc || kk) ? 1u : 0u);
+        }
       };
+      // S^T(s+1) goes in as soon as the compute warps hold S^T(s) in registers, so their
+      // exponentials of step s+1 run under dV / dK(s) and dP^T(s+1); dP^T(s+1) follows dV / dK(s),
+      // which read P^T(s) and dS^T(s) over the dP^T columns.
       for (int rr = 0; ok; ++rr) {
         const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
         if (w < 0) break;
@@ -448,35 +510,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         item(w, b, g, kt);
         const int n = G * (nqt - kt);
         if (!mbar_wait(kv_full, rr & 1, abort, status)) break;
+        if (!mbar_wait(&qd_full[qdit & 1], (qdit >> 1) & 1, abort, status)) break;
+        if (!first) {
+          if (!mbar_wait(s_free, sf & 1, abort, status)) break;
+          ++sf;
+        }
+        first = false;
+        tc_fence_after();
+        issue_s(qdit & 1);
+        issue_dp(qdit & 1);
         for (int s = 0; s < n; ++s) {
-          const int cur = qdit + s, st = cur & 1;
-          if (!mbar_wait(&qd_full[st], (cur >> 1) & 1, abort, status)) { ok = false; break; }
-          if (s > 0) {  // finish step s-1 before S^T_s overwrites its P^T
-            if (!mbar_wait(p_full, pc & 1, abort, status)) { ok = false; break; }
-            ++pc;
-            if (s == 1 && !mbar_wait(acc_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
+          const int cur = qdit + s, st = cur & 1, nst = (cur + 1) & 1;
+          if (s + 1 < n) {
+            if (!mbar_wait(&qd_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
+            if (!mbar_wait(s_free, sf & 1, abort, status)) { ok = false; break; }
+            ++sf;
             tc_fence_after();
-            issue_acc((cur - 1) & 1, s > 1);
-            umma_commit(&qd_empty[(cur - 1) & 1]);
+            issue_s(nst);
           }
+          if (!mbar_wait(p_full, pc & 1, abort, status)) { ok = false; break; }
+          ++pc;
+          if (s == 0 && !mbar_wait(acc_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t qd = sdesc_kmajor_sw128(sQD + st * C::STAGE);
-          const uint64_t dod = sdesc_kmajor_sw128(sQD + st * C::STAGE + C::TILE);
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk)
-            umma_bf16_ss(tbase + S_COL, kd + kstep(kk, C::HALF), qd + kstep(kk, C::HALF), IDESC_S, kk != 0);
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk)
-            umma_bf16_ss(tbase + P_COL, vd + kstep(kk, C::HALF), dod + kstep(kk, C::HALF), IDESC_S, kk != 0);
-          umma_commit(s_full);
+          issue_acc(st, s > 0);
+          umma_commit(&qd_empty[st]);
+          if (s + 1 < n) issue_dp(nst);
         }
         if (!ok) break;
-        if (!mbar_wait(p_full, pc & 1, abort, status)) break;
-        ++pc;
-        if (n == 1 && !mbar_wait(acc_empty, (rr & 1) ^ 1, abort, status)) break;
-        tc_fence_after();
-        issue_acc((qdit + n - 1) & 1, n > 1);
-        umma_commit(&qd_empty[(qdit + n - 1) & 1]);
         umma_commit(kv_empty);
         umma_commit(acc_full);
         qdit += n;
@@ -515,28 +575,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int q0 = qt * BT, cmax = a.S - q0, cmin = key - q0;
         const bool masked = __any_sync(0xffffffffu, cmin > 64 * half || cmax < 64 * half + 64);  // warp-uniform
         const float2 sl2v = make_float2(sl2, sl2), scalev = make_float2(a.scale, a.scale);
-        // the second chunk's TMEM loads are in flight while the first is processed
-        uint32_t sv[2][32], pv[2][32];
+        // phase 1: this half's 64 scores into registers (S^T's columns are then free for the next
+        // step), P^T = 2^(s sl2 - lse) in float32
+        uint32_t sv[2][32];
         tmem_ld32(s_tmem + 64 * half, sv[0]);
-        tmem_ld32(p_tmem + 64 * half, pv[0]);
+        tmem_ld32(s_tmem + 64 * half + 32, sv[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = 2 * half + cc;
-          tmem_ld_wait();
-          if (cc == 0) {
-            tmem_ld32(s_tmem + 64 * half + 32, sv[1]);
-            tmem_ld32(p_tmem + 64 * half + 32, pv[1]);
-          }
-          uint32_t pp[16], pd[16];
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {  // lse and D of four query columns per shared-memory load
+          for (int e4 = 0; e4 < 8; ++e4) {  // lse of four query columns per shared-memory load
             const float4 l4 = *(const float4*)(lse2 + c * 32 + 4 * e4);
-            const float4 d4 = *(const float4*)(dsum + c * 32 + 4 * e4);
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
               const int e = 2 * e4 + k, c0 = c * 32 + 2 * e;
               const float2 nl = k ? make_float2(-l4.z, -l4.w) : make_float2(-l4.x, -l4.y);
-              const float2 nd = k ? make_float2(-d4.z, -d4.w) : make_float2(-d4.x, -d4.y);
               const float2 x2 = __ffma2_rn(make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1])),
                                            sl2v, nl);
               float p0 = ex2(x2.x), p1 = ex2(x2.y);
@@ -544,15 +601,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 p0 = (c0 < cmax && c0 >= cmin) ? p0 : 0.f;
                 p1 = (c0 + 1 < cmax && c0 + 1 >= cmin) ? p1 : 0.f;
               }
-              pp[e] = pack2(p0, p1);
-              const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(pv[cc][2 * e]), __uint_as_float(pv[cc][2 * e + 1])),
-                                           nd);
-              const float2 r2 = __fmul2_rn(__fmul2_rn(make_float2(p0, p1), scalev), d2);
+              sv[cc][2 * e] = __float_as_uint(p0);
+              sv[cc][2 * e + 1] = __float_as_uint(p1);
+            }
+          }
+        }
+        // phase 2: dS^T = scale P^T (dP^T - D); P^T and dS^T packed over this half's dP^T columns,
+        // chunk cc at [32 cc, 32 cc + 16) and [32 cc + 16, 32 cc + 32) of the half
+        if (!mbar_wait(dp_full, sit & 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {  // chunk by chunk: a chunk's outputs go only over its own inputs
+          const int c = 2 * half + cc;
+          uint32_t pv[32];
+          tmem_ld32(p_tmem + 64 * half + 32 * cc, pv);
+          tmem_ld_wait();
+          uint32_t pp[16], pd[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 d4 = *(const float4*)(dsum + c * 32 + 4 * e4);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int e = 2 * e4 + k;
+              const float2 nd = k ? make_float2(-d4.z, -d4.w) : make_float2(-d4.x, -d4.y);
+              const float2 p2 = make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1]));
+              pp[e] = pack2(p2.x, p2.y);
+              const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(pv[2 * e]), __uint_as_float(pv[2 * e + 1])), nd);
+              const float2 r2 = __fmul2_rn(__fmul2_rn(p2, scalev), d2);
               pd[e] = pack2(r2.x, r2.y);
             }
           }
-          tmem_st16(s_tmem + 64 * half + cc * 16, pp);
-          tmem_st16(p_tmem + 64 * half + cc * 16, pd);
+          tmem_st16(p_tmem + 64 * half + 32 * cc, pp);
+          tmem_st16(p_tmem + 64 * half + 32 * cc + 16, pd);
         }
         tmem_st_wait();
         tc_fence_before();
