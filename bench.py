@@ -419,10 +419,10 @@ def run_train(args, rank, world, local_rank):
 def train_kernels() -> int:
     """Kernel launches of one training step: the 10 of the prefill, then the backward's weight
     transposes (2), D, the two attention-backward kernels, the router pre-activation GEMM, the EMA
-    and recalled-mean recomputes (2), the router backward, the dq GEMM and its combine (2), the
-    recall lists (3), the memory adjoint (4), the dX GEMM, the activation transposes (4) and the
-    two weight-gradient GEMMs."""
-    return 10 + 2 + 1 + 2 + 1 + 2 + 1 + 2 + 3 + 4 + 1 + 4 + 2
+    and recalled-mean recomputes (2), the router backward, the dq GEMM (which adds the attention's
+    dq in its epilogue), the recall lists (3), the memory adjoint (4), the dX GEMM, the activation
+    transposes (4) and the two weight-gradient GEMMs."""
+    return 10 + 2 + 1 + 2 + 1 + 2 + 1 + 1 + 3 + 4 + 1 + 4 + 2
 
 
 def run_decode(args, cfg_prefill, inp_unused, weights_unused, dev, layer_pack=None):

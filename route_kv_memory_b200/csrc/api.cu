@@ -763,7 +763,7 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
 struct TrainWs {
   PrefillWs fw;
   int Spad, Tp, ncat, nball;
-  size_t lse, dsum, dq, dy, ema, m3, hrec, dlam, dh, dqr, gsum, rsum, cs, acat, wcatT, wr1, xT, acatT, qT, dhT;
+  size_t lse, dsum, dq, dy, ema, m3, hrec, dlam, dh, gsum, rsum, cs, acat, wcatT, wr1, xT, acatT, qT, dhT;
   size_t nrec, recoff, cursor, pairoff, pairbj, list, total;
 };
 static TrainWs train_ws(const Dims& d) {
@@ -785,7 +785,6 @@ static TrainWs train_ws(const Dims& d) {
   w.hrec = o; o += al(T * 2 * d.rh * 4);
   w.dlam = o; o += al(T * 3 * 4);
   w.dh = o; o += al(T * d.rh * 2);
-  w.dqr = o; o += al(T * d.dq * 4);
   w.gsum = o; o += al(nbj * W * 4);
   w.rsum = o; o += al((size_t)d.B * w.nball * W * 4);
   w.cs = o; o += al((size_t)d.B * (w.nball + 1) * W * 4);
@@ -866,7 +865,6 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
   float* hrec = (float*)P(ws, W.hrec);
   float* dlam = dlambda_out ? dlambda_out : (float*)P(ws, W.dlam);
   void* dh = P(ws, W.dh);
-  float* dqr = (float*)P(ws, W.dqr);
   void* acat = P(ws, W.acat);
   void* wcatT = P(ws, W.wcatT);
   void* wr1 = P(ws, W.wr1);
@@ -912,14 +910,13 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
   rb.B = d.B; rb.S = d.S; rb.route_mode = d.route; rb.tiers = d.tiers;
   CUDA_TRY(router_backward(rb, s));
   STAGE(s);
-  // dq = dq (attention) + dh W_r1^T, into the first dq columns of [dq | U] (bf16)
+  // dq = dh W_r1^T + dq (attention, added in the epilogue), into the first dq columns of [dq | U] (bf16)
   {
     Epilogue ep{};
     ep.nseg = 1;
-    ep.seg[0] = OutSeg{0, d.dq, dqr, d.dq, 0};
+    ep.seg[0] = OutSeg{0, d.dq, acat, W.ncat, 1, dq, d.dq};
     CUDA_TRY(gemm_tn_bf16_tc(dh, d.rh, wr1, d.rh, (int)T, d.dq, d.rh, ep, status_ptr(), s));
   }
-  CUDA_TRY(add_to_bf16(dq, dqr, (long long)T, d.dq, acat, W.ncat, s));
   STAGE(s);
   // U = lam1 dY + EMA^T(lam2 dY) + M^T(lam3 dY), into the last 2 dkv columns
   {

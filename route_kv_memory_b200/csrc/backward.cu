@@ -243,21 +243,6 @@ __global__ void __launch_bounds__(64) ema_adj_apply_kernel(const float* __restri
   }
 }
 
-// out[t][0:n] = bf16(a[t] + b[t]) (float32 rows of n), row stride ldo.
-__global__ void add_to_bf16_kernel(const float* __restrict__ x, const float* __restrict__ y, long long rows, int n,
-                                   bf16* __restrict__ out, int ldo) {
-  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-  if (i >= rows * n) return;
-  const long long r = i / n;
-  const int c = (int)(i - r * n);
-  const float4 p = *(const float4*)(x + i), q = *(const float4*)(y + i);
-  __nv_bfloat162 a0 = __floats2bfloat162_rn(p.x + q.x, p.y + q.y), a1 = __floats2bfloat162_rn(p.z + q.z, p.w + q.w);
-  uint2 pk;
-  pk.x = *(uint32_t*)&a0;
-  pk.y = *(uint32_t*)&a1;
-  *(uint2*)(out + r * ldo + c) = pk;
-}
-
 }  // namespace
 
 cudaError_t attention_dsum(const void* dout, const void* o, int B, int S, int Hq, int dh, int ld, float* dsum,
@@ -304,14 +289,6 @@ cudaError_t memory_adjoint(const MemAdjArgs& a, cudaStream_t s) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ema_adj_apply_kernel<<<dim3(gx, nball, a.B), 64, 0, s>>>(a.dy, a.width, a.lam, a.S, nball, a.nblk, a.blk, a.alpha,
                                                            a.cs, a.gsum, (bf16*)a.u, a.ldu);
-  return cudaGetLastError();
-}
-
-cudaError_t add_to_bf16(const float* x, const float* y, long long rows, int n, void* out, int ldo, cudaStream_t s) {
-  if (rows <= 0) return cudaSuccess;
-  if (n % 4 || ldo % 4) return cudaErrorInvalidValue;
-  const long long m = rows * n / 4;
-  add_to_bf16_kernel<<<(unsigned)((m + 255) / 256), 256, 0, s>>>(x, y, rows, n, (bf16*)out, ldo);
   return cudaGetLastError();
 }
 

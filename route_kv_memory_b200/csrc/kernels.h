@@ -16,6 +16,8 @@ struct OutSeg {
   void* ptr;           // element (m, n) goes to ptr[m * ld + (n - n_begin)]
   int ld;
   int is_bf16;         // 1: bf16 store, 0: float32 store
+  const float* add = nullptr;  // when set, add[m * ld_add + (n - n_begin)] is added before the store
+  int ld_add = 0;              //   (ld_add % 4 == 0, 16-byte aligned)
 };
 constexpr int kMaxSegs = 6;
 struct Epilogue {
@@ -213,8 +215,6 @@ struct MemAdjArgs {
   void* u; int ldu;  // bf16 rows of U (stride ldu)
 };
 cudaError_t memory_adjoint(const MemAdjArgs& a, cudaStream_t s);
-// out[r][0:n] = bf16(x[r] + y[r]) for float32 rows of n (out row stride ldo).
-cudaError_t add_to_bf16(const float* x, const float* y, long long rows, int n, void* out, int ldo, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode
 struct DecodeArgs {

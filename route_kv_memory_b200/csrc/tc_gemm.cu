@@ -49,13 +49,24 @@ __device__ __forceinline__ void store1(const Epilogue& ep, int m, int n, float v
 }
 
 // Columns n .. n+31 of row m.
-__device__ __forceinline__ void store_chunk(const Epilogue& ep, int m, int n, const uint32_t (&r)[32], int N) {
+__device__ __forceinline__ void store_chunk(const Epilogue& ep, int m, int n, uint32_t (&r)[32], int N) {
 #pragma unroll
   for (int s = 0; s < kMaxSegs; ++s) {
     if (s >= ep.nseg) break;
     const OutSeg& g = ep.seg[s];
     if (n >= g.n_begin && n + 32 <= g.n_end && n + 32 <= N) {
       const size_t off = (size_t)m * g.ld + (n - g.n_begin);
+      if (g.add) {  // a float32 addend row (e.g. another contribution to the same gradient)
+        const float4* ad = (const float4*)(g.add + (size_t)m * g.ld_add + (n - g.n_begin));
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 x = ad[v];
+          r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + x.x);
+          r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + x.y);
+          r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + x.z);
+          r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + x.w);
+        }
+      }
       if (g.is_bf16) {
         bf16* p = (bf16*)g.ptr + off;
         if ((off & 7) == 0) {
