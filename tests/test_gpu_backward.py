@@ -94,6 +94,9 @@ CASES = [
     small("bwd_top2", route_mode="top2", seed=203),
     small("bwd_l1_l2_only", tiers=3, seed=204),
     small("bwd_short_no_blocks", seq=24, block=32, seed=205),
+    small("bwd_mha_dh128", seq=320, n_q_heads=2, n_kv_heads=2, d_head=128, router_hidden=128, block=64, seed=206),
+    small("bwd_blocks_of_256", batch=2, seq=600, n_q_heads=8, n_kv_heads=2, d_head=64, block=256, recall_r=2,
+          seed=207),
 ]
 
 
