@@ -291,8 +291,8 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
-BACKWARD_STAGES = ["weight_transposes", "dsum", "attention_bwd", "router_preact_gemm", "router_bwd", "dq_gemm",
-                   "memory_adjoint", "dx_gemm", "act_transposes", "weight_grad_gemms"]
+BACKWARD_STAGES = ["dsum", "attention_bwd", "router_preact_gemm", "router_bwd", "dq_gemm", "memory_adjoint", "dx_gemm",
+                   "weight_grad_gemms"]
 
 
 def train_flops(cfg) -> dict:
@@ -417,12 +417,12 @@ def run_train(args, rank, world, local_rank):
 
 
 def train_kernels() -> int:
-    """Kernel launches of one training step: the 10 of the prefill, then the backward's weight
-    transposes (2), D, the two attention-backward kernels, the router pre-activation GEMM, the EMA
-    and recalled-mean recomputes (2), the router backward, the dq GEMM (which adds the attention's
-    dq in its epilogue), the recall lists (3), the memory adjoint (4), the dX GEMM, the activation
-    transposes (4) and the two weight-gradient GEMMs."""
-    return 10 + 2 + 1 + 2 + 1 + 2 + 1 + 1 + 3 + 4 + 1 + 4 + 2
+    """Kernel launches of one training step: the 10 of the prefill, then the backward's D, the two
+    attention-backward kernels, the router pre-activation GEMM, the EMA and recalled-mean recomputes
+    (2), the router backward, the dq GEMM (which adds the attention's dq in its epilogue), the recall
+    lists (3), the memory adjoint (4), the dX GEMM and the two weight-gradient GEMMs (their operands
+    read MN-major as stored, no transposes)."""
+    return 10 + 1 + 2 + 1 + 2 + 1 + 1 + 3 + 4 + 1 + 2
 
 
 def run_decode(args, cfg_prefill, inp_unused, weights_unused, dev, layer_pack=None):

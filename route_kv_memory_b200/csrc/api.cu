@@ -762,8 +762,8 @@ int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x
 // by the attention normalisers the training forward writes and the backward's own scratch.
 struct TrainWs {
   PrefillWs fw;
-  int Spad, Tp, ncat, nball;
-  size_t lse, dsum, dq, dy, ema, m3, hrec, dlam, dh, gsum, rsum, cs, acat, wcatT, wr1, xT, acatT, qT, dhT;
+  int Spad, ncat, nball;
+  size_t lse, dsum, dq, dy, ema, m3, hrec, dlam, dh, gsum, rsum, cs, acat;
   size_t nrec, recoff, cursor, pairoff, pairbj, list, total;
 };
 static TrainWs train_ws(const Dims& d) {
@@ -771,7 +771,6 @@ static TrainWs train_ws(const Dims& d) {
   w.fw = prefill_ws(d);
   const size_t T = d.T, W = d.width;
   w.Spad = (d.S + 127) / 128 * 128;
-  w.Tp = (int)((T + 7) / 8 * 8);  // K of the weight-gradient products, padded with zero columns
   w.ncat = d.dq + 2 * d.dkv;      // [dq | U] columns
   w.nball = (d.S + d.blk - 1) / d.blk;
   const size_t nbj = (size_t)d.B * d.nblk;
@@ -789,12 +788,6 @@ static TrainWs train_ws(const Dims& d) {
   w.rsum = o; o += al((size_t)d.B * w.nball * W * 4);
   w.cs = o; o += al((size_t)d.B * (w.nball + 1) * W * 4);
   w.acat = o; o += al(T * w.ncat * 2);
-  w.wcatT = o; o += al((size_t)d.d * w.ncat * 2);
-  w.wr1 = o; o += al((size_t)d.dq * d.rh * 2);
-  w.xT = o; o += al((size_t)d.d * w.Tp * 2);
-  w.acatT = o; o += al((size_t)w.ncat * w.Tp * 2);
-  w.qT = o; o += al((size_t)d.dq * w.Tp * 2);
-  w.dhT = o; o += al((size_t)d.rh * w.Tp * 2);
   w.nrec = o; o += al(nbj * 4);
   w.recoff = o; o += al(nbj * 4);
   w.cursor = o; o += al(nbj * 4);
@@ -866,17 +859,11 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
   float* dlam = dlambda_out ? dlambda_out : (float*)P(ws, W.dlam);
   void* dh = P(ws, W.dh);
   void* acat = P(ws, W.acat);
-  void* wcatT = P(ws, W.wcatT);
-  void* wr1 = P(ws, W.wr1);
   const float* lam = (const float*)P(ws, F.lam);
   const int* idx = (const int*)P(ws, F.idx);
   const int* cnt = (const int*)P(ws, F.cnt);
 
   prof_begin();
-  STAGE(s);
-  // weights in the orientation of the backward products: [W_q | W_k | W_v] as [d][dq + 2 dkv], W_r1 as [dq][rh]
-  CUDA_TRY(transpose(wcat, W.ncat, d.d, d.d, wcatT, W.ncat, 2, 0, s));
-  CUDA_TRY(transpose(P((void*)packed, PL.wr1T), d.rh, d.dq, d.dq, wr1, d.rh, 2, 0, s));
   STAGE(s);
   // attention: D = rowsum(dO * O), then dQ and [dK | dV]
   CUDA_TRY(cudaMemsetAsync(dsum, 0, (size_t)d.B * d.Hq * W.Spad * 4, s));
@@ -910,12 +897,13 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
   rb.B = d.B; rb.S = d.S; rb.route_mode = d.route; rb.tiers = d.tiers;
   CUDA_TRY(router_backward(rb, s));
   STAGE(s);
-  // dq = dh W_r1^T + dq (attention, added in the epilogue), into the first dq columns of [dq | U] (bf16)
+  // dq = dh W_r1^T + dq (attention, added in the epilogue), into the first dq columns of [dq | U] (bf16);
+  // the packed W_r1^T [rh][dq] is the MN-major B
   {
     Epilogue ep{};
     ep.nseg = 1;
     ep.seg[0] = OutSeg{0, d.dq, acat, W.ncat, 1, dq, d.dq};
-    CUDA_TRY(gemm_tn_bf16_tc(dh, d.rh, wr1, d.rh, (int)T, d.dq, d.rh, ep, status_ptr(), s));
+    CUDA_TRY(gemm_bf16_tc(dh, d.rh, 0, P((void*)packed, PL.wr1T), d.dq, 1, (int)T, d.dq, d.rh, ep, status_ptr(), s));
   }
   STAGE(s);
   // U = lam1 dY + EMA^T(lam2 dY) + M^T(lam3 dY), into the last 2 dkv columns
@@ -935,43 +923,29 @@ int mka_prefill_backward(const mka_config* cfg, const void* packed, const void* 
     CUDA_TRY(memory_adjoint(ma, s));
   }
   STAGE(s);
-  // dX = [dq | U] [W_q | W_k | W_v]^T
+  // dX = [dq | U] [W_q | W_k | W_v]^T; the packed rows [W_q | W_k | W_v]^T ([dq + 2 dkv][d]) are the MN-major B
   {
     Epilogue ep{};
     ep.nseg = 1;
     ep.seg[0] = OutSeg{0, d.d, dx, d.d, 1};
-    CUDA_TRY(gemm_tn_bf16_tc(acat, W.ncat, wcatT, W.ncat, (int)T, d.d, W.ncat, ep, status_ptr(), s));
+    CUDA_TRY(gemm_bf16_tc(acat, W.ncat, 0, wcat, d.d, 1, (int)T, d.d, W.ncat, ep, status_ptr(), s));
   }
   STAGE(s);
-  // weight gradients: [dW_q | dW_k | dW_v] = X^T [dq | U], dW_r1 = q^T dh, with the token axis as K
-  void* xT = P(ws, W.xT);
-  void* acatT = P(ws, W.acatT);
-  void* qT = P(ws, W.qT);
-  void* dhT = P(ws, W.dhT);
-  if ((size_t)W.Tp != T) {  // zero K padding
-    CUDA_TRY(cudaMemsetAsync(xT, 0, (size_t)d.d * W.Tp * 2, s));
-    CUDA_TRY(cudaMemsetAsync(acatT, 0, (size_t)W.ncat * W.Tp * 2, s));
-    CUDA_TRY(cudaMemsetAsync(qT, 0, (size_t)d.dq * W.Tp * 2, s));
-    CUDA_TRY(cudaMemsetAsync(dhT, 0, (size_t)d.rh * W.Tp * 2, s));
-  }
-  CUDA_TRY(transpose(x, (int)T, d.d, d.d, xT, W.Tp, 2, 0, s));
-  CUDA_TRY(transpose(acat, (int)T, W.ncat, W.ncat, acatT, W.Tp, 2, 0, s));
-  CUDA_TRY(transpose(P(ws, F.q), (int)T, d.dq, d.dq, qT, W.Tp, 2, 0, s));
-  CUDA_TRY(transpose(dh, (int)T, d.rh, d.rh, dhT, W.Tp, 2, 0, s));
-  STAGE(s);
+  // weight gradients: [dW_q | dW_k | dW_v] = X^T [dq | U], dW_r1 = q^T dh, with the token axis as K:
+  // X, [dq | U], q and dh are the MN-major operands as they are stored
   {
     Epilogue ep{};
     ep.nseg = 3;
     ep.seg[0] = OutSeg{0, d.dq, dw_q, d.dq, 0};
     ep.seg[1] = OutSeg{d.dq, d.dq + d.dkv, dw_k, d.dkv, 0};
     ep.seg[2] = OutSeg{d.dq + d.dkv, W.ncat, dw_v, d.dkv, 0};
-    CUDA_TRY(gemm_tn_bf16_tc(xT, W.Tp, acatT, W.Tp, d.d, W.ncat, W.Tp, ep, status_ptr(), s));
+    CUDA_TRY(gemm_bf16_tc(x, d.d, 1, acat, W.ncat, 1, d.d, W.ncat, (int)T, ep, status_ptr(), s));
   }
   {
     Epilogue ep{};
     ep.nseg = 1;
     ep.seg[0] = OutSeg{0, d.rh, dw_r1, d.rh, 0};
-    CUDA_TRY(gemm_tn_bf16_tc(qT, W.Tp, dhT, W.Tp, d.dq, d.rh, W.Tp, ep, status_ptr(), s));
+    CUDA_TRY(gemm_bf16_tc(P(ws, F.q), d.dq, 1, dh, d.rh, 1, d.dq, d.rh, (int)T, ep, status_ptr(), s));
   }
   STAGE(s);
   return MKA_OK;

@@ -38,6 +38,11 @@ struct Epilogue {
 // A and B 16-byte aligned); a bounded wait that runs out records MKA_ERR_DEVICE_TIMEOUT in *status.
 cudaError_t gemm_tn_bf16_tc(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
                             int* status, cudaStream_t s);
+// The same product with either operand stored MN-major instead (a_mn: A given as [K][M] with row
+// stride lda, i.e. C = A^T-of-storage * ...; b_mn: B given as [K][N] with row stride ldb); the
+// MN dimension of an MN-major operand a multiple of 8.
+cudaError_t gemm_bf16_tc(const void* A, int lda, int a_mn, const void* B, int ldb, int b_mn, int M, int N, int K,
+                         const Epilogue& ep, int* status, cudaStream_t s);
 cudaError_t gemm_tn_ffma(const void* A, int lda, int a_bf16, const void* B, int ldb, int b_bf16, int M, int N, int K,
                          const Epilogue& ep, cudaStream_t s);
 

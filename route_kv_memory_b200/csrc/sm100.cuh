@@ -113,12 +113,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// MN-major (V) descriptor: 8-key groups of 128-B rows 1024 B apart (stride byte
-// offset), 64-column halves of the head dimension 16 KB apart (leading byte offset).
-__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(const void* tile) {
+// MN-major descriptor (operand stored [K][MN], MN contiguous): 8-row groups of the K dimension,
+// 128-B rows, 1024 B apart (stride byte offset); 64-element chunks of the MN dimension `chunk`
+// bytes apart (leading byte offset; 16 KB for a 128-row tile of the attention's V).
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(const void* tile, uint32_t chunk = 16384) {
   const uint64_t addr = smem_u32(tile);
   uint64_t d = (addr >> 4) & 0x3FFFull;
-  d |= (uint64_t)(16384 >> 4) << 16;
+  d |= (uint64_t)(chunk >> 4) << 16;
   d |= (uint64_t)(1024 >> 4) << 32;
   d |= 1ull << 46;
   d |= 2ull << 61;

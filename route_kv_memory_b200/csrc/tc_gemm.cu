@@ -281,9 +281,14 @@ constexpr int PAIR_STAGE_BYTES = 2 * HALF_ROWS * BK * 2;  // A rows + B rows of 
 constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * PAIR_STAGE_BYTES + 1024 + 256;
 constexpr uint32_t PAIR_IDESC = idesc_bf16_f32(PAIR_BM, BN);
 
+// AMN / BMN: the operand is stored MN-major ([K][M] or [K][N], row stride lda / ldb): its 128 rows
+// of a stage come as two 64 x 64 boxes (64 MN elements by 64 K rows, 8 KB apart).
+template <bool AMN, bool BMN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                     int K, Epilogue ep, int* status) {
+  constexpr uint32_t IDESC2 = PAIR_IDESC | (AMN ? 1u << 15 : 0u) | (BMN ? 1u << 16 : 0u);
+  constexpr int CHUNK = 64 * BK * 2;  // one 64 x 64 MN-major box
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(smem + PAIR_STAGES * PAIR_STAGE_BYTES);  // rank 0's copy is used
@@ -333,8 +338,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!mbar_wait(&empty[s], ph ^ 1, abort, status)) goto producer_done;
           uint8_t* st = smem + s * PAIR_STAGE_BYTES;
           if (rank == 0) mbar_expect_tx(&full[s], 2 * PAIR_STAGE_BYTES);
-          tma_load_2d_pair(st, &tmA, &full[s], k * BK, ma);
-          tma_load_2d_pair(st + HALF_ROWS * BK * 2, &tmB, &full[s], k * BK, nb);
+          if constexpr (AMN) {
+            tma_load_2d_pair(st, &tmA, &full[s], ma, k * BK);
+            tma_load_2d_pair(st + CHUNK, &tmA, &full[s], ma + 64, k * BK);
+          } else {
+            tma_load_2d_pair(st, &tmA, &full[s], k * BK, ma);
+          }
+          if constexpr (BMN) {
+            tma_load_2d_pair(st + HALF_ROWS * BK * 2, &tmB, &full[s], nb, k * BK);
+            tma_load_2d_pair(st + HALF_ROWS * BK * 2 + CHUNK, &tmB, &full[s], nb + 64, k * BK);
+          } else {
+            tma_load_2d_pair(st + HALF_ROWS * BK * 2, &tmB, &full[s], k * BK, nb);
+          }
         }
       }
     producer_done:
@@ -367,12 +382,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           tc_fence_after();
           const uint8_t* st = smem + s * PAIR_STAGE_BYTES;
-          const uint64_t a_desc = sdesc_kmajor_sw128(st);
-          const uint64_t b_desc = sdesc_kmajor_sw128(st + HALF_ROWS * BK * 2);
+          const uint64_t a_desc = AMN ? sdesc_mnmajor_sw128(st, CHUNK) : sdesc_kmajor_sw128(st);
+          const uint64_t b_desc = BMN ? sdesc_mnmajor_sw128(st + HALF_ROWS * BK * 2, CHUNK)
+                                      : sdesc_kmajor_sw128(st + HALF_ROWS * BK * 2);
+          // K-step kk: 32 bytes along a K-major row, or 16 K rows (2 KB) of an MN-major box
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            umma2_bf16_ss(d_tmem, a_desc + (uint64_t)(kk * 2), b_desc + (uint64_t)(kk * 2), PAIR_IDESC,
-                          (k | kk) != 0);
+            umma2_bf16_ss(d_tmem, a_desc + (uint64_t)(AMN ? kk * (2048 >> 4) : kk * 2),
+                          b_desc + (uint64_t)(BMN ? kk * (2048 >> 4) : kk * 2), IDESC2, (k | kk) != 0);
           umma2_commit_mc(&empty[s], 0x3);
         }
         if (!ok) break;
@@ -454,41 +471,52 @@ cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, int d0, int d1
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t gemm_tn_bf16_tc(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
-                            int* status, cudaStream_t s) {
+template <bool AMN, bool BMN>
+static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const Epilogue& ep,
+                               int* status, int sms, cudaStream_t s) {
+  cudaError_t e = set_max_smem(tcg::gemm_tc2_kernel<AMN, BMN>, tcg::PAIR_SMEM_BYTES, s);
+  if (e != cudaSuccess) return e;
+  const int ntiles = ((M + tcg::PAIR_BM - 1) / tcg::PAIR_BM) * ((N + tcg::BN - 1) / tcg::BN);
+  int pairs = sms / 2;
+  if (ntiles < pairs) pairs = ntiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(tcg::NTHREADS);
+  cfg.dynamicSmemBytes = tcg::PAIR_SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tcg::gemm_tc2_kernel<AMN, BMN>, ta, tb, M, N, K, ep, status);
+}
+
+cudaError_t gemm_bf16_tc(const void* A, int lda, int a_mn, const void* B, int ldb, int b_mn, int M, int N, int K,
+                         const Epilogue& ep, int* status, cudaStream_t s) {
   if (M <= 0 || N <= 0) return cudaSuccess;
-  if ((K % 8) || (lda % 8) || (ldb % 8) || ((uintptr_t)A & 15) || ((uintptr_t)B & 15)) return cudaErrorInvalidValue;
+  if ((lda % 8) || (ldb % 8) || ((uintptr_t)A & 15) || ((uintptr_t)B & 15) || (!a_mn && K % 8) ||
+      (a_mn && M % 8) || (!b_mn && K % 8) || (b_mn && N % 8))
+    return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
-  cudaError_t e = make_tmap_bf16(&ta, A, M, K, lda, tcg::BM);
+  // K-major: [M][K] rows, boxes of 64 K by 128 (A) / 128 (B, per CTA of a pair) rows;
+  // MN-major: [K][M] rows, boxes of 64 x 64
+  cudaError_t e = a_mn ? make_tmap_bf16(&ta, A, K, M, lda, 64) : make_tmap_bf16(&ta, A, M, K, lda, tcg::BM);
+  if (e != cudaSuccess) return e;
+  e = b_mn ? make_tmap_bf16(&tb, B, K, N, ldb, 64) : make_tmap_bf16(&tb, B, N, K, ldb, tcg::HALF_ROWS);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // CTA pairs: 256 x 256 tiles, two SMs per tile, grid of whole pairs
-  {
-    e = make_tmap_bf16(&tb, B, N, K, ldb, tcg::HALF_ROWS);
-    if (e != cudaSuccess) return e;
-    e = set_max_smem(tcg::gemm_tc2_kernel, tcg::PAIR_SMEM_BYTES, s);
-    if (e != cudaSuccess) return e;
-    const int ntiles = ((M + tcg::PAIR_BM - 1) / tcg::PAIR_BM) * ((N + tcg::BN - 1) / tcg::BN);
-    int pairs = sms / 2;
-    if (ntiles < pairs) pairs = ntiles;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(tcg::NTHREADS);
-    cfg.dynamicSmemBytes = tcg::PAIR_SMEM_BYTES;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, tcg::gemm_tc2_kernel, ta, tb, M, N, K, ep, status);
-    if (e == cudaSuccess) return cudaSuccess;
-    cudaGetLastError();  // a device or partition that cannot place 2-CTA clusters: one CTA per tile
-  }
+  if (a_mn && b_mn) e = launch_pair<true, true>(ta, tb, M, N, K, ep, status, sms, s);
+  else if (a_mn) e = launch_pair<true, false>(ta, tb, M, N, K, ep, status, sms, s);
+  else if (b_mn) e = launch_pair<false, true>(ta, tb, M, N, K, ep, status, sms, s);
+  else e = launch_pair<false, false>(ta, tb, M, N, K, ep, status, sms, s);
+  if (e == cudaSuccess || a_mn || b_mn) return e;  // the single-CTA fallback takes K-major operands only
+  cudaGetLastError();  // a device or partition that cannot place 2-CTA clusters: one CTA per tile
   e = make_tmap_bf16(&tb, B, N, K, ldb, tcg::BN);
   if (e != cudaSuccess) return e;
   e = set_max_smem(tcg::gemm_tc_kernel, tcg::SMEM_BYTES, s);
@@ -496,6 +524,11 @@ cudaError_t gemm_tn_bf16_tc(const void* A, int lda, const void* B, int ldb, int 
   const int ntiles1 = ((M + tcg::BM - 1) / tcg::BM) * ((N + tcg::BN - 1) / tcg::BN);
   tcg::gemm_tc_kernel<<<ntiles1 < sms ? ntiles1 : sms, tcg::NTHREADS, tcg::SMEM_BYTES, s>>>(ta, tb, M, N, K, ep, status);
   return cudaGetLastError();
+}
+
+cudaError_t gemm_tn_bf16_tc(const void* A, int lda, const void* B, int ldb, int M, int N, int K, const Epilogue& ep,
+                            int* status, cudaStream_t s) {
+  return gemm_bf16_tc(A, lda, 0, B, ldb, 0, M, N, K, ep, status, s);
 }
 
 }  // namespace mka
