@@ -6,14 +6,15 @@
 // dK and dV summed over the G = Hq / Hkv query heads of a KV group.  Two kernels, no atomics:
 //
 //   attn_bwd_dq_kernel    per (sequence, query head, 128-row query tile), streaming the key
-//                         tiles j <= its own: S = Q K_j^T and dP = dO V_j^T into TMEM, four warps
-//                         turn them into scale * dS (bf16, written over S), then dQ += dS K_j
-//                         with dS read from TMEM and K_j as an MN-major operand.
+//                         tiles j <= its own (K in a 3-stage ring, V in a 2-stage one):
+//                         S = Q K_j^T and dP = dO V_j^T into TMEM, the compute warps turn them
+//                         into scale * dS (bf16, packed over dP), then dQ += dS K_j with dS read
+//                         from TMEM and K_j as an MN-major operand.
 //   attn_bwd_dkdv_kernel  per (sequence, KV group, 128-key tile), K and V staying in shared
 //                         memory while the query tiles t >= its own of all G heads stream through
-//                         a 2-stage ring (Q, dO and their lse and D rows): S^T = K Q^T and
-//                         dP^T = V dO^T into TMEM, four warps write P^T and scale * dS^T (bf16)
-//                         over them, then dV += P^T dO and dK += dS^T Q accumulate in TMEM.
+//                         two 2-stage rings (Q with its lse and D rows; dO): S^T = K Q^T and
+//                         dP^T = V dO^T into TMEM, the compute warps write P^T and scale * dS^T
+//                         (bf16) over dP^T, then dK += dS^T Q and dV += P^T dO accumulate in TMEM.
 // Warp 0 loads (TMA), warp 1 issues the MMAs, warps 2-9 compute: two warps per TMEM lane quadrant,
 // each taking 64 of a row's 128 columns; a warp packs its bf16 results into the first 32 columns of
 // its own 64-column range (so neither half overwrites what the other still reads), and the MMAs
@@ -45,9 +46,10 @@ struct Cfg {
   static constexpr int TILE = BT * DH * 2;       // one 128-row bf16 tile
   static constexpr int HALF = BT * 64 * 2;       // one 128-row x 64-column swizzled box
   static constexpr int VEC = BT * 4;             // 128 floats (lse or D of a query tile)
-  static constexpr int STAGE = 2 * TILE + 1024;  // dK/dV ring stage: Q, dO, lse, D (1024-aligned)
-  static constexpr int SMEM_DQ = 2 * TILE + 2 * 2 * TILE + 1024 + 256;
-  static constexpr int SMEM_DKDV = 2 * TILE + 2 * STAGE + 1024 + 256;
+  static constexpr int QSTAGE = TILE + 1024;     // dK/dV Q ring stage: Q, lse, D (1024-aligned)
+  static constexpr int KST = 3, VST = 2;           // dQ kernel: K ring stages, V ring stages
+  static constexpr int SMEM_DQ = (2 + KST + VST) * TILE + 1024 + 256;
+  static constexpr int SMEM_DKDV = 2 * TILE + 2 * QSTAGE + 2 * TILE + 1024 + 256;
 };
 
 __device__ __forceinline__ int snake(int r, int grid, int cta, int nwork) {
@@ -79,28 +81,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
   uint8_t* sdO = smem + C::TILE;
-  uint8_t* sKV = smem + 2 * C::TILE;  // stage st: K at st * 2 TILE, V at + TILE
-  uint64_t* bars = (uint64_t*)(smem + 6 * C::TILE);
+  // K and V rings of their own: K_j is read by S(j) and dQ(j), V_j only by dP(j), which ends a
+  // whole step earlier, so K takes one stage more
+  uint8_t* sK = smem + 2 * C::TILE;                // stage st at st * TILE
+  uint8_t* sV = smem + (2 + C::KST) * C::TILE;
+  uint64_t* bars = (uint64_t*)(smem + (2 + C::KST + C::VST) * C::TILE);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;   // [2]
-  uint64_t* kv_empty = bars + 4;  // [2]
-  uint64_t* s_full = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* dq_full = bars + 8;
-  uint64_t* dq_empty = bars + 9;
-  uint64_t* drain = bars + 10;
-  uint64_t* s_free = bars + 11;   // the compute warps hold S in registers: its columns are free
-  uint64_t* dp_full = bars + 12;  // dP has landed
-  uint32_t* tmem_slot = (uint32_t*)(bars + 13);
+  uint64_t* k_full = bars + 2;                 // [KST]
+  uint64_t* k_empty = k_full + C::KST;         // [KST]
+  uint64_t* v_full = k_empty + C::KST;         // [VST]
+  uint64_t* v_empty = v_full + C::VST;         // [VST]
+  uint64_t* s_full = v_empty + C::VST;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* dq_full = s_full + 2;
+  uint64_t* dq_empty = s_full + 3;
+  uint64_t* drain = s_full + 4;
+  uint64_t* s_free = s_full + 5;   // the compute warps hold S in registers: its columns are free
+  uint64_t* dp_full = s_full + 6;  // dP has landed
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 7);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+    for (int i = 0; i < C::KST; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < C::VST; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, NCOMPUTE);
@@ -151,17 +162,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_2d(sdO + hb * C::HALF, &tmdO, q_full, h * DH + hb * 64, b * a.S + qt * BT);
         }
         for (int j = 0; j <= qt; ++j, ++kvit) {
-          const int st = kvit & 1;
-          if (!mbar_wait(&kv_empty[st], ((kvit >> 1) & 1) ^ 1, abort, status)) {
+          const int ks = kvit % C::KST, vs = kvit % C::VST;
+          if (!mbar_wait(&k_empty[ks], ((kvit / C::KST) & 1) ^ 1, abort, status)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(&kv_full[st], 2 * C::TILE);
-          uint8_t* dst = sKV + st * 2 * C::TILE;
-          for (int hb = 0; hb < C::NH; ++hb) {
-            tma_load_2d(dst + hb * C::HALF, &tmK, &kv_full[st], (h / G) * DH + hb * 64, b * a.S + j * BT);
-            tma_load_2d(dst + C::TILE + hb * C::HALF, &tmV, &kv_full[st], (h / G) * DH + hb * 64, b * a.S + j * BT);
+          mbar_expect_tx(&k_full[ks], C::TILE);
+          for (int hb = 0; hb < C::NH; ++hb)
+            tma_load_2d(sK + ks * C::TILE + hb * C::HALF, &tmK, &k_full[ks], (h / G) * DH + hb * 64, b * a.S + j * BT);
+          if (!mbar_wait(&v_empty[vs], ((kvit / C::VST) & 1) ^ 1, abort, status)) {
+            ok = false;
+            break;
           }
+          mbar_expect_tx(&v_full[vs], C::TILE);
+          for (int hb = 0; hb < C::NH; ++hb)
+            tma_load_2d(sV + vs * C::TILE + hb * C::HALF, &tmV, &v_full[vs], (h / G) * DH + hb * 64, b * a.S + j * BT);
         }
       }
       if (*abort) {
@@ -170,83 +185,86 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint64_t qd = sdesc_kmajor_sw128(sQ), dod = sdesc_kmajor_sw128(sdO);
-      int kvit = 0, pc = 0, sf = 0;
-      bool ok = true, first = true;
-      // S = Q K^T for the key tile in ring slot `st`
-      auto issue_s = [&](int st) {
-        const uint64_t kd = sdesc_kmajor_sw128(sKV + st * 2 * C::TILE);
+  } else if (warp == 1) {  // the whole warp runs the MMA role; one elected lane issues
+    const uint64_t qd = sdesc_kmajor_sw128(sQ), dod = sdesc_kmajor_sw128(sdO);
+    int kvit = 0, pc = 0, sf = 0;
+    bool ok = true, first = true;
+    // S = Q K^T for the key tile in K ring slot `st`
+    auto issue_s = [&](int st) {
+      const uint64_t kd = sdesc_kmajor_sw128(sK + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk)
-          umma_bf16_ss(tbase + S_COL, qd + kstep(kk, C::HALF), kd + kstep(kk, C::HALF), IDESC_S, kk != 0);
-        umma_commit(s_full);
-      };
-      // dP = dO V^T
-      auto issue_dp = [&](int st) {
-        const uint64_t vd = sdesc_kmajor_sw128(sKV + st * 2 * C::TILE + C::TILE);
+      for (int kk = 0; kk < DH / 16; ++kk)
+        umma_bf16_ss_w(tbase + S_COL, qd + kstep(kk, C::HALF), kd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+      umma_commit_w(s_full);
+    };
+    // dP = dO V^T, V in V ring slot `st` (freed when dP lands)
+    auto issue_dp = [&](int st) {
+      const uint64_t vd = sdesc_kmajor_sw128(sV + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk)
-          umma_bf16_ss(tbase + P_COL, dod + kstep(kk, C::HALF), vd + kstep(kk, C::HALF), IDESC_S, kk != 0);
-        umma_commit(dp_full);
-      };
-      // dQ += scale*dS K_j, dS packed over the dP columns
-      auto issue_dq = [&](int st, bool acc) {
-        const uint64_t kd = sdesc_mnmajor_sw128(sKV + st * 2 * C::TILE);
+      for (int kk = 0; kk < DH / 16; ++kk)
+        umma_bf16_ss_w(tbase + P_COL, dod + kstep(kk, C::HALF), vd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+      umma_commit_w(dp_full);
+      umma_commit_w(&v_empty[st]);
+    };
+    // dQ += scale*dS K_j, dS packed over the dP columns
+    auto issue_dq = [&](int st, bool acc) {
+      const uint64_t kd = sdesc_mnmajor_sw128(sK + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_ts(tbase + Q_COL, tbase + P_COL + packed_col(kk), kd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
-                       (acc || kk) ? 1u : 0u);
-      };
-      // S(j+1) goes in as soon as the compute warps hold S(j) in registers, so their exponentials
-      // of tile j+1 run under dQ(j) and dP(j+1); dP(j+1) follows dQ(j), which reads dS(j) over dP.
-      for (int rr = 0; ok; ++rr) {
-        const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
-        if (w < 0) break;
-        int b, h, qt;
-        item(w, b, h, qt);
-        const int n = qt + 1;
-        if (!mbar_wait(q_full, rr & 1, abort, status)) break;
-        if (!mbar_wait(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
-        if (!first) {
-          if (!mbar_wait(s_free, sf & 1, abort, status)) break;
-          ++sf;
-        }
-        first = false;
-        tc_fence_after();
-        issue_s(kvit & 1);
-        issue_dp(kvit & 1);
-        if (n == 1) umma_commit(q_empty);
-        for (int j = 0; j < n; ++j) {
-          const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
-          if (j + 1 < n) {
-            if (!mbar_wait(&kv_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
-            if (!mbar_wait(s_free, sf & 1, abort, status)) { ok = false; break; }
-            ++sf;
-            tc_fence_after();
-            issue_s(nst);
-          }
-          if (!mbar_wait(p_full, pc & 1, abort, status)) { ok = false; break; }
-          ++pc;
-          if (j == 0 && !mbar_wait(dq_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
-          tc_fence_after();
-          issue_dq(st, j > 0);
-          umma_commit(&kv_empty[st]);
-          if (j + 1 < n) {
-            issue_dp(nst);
-            if (j + 2 == n) umma_commit(q_empty);  // Q and dO's last use
-          }
-        }
-        if (!ok) break;
-        umma_commit(dq_full);
-        kvit += n;
+      for (int kk = 0; kk < BT / 16; ++kk)
+        umma_bf16_ts_w(tbase + Q_COL, tbase + P_COL + packed_col(kk), kd + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+                     (acc || kk) ? 1u : 0u);
+    };
+    // S(j+1) goes in as soon as the compute warps hold S(j) in registers, so their exponentials
+    // of tile j+1 run under dQ(j) and dP(j+1); dP(j+1) follows dQ(j), which reads dS(j) over dP.
+    for (int rr = 0; ok; ++rr) {
+      const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
+      if (w < 0) break;
+      int b, h, qt;
+      item(w, b, h, qt);
+      const int n = qt + 1;
+      if (!mbar_wait_warp(q_full, rr & 1, abort, status)) break;
+      if (!mbar_wait_warp(&k_full[kvit % C::KST], (kvit / C::KST) & 1, abort, status)) break;
+      if (!first) {
+        if (!mbar_wait_warp(s_free, sf & 1, abort, status)) break;
+        ++sf;
       }
-      if (*abort) {
-        umma_commit(drain);
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
+      first = false;
+      tc_fence_after();
+      issue_s(kvit % C::KST);
+      if (!mbar_wait_warp(&v_full[kvit % C::VST], (kvit / C::VST) & 1, abort, status)) break;
+      tc_fence_after();
+      issue_dp(kvit % C::VST);
+      if (n == 1) umma_commit_w(q_empty);
+      for (int j = 0; j < n; ++j) {
+        const int cur = kvit + j, nxt = cur + 1;
+        if (j + 1 < n) {
+          if (!mbar_wait_warp(&k_full[nxt % C::KST], (nxt / C::KST) & 1, abort, status)) { ok = false; break; }
+          if (!mbar_wait_warp(s_free, sf & 1, abort, status)) { ok = false; break; }
+          ++sf;
+          tc_fence_after();
+          issue_s(nxt % C::KST);
         }
+        if (!mbar_wait_warp(p_full, pc & 1, abort, status)) { ok = false; break; }
+        ++pc;
+        if (j == 0 && !mbar_wait_warp(dq_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        issue_dq(cur % C::KST, j > 0);
+        umma_commit_w(&k_empty[cur % C::KST]);
+        if (j + 1 < n) {
+          if (!mbar_wait_warp(&v_full[nxt % C::VST], (nxt / C::VST) & 1, abort, status)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(nxt % C::VST);
+          if (j + 2 == n) umma_commit_w(q_empty);  // Q and dO's last use
+        }
+      }
+      if (!ok) break;
+      umma_commit_w(dq_full);
+      kvit += n;
+    }
+    if (__any_sync(0xffffffffu, *abort)) {
+      umma_commit_w(drain);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
   } else {
@@ -370,28 +388,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sK = smem;
   uint8_t* sV = smem + C::TILE;
-  uint8_t* sQD = smem + 2 * C::TILE;  // stage st at st * STAGE: Q, dO, lse[128], D[128]
-  uint64_t* bars = (uint64_t*)(smem + 2 * C::TILE + 2 * C::STAGE);
+  // Q (with its lse and D rows) and dO in rings of their own: dK(s), the last reader of Q(s), is
+  // issued before dV(s), so Q(s + 2), all that S^T(s + 2) needs, loads while dV(s) runs
+  uint8_t* sQ = smem + 2 * C::TILE;                  // stage st at st * QSTAGE: Q, lse[128], D[128]
+  uint8_t* sdO = sQ + 2 * C::QSTAGE;                 // stage st at st * TILE
+  uint64_t* bars = (uint64_t*)(sdO + 2 * C::TILE);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* qd_full = bars + 2;   // [2]
-  uint64_t* qd_empty = bars + 4;  // [2]
-  uint64_t* s_full = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* acc_full = bars + 8;
-  uint64_t* acc_empty = bars + 9;
-  uint64_t* drain = bars + 10;
-  uint64_t* s_free = bars + 11;   // the compute warps hold S^T in registers: its columns are free
-  uint64_t* dp_full = bars + 12;  // dP^T has landed
-  uint32_t* tmem_slot = (uint32_t*)(bars + 13);
+  uint64_t* q_full = bars + 2;    // [2]
+  uint64_t* q_empty = bars + 4;   // [2]
+  uint64_t* do_full = bars + 6;   // [2]
+  uint64_t* do_empty = bars + 8;  // [2]
+  uint64_t* s_full = bars + 10;
+  uint64_t* p_full = bars + 11;
+  uint64_t* acc_full = bars + 12;
+  uint64_t* acc_empty = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint64_t* s_free = bars + 15;   // the compute warps hold S^T in registers: its columns are free
+  uint64_t* dp_full = bars + 16;  // dP^T has landed
+  uint32_t* tmem_slot = (uint32_t*)(bars + 17);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&qd_full[i], 1);
-      mbar_init(&qd_empty[i], 1);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&do_full[i], 1);
+      mbar_init(&do_empty[i], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, NCOMPUTE);
@@ -444,20 +469,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         const int nq = nqt - kt;
         for (int s = 0; s < G * nq; ++s, ++qdit) {
-          const int h = g * G + s / nq, qt = kt + s % nq, st = qdit & 1;
-          if (!mbar_wait(&qd_empty[st], ((qdit >> 1) & 1) ^ 1, abort, status)) {
+          const int h = g * G + s / nq, qt = kt + s % nq, st = qdit & 1, ph = ((qdit >> 1) & 1) ^ 1;
+          if (!mbar_wait(&q_empty[st], ph, abort, status)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(&qd_full[st], 2 * C::TILE + 2 * C::VEC);
-          uint8_t* dst = sQD + st * C::STAGE;
-          for (int hb = 0; hb < C::NH; ++hb) {
-            tma_load_2d(dst + hb * C::HALF, &tmQ, &qd_full[st], h * DH + hb * 64, b * a.S + qt * BT);
-            tma_load_2d(dst + C::TILE + hb * C::HALF, &tmdO, &qd_full[st], h * DH + hb * 64, b * a.S + qt * BT);
-          }
+          mbar_expect_tx(&q_full[st], C::TILE + 2 * C::VEC);
+          uint8_t* dst = sQ + st * C::QSTAGE;
+          for (int hb = 0; hb < C::NH; ++hb)
+            tma_load_2d(dst + hb * C::HALF, &tmQ, &q_full[st], h * DH + hb * 64, b * a.S + qt * BT);
           const size_t li = ((size_t)b * a.Hq + h) * a.lse_ld + (size_t)qt * BT;
-          bulk_load(dst + 2 * C::TILE, a.lse + li, C::VEC, &qd_full[st]);
-          bulk_load(dst + 2 * C::TILE + C::VEC, a.dsum + li, C::VEC, &qd_full[st]);
+          bulk_load(dst + C::TILE, a.lse + li, C::VEC, &q_full[st]);
+          bulk_load(dst + C::TILE + C::VEC, a.dsum + li, C::VEC, &q_full[st]);
+          if (!mbar_wait(&do_empty[st], ph, abort, status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&do_full[st], C::TILE);
+          for (int hb = 0; hb < C::NH; ++hb)
+            tma_load_2d(sdO + st * C::TILE + hb * C::HALF, &tmdO, &do_full[st], h * DH + hb * 64, b * a.S + qt * BT);
         }
       }
       if (*abort) {
@@ -466,86 +496,96 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint64_t kd = sdesc_kmajor_sw128(sK), vd = sdesc_kmajor_sw128(sV);
-      int qdit = 0, pc = 0, sf = 0;
-      bool ok = true, first = true;
-      // S^T = K Q^T for the query stage `st`
-      auto issue_s = [&](int st) {
-        const uint64_t qd = sdesc_kmajor_sw128(sQD + st * C::STAGE);
+  } else if (warp == 1) {  // the whole warp runs the MMA role; one elected lane issues
+    const uint64_t kd = sdesc_kmajor_sw128(sK), vd = sdesc_kmajor_sw128(sV);
+    int qdit = 0, pc = 0, sf = 0;
+    bool ok = true, first = true;
+    // S^T = K Q^T for the query stage `st`
+    auto issue_s = [&](int st) {
+      const uint64_t qd = sdesc_kmajor_sw128(sQ + st * C::QSTAGE);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk)
-          umma_bf16_ss(tbase + S_COL, kd + kstep(kk, C::HALF), qd + kstep(kk, C::HALF), IDESC_S, kk != 0);
-        umma_commit(s_full);
-      };
-      // dP^T = V dO^T
-      auto issue_dp = [&](int st) {
-        const uint64_t dod = sdesc_kmajor_sw128(sQD + st * C::STAGE + C::TILE);
+      for (int kk = 0; kk < DH / 16; ++kk)
+        umma_bf16_ss_w(tbase + S_COL, kd + kstep(kk, C::HALF), qd + kstep(kk, C::HALF), IDESC_S, kk != 0);
+      umma_commit_w(s_full);
+    };
+    // dP^T = V dO^T
+    auto issue_dp = [&](int st) {
+      const uint64_t dod = sdesc_kmajor_sw128(sdO + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk)
-          umma_bf16_ss(tbase + P_COL, vd + kstep(kk, C::HALF), dod + kstep(kk, C::HALF), IDESC_S, kk != 0);
-        umma_commit(dp_full);
-      };
-      // dV += P^T dO and dK += scale*dS^T Q; the compute warps pack P^T and dS^T over the dP^T
-      // columns: K-step kk (16 queries) of P^T at 64 (kk / 4) + 32 ((kk / 2) % 2) + 8 (kk % 2), of dS^T 16 further
-      auto issue_acc = [&](int st, bool acc) {
-        const uint64_t dq = sdesc_mnmajor_sw128(sQD + st * C::STAGE);
-        const uint64_t dd = sdesc_mnmajor_sw128(sQD + st * C::STAGE + C::TILE);
+      for (int kk = 0; kk < DH / 16; ++kk)
+        umma_bf16_ss_w(tbase + P_COL, vd + kstep(kk, C::HALF), dod + kstep(kk, C::HALF), IDESC_S, kk != 0);
+      umma_commit_w(dp_full);
+    };
+    // dK += scale*dS^T Q, then dV += P^T dO, each freeing its ring slot; the compute warps pack
+    // P^T and dS^T over the dP^T columns: K-step kk (16 queries) of P^T at
+    // 64 (kk / 4) + 32 ((kk / 2) % 2) + 8 (kk % 2), of dS^T 16 further
+    auto issue_acc = [&](int st, bool acc) {
+      const uint64_t dq = sdesc_mnmajor_sw128(sQ + st * C::QSTAGE);
+      const uint64_t dd = sdesc_mnmajor_sw128(sdO + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk) {
-          const uint32_t pcol = P_COL + 64 * (kk >> 2) + 32 * ((kk >> 1) & 1) + 8 * (kk & 1);
-          umma_bf16_ts(tbase + V_COL, tbase + pcol, dd + (uint64_t)(kk * (2048 >> 4)), IDESC_D, (acc || kk) ? 1u : 0u);
-          umma_bf16_ts(tbase + K_COL, tbase + pcol + 16, dq + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
-                       (acc || kk) ? 1u : 0u);
-        }
-      };
-      // S^T(s+1) goes in as soon as the compute warps hold S^T(s) in registers, so their
-      // exponentials of step s+1 run under dV / dK(s) and dP^T(s+1); dP^T(s+1) follows dV / dK(s),
-      // which read P^T(s) and dS^T(s) over the dP^T columns.
-      for (int rr = 0; ok; ++rr) {
-        const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
-        if (w < 0) break;
-        int b, g, kt;
-        item(w, b, g, kt);
-        const int n = G * (nqt - kt);
-        if (!mbar_wait(kv_full, rr & 1, abort, status)) break;
-        if (!mbar_wait(&qd_full[qdit & 1], (qdit >> 1) & 1, abort, status)) break;
-        if (!first) {
-          if (!mbar_wait(s_free, sf & 1, abort, status)) break;
-          ++sf;
-        }
-        first = false;
-        tc_fence_after();
-        issue_s(qdit & 1);
-        issue_dp(qdit & 1);
-        for (int s = 0; s < n; ++s) {
-          const int cur = qdit + s, st = cur & 1, nst = (cur + 1) & 1;
-          if (s + 1 < n) {
-            if (!mbar_wait(&qd_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
-            if (!mbar_wait(s_free, sf & 1, abort, status)) { ok = false; break; }
-            ++sf;
-            tc_fence_after();
-            issue_s(nst);
-          }
-          if (!mbar_wait(p_full, pc & 1, abort, status)) { ok = false; break; }
-          ++pc;
-          if (s == 0 && !mbar_wait(acc_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
-          tc_fence_after();
-          issue_acc(st, s > 0);
-          umma_commit(&qd_empty[st]);
-          if (s + 1 < n) issue_dp(nst);
-        }
-        if (!ok) break;
-        umma_commit(kv_empty);
-        umma_commit(acc_full);
-        qdit += n;
+      for (int kk = 0; kk < BT / 16; ++kk) {
+        const uint32_t pcol = P_COL + 64 * (kk >> 2) + 32 * ((kk >> 1) & 1) + 8 * (kk & 1);
+        umma_bf16_ts_w(tbase + K_COL, tbase + pcol + 16, dq + (uint64_t)(kk * (2048 >> 4)), IDESC_D,
+                     (acc || kk) ? 1u : 0u);
       }
-      if (*abort) {
-        umma_commit(drain);
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
+      umma_commit_w(&q_empty[st]);
+#pragma unroll
+      for (int kk = 0; kk < BT / 16; ++kk) {
+        const uint32_t pcol = P_COL + 64 * (kk >> 2) + 32 * ((kk >> 1) & 1) + 8 * (kk & 1);
+        umma_bf16_ts_w(tbase + V_COL, tbase + pcol, dd + (uint64_t)(kk * (2048 >> 4)), IDESC_D, (acc || kk) ? 1u : 0u);
+      }
+      umma_commit_w(&do_empty[st]);
+    };
+    // S^T(s+1) goes in as soon as the compute warps hold S^T(s) in registers, so their
+    // exponentials of step s+1 run under dV / dK(s) and dP^T(s+1); dP^T(s+1) follows dV / dK(s),
+    // which read P^T(s) and dS^T(s) over the dP^T columns.
+    for (int rr = 0; ok; ++rr) {
+      const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
+      if (w < 0) break;
+      int b, g, kt;
+      item(w, b, g, kt);
+      const int n = G * (nqt - kt);
+      if (!mbar_wait_warp(kv_full, rr & 1, abort, status)) break;
+      if (!mbar_wait_warp(&q_full[qdit & 1], (qdit >> 1) & 1, abort, status)) break;
+      if (!first) {
+        if (!mbar_wait_warp(s_free, sf & 1, abort, status)) break;
+        ++sf;
+      }
+      first = false;
+      tc_fence_after();
+      issue_s(qdit & 1);
+      if (!mbar_wait_warp(&do_full[qdit & 1], (qdit >> 1) & 1, abort, status)) break;
+      tc_fence_after();
+      issue_dp(qdit & 1);
+      for (int s = 0; s < n; ++s) {
+        const int cur = qdit + s, st = cur & 1, nst = (cur + 1) & 1, nph = ((cur + 1) >> 1) & 1;
+        if (s + 1 < n) {
+          if (!mbar_wait_warp(&q_full[nst], nph, abort, status)) { ok = false; break; }
+          if (!mbar_wait_warp(s_free, sf & 1, abort, status)) { ok = false; break; }
+          ++sf;
+          tc_fence_after();
+          issue_s(nst);
         }
+        if (!mbar_wait_warp(p_full, pc & 1, abort, status)) { ok = false; break; }
+        ++pc;
+        if (s == 0 && !mbar_wait_warp(acc_empty, (rr & 1) ^ 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        issue_acc(st, s > 0);
+        if (s + 1 < n) {
+          if (!mbar_wait_warp(&do_full[nst], nph, abort, status)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(nst);
+        }
+      }
+      if (!ok) break;
+      umma_commit_w(kv_empty);
+      umma_commit_w(acc_full);
+      qdit += n;
+    }
+    if (__any_sync(0xffffffffu, *abort)) {
+      umma_commit_w(drain);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
   } else {
@@ -564,12 +604,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       bool ok = true;
       for (int s = 0; s < n; ++s, ++sit) {
         const int qt = kt + s % nq, st = sit & 1;
-        // the stage's lse and D rows: landed with its Q and dO (the stage is not refilled before
-        // this step's dV / dK MMAs, which wait for this warp)
-        if (!mbar_wait(&qd_full[st], (sit >> 1) & 1, abort, status)) { ok = false; break; }
+        // the stage's lse and D rows: landed with its Q (the stage is not refilled before this
+        // step's dK MMAs, which wait for this warp)
+        if (!mbar_wait(&q_full[st], (sit >> 1) & 1, abort, status)) { ok = false; break; }
         if (!mbar_wait(s_full, sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
-        const float* lse2 = (const float*)(sQD + st * C::STAGE + 2 * C::TILE);
+        const float* lse2 = (const float*)(sQ + st * C::QSTAGE + C::TILE);
         const float* dsum = lse2 + BT;
         // query column c is used iff it is a real row at or after this key: q0 + c < S, q0 + c >= key
         const int q0 = qt * BT, cmax = a.S - q0, cmin = key - q0;
