@@ -340,105 +340,104 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int kvit = 0, pc[2] = {0, 0};
-      bool ok = true;
-      const uint64_t qd0 = sdesc_kmajor_sw128(sQ), qd1 = sdesc_kmajor_sw128(sQ + C::Q_BYTES);
-      auto issue_s = [&](int t, int st) {
-        const uint64_t kd = sdesc_kmajor_sw128(sKV + st * C::KV_BYTES);
+    // (the whole warp runs the role, converged; one elected lane issues)
+    int kvit = 0, pc[2] = {0, 0};
+    bool ok = true;
+    const uint64_t qd0 = sdesc_kmajor_sw128(sQ), qd1 = sdesc_kmajor_sw128(sQ + C::Q_BYTES);
+    auto issue_s = [&](int t, int st) {
+      const uint64_t kd = sdesc_kmajor_sw128(sKV + st * C::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint64_t off = (uint64_t)((kk >> 2) * (C::HALF >> 4) + (kk & 3) * 2);
-          umma_bf16_ss(tbase + S_COL(t), (t ? qd1 : qd0) + off, kd + off, IDESC_S, kk != 0);
-        }
-        umma_commit(&s_full[t]);
-      };
-      auto issue_pv = [&](int t, int st, int j) {
-        const uint64_t vd = sdesc_mnmajor_sw128(sKV + st * C::KV_BYTES + C::K_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)
-          umma_bf16_ts(tbase + O_COL(t), tbase + S_COL(t) + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
-                       (j | kk) != 0);
-        umma_commit(&pv_done[t]);
-      };
-      int nx0 = 0, nx1 = 0;  // tiles of the next item, looked up while this one runs
-      {
-        const int w0 = snake_item(0, gridDim.x, blockIdx.x, nwork);
-        if (w0 >= 0) item_tiles(w0, nx0, nx1);
+      for (int kk = 0; kk < DH / 16; ++kk) {
+        const uint64_t off = (uint64_t)((kk >> 2) * (C::HALF >> 4) + (kk & 3) * 2);
+        umma_bf16_ss_w(tbase + S_COL(t), (t ? qd1 : qd0) + off, kd + off, IDESC_S, kk != 0);
       }
-      for (int rr = 0; rr * (int)gridDim.x < nwork && ok; ++rr) {
-        const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
-        if (w < 0) break;
-        const int wi = rr;  // items this CTA has started before this one
-        const int n0 = nx0, n1 = nx1;  // n0 <= n1, n1 >= 1
-        if (!mbar_wait(&q_full[0], wi & 1, abort, status)) break;
-        if (n1 > 0 && !mbar_wait(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
-        tc_fence_after();
-        if (n0 > 0) issue_s(0, kvit & 1);
-        if (n0 <= 1) umma_commit(&q_empty[0]);  // Q_0's last use (or none)
-        // No key tile: the epilogue adds nothing from TMEM, but o_full still moves one phase per
-        // item, and only after the previous item's epilogue released O_t: without that wait two
-        // items in a row could commit two phases before the softmax warps wait for the first,
-        // which then reads as the wrong parity and never completes.
-        if (n0 == 0) {
-          if (!mbar_wait(&o_empty[0], (wi & 1) ^ 1, abort, status)) break;
-          umma_commit(&o_full[0]);
-        }
-        if (!mbar_wait(&q_full[1], wi & 1, abort, status)) break;
-        tc_fence_after();
-        if (n1 > 0) issue_s(1, kvit & 1);
-        if (n1 <= 1) umma_commit(&q_empty[1]);
-        if (n1 == 0) {
-          if (!mbar_wait(&o_empty[1], (wi & 1) ^ 1, abort, status)) break;
-          umma_commit(&o_full[1]);
-        }
-        {  // the next item's tile counts, looked up while these S MMAs and the softmax run
-          const int wn = snake_item(rr + 1, gridDim.x, blockIdx.x, nwork);
-          if (wn >= 0) item_tiles(wn, nx0, nx1);
-        }
-        for (int j = 0; j < n1; ++j) {
-          const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
-          bool next_ready = false;
-          if (j < n0) {
-            if (!mbar_wait(&p_full[0], pc[0] & 1, abort, status)) { ok = false; break; }
-            if (j == 0 && !mbar_wait(&o_empty[0], (wi & 1) ^ 1, abort, status)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(0, st, j);
-            ++pc[0];
-            if (j + 1 == n0) umma_commit(&o_full[0]);
-            if (j + 1 < n0) {
-              if (!mbar_wait(&kv_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
-              tc_fence_after();
-              next_ready = true;
-              issue_s(0, nst);
-              if (j + 2 == n0) umma_commit(&q_empty[0]);  // Q_0's last use
-            }
-          }
-          if (!mbar_wait(&p_full[1], pc[1] & 1, abort, status)) { ok = false; break; }
-          if (j == 0 && !mbar_wait(&o_empty[1], (wi & 1) ^ 1, abort, status)) { ok = false; break; }
+      umma_commit_w(&s_full[t]);
+    };
+    auto issue_pv = [&](int t, int st, int j) {
+      const uint64_t vd = sdesc_mnmajor_sw128(sKV + st * C::KV_BYTES + C::K_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < BKV / 16; ++kk)
+        umma_bf16_ts_w(tbase + O_COL(t), tbase + S_COL(t) + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
+                     (j | kk) != 0);
+      umma_commit_w(&pv_done[t]);
+    };
+    int nx0 = 0, nx1 = 0;  // tiles of the next item, looked up while this one runs
+    {
+      const int w0 = snake_item(0, gridDim.x, blockIdx.x, nwork);
+      if (w0 >= 0) item_tiles(w0, nx0, nx1);
+    }
+    for (int rr = 0; rr * (int)gridDim.x < nwork && ok; ++rr) {
+      const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
+      if (w < 0) break;
+      const int wi = rr;  // items this CTA has started before this one
+      const int n0 = nx0, n1 = nx1;  // n0 <= n1, n1 >= 1
+      if (!mbar_wait_warp(&q_full[0], wi & 1, abort, status)) break;
+      if (n1 > 0 && !mbar_wait_warp(&kv_full[kvit & 1], (kvit >> 1) & 1, abort, status)) break;
+      tc_fence_after();
+      if (n0 > 0) issue_s(0, kvit & 1);
+      if (n0 <= 1) umma_commit_w(&q_empty[0]);  // Q_0's last use (or none)
+      // No key tile: the epilogue adds nothing from TMEM, but o_full still moves one phase per
+      // item, and only after the previous item's epilogue released O_t: without that wait two
+      // items in a row could commit two phases before the softmax warps wait for the first,
+      // which then reads as the wrong parity and never completes.
+      if (n0 == 0) {
+        if (!mbar_wait_warp(&o_empty[0], (wi & 1) ^ 1, abort, status)) break;
+        umma_commit_w(&o_full[0]);
+      }
+      if (!mbar_wait_warp(&q_full[1], wi & 1, abort, status)) break;
+      tc_fence_after();
+      if (n1 > 0) issue_s(1, kvit & 1);
+      if (n1 <= 1) umma_commit_w(&q_empty[1]);
+      if (n1 == 0) {
+        if (!mbar_wait_warp(&o_empty[1], (wi & 1) ^ 1, abort, status)) break;
+        umma_commit_w(&o_full[1]);
+      }
+      {  // the next item's tile counts, looked up while these S MMAs and the softmax run
+        const int wn = snake_item(rr + 1, gridDim.x, blockIdx.x, nwork);
+        if (wn >= 0) item_tiles(wn, nx0, nx1);
+      }
+      for (int j = 0; j < n1; ++j) {
+        const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
+        bool next_ready = false;
+        if (j < n0) {
+          if (!mbar_wait_warp(&p_full[0], pc[0] & 1, abort, status)) { ok = false; break; }
+          if (j == 0 && !mbar_wait_warp(&o_empty[0], (wi & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(1, st, j);
-          ++pc[1];
-          umma_commit(&kv_empty[st]);
-          if (j + 1 < n1) {
-            if (!next_ready) {
-              if (!mbar_wait(&kv_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
-              tc_fence_after();
-            }
-            issue_s(1, nst);
-            if (j + 2 == n1) umma_commit(&q_empty[1]);  // Q_1's last use
-          } else {
-            umma_commit(&o_full[1]);
+          issue_pv(0, st, j);
+          ++pc[0];
+          if (j + 1 == n0) umma_commit_w(&o_full[0]);
+          if (j + 1 < n0) {
+            if (!mbar_wait_warp(&kv_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
+            tc_fence_after();
+            next_ready = true;
+            issue_s(0, nst);
+            if (j + 2 == n0) umma_commit_w(&q_empty[0]);  // Q_0's last use
           }
         }
-        if (!ok) break;
-        kvit += n1;
-      }
-      if (*abort) {
-        umma_commit(drain);
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
+        if (!mbar_wait_warp(&p_full[1], pc[1] & 1, abort, status)) { ok = false; break; }
+        if (j == 0 && !mbar_wait_warp(&o_empty[1], (wi & 1) ^ 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, st, j);
+        ++pc[1];
+        umma_commit_w(&kv_empty[st]);
+        if (j + 1 < n1) {
+          if (!next_ready) {
+            if (!mbar_wait_warp(&kv_full[nst], ((cur + 1) >> 1) & 1, abort, status)) { ok = false; break; }
+            tc_fence_after();
+          }
+          issue_s(1, nst);
+          if (j + 2 == n1) umma_commit_w(&q_empty[1]);  // Q_1's last use
+        } else {
+          umma_commit_w(&o_full[1]);
         }
+      }
+      if (!ok) break;
+      kvit += n1;
+    }
+    if (__any_sync(0xffffffffu, *abort)) {
+      umma_commit_w(drain);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
   } else {
