@@ -207,40 +207,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      int it = 0, tl = 0;
-      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
-        const int acc = tl & 1;
-        const uint32_t aph = (tl >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], aph ^ 1, abort, status)) break;
+  } else if (warp == 1) {  // the whole warp runs the MMA role; one elected lane issues
+    int it = 0, tl = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
+      const int acc = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1;
+      if (!mbar_wait_warp(&tempty[acc], aph ^ 1, abort, status)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tbase + acc * BN;
+      bool ok = true;
+      for (int k = 0; k < kblocks; ++k, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait_warp(&full[s], ph, abort, status)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tbase + acc * BN;
-        bool ok = true;
-        for (int k = 0; k < kblocks; ++k, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&full[s], ph, abort, status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint8_t* st = smem + s * STAGE_BYTES;
-          const uint64_t a_desc = sdesc_kmajor_sw128(st);
-          const uint64_t b_desc = sdesc_kmajor_sw128(st + A_BYTES);
+        const uint8_t* st = smem + s * STAGE_BYTES;
+        const uint64_t a_desc = sdesc_kmajor_sw128(st);
+        const uint64_t b_desc = sdesc_kmajor_sw128(st + A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16_ss(d_tmem, a_desc + (uint64_t)(kk * 2), b_desc + (uint64_t)(kk * 2), IDESC, (k | kk) != 0);
-          umma_commit(&empty[s]);
-        }
-        if (!ok) break;
-        umma_commit(&tfull[acc]);
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_bf16_ss_w(d_tmem, a_desc + (uint64_t)(kk * 2), b_desc + (uint64_t)(kk * 2), IDESC, (k | kk) != 0);
+        umma_commit_w(&empty[s]);
       }
-      if (*abort) {  // let the MMAs already issued finish before the TMEM is released
-        umma_commit(drain);
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
-        }
+      if (!ok) break;
+      umma_commit_w(&tfull[acc]);
+    }
+    if (__any_sync(0xffffffffu, *abort)) {  // let the MMAs already issued finish before the TMEM is released
+      umma_commit_w(drain);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
   } else {
@@ -363,46 +361,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      int it = 0, tl = 0;
-      for (int tile = pair; tile < ntiles; tile += npairs, ++tl) {
-        const int acc = tl & 1;
-        const uint32_t aph = (tl >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], aph ^ 1, abort, status)) break;
+  } else if (warp == 1 && rank == 0) {  // the whole warp runs the MMA role; one elected lane issues
+    int it = 0, tl = 0;
+    for (int tile = pair; tile < ntiles; tile += npairs, ++tl) {
+      const int acc = tl & 1;
+      const uint32_t aph = (tl >> 1) & 1;
+      if (!mbar_wait_warp(&tempty[acc], aph ^ 1, abort, status)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tbase + acc * BN;
+      bool ok = true;
+      for (int k = 0; k < kblocks; ++k, ++it) {
+        const int s = it % PAIR_STAGES;
+        const uint32_t ph = (it / PAIR_STAGES) & 1;
+        if (!mbar_wait_warp(&full[s], ph, abort, status)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tbase + acc * BN;
-        bool ok = true;
-        for (int k = 0; k < kblocks; ++k, ++it) {
-          const int s = it % PAIR_STAGES;
-          const uint32_t ph = (it / PAIR_STAGES) & 1;
-          if (!mbar_wait(&full[s], ph, abort, status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint8_t* st = smem + s * PAIR_STAGE_BYTES;
-          const uint64_t a_desc = AMN ? sdesc_mnmajor_sw128(st, CHUNK) : sdesc_kmajor_sw128(st);
-          const uint64_t b_desc = BMN ? sdesc_mnmajor_sw128(st + HALF_ROWS * BK * 2, CHUNK)
-                                      : sdesc_kmajor_sw128(st + HALF_ROWS * BK * 2);
-          // K-step kk: 32 bytes along a K-major row, or 16 K rows (2 KB) of an MN-major box
+        const uint8_t* st = smem + s * PAIR_STAGE_BYTES;
+        const uint64_t a_desc = AMN ? sdesc_mnmajor_sw128(st, CHUNK) : sdesc_kmajor_sw128(st);
+        const uint64_t b_desc = BMN ? sdesc_mnmajor_sw128(st + HALF_ROWS * BK * 2, CHUNK)
+                                    : sdesc_kmajor_sw128(st + HALF_ROWS * BK * 2);
+        // K-step kk: 32 bytes along a K-major row, or 16 K rows (2 KB) of an MN-major box
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma2_bf16_ss(d_tmem, a_desc + (uint64_t)(AMN ? kk * (2048 >> 4) : kk * 2),
-                          b_desc + (uint64_t)(BMN ? kk * (2048 >> 4) : kk * 2), IDESC2, (k | kk) != 0);
-          umma2_commit_mc(&empty[s], 0x3);
-        }
-        if (!ok) break;
-        umma2_commit_mc(&tfull[acc], 0x3);
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma2_bf16_ss_w(d_tmem, a_desc + (uint64_t)(AMN ? kk * (2048 >> 4) : kk * 2),
+                        b_desc + (uint64_t)(BMN ? kk * (2048 >> 4) : kk * 2), IDESC2, (k | kk) != 0);
+        umma2_commit_mc_w(&empty[s], 0x3);
       }
-      if (*abort) {  // let the MMAs already issued finish before the TMEM is released
-        umma2_commit_mc(drain, 0x1);
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
-        }
+      if (!ok) break;
+      umma2_commit_mc_w(&tfull[acc], 0x3);
+    }
+    if (__any_sync(0xffffffffu, *abort)) {  // let the MMAs already issued finish before the TMEM is released
+      umma2_commit_mc_w(drain, 0x1);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
-  } else {
+  } else if (warp >= 2) {
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     int tl = 0;
     for (int tile = pair; tile < ntiles; tile += npairs, ++tl) {
