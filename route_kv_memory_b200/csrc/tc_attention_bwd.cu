@@ -13,8 +13,9 @@
 //   attn_bwd_dkdv_kernel  per (sequence, KV group, 128-key tile), K and V staying in shared
 //                         memory while the query tiles t >= its own of all G heads stream through
 //                         two 2-stage rings (Q with its lse and D rows; dO): S^T = K Q^T and
-//                         dP^T = V dO^T into TMEM, the compute warps write P^T and scale * dS^T
-//                         (bf16) over dP^T, then dK += dS^T Q and dV += P^T dO accumulate in TMEM.
+//                         dP^T = V dO^T into TMEM, the compute warps write P^T and dS^T (bf16)
+//                         over dP^T, then dK += dS^T Q and dV += P^T dO accumulate in TMEM (dK
+//                         takes its factor scale when it is written out).
 // Warp 0 loads (TMA), warp 1 issues the MMAs, warps 2-9 compute: two warps per TMEM lane quadrant,
 // each taking 64 of a row's 128 columns; a warp packs its bf16 results into the first 32 columns of
 // its own 64-column range (so neither half overwrites what the other still reads), and the MMAs
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t s_tmem = tbase + lane_off + S_COL, p_tmem = tbase + lane_off + P_COL;
     const uint32_t q_tmem = tbase + lane_off + Q_COL + half * (DH / 2);
-    const float sl2 = a.scale * 1.4426950408889634f;
+    const float sl2 = a.scale * 1.4426950408889634f, l2scale = log2f(a.scale);
     int sit = 0;
     for (int rr = 0;; ++rr) {
       const int w = snake(rr, gridDim.x, blockIdx.x, nwork);
@@ -283,9 +284,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int n = qt + 1, row = qt * BT + r;
       const bool valid = row < a.S;
       const size_t li = ((size_t)b * a.Hq + h) * a.lse_ld + (valid ? row : 0);
-      const float lse2 = valid ? a.lse[li] : 0.f, drow = valid ? a.dsum[li] : 0.f;
+      // scale * P = 2^(s sl2 - lse + log2 scale): dQ's factor scale rides in the exponent
+      const float lse2 = (valid ? a.lse[li] : 0.f) - l2scale, drow = valid ? a.dsum[li] : 0.f;
       const float2 sl2v = make_float2(sl2, sl2), nlse2v = make_float2(-lse2, -lse2);
-      const float2 ndrowv = make_float2(-drow, -drow), scalev = make_float2(a.scale, a.scale);
+      const float2 ndrowv = make_float2(-drow, -drow);
       bool ok = true;
       for (int j = 0; j < n; ++j, ++sit) {
         if (!mbar_wait(s_full, sit & 1, abort, status)) { ok = false; break; }
@@ -318,7 +320,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             sv[cc][2 * e + 1] = __float_as_uint(p1);
           }
         }
-        // phase 2: dS = scale P (dP - D), packed over the first 32 of this half's dP columns
+        // phase 2: scale dS = (scale P) (dP - D), packed over the first 32 of this half's dP columns
         if (!mbar_wait(dp_full, sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
         uint32_t pv[2][32];
@@ -332,8 +334,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int e = 0; e < 16; ++e) {
             const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(pv[cc][2 * e]), __uint_as_float(pv[cc][2 * e + 1])),
                                          ndrowv);
-            const float2 r2 = __fmul2_rn(
-                __fmul2_rn(make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1])), scalev), d2);
+            const float2 r2 = __fmul2_rn(make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1])), d2);
             pk[e] = pack2(r2.x, r2.y);
           }
           tmem_st16(p_tmem + 64 * half + cc * 16, pk);
@@ -516,7 +517,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         umma_bf16_ss_w(tbase + P_COL, vd + kstep(kk, C::HALF), dod + kstep(kk, C::HALF), IDESC_S, kk != 0);
       umma_commit_w(dp_full);
     };
-    // dK += scale*dS^T Q, then dV += P^T dO, each freeing its ring slot; the compute warps pack
+    // dK += dS^T Q, then dV += P^T dO, each freeing its ring slot; the compute warps pack
     // P^T and dS^T over the dP^T columns: K-step kk (16 queries) of P^T at
     // 64 (kk / 4) + 32 ((kk / 2) % 2) + 8 (kk % 2), of dS^T 16 further
     auto issue_acc = [&](int st, bool acc) {
@@ -614,7 +615,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // query column c is used iff it is a real row at or after this key: q0 + c < S, q0 + c >= key
         const int q0 = qt * BT, cmax = a.S - q0, cmin = key - q0;
         const bool masked = __any_sync(0xffffffffu, cmin > 64 * half || cmax < 64 * half + 64);  // warp-uniform
-        const float2 sl2v = make_float2(sl2, sl2), scalev = make_float2(a.scale, a.scale);
+        const float2 sl2v = make_float2(sl2, sl2);
         // phase 1: this half's 64 scores into registers (S^T's columns are then free for the next
         // step), P^T = 2^(s sl2 - lse) in float32
         uint32_t sv[2][32];
@@ -646,7 +647,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
           }
         }
-        // phase 2: dS^T = scale P^T (dP^T - D); P^T and dS^T packed over this half's dP^T columns,
+        // phase 2: dS^T = P^T (dP^T - D) (dK takes its factor scale in the epilogue); P^T and dS^T
+        // packed over this half's dP^T columns,
         // chunk cc at [32 cc, 32 cc + 16) and [32 cc + 16, 32 cc + 32) of the half
         if (!mbar_wait(dp_full, sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
@@ -667,7 +669,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const float2 p2 = make_float2(__uint_as_float(sv[cc][2 * e]), __uint_as_float(sv[cc][2 * e + 1]));
               pp[e] = pack2(p2.x, p2.y);
               const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(pv[2 * e]), __uint_as_float(pv[2 * e + 1])), nd);
-              const float2 r2 = __fmul2_rn(__fmul2_rn(p2, scalev), d2);
+              const float2 r2 = __fmul2_rn(p2, d2);
               pd[e] = pack2(r2.x, r2.y);
             }
           }
@@ -685,14 +687,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const bool valid = key < a.S;
       const int wkv = 2 * a.Hkv * DH;
       float* dst = a.dkv + ((size_t)b * a.S + (valid ? key : 0)) * (size_t)wkv + (size_t)g * DH;
-      {  // the first warpgroup writes dK (columns [0, dkv)), the second dV ([dkv, 2 dkv))
+      {  // the first warpgroup writes dK (columns [0, dkv)) = scale * sum dS^T Q, the second dV ([dkv, 2 dkv))
         const uint32_t src = tbase + lane_off + (half ? V_COL : K_COL);
         float* d = dst + (half ? a.Hkv * DH : 0);
+        const float f = half ? 1.f : a.scale;
 #pragma unroll
         for (int c = 0; c < DH; c += 32) {
           uint32_t v[32];
           tmem_ld32(src + c, v);
           tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
           if (valid) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
