@@ -135,8 +135,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* pv_done = bars + 12;  // [2]
   uint64_t* o_full = bars + 14;   // [2]
   uint64_t* o_empty = bars + 16;  // [2]
-  uint64_t* drain = bars + 18;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 19);
+  uint64_t* p_half = bars + 18;   // [2] keys 0-63 of P_t are in TMEM
+  uint64_t* drain = bars + 20;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 21);
   int* stok = (int*)(smem + 2 * C::Q_BYTES + 2 * C::KV_BYTES + 256);  // MODE 1: loader's tokens, [2][BQ]
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&pv_done[i], 1);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_empty[i], 4);
+      mbar_init(&p_half[i], 4);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -353,13 +355,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       umma_commit_w(&s_full[t]);
     };
-    auto issue_pv = [&](int t, int st, int j) {
+    // P V in two halves of four K-steps: keys 0-63 as soon as the softmax has packed them, keys
+    // 64-127 after p_full
+    auto issue_pv_half = [&](int t, int st, int j, int hh) {
       const uint64_t vd = sdesc_mnmajor_sw128(sKV + st * C::KV_BYTES + C::K_BYTES);
 #pragma unroll
-      for (int kk = 0; kk < BKV / 16; ++kk)
+      for (int k4 = 0; k4 < BKV / 32; ++k4) {
+        const int kk = hh * (BKV / 32) + k4;
         umma_bf16_ts_w(tbase + O_COL(t), tbase + S_COL(t) + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
-                     (j | kk) != 0);
-      umma_commit_w(&pv_done[t]);
+                       (j | kk) != 0);
+      }
+      if (hh) umma_commit_w(&pv_done[t]);
     };
     int nx0 = 0, nx1 = 0;  // tiles of the next item, looked up while this one runs
     {
@@ -400,10 +406,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int cur = kvit + j, st = cur & 1, nst = (cur + 1) & 1;
         bool next_ready = false;
         if (j < n0) {
-          if (!mbar_wait_warp(&p_full[0], pc[0] & 1, abort, status)) { ok = false; break; }
+          if (!mbar_wait_warp(&p_half[0], pc[0] & 1, abort, status)) { ok = false; break; }
           if (j == 0 && !mbar_wait_warp(&o_empty[0], (wi & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(0, st, j);
+          issue_pv_half(0, st, j, 0);
+          if (!mbar_wait_warp(&p_full[0], pc[0] & 1, abort, status)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv_half(0, st, j, 1);
           ++pc[0];
           if (j + 1 == n0) umma_commit_w(&o_full[0]);
           if (j + 1 < n0) {
@@ -414,10 +423,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (j + 2 == n0) umma_commit_w(&q_empty[0]);  // Q_0's last use
           }
         }
-        if (!mbar_wait_warp(&p_full[1], pc[1] & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait_warp(&p_half[1], pc[1] & 1, abort, status)) { ok = false; break; }
         if (j == 0 && !mbar_wait_warp(&o_empty[1], (wi & 1) ^ 1, abort, status)) { ok = false; break; }
         tc_fence_after();
-        issue_pv(1, st, j);
+        issue_pv_half(1, st, j, 0);
+        if (!mbar_wait_warp(&p_full[1], pc[1] & 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv_half(1, st, j, 1);
         ++pc[1];
         umma_commit_w(&kv_empty[st]);
         if (j + 1 < n1) {
@@ -526,8 +538,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           m_ref = mx;
           l *= corr;
         }
+        // rescale the O rows (rare with the lazy threshold) before pass 2, since the first half of
+        // P_j V_j starts while pass 2 runs.  S_j landing means P_{j-1} V_{j-1}, issued before QK_j,
+        // has completed, so the wait below returns at once.
+        if (__ballot_sync(0xffffffffu, rescale)) {
+          if (!mbar_wait(&pv_done[t], (sit - 1) & 1, abort, status)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < DH; c += 32) {
+            uint32_t ov[32];
+            tmem_ld32(o_tmem + c, ov);
+            tmem_ld_wait();
+            const float2 c2 = make_float2(corr, corr);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), c2);
+              ov[e] = __float_as_uint(o2.x);
+              ov[e + 1] = __float_as_uint(o2.y);
+            }
+            tmem_st16(o_tmem + c, *reinterpret_cast<const uint32_t(*)[16]>(&ov[0]));
+            tmem_st16(o_tmem + c + 16, *reinterpret_cast<const uint32_t(*)[16]>(&ov[16]));
+          }
+        }
         // pass 2: P = 2^(s*sl2 - m_ref) as bf16 pairs over the first 64 columns of S; the
-        // TMEM load of chunk c+1 is in flight while chunk c is exponentiated
+        // TMEM load of chunk c+1 is in flight while chunk c is exponentiated.  Keys 0-63 (chunks 0
+        // and 1) are signalled on p_half so that their half of P V can start.
         const float nm = -m_ref;
         const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(nm, nm);
         float2 lsum2 = make_float2(0.f, 0.f);
@@ -553,31 +588,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pk[e] = *(uint32_t*)&hb;
           }
           tmem_st16(s_tmem + c * 16, pk);
+          if (c == 1) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_half[t]);
+          }
         }
         const float lsum = lsum2.x + lsum2.y;
         l += lsum;
-        // rescale the O rows (rare with the lazy threshold).  S_j landing means PV_{j-1},
-        // issued before QK_j, has completed, so the wait below returns at once.  PV_j is
-        // issued only after p_full, so it accumulates onto the rescaled rows.
-        if (__ballot_sync(0xffffffffu, rescale)) {
-          if (!mbar_wait(&pv_done[t], (sit - 1) & 1, abort, status)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < DH; c += 32) {
-            uint32_t ov[32];
-            tmem_ld32(o_tmem + c, ov);
-            tmem_ld_wait();
-            const float2 c2 = make_float2(corr, corr);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), c2);
-              ov[e] = __float_as_uint(o2.x);
-              ov[e + 1] = __float_as_uint(o2.y);
-            }
-            tmem_st16(o_tmem + c, *reinterpret_cast<const uint32_t(*)[16]>(&ov[0]));
-            tmem_st16(o_tmem + c + 16, *reinterpret_cast<const uint32_t(*)[16]>(&ov[16]));
-          }
-        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
