@@ -101,3 +101,27 @@ def check_out(o_gpu: torch.Tensor, o_ref: np.ndarray, dtype: str, rows=None):
     else:
         assert rel_l2 <= BF16_REL_L2 and max_abs <= BF16_ATOL, f"bf16 rel-L2 {rel_l2:.3e} max-abs {max_abs:.3e}"
     return max_abs, rel_l2
+
+
+def bf16_round(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).double().numpy()
+
+
+def lazy_rescales(q: np.ndarray, K: np.ndarray, scale: float, tile: int = 128, threshold: float = 8.0) -> int:
+    """Row-tiles of one sequence at which a tiled online softmax that moves its reference maximum only when
+    it is exceeded by more than 2^threshold (log2 units) moves it after the row's first tile.  Counted from
+    the oracle's q [S, Hq, dh] and K [S, Hkv, dh]."""
+    S, Hq, dh = q.shape
+    G = Hq // K.shape[1]
+    c = scale * 1.4426950408889634
+    n = 0
+    for h in range(Hq):
+        s = (q[:, h] @ K[:, h // G].T) * c
+        for t in range(S):
+            m = -np.inf
+            for j in range(t // tile + 1):
+                mx = s[t, j * tile:min(t + 1, (j + 1) * tile)].max()
+                if mx > m + threshold:
+                    n += m != -np.inf
+                    m = mx
+    return n

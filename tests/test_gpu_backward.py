@@ -17,7 +17,7 @@ import torch
 
 import oracle
 from fastmka_inputs import CONFIGS, FastMKAConfig, make_inputs
-from gpu_util import check_out, gpu_weights, oracle_weights
+from gpu_util import check_out, gpu_weights, lazy_rescales, oracle_weights
 
 pytestmark = pytest.mark.gpu
 
@@ -69,12 +69,24 @@ def oracle_backward(cfg, inp, dout, idx):
     return fwd, oracle.fastmka_backward(X, w, cfg, dout.float().numpy().astype(np.float64), fwd)
 
 
-def check_grads(cfg, seed=7):
+def check_grads(cfg, seed=7, ramp=None):
     inp = make_inputs(cfg)
+    if ramp is not None:  # scale the inputs up along the sequence by 1 -> ramp
+        import dataclasses
+        r = torch.linspace(1.0, ramp, cfg.seq)
+        x = inp.x.float()
+        x[:, :cfg.seq] *= r[None, :, None]
+        inp = dataclasses.replace(inp, x=x.to(inp.x.dtype))
     dout = output_gradient(cfg, seed)
     out, g, idx = gpu_backward(cfg, inp, dout)
     fwd, ref = oracle_backward(cfg, inp, dout, idx)
-    check_out(out, fwd["O"], "bf16")
+    if ramp is not None:  # the forward's reference maximum really moves after a row's first tile
+        assert lazy_rescales(fwd["q"][0], fwd["K"][0], 1.0 / np.sqrt(cfg.d_head)) > 200
+    if ramp is None:
+        check_out(out, fwd["O"], "bf16")
+    else:  # outputs of several units: the relative bound only (the absolute one assumes unit scale)
+        o = out.float().cpu().double().numpy().reshape(fwd["O"].shape)
+        assert np.linalg.norm(o - fwd["O"]) <= 1e-2 * np.linalg.norm(fwd["O"])
     errs = {}
     for k in GRADS:
         a, r = g[k].reshape(ref[k].shape), ref[k]
@@ -103,6 +115,13 @@ CASES = [
 @pytest.mark.parametrize("cfg", CASES, ids=[c.name for c in CASES])
 def test_layer_backward(cfg):
     check_grads(cfg)
+
+
+def test_layer_backward_rescaled_softmax():
+    """Inputs scaled up along the sequence (x 1 -> 3): the forward's tiled softmax moves its reference
+    maximum (and rescales O) in many row-tiles, so the row normalisers it leaves for the backward must
+    account for the moves."""
+    check_grads(small("bwd_rescaled", seq=512, d_head=128, router_hidden=128, block=64, seed=208), ramp=3.0)
 
 
 @pytest.mark.slow

@@ -7,8 +7,8 @@ import torch
 
 import oracle
 from fastmka_inputs import CONFIGS, FastMKAConfig, make_inputs, sample_rows, to_f64
-from gpu_util import (check_lambda, check_out, check_recall, gpu_prefill, gpu_weights, oracle_prefill,
-                      oracle_weights, out_errors, F32_ATOL)
+from gpu_util import (BF16_REL_L2, bf16_round, check_lambda, check_out, check_recall, gpu_prefill, gpu_weights,
+                      lazy_rescales, oracle_prefill, oracle_weights, out_errors, F32_ATOL)
 
 pytestmark = pytest.mark.gpu
 
@@ -65,6 +65,33 @@ def test_layer_edge_cases(cfg):
     check_lambda(lam, ref["lam"])
     check_recall(idx, ref)
     check_out(out, ref["O"], cfg.dtype)
+
+
+def test_attention_rescale_path():
+    """Inputs scaled up along the sequence (x 1 -> 4): a row's later key tiles beat its first by up to 2^48,
+    so the tiled softmax moves its reference maximum and rescales O in about a quarter of the row-tiles
+    (the rare path of the lazy max-shift, notes §4).  The layer's O is compared with the oracle's causal
+    attention over the oracle's own q, K, V rounded to bf16, the precision the attention reads them in, so
+    that the peaked softmax does not magnify the projections' rounding."""
+    import dataclasses
+    cfg = small("bf16_rescale", "bf16", seq=640, n_q_heads=4, n_kv_heads=2, d_head=128, block=64, seed=31)
+    inp = make_inputs(cfg)
+    ramp = torch.linspace(1.0, 4.0, cfg.seq)
+    inp = dataclasses.replace(inp, x=(inp.x.float() * ramp[None, :, None]).to(torch.bfloat16))
+    ref = oracle_prefill(cfg, inp)
+    scale = 1.0 / math.sqrt(cfg.d_head)
+    assert lazy_rescales(ref["q"][0], ref["K"][0], scale) > 1000
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    check_recall(idx, ref)
+    O16 = oracle.causal_gqa_attention(bf16_round(ref["q"][0]), np.arange(cfg.seq), bf16_round(ref["K"][0]),
+                                      bf16_round(ref["V"][0]), cfg.n_kv_heads, scale)
+    g = out.float().cpu().double().numpy().reshape(O16.shape)
+    max_abs, rel_l2 = out_errors(g, O16)
+    # The outputs here reach several units (V grows with the ramp): bound the largest error relative to
+    # the largest output.  P and O are rounded to bf16 once each (<= 2^-9 relative), so about 0.4% is
+    # expected; a missed or doubled rescale would be off by factors up to 2^48.
+    assert rel_l2 <= BF16_REL_L2 and max_abs <= 1e-2 * np.abs(O16).max(), (rel_l2, max_abs, np.abs(O16).max())
 
 
 def test_qwen7b_4k_layer():
