@@ -152,36 +152,14 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulator.  One thread issues.
-__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem desc]^T (A read from tensor memory).
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Arrives once on `bar` when every tcgen05 op issued so far by this thread has completed.
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-// Warp-wide forms: the whole (converged) warp executes them and one lane, chosen by elect.sync,
-// issues.  Descriptor and address arithmetic then stays in converged code, where it can use the
-// uniform datapath, instead of a one-lane branch; every tcgen05 op of the role must come from the
-// same elected lane (elect.sync over a converged full warp picks the same one each time).
+// tcgen05.mma kind::f16 (bf16 inputs, fp32 accumulator) and commit, in warp-wide form: the whole
+// (converged) warp executes them and one lane, chosen by elect.sync, issues.  Descriptor and address
+// arithmetic then stays in converged code, where it can use the uniform datapath, instead of a
+// one-lane branch.  Every tcgen05 op of the role must come from the same elected lane (elect.sync
+// over a converged full warp picks the same one each time).
+//   umma_bf16_ss_w: D[tmem] (+)= A[smem desc] * B[smem desc]^T
+//   umma_bf16_ts_w: D[tmem] (+)= A[tmem] * B[smem desc]^T (A read from tensor memory)
+//   umma_commit_w:  arrive once on `bar` when every tcgen05 op issued so far by the lane has completed
 __device__ __forceinline__ void umma_bf16_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                uint32_t accumulate) {
   asm volatile(
@@ -268,27 +246,11 @@ __device__ __forceinline__ void tmem_alloc2(uint32_t* dst_smem, uint32_t ncols) 
 __device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
-// D[tmem] (+)= A * B^T over both CTAs of the pair (M = 256); issued by one thread of rank 0.
-__device__ __forceinline__ void umma2_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                              uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
-      "r"(0u), "r"(0u)
-      : "memory");
-}
-// Arrives once on `bar` in every CTA of `cta_mask` when the pair's MMAs issued so far have completed.
-__device__ __forceinline__ void umma2_commit_mc(uint64_t* bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          smem_u32(bar)),
-      "h"(cta_mask)
-      : "memory");
-}
-// Warp-wide forms of the two above (see umma_bf16_ss_w): one elected lane of a converged warp issues.
+// Over both CTAs of the pair, warp-wide like umma_bf16_ss_w (one elected lane of a converged warp of
+// rank 0 issues):
+//   umma2_bf16_ss_w:   D[tmem] (+)= A * B^T with M = 256, each CTA holding its half of A and of B
+//   umma2_commit_mc_w: arrive once on `bar` in every CTA of `cta_mask` when the pair's MMAs issued so
+//                      far have completed
 __device__ __forceinline__ void umma2_bf16_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                 uint32_t accumulate) {
   asm volatile(
