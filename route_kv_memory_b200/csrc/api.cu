@@ -803,7 +803,7 @@ static int check_train(const mka_config* cfg, Dims* d) {
   if (rc) return rc;
   if (!d->bf16 || d->paths != 1 || d->block_sparse)
     return fail(MKA_ERR_UNSUPPORTED, "the layer backward needs bf16 FastMKA (attention_paths 1, no block_sparse)");
-  if (d->rh % 32 || d->rh > 512) return fail(MKA_ERR_UNSUPPORTED, "the layer backward needs router_hidden % 32 == 0, <= 512");
+  if (d->rh % 32 || d->rh > 512) return fail(MKA_ERR_UNSUPPORTED, "the layer backward needs router_hidden a multiple of 32, at most 512");
   return MKA_OK;
 }
 
