@@ -461,6 +461,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t s_tmem = tbase + lane_off + S_COL(t);
     const uint32_t o_tmem = tbase + lane_off + O_COL(t);
     const float sl2 = a.scale * 1.4426950408889634f;
+    // causal output rows start on 32-byte boundaries: one 32-byte store per 16 columns
+    const bool o32 = !GA && ((uintptr_t)a.o & 31) == 0 && a.o_ld % 16 == 0 && a.o_bstride % 16 == 0;
     int sit = 0;
     for (int rr = 0; rr * (int)gridDim.x < nwork; ++rr) {
       const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
@@ -637,7 +639,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                                         __uint_as_float(ov[v >> 1][(v & 1) * 16 + 2 * e + 1]) * inv);
               wv[e] = *(uint32_t*)&hb;
             }
-            if constexpr (GA) {
+            if (GA || o32) {
               st_global_v8(orow + c + v * 16, wv);
             } else {
               *(uint4*)(orow + c + v * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
