@@ -69,7 +69,18 @@ __device__ __forceinline__ void store_chunk(const Epilogue& ep, int m, int n, ui
       }
       if (g.is_bf16) {
         bf16* p = (bf16*)g.ptr + off;
-        if ((off & 7) == 0) {
+        if (((uintptr_t)p & 31) == 0) {  // one 32-byte store per 16 columns
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[v * 16 + 2 * e]), __uint_as_float(r[v * 16 + 2 * e + 1]));
+              w[e] = *(uint32_t*)&h;
+            }
+            st_global_v8(p + v * 16, w);
+          }
+        } else if ((off & 7) == 0) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 u;
@@ -87,7 +98,14 @@ __device__ __forceinline__ void store_chunk(const Epilogue& ep, int m, int n, ui
         }
       } else {
         float* p = (float*)g.ptr + off;
-        if ((off & 3) == 0) {
+        if (((uintptr_t)p & 31) == 0) {  // one 32-byte store per 8 columns
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t w[8] = {r[8 * v], r[8 * v + 1], r[8 * v + 2], r[8 * v + 3],
+                                   r[8 * v + 4], r[8 * v + 5], r[8 * v + 6], r[8 * v + 7]};
+            st_global_v8(p + v * 8, w);
+          }
+        } else if ((off & 3) == 0) {
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             *(float4*)(p + v * 4) = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
