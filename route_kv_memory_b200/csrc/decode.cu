@@ -472,11 +472,6 @@ __device__ void attn_unit(const DecodeArgs& a, const int split, const int g, con
   }
   __syncthreads();  // the next unit of this CTA reuses the shared memory
 }
-template <int DH>
-__global__ void __launch_bounds__(NWD * 32) decode_attn_kernel(DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  attn_unit<DH>(a, blockIdx.x, blockIdx.y, blockIdx.z, a.pos[blockIdx.z], a.qf, a.dq, smem_raw);
-}
 }  // namespace dk
 
 // float32 split-KV attention (CUDA cores): grid (nsplit, Hq, B), one warp per position stride.
