@@ -191,10 +191,8 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     barrier(world)
     step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
-    ms = statistics.mean(step_ms)
-    ms = max_over_ranks(ms, world)
+    value, ms = job_throughput(cfg.tokens, statistics.mean(step_ms), world)
     launches_per_step = prefill_kernels(cfg)
-    value = world * cfg.tokens / (ms / 1e3)
 
     peaks = load_peaks()
     fl = prefill_flops(cfg)
@@ -251,8 +249,8 @@ def run_ours(args, rank, world, local_rank):
         return t0.elapsed_time(t1) / n
 
     e2e_run(3, False)
-    e2e_ms = max_over_ranks(e2e_run(n_e2e, True), world)
-    e2e = {"value": world * cfg.tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+    e2e_value, e2e_ms = job_throughput(cfg.tokens, e2e_run(n_e2e, True), world)
+    e2e = {"value": e2e_value, "unit": "tokens/s",
            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
            "d2h_bytes_per_step": o_host[0].numel() * o_host[0].element_size(), "ms_per_step": round(e2e_ms, 4),
            "steps": n_e2e,
@@ -362,7 +360,7 @@ def run_train(args, rank, world, local_rank):
             ev1[i].record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(ev0, ev1)), world)
+    value, ms = job_throughput(cfg.tokens, statistics.mean(a.elapsed_time(b) for a, b in zip(ev0, ev1)), world)
     assert mka.mka_status() == 0
 
     # end to end: X and dO from pinned host memory, dX back, every step (sequential)
@@ -380,7 +378,7 @@ def run_train(args, rank, world, local_rank):
         dx_host.copy_(grads["dx"], non_blocking=True)
     t1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(t0.elapsed_time(t1) / n_e2e, world)
+    e2e_value, e2e_ms = job_throughput(cfg.tokens, t0.elapsed_time(t1) / n_e2e, world)
 
     peaks = load_peaks()
     fl = train_flops(cfg)
@@ -388,7 +386,7 @@ def run_train(args, rank, world, local_rank):
     ab_tf = fl["attention_bwd"] / (ab_ms / 1e3) / 1e12
     return {
         "metric": "FastMKA layer training step (forward + backward) tokens/s",
-        "value": round(world * cfg.tokens / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world,
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) inputs and output gradient, N(0,1/d_in) weights)",
@@ -407,7 +405,7 @@ def run_train(args, rank, world, local_rank):
         "layer_tflops": round(sum(fl.values()) / (ms / 1e3) / 1e12, 1),
         "forward_stage_ms": {n: round(float(v), 4) for n, v in zip(PREFILL_STAGES, fw_st)},
         "backward_stage_ms": {n: round(float(v), 4) for n, v in zip(BACKWARD_STAGES, bw_st)},
-        "e2e": {"value": round(world * cfg.tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": 2 * x_host.numel() * x_host.element_size(),
                 "d2h_bytes_per_step": dx_host.numel() * dx_host.element_size(), "ms_per_step": round(e2e_ms, 4),
                 "how": "pinned host X and dO -> device, training step, device dX -> pinned host, sequential"},
@@ -571,11 +569,21 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of the ranks' values, returned on every rank.  The collective's tensor lives where
+    the process group's backend wants it: on the GPU for NCCL, in host memory for gloo."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, ms: float, world: int):
+    """Whole-job units per second and the job's time per step: every rank processes units_per_rank
+    in its own `ms`, and the job takes as long as its slowest rank.  Returns (units/s, max ms)."""
+    ms_max = max_over_ranks(ms, world)
+    return world * units_per_rank / (ms_max / 1e3), ms_max
 
 
 def main():
