@@ -19,7 +19,7 @@ from .fastmka import (  # noqa: F401
     recall_select, longterm_recall, fuse_sources, kv_project, causal_gqa_attention,
     online_softmax_attend, fastmka_prefill, fastmka_decode, Weights64, weights_f64,
     recalled_block_attention, mka_full_prefill, block_sparse_gqa_attention,
-    EXCUSE_EPS,
+    EXCUSE_EPS, recall_mismatch_excused, recall_mismatches,
 )
 from .backward import (  # noqa: F401
     fastmka_backward, causal_gqa_attention_backward, session_ema_backward, longterm_recall_backward,

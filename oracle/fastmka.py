@@ -38,9 +38,10 @@ from typing import Optional
 import numpy as np
 from scipy.special import erfc
 
-# A recalled-index mismatch at token t is excused only if one of the hash
-# projections that decide it (the token's own, or an eligible block's) is
-# closer to zero than this.
+# Hash bits whose projection lies closer to zero than this may come out either
+# way on another machine: a recalled-index mismatch is excused only when the
+# other side's list is the recall under some flip of such bits
+# (recall_mismatch_excused).
 EXCUSE_EPS = 1e-4
 
 
@@ -182,23 +183,19 @@ def recall_select(code_t: int, summary_codes: np.ndarray, n_eligible: int, R: in
 
 
 def longterm_recall(x_rows: np.ndarray, positions: np.ndarray, summaries: np.ndarray, P: np.ndarray,
-                    b: int, R: int, summary_proj: Optional[np.ndarray] = None):
+                    b: int, R: int):
     """L3 long-term memory for the rows of ONE sequence.
 
     x_rows [n, d] are the raw tokens at `positions` [n]; summaries [nblk, d] the
     block means of the whole sequence.  Block j is eligible at t iff (j+1)*b <= t.
-    Returns (idx [n, R] with -1 padding, count [n], M3 [n, d], excuse [n], x_codes [n], x_proj [n, nb]).
+    Returns (idx [n, R] with -1 padding, count [n], M3 [n, d], x_codes [n], x_proj [n, nb]).
     """
     n, d = x_rows.shape
-    s_codes, s_proj = hash_codes(summaries, P)
-    if summary_proj is not None:
-        s_proj = summary_proj
+    s_codes, _ = hash_codes(summaries, P)
     x_codes, x_proj = hash_codes(x_rows, P)
     idx = np.full((n, R), -1, dtype=np.int64)
     count = np.zeros(n, dtype=np.int64)
     M3 = np.zeros((n, d))
-    excuse = np.zeros(n, dtype=bool)
-    near_zero_block = (np.abs(s_proj) < EXCUSE_EPS).any(axis=-1) if len(summaries) else np.zeros(0, bool)
     for i, t in enumerate(positions):
         n_elig = min(int(t) // b, len(summaries))
         sel = recall_select(int(x_codes[i]), s_codes, n_elig, R)
@@ -206,8 +203,87 @@ def longterm_recall(x_rows: np.ndarray, positions: np.ndarray, summaries: np.nda
         count[i] = len(sel)
         if len(sel):
             M3[i] = summaries[sel].mean(axis=0)
-        excuse[i] = bool((np.abs(x_proj[i]) < EXCUSE_EPS).any() or near_zero_block[:n_elig].any())
-    return idx, count, M3, excuse, x_codes, x_proj
+    return idx, count, M3, x_codes, x_proj
+
+
+def recall_mismatch_excused(got, x_proj_t: np.ndarray, s_proj: np.ndarray, n_eligible: int, R: int,
+                            eps: float = EXCUSE_EPS, max_token_bits: int = 16) -> bool:
+    """Whether the recalled list `got` is the L3 recall of token t once some of the hash bits
+    that lie within eps of zero are flipped.
+
+    notes §1 (L3 hash recall) with the sign-code reading: bit k of a code is [p_k > 0].  A bit
+    whose projection has |p_k| < eps may come out either way under another summation order, so
+    any recall that some such flip produces is as correct as the oracle's.  x_proj_t [nb] is
+    token t's projection, s_proj [nblk, nb] the summaries'; `got` the other side's recalled
+    indices in order (-1 padding ignored).  Bits further than eps from zero are fixed, so a
+    near-zero component that cannot move the selection excuses nothing.
+
+    Exact: the token's near-zero bits are enumerated (at most max_token_bits of them); a
+    block's own near-zero bits can move its distance to any value in [d - u, d + v] (u of them
+    differ from the token's bit, v agree), and the selection is the first min(R, n_eligible)
+    blocks in (distance, index) order, so `got` is reachable iff the greedy choice -- the
+    lowest distances for the blocks of `got` in its order, the highest for every other
+    eligible block -- keeps that order.
+    """
+    got = [int(j) for j in got if int(j) >= 0]
+    n_eligible = min(int(n_eligible), len(s_proj))
+    if len(got) != min(R, n_eligible) or len(set(got)) != len(got) or any(j >= n_eligible for j in got):
+        return False
+    if not got:
+        return True
+    nb = len(x_proj_t)
+    place = np.left_shift(np.uint64(1), np.arange(nb, dtype=np.uint64))
+    sp = np.asarray(s_proj[:n_eligible], np.float64)
+    s_bits = (sp > 0)
+    s_free = np.abs(sp) < eps                                    # [n_eligible, nb]
+    t_bits = np.asarray(x_proj_t, np.float64) > 0
+    t_free = np.flatnonzero(np.abs(np.asarray(x_proj_t, np.float64)) < eps)
+    if len(t_free) > max_token_bits:
+        raise ValueError(f"{len(t_free)} near-zero token bits: too many to enumerate")
+    others = np.setdiff1d(np.arange(n_eligible), got)
+    for flips in range(1 << len(t_free)):
+        tb = t_bits.copy()
+        for k_i, k in enumerate(t_free):
+            if (flips >> k_i) & 1:
+                tb[k] = not tb[k]
+        differ = s_bits != tb[None, :]                           # XOR bits
+        dist = differ.sum(axis=1)
+        lo = dist - (differ & s_free).sum(axis=1)                # flip free bits that differ
+        hi = dist + (~differ & s_free).sum(axis=1)               # flip free bits that agree
+        ok, prev = True, None
+        for j in got:
+            dj = int(lo[j]) if prev is None else max(int(lo[j]), prev[0] + (0 if j > prev[1] else 1))
+            if dj > hi[j]:
+                ok = False
+                break
+            prev = (dj, j)
+        if ok and len(others):
+            ok = bool(np.all((hi[others] > prev[0]) | ((hi[others] == prev[0]) & (others > prev[1]))))
+        if ok:
+            return True
+    return False
+
+
+def recall_mismatches(got_idx: np.ndarray, ref: dict, rows=None):
+    """Counts (unexcused, excused) tokens whose recalled list `got_idx` [B, S or len(rows), R]
+    differs from the oracle's `ref` (a fastmka_prefill / mka_full_prefill result); a mismatch is
+    excused by recall_mismatch_excused only.  Returns the two counts and the unexcused (b, t)."""
+    ref_idx = ref["idx"] if rows is None else ref["idx"][:, rows]
+    pos = np.arange(ref["idx"].shape[1]) if rows is None else np.asarray(rows)
+    got_idx = np.asarray(got_idx).reshape(ref_idx.shape)
+    R = ref_idx.shape[-1]
+    nblk = ref["summary_proj"].shape[1]
+    b = ref["block"]
+    unexcused, excused, where = 0, 0, []
+    for bi, ti in zip(*np.nonzero((got_idx != ref_idx).any(axis=-1))):
+        t = int(pos[ti])
+        if recall_mismatch_excused(got_idx[bi, ti], ref["x_proj"][bi, t], ref["summary_proj"][bi],
+                                   min(t // b, nblk), R):
+            excused += 1
+        else:
+            unexcused += 1
+            where.append((int(bi), t))
+    return unexcused, excused, where
 
 
 # ----------------------------------------------------------------------------- fuse + K/V
@@ -334,7 +410,7 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
         "lam": np.zeros((B, S, 3)),
         "idx": np.full((B, S, R), -1, np.int64),
         "count": np.zeros((B, S), np.int64),
-        "excuse": np.zeros((B, S), bool),
+        "block": b,
         "x_codes": np.zeros((B, S), np.uint32),
         "x_proj": np.zeros((B, S, w.P.shape[1])),
         "summary_codes": np.zeros((B, nblk), np.uint32),
@@ -369,7 +445,7 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
             out["route_margin"][bi, r0:r1] = route_margin(z, mode, tiers)
             M2, m2 = session_ema(xc, cfg.alpha, m2)
             pos = np.arange(r0, r1)
-            idx, cnt, M3, exc, xcodes, xproj = longterm_recall(xc[0], pos, summ, w.P, b, R, s_proj)
+            idx, cnt, M3, xcodes, xproj = longterm_recall(xc[0], pos, summ, w.P, b, R)
             if recall_fixed is not None:
                 idx = np.asarray(recall_fixed[0][bi, r0:r1], np.int64)
                 cnt = np.asarray(recall_fixed[1][bi, r0:r1], np.int64)
@@ -378,7 +454,7 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
             Xf = fuse_sources(lam, xc[0], M2[0], M3)
             Kc, Vc = kv_project(Xf, w.w_k, w.w_v)
             out["lam"][bi, r0:r1] = lam
-            out["idx"][bi, r0:r1], out["count"][bi, r0:r1], out["excuse"][bi, r0:r1] = idx, cnt, exc
+            out["idx"][bi, r0:r1], out["count"][bi, r0:r1] = idx, cnt
             out["x_codes"][bi, r0:r1], out["x_proj"][bi, r0:r1] = xcodes, xproj
             out["K"][bi, r0:r1] = Kc.reshape(-1, Hkv, dh)
             out["V"][bi, r0:r1] = Vc.reshape(-1, Hkv, dh)
@@ -484,8 +560,10 @@ def mka_full_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray
     b, R = cfg.block, cfg.recall_r
     G = Hq // Hkv
     rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    nb = w.P.shape[1]
     out = {"rows": rows, "lam": np.zeros((B, S, 3)), "idx": np.zeros((B, S, R), np.int64),
-           "count": np.zeros((B, S), np.int64), "excuse": np.zeros((B, S), bool),
+           "count": np.zeros((B, S), np.int64), "block": b, "x_proj": np.zeros((B, S, nb)),
+           "summary_proj": np.zeros((B, S // b, nb)),
            "O": np.zeros((B, len(rows), Hq * dh)), "route_margin": np.zeros((B, S))}
     mode, tiers = getattr(cfg, "route_mode", "soft"), getattr(cfg, "tiers", 7)
     for bi in range(B):
@@ -499,7 +577,8 @@ def mka_full_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray
         M2, _ = session_ema(Xb[None], cfg.alpha)
         V2 = (M2[0] @ w.w_v).reshape(S, Hkv, dh)
         summ = block_summaries(Xb[None], b)[0]
-        idx, cnt, _, exc, _, _ = longterm_recall(Xb, np.arange(S), summ, w.P, b, R)
+        idx, cnt, _, _, xproj = longterm_recall(Xb, np.arange(S), summ, w.P, b, R)
+        out["x_proj"][bi], out["summary_proj"][bi] = xproj, hash_codes(summ, w.P)[1]
         qr = q[rows].reshape(len(rows), Hq, dh)
         a1 = causal_gqa_attention(qr, rows, K1, V1, Hkv, cfg.scale)
         a2 = V2[rows][:, np.arange(Hq) // G]
@@ -507,6 +586,6 @@ def mka_full_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray
         lr = lam[rows]
         O = lr[:, 0, None, None] * a1 + lr[:, 1, None, None] * a2 + lr[:, 2, None, None] * a3
         out["O"][bi] = O.reshape(len(rows), Hq * dh)
-        out["lam"][bi], out["idx"][bi], out["count"][bi], out["excuse"][bi] = lam, idx, cnt, exc
+        out["lam"][bi], out["idx"][bi], out["count"][bi] = lam, idx, cnt
         out["route_margin"][bi] = route_margin(z, mode, tiers)
     return out

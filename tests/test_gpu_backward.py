@@ -1,8 +1,8 @@
 """GPU parity of the layer backward (mka_prefill_forward_train + mka_prefill_backward) against the
 oracle's float64 backward on the same bf16-rounded inputs and output gradient.
 
-The oracle follows the GPU's recall (recall_fixed): the backward holds the recall fixed, so the
-discrete choice is not under test here (the forward parity tests check it).
+The oracle computes its own recall, and the GPU's recalled indices must equal it bit for bit; the
+backward then holds that recall fixed (straight-through) on both sides.
 
 Tolerance: relative L2 error <= 2e-2 per gradient tensor.  The GPU differentiates its own bf16
 forward (q, K, V, O rounded) with bf16 operands on the tensor cores (P and dS of the attention
@@ -61,11 +61,13 @@ def gpu_backward(cfg, inp, dout):
     return out, {k: v.float().cpu().double().numpy() for k, v in g.items()}, idx.cpu().numpy().astype(np.int64)
 
 
-def oracle_backward(cfg, inp, dout, idx):
+def oracle_backward(cfg, inp, dout, idx_gpu):
+    """The oracle's forward with its own recall, then its backward; the GPU's recall must be the same."""
     X = inp.x[:, :cfg.seq].float().numpy()
     w = oracle_weights(inp)
-    count = (idx >= 0).sum(-1)
-    fwd = oracle.fastmka_prefill(X, w, cfg, keep_d_space=True, recall_fixed=(idx, count))
+    fwd = oracle.fastmka_prefill(X, w, cfg, keep_d_space=True)
+    mism = np.flatnonzero((idx_gpu != fwd["idx"]).any(-1).reshape(-1))
+    assert mism.size == 0, f"{mism.size} tokens recall different blocks on the GPU (first {mism[:8]})"
     return fwd, oracle.fastmka_backward(X, w, cfg, dout.float().numpy().astype(np.float64), fwd)
 
 

@@ -26,12 +26,14 @@ def test_prefill_full_size(name, max_rows):
     torch.cuda.empty_cache()
     ref = oracle_prefill(cfg, inp, rows=rows)
     lam_err = check_lambda(lam_h, ref["lam"])
-    _, excused = check_recall(idx_h, ref)
+    # the GPU decides every hash sign exactly (fp64 where the fp32 value is in doubt): no
+    # mismatch at all, excused or not
+    _, excused = check_recall(idx_h, ref, allow_excused=False)
     max_abs, rel = check_out(out_h, ref["O"], cfg.dtype, rows=rows)
     print(f"{name}: lambda rel {lam_err:.2e}, recall excused {excused}, O rel-L2 {rel:.2e} max-abs {max_abs:.2e}")
 
 
-@pytest.mark.parametrize("ctx", [4096, 32768, 131072])
+@pytest.mark.parametrize("ctx", [4096, 32768, 131072, 262144])
 def test_decode_full_context(ctx):
     """Qwen decode: prefill `ctx` rows into a state, decode 256 tokens; check a sample of them."""
     import route_kv_memory_b200 as mka

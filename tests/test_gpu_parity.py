@@ -94,6 +94,31 @@ def test_attention_rescale_path():
     assert rel_l2 <= BF16_REL_L2 and max_abs <= 1e-2 * np.abs(O16).max(), (rel_l2, max_abs, np.abs(O16).max())
 
 
+def test_attention_rescale_path_layer_tolerance():
+    """The lazy max-shift's rescale path held to the layer's own bf16 bound (rel-L2 <= 1e-2 and
+    max-abs <= 3e-2 against the float64 layer oracle).  A fixed direction u is added to every token
+    with a weight that grows from 0 to 3 along the sequence, so for heads whose (u W_q).(u W_k) is
+    positive the later keys score higher and a row's reference maximum moves after its first tile
+    in more than 500 row-tiles (notes §4, exp(mu_prev - mu_new)).  Scores that grow through a shared
+    direction add terms of one sign, so bf16 rounding of q and K perturbs them far less than scores
+    grown by scaling random inputs; W_v is divided by 3 so the outputs stay near unit size."""
+    import dataclasses
+    cfg = small("bf16_rescale_layer", "bf16", seq=640, n_q_heads=4, n_kv_heads=2, d_head=128, block=64, seed=31)
+    inp = make_inputs(cfg)
+    u = torch.randn(cfg.d_model, generator=torch.Generator().manual_seed(77))
+    ramp = torch.linspace(0.0, 3.0, cfg.seq)
+    inp = dataclasses.replace(inp, x=(inp.x.float() + ramp[None, :, None] * u).to(torch.bfloat16),
+                              w_v=(inp.w_v.float() / 3.0).to(torch.bfloat16))
+    ref = oracle_prefill(cfg, inp)
+    moves = lazy_rescales(ref["q"][0], ref["K"][0], 1.0 / math.sqrt(cfg.d_head))
+    assert moves > 500, moves
+    out, lam, idx, *_ = gpu_prefill(cfg, inp)
+    check_lambda(lam, ref["lam"])
+    check_recall(idx, ref)
+    max_abs, rel = check_out(out, ref["O"], "bf16")
+    print(f"rescale path at the layer tolerance: {moves} moves, rel-L2 {rel:.2e} max-abs {max_abs:.2e}")
+
+
 def test_qwen7b_4k_layer():
     """Qwen2.5-7B-shaped layer, batch 2 x 4096, bf16: lambda and recall on every row, O on a row sample."""
     cfg = CONFIGS["qwen7b_4k"]
@@ -102,7 +127,7 @@ def test_qwen7b_4k_layer():
     ref = oracle_prefill(cfg, inp, rows=rows)
     out, lam, idx, *_ = gpu_prefill(cfg, inp)
     lam_err = check_lambda(lam, ref["lam"])
-    unexc, exc = check_recall(idx, ref)
+    unexc, exc = check_recall(idx, ref, allow_excused=False)
     max_abs, rel = check_out(out, ref["O"], "bf16", rows=rows)
     print(f"qwen7b_4k: lambda rel {lam_err:.2e}, recall excused {exc}, O rel-L2 {rel:.2e} max-abs {max_abs:.2e}")
 
@@ -314,10 +339,14 @@ def test_longterm_recall_entry(mka, dtype):
     P = to_f64(inp.hash_proj)
     for bi in range(cfg.batch):
         summ = oracle.block_summaries(X[bi:bi + 1], cfg.block)[0]
-        ridx, rcnt, rM3, exc, *_ = oracle.longterm_recall(X[bi], np.arange(cfg.seq), summ, P, cfg.block, cfg.recall_r)
+        ridx, rcnt, rM3, _, xproj = oracle.longterm_recall(X[bi], np.arange(cfg.seq), summ, P, cfg.block,
+                                                           cfg.recall_r)
         g = idx[bi].cpu().numpy()
         bad = (g != ridx).any(-1)
-        assert int((bad & ~exc).sum()) == 0
+        sproj = oracle.hash_codes(summ, P)[1]
+        unexcused = [t for t in np.flatnonzero(bad) if not oracle.recall_mismatch_excused(
+            g[t], xproj[t], sproj, t // cfg.block, cfg.recall_r)]
+        assert not unexcused, f"tokens {unexcused[:8]} recall different blocks"
         assert np.array_equal(cnt[bi].cpu().numpy(), rcnt)
         ok = ~bad
         assert np.abs(m3[bi].cpu().double().numpy()[ok] - rM3[ok]).max() <= F32_ATOL

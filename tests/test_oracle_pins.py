@@ -137,7 +137,7 @@ def check_recall_brute_force(recall_fn, b=4, R=3, nb=4, S=60, d=5, seed=7):
     X1 = rng.standard_normal((S, d))
     P = rng.standard_normal((d, nb))
     summ = brute_summaries(X1, b)
-    idx, count, M3, excuse, xcodes, _ = recall_fn(X1, np.arange(S), summ, P, b, R)
+    idx, count, M3, xcodes, _ = recall_fn(X1, np.arange(S), summ, P, b, R)
     scodes = [brute_code(s, P) for s in summ]
     for t in range(S):
         xc = brute_code(X1[t], P)
@@ -181,6 +181,125 @@ def test_recall_special_cases():
     summ_big = O.block_summaries(X1[None], 64)[0]
     _, count, M3, *_ = O.longterm_recall(X1, np.arange(40), summ_big, P, 64, 2)
     assert np.all(count == 0) and np.all(M3 == 0)
+
+
+def brute_reachable_recalls(x_proj_t, s_proj, n_elig, R, eps):
+    """Every recalled list (as a tuple) that some flip of the hash bits with |p| < eps produces,
+    found by enumerating all subsets of those bits (token's and blocks') and sorting by hand."""
+    nb = len(x_proj_t)
+    free = [("t", None, k) for k in range(nb) if abs(x_proj_t[k]) < eps]
+    free += [("s", j, k) for j in range(n_elig) for k in range(nb) if abs(s_proj[j, k]) < eps]
+    out = set()
+    for m in range(1 << len(free)):
+        tb = [x_proj_t[k] > 0 for k in range(nb)]
+        sb = [[s_proj[j, k] > 0 for k in range(nb)] for j in range(n_elig)]
+        for i, (who, j, k) in enumerate(free):
+            if (m >> i) & 1:
+                if who == "t":
+                    tb[k] = not tb[k]
+                else:
+                    sb[j][k] = not sb[j][k]
+        keys = sorted((sum(tb[k] != sb[j][k] for k in range(nb)), j) for j in range(n_elig))
+        out.add(tuple(j for _, j in keys[:R]))
+    return out
+
+
+def check_recall_excuse_exact(excused_fn, seed, nb=4, nblk=7, R=3, n_free=3):
+    """The excuse accepts exactly the lists that a flip of near-zero bits reaches (brute force),
+    for a token with near-zero bits planted at random among its own and the blocks' projections."""
+    rng = np.random.default_rng(seed)
+    eps = 1e-4
+    x = rng.standard_normal(nb)
+    sp = rng.standard_normal((nblk, nb))
+    for _ in range(n_free):                      # plant near-zero components
+        if rng.random() < 0.3:
+            x[rng.integers(nb)] = rng.uniform(-0.9, 0.9) * eps
+        else:
+            sp[rng.integers(nblk), rng.integers(nb)] = rng.uniform(-0.9, 0.9) * eps
+    for n_elig in range(nblk + 1):
+        reach = brute_reachable_recalls(x, sp, n_elig, R, eps)
+        for lst in reach:
+            assert excused_fn(list(lst), x, sp, n_elig, R, eps)
+        cands = set()
+        for _ in range(40):                       # wrong lists: random picks, orders and counts
+            k = min(R, n_elig) if rng.random() < 0.8 else int(rng.integers(0, R + 1))
+            cands.add(tuple(int(j) for j in rng.permutation(max(n_elig, 1))[:k] if j < n_elig))
+        for lst in cands - reach:
+            assert not excused_fn(list(lst), x, sp, n_elig, R, eps), (lst, reach)
+
+
+def test_recall_excuse_matches_brute_force():
+    for seed in range(30):
+        check_recall_excuse_exact(O.recall_mismatch_excused, seed)
+    check_recall_excuse_exact(O.recall_mismatch_excused, 99, nb=6, nblk=9, R=4, n_free=5)
+
+
+def test_recall_excuse_needs_a_deciding_bit():
+    """A near-zero component excuses a mismatch only where it can move the selection."""
+    eps = 1e-4
+    # token code 0000; blocks at distances 0, 1, 2, 4 (block 3's bit 0 projection is near zero)
+    x = np.array([-1.0, -1.0, -1.0, -1.0])
+    sp = np.array([[-1.0, -1.0, -1.0, -1.0],     # d 0
+                   [1.0, -1.0, -1.0, -1.0],      # d 1
+                   [1.0, 1.0, -1.0, -1.0],       # d 2
+                   [0.5 * eps, 1.0, 1.0, 1.0]])  # d 4, bit 0 undecided -> d in {3, 4}
+    assert O.recall_mismatch_excused([0, 1], x, sp, 4, 2)
+    # block 3 is far from the R = 2 cutoff whatever its bit 0: it excuses no other list
+    for wrong in ([0, 2], [1, 0], [0, 3], [1, 2], [0]):
+        assert not O.recall_mismatch_excused(wrong, x, sp, 4, 2)
+    # with R = 3 the cutoff sits at distance 2 vs 3-or-4: still fixed, (2 beats 3)
+    assert not O.recall_mismatch_excused([0, 1, 3], x, sp, 4, 3)
+    # make block 3's distance reach 2 (two undecided bits): now it can tie block 2 at d 2, and wins
+    # only on (distance, index) order if its distance drops below 2 -- it cannot, so [0, 1, 3] stays out
+    sp2 = sp.copy()
+    sp2[3, 1] = -0.5 * eps
+    assert O.recall_mismatch_excused([0, 1, 2], x, sp2, 4, 3)
+    assert not O.recall_mismatch_excused([0, 1, 3], x, sp2, 4, 3)
+    # three undecided bits: block 3 reaches distance 1 and ties block 1, which it loses on the index,
+    # but it beats block 2 (distance 2): [0, 1, 3] becomes reachable, and so does [0, 3, 1]? no: index order
+    sp3 = sp2.copy()
+    sp3[3, 2] = 0.25 * eps
+    assert O.recall_mismatch_excused([0, 1, 3], x, sp3, 4, 3)
+    assert not O.recall_mismatch_excused([0, 3, 1], x, sp3, 4, 3)
+    # a token's own undecided bit moves every block: flipping bit 3 of the token makes block 3 nearer
+    xt = x.copy()
+    xt[3] = 0.1 * eps
+    assert O.recall_mismatch_excused([0, 1], xt, sp, 4, 2)
+    assert not O.recall_mismatch_excused([2, 3], xt, sp, 4, 2)
+
+
+def test_recall_excuse_planted_broad_rule_is_caught():
+    """The broad rule -- excuse a token whenever any eligible block has a near-zero component --
+    would excuse a recall that no flip reaches; the exact rule and brute force both reject it."""
+    eps = 1e-4
+    x = np.array([-1.0, -1.0, -1.0, -1.0])
+    sp = np.array([[-1.0, -1.0, -1.0, -1.0], [1.0, -1.0, -1.0, -1.0], [1.0, 1.0, -1.0, -1.0],
+                   [0.5 * eps, 1.0, 1.0, 1.0]])
+
+    def broad(got, x_proj_t, s_proj, n_elig, R, eps=eps):
+        return bool((np.abs(x_proj_t) < eps).any() or (np.abs(s_proj[:n_elig]) < eps).any())
+
+    assert (1, 0) not in brute_reachable_recalls(x, sp, 4, 2, eps)
+    assert broad([1, 0], x, sp, 4, 2) and not O.recall_mismatch_excused([1, 0], x, sp, 4, 2)
+    with pytest.raises(AssertionError):
+        check_recall_excuse_exact(broad, 0)
+
+
+def test_recall_mismatches_counts():
+    """recall_mismatches counts a mismatch the flip excuses and one it does not."""
+    rng = np.random.default_rng(5)
+    cfg = tiny_cfg(seq=24, block=4, recall_r=2, hash_bits=4)
+    X = rng.standard_normal((1, cfg.seq, cfg.d_model))
+    ref = O.fastmka_prefill(X, tiny_weights(cfg, rng), cfg, rows=np.array([23]))
+    got = ref["idx"].copy()
+    assert O.recall_mismatches(got, ref) == (0, 0, [])
+    t = 20                                       # 5 eligible blocks
+    got[0, t] = got[0, t][::-1]                  # reversed order: no flip reaches it (no bit is near zero)
+    assert O.recall_mismatches(got, ref)[:2] == (1, 0)
+    ref["x_proj"][0, t] = 0.0                    # every token bit undecided: brute force decides
+    reach = brute_reachable_recalls(ref["x_proj"][0, t], ref["summary_proj"][0], 5, 2, O.EXCUSE_EPS)
+    want = (0, 1) if tuple(got[0, t]) in reach else (1, 0)
+    assert O.recall_mismatches(got, ref)[:2] == want
 
 
 def test_hash_bit_order_and_zero():
