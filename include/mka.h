@@ -186,7 +186,9 @@ MKA_API int mka_longterm_recall(const mka_config* cfg, const void* x, const void
  * skip): lambda_out [B*S, 3] float32, recall_idx_out [B, S, R] int32.  When `state`
  * is not NULL (mka_state_init'ed, max_positions >= S), the fused K/V rows, M2[S],
  * the finished block summaries and the unfinished block's partial sums are left in
- * it and its position is set to S, ready for mka_decode_step.
+ * it and its position is set to S, ready for mka_decode_step.  Everything a decode
+ * step reads is rewritten (the codes of blocks not yet finished are zeroed), so a
+ * state that was used before can be refilled without mka_state_init.
  * ws: mka_workspace_size(cfg) bytes, 16-byte aligned (32-byte aligned for full MKA and
  * block-sparse attention, whose partial results are written 32 bytes at a time). */
 MKA_API int mka_prefill_forward(const mka_config* cfg, const void* packed, const void* x, void* out, float* lambda_out,
@@ -225,7 +227,13 @@ MKA_API int mka_prefill_backward(const mka_config* cfg, const void* packed, cons
  * merge), then advances M2, the block sums and the position.  The position lives
  * in device memory, so a sequence of steps can be captured in a CUDA graph.  A
  * step on a full cache records MKA_ERR_CAPACITY in the status word and changes
- * nothing.  ws: mka_decode_workspace_size(cfg, max_positions) bytes. */
+ * nothing.  ws: mka_decode_workspace_size(cfg, max_positions) bytes.
+ * A step whose bounded device-side wait ran out records MKA_ERR_DEVICE_TIMEOUT and
+ * may have applied part of its update: the state's position, cache row and memories
+ * are then unspecified, and the out row too.  Refill the state with
+ * mka_prefill_forward (a prefill into a state redefines all of it) before decoding
+ * on.  The step's grid barrier is reset by the last CTA to leave every launch, so
+ * a timed-out step does not affect the barrier of the next. */
 MKA_API int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size_t state_bytes,
                     int32_t max_positions, const void* x_new, void* out, void* ws, size_t ws_bytes, void* stream);
 
@@ -248,7 +256,10 @@ MKA_API int mka_decode_step(const mka_config* cfg, const void* packed, void* sta
  *     MKA_ERR_WORKSPACE and a message naming both sizes; use mka_session_ema.
  *   - The first call on a device looks up the array's device address with that
  *     device current (cudaGetSymbolAddress) and caches it; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The cache is kept per device index for the life
+ *     of the process: it is not valid after cudaDeviceReset, nor while the calling
+ *     thread has a context other than the device's primary context current (the
+ *     library's image, and so the array, is then loaded at another address).
  *   - All calls share the one array, and each call overwrites what the previous
  *     one left there before reading it.  Calls that overlap on the GPU (on two
  *     streams or from two host threads) race on it: serialise them.
@@ -284,6 +295,22 @@ MKA_API int mka_profile_read(float* ms, int max_stages);
  * up, records MKA_ERR_DEVICE_TIMEOUT in the status word (read it with mka_status) and
  * the kernel returns.  *result (device int) is set to 0, or to 1 if the wait completed. */
 MKA_API int mka_selftest_wait_timeout(int limit_us, int* result, void* stream);
+
+/* Wait classes of mka_set_wait_limit. */
+#define MKA_WAIT_PIPELINE 1 /* mbarrier waits of the TMA / tensor-core pipelines (GEMM, attention) */
+#define MKA_WAIT_GRID 2     /* grid barriers of the cooperative bf16 decode step */
+
+/* Testing aid (not part of the layer; the paper has no counterpart): replaces the
+ * built-in limit (2 s) of every bounded device-side wait of the classes in the mask
+ * wait_classes with limit_ns nanoseconds, on the current device, for the kernels
+ * launched after the call.  limit_ns = 0 restores the built-in limits.  A short
+ * limit makes ordinary waits run out, so a test can drive the production kernels'
+ * timeout path: they record MKA_ERR_DEVICE_TIMEOUT, let their copies and MMAs in
+ * flight finish (drain waits keep their own limits), free their tensor memory and
+ * return, and the context stays usable.  Synchronises the device; call it only
+ * while no work of this library is running on it.  MKA_ERR_INVALID_ARG for an
+ * unknown bit in wait_classes. */
+MKA_API int mka_set_wait_limit(unsigned long long limit_ns, int wait_classes);
 
 /* Library version string. */
 MKA_API const char* mka_version(void);

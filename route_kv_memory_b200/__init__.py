@@ -42,7 +42,7 @@ EXPORTED = [
     "mka_state_init", "mka_router", "mka_session_ema", "mka_longterm_recall", "mka_prefill_forward",
     "mka_decode_step", "mka_status", "mka_last_error", "mka_version", "mka_profile_enable", "mka_profile_read",
     "mka_session_ema_noalloc", "mka_selftest_wait_timeout", "mka_train_workspace_size", "mka_prefill_forward_train",
-    "mka_prefill_backward",
+    "mka_prefill_backward", "mka_set_wait_limit",
 ]
 
 
@@ -87,6 +87,7 @@ _SIGS = {
     "mka_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "mka_session_ema_noalloc": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _vp]),
     "mka_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int, _vp, _vp]),
+    "mka_set_wait_limit": (ctypes.c_int, [ctypes.c_ulonglong, ctypes.c_int]),
     "mka_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -248,6 +249,14 @@ def mka_profile_read(max_stages: int = 16) -> list:
 
 def mka_selftest_wait_timeout(limit_us: int, result: torch.Tensor, stream=None) -> None:
     _check(_lib.mka_selftest_wait_timeout(limit_us, _ptr(result), _stream(stream)), "mka_selftest_wait_timeout")
+
+
+MKA_WAIT_PIPELINE, MKA_WAIT_GRID = 1, 2
+
+
+def mka_set_wait_limit(limit_ns: int, wait_classes: int) -> None:
+    """Testing aid: the limit of the device-side waits of the given classes (0 restores the built-in one)."""
+    _check(_lib.mka_set_wait_limit(limit_ns, wait_classes), "mka_set_wait_limit")
 
 
 def mka_version() -> str:

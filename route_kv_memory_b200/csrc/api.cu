@@ -13,8 +13,9 @@
 
 using namespace mka;
 
-// Device status word: kernels record device-side errors here (never trap).
-__device__ int g_mka_status = 0;
+// Device status block: kernels record device-side errors in word 0 (never trap); words 1-3
+// hold the test-only wait-limit override (see wait_limit in common.cuh).
+__device__ __align__(16) int g_mka_status[4] = {0, 0, 0, 0};
 
 namespace {
 
@@ -214,7 +215,7 @@ StateLayout state_layout(const Dims& d, int Lmax) {
   s.maxblk = Lmax / d.blk;
   size_t o = 0, B = d.B;
   s.pos = o; o += al(B * 4);
-  s.sync = o; o += al(2 * 4);
+  s.sync = o; o += al(3 * 4);
   s.kc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.vc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.ema = o; o += al(B * d.width * 4);
@@ -324,6 +325,17 @@ int mka_selftest_wait_timeout(int limit_us, int* result, void* stream) {
   int* st = status_ptr();
   if (!st) return fail(MKA_ERR_CUDA, "no CUDA device");
   CUDA_TRY(selftest_wait_timeout(limit_us, st, result, (cudaStream_t)stream));
+  return MKA_OK;
+}
+
+int mka_set_wait_limit(unsigned long long limit_ns, int wait_classes) {
+  if (wait_classes & ~(MKA_WAIT_PIPELINE | MKA_WAIT_GRID))
+    return fail(MKA_ERR_INVALID_ARG, "wait_classes must be a mask of MKA_WAIT_PIPELINE and MKA_WAIT_GRID");
+  int* st = status_ptr();
+  if (!st) return fail(MKA_ERR_CUDA, "no CUDA device");
+  int words[3] = {limit_ns ? wait_classes : 0, (int)(limit_ns & 0xffffffffull), (int)(limit_ns >> 32)};
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpy(st + 1, words, sizeof(words), cudaMemcpyHostToDevice));
   return MKA_OK;
 }
 
@@ -620,6 +632,10 @@ static int prefill_forward(const mka_config* cfg, const void* packed, const void
     return prefill_tail_state(xkv, d.width, d.width, x, d.bf16, d.d, d.B, d.S, d.blk, (float*)P(state, SL.blk_sum),
                               (double*)P(state, SL.blk_x), (int*)P(state, SL.pos), st);
   };
+  // A decode step ORs the bits of a block's code in when the block closes: the codes of the
+  // blocks this prefill does not finish start at zero, so a prefill redefines the whole state.
+  if (state && SL.maxblk > d.nblk)
+    CUDA_TRY(cudaMemset2DAsync(scode + d.nblk, (size_t)SL.maxblk * 4, 0, (size_t)(SL.maxblk - d.nblk) * 4, d.B, s));
   std::unique_lock<std::mutex> aux_lock(aux_mutex(), std::defer_lock);
   AuxStreams* ax = nullptr;
   if (!g_prof.on) {

@@ -19,6 +19,19 @@ __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// The status block every kernel receives (16 bytes, 16-byte aligned): word 0 is the device
+// status code above; word 1 a mask of the wait classes that take the limit in words 2-3 (an
+// unsigned 64-bit count of nanoseconds; 0 = none) in place of their built-in limit.  Only the
+// host writes words 1-3, and only while no kernel of the library runs.
+constexpr int kWaitPipeline = 1;  // mbarrier waits of the TMA / tensor-core pipelines
+constexpr int kWaitGrid = 2;      // grid barriers of the cooperative decode step
+__device__ __forceinline__ unsigned long long wait_limit(const int* status, int wait_class,
+                                                         unsigned long long builtin_ns) {
+  if (!status || !(status[1] & wait_class)) return builtin_ns;
+  const unsigned long long o = *(const unsigned long long*)(status + 2);
+  return o ? o : builtin_ns;
+}
+
 template <typename T> __device__ __forceinline__ float to_f(T v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f<bf16>(bf16 v) { return __bfloat162float(v); }

@@ -711,7 +711,9 @@ __device__ void token_slice(const DecodeArgs& a, const int bi, const int pos, co
 //      term (its score against the appended K row, weight on the appended V row)
 // The two barriers are counters in the decode state, each wait bounded by a time
 // limit that records MKA_ERR_DEVICE_TIMEOUT.  All CTAs are co-resident
-// (cooperative launch), so the barrier cannot deadlock on scheduling.
+// (cooperative launch), so the barrier cannot deadlock on scheduling.  A CTA whose
+// wait ran out leaves the step; every CTA counts itself out on the way, and the
+// last to leave clears the barrier's arrival count for the next launch.
 constexpr int kFusedRing = 2 * 2 * dk::NWD * dk::TP * 128 * 2;  // 64 KB: GEMV chunks, then K/V tiles
 static_assert(kFusedRing >= dk::NWD * 16 * 128 * 4, "attention merge scratch must fit the ring");
 
@@ -728,8 +730,9 @@ __device__ bool grid_sync(unsigned* count, unsigned* gen, unsigned nblocks, int*
       atomicAdd(gen, 1u);
     } else {
       const unsigned long long t0 = sm100::globaltimer();
+      const unsigned long long lim = wait_limit(status, kWaitGrid, sm100::kWaitLimitNs);
       while (*(volatile unsigned*)gen == g) {
-        if (sm100::globaltimer() - t0 > sm100::kWaitLimitNs) {
+        if (sm100::globaltimer() - t0 > lim) {
           set_status(status, kStatusTimeout);
           s_ok = 0;
           break;
@@ -741,6 +744,22 @@ __device__ bool grid_sync(unsigned* count, unsigned* gen, unsigned nblocks, int*
   }
   __syncthreads();
   return s_ok != 0;
+}
+
+// Every CTA of a fused decode launch leaves through here, after its last use of the grid
+// barrier (sync[0] arrivals, sync[1] generation, sync[2] CTAs gone).  The last CTA to leave
+// zeroes the arrival count: a step in which some CTAs gave up on a barrier leaves arrivals
+// counted, and the next launch would otherwise pass its first barrier early.
+__device__ void grid_exit(unsigned* sync, unsigned nblocks) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(sync + 2, 1u) == nblocks - 1) {
+      atomicExch(sync, 0u);
+      atomicExch(sync + 2, 0u);
+      __threadfence();
+    }
+  }
 }
 
 __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -820,7 +839,7 @@ __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, cons
 }
 
 template <int DH>
-__global__ void __launch_bounds__(dk::NWD * 32, 2) decode_fused_kernel(DecodeArgs a) {
+__device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
   bf16* sx = (bf16*)(smem + kFusedRing);
@@ -856,11 +875,25 @@ __global__ void __launch_bounds__(dk::NWD * 32, 2) decode_fused_kernel(DecodeArg
           bulk_copy(dst + (size_t)(r - ra) * row_bytes, W + (size_t)r * a.d, (uint32_t)row_bytes, &gbar[c & 1]);
       }
     };
-    volatile int abort_flag = 0;
+    __shared__ int abort_flag;
+    if (tid == 0) abort_flag = 0;
+    __syncthreads();
     if (nch > 0) issue(0);
     for (int c = 0; c < nch; ++c) {
       if (c + 1 < nch) issue(c + 1);
-      if (!sm100::mbar_wait(&gbar[c & 1], (c >> 1) & 1, &abort_flag, a.status)) return;
+      const bool ok = sm100::mbar_wait(&gbar[c & 1], (c >> 1) & 1, (volatile int*)&abort_flag, a.status);
+      // one decision for the whole CTA (a wait that ran out raised abort_flag for the others);
+      // before leaving, let the copies in flight (chunks c and c + 1) land, within a fixed bound
+      if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+          const unsigned long long t0 = sm100::globaltimer();
+          for (int cc = c; cc < min(c + 2, nch); ++cc)
+            while (!sm100::mbar_try_wait(&gbar[cc & 1], (cc >> 1) & 1) && sm100::globaltimer() - t0 < 100000000ull) {
+            }
+        }
+        __syncthreads();
+        return;
+      }
       const int ra = r0 + c * CR, rb = min(r1, ra + CR);
       const bf16* wst = (const bf16*)(ring + (size_t)(c & 1) * CR * row_bytes);
       for (int r = ra + warp; r < rb; r += NW) {
@@ -961,6 +994,12 @@ __global__ void __launch_bounds__(dk::NWD * 32, 2) decode_fused_kernel(DecodeArg
       }
     }
   }
+}
+
+template <int DH>
+__global__ void __launch_bounds__(dk::NWD * 32, 2) decode_fused_kernel(DecodeArgs a) {
+  decode_fused_body<DH>(a);
+  grid_exit(a.sync, gridDim.x);
 }
 
 size_t decode_fused_smem(int B, int d) { return kFusedRing + (((size_t)B * d * 2 + 15) & ~(size_t)15) + 64; }

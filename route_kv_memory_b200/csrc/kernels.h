@@ -242,7 +242,7 @@ struct DecodeArgs {
   float* qf;                     // [B, dq] float32 query
   float* part;                   // split-KV partials
   int nsplit;
-  unsigned* sync;                // 2 words in the decode state: grid-barrier count and generation
+  unsigned* sync;                // 3 words in the decode state: grid-barrier count, generation, CTAs gone
   int* status;
   cudaEvent_t* prof;             // 5 events around the 4 stages, or NULL
 };

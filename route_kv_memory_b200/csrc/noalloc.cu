@@ -24,7 +24,9 @@ __device__ __align__(256) unsigned char g_ema_scratch[MKA_NOALLOC_SCRATCH_BYTES]
 
 // Host code may not use g_ema_scratch as a device address (in host code the
 // name is a host-side stand-in).  Its device address is looked up once per
-// device, with that device current, and cached.
+// device, with that device current, and cached.  The address belongs to the
+// device's primary context: the cache does not follow cudaDeviceReset or a
+// non-primary context, which load the image again elsewhere.
 void* scratch_address(int* err) {
   static std::mutex mu;
   static void* addr[64] = {};

@@ -46,21 +46,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Waits for the phase of `bar` with the given parity.  Returns false (and the
 // kernel must unwind) when another role of the CTA raised *abort, or when the
-// wait ran past kWaitLimitNs, in which case it raises *abort and records the
-// timeout in the status word.
+// wait ran past its limit (limit_ns, or the pipeline-wait limit set in the
+// status block), in which case it raises *abort and records the timeout in the
+// status word.  Limits shorter than the built-in one are checked on every poll.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
                                           unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
+  const unsigned long long lim = wait_limit(status, kWaitPipeline, limit_ns);
+  const uint32_t every = lim < kWaitLimitNs ? 0u : 31u;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0u) {
+    if ((i & every) == 0u) {
       if (*abort) return false;
-      if (globaltimer() - t0 > limit_ns) {
+      if (globaltimer() - t0 > lim) {
         *abort = 1;
         set_status(status, kStatusTimeout);
         return false;
       }
+    }
+  }
+}
+
+// End of a CTA in which some role raised *abort.  A consumer can give up after the loader has
+// issued its last copies, so copies may still be landing in this CTA's shared memory: the CTA
+// stays resident for a fixed bound (far above any copy's latency) before it exits.  Called by
+// one thread after the CTA's final barrier, by which every role that gave up has raised *abort.
+constexpr unsigned long long kDrainNs = 50000000ull;
+__device__ __forceinline__ void linger_after_abort(volatile int* abort) {
+  if (*abort) {
+    const unsigned long long t0 = globaltimer();
+    while (globaltimer() - t0 < kDrainNs) {
     }
   }
 }

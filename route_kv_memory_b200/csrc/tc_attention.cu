@@ -288,11 +288,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         w = snake_item(rr + 1, gridDim.x, blockIdx.x, nwork);
         if (w >= 0) lookup(w);
       }
-      if (lane == 0 && *abort) {  // let issued copies land (bounded) before unwinding
-        const unsigned long long t0 = globaltimer();
-        while (globaltimer() - t0 < 50000000ull) {
-        }
-      }
     } else if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -333,11 +328,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         if (!ok) break;
-      }
-      if (*abort) {  // let issued copies land (bounded) before unwinding
-        const unsigned long long t0 = globaltimer();
-        while (globaltimer() - t0 < 50000000ull) {
-        }
       }
     }
   } else if (warp == 1) {
@@ -658,6 +648,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
+    if (lane == 0) linger_after_abort(abort);  // copies issued before a role gave up land first
   }
 #undef O_COL
 #undef S_COL

@@ -180,11 +180,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_2d(sV + vs * C::TILE + hb * C::HALF, &tmV, &v_full[vs], (h / G) * DH + hb * 64, b * a.S + j * BT);
         }
       }
-      if (*abort) {
-        const unsigned long long t0 = globaltimer();
-        while (globaltimer() - t0 < 50000000ull) {
-        }
-      }
     }
   } else if (warp == 1) {  // the whole warp runs the MMA role; one elected lane issues
     const uint64_t qd = sdesc_kmajor_sw128(sQ), dod = sdesc_kmajor_sw128(sdO);
@@ -373,6 +368,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
+    if (lane == 0) linger_after_abort(abort);  // copies issued before a role gave up land first
   }
 }
 
@@ -489,11 +485,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_expect_tx(&do_full[st], C::TILE);
           for (int hb = 0; hb < C::NH; ++hb)
             tma_load_2d(sdO + st * C::TILE + hb * C::HALF, &tmdO, &do_full[st], h * DH + hb * 64, b * a.S + qt * BT);
-        }
-      }
-      if (*abort) {
-        const unsigned long long t0 = globaltimer();
-        while (globaltimer() - t0 < 50000000ull) {
         }
       }
     }
@@ -718,6 +709,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
+    if (lane == 0) linger_after_abort(abort);  // copies issued before a role gave up land first
   }
 }
 

@@ -281,6 +281,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
+    if (lane == 0) linger_after_abort(abort);  // copies issued before a role gave up land first
   }
 }
 

@@ -148,3 +148,9 @@ def test_product_path_has_no_fallback():
     src = open(os.path.join(ROOT, "route_kv_memory_b200", "__init__.py")).read()
     assert "oracle" not in src.replace("no CPU fallback", "")
     assert "raise ImportError" in src
+
+
+def test_set_wait_limit_rejects_unknown_classes_on_the_host(mka):
+    """The testing aid checks its mask before it touches a device."""
+    assert mka._lib.mka_set_wait_limit(1000, 4) == mka.MKA_ERR_INVALID_ARG
+    assert b"wait_classes" in mka._lib.mka_last_error()

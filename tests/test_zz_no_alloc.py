@@ -50,6 +50,32 @@ def test_noalloc_matches_caller_scratch_on_two_calls(dtype):
         assert np.abs((out - ref_out).cpu().numpy()).max() <= ATOL, f"call {call}"
 
 
+@pytest.mark.parametrize("seq,with_carry", [(40, True), (300, False), (40, False)])
+def test_noalloc_short_sequences_and_no_carries(seq, with_carry):
+    """Sequences shorter than one 64-row chunk (no chunk end states) and calls without carry_in /
+    carry_out, against mka_session_ema on the same arguments."""
+    import route_kv_memory_b200 as mka
+    cfg = _cfg("f32", seq, 80 + seq)
+    inp = make_inputs(cfg)
+    c = mka.make_config(cfg)
+    x = inp.x.cuda()
+    cin = torch.randn(cfg.batch, cfg.d_model, generator=torch.Generator().manual_seed(seq)).cuda() if with_carry else None
+    ref_m2 = torch.empty(cfg.batch, seq, cfg.d_model, device="cuda")
+    ref_out = torch.empty(cfg.batch, cfg.d_model, device="cuda") if with_carry else None
+    ws = mka.buffer(mka.mka_session_ema_workspace_size(c))
+    mka.mka_session_ema(c, x, cin, ref_m2, ref_out, ws)
+    m2 = torch.full_like(ref_m2, float("nan"))
+    out = torch.full_like(ref_out, float("nan")) if with_carry else None
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None
+    rc = mka._lib.mka_session_ema_noalloc(ctypes.byref(c), ptr(x), ptr(cin), ptr(m2), ptr(out),
+                                           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == mka.MKA_OK, mka._lib.mka_last_error()
+    torch.cuda.synchronize()
+    assert np.abs((m2 - ref_m2).cpu().numpy()).max() <= ATOL
+    if with_carry:
+        assert np.abs((out - ref_out).cpu().numpy()).max() <= ATOL
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     import route_kv_memory_b200 as mka
     cfg = FastMKAConfig("big", 4, 65536, 4096, 32, 8, 128, 256, 0.99, 256, 16, 32, "bf16", 0)
