@@ -1,14 +1,17 @@
 #!/usr/bin/env python
 """FastMKA layer benchmark on B200.
 
-Headline: prefill tokens/s of the Qwen2.5-7B-shaped FastMKA layer (batch 2 x
-seq 4096, bf16; every step runs the whole layer: projections, router, L2 EMA,
-L3 hash recall, route-fuse, causal GQA attention).  Also reported: decode
-us/token over a 131072-position fused cache (256 steps in one CUDA graph), the
-roofline fraction of the dominant kernel (measured live with CUDA events on the
-launching stream), the end-to-end rate through host buffers, and the CPU oracle.
+Headline: prefill tokens/s of the Llama-3.1-8B-shaped FastMKA layer (batch 1 x
+seq 131072, bf16; every step runs the whole layer: projections, router, L2 EMA,
+L3 hash recall, route-fuse, causal GQA attention), the largest workload that
+fits one GPU.  Alongside it: the same measurement for the smaller prefill
+workloads (by_workload), decode us/token over fused caches of 4K-256K positions
+(256 steps in one CUDA graph), the roofline fraction of the attention and the
+HBM fraction of every bandwidth-bound stage (measured live with CUDA events on
+the launching stream), the end-to-end rate through host buffers, the recalled
+blocks checked against the CPU oracle, and the CPU oracle's own rate.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 With N > 1 (torchrun, one rank per GPU) every rank runs an independent replica
 of the workload (the layer shards by sequence with no exchange): weak scaling.
@@ -145,12 +148,83 @@ def prefill_kernels(cfg) -> int:
     return 10
 
 
-# ------------------------------------------------------------------ our arm
-def run_ours(args, rank, world, local_rank):
+FFMA_LANES_PER_SM = 128  # fp32 FMA lanes of an sm_100 SM (4 SMSPs x 32)
+
+
+def ffma_peak_tflops(sm_max_mhz: float = 1965.0, sms: int = 148) -> float:
+    """Dense fp32 FFMA peak: SMs x FMA lanes x 2 flops x the maximum SM clock."""
+    return sms * FFMA_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+
+
+def prefill_hbm_bytes(cfg) -> dict:
+    """Algorithmic DRAM bytes per prefill call of each bandwidth-bound stage (each input read once,
+    each output written once; workspace tensors the GEMM wrote count as reads)."""
+    T, d, W, nb, R = cfg.tokens, cfg.d_model, 2 * cfg.dkv, cfg.hash_bits, cfg.recall_r
+    elem = 4 if cfg.dtype == "f32" else 2
+    nblk = cfg.batch * (cfg.seq // cfg.block)
+    rh_parts = max(1, cfg.router_hidden // 128)
+    return {
+        "router_tail": T * rh_parts * 3 * 4 + T * 3 * 4,
+        "token_codes": T * nb * 4 + T * 4,
+        "block_sums": T * W * 4 + nblk * 9 * W * 4,
+        "block_codes": T * d * elem + nblk * 4,
+        "recall": T * 4 + nblk * 4 + T * (R + 1) * 4,
+        "route_fuse": T * W * 4 + T * 3 * 4 + T * R * 4 + nblk * W * 4 + T * W * elem,
+    }
+
+
+def workload_config(cfg, world: int) -> dict:
+    """The `config` object of the JSON line, the same for both arms."""
+    return {"workload": f"{cfg.name}: {model_name(cfg)}-shaped FastMKA layer prefill, batch {cfg.batch} x seq "
+                        f"{cfg.seq}, d_model {cfg.d_model}, {cfg.n_q_heads}/{cfg.n_kv_heads} heads, d_h "
+                        f"{cfg.d_head}, router {cfg.dq}->{cfg.router_hidden}->3, alpha {cfg.alpha}, L3 block "
+                        f"{cfg.block}, R {cfg.recall_r}, nbits {cfg.hash_bits}, {cfg.dtype}, seed {cfg.seed}"
+                        + ("" if (cfg.route_mode, cfg.tiers) == ("soft", 7) else
+                           f"; routing {cfg.route_mode}, tiers mask {cfg.tiers}")
+                        + ("; full MKA, three attention paths" if cfg.attention_paths == 3 else "")
+                        + ("; Block-MKA block-sparse attention" if cfg.block_sparse else ""),
+            "global_batch": cfg.batch * world, "seq_len": cfg.seq,
+            "parallelism": f"replicas x{world} (independent sequences, no exchange)",
+            "l2": "flushed (512 MB write) before every timed step"}
+
+
+def attention_roofline(cfg, attn_ms: float, peaks: dict, clk_max_mhz: float = 1965.0) -> dict:
+    fl = prefill_flops(cfg)["attention"]
+    tf = fl / (attn_ms / 1e3) / 1e12
+    kernel = (("attention (Block-MKA block-sparse: own block + recalled blocks)" if cfg.block_sparse else
+               "attention (causal GQA, online max-shift)") if cfg.attention_paths == 1 else
+              "attention (full MKA: causal pass + recalled-block pass)")
+    if cfg.dtype == "f32":
+        peak = ffma_peak_tflops(clk_max_mhz)
+        return {"kernel": kernel + ", fp32 FFMA", "bound": "alu", "achieved": round(tf, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+                "peak_source": f"derived: 148 SMs x {FFMA_LANES_PER_SM} FP32 lanes x 2 x {clk_max_mhz:.0f} MHz",
+                "traffic": None, "avg_ms": round(attn_ms, 4), "flops_per_launch": fl}
+    return {"kernel": kernel, "bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+            "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)",
+            "traffic": traffic_from_profiles("attention_tc"), "avg_ms": round(attn_ms, 4), "flops_per_launch": fl}
+
+
+def hbm_rooflines(cfg, stage_ms: dict, peaks: dict) -> dict:
+    """GB/s and fraction of the measured HBM copy bandwidth of each bandwidth-bound stage, from its
+    algorithmic bytes and its own CUDA-event time (stages run one after another when timed)."""
+    out = {}
+    for k, b in prefill_hbm_bytes(cfg).items():
+        ms = stage_ms.get(k)
+        if not ms:
+            continue
+        gbs = b / (ms / 1e3) / 1e9
+        out[k] = {"bytes": int(b), "ms": round(ms, 4), "achieved": round(gbs, 1), "unit": "GB/s",
+                  "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    return {"peak": peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy bandwidth", "kernels": out}
+
+
+def measure_prefill(args, cfg, dev, world, steps, warmup, with_e2e=False, with_clocks=False):
+    """Prefill tokens/s of one workload: `warmup` untimed calls, stage times from profiled calls
+    (every stage alone on the caller's stream), then `steps` timed calls with L2 flushed before
+    each (device time by CUDA events, independent memory kernels as concurrent branches)."""
     import route_kv_memory_b200 as mka
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    cfg = workload_cfg(args, args.workload)
     inp = make_inputs(cfg)
     weights = {k: v.to(dev) for k, v in inp.tensors().items() if k != "x"}
     layer = mka.FastMKALayer(cfg, weights, dev)
@@ -159,67 +233,78 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     stream = torch.cuda.current_stream()
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         layer.prefill(x, out)
     torch.cuda.synchronize()
     assert mka.mka_status() == 0
 
-    # ---- stage breakdown: profiled calls, in which the library runs every stage on the
-    # caller's stream one after another (outside the timed region)
     stage_ms = []
     mka.mka_profile_enable(True)
-    for i in range(min(args.steps, 10)):
+    for i in range(min(steps, 10)):
         flush.zero_()
         layer.prefill(x, out)
         stage_ms.append(mka.mka_profile_read())
     mka.mka_profile_enable(False)
     torch.cuda.synchronize()
-    stages = np.array(stage_ms).mean(axis=0)
+    stages = {n: float(v) for n, v in zip(PREFILL_STAGES, np.array(stage_ms).mean(axis=0))}
 
-    # ---- timed region: K prefill steps, L2 flushed before each, device time by CUDA events;
-    # profiling off, so the independent memory kernels run as concurrent branches
-    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        for i in range(args.steps):
-            flush.zero_()
-            ev0[i].record(stream)
-            layer.prefill(x, out)
-            ev1[i].record(stream)
-        torch.cuda.synchronize()
+    clk = ClockSampler(dev.index or 0) if with_clocks else None
+    if clk:
+        clk.__enter__()
+    for i in range(steps):
+        flush.zero_()
+        ev0[i].record(stream)
+        layer.prefill(x, out)
+        ev1[i].record(stream)
+    torch.cuda.synchronize()
+    if clk:
+        clk.__exit__()
     barrier(world)
+    assert mka.mka_status() == 0
     step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     value, ms = job_throughput(cfg.tokens, statistics.mean(step_ms), world)
-    launches_per_step = prefill_kernels(cfg)
 
     peaks = load_peaks()
     fl = prefill_flops(cfg)
-    attn_ms = float(stages[8])
-    attn_tflops = fl["attention"] / (attn_ms / 1e3) / 1e12
-    roofline = {"kernel": ("attention (Block-MKA block-sparse: own block + recalled blocks)" if cfg.block_sparse else
-                           "attention (causal GQA, online max-shift)") if cfg.attention_paths == 1 else
-                "attention (full MKA: causal pass + recalled-block pass)", "bound": "tensor",
-                "achieved": round(attn_tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
-                "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)",
-                "traffic": traffic_from_profiles("attention_tc"), "avg_ms": round(attn_ms, 4),
-                "flops_per_launch": fl["attention"]}
-    layer_tflops = (fl["projections"] + fl["attention"]) / (ms / 1e3) / 1e12
+    res = {"value": round(value, 1), "unit": "tokens/s", "ms_per_step": round(ms, 4), "steps": steps,
+           "roofline": attention_roofline(cfg, stages["attention"], peaks),
+           "hbm": hbm_rooflines(cfg, stages, peaks),
+           "layer_tflops": round((fl["projections"] + fl["attention"]) / (ms / 1e3) / 1e12, 1),
+           "stage_ms": {n: round(v, 4) for n, v in stages.items()},
+           "gpu_launches": prefill_kernels(cfg) * steps}
+    if clk:
+        res["clocks"] = clk.summary()
+    if with_e2e:
+        res["e2e"] = measure_e2e(layer, inp, cfg, x, out, flush, world, max(4, steps // 4))
+    res["_recall_gpu"] = None
+    if getattr(args, "recall_check", True) and cfg.tiers & 4 and cfg.attention_paths == 1:
+        idx = torch.empty(cfg.batch, cfg.seq, cfg.recall_r, dtype=torch.int32, device=dev)
+        layer.prefill(x, out, None, idx)
+        torch.cuda.synchronize()
+        assert mka.mka_status() == 0
+        res["_recall_gpu"] = idx.cpu().numpy().astype(np.int64)
+    del layer, x, out, flush, weights
+    torch.cuda.empty_cache()
+    return res, inp
 
-    # ---- end to end through host buffers (pinned): every step copies its X in (H2D), runs the
-    # layer and copies its O out (D2H), all inside the timed region.  Steps are pipelined the way
-    # a serving loop streams batches: three streams and double-buffered device X / O, so the
-    # copy-in of step i+1 and the copy-out of step i-1 (separate copy engines, full-duplex PCIe)
-    # overlap the layer of step i.  L2 is flushed before every layer call, as in the timed loop.
-    n_e2e = max(4, args.steps // 4)
+
+def measure_e2e(layer, inp, cfg, x, out, flush, world, n_e2e):
+    """End to end through host buffers (pinned): every step copies its X in (H2D), runs the layer and
+    copies its O out (D2H), all inside the timed region.  Steps are pipelined the way a serving loop
+    streams batches: three streams and double-buffered device X / O, so the copy-in of step i+1 and the
+    copy-out of step i-1 (separate copy engines, full-duplex PCIe) overlap the layer of step i.  L2 is
+    flushed before every layer call, as in the timed loop."""
+    dev = x.device
     x_host = inp.x[:, :cfg.seq].contiguous().pin_memory()
     o_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     xb, ob = [x, torch.empty_like(x)], [out, torch.empty_like(out)]
     s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_run(n, timed):
+    def e2e_run(n):
         ev_in = [torch.cuda.Event() for _ in range(n)]
         ev_cmp = [torch.cuda.Event() for _ in range(n)]
         ev_out = [torch.cuda.Event() for _ in range(n)]
@@ -248,44 +333,54 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         return t0.elapsed_time(t1) / n
 
-    e2e_run(3, False)
-    e2e_value, e2e_ms = job_throughput(cfg.tokens, e2e_run(n_e2e, True), world)
-    e2e = {"value": e2e_value, "unit": "tokens/s",
-           "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-           "d2h_bytes_per_step": o_host[0].numel() * o_host[0].element_size(), "ms_per_step": round(e2e_ms, 4),
-           "steps": n_e2e,
-           "how": "pinned host X -> device, layer, device O -> pinned host, every step; steps pipelined over "
-                  "copy-in / compute / copy-out streams with double-buffered device X and O"}
-    del x_host, o_host, xb, ob
+    e2e_run(3)
+    e2e_value, e2e_ms = job_throughput(cfg.tokens, e2e_run(n_e2e), world)
+    return {"value": round(e2e_value, 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": o_host[0].numel() * o_host[0].element_size(), "ms_per_step": round(e2e_ms, 4),
+            "steps": n_e2e,
+            "how": "pinned host X -> device, layer, device O -> pinned host, every step; steps pipelined over "
+                   "copy-in / compute / copy-out streams with double-buffered device X and O"}
 
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = workload_cfg(args, args.workload)
+    head, inp = measure_prefill(args, cfg, dev, world, args.steps, args.warmup, with_e2e=True, with_clocks=True)
+    recall_gpu = head.pop("_recall_gpu")
     result = {
         "metric": "FastMKA layer prefill tokens/s (decode us/token and roofline fraction alongside)",
-        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded N(0,1) inputs, N(0,1/d_in) weights)",
-        "config": {"workload": f"{cfg.name}: {model_name(cfg)}-shaped FastMKA layer prefill, batch {cfg.batch} x seq "
-                               f"{cfg.seq}, d_model {cfg.d_model}, {cfg.n_q_heads}/{cfg.n_kv_heads} heads, d_h "
-                               f"{cfg.d_head}, router {cfg.dq}->{cfg.router_hidden}->3, alpha {cfg.alpha}, L3 block "
-                               f"{cfg.block}, R {cfg.recall_r}, nbits {cfg.hash_bits}, seed {cfg.seed}"
-                               + ("" if (cfg.route_mode, cfg.tiers) == ("soft", 7) else
-                                  f"; routing {cfg.route_mode}, tiers mask {cfg.tiers}")
-                               + ("; full MKA, three attention paths" if cfg.attention_paths == 3 else "")
-                               + ("; Block-MKA block-sparse attention" if cfg.block_sparse else ""),
-                   "global_batch": cfg.batch * world, "seq_len": cfg.seq,
-                   "parallelism": f"replicas x{world} (independent sequences, no exchange)",
-                   "l2": "flushed (512 MB write) before every timed step"},
-        "roofline": roofline,
-        "layer_tflops": round(layer_tflops, 1),
-        "stage_ms": {n: round(float(v), 4) for n, v in zip(PREFILL_STAGES, stages)},
-        "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": cfg.dtype, "data": "synthetic (seeded N(0,1) inputs, N(0,1/d_in) weights)",
+        "config": workload_config(cfg, world),
+        "roofline": head["roofline"],
+        "hbm_roofline": head["hbm"],
+        "layer_tflops": head["layer_tflops"],
+        "stage_ms": head["stage_ms"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
     }
-    del flush
+    others = [w for w in args.by_workload if w != cfg.name]
+    if others:
+        result["by_workload"] = {}
+        for name in others:
+            c = workload_cfg(args, name)
+            r, _ = measure_prefill(args, c, dev, world, min(args.steps, 20), args.warmup)
+            rec = r.pop("_recall_gpu")
+            if rank == 0 and world == 1 and not args.no_cpu_baseline and rec is not None:
+                r["recall"] = recall_check(c, make_inputs(c), rec)
+            r["config"] = workload_config(c, world)["workload"]
+            result["by_workload"][name] = r
     if world == 1 and not args.no_decode and args.paths == 1 and not args.block_sparse:  # prefill-only variants
-        result["decode"] = run_decode(args, cfg, inp, weights, dev, layer_pack=None)
+        result["decode"] = run_decode(args, cfg, None, None, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(cfg, inp, budget_rows=args.cpu_rows)
+        result["cpu_baseline"] = cpu_baseline(cfg, inp, prefix_tokens=args.cpu_prefix, attn_rows=args.cpu_rows)
+        if recall_gpu is not None:
+            result["recall"] = recall_check(cfg, inp, recall_gpu)
     return result
 
 
@@ -495,15 +590,20 @@ def run_decode(args, cfg_prefill, inp_unused, weights_unused, dev, layer_pack=No
 
 
 # ------------------------------------------------------------------ CPU oracle
-def cpu_baseline(cfg, inp, budget_rows=48):
-    """The oracle as it stands on this host's cores: all linear parts of the layer for every token, the
-    attention for a strided row sample, extrapolated to all rows by the causal pair count."""
+def cpu_baseline(cfg, inp, prefix_tokens=8192, attn_rows=32):
+    """The oracle as it stands on this host's cores, on a bounded sample of the workload: the whole
+    layer over the first rows of every sequence (prefix_tokens in all; causality makes those rows
+    exactly the full layer's first rows) with the attention on a strided sample of them, then
+    extrapolated to the full workload: the linear parts (projections, router, EMA, L3, fuse, K/V)
+    by token count, the attention by causal pair count."""
     import oracle
-    X = inp.x[:, :cfg.seq].float().numpy()
+    P = max(cfg.block, min(cfg.seq, prefix_tokens // cfg.batch))
+    c = cfg.replace(seq=P)
+    X = inp.x[:, :P].float().numpy()
     w = oracle.weights_f64(*(to_f64(t) for t in (inp.w_q, inp.w_k, inp.w_v, inp.w_r1, inp.w_r2, inp.hash_proj)))
-    rows = sample_rows(cfg.seq, cfg.block, max_rows=budget_rows)
+    rows = sample_rows(P, cfg.block, max_rows=attn_rows)
     t0 = time.perf_counter()
-    out = oracle.fastmka_prefill(X, w, cfg, rows=rows)
+    out = oracle.fastmka_prefill(X, w, c, rows=rows)
     t_total = time.perf_counter() - t0
     t1 = time.perf_counter()
     for bi in range(cfg.batch):
@@ -512,13 +612,49 @@ def cpu_baseline(cfg, inp, budget_rows=48):
     t_lin = max(t_total - t_attn, 0.0)
     pairs_all = cfg.seq * (cfg.seq + 1) / 2
     pairs_sample = float(np.sum(rows + 1))
-    t_full = t_lin + t_attn * pairs_all / pairs_sample
+    t_full = t_lin * cfg.seq / P + t_attn * pairs_all / pairs_sample
     cores = len(os.sched_getaffinity(0))
-    return {"value": round(cfg.tokens / t_full, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"float64 NumPy oracle, {cfg.name}: projections/router/EMA/L3/fuse/K,V for all "
-                      f"{cfg.tokens} tokens ({t_lin:.1f} s) + attention for {len(rows)} strided query rows per "
-                      f"sequence ({t_attn:.1f} s), extrapolated by causal pair count to {t_full:.1f} s per layer",
+    return {"value": round(cfg.tokens / t_full, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "value_is": "extrapolated from the measured sample to the whole workload",
+            "sample": f"float64 NumPy oracle, {cfg.name}: the layer over the first {P} rows of each of {cfg.batch} "
+                      f"sequence(s) ({t_lin:.2f} s for projections/router/EMA/L3/fuse/K,V) with the attention on "
+                      f"{len(rows)} strided rows per sequence ({t_attn:.2f} s); extrapolated by token count "
+                      f"(x{cfg.seq / P:.0f}) and causal pair count (x{pairs_all / pairs_sample:.0f}) to "
+                      f"{t_full:.0f} s per layer",
             "measured_s": round(t_total, 2)}
+
+
+def recall_check(cfg, inp, idx_gpu, max_rows=16384):
+    """The GPU's recalled block indices against the oracle's L3 recall on the same inputs: every
+    row for workloads up to max_rows tokens per sequence, else a strided row sample.  A mismatch is
+    excused only where the GPU's list is the recall under a flip of hash bits within 1e-4 of zero."""
+    import oracle
+    P = to_f64(inp.hash_proj)
+    S, b = cfg.seq, cfg.block
+    stride = max(1, -(-S // max_rows))
+    rows = np.arange(0, S, stride)
+    nblk = S // b
+    t0 = time.perf_counter()
+    ref = {"idx": np.full((cfg.batch, len(rows), cfg.recall_r), -1, np.int64), "block": b,
+           "x_proj": np.zeros((cfg.batch, S, P.shape[1])), "summary_proj": np.zeros((cfg.batch, nblk, P.shape[1]))}
+    for bi in range(cfg.batch):
+        summ = np.zeros((nblk, cfg.d_model))
+        for j0 in range(0, nblk, 64):  # block means, 64 blocks of rows widened at a time
+            j1 = min(nblk, j0 + 64)
+            summ[j0:j1] = oracle.block_summaries(to_f64(inp.x[bi:bi + 1, j0 * b:j1 * b]), b)[0]
+        xr = to_f64(inp.x[bi, :S][torch.from_numpy(rows)])
+        idx, _, _, _, xproj = oracle.longterm_recall(xr, rows, summ, P, b, cfg.recall_r)
+        ref["idx"][bi] = idx
+        ref["x_proj"][bi, rows] = xproj
+        ref["summary_proj"][bi] = oracle.hash_codes(summ, P)[1]
+    full_ref = dict(ref, idx=np.full((cfg.batch, S, cfg.recall_r), -1, np.int64))
+    full_ref["idx"][:, rows] = ref["idx"]
+    unexcused, excused, _ = oracle.recall_mismatches(idx_gpu[:, rows], full_ref, rows)
+    return {"rows_checked": int(cfg.batch * len(rows)), "rows_total": int(cfg.tokens),
+            "rows": "all" if stride == 1 else f"every {stride}th row of each sequence",
+            "mismatches_unexcused": unexcused, "mismatches_excused": excused,
+            "rule": "bit-exact; excused only where a flip of hash bits with |p| < 1e-4 gives the GPU's list",
+            "oracle_s": round(time.perf_counter() - t0, 1)}
 
 
 def run_reference(args, rank, world):
@@ -529,20 +665,21 @@ def run_reference(args, rank, world):
     inp = make_inputs(cfg)
     vals = []
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(cfg, inp, budget_rows=max(8, args.cpu_rows // 4))
+        r = cpu_baseline(cfg, inp, prefix_tokens=args.ref_prefix, attn_rows=max(4, args.cpu_rows // 4))
         if i >= args.warmup:
             vals.append(r)
     v = statistics.mean(r["value"] for r in vals)
-    ms = statistics.mean(cfg.tokens / r["value"] * 1e3 for r in vals)
+    ms = statistics.mean(r["measured_s"] for r in vals) * 1e3
     return {"impl": "reference", "metric": "FastMKA layer prefill tokens/s (decode us/token and roofline fraction "
-                                           "alongside)", "value": round(v, 2), "unit": "tokens/s", "n_gpus": world,
+                                           "alongside)", "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "global_batch": cfg.batch, "seq_len": cfg.seq,
-                       "parallelism": "CPU oracle, rank 0 only"},
-            "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "cores": vals[-1]["cores"], "kind": "oracle",
+            "config": workload_config(cfg, world),
+            "value_is": "tokens/s of the whole workload, extrapolated from each step's measured sample; "
+                        "ms_per_step is the measured time of one sampled step",
+            "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": vals[-1]["cores"], "kind": "oracle",
                              "sample": vals[-1]["sample"]},
-            "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def traffic_from_profiles(kernel: str):
@@ -589,10 +726,14 @@ def job_throughput(units_per_rank: float, ms: float, world: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen7b_4k")
+    ap.add_argument("--workload", default=None,
+                    help="the headline workload (default: llama8b_128k, the largest single-GPU prefill; "
+                         "qwen7b_4k with --train)")
+    ap.add_argument("--by-workload", nargs="*", default=["tiny_f32", "qwen7b_4k", "qwen7b_32k"],
+                    help="further prefill workloads reported under by_workload (none: pass the flag alone)")
     ap.add_argument("--route", default="soft", choices=["soft", "fixed", "top1", "top2"],
                     help="routing gate variant (the published layer is soft)")
     ap.add_argument("--tiers", type=int, default=7, help="memory tier mask: 1 L1, 2 L2, 4 L3 (7 = all)")
@@ -602,13 +743,18 @@ def main():
                     help="Block-MKA block-sparse attention: own block + recalled blocks (prefill only)")
     ap.add_argument("--train", action="store_true",
                     help="time the layer training step (forward keeping activations + backward) instead of prefill")
-    ap.add_argument("--decode-ctx", type=int, nargs="*", default=[131072])
+    ap.add_argument("--decode-ctx", type=int, nargs="*", default=[4096, 32768, 131072, 262144])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode measurement (no prefill line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=48)
+    ap.add_argument("--cpu-rows", type=int, default=32, help="oracle attention rows per sequence in its sample")
+    ap.add_argument("--cpu-prefix", type=int, default=8192, help="tokens of the oracle's prefix sample (main arm)")
+    ap.add_argument("--ref-prefix", type=int, default=2048, help="tokens of each reference-arm step's prefix sample")
+    ap.add_argument("--no-recall-check", dest="recall_check", action="store_false")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.workload is None:
+        args.workload = "qwen7b_4k" if args.train else "llama8b_128k"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -82,7 +82,8 @@ __device__ __forceinline__ void linger_after_abort(volatile int* abort) {
 }
 
 // mbar_wait by every lane of a warp, with one answer for all: false if any lane's wait failed,
-// so the warp leaves its loop together (the warp-wide tcgen05 forms need it converged).
+// so the warp leaves its loop together (the warp-wide tcgen05 forms need it converged).  Every
+// role whose warps go on to warp-wide instructions (tcgen05.ld / st, shuffles) waits this way.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
 }

@@ -486,7 +486,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv; ++j, ++sit) {
-        if (!mbar_wait(&s_full[t], sit & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait_warp(&s_full[t], sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
         const bool diag = GA ? masked : (j == nkv - 1);
         // keys c > lim of this tile are in the future of this row
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // P_j V_j starts while pass 2 runs.  S_j landing means P_{j-1} V_{j-1}, issued before QK_j,
         // has completed, so the wait below returns at once.
         if (__ballot_sync(0xffffffffu, rescale)) {
-          if (!mbar_wait(&pv_done[t], (sit - 1) & 1, abort, status)) { ok = false; break; }
+          if (!mbar_wait_warp(&pv_done[t], (sit - 1) & 1, abort, status)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < DH; c += 32) {
@@ -596,7 +596,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (!ok) break;
       // epilogue: O_t / l -> bf16 -> global
-      if (!mbar_wait(&o_full[t], wi & 1, abort, status)) break;
+      if (!mbar_wait_warp(&o_full[t], wi & 1, abort, status)) break;
       tc_fence_after();
       const float inv = 1.f / l;
       // causal: row `row` of the output; MODE 1: slot `slot` of the token's partial results

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float2 ndrowv = make_float2(-drow, -drow);
       bool ok = true;
       for (int j = 0; j < n; ++j, ++sit) {
-        if (!mbar_wait(s_full, sit & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait_warp(s_full, sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
         const int lim = valid ? row - j * BT : -1;  // keys c > lim are masked (all, for a padding row)
         const bool diag = __any_sync(0xffffffffu, j == n - 1 || !valid);  // warp-uniform
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         // phase 2: scale dS = (scale P) (dP - D), packed over the first 32 of this half's dP columns
-        if (!mbar_wait(dp_full, sit & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait_warp(dp_full, sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
         uint32_t pv[2][32];
         tmem_ld32(p_tmem + 64 * half, pv[0]);
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) mbar_arrive(p_full);
       }
       if (!ok) break;
-      if (!mbar_wait(dq_full, rr & 1, abort, status)) break;
+      if (!mbar_wait_warp(dq_full, rr & 1, abort, status)) break;
       tc_fence_after();
       float* dst = a.dq + ((size_t)b * a.S + (valid ? row : 0)) * (size_t)(a.Hq * DH) + (size_t)h * DH +
                    half * (DH / 2);
@@ -598,8 +598,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int qt = kt + s % nq, st = sit & 1;
         // the stage's lse and D rows: landed with its Q (the stage is not refilled before this
         // step's dK MMAs, which wait for this warp)
-        if (!mbar_wait(&q_full[st], (sit >> 1) & 1, abort, status)) { ok = false; break; }
-        if (!mbar_wait(s_full, sit & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait_warp(&q_full[st], (sit >> 1) & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait_warp(s_full, sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
         const float* lse2 = (const float*)(sQ + st * C::QSTAGE + C::TILE);
         const float* dsum = lse2 + BT;
@@ -641,7 +641,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // phase 2: dS^T = P^T (dP^T - D) (dK takes its factor scale in the epilogue); P^T and dS^T
         // packed over this half's dP^T columns,
         // chunk cc at [32 cc, 32 cc + 16) and [32 cc + 16, 32 cc + 32) of the half
-        if (!mbar_wait(dp_full, sit & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait_warp(dp_full, sit & 1, abort, status)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {  // chunk by chunk: a chunk's outputs go only over its own inputs
@@ -673,7 +673,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) mbar_arrive(p_full);
       }
       if (!ok) break;
-      if (!mbar_wait(acc_full, rr & 1, abort, status)) break;
+      if (!mbar_wait_warp(acc_full, rr & 1, abort, status)) break;
       tc_fence_after();
       const bool valid = key < a.S;
       const int wkv = 2 * a.Hkv * DH;

@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
       const int acc = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], aph, abort, status)) break;
+      if (!mbar_wait_warp(&tfull[acc], aph, abort, status)) break;
       tc_fence_after();
       const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
       const int m = m0 + q * 32 + lane;
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int tile = pair; tile < ntiles; tile += npairs, ++tl) {
       const int acc = tl & 1;
       const uint32_t aph = (tl >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], aph, abort, status)) break;
+      if (!mbar_wait_warp(&tfull[acc], aph, abort, status)) break;
       tc_fence_after();
       const int n0 = (tile % nN) * BN;
       const int m = (tile / nN) * PAIR_BM + (int)rank * HALF_ROWS + q * 32 + lane;

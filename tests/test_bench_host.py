@@ -68,3 +68,47 @@ def test_reference_arm_runs_on_rank_zero_only():
     """The other ranks of a torchrun launch leave at once, with no oracle work and nothing printed."""
     args = argparse.Namespace(workload="qwen7b_4k", warmup=3, steps=1, cpu_rows=8)
     assert bench.run_reference(args, rank=1, world=2) is None
+
+
+def _ref_args(**kw):
+    a = dict(workload="tiny_f32", warmup=0, steps=1, cpu_rows=16, ref_prefix=256, route="soft", tiers=7, paths=1,
+             block_sparse=False)
+    a.update(kw)
+    return argparse.Namespace(**a)
+
+
+def test_reference_arm_prints_the_main_arms_config():
+    """Both arms describe the workload with the same config object, so the two lines compare."""
+    args = _ref_args()
+    res = bench.run_reference(args, rank=0, world=1)
+    assert res["impl"] == "reference"
+    assert res["config"] == bench.workload_config(bench.workload_cfg(args, "tiny_f32"), 1)
+    assert res["value"] > 0 and res["ms_per_step"] > 0
+    assert "extrapolated" in res["value_is"]
+
+
+def test_recall_check_counts_a_planted_mismatch():
+    """The bench's recall check finds no mismatch for the oracle's own recall, and counts one row
+    whose list is reversed (no hash bit of these inputs lies within 1e-4 of zero)."""
+    import numpy as np
+    import oracle
+    from fastmka_inputs import CONFIGS, make_inputs, to_f64
+    cfg = CONFIGS["tiny_f32"]
+    inp = make_inputs(cfg)
+    X = to_f64(inp.x)
+    summ = oracle.block_summaries(X, cfg.block)[0]
+    idx, *_ = oracle.longterm_recall(X[0], np.arange(cfg.seq), summ, to_f64(inp.hash_proj), cfg.block, cfg.recall_r)
+    got = idx[None].copy()
+    r = bench.recall_check(cfg, inp, got)
+    assert (r["mismatches_unexcused"], r["mismatches_excused"], r["rows_checked"]) == (0, 0, cfg.seq)
+    got[0, 200] = got[0, 200][::-1]
+    assert bench.recall_check(cfg, inp, got)["mismatches_unexcused"] == 1
+
+
+def test_hbm_bytes_of_the_headline_workload():
+    """The fuse reads the projected sources once and writes K and V once: at 1 x 131072 with
+    2 * d_kv = 2048 columns that is at least 1.07 GB + 0.54 GB."""
+    from fastmka_inputs import CONFIGS
+    b = bench.prefill_hbm_bytes(CONFIGS["llama8b_128k"])
+    assert b["route_fuse"] >= 131072 * 2048 * (4 + 2)
+    assert b["block_codes"] >= 131072 * 4096 * 2
