@@ -112,3 +112,15 @@ def test_hbm_bytes_of_the_headline_workload():
     b = bench.prefill_hbm_bytes(CONFIGS["llama8b_128k"])
     assert b["route_fuse"] >= 131072 * 2048 * (4 + 2)
     assert b["block_codes"] >= 131072 * 4096 * 2
+
+
+def test_sustained_peak_only_under_the_power_cap():
+    peaks = {"bf16_tflops": 1654.3, "bf16_tflops_sustained": 1391.4, "hbm_gbs": 6457.7, "source": "measured"}
+    from fastmka_inputs import CONFIGS
+    cfg = CONFIGS["llama8b_128k"]
+    capped = {"sm_mhz": 1552.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.power_capped(capped) and not bench.power_capped(full) and not bench.power_capped(None)
+    r = bench.attention_roofline(cfg, 140.0, peaks, sustained=True)
+    assert r["peak"] == 1391.4 and r["frac_of_burst_peak"] < r["frac"]
+    assert bench.attention_roofline(cfg, 140.0, peaks)["peak"] == 1654.3

@@ -66,8 +66,9 @@ def oracle_backward(cfg, inp, dout, idx_gpu):
     X = inp.x[:, :cfg.seq].float().numpy()
     w = oracle_weights(inp)
     fwd = oracle.fastmka_prefill(X, w, cfg, keep_d_space=True)
-    mism = np.flatnonzero((idx_gpu != fwd["idx"]).any(-1).reshape(-1))
-    assert mism.size == 0, f"{mism.size} tokens recall different blocks on the GPU (first {mism[:8]})"
+    if cfg.tiers & 4:  # with L3 off its weight is 0 and the GPU computes no recall (indices -1)
+        mism = np.flatnonzero((idx_gpu != fwd["idx"]).any(-1).reshape(-1))
+        assert mism.size == 0, f"{mism.size} tokens recall different blocks on the GPU (first {mism[:8]})"
     return fwd, oracle.fastmka_backward(X, w, cfg, dout.float().numpy().astype(np.float64), fwd)
 
 
