@@ -446,6 +446,8 @@ def fastmka_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray]
             M2, m2 = session_ema(xc, cfg.alpha, m2)
             pos = np.arange(r0, r1)
             idx, cnt, M3, xcodes, xproj = longterm_recall(xc[0], pos, summ, w.P, b, R)
+            if not tiers & 4:  # the L3 tier removed: no long-term memory at all (no recall, M3 = 0)
+                idx, cnt, M3 = np.full_like(idx, -1), np.zeros_like(cnt), np.zeros_like(M3)
             if recall_fixed is not None:
                 idx = np.asarray(recall_fixed[0][bi, r0:r1], np.int64)
                 cnt = np.asarray(recall_fixed[1][bi, r0:r1], np.int64)
@@ -500,7 +502,8 @@ def fastmka_decode(X: np.ndarray, w: Weights64, cfg) -> np.ndarray:
             lam = router(q[None], w.w_r1, w.w_r2, getattr(cfg, "route_mode", "soft"), getattr(cfg, "tiers", 7))[0]
             code_t, _ = hash_codes(x[None], w.P)
             s_arr = np.array(summaries).reshape(-1, d)
-            sel = recall_select(int(code_t[0]), np.array(codes, np.uint32), len(summaries), R)
+            n_rec = len(summaries) if getattr(cfg, "tiers", 7) & 4 else 0  # L3 removed: nothing recalled
+            sel = recall_select(int(code_t[0]), np.array(codes, np.uint32), n_rec, R)
             M3 = s_arr[sel].mean(axis=0) if len(sel) else np.zeros(d)
             xf = fuse_sources(lam[None], x[None], m2[None], M3[None])
             k, v = kv_project(xf, w.w_k, w.w_v)
@@ -578,6 +581,8 @@ def mka_full_prefill(X: np.ndarray, w: Weights64, cfg, rows: Optional[np.ndarray
         V2 = (M2[0] @ w.w_v).reshape(S, Hkv, dh)
         summ = block_summaries(Xb[None], b)[0]
         idx, cnt, _, _, xproj = longterm_recall(Xb, np.arange(S), summ, w.P, b, R)
+        if not tiers & 4:  # the L3 tier removed: no recall
+            idx, cnt = np.full_like(idx, -1), np.zeros_like(cnt)
         out["x_proj"][bi], out["summary_proj"][bi] = xproj, hash_codes(summ, w.P)[1]
         qr = q[rows].reshape(len(rows), Hq, dh)
         a1 = causal_gqa_attention(qr, rows, K1, V1, Hkv, cfg.scale)

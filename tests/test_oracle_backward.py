@@ -44,7 +44,7 @@ def check_gradients(backward_fn, cfg, seed=5, per_tensor=6):
     X, w, dO = tiny_problem(cfg, seed)
     fwd = O.fastmka_prefill(X, w, cfg, keep_d_space=True)
     fixed = (fwd["idx"], fwd["count"])
-    assert fixed[1].max() > 0, "the problem must recall some blocks"
+    assert fixed[1].max() > 0 or not cfg.tiers & 4, "the problem must recall some blocks"
     g = backward_fn(X, w, cfg, dO, fwd)
     rng = np.random.default_rng(seed + 1)
     # X: rows of the first blocks (recalled, EMA-weighted from far), a middle row and the last row
