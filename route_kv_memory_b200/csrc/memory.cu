@@ -517,9 +517,195 @@ __global__ void __launch_bounds__(64 * kRG) fuse_kernel(FuseArgs a) {
   if (r1 == a.S && rb == nr && rb > ra && a.state_ema) *(float4*)(a.state_ema + (size_t)bi * a.width + c) = m2;
 }
 
+// ---------------------------------------------------------------- route-fuse with staged summaries
+// The same fuse, organised around the recalled-block gather.  A CTA owns one sequence, a 64-column
+// slice of the projected sources and a range of blocks.  It first stages that slice of the mean of
+// every block its tokens can recall (the blocks before its last one) in shared memory, so the
+// R-way gather-mean of each token reads shared memory instead of L2.  bf16 layers stage the means
+// in bf16: 2^-9 relative on M3, the size of the rounding of the K/V it feeds; float32 layers stage
+// float32.  Threads: 8 columns each, 8 threads per row, the kRG row groups of a block (EMA carried
+// in from block_reduce's group end states), kFsBlocks blocks at a time; the projected rows, counts
+// and gates are loaded two rows ahead.
+constexpr int kFsCols = 64, kFsLaneCols = 8, kFsLanes = kFsCols / kFsLaneCols;
+constexpr int kFsThreads = 256, kFsBlocks = kFsThreads / (kFsLanes * kRG), kFsBlocksPerCta = 2 * kFsBlocks;
+constexpr size_t kFsMaxSmem = 200 * 1024;
+
+template <typename ST> struct Staged8;
+template <> struct Staged8<bf16> {
+  static __device__ __forceinline__ void put(bf16* p, float4 a, float4 b, float sc) {
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x * sc, a.y * sc), h1 = __floats2bfloat162_rn(a.z * sc, a.w * sc);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x * sc, b.y * sc), h3 = __floats2bfloat162_rn(b.z * sc, b.w * sc);
+    *(uint4*)p = make_uint4(*(uint32_t*)&h0, *(uint32_t*)&h1, *(uint32_t*)&h2, *(uint32_t*)&h3);
+  }
+  static __device__ __forceinline__ void add(const bf16* p, float* acc) {
+    const uint4 u = *(const uint4*)p;
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += __uint_as_float(w[i] << 16);
+      acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+template <> struct Staged8<float> {
+  static __device__ __forceinline__ void put(float* p, float4 a, float4 b, float sc) {
+    *(float4*)p = f4_scale(sc, a);
+    *(float4*)(p + 4) = f4_scale(sc, b);
+  }
+  static __device__ __forceinline__ void add(const float* p, float* acc) {
+    const float4 a = *(const float4*)p, b = *(const float4*)(p + 4);
+    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+  }
+};
+
+template <typename OutT> __device__ __forceinline__ void store8(OutT* p, const float* v);
+template <> __device__ __forceinline__ void store8<float>(float* p, const float* v) {
+  *(float4*)p = make_float4(v[0], v[1], v[2], v[3]);
+  *(float4*)(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *(uint32_t*)&h;
+  }
+  *(uint4*)p = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+struct FsRow {  // what one row needs besides the staged means: its 8 sources, count and gates
+  float4 xa, xb;
+  int cnt;
+  float l0, l1, l2;
+};
+
+template <typename OutT, typename ST>
+__global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, int blocks_per_cta) {
+  extern __shared__ __align__(16) uint8_t fs_smem[];
+  ST* smean = (ST*)fs_smem;  // [nstage][kFsCols] block means of this slice
+  const int bi = blockIdx.z, c0 = blockIdx.x * kFsCols;
+  const int nb_all = (a.S + a.blk - 1) / a.blk;  // the unfinished block included
+  const int J0 = blockIdx.y * blocks_per_cta, J1 = min(nb_all, J0 + blocks_per_cta);
+  if (J0 >= J1) return;
+  const int nstage = min(J1 - 1, a.nblk);  // a token of block j recalls blocks < j only
+  const float invb = 1.f / (float)a.blk;
+  const float* bs = a.bsum + (size_t)bi * a.bsum_bstride + c0;
+  for (int i = threadIdx.x; i < nstage * kFsLanes; i += blockDim.x) {
+    const int jj = i / kFsLanes, cc = (i % kFsLanes) * kFsLaneCols;
+    const float* src = bs + (size_t)jj * a.width + cc;
+    Staged8<ST>::put(smean + jj * kFsCols + cc, *(const float4*)src, *(const float4*)(src + 4), invb);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x % kFsLanes, rg = (threadIdx.x / kFsLanes) % kRG, bl = threadIdx.x / (kFsLanes * kRG);
+  const int cs = lane * kFsLaneCols, c = c0 + cs;
+  const bool is_k = c < a.dkv;
+  const float al = a.alpha, om = 1.f - a.alpha;
+  for (int j = J0 + bl; j < J1; j += kFsBlocks) {
+    const int r0 = j * a.blk, nr = min(a.blk, a.S - r0);
+    // EMA value at this group's first row: the block's carry advanced over the preceding groups
+    const float* cp = a.carry + ((size_t)bi * (a.nblk + 1) + j) * a.width + c;
+    float4 ma = *(const float4*)cp, mb = *(const float4*)(cp + 4);
+    int ra, rb;
+    if (j < a.nblk) {
+      group_rows(rg, a.blk, ra, rb);
+      for (int g = 0; g < rg; ++g) {
+        int ga, gb;
+        group_rows(g, a.blk, ga, gb);
+        float ap = 1.f;
+        for (int i = ga; i < gb; ++i) ap *= al;
+        const float* ge = a.gend + (((size_t)bi * a.nblk + j) * kRG + g) * a.width + c;
+        ma = f4_add(f4_scale(ap, ma), *(const float4*)ge);
+        mb = f4_add(f4_scale(ap, mb), *(const float4*)(ge + 4));
+      }
+    } else {  // the unfinished last block: one group walks all its rows
+      ra = 0;
+      rb = rg == 0 ? nr : 0;
+    }
+    float m2[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+    const size_t tg0 = (size_t)bi * a.S + r0;
+    OutT* dst = (OutT*)(is_k ? a.k_out : a.v_out) + (size_t)bi * a.kv_bstride + (size_t)r0 * a.dkv +
+                (is_k ? c : c - a.dkv);
+    auto fetch = [&](int r, FsRow& f) {
+      if (r < rb) {
+        const size_t t = tg0 + r;
+        const float* xp = a.xkv + t * a.ld + c;
+        f.xa = __ldcs((const float4*)xp);
+        f.xb = __ldcs((const float4*)(xp + 4));
+        f.cnt = __ldg(a.count + t);
+        f.l0 = __ldg(a.lam + t * 3);
+        f.l1 = __ldg(a.lam + t * 3 + 1);
+        f.l2 = __ldg(a.lam + t * 3 + 2);
+      }
+    };
+    FsRow cur[2], nxt[2];
+    fetch(ra, cur[0]);
+    fetch(ra + 1, cur[1]);
+    for (int r = ra; r < rb; r += 2) {
+      fetch(r + 2, nxt[0]);
+      fetch(r + 3, nxt[1]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (r + u < rb) {
+          const FsRow& f = cur[u];
+          const size_t t = tg0 + r + u;
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          const int* ip = a.idx + t * a.R;
+          for (int q = 0; q < f.cnt; ++q) {
+            const int jq = __ldg(ip + q);
+            if ((unsigned)jq < (unsigned)nstage) Staged8<ST>::add(smean + jq * kFsCols + cs, acc);
+          }
+          const float s3 = f.cnt ? f.l2 / (float)f.cnt : 0.f;
+          const float x[8] = {f.xa.x, f.xa.y, f.xa.z, f.xa.w, f.xb.x, f.xb.y, f.xb.z, f.xb.w};
+          float o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            o[i] = fmaf(f.l0, x[i], fmaf(f.l1, m2[i], s3 * acc[i]));
+            m2[i] = fmaf(al, m2[i], om * x[i]);
+          }
+          store8<OutT>(dst + (size_t)(r + u) * a.dkv, o);
+        }
+      }
+      cur[0] = nxt[0];
+      cur[1] = nxt[1];
+    }
+    if (r0 + rb == a.S && rb > ra && a.state_ema) {
+      float* se = a.state_ema + (size_t)bi * a.width + c;
+      *(float4*)se = make_float4(m2[0], m2[1], m2[2], m2[3]);
+      *(float4*)(se + 4) = make_float4(m2[4], m2[5], m2[6], m2[7]);
+    }
+  }
+}
+
+// Shared-memory bytes of the staged fuse (0: it does not apply, use fuse_kernel).
+size_t fuse_staged_smem(const FuseArgs& a) {
+  if (a.v2_out || a.width % kFsCols || a.dkv % kFsCols) return 0;
+  const size_t b = (size_t)a.nblk * kFsCols * (a.out_bf16 ? 2 : 4);
+  return b <= kFsMaxSmem ? (b > 16 ? b : 16) : 0;
+}
+
 cudaError_t fuse_kv(const FuseArgs& a, cudaStream_t s) {
   if (a.B <= 0 || a.S <= 0) return cudaSuccess;
   int nb_all = (a.S + a.blk - 1) / a.blk;
+  if (const size_t fsm = fuse_staged_smem(a)) {
+    // many short CTAs (two passes of kFsBlocks blocks of one column slice each) balance the SMs;
+    // two are resident per SM, so one stages while the other streams
+    const int slices = a.width / kFsCols;
+    const int bpc = kFsBlocksPerCta;
+    const int nchunk = (nb_all + bpc - 1) / bpc;
+    dim3 grid(slices, nchunk, a.B);
+    cudaError_t e;
+    if (a.out_bf16) {
+      e = set_max_smem(fuse_staged_kernel<bf16, bf16>, fsm, s);
+      if (e != cudaSuccess) return e;
+      fuse_staged_kernel<bf16, bf16><<<grid, kFsThreads, fsm, s>>>(a, bpc);
+    } else {
+      e = set_max_smem(fuse_staged_kernel<float, float>, fsm, s);
+      if (e != cudaSuccess) return e;
+      fuse_staged_kernel<float, float><<<grid, kFsThreads, fsm, s>>>(a, bpc);
+    }
+    return cudaGetLastError();
+  }
   dim3 grid((a.width / 4 + 63) / 64, nb_all, a.B);
   size_t sm = (size_t)a.blk * (3 * sizeof(float) + (a.R + 1) * sizeof(int));
   if (a.out_bf16) {

@@ -54,6 +54,12 @@ EDGE = [
           recall_r=8, hash_bits=32, seed=14),
     small("bf16_b2_s129", "bf16", batch=2, seq=129, n_q_heads=4, n_kv_heads=4, d_head=128, seed=15),
     small("bf16_s1", "bf16", seq=1, d_head=128, seed=16),
+    # more blocks (2000) than the fuse stages in shared memory: the unstaged fuse kernel runs
+    small("bf16_blocks_of_1", "bf16", seq=2000, block=1, recall_r=3, hash_bits=8, seed=17),
+    small("f32_blocks_of_2_many", "f32", seq=1700, block=2, recall_r=2, hash_bits=6, seed=18),
+    # many staged blocks, several passes per CTA, a ragged last block
+    small("bf16_staged_passes", "bf16", batch=2, seq=1100, d_head=128, n_q_heads=4, n_kv_heads=2, block=16,
+          recall_r=5, hash_bits=12, seed=19),
 ]
 
 
