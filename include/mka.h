@@ -230,10 +230,10 @@ MKA_API int mka_prefill_backward(const mka_config* cfg, const void* packed, cons
  * nothing.  ws: mka_decode_workspace_size(cfg, max_positions) bytes.
  * A step whose bounded device-side wait ran out records MKA_ERR_DEVICE_TIMEOUT and
  * may have applied part of its update: the state's position, cache row and memories
- * are then unspecified, and the out row too.  Refill the state with
- * mka_prefill_forward (a prefill into a state redefines all of it) before decoding
- * on.  The step's grid barrier is reset by the last CTA to leave every launch, so
- * a timed-out step does not affect the barrier of the next. */
+ * are then unspecified, and the out row too, and so is the step's grid barrier (an
+ * arrival count in the state).  Refill the state with mka_prefill_forward (a prefill
+ * into a state redefines all of it, the barrier included) or mka_state_init before
+ * decoding on. */
 MKA_API int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size_t state_bytes,
                     int32_t max_positions, const void* x_new, void* out, void* ws, size_t ws_bytes, void* stream);
 

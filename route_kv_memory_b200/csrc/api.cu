@@ -215,7 +215,7 @@ StateLayout state_layout(const Dims& d, int Lmax) {
   s.maxblk = Lmax / d.blk;
   size_t o = 0, B = d.B;
   s.pos = o; o += al(B * 4);
-  s.sync = o; o += al(3 * 4);
+  s.sync = o; o += al(8);
   s.kc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.vc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.ema = o; o += al(B * d.width * 4);
@@ -251,7 +251,7 @@ DecodeWs decode_ws(const Dims& d, int Lmax) {
   size_t o = 0, B = d.B;
   w.y = o; o += al(B * p.Ntot * 4);
   w.qf = o; o += al(B * d.dq * 4);
-  w.part = o; o += al(B * d.Hq * (size_t)w.nsplit * (d.dh + 2) * 4);
+  w.part = o; o += al(B * d.Hq * (size_t)w.nsplit * (d.dh + 4) * 4);  // records of part_rec(dh) floats
   w.total = o;
   return w;
 }
@@ -636,6 +636,8 @@ static int prefill_forward(const mka_config* cfg, const void* packed, const void
   // blocks this prefill does not finish start at zero, so a prefill redefines the whole state.
   if (state && SL.maxblk > d.nblk)
     CUDA_TRY(cudaMemset2DAsync(scode + d.nblk, (size_t)SL.maxblk * 4, 0, (size_t)(SL.maxblk - d.nblk) * 4, d.B, s));
+  // and the decode step's grid barrier starts from zero arrivals
+  if (state) CUDA_TRY(cudaMemsetAsync(P(state, SL.sync), 0, 8, s));
   std::unique_lock<std::mutex> aux_lock(aux_mutex(), std::defer_lock);
   AuxStreams* ax = nullptr;
   if (!g_prof.on) {
@@ -996,7 +998,7 @@ int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size
   a.ema = (float*)P(state, SL.ema); a.blk_sum = (float*)P(state, SL.blk_sum); a.blk_x = (double*)P(state, SL.blk_x);
   a.summ = (float*)P(state, SL.summ); a.scode = (uint32_t*)P(state, SL.scode);
   a.y = (float*)P(ws, W.y); a.qf = (float*)P(ws, W.qf); a.part = (float*)P(ws, W.part); a.nsplit = W.nsplit;
-  a.sync = (unsigned*)P(state, SL.sync);
+  a.sync = (unsigned long long*)P(state, SL.sync);
   a.status = status_ptr();
   prof_begin();
   a.prof = g_prof.on ? g_prof.ev : nullptr;

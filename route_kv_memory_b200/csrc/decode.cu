@@ -11,6 +11,11 @@
 
 namespace mka {
 
+// ---------------------------------------------------------------- split-KV partial records
+// One record per (sequence, query head, split): o[DH] (unnormalised), then m (log2 units) and
+// l, padded to a multiple of four floats so that every record's o starts 16-byte aligned.
+__host__ __device__ constexpr int part_rec(int dh) { return dh + 4; }
+
 // ---------------------------------------------------------------- 1. GEMV
 constexpr int kMaxDecodeBatch = 8;
 
@@ -449,15 +454,15 @@ __device__ void attn_unit(const DecodeArgs& a, const int split, const int g, con
     }
   }
   __syncthreads();
-  // partial record per (b, head, split): [m (log2 units), l, o[DH] (unnormalised)]
-  const int rec = DH + 2;
+  // partial record per (b, head, split): [o[DH] (unnormalised), m (log2 units), l]
+  constexpr int rec = part_rec(DH);
   for (int i = tid; i < G * DH; i += NWD * 32) {
     int r = i / DH, c = i % DH;
     int hq = g * G + r;
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < NWD; ++w) v += so[((size_t)w * 16 + r) * DH + c];
-    a.part[(((size_t)bi * a.Hq + hq) * a.nsplit + split) * rec + 2 + c] = v;
+    a.part[(((size_t)bi * a.Hq + hq) * a.nsplit + split) * rec + c] = v;
   }
   if (warp == 0 && (lane & 3) == 0) {
 #pragma unroll
@@ -465,8 +470,8 @@ __device__ void attn_unit(const DecodeArgs& a, const int split, const int g, con
       int row = (lane >> 2) + 8 * r;
       if (row < G) {
         float* pr = a.part + (((size_t)bi * a.Hq + g * G + row) * a.nsplit + split) * rec;
-        pr[0] = M[r];
-        pr[1] = Lsum[r];
+        pr[DH] = M[r];
+        pr[DH + 1] = Lsum[r];
       }
     }
   }
@@ -526,14 +531,14 @@ __global__ void decode_attn_f32_kernel(DecodeArgs a) {
 #pragma unroll
       for (int i = 0; i < PER; ++i) out[i] += s_o[w][lane + 32 * i] * wg;
     }
-    const int rec = DH + 2;
+    constexpr int rec = part_rec(DH);
     float* pr = a.part + (((size_t)bi * a.Hq + hq) * a.nsplit + split) * rec;
     if (lane == 0) {
-      pr[0] = M;
-      pr[1] = Ls;
+      pr[DH] = M;
+      pr[DH + 1] = Ls;
     }
 #pragma unroll
-    for (int i = 0; i < PER; ++i) pr[2 + lane + 32 * i] = out[i];
+    for (int i = 0; i < PER; ++i) pr[lane + 32 * i] = out[i];
   }
 }
 
@@ -541,20 +546,20 @@ __global__ void decode_attn_f32_kernel(DecodeArgs a) {
 template <typename T>
 __global__ void decode_merge_kernel(DecodeArgs a) {
   const int hq = blockIdx.x, bi = blockIdx.y;
-  const int rec = a.dh + 2;
+  const int rec = part_rec(a.dh), dh = a.dh;
   const float* pr = a.part + ((size_t)bi * a.Hq + hq) * a.nsplit * rec;
   float M = -INFINITY;
-  for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, pr[(size_t)s * rec]);
+  for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, pr[(size_t)s * rec + dh]);
   float Ls = 0.f;
   for (int s = 0; s < a.nsplit; ++s) {
-    float m = pr[(size_t)s * rec];
-    if (m != -INFINITY) Ls += pr[(size_t)s * rec + 1] * exp2f(m - M);
+    float m = pr[(size_t)s * rec + dh];
+    if (m != -INFINITY) Ls += pr[(size_t)s * rec + dh + 1] * exp2f(m - M);
   }
   for (int c = threadIdx.x; c < a.dh; c += blockDim.x) {
     float acc = 0.f;
     for (int s = 0; s < a.nsplit; ++s) {
-      float m = pr[(size_t)s * rec];
-      if (m != -INFINITY) acc += pr[(size_t)s * rec + 2 + c] * exp2f(m - M);
+      float m = pr[(size_t)s * rec + dh];
+      if (m != -INFINITY) acc += pr[(size_t)s * rec + c] * exp2f(m - M);
     }
     ((T*)a.out)[(size_t)bi * a.dq + (size_t)hq * a.dh + c] = from_f<T>(acc / Ls);
   }
@@ -709,57 +714,46 @@ __device__ void token_slice(const DecodeArgs& a, const int bi, const int pos, co
 //   -- grid barrier --
 //   C  per (sequence, query head): merge the split partials and the new row's own
 //      term (its score against the appended K row, weight on the appended V row)
-// The two barriers are counters in the decode state, each wait bounded by a time
-// limit that records MKA_ERR_DEVICE_TIMEOUT.  All CTAs are co-resident
-// (cooperative launch), so the barrier cannot deadlock on scheduling.  A CTA whose
-// wait ran out leaves the step; every CTA counts itself out on the way, and the
-// last to leave clears the barrier's arrival count for the next launch.
+// The two barriers share one arrival count in the decode state, each wait bounded by a
+// time limit that records MKA_ERR_DEVICE_TIMEOUT.  All CTAs are co-resident (cooperative
+// launch), so the barrier cannot deadlock on scheduling.  A CTA whose wait ran out leaves
+// the step.
 constexpr int kFusedRing = 2 * 2 * dk::NWD * dk::TP * 128 * 2;  // 64 KB: GEMV chunks, then K/V tiles
 static_assert(kFusedRing >= dk::NWD * 16 * 128 * 4, "attention merge scratch must fit the ring");
 
-__device__ bool grid_sync(unsigned* count, unsigned* gen, unsigned nblocks, int* status) {
+// Grid barrier on a 64-bit arrival count that only grows: a CTA's own arrival number tells it
+// which barrier it is in (every launch passes whole barriers of nblocks arrivals), so the barrier
+// is released by the last arrival itself, with no reset and no second word.  A step whose wait
+// ran out leaves the count mid-barrier; a prefill into the state (or mka_state_init) zeroes it.
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ bool grid_sync(unsigned long long* count, unsigned nblocks, int* status) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
     s_ok = 1;
-    const unsigned g = *(volatile unsigned*)gen;
     __threadfence();
-    if (atomicAdd(count, 1u) == nblocks - 1) {
-      atomicExch(count, 0u);
-      __threadfence();
-      atomicAdd(gen, 1u);
-    } else {
+    const unsigned long long arrival = atomicAdd(count, 1ull);
+    const unsigned long long target = (arrival / nblocks + 1) * nblocks;
+    if (ld_acquire_u64(count) < target) {
       const unsigned long long t0 = sm100::globaltimer();
       const unsigned long long lim = wait_limit(status, kWaitGrid, sm100::kWaitLimitNs);
-      while (*(volatile unsigned*)gen == g) {
+      while (ld_acquire_u64(count) < target) {
         if (sm100::globaltimer() - t0 > lim) {
           set_status(status, kStatusTimeout);
           s_ok = 0;
           break;
         }
-        __nanosleep(64);
+        __nanosleep(32);
       }
     }
     __threadfence();
   }
   __syncthreads();
   return s_ok != 0;
-}
-
-// Every CTA of a fused decode launch leaves through here, after its last use of the grid
-// barrier (sync[0] arrivals, sync[1] generation, sync[2] CTAs gone).  The last CTA to leave
-// zeroes the arrival count: a step in which some CTAs gave up on a barrier leaves arrivals
-// counted, and the next launch would otherwise pass its first barrier early.
-__device__ void grid_exit(unsigned* sync, unsigned nblocks) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(sync + 2, 1u) == nblocks - 1) {
-      atomicExch(sync, 0u);
-      atomicExch(sync + 2, 0u);
-      __threadfence();
-    }
-  }
 }
 
 __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -787,14 +781,17 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) 
 
 constexpr int kMaxSplits = 512;
 
-// Combines the split partials (m in log2 units, l, unnormalised o) of (sequence bi, query
-// head hq) and, when the step appended a row at pos_old, that row's own term.
+// Combines the split partials (unnormalised o, m in log2 units, l) of (sequence bi, query head
+// hq) and, when the step appended a row at pos_old, that row's own term.  The splits are
+// shared out over the warps (16-byte loads of o, independent across splits), then summed over
+// the warps in a fixed order: deterministic.
 template <int DH>
 __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, const int pos_old) {
   __shared__ float s_w[kMaxSplits];
   __shared__ float red[32];
-  const int tid = threadIdx.x;
-  const int rec = DH + 2;
+  __shared__ float4 s_acc[dk::NWD][DH / 4];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int rec = part_rec(DH);
   const int g = hq / (a.Hq / a.Hkv);
   const float* pr = a.part + ((size_t)bi * a.Hq + hq) * a.nsplit * rec;
   const bool has_new = pos_old < a.Lmax;
@@ -804,11 +801,11 @@ __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, cons
   float s = 0.f;
   if (has_new)
     for (int c = tid; c < DH; c += blockDim.x)
-      s = fmaf(__bfloat162float(__float2bfloat16_rn(q[c])), __bfloat162float(kn[c]), s);
+      s = fmaf(__bfloat162float(__float2bfloat16_rn(__ldcg(q + c))), __bfloat162float(kn[c]), s);
   const float snew = block_reduce(s, false, red) * a.scale * 1.4426950408889634f;
   float mloc = has_new ? snew : -INFINITY;
   for (int sp = tid; sp < a.nsplit; sp += blockDim.x) {
-    const float m = pr[(size_t)sp * rec];
+    const float m = __ldcg(pr + (size_t)sp * rec + DH);
     s_w[sp] = m;
     mloc = fmaxf(mloc, m);
   }
@@ -818,22 +815,43 @@ __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, cons
     const float m = s_w[sp];
     const float w = m == -INFINITY ? 0.f : exp2f(m - M);
     s_w[sp] = w;
-    lloc += w * pr[(size_t)sp * rec + 1];
+    lloc += w * __ldcg(pr + (size_t)sp * rec + DH + 1);
   }
   const float wn = has_new ? exp2f(snew - M) : 0.f;
   const float Ls = block_reduce(lloc, false, red) + wn;  // also orders the s_w writes before the reads below
   const float inv = 1.f / Ls;
-  for (int c = tid; c < DH; c += blockDim.x) {
-    float a0 = has_new ? wn * __bfloat162float(vn[c]) : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    int sp = 0;
-    for (; sp + 3 < a.nsplit; sp += 4) {
-      a0 = fmaf(pr[(size_t)sp * rec + 2 + c], s_w[sp], a0);
-      a1 = fmaf(pr[(size_t)(sp + 1) * rec + 2 + c], s_w[sp + 1], a1);
-      a2 = fmaf(pr[(size_t)(sp + 2) * rec + 2 + c], s_w[sp + 2], a2);
-      a3 = fmaf(pr[(size_t)(sp + 3) * rec + 2 + c], s_w[sp + 3], a3);
+  if (lane < DH / 4) {
+    float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+    int sp = warp;
+    for (; sp + dk::NWD < a.nsplit; sp += 2 * dk::NWD) {
+      const float4 v0 = __ldcg((const float4*)(pr + (size_t)sp * rec) + lane);
+      const float4 v1 = __ldcg((const float4*)(pr + (size_t)(sp + dk::NWD) * rec) + lane);
+      const float w0 = s_w[sp], w1 = s_w[sp + dk::NWD];
+      acc0 = make_float4(fmaf(v0.x, w0, acc0.x), fmaf(v0.y, w0, acc0.y), fmaf(v0.z, w0, acc0.z), fmaf(v0.w, w0, acc0.w));
+      acc1 = make_float4(fmaf(v1.x, w1, acc1.x), fmaf(v1.y, w1, acc1.y), fmaf(v1.z, w1, acc1.z), fmaf(v1.w, w1, acc1.w));
     }
-    for (; sp < a.nsplit; ++sp) a0 = fmaf(pr[(size_t)sp * rec + 2 + c], s_w[sp], a0);
-    ((bf16*)a.out)[(size_t)bi * a.dq + (size_t)hq * DH + c] = __float2bfloat16_rn(((a0 + a1) + (a2 + a3)) * inv);
+    if (sp < a.nsplit) {
+      const float4 v0 = __ldcg((const float4*)(pr + (size_t)sp * rec) + lane);
+      const float w0 = s_w[sp];
+      acc0 = make_float4(fmaf(v0.x, w0, acc0.x), fmaf(v0.y, w0, acc0.y), fmaf(v0.z, w0, acc0.z), fmaf(v0.w, w0, acc0.w));
+    }
+    s_acc[warp][lane] = make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
+  }
+  __syncthreads();
+  if (tid < DH / 4) {
+    float4 t = s_acc[0][tid];
+#pragma unroll
+    for (int w = 1; w < dk::NWD; ++w) {
+      const float4 u = s_acc[w][tid];
+      t = make_float4(t.x + u.x, t.y + u.y, t.z + u.z, t.w + u.w);
+    }
+    float o[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = 4 * tid + e;
+      if (has_new) o[e] = fmaf(wn, __bfloat162float(vn[c]), o[e]);
+      ((bf16*)a.out)[(size_t)bi * a.dq + (size_t)hq * DH + c] = __float2bfloat16_rn(o[e] * inv);
+    }
   }
   __syncthreads();
 }
@@ -848,17 +866,72 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int NW = dk::NWD;
   const unsigned nblk = gridDim.x;
-  if (tid < a.B) s_pos[tid] = a.pos[tid];  // positions before this step changes them
-  if (tid == 0) {
-    sm100::mbar_init(&gbar[0], 1);
-    sm100::mbar_init(&gbar[1], 1);
-    sm100::fence_barrier_init();
+  // positions before this step changes them (visible to the CTA after the first grid barrier)
+  if (tid < a.B) s_pos[tid] = a.pos[tid];
+  // batch 1 with d_model a multiple of 256 up to 4096: phase A streams the weight rows through
+  // registers (no shared-memory ring, no set-up barrier)
+  const bool reg_gemv = a.B == 1 && (a.d & 255) == 0 && a.d <= 4096;
+  if (!reg_gemv) {
+    if (tid == 0) {
+      sm100::mbar_init(&gbar[0], 1);
+      sm100::mbar_init(&gbar[1], 1);
+      sm100::fence_barrier_init();
+    }
+    for (int i = tid; i < a.B * a.d / 8; i += blockDim.x) ((uint4*)sx)[i] = ((const uint4*)a.x_new)[i];
+    __syncthreads();
   }
-  for (int i = tid; i < a.B * a.d / 8; i += blockDim.x) ((uint4*)sx)[i] = ((const uint4*)a.x_new)[i];
-  __syncthreads();
 
   // ---- A: projection row, this CTA's share of the packed weight rows
-  {
+  if (reg_gemv) {
+    // Every warp of the grid takes the rows r = gw, gw + TW, ... two at a time; a lane holds the
+    // 16-byte vectors lane + 32 k (k < d / 256) of both rows, all of a row's loads issued before
+    // its dot products, so each SM keeps ~100 KB of weights in flight.
+    const int TW = (int)nblk * NW, gw = (int)blockIdx.x * NW + warp;
+    const int kv = a.d / 256;
+    const uint4* W = (const uint4*)a.wcatT;
+    const size_t rowv = (size_t)a.d / 8;
+    const uint4* xv = (const uint4*)a.x_new;  // read through L1: every warp reads the same 16 B pieces
+    for (int r = gw; r < a.Ntot; r += 2 * TW) {
+      const int r2 = r + TW;
+      const bool two = r2 < a.Ntot;
+      uint4 w1[16], w2[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        if (k < kv) {
+          w1[k] = __ldg(W + (size_t)r * rowv + lane + 32 * k);
+          if (two) w2[k] = __ldg(W + (size_t)r2 * rowv + lane + 32 * k);
+        }
+      }
+      float a1[2] = {0.f, 0.f}, a2[2] = {0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        if (k < kv) {
+          const uint4 xu = __ldg(xv + lane + 32 * k);
+          const __nv_bfloat162* xh = (const __nv_bfloat162*)&xu;
+          const __nv_bfloat162* h1 = (const __nv_bfloat162*)&w1[k];
+          const __nv_bfloat162* h2 = (const __nv_bfloat162*)&w2[k];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 xf = __bfloat1622float2(xh[e]);
+            const float2 f1 = __bfloat1622float2(h1[e]);
+            a1[k & 1] = fmaf(f1.x, xf.x, a1[k & 1]);
+            a1[k & 1] = fmaf(f1.y, xf.y, a1[k & 1]);
+            if (two) {
+              const float2 f2 = __bfloat1622float2(h2[e]);
+              a2[k & 1] = fmaf(f2.x, xf.x, a2[k & 1]);
+              a2[k & 1] = fmaf(f2.y, xf.y, a2[k & 1]);
+            }
+          }
+        }
+      }
+      const float v1 = warp_sum(a1[0] + a1[1]);
+      const float v2 = two ? warp_sum(a2[0] + a2[1]) : 0.f;
+      if (lane == 0) {
+        a.y[r] = v1;
+        if (two) a.y[r2] = v2;
+      }
+    }
+  } else {
     const int rpc = (a.Ntot + (int)nblk - 1) / (int)nblk;
     const int r0 = blockIdx.x * rpc, r1 = min(a.Ntot, r0 + rpc);
     const size_t row_bytes = (size_t)a.d * 2;
@@ -936,7 +1009,7 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
       __syncthreads();  // stage (c & 1) is free for chunk c + 2
     }
   }
-  if (!grid_sync(a.sync, a.sync + 1, nblk, a.status)) return;
+  if (!grid_sync(a.sync, nblk, a.status)) return;
 
   // ---- B: split-KV attention over the old rows (units handed out from CTA ntok on), and the
   // token update, split over the first ntok CTAs
@@ -968,7 +1041,7 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
         a.pos[threadIdx.x] = s_pos[threadIdx.x] + 1;
     }
   }
-  if (!grid_sync(a.sync, a.sync + 1, nblk, a.status)) return;
+  if (!grid_sync(a.sync, nblk, a.status)) return;
 
   // ---- C: merge, and finish a block completed by this token: its projected sum becomes
   // the summary, its code the signs of the exact float64 d_model-space sum projected on P
@@ -999,7 +1072,6 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
 template <int DH>
 __global__ void __launch_bounds__(dk::NWD * 32, 2) decode_fused_kernel(DecodeArgs a) {
   decode_fused_body<DH>(a);
-  grid_exit(a.sync, gridDim.x);
 }
 
 size_t decode_fused_smem(int B, int d) { return kFusedRing + (((size_t)B * d * 2 + 15) & ~(size_t)15) + 64; }

@@ -242,7 +242,7 @@ struct DecodeArgs {
   float* qf;                     // [B, dq] float32 query
   float* part;                   // split-KV partials
   int nsplit;
-  unsigned* sync;                // 3 words in the decode state: grid-barrier count, generation, CTAs gone
+  unsigned long long* sync;      // the decode state's grid-barrier arrival count (only grows)
   int* status;
   cudaEvent_t* prof;             // 5 events around the 4 stages, or NULL
 };

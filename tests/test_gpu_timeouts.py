@@ -87,9 +87,9 @@ def test_prefill_and_training_waits_run_out_then_the_layer_recovers(mka):
 
 def test_decode_grid_barrier_runs_out_then_a_refilled_state_decodes(mka):
     """The cooperative decode step with a 1 ns grid-barrier limit: CTAs that reach a barrier early
-    give up and leave.  The state is then refilled by a prefill, without mka_state_init, so its
-    barrier words are the ones the timed-out step left; the step's exit protocol must have cleared
-    them, or the next steps would pass their barriers early and decode wrong rows."""
+    give up and leave, and the barrier's arrival count is left mid-barrier.  The state is then
+    refilled by a prefill, without mka_state_init: the refill must reset the barrier too, or the
+    next steps would pass their barriers early and decode wrong rows."""
     cfg = _cfg("timeout_decode", seq=1100, n_q_heads=8, block=64, recall_r=4, seed=91)
     inp = make_inputs(cfg)
     ctx, n_new, lmax = 1000, 64, 1200
