@@ -527,8 +527,9 @@ __global__ void __launch_bounds__(64 * kRG) fuse_kernel(FuseArgs a) {
 // in from block_reduce's group end states), kFsBlocks blocks at a time; the projected rows, counts
 // and gates are loaded two rows ahead.
 constexpr int kFsCols = 64, kFsLaneCols = 8, kFsLanes = kFsCols / kFsLaneCols;
-constexpr int kFsThreads = 256, kFsBlocks = kFsThreads / (kFsLanes * kRG), kFsBlocksPerCta = 2 * kFsBlocks;
+constexpr int kFsThreads = 256, kFsBlocks = kFsThreads / (kFsLanes * kRG), kFsBlocksPerCta = kFsBlocks;
 constexpr size_t kFsMaxSmem = 200 * 1024;
+constexpr int kFsBatch = 8;  // staging loads in flight per thread
 
 template <typename ST> struct Staged8;
 template <> struct Staged8<bf16> {
@@ -574,100 +575,153 @@ template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v
   *(uint4*)p = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-struct FsRow {  // what one row needs besides the staged means: its 8 sources, count and gates
-  float4 xa, xb;
-  int cnt;
-  float l0, l1, l2;
-};
+// Shared memory of one CTA: the staged means, then the pass's recalled indices (16-bit), counts
+// and gates.
+template <typename ST>
+__device__ __forceinline__ size_t fs_mean_bytes(int nstage) {
+  return ((size_t)nstage * kFsCols * sizeof(ST) + 15) & ~(size_t)15;
+}
 
 template <typename OutT, typename ST>
 __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, int blocks_per_cta) {
   extern __shared__ __align__(16) uint8_t fs_smem[];
-  ST* smean = (ST*)fs_smem;  // [nstage][kFsCols] block means of this slice
   const int bi = blockIdx.z, c0 = blockIdx.x * kFsCols;
   const int nb_all = (a.S + a.blk - 1) / a.blk;  // the unfinished block included
   const int J0 = blockIdx.y * blocks_per_cta, J1 = min(nb_all, J0 + blocks_per_cta);
   if (J0 >= J1) return;
   const int nstage = min(J1 - 1, a.nblk);  // a token of block j recalls blocks < j only
+  ST* smean = (ST*)fs_smem;                // [nstage][kFsCols] block means of this slice
+  const int prows = kFsBlocks * a.blk;     // rows of one pass
+  uint16_t* sidx = (uint16_t*)(fs_smem + fs_mean_bytes<ST>(nstage));  // [prows][R]
+  float* slam = (float*)(sidx + (((size_t)prows * a.R + 7) & ~(size_t)7));  // [prows][3]
+  uint16_t* scnt = (uint16_t*)(slam + (size_t)prows * 3);                  // [prows]
   const float invb = 1.f / (float)a.blk;
   const float* bs = a.bsum + (size_t)bi * a.bsum_bstride + c0;
-  for (int i = threadIdx.x; i < nstage * kFsLanes; i += blockDim.x) {
-    const int jj = i / kFsLanes, cc = (i % kFsLanes) * kFsLaneCols;
-    const float* src = bs + (size_t)jj * a.width + cc;
-    Staged8<ST>::put(smean + jj * kFsCols + cc, *(const float4*)src, *(const float4*)(src + 4), invb);
+  // staging loads are batched (kFsBatch per thread in flight before any store): one L2 round
+  // trip per batch instead of one per element
+  for (int i0 = 0; i0 < nstage * kFsLanes; i0 += kFsBatch * kFsThreads) {
+    float4 va[kFsBatch], vb[kFsBatch];
+#pragma unroll
+    for (int u = 0; u < kFsBatch; ++u) {
+      const int i = i0 + u * kFsThreads + (int)threadIdx.x;
+      if (i < nstage * kFsLanes) {
+        const float* src = bs + (size_t)(i / kFsLanes) * a.width + (i % kFsLanes) * kFsLaneCols;
+        va[u] = *(const float4*)src;
+        vb[u] = *(const float4*)(src + 4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kFsBatch; ++u) {
+      const int i = i0 + u * kFsThreads + (int)threadIdx.x;
+      if (i < nstage * kFsLanes)
+        Staged8<ST>::put(smean + (i / kFsLanes) * kFsCols + (i % kFsLanes) * kFsLaneCols, va[u], vb[u], invb);
+    }
   }
-  __syncthreads();
   const int lane = threadIdx.x % kFsLanes, rg = (threadIdx.x / kFsLanes) % kRG, bl = threadIdx.x / (kFsLanes * kRG);
   const int cs = lane * kFsLaneCols, c = c0 + cs;
   const bool is_k = c < a.dkv;
   const float al = a.alpha, om = 1.f - a.alpha;
-  for (int j = J0 + bl; j < J1; j += kFsBlocks) {
+  for (int jp = J0; jp < J1; jp += kFsBlocks) {
+    // this pass's rows: their recalled indices, counts and gates, staged once for all columns
+    const int pr0 = jp * a.blk, pr1 = min(a.S, min(J1, jp + kFsBlocks) * a.blk), np = pr1 - pr0;
+    const size_t tp0 = (size_t)bi * a.S + pr0;
+    __syncthreads();  // the previous pass is done with the staged rows
+    {
+      const int* gi = a.idx + tp0 * a.R;
+      const float* gl = a.lam + tp0 * 3;
+      const int* gc = a.count + tp0;
+      const int ni = np * a.R, nl = np * 3;
+      for (int i0 = 0; i0 < ni + nl + np; i0 += 2 * kFsBatch * kFsThreads) {
+        uint32_t v[2 * kFsBatch];
+#pragma unroll
+        for (int u = 0; u < 2 * kFsBatch; ++u) {
+          const int i = i0 + u * kFsThreads + (int)threadIdx.x;
+          v[u] = i < ni ? (uint32_t)gi[i] : i < ni + nl ? __float_as_uint(gl[i - ni]) : i < ni + nl + np ? (uint32_t)gc[i - ni - nl] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 2 * kFsBatch; ++u) {
+          const int i = i0 + u * kFsThreads + (int)threadIdx.x;
+          if (i < ni) sidx[i] = (uint16_t)v[u];
+          else if (i < ni + nl) slam[i - ni] = __uint_as_float(v[u]);
+          else if (i < ni + nl + np) scnt[i - ni - nl] = (uint16_t)min((int)v[u], 65535);
+        }
+      }
+    }
+    __syncthreads();
+    const int j = jp + bl;
+    if (j >= J1) continue;
     const int r0 = j * a.blk, nr = min(a.blk, a.S - r0);
-    // EMA value at this group's first row: the block's carry advanced over the preceding groups
-    const float* cp = a.carry + ((size_t)bi * (a.nblk + 1) + j) * a.width + c;
-    float4 ma = *(const float4*)cp, mb = *(const float4*)(cp + 4);
     int ra, rb;
     if (j < a.nblk) {
       group_rows(rg, a.blk, ra, rb);
-      for (int g = 0; g < rg; ++g) {
-        int ga, gb;
-        group_rows(g, a.blk, ga, gb);
-        float ap = 1.f;
-        for (int i = ga; i < gb; ++i) ap *= al;
-        const float* ge = a.gend + (((size_t)bi * a.nblk + j) * kRG + g) * a.width + c;
-        ma = f4_add(f4_scale(ap, ma), *(const float4*)ge);
-        mb = f4_add(f4_scale(ap, mb), *(const float4*)(ge + 4));
-      }
     } else {  // the unfinished last block: one group walks all its rows
       ra = 0;
       rb = rg == 0 ? nr : 0;
     }
-    float m2[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
     const size_t tg0 = (size_t)bi * a.S + r0;
+    const int prow0 = r0 - pr0;  // this block's first row within the pass
     OutT* dst = (OutT*)(is_k ? a.k_out : a.v_out) + (size_t)bi * a.kv_bstride + (size_t)r0 * a.dkv +
                 (is_k ? c : c - a.dkv);
-    auto fetch = [&](int r, FsRow& f) {
+    // projected rows streamed two ahead of their use (the first two issued before the carry)
+    float4 xa[2], xb[2], na[2], nb[2];
+    auto fetch = [&](int r, float4& fa, float4& fb) {
       if (r < rb) {
-        const size_t t = tg0 + r;
-        const float* xp = a.xkv + t * a.ld + c;
-        f.xa = __ldcs((const float4*)xp);
-        f.xb = __ldcs((const float4*)(xp + 4));
-        f.cnt = __ldg(a.count + t);
-        f.l0 = __ldg(a.lam + t * 3);
-        f.l1 = __ldg(a.lam + t * 3 + 1);
-        f.l2 = __ldg(a.lam + t * 3 + 2);
+        const float* xp = a.xkv + (tg0 + r) * a.ld + c;
+        fa = __ldcs((const float4*)xp);
+        fb = __ldcs((const float4*)(xp + 4));
       }
     };
-    FsRow cur[2], nxt[2];
-    fetch(ra, cur[0]);
-    fetch(ra + 1, cur[1]);
+    fetch(ra, xa[0], xb[0]);
+    fetch(ra + 1, xa[1], xb[1]);
+    // EMA value at this group's first row: the block's carry advanced over the preceding groups
+    const float* cp = a.carry + ((size_t)bi * (a.nblk + 1) + j) * a.width + c;
+    float4 ma = *(const float4*)cp, mb = *(const float4*)(cp + 4);
+    if (j < a.nblk) {
+#pragma unroll
+      for (int g = 0; g < kRG - 1; ++g) {
+        if (g < rg) {
+          int ga, gb;
+          group_rows(g, a.blk, ga, gb);
+          float ap = 1.f;
+          for (int i = ga; i < gb; ++i) ap *= al;
+          const float* ge = a.gend + (((size_t)bi * a.nblk + j) * kRG + g) * a.width + c;
+          ma = f4_add(f4_scale(ap, ma), *(const float4*)ge);
+          mb = f4_add(f4_scale(ap, mb), *(const float4*)(ge + 4));
+        }
+      }
+    }
+    float m2[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
     for (int r = ra; r < rb; r += 2) {
-      fetch(r + 2, nxt[0]);
-      fetch(r + 3, nxt[1]);
+      fetch(r + 2, na[0], nb[0]);
+      fetch(r + 3, na[1], nb[1]);
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         if (r + u < rb) {
-          const FsRow& f = cur[u];
-          const size_t t = tg0 + r + u;
+          const int pr = prow0 + r + u;
+          const int cnt = scnt[pr];
+          const uint16_t* ip = sidx + (size_t)pr * a.R;
           float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          const int* ip = a.idx + t * a.R;
-          for (int q = 0; q < f.cnt; ++q) {
-            const int jq = __ldg(ip + q);
-            if ((unsigned)jq < (unsigned)nstage) Staged8<ST>::add(smean + jq * kFsCols + cs, acc);
+#pragma unroll 4
+          for (int q = 0; q < cnt; ++q) {
+            const int jq = ip[q];
+            if (jq < nstage) Staged8<ST>::add(smean + jq * kFsCols + cs, acc);
           }
-          const float s3 = f.cnt ? f.l2 / (float)f.cnt : 0.f;
-          const float x[8] = {f.xa.x, f.xa.y, f.xa.z, f.xa.w, f.xb.x, f.xb.y, f.xb.z, f.xb.w};
+          const float l0 = slam[pr * 3], l1 = slam[pr * 3 + 1], l2 = slam[pr * 3 + 2];
+          const float s3 = cnt ? l2 / (float)cnt : 0.f;
+          const float x[8] = {xa[u].x, xa[u].y, xa[u].z, xa[u].w, xb[u].x, xb[u].y, xb[u].z, xb[u].w};
           float o[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            o[i] = fmaf(f.l0, x[i], fmaf(f.l1, m2[i], s3 * acc[i]));
+            o[i] = fmaf(l0, x[i], fmaf(l1, m2[i], s3 * acc[i]));
             m2[i] = fmaf(al, m2[i], om * x[i]);
           }
           store8<OutT>(dst + (size_t)(r + u) * a.dkv, o);
         }
       }
-      cur[0] = nxt[0];
-      cur[1] = nxt[1];
+      xa[0] = na[0];
+      xb[0] = nb[0];
+      xa[1] = na[1];
+      xb[1] = nb[1];
     }
     if (r0 + rb == a.S && rb > ra && a.state_ema) {
       float* se = a.state_ema + (size_t)bi * a.width + c;
@@ -677,18 +731,22 @@ __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, 
   }
 }
 
-// Shared-memory bytes of the staged fuse (0: it does not apply, use fuse_kernel).
+// Shared-memory bytes of the staged fuse (0: it does not apply, use fuse_kernel): the means of
+// every block, then one pass's recalled indices, gates and counts.
 size_t fuse_staged_smem(const FuseArgs& a) {
-  if (a.v2_out || a.width % kFsCols || a.dkv % kFsCols) return 0;
-  const size_t b = (size_t)a.nblk * kFsCols * (a.out_bf16 ? 2 : 4);
-  return b <= kFsMaxSmem ? (b > 16 ? b : 16) : 0;
+  if (a.v2_out || a.width % kFsCols || a.dkv % kFsCols || a.nblk > 65535) return 0;
+  const size_t prows = (size_t)kFsBlocks * a.blk;
+  const size_t means = ((size_t)a.nblk * kFsCols * (a.out_bf16 ? 2 : 4) + 15) & ~(size_t)15;
+  const size_t rows = (((prows * a.R + 7) & ~(size_t)7) * 2) + prows * 3 * 4 + prows * 2;
+  const size_t b = means + rows;
+  return b <= kFsMaxSmem ? b : 0;
 }
 
 cudaError_t fuse_kv(const FuseArgs& a, cudaStream_t s) {
   if (a.B <= 0 || a.S <= 0) return cudaSuccess;
   int nb_all = (a.S + a.blk - 1) / a.blk;
   if (const size_t fsm = fuse_staged_smem(a)) {
-    // many short CTAs (two passes of kFsBlocks blocks of one column slice each) balance the SMs;
+    // many short CTAs (one pass of kFsBlocks blocks of one column slice each) balance the SMs;
     // two are resident per SM, so one stages while the other streams
     const int slices = a.width / kFsCols;
     const int bpc = kFsBlocksPerCta;
