@@ -248,6 +248,12 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)_
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
 }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(src));
+}
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N> __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 __device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
@@ -574,8 +580,20 @@ struct TokenDecision {
   int idx[64];
 };
 
+// Values of one sequence's token update that do not depend on the step's projection row, loaded
+// by a token CTA into shared memory before phase A (batch 1): the block codes and this CTA's
+// slices of the EMA state, the block sums, the d_model-space block sum and x_new.
+struct TokenPrefetch {
+  const uint32_t* bc;  // [maxblk] block codes
+  const float* ema;    // [c1 - c0]
+  const float* bsum;   // [c1 - c0]
+  const double* bx;    // [i1 - i0]
+  const bf16* xn;      // [i1 - i0]
+};
+
 template <typename T>
-__device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, TokenDecision* td) {
+__device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, TokenDecision* td,
+                             const TokenPrefetch* pf = nullptr) {
   __shared__ float s_red[32][3];
   __shared__ unsigned s_code;
   __shared__ int s_base[34], s_run[34];
@@ -631,7 +649,7 @@ __device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, T
   }
   // recall among the finished blocks: counting select by (distance, index)
   const int n_elig = min(pos / a.blk, a.maxblk);
-  const uint32_t* bc = a.scode + (size_t)bi * a.maxblk;
+  const uint32_t* bc = pf ? pf->bc : a.scode + (size_t)bi * a.maxblk;
   if (warp == 0) {
     const uint32_t code = s_code;
     for (int i = lane; i < 34; i += 32) {
@@ -676,7 +694,7 @@ __device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, T
 // at the start of a block (pos % b == 0) starts the block sums from zero.
 template <typename T>
 __device__ void token_slice(const DecodeArgs& a, const int bi, const int pos, const TokenDecision* td, const int c0,
-                            const int c1, const int i0, const int i1) {
+                            const int c1, const int i0, const int i1, const TokenPrefetch* pf = nullptr) {
   const int width = 2 * a.dkv;
   const float* xkv = a.y + (size_t)bi * a.Ntot + a.dq;
   const T* xn = (const T*)a.x_new + (size_t)bi * a.d;
@@ -689,17 +707,25 @@ __device__ void token_slice(const DecodeArgs& a, const int bi, const int pos, co
   float* bsum = a.blk_sum + (size_t)bi * width;
   for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
     const float xv = xkv[c];
-    const float m2 = ema[c];
+    const float m2 = pf ? pf->ema[c - c0] : ema[c];
+    // the recalled summaries' loads are independent: issued eight at a time
     float m3 = 0.f;
-    for (int r = 0; r < cnt; ++r) m3 += summ[(size_t)td->idx[r] * width + c];
+    for (int r0 = 0; r0 < cnt; r0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = r0 + u < cnt ? summ[(size_t)td->idx[r0 + u] * width + c] : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) m3 += v[u];
+    }
     const float o = fmaf(l0, xv, fmaf(l1, m2, l2 * s3 * m3));
     T* dst = (T*)(c < a.dkv ? a.kcache : a.vcache) + ((size_t)bi * a.Lmax + pos) * a.dkv + (c < a.dkv ? c : c - a.dkv);
     *dst = from_f<T>(o);
     ema[c] = fmaf(a.alpha, m2, (1.f - a.alpha) * xv);
-    bsum[c] = (fresh ? 0.f : bsum[c]) + xv;
+    bsum[c] = (fresh ? 0.f : (pf ? pf->bsum[c - c0] : bsum[c])) + xv;
   }
   double* bx = a.blk_x + (size_t)bi * a.d;
-  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) bx[i] = (fresh ? 0.0 : bx[i]) + to_d<T>(xn[i]);
+  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x)
+    bx[i] = (fresh ? 0.0 : (pf ? pf->bx[i - i0] : bx[i])) + to_d<T>(pf ? (T)pf->xn[i - i0] : xn[i]);
 }
 
 // ---------------------------------------------------------------- fused decode step (bf16)
@@ -718,6 +744,9 @@ __device__ void token_slice(const DecodeArgs& a, const int bi, const int pos, co
 // time limit that records MKA_ERR_DEVICE_TIMEOUT.  All CTAs are co-resident (cooperative
 // launch), so the barrier cannot deadlock on scheduling.  A CTA whose wait ran out leaves
 // the step.
+// the token CTAs' prefetch area (batch 1): block codes, EMA and block-sum slices, d_model slices
+constexpr int kPfCodes = 2048, kPfCols = 256, kPfD = 128;
+constexpr size_t kPfBytes = (size_t)kPfCodes * 4 + 2 * kPfCols * 4 + kPfD * (8 + 2);
 constexpr int kFusedRing = 2 * 2 * dk::NWD * dk::TP * 128 * 2;  // 64 KB: GEMV chunks, then K/V tiles
 static_assert(kFusedRing >= dk::NWD * 16 * 128 * 4, "attention merge scratch must fit the ring");
 
@@ -781,14 +810,34 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) 
 
 constexpr int kMaxSplits = 512;
 
+// Block-wide (sum, max) of a pair of values in one pass (blockDim.x <= 1024).
+__device__ __forceinline__ float2 block_reduce_sum_max(float s, float m, float2* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = make_float2(s, m);
+  __syncthreads();
+  float2 t = red[0];
+  for (int w = 1; w < nw; ++w) t = make_float2(t.x + red[w].x, fmaxf(t.y, red[w].y));
+  return t;
+}
+
+constexpr int kMergeBatch = 16;  // splits whose o a warp holds in registers at a time
+
 // Combines the split partials (unnormalised o, m in log2 units, l) of (sequence bi, query head
-// hq) and, when the step appended a row at pos_old, that row's own term.  The splits are
-// shared out over the warps (16-byte loads of o, independent across splits), then summed over
-// the warps in a fixed order: deterministic.
+// hq) and, when the step appended a row at pos_old, that row's own term.  Every load that needs
+// no reduction goes out first (the new row's terms, each split's m and l, a warp's first
+// kMergeBatch splits' o); the splits are shared out over the warps (16-byte loads of o), then
+// summed over the warps in a fixed order: deterministic.
 template <int DH>
 __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, const int pos_old) {
   __shared__ float s_w[kMaxSplits];
   __shared__ float red[32];
+  __shared__ float2 red2[32];
   __shared__ float4 s_acc[dk::NWD][DH / 4];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int rec = part_rec(DH);
@@ -802,40 +851,47 @@ __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, cons
   if (has_new)
     for (int c = tid; c < DH; c += blockDim.x)
       s = fmaf(__bfloat162float(__float2bfloat16_rn(__ldcg(q + c))), __bfloat162float(kn[c]), s);
-  const float snew = block_reduce(s, false, red) * a.scale * 1.4426950408889634f;
-  float mloc = has_new ? snew : -INFINITY;
+  float mloc = -INFINITY, lfirst = 0.f;
   for (int sp = tid; sp < a.nsplit; sp += blockDim.x) {
     const float m = __ldcg(pr + (size_t)sp * rec + DH);
+    if (sp == tid) lfirst = __ldcg(pr + (size_t)sp * rec + DH + 1);
     s_w[sp] = m;
     mloc = fmaxf(mloc, m);
   }
-  const float M = block_reduce(mloc, true, red);
+  float4 ov[kMergeBatch];
+  const bool olane = lane < DH / 4;
+#pragma unroll
+  for (int i = 0; i < kMergeBatch; ++i) {
+    const int sp = warp + i * dk::NWD;
+    ov[i] = olane && sp < a.nsplit ? __ldcg((const float4*)(pr + (size_t)sp * rec) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float2 sm = block_reduce_sum_max(s, mloc, red2);
+  const float snew = sm.x * a.scale * 1.4426950408889634f;
+  const float M = has_new ? fmaxf(sm.y, snew) : sm.y;
   float lloc = 0.f;
   for (int sp = tid; sp < a.nsplit; sp += blockDim.x) {
     const float m = s_w[sp];
     const float w = m == -INFINITY ? 0.f : exp2f(m - M);
     s_w[sp] = w;
-    lloc += w * __ldcg(pr + (size_t)sp * rec + DH + 1);
+    lloc += w * (sp == tid ? lfirst : __ldcg(pr + (size_t)sp * rec + DH + 1));
   }
   const float wn = has_new ? exp2f(snew - M) : 0.f;
   const float Ls = block_reduce(lloc, false, red) + wn;  // also orders the s_w writes before the reads below
   const float inv = 1.f / Ls;
-  if (lane < DH / 4) {
-    float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-    int sp = warp;
-    for (; sp + dk::NWD < a.nsplit; sp += 2 * dk::NWD) {
-      const float4 v0 = __ldcg((const float4*)(pr + (size_t)sp * rec) + lane);
-      const float4 v1 = __ldcg((const float4*)(pr + (size_t)(sp + dk::NWD) * rec) + lane);
-      const float w0 = s_w[sp], w1 = s_w[sp + dk::NWD];
-      acc0 = make_float4(fmaf(v0.x, w0, acc0.x), fmaf(v0.y, w0, acc0.y), fmaf(v0.z, w0, acc0.z), fmaf(v0.w, w0, acc0.w));
-      acc1 = make_float4(fmaf(v1.x, w1, acc1.x), fmaf(v1.y, w1, acc1.y), fmaf(v1.z, w1, acc1.z), fmaf(v1.w, w1, acc1.w));
+  if (olane) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kMergeBatch; ++i) {
+      const int sp = warp + i * dk::NWD;
+      const float w = sp < a.nsplit ? s_w[sp] : 0.f;
+      acc = make_float4(fmaf(ov[i].x, w, acc.x), fmaf(ov[i].y, w, acc.y), fmaf(ov[i].z, w, acc.z), fmaf(ov[i].w, w, acc.w));
     }
-    if (sp < a.nsplit) {
-      const float4 v0 = __ldcg((const float4*)(pr + (size_t)sp * rec) + lane);
-      const float w0 = s_w[sp];
-      acc0 = make_float4(fmaf(v0.x, w0, acc0.x), fmaf(v0.y, w0, acc0.y), fmaf(v0.z, w0, acc0.z), fmaf(v0.w, w0, acc0.w));
+    for (int sp = warp + kMergeBatch * dk::NWD; sp < a.nsplit; sp += dk::NWD) {  // more splits than a batch
+      const float4 v = __ldcg((const float4*)(pr + (size_t)sp * rec) + lane);
+      const float w = s_w[sp];
+      acc = make_float4(fmaf(v.x, w, acc.x), fmaf(v.y, w, acc.y), fmaf(v.z, w, acc.z), fmaf(v.w, w, acc.w));
     }
-    s_acc[warp][lane] = make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
+    s_acc[warp][lane] = acc;
   }
   __syncthreads();
   if (tid < DH / 4) {
@@ -879,6 +935,36 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
     }
     for (int i = tid; i < a.B * a.d / 8; i += blockDim.x) ((uint4*)sx)[i] = ((const uint4*)a.x_new)[i];
     __syncthreads();
+  }
+
+  // Batch 1: a token CTA copies what its token update reads from the state (not from this step's
+  // projection row) into shared memory while phase A runs (cp.async: the thread does not wait)
+  const int ntok = min((int)nblk, 32);
+  const int width = 2 * a.dkv;
+  const int cpc = (width + ntok - 1) / ntok;  // fused columns per token CTA
+  const int dpc = (a.d + ntok - 1) / ntok;    // d_model elements per token CTA
+  const bool tok_pf = reg_gemv && (int)blockIdx.x < ntok && a.maxblk <= kPfCodes && cpc <= kPfCols && dpc <= kPfD &&
+                      (dpc & 1) == 0;
+  TokenPrefetch pf{};
+  if (tok_pf) {
+    uint8_t* pfa = smem + kFusedRing + (((size_t)a.B * a.d * 2 + 15) & ~(size_t)15) + 64;
+    uint32_t* pbc = (uint32_t*)pfa;
+    float* pema = (float*)(pbc + kPfCodes);
+    float* pbs = pema + kPfCols;
+    double* pbx = (double*)(pbs + kPfCols);
+    bf16* pxn = (bf16*)(pbx + kPfD);
+    const int c0 = min(width, (int)blockIdx.x * cpc), c1 = min(width, c0 + cpc);
+    const int i0 = min(a.d, (int)blockIdx.x * dpc), i1 = min(a.d, i0 + dpc);
+    for (int k = tid; k < a.maxblk; k += blockDim.x) dk::cp_async4(dk::smem_u32(pbc + k), a.scode + k);
+    for (int k = tid; k < c1 - c0; k += blockDim.x) {
+      dk::cp_async4(dk::smem_u32(pema + k), a.ema + c0 + k);
+      dk::cp_async4(dk::smem_u32(pbs + k), a.blk_sum + c0 + k);
+    }
+    for (int k = tid; k < i1 - i0; k += blockDim.x) dk::cp_async8(dk::smem_u32(pbx + k), a.blk_x + i0 + k);
+    for (int k = 2 * tid; k < i1 - i0; k += 2 * blockDim.x)
+      dk::cp_async4(dk::smem_u32(pxn + k), (const bf16*)a.x_new + i0 + k);
+    dk::cp_commit();
+    pf = TokenPrefetch{pbc, pema, pbs, pbx, pxn};
   }
 
   // ---- A: projection row, this CTA's share of the packed weight rows
@@ -1009,12 +1095,12 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
       __syncthreads();  // stage (c & 1) is free for chunk c + 2
     }
   }
+  if (tok_pf) dk::cp_wait<0>();  // the prefetched values, visible to the CTA after the barrier
   if (!grid_sync(a.sync, nblk, a.status)) return;
 
   // ---- B: split-KV attention over the old rows (units handed out from CTA ntok on), and the
   // token update, split over the first ntok CTAs
   {
-    const int ntok = min((int)nblk, 32);
     const int units = a.B * a.Hkv * a.nsplit;
     for (int u = ((int)blockIdx.x - ntok + (int)nblk) % (int)nblk; u < units; u += nblk) {
       const int split = u % a.nsplit, g = (u / a.nsplit) % a.Hkv, bi = u / (a.nsplit * a.Hkv);
@@ -1022,9 +1108,6 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
     }
     if ((int)blockIdx.x < ntok) {
       __shared__ TokenDecision td;
-      const int width = 2 * a.dkv;
-      const int cpc = (width + ntok - 1) / ntok;  // fused columns per CTA
-      const int dpc = (a.d + ntok - 1) / ntok;    // d_model elements per CTA
       for (int bi = 0; bi < a.B; ++bi) {
         const int pos = s_pos[bi];
         if (pos < 0 || pos >= a.Lmax) {
@@ -1033,8 +1116,8 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
         }
         const int c0 = min(width, (int)blockIdx.x * cpc), c1 = min(width, c0 + cpc);
         const int i0 = min(a.d, (int)blockIdx.x * dpc), i1 = min(a.d, i0 + dpc);
-        token_decide<bf16>(a, bi, pos, &td);
-        token_slice<bf16>(a, bi, pos, &td, c0, c1, i0, i1);
+        token_decide<bf16>(a, bi, pos, &td, tok_pf ? &pf : nullptr);
+        token_slice<bf16>(a, bi, pos, &td, c0, c1, i0, i1, tok_pf ? &pf : nullptr);
         __syncthreads();
       }
       if (blockIdx.x == 0 && threadIdx.x < a.B && s_pos[threadIdx.x] < a.Lmax)
@@ -1074,7 +1157,9 @@ __global__ void __launch_bounds__(dk::NWD * 32, 2) decode_fused_kernel(DecodeArg
   decode_fused_body<DH>(a);
 }
 
-size_t decode_fused_smem(int B, int d) { return kFusedRing + (((size_t)B * d * 2 + 15) & ~(size_t)15) + 64; }
+size_t decode_fused_smem(int B, int d) {
+  return kFusedRing + (((size_t)B * d * 2 + 15) & ~(size_t)15) + 64 + (B == 1 ? kPfBytes : 0);
+}
 
 cudaError_t decode_step(const DecodeArgs& a, cudaStream_t s) {
   if (a.B <= 0) return cudaSuccess;
