@@ -132,10 +132,13 @@ def decode_bytes_per_token(cfg, ctx: int, ntot: int) -> float:
 
 
 def workload_cfg(args, name):
-    """The named workload with the routing gate / memory tiers the command line selects."""
-    return CONFIGS[name].replace(route_mode=args.route, tiers=args.tiers,
-                                 attention_paths=getattr(args, "paths", 1),
-                                 block_sparse=int(getattr(args, "block_sparse", False)))
+    """The named workload with the routing gate / memory tiers the command line selects (and, for
+    profiling runs, another sequence length of the same shape)."""
+    c = CONFIGS[name].replace(route_mode=args.route, tiers=args.tiers,
+                              attention_paths=getattr(args, "paths", 1),
+                              block_sparse=int(getattr(args, "block_sparse", False)))
+    seq = getattr(args, "seq", None)
+    return c.replace(seq=seq) if seq and name == args.workload else c
 
 
 def model_name(cfg) -> str:
@@ -763,6 +766,8 @@ def main():
     ap.add_argument("--cpu-prefix", type=int, default=8192, help="tokens of the oracle's prefix sample (main arm)")
     ap.add_argument("--ref-prefix", type=int, default=2048, help="tokens of each reference-arm step's prefix sample")
     ap.add_argument("--no-recall-check", dest="recall_check", action="store_false")
+    ap.add_argument("--seq", type=int, default=None,
+                    help="profiling: run the headline workload's shape at this sequence length instead")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.workload is None:

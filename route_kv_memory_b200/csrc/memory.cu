@@ -538,14 +538,13 @@ template <> struct Staged8<bf16> {
     __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x * sc, b.y * sc), h3 = __floats2bfloat162_rn(b.z * sc, b.w * sc);
     *(uint4*)p = make_uint4(*(uint32_t*)&h0, *(uint32_t*)&h1, *(uint32_t*)&h2, *(uint32_t*)&h3);
   }
-  static __device__ __forceinline__ void add(const bf16* p, float* acc) {
+  // bf16 pair -> two floats by a shift and a mask; packed FP32x2 adds
+  static __device__ __forceinline__ void add(const bf16* p, float2* acc) {
     const uint4 u = *(const uint4*)p;
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[2 * i] += __uint_as_float(w[i] << 16);
-      acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
-    }
+    for (int i = 0; i < 4; ++i)
+      acc[i] = __fadd2_rn(acc[i], make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u)));
   }
 };
 template <> struct Staged8<float> {
@@ -553,10 +552,12 @@ template <> struct Staged8<float> {
     *(float4*)p = f4_scale(sc, a);
     *(float4*)(p + 4) = f4_scale(sc, b);
   }
-  static __device__ __forceinline__ void add(const float* p, float* acc) {
+  static __device__ __forceinline__ void add(const float* p, float2* acc) {
     const float4 a = *(const float4*)p, b = *(const float4*)(p + 4);
-    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    acc[0] = __fadd2_rn(acc[0], make_float2(a.x, a.y));
+    acc[1] = __fadd2_rn(acc[1], make_float2(a.z, a.w));
+    acc[2] = __fadd2_rn(acc[2], make_float2(b.x, b.y));
+    acc[3] = __fadd2_rn(acc[3], make_float2(b.z, b.w));
   }
 };
 
@@ -575,12 +576,27 @@ template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v
   *(uint4*)p = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Shared memory of one CTA: the staged means, then the pass's recalled indices (16-bit), counts
-// and gates.
+// Shared memory of one CTA: the staged means of every block, then one ring per row group of
+// kFsDepth rows in flight: the projected columns of its 8 lanes and the row's recalled indices,
+// gates and count (cp.async, no registers held while the copies fly).
+constexpr int kFsDepth = 4;
+constexpr int kFsGroups = kFsThreads / kFsLanes;  // row groups of a CTA
 template <typename ST>
-__device__ __forceinline__ size_t fs_mean_bytes(int nstage) {
-  return ((size_t)nstage * kFsCols * sizeof(ST) + 15) & ~(size_t)15;
+__host__ __device__ __forceinline__ size_t fs_mean_bytes(int nblk) {
+  return ((size_t)nblk * kFsCols * sizeof(ST) + 15) & ~(size_t)15;
 }
+__host__ __device__ __forceinline__ int fs_meta(int R) { return (R + 4 + 3) & ~3; }  // idx[R], lam[3], cnt
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <typename OutT, typename ST>
 __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, int blocks_per_cta) {
@@ -591,14 +607,12 @@ __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, 
   if (J0 >= J1) return;
   const int nstage = min(J1 - 1, a.nblk);  // a token of block j recalls blocks < j only
   ST* smean = (ST*)fs_smem;                // [nstage][kFsCols] block means of this slice
-  const int prows = kFsBlocks * a.blk;     // rows of one pass
-  uint16_t* sidx = (uint16_t*)(fs_smem + fs_mean_bytes<ST>(nstage));  // [prows][R]
-  float* slam = (float*)(sidx + (((size_t)prows * a.R + 7) & ~(size_t)7));  // [prows][3]
-  uint16_t* scnt = (uint16_t*)(slam + (size_t)prows * 3);                  // [prows]
+  const int meta = fs_meta(a.R);
+  float* ring_x = (float*)(fs_smem + fs_mean_bytes<ST>(a.nblk));        // [groups][depth][kFsCols]
+  uint32_t* ring_m = (uint32_t*)(ring_x + kFsGroups * kFsDepth * kFsCols);  // [groups][depth][meta]
   const float invb = 1.f / (float)a.blk;
   const float* bs = a.bsum + (size_t)bi * a.bsum_bstride + c0;
-  // staging loads are batched (kFsBatch per thread in flight before any store): one L2 round
-  // trip per batch instead of one per element
+  // staging loads are batched (kFsBatch per thread in flight before any store)
   for (int i0 = 0; i0 < nstage * kFsLanes; i0 += kFsBatch * kFsThreads) {
     float4 va[kFsBatch], vb[kFsBatch];
 #pragma unroll
@@ -617,39 +631,16 @@ __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, 
         Staged8<ST>::put(smean + (i / kFsLanes) * kFsCols + (i % kFsLanes) * kFsLaneCols, va[u], vb[u], invb);
     }
   }
-  const int lane = threadIdx.x % kFsLanes, rg = (threadIdx.x / kFsLanes) % kRG, bl = threadIdx.x / (kFsLanes * kRG);
+  __syncthreads();
+  const int lane = threadIdx.x % kFsLanes, gid = threadIdx.x / kFsLanes;
+  const int rg = gid % kRG, bl = gid / kRG;
+  const unsigned gmask = 0xffu << (8 * (gid & 3));  // this group's 8 lanes within the warp
   const int cs = lane * kFsLaneCols, c = c0 + cs;
   const bool is_k = c < a.dkv;
   const float al = a.alpha, om = 1.f - a.alpha;
-  for (int jp = J0; jp < J1; jp += kFsBlocks) {
-    // this pass's rows: their recalled indices, counts and gates, staged once for all columns
-    const int pr0 = jp * a.blk, pr1 = min(a.S, min(J1, jp + kFsBlocks) * a.blk), np = pr1 - pr0;
-    const size_t tp0 = (size_t)bi * a.S + pr0;
-    __syncthreads();  // the previous pass is done with the staged rows
-    {
-      const int* gi = a.idx + tp0 * a.R;
-      const float* gl = a.lam + tp0 * 3;
-      const int* gc = a.count + tp0;
-      const int ni = np * a.R, nl = np * 3;
-      for (int i0 = 0; i0 < ni + nl + np; i0 += 2 * kFsBatch * kFsThreads) {
-        uint32_t v[2 * kFsBatch];
-#pragma unroll
-        for (int u = 0; u < 2 * kFsBatch; ++u) {
-          const int i = i0 + u * kFsThreads + (int)threadIdx.x;
-          v[u] = i < ni ? (uint32_t)gi[i] : i < ni + nl ? __float_as_uint(gl[i - ni]) : i < ni + nl + np ? (uint32_t)gc[i - ni - nl] : 0u;
-        }
-#pragma unroll
-        for (int u = 0; u < 2 * kFsBatch; ++u) {
-          const int i = i0 + u * kFsThreads + (int)threadIdx.x;
-          if (i < ni) sidx[i] = (uint16_t)v[u];
-          else if (i < ni + nl) slam[i - ni] = __uint_as_float(v[u]);
-          else if (i < ni + nl + np) scnt[i - ni - nl] = (uint16_t)min((int)v[u], 65535);
-        }
-      }
-    }
-    __syncthreads();
-    const int j = jp + bl;
-    if (j >= J1) continue;
+  float* gx = ring_x + (size_t)gid * kFsDepth * kFsCols;
+  uint32_t* gm = ring_m + (size_t)gid * kFsDepth * meta;
+  for (int j = J0 + bl; j < J1; j += kFsBlocks) {
     const int r0 = j * a.blk, nr = min(a.blk, a.S - r0);
     int ra, rb;
     if (j < a.nblk) {
@@ -659,20 +650,28 @@ __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, 
       rb = rg == 0 ? nr : 0;
     }
     const size_t tg0 = (size_t)bi * a.S + r0;
-    const int prow0 = r0 - pr0;  // this block's first row within the pass
     OutT* dst = (OutT*)(is_k ? a.k_out : a.v_out) + (size_t)bi * a.kv_bstride + (size_t)r0 * a.dkv +
                 (is_k ? c : c - a.dkv);
-    // projected rows streamed two ahead of their use (the first two issued before the carry)
-    float4 xa[2], xb[2], na[2], nb[2];
-    auto fetch = [&](int r, float4& fa, float4& fb) {
+    // row r into ring slot (r - ra) % kFsDepth: each lane its 8 columns, the indices, gates and
+    // count shared out over the 8 lanes
+    auto issue = [&](int r) {
       if (r < rb) {
-        const float* xp = a.xkv + (tg0 + r) * a.ld + c;
-        fa = __ldcs((const float4*)xp);
-        fb = __ldcs((const float4*)(xp + 4));
+        const size_t t = tg0 + r;
+        const int slot = (r - ra) % kFsDepth;
+        const float* xp = a.xkv + t * a.ld + c;
+        cp_async16(gx + slot * kFsCols + cs, xp);
+        cp_async16(gx + slot * kFsCols + cs + 4, xp + 4);
+        uint32_t* m = gm + slot * meta;
+        for (int k = lane; k < a.R + 4; k += kFsLanes) {
+          const void* src = k < a.R ? (const void*)(a.idx + t * a.R + k)
+                            : k < a.R + 3 ? (const void*)(a.lam + t * 3 + (k - a.R)) : (const void*)(a.count + t);
+          cp_async4(m + k, src);
+        }
       }
+      cp_commit();  // one group per row (empty past the end), so the waits below count rows
     };
-    fetch(ra, xa[0], xb[0]);
-    fetch(ra + 1, xa[1], xb[1]);
+#pragma unroll
+    for (int d = 0; d < kFsDepth; ++d) issue(ra + d);
     // EMA value at this group's first row: the block's carry advanced over the preceding groups
     const float* cp = a.carry + ((size_t)bi * (a.nblk + 1) + j) * a.width + c;
     float4 ma = *(const float4*)cp, mb = *(const float4*)(cp + 4);
@@ -691,38 +690,35 @@ __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, 
       }
     }
     float m2[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
-    for (int r = ra; r < rb; r += 2) {
-      fetch(r + 2, na[0], nb[0]);
-      fetch(r + 3, na[1], nb[1]);
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (r + u < rb) {
-          const int pr = prow0 + r + u;
-          const int cnt = scnt[pr];
-          const uint16_t* ip = sidx + (size_t)pr * a.R;
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int r = ra; r < rb; ++r) {
+      cp_wait<kFsDepth - 1>();  // row r landed (this lane's copies)
+      __syncwarp(gmask);        // and the other lanes' share of its indices
+      const int slot = (r - ra) % kFsDepth;
+      const float* xs = gx + slot * kFsCols + cs;
+      const uint32_t* m = gm + slot * meta;
+      const int cnt = (int)m[a.R + 3];
+      const float l0 = __uint_as_float(m[a.R]), l1 = __uint_as_float(m[a.R + 1]), l2 = __uint_as_float(m[a.R + 2]);
+      float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll 4
-          for (int q = 0; q < cnt; ++q) {
-            const int jq = ip[q];
-            if (jq < nstage) Staged8<ST>::add(smean + jq * kFsCols + cs, acc);
-          }
-          const float l0 = slam[pr * 3], l1 = slam[pr * 3 + 1], l2 = slam[pr * 3 + 2];
-          const float s3 = cnt ? l2 / (float)cnt : 0.f;
-          const float x[8] = {xa[u].x, xa[u].y, xa[u].z, xa[u].w, xb[u].x, xb[u].y, xb[u].z, xb[u].w};
-          float o[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            o[i] = fmaf(l0, x[i], fmaf(l1, m2[i], s3 * acc[i]));
-            m2[i] = fmaf(al, m2[i], om * x[i]);
-          }
-          store8<OutT>(dst + (size_t)(r + u) * a.dkv, o);
-        }
+      for (int q = 0; q < cnt; ++q) {
+        const uint32_t jq = m[q];
+        if (jq < (uint32_t)nstage) Staged8<ST>::add(smean + jq * kFsCols + cs, acc2);
       }
-      xa[0] = na[0];
-      xb[0] = nb[0];
-      xa[1] = na[1];
-      xb[1] = nb[1];
+      const float acc[8] = {acc2[0].x, acc2[0].y, acc2[1].x, acc2[1].y, acc2[2].x, acc2[2].y, acc2[3].x, acc2[3].y};
+      const float4 xa = *(const float4*)xs, xb = *(const float4*)(xs + 4);
+      const float x[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+      const float s3 = cnt ? l2 / (float)cnt : 0.f;
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[i] = fmaf(l0, x[i], fmaf(l1, m2[i], s3 * acc[i]));
+        m2[i] = fmaf(al, m2[i], om * x[i]);
+      }
+      store8<OutT>(dst + (size_t)r * a.dkv, o);
+      __syncwarp(gmask);  // the slot is read by all 8 lanes before it is refilled
+      issue(r + kFsDepth);
     }
+    cp_wait<0>();
     if (r0 + rb == a.S && rb > ra && a.state_ema) {
       float* se = a.state_ema + (size_t)bi * a.width + c;
       *(float4*)se = make_float4(m2[0], m2[1], m2[2], m2[3]);
@@ -731,14 +727,19 @@ __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, 
   }
 }
 
-// Shared-memory bytes of the staged fuse (0: it does not apply, use fuse_kernel): the means of
-// every block, then one pass's recalled indices, gates and counts.
+// Shared-memory bytes of the staged fuse (0: it does not apply, use fuse_kernel).  Staging pays
+// when a token's gather is large: the unstaged kernel reads R * width floats per token from L2
+// (17 GB at 1 x 131072 with R = 16 and width 2048, where it is L2-bound), while the staged one
+// spends about two instructions per gathered element (bf16 unpack and add) and is issue-bound.
+// Measured crossover: staged 1.16 ms against 1.24 at R * width = 32768; unstaged 0.187 ms
+// against 0.217 at R * width = 8192 (2 x 32768 tokens).
+constexpr int kFsMinGather = 16384;
 size_t fuse_staged_smem(const FuseArgs& a) {
-  if (a.v2_out || a.width % kFsCols || a.dkv % kFsCols || a.nblk > 65535) return 0;
-  const size_t prows = (size_t)kFsBlocks * a.blk;
-  const size_t means = ((size_t)a.nblk * kFsCols * (a.out_bf16 ? 2 : 4) + 15) & ~(size_t)15;
-  const size_t rows = (((prows * a.R + 7) & ~(size_t)7) * 2) + prows * 3 * 4 + prows * 2;
-  const size_t b = means + rows;
+  if (a.v2_out || a.width % kFsCols || a.dkv % kFsCols || a.R > 64) return 0;
+  if ((long long)a.R * a.width < kFsMinGather) return 0;
+  const size_t means = a.out_bf16 ? fs_mean_bytes<bf16>(a.nblk) : fs_mean_bytes<float>(a.nblk);
+  const size_t rings = (size_t)kFsGroups * kFsDepth * (kFsCols + fs_meta(a.R)) * 4;
+  const size_t b = means + rings;
   return b <= kFsMaxSmem ? b : 0;
 }
 

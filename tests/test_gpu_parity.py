@@ -54,12 +54,15 @@ EDGE = [
           recall_r=8, hash_bits=32, seed=14),
     small("bf16_b2_s129", "bf16", batch=2, seq=129, n_q_heads=4, n_kv_heads=4, d_head=128, seed=15),
     small("bf16_s1", "bf16", seq=1, d_head=128, seed=16),
-    # more blocks (2000) than the fuse stages in shared memory: the unstaged fuse kernel runs
+    # many small blocks (2000, 850): the fuse gathers from L2 (unstaged kernel)
     small("bf16_blocks_of_1", "bf16", seq=2000, block=1, recall_r=3, hash_bits=8, seed=17),
     small("f32_blocks_of_2_many", "f32", seq=1700, block=2, recall_r=2, hash_bits=6, seed=18),
-    # many staged blocks, several passes per CTA, a ragged last block
-    small("bf16_staged_passes", "bf16", batch=2, seq=1100, d_head=128, n_q_heads=4, n_kv_heads=2, block=16,
-          recall_r=5, hash_bits=12, seed=19),
+    # R * 2 d_kv >= 16384: the fuse stages the block means in shared memory; many blocks, a
+    # ragged last block, two sequences
+    small("bf16_staged_fuse", "bf16", batch=2, seq=1100, d_head=128, n_q_heads=8, n_kv_heads=4, block=16,
+          recall_r=16, hash_bits=12, seed=19),
+    small("f32_staged_fuse", "f32", seq=700, d_head=128, n_q_heads=4, n_kv_heads=4, block=32, recall_r=16,
+          hash_bits=10, seed=20),
 ]
 
 
@@ -444,3 +447,44 @@ def test_bounded_wait_reports_timeout(mka):
     # the context is still usable
     x = torch.ones(4, device="cuda")
     assert float((x * 2).sum().item()) == 8.0
+
+
+def test_block_codes_exact_refinement(mka):
+    """Blocks whose rows cancel in pairs except one small row w: each block sum is exactly w, and w
+    is chosen so that every projection |w . P_k| lies between 5e-3 and 5e-2, inside the float32
+    summation bound of the block-code kernel (rows of size ~100 make it ~0.08) but far above the
+    1e-4 excuse threshold.  Every bit is then decided by the exact float64 recomputation, and the
+    recalled indices must equal the oracle's exactly."""
+    cfg = small("codes_refine", "bf16", seq=256, block=32, recall_r=2, hash_bits=32, seed=90)
+    inp = make_inputs(cfg)
+    g = torch.Generator().manual_seed(91)
+    P = inp.hash_proj.double()
+    b, nblk, d = cfg.block, cfg.seq // cfg.block, cfg.d_model
+    X = torch.zeros(1, cfg.seq, d, dtype=torch.float64)
+    for j in range(nblk):
+        half = (b - 2) // 2
+        xp = (100.0 * torch.randn(half, d, generator=g)).to(torch.bfloat16).double()
+        X[0, j * b:j * b + 2 * half:2] = xp
+        X[0, j * b + 1:j * b + 2 * half:2] = -xp
+        # w with prescribed projections t (signs random, sizes 1e-2 .. 2e-2): w = P (P^T P)^-1 t
+        sgn = torch.randint(0, 2, (cfg.hash_bits,), generator=g).double() * 2 - 1
+        t = sgn * 1e-2 * (1 + torch.rand(cfg.hash_bits, generator=g, dtype=torch.float64))
+        w = (P @ torch.linalg.solve(P.T @ P, t)).to(torch.bfloat16).double()
+        pr = (w @ P).abs()
+        assert pr.min() > 5e-3 and pr.max() < 5e-2, (float(pr.min()), float(pr.max()))
+        X[0, j * b + 2 * half] = w
+    x = X.to(torch.bfloat16)
+    assert torch.equal(x.double(), X)
+    c = mka.make_config(cfg)
+    idx = torch.empty(1, cfg.seq, cfg.recall_r, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(1, cfg.seq, dtype=torch.int32, device="cuda")
+    ws = mka.buffer(mka.mka_longterm_recall_workspace_size(c))
+    mka.mka_longterm_recall(c, x.cuda(), inp.hash_proj.cuda(), idx, cnt, None, ws)
+    torch.cuda.synchronize()
+    assert mka.mka_status() == 0
+    Xn = X[0].numpy()
+    summ = oracle.block_summaries(Xn[None], b)[0]
+    ridx, rcnt, *_ = oracle.longterm_recall(Xn, np.arange(cfg.seq), summ, to_f64(inp.hash_proj), b, cfg.recall_r)
+    assert np.abs(oracle.hash_codes(summ, to_f64(inp.hash_proj))[1]).min() > 1e-4
+    assert np.array_equal(idx[0].cpu().numpy(), ridx), "recall after the exact refinement differs from the oracle"
+    assert np.array_equal(cnt[0].cpu().numpy(), rcnt)
