@@ -217,7 +217,8 @@ def attention_roofline(cfg, attn_ms: float, peaks: dict, clk_max_mhz: float = 19
             "unit": "TFLOP/s", "frac": round(tf / peak, 4),
             "peak_source": f"{peaks['source']} bf16 dense cuBLAS ({how})",
             "frac_of_burst_peak": round(tf / peaks["bf16_tflops"], 4),
-            "traffic": traffic_from_profiles("attention_tc"), "avg_ms": round(attn_ms, 4), "flops_per_launch": fl}
+            "traffic": traffic_from_profiles("attention_tc", cfg.name), "avg_ms": round(attn_ms, 4),
+            "flops_per_launch": fl}
 
 
 def hbm_rooflines(cfg, stage_ms: dict, peaks: dict) -> dict:
@@ -510,7 +511,7 @@ def run_train(args, rank, world, local_rank):
                      "achieved": round(ab_tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(ab_tf / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} bf16 dense (burst, kernel timed per step)",
-                     "traffic": traffic_from_profiles("attention_bwd"),
+                     "traffic": traffic_from_profiles("attention_bwd", cfg.name),
                      "avg_ms": round(ab_ms, 4), "flops_per_launch": fl["attention_bwd"]},
         "layer_tflops": round(sum(fl.values()) / (ms / 1e3) / 1e12, 1),
         "forward_stage_ms": {n: round(float(v), 4) for n, v in zip(PREFILL_STAGES, fw_st)},
@@ -697,9 +698,10 @@ def run_reference(args, rank, world):
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def traffic_from_profiles(kernel: str):
-    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary profiles/traffic.txt,
-    or None when the kernel's source changed after the counters were taken."""
+def traffic_from_profiles(kernel: str, workload: str = None):
+    """DRAM bytes (read + write) per launch of `kernel` at `workload` from the committed ncu summary
+    profiles/traffic.txt; None when there is no capture of that workload or the kernel's source
+    changed after the counters were taken."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
@@ -711,7 +713,8 @@ def traffic_from_profiles(kernel: str):
     with open(os.path.join(ROOT, d["source"]), "rb") as f:
         if hashlib.sha1(f.read()).hexdigest() != d["source_sha1"]:
             return None
-    return d["dram_bytes_per_launch"]
+    per = d["dram_bytes_per_launch"]
+    return per.get(workload) if isinstance(per, dict) else per
 
 
 # ------------------------------------------------------------------ distributed plumbing

@@ -245,6 +245,29 @@ __global__ void __launch_bounds__(1024) token_kernel(DecodeArgs a) {
 // ---------------------------------------------------------------- 3. split-KV attention, bf16 tensor cores
 namespace dk {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+// L2 cache policies: the K/V cache streams through once per step (evict first); the packed weights
+// are read every step (evict last), so they stay in L2 while long caches stream past them.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void* src, int src_bytes, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src), "r"(src_bytes),
+               "l"(pol));
+}
+__device__ __forceinline__ uint4 ldg_nc_hint(const uint4* p, uint64_t pol) {
+  uint4 v;
+  asm("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p), "l"(pol));
+  return v;
+}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
 }
@@ -319,6 +342,7 @@ __device__ void attn_unit(const DecodeArgs& a, const int split, const int g, con
       qf[kk][3] = pack_bf16(w10, w11);
     }
   }
+  const uint64_t pol_kv = l2_evict_first();
   auto load = [&](int stage, int base) {
     for (int i = tid; i < NWD * TP * CH; i += NWD * 32) {
       int w = i / (TP * CH), rem = i % (TP * CH), r = rem / CH, c = rem % CH;
@@ -326,8 +350,10 @@ __device__ void attn_unit(const DecodeArgs& a, const int split, const int g, con
       bool ok = j < p1;
       bf16* k = sK + (stage * NWD + w) * TILE;
       bf16* v = sV + (stage * NWD + w) * TILE;
-      cp_async16(smem_u32(k + swz<DH>(r, c)), ok ? (const void*)(Kp + (size_t)j * a.dkv + c * 8) : (const void*)Kp, ok ? 16 : 0);
-      cp_async16(smem_u32(v + swz<DH>(r, c)), ok ? (const void*)(Vp + (size_t)j * a.dkv + c * 8) : (const void*)Vp, ok ? 16 : 0);
+      cp_async16_hint(smem_u32(k + swz<DH>(r, c)), ok ? (const void*)(Kp + (size_t)j * a.dkv + c * 8) : (const void*)Kp,
+                      ok ? 16 : 0, pol_kv);
+      cp_async16_hint(smem_u32(v + swz<DH>(r, c)), ok ? (const void*)(Vp + (size_t)j * a.dkv + c * 8) : (const void*)Vp,
+                      ok ? 16 : 0, pol_kv);
     }
   };
   const float sl2 = a.scale * 1.4426950408889634f;
@@ -977,6 +1003,7 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
     const uint4* W = (const uint4*)a.wcatT;
     const size_t rowv = (size_t)a.d / 8;
     const uint4* xv = (const uint4*)a.x_new;  // read through L1: every warp reads the same 16 B pieces
+    const uint64_t pol_w = dk::l2_evict_last();
     for (int r = gw; r < a.Ntot; r += 2 * TW) {
       const int r2 = r + TW;
       const bool two = r2 < a.Ntot;
@@ -984,8 +1011,8 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         if (k < kv) {
-          w1[k] = __ldg(W + (size_t)r * rowv + lane + 32 * k);
-          if (two) w2[k] = __ldg(W + (size_t)r2 * rowv + lane + 32 * k);
+          w1[k] = dk::ldg_nc_hint(W + (size_t)r * rowv + lane + 32 * k, pol_w);
+          if (two) w2[k] = dk::ldg_nc_hint(W + (size_t)r2 * rowv + lane + 32 * k, pol_w);
         }
       }
       float a1[2] = {0.f, 0.f}, a2[2] = {0.f, 0.f};

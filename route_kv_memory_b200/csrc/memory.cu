@@ -538,13 +538,17 @@ template <> struct Staged8<bf16> {
     __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x * sc, b.y * sc), h3 = __floats2bfloat162_rn(b.z * sc, b.w * sc);
     *(uint4*)p = make_uint4(*(uint32_t*)&h0, *(uint32_t*)&h1, *(uint32_t*)&h2, *(uint32_t*)&h3);
   }
-  // bf16 pair -> two floats by a shift and a mask; packed FP32x2 adds
+  // sm_100 mixed-precision adds: each bf16 half of a word goes straight into its fp32 sum (the
+  // same round-to-nearest fp32 sum as widening first), one instruction per element
   static __device__ __forceinline__ void add(const bf16* p, float2* acc) {
     const uint4 u = *(const uint4*)p;
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      acc[i] = __fadd2_rn(acc[i], make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u)));
+      asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+          "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+          : "+f"(acc[i].x), "+f"(acc[i].y)
+          : "r"(w[i]));
   }
 };
 template <> struct Staged8<float> {
