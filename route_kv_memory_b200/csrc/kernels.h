@@ -131,6 +131,7 @@ struct AttnArgs {
   // causal mode, when set: each row's softmax normaliser in log2 units, m + log2(l) with the
   // scores taken as scale * log2(e) * q.k, at lse[(b * Hq + h) * lse_ld + t] (for the backward)
   float* lse = nullptr; int lse_ld = 0;
+  int chunk = 1;  // causal mode: (sequence, KV group) streams per chunk of the work order (set by attention_prefill_tc)
   // Block-gathered attention (set g_pairoff to select it; bf16, tcgen05 only).  The rows of a
   // work item are (token, query head) pairs that all attend to the keys of one L3 block j of
   // sequence b: the tokens of block j's list (its own tokens first when g_own, under the causal

@@ -538,10 +538,13 @@ template <> struct Staged8<bf16> {
     __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x * sc, b.y * sc), h3 = __floats2bfloat162_rn(b.z * sc, b.w * sc);
     *(uint4*)p = make_uint4(*(uint32_t*)&h0, *(uint32_t*)&h1, *(uint32_t*)&h2, *(uint32_t*)&h3);
   }
+  // a row's 8 staged columns, loaded before they are added so that several gathers are in flight
+  using V = uint4;
+  static __device__ __forceinline__ V load(const bf16* p) { return *(const uint4*)p; }
+  static __device__ __forceinline__ V zero() { return make_uint4(0, 0, 0, 0); }
   // sm_100 mixed-precision adds: each bf16 half of a word goes straight into its fp32 sum (the
   // same round-to-nearest fp32 sum as widening first), one instruction per element
-  static __device__ __forceinline__ void add(const bf16* p, float2* acc) {
-    const uint4 u = *(const uint4*)p;
+  static __device__ __forceinline__ void accum(V u, float2* acc) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -556,12 +559,16 @@ template <> struct Staged8<float> {
     *(float4*)p = f4_scale(sc, a);
     *(float4*)(p + 4) = f4_scale(sc, b);
   }
-  static __device__ __forceinline__ void add(const float* p, float2* acc) {
-    const float4 a = *(const float4*)p, b = *(const float4*)(p + 4);
-    acc[0] = __fadd2_rn(acc[0], make_float2(a.x, a.y));
-    acc[1] = __fadd2_rn(acc[1], make_float2(a.z, a.w));
-    acc[2] = __fadd2_rn(acc[2], make_float2(b.x, b.y));
-    acc[3] = __fadd2_rn(acc[3], make_float2(b.z, b.w));
+  struct V {
+    float4 a, b;
+  };
+  static __device__ __forceinline__ V load(const float* p) { return {*(const float4*)p, *(const float4*)(p + 4)}; }
+  static __device__ __forceinline__ V zero() { return {make_float4(0, 0, 0, 0), make_float4(0, 0, 0, 0)}; }
+  static __device__ __forceinline__ void accum(const V& v, float2* acc) {
+    acc[0] = __fadd2_rn(acc[0], make_float2(v.a.x, v.a.y));
+    acc[1] = __fadd2_rn(acc[1], make_float2(v.a.z, v.a.w));
+    acc[2] = __fadd2_rn(acc[2], make_float2(v.b.x, v.b.y));
+    acc[3] = __fadd2_rn(acc[3], make_float2(v.b.z, v.b.w));
   }
 };
 
@@ -584,12 +591,14 @@ template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v
 // kFsDepth rows in flight: the projected columns of its 8 lanes and the row's recalled indices,
 // gates and count (cp.async, no registers held while the copies fly).
 constexpr int kFsDepth = 4;
+constexpr int kFsInflight = 8;  // gathers of one row in flight per lane
 constexpr int kFsGroups = kFsThreads / kFsLanes;  // row groups of a CTA
 template <typename ST>
 __host__ __device__ __forceinline__ size_t fs_mean_bytes(int nblk) {
   return ((size_t)nblk * kFsCols * sizeof(ST) + 15) & ~(size_t)15;
 }
-__host__ __device__ __forceinline__ int fs_meta(int R) { return (R + 4 + 3) & ~3; }  // idx[R], lam[3], cnt
+// idx[R], lam[3], cnt, rounded up to 4 words: at least R rounded up to kFsInflight
+__host__ __device__ __forceinline__ int fs_meta(int R) { return (R + 4 + 3) & ~3; }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
@@ -703,10 +712,22 @@ __global__ void __launch_bounds__(kFsThreads, 2) fuse_staged_kernel(FuseArgs a, 
       const int cnt = (int)m[a.R + 3];
       const float l0 = __uint_as_float(m[a.R]), l1 = __uint_as_float(m[a.R + 1]), l2 = __uint_as_float(m[a.R + 2]);
       float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll 4
-      for (int q = 0; q < cnt; ++q) {
-        const uint32_t jq = m[q];
-        if (jq < (uint32_t)nstage) Staged8<ST>::add(smean + jq * kFsCols + cs, acc2);
+      // kFsInflight gathers issued before their adds; indices read four at a time (a slot's meta
+      // words run to a multiple of 4 past R, so the reads stay in the slot; entries past cnt and
+      // indices outside the staged blocks add nothing)
+      for (int q0 = 0; q0 < cnt; q0 += kFsInflight) {
+        typename Staged8<ST>::V v[kFsInflight];
+#pragma unroll
+        for (int k = 0; k < kFsInflight; k += 4) {
+          const uint4 j4 = *(const uint4*)(m + q0 + k);
+          const uint32_t jj[4] = {j4.x, j4.y, j4.z, j4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            v[k + u] = q0 + k + u < cnt && jj[u] < (uint32_t)nstage ? Staged8<ST>::load(smean + jj[u] * kFsCols + cs)
+                                                                    : Staged8<ST>::zero();
+        }
+#pragma unroll
+        for (int k = 0; k < kFsInflight; ++k) Staged8<ST>::accum(v[k], acc2);
       }
       const float acc[8] = {acc2[0].x, acc2[0].y, acc2[1].x, acc2[1].y, acc2[2].x, acc2[2].y, acc2[3].x, acc2[3].y};
       const float4 xa = *(const float4*)xs, xb = *(const float4*)(xs + 4);

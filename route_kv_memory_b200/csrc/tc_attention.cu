@@ -59,13 +59,24 @@ struct Cfg {
 struct Work {
   int b, h, pair;
 };
-__device__ __forceinline__ Work work_item(int w, int B, int Hq, int npairs) {
+// Items run in chunks of `chunk` streams, a stream being one (sequence, KV group): chunk by
+// chunk, within a chunk the longest query-tile pairs first, and for one pair the chunk's streams
+// with their G query heads next to each other (the heads that share a K/V tile run together).  The
+// CTAs at work then share the K/V of a chunk's streams in L2 (one stream is 67 MB at 131072 keys)
+// instead of streaming every group's K/V from DRAM each round of items.  Rounds of items must still
+// span few pair lengths, which the static snake schedule needs for its balance; chunk = B * Hkv is
+// plain longest-first over all heads.
+__device__ __forceinline__ Work work_item(int w, int B, int Hq, int Hkv, int npairs, int chunk) {
   Work r;
-  const int per = B * Hq;
-  r.pair = npairs - 1 - w / per;  // longest rows first
-  const int rem = w % per;
-  r.h = rem % Hq;
-  r.b = rem / Hq;
+  const int G = Hq / Hkv, NS = B * Hkv;
+  const int k = w / (chunk * G * npairs);  // chunk (the last one may hold fewer streams)
+  const int cs = min(chunk, NS - k * chunk);
+  const int rem = w - k * chunk * G * npairs;
+  r.pair = npairs - 1 - rem / (cs * G);  // longest rows first
+  const int r2 = rem % (cs * G);
+  const int st = k * chunk + r2 / G;
+  r.b = st / Hkv;
+  r.h = (st % Hkv) * G + r2 % G;
   return r;
 }
 
@@ -187,7 +198,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       n0 = (a.g_pinfo[w / a.Hkv] >> 30) & 1 ? mt : 0;
       n1 = mt;
     } else {
-      const Work it = work_item(w, a.B, a.Hq, npairs);
+      const Work it = work_item(w, a.B, a.Hq, a.Hkv, npairs, a.chunk);
       n0 = 2 * it.pair + 1;
       n1 = 2 * it.pair + 2;
     }
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
         if (w < 0) break;
         const int wi = rr;  // items this CTA has started before this one
-        const Work it = work_item(w, a.B, a.Hq, npairs);
+        const Work it = work_item(w, a.B, a.Hq, a.Hkv, npairs, a.chunk);
         const int g = it.h / G;
         bool qok = true;
         for (int t = 0; t < 2; ++t) {  // each tile as soon as the previous item's last S_t has read it
@@ -474,7 +485,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         row_lim = row >= 0 && row / a.blk == it.j ? row : kNoMask;  // the block's own tokens only
         masked = __any_sync(0xffffffffu, row_lim != kNoMask);
       } else {
-        const Work it = work_item(w, a.B, a.Hq, npairs);
+        const Work it = work_item(w, a.B, a.Hq, a.Hkv, npairs, a.chunk);
         const int qt = 2 * it.pair + t;
         b = it.b;
         h = it.h;
@@ -702,9 +713,23 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
   const int nqt = (a.S + tca::BQ - 1) / tca::BQ;
   const int nwork = a.B * a.Hq * ((nqt + 1) / 2);
   const int grid = ga ? sms : (nwork < sms ? nwork : sms);
+  // causal mode: streams per chunk of the work order.  When the K/V of all streams about fits in
+  // L2 (at most 1.5x its size), one chunk of all streams; otherwise the fewest streams for which
+  // one round of `grid` items spans at most an eighth of the pair lengths.  Measured at 1 x 131072
+  // (8 streams of 67 MB): 1 stream per chunk, 12 GB of DRAM reads per launch against 174 GB for a
+  // single chunk, and 4.7% less time; at 2 x 32768 (134 MB of K/V) the single chunk is 1% faster.
+  AttnArgs c = a;
+  if (!ga) {
+    const int G = a.Hq / a.Hkv, NS = a.B * a.Hkv, npairs = (nqt + 1) / 2;
+    int l2 = 0;
+    cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
+    const double kv_bytes = 2.0 * NS * (double)a.S * a.dh * 2;  // K and V, bf16
+    const int want = (8 * grid + G * npairs - 1) / (G * npairs);
+    c.chunk = kv_bytes <= 1.5 * l2 ? NS : (want < 1 ? 1 : (want > NS ? NS : want));
+  }
   if (a.dh == 128)
-    return ga ? launch_attn<128, 1>(tq, tk, tv, a, status, grid, s) : launch_attn<128, 0>(tq, tk, tv, a, status, grid, s);
-  return ga ? launch_attn<64, 1>(tq, tk, tv, a, status, grid, s) : launch_attn<64, 0>(tq, tk, tv, a, status, grid, s);
+    return ga ? launch_attn<128, 1>(tq, tk, tv, c, status, grid, s) : launch_attn<128, 0>(tq, tk, tv, c, status, grid, s);
+  return ga ? launch_attn<64, 1>(tq, tk, tv, c, status, grid, s) : launch_attn<64, 0>(tq, tk, tv, c, status, grid, s);
 }
 
 }  // namespace mka
