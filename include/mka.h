@@ -230,10 +230,10 @@ MKA_API int mka_prefill_backward(const mka_config* cfg, const void* packed, cons
  * nothing.  ws: mka_decode_workspace_size(cfg, max_positions) bytes.
  * A step whose bounded device-side wait ran out records MKA_ERR_DEVICE_TIMEOUT and
  * may have applied part of its update: the state's position, cache row and memories
- * are then unspecified, and the out row too, and so is the step's grid barrier (an
- * arrival count in the state).  Refill the state with mka_prefill_forward (a prefill
- * into a state redefines all of it, the barrier included) or mka_state_init before
- * decoding on. */
+ * are then unspecified, and the out row too, and so are the step's grid barrier and
+ * completion counts (arrival counts in the state).  Refill the state with
+ * mka_prefill_forward (a prefill into a state redefines all of it, the counts
+ * included) or mka_state_init before decoding on. */
 MKA_API int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size_t state_bytes,
                     int32_t max_positions, const void* x_new, void* out, void* ws, size_t ws_bytes, void* stream);
 
@@ -298,7 +298,7 @@ MKA_API int mka_selftest_wait_timeout(int limit_us, int* result, void* stream);
 
 /* Wait classes of mka_set_wait_limit. */
 #define MKA_WAIT_PIPELINE 1 /* mbarrier waits of the TMA / tensor-core pipelines (GEMM, attention) */
-#define MKA_WAIT_GRID 2     /* grid barriers of the cooperative bf16 decode step */
+#define MKA_WAIT_GRID 2     /* grid barrier and completion-count waits of the cooperative bf16 decode step */
 
 /* Testing aid (not part of the layer; the paper has no counterpart): replaces the
  * built-in limit (2 s) of every bounded device-side wait of the classes in the mask

@@ -215,7 +215,7 @@ StateLayout state_layout(const Dims& d, int Lmax) {
   s.maxblk = Lmax / d.blk;
   size_t o = 0, B = d.B;
   s.pos = o; o += al(B * 4);
-  s.sync = o; o += al(8);
+  s.sync = o; o += al(8 * decode_sync_words(d.B, d.Hkv));
   s.kc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.vc = o; o += al(B * Lmax * d.dkv * d.elem);
   s.ema = o; o += al(B * d.width * 4);
@@ -636,8 +636,8 @@ static int prefill_forward(const mka_config* cfg, const void* packed, const void
   // blocks this prefill does not finish start at zero, so a prefill redefines the whole state.
   if (state && SL.maxblk > d.nblk)
     CUDA_TRY(cudaMemset2DAsync(scode + d.nblk, (size_t)SL.maxblk * 4, 0, (size_t)(SL.maxblk - d.nblk) * 4, d.B, s));
-  // and the decode step's grid barrier starts from zero arrivals
-  if (state) CUDA_TRY(cudaMemsetAsync(P(state, SL.sync), 0, 8, s));
+  // and the decode step's grid barrier and completion counts start from zero
+  if (state) CUDA_TRY(cudaMemsetAsync(P(state, SL.sync), 0, 8 * decode_sync_words(d.B, d.Hkv), s));
   std::unique_lock<std::mutex> aux_lock(aux_mutex(), std::defer_lock);
   AuxStreams* ax = nullptr;
   if (!g_prof.on) {

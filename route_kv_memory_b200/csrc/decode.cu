@@ -785,7 +785,7 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ bool grid_sync(unsigned long long* count, unsigned nblocks, int* status) {
+__device__ bool grid_sync(unsigned long long* count, unsigned nblocks, int* status, unsigned long long* index = nullptr) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -793,6 +793,7 @@ __device__ bool grid_sync(unsigned long long* count, unsigned nblocks, int* stat
     __threadfence();
     const unsigned long long arrival = atomicAdd(count, 1ull);
     const unsigned long long target = (arrival / nblocks + 1) * nblocks;
+    if (index) *index = arrival / nblocks;  // barriers since the count was zeroed
     if (ld_acquire_u64(count) < target) {
       const unsigned long long t0 = sm100::globaltimer();
       const unsigned long long lim = wait_limit(status, kWaitGrid, sm100::kWaitLimitNs);
@@ -809,6 +810,36 @@ __device__ bool grid_sync(unsigned long long* count, unsigned nblocks, int* stat
   }
   __syncthreads();
   return s_ok != 0;
+}
+
+// Thread 0 waits until *count reaches target (acquire), then the CTA goes on; false (status set) if
+// the wait ran out.
+__device__ bool wait_count(const unsigned long long* count, unsigned long long target, int* status) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_ok = 1;
+    if (ld_acquire_u64(count) < target) {
+      const unsigned long long t0 = sm100::globaltimer();
+      const unsigned long long lim = wait_limit(status, kWaitGrid, sm100::kWaitLimitNs);
+      while (ld_acquire_u64(count) < target) {
+        if (sm100::globaltimer() - t0 > lim) {
+          set_status(status, kStatusTimeout);
+          s_ok = 0;
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+// All threads' writes so far, then one arrival on *count (release).
+__device__ __forceinline__ void count_done(unsigned long long* count) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) atomicAdd(count, 1ull);
 }
 
 __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -1123,7 +1154,11 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
     }
   }
   if (tok_pf) dk::cp_wait<0>();  // the prefetched values, visible to the CTA after the barrier
-  if (!grid_sync(a.sync, nblk, a.status)) return;
+  __shared__ unsigned long long s_step;  // index of this step since the counts were zeroed
+  if (!grid_sync(a.sync, nblk, a.status, &s_step)) return;
+  const unsigned long long step = s_step;
+  unsigned long long* att_done = a.sync + 1;            // [B][Hkv] units of split attention finished
+  unsigned long long* tok_done = a.sync + 1 + a.B * a.Hkv;  // [B] token-update CTAs finished
 
   // ---- B: split-KV attention over the old rows (units handed out from CTA ntok on), and the
   // token update, split over the first ntok CTAs
@@ -1132,6 +1167,7 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
     for (int u = ((int)blockIdx.x - ntok + (int)nblk) % (int)nblk; u < units; u += nblk) {
       const int split = u % a.nsplit, g = (u / a.nsplit) % a.Hkv, bi = u / (a.nsplit * a.Hkv);
       dk::attn_unit<DH>(a, split, g, bi, min(s_pos[bi], a.Lmax), a.y, a.Ntot, ring);
+      count_done(&att_done[bi * a.Hkv + g]);
     }
     if ((int)blockIdx.x < ntok) {
       __shared__ TokenDecision td;
@@ -1139,23 +1175,32 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
         const int pos = s_pos[bi];
         if (pos < 0 || pos >= a.Lmax) {
           if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, kStatusCapacity);
+          count_done(&tok_done[bi]);
           continue;
         }
         const int c0 = min(width, (int)blockIdx.x * cpc), c1 = min(width, c0 + cpc);
         const int i0 = min(a.d, (int)blockIdx.x * dpc), i1 = min(a.d, i0 + dpc);
         token_decide<bf16>(a, bi, pos, &td, tok_pf ? &pf : nullptr);
         token_slice<bf16>(a, bi, pos, &td, c0, c1, i0, i1, tok_pf ? &pf : nullptr);
-        __syncthreads();
+        count_done(&tok_done[bi]);
       }
       if (blockIdx.x == 0 && threadIdx.x < a.B && s_pos[threadIdx.x] < a.Lmax)
         a.pos[threadIdx.x] = s_pos[threadIdx.x] + 1;
     }
   }
-  if (!grid_sync(a.sync, nblk, a.status)) return;
 
   // ---- C: merge, and finish a block completed by this token: its projected sum becomes
-  // the summary, its code the signs of the exact float64 d_model-space sum projected on P
-  for (int u = blockIdx.x; u < a.B * a.Hq; u += nblk) merge_unit<DH>(a, u / a.Hq, u % a.Hq, s_pos[u / a.Hq]);
+  // the summary, its code the signs of the exact float64 d_model-space sum projected on P.  No grid
+  // barrier: a CTA with work here waits only for the counts it needs (this step's split units of
+  // the head's KV group, and the sequence's token-update CTAs); the others leave.
+  const int ntok_run = ntok;
+  for (int u = blockIdx.x; u < a.B * a.Hq; u += nblk) {
+    const int bi = u / a.Hq, hq = u % a.Hq, g = hq / (a.Hq / a.Hkv);
+    if (!wait_count(&att_done[bi * a.Hkv + g], (step + 1) * (unsigned long long)a.nsplit, a.status) ||
+        !wait_count(&tok_done[bi], (step + 1) * (unsigned long long)ntok_run, a.status))
+      return;
+    merge_unit<DH>(a, bi, hq, s_pos[bi]);
+  }
   {
     const int width = 2 * a.dkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1165,9 +1210,14 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
       const int j = pos / a.blk;
       const float* bsum = a.blk_sum + (size_t)bi * width;
       float* summ = a.summ + ((size_t)bi * a.maxblk + j) * width;
-      for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < width; c += nblk * blockDim.x) summ[c] = bsum[c];
       // bit k on CTA (nblk - 1 - k), one warp per bit
       const int k = (int)nblk - 1 - (int)blockIdx.x;
+      // the block's sums are final once every token-update CTA of this step has finished
+      const bool copies = (int)blockIdx.x * (int)blockDim.x < width;
+      if ((copies || (k >= 0 && k < a.nb)) &&
+          !wait_count(&tok_done[bi], (step + 1) * (unsigned long long)ntok_run, a.status))
+        return;
+      for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < width; c += nblk * blockDim.x) summ[c] = bsum[c];
       if (k >= 0 && k < a.nb && warp == 0) {
         const double* bx = a.blk_x + (size_t)bi * a.d;
         double v = 0.0;

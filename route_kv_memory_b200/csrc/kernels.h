@@ -122,6 +122,12 @@ cudaError_t prefill_tail_state(const float* xkv, int ld, int width, const void* 
                                int blk, float* blk_sum, double* blk_x, int* pos, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
+// 64-bit words of the decode step's synchronisation area in the state: the grid barrier's arrival
+// count, then per (sequence, KV group) the split-attention units finished, then per sequence the
+// token-update CTAs finished.  All of them only grow; a prefill with a state, or state_init, zeroes
+// them.
+inline size_t decode_sync_words(int B, int Hkv) { return 1 + (size_t)B * (Hkv + 1); }
+
 struct AttnArgs {
   const void* q; long long q_bstride; int q_ld;      // q[b][t][h*dh + i]: b*q_bstride + t*q_ld + h*dh + i
   const void* k; const void* v; long long kv_bstride; int kv_ld;  // k[b][j][g*dh + i]
