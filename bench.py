@@ -295,7 +295,7 @@ def measure_prefill(args, cfg, dev, world, steps, warmup, with_e2e=False, with_c
     if clk:
         res["clocks"] = clocks
     if with_e2e:
-        res["e2e"] = measure_e2e(layer, inp, cfg, x, out, flush, world, max(4, steps // 4))
+        res["e2e"] = measure_e2e(layer, inp, cfg, x, out, flush, world, max(4, steps))
     res["_recall_gpu"] = None
     if getattr(args, "recall_check", True) and cfg.tiers & 4 and cfg.attention_paths == 1:
         idx = torch.empty(cfg.batch, cfg.seq, cfg.recall_r, dtype=torch.int32, device=dev)

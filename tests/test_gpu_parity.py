@@ -411,6 +411,49 @@ def test_decode_bf16_small():
     check_out(got, ref["O"], "bf16")
 
 
+def test_decode_bf16_from_empty_state():
+    """The fused bf16 step from position 0 of a fresh state (two sequences, blocks of 8): every step's
+    merge waits on completion counts that start at zero, and five blocks close on the way."""
+    cfg = small("decbf0", "bf16", batch=2, seq=40, d_head=128, n_q_heads=4, n_kv_heads=2, block=8, recall_r=3,
+                hash_bits=8, seed=64)
+    inp = make_inputs(cfg)
+    got = decode_run(cfg, inp, 0, cfg.seq, 48)
+    ref = oracle_prefill(cfg, inp, rows=np.arange(0, cfg.seq))
+    check_out(got, ref["O"], "bf16")
+
+
+def test_decode_capacity_bf16_fused(mka):
+    """The fused bf16 step on a full cache records MKA_ERR_CAPACITY and still returns: its attention
+    units and token-update CTAs are counted, so the merging CTAs' waits are met; a refill by prefill
+    then decodes on as before."""
+    cfg = small("capbf", "bf16", seq=64, d_head=128, block=16, hash_bits=8, seed=63)
+    inp = make_inputs(cfg, seq_total=66)
+    layer = mka.FastMKALayer(cfg, gpu_weights(inp))
+    x = inp.x.cuda()
+    state = layer.new_state(64)
+    out = torch.empty(1, 64, cfg.dq, dtype=x.dtype, device="cuda")
+    layer.prefill(x[:, :64].contiguous(), out, state=state, max_positions=64)
+    for t in (64, 65):
+        o = torch.empty(1, cfg.dq, dtype=x.dtype, device="cuda")
+        layer.decode(state, 64, x[:, t].contiguous(), o)
+        torch.cuda.synchronize()
+        assert mka.mka_status() == mka.MKA_ERR_CAPACITY
+    assert mka.mka_status() == 0
+    # refill 48 rows into a state of 64 positions, decode 16 and check them
+    layer48 = mka.FastMKALayer(cfg.replace(seq=48), gpu_weights(inp))
+    out48 = torch.empty(1, 48, cfg.dq, dtype=x.dtype, device="cuda")
+    layer48.prefill(x[:, :48].contiguous(), out48, state=state, max_positions=64)
+    outs = []
+    for t in range(48, 64):
+        o = torch.empty(1, cfg.dq, dtype=x.dtype, device="cuda")
+        layer48.decode(state, 64, x[:, t].contiguous(), o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert mka.mka_status() == 0
+    ref = oracle_prefill(cfg, inp, rows=np.arange(48, 64))
+    check_out(torch.stack(outs, 1), ref["O"], "bf16")
+
+
 def test_decode_qwen_shape_4k():
     """Qwen decode shapes (28/4 heads, d 3584, block 256, R 8): 4096-token prefix, 24 decoded tokens."""
     cfg = CONFIGS["qwen7b_decode"].replace(seq=4096 + 24, decode_new=0)
