@@ -835,11 +835,14 @@ __device__ bool wait_count(const unsigned long long* count, unsigned long long t
   __syncthreads();
   return s_ok != 0;
 }
-// All threads' writes so far, then one arrival on *count (release).
+// One arrival on *count once all of the CTA's writes so far are visible (the barrier orders them
+// before thread 0's fence, as in grid_sync).
 __device__ __forceinline__ void count_done(unsigned long long* count) {
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) atomicAdd(count, 1ull);
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(count, 1ull);
+  }
 }
 
 __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
