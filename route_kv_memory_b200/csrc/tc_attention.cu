@@ -303,6 +303,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      // L2: a query tile is read by this item only, while the K/V of the chunk's streams are read
+      // by every item of the chunk: the Q tiles (and the O rows) must not age the K/V out of L2
+      const uint64_t pol_once = policy_evict_first(), pol_kv = policy_evict_last();
       int kvit = 0;
       for (int rr = 0; rr * (int)gridDim.x < nwork; ++rr) {
         const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
@@ -319,7 +322,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_expect_tx(&q_full[t], C::Q_BYTES);
           const int qy = (int)(it.b * q_rows_per_b) + (2 * it.pair + t) * BQ;
           for (int hb = 0; hb < NH; ++hb)
-            tma_load_2d(sQ + t * C::Q_BYTES + hb * C::HALF, &tmQ, &q_full[t], it.h * DH + hb * 64, qy);
+            tma_load_2d_hint(sQ + t * C::Q_BYTES + hb * C::HALF, &tmQ, &q_full[t], it.h * DH + hb * 64, qy, pol_once);
         }
         if (!qok) break;
         const int nkv = 2 * it.pair + 2;
@@ -334,8 +337,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint8_t* kdst = sKV + st * C::KV_BYTES;
           const int ky = (int)(it.b * kv_rows_per_b) + j * BKV;
           for (int hb = 0; hb < NH; ++hb) {
-            tma_load_2d(kdst + hb * C::HALF, &tmK, &kv_full[st], g * DH + hb * 64, ky);
-            tma_load_2d(kdst + C::K_BYTES + hb * C::HALF, &tmV, &kv_full[st], g * DH + hb * 64, ky);
+            tma_load_2d_hint(kdst + hb * C::HALF, &tmK, &kv_full[st], g * DH + hb * 64, ky, pol_kv);
+            tma_load_2d_hint(kdst + C::K_BYTES + hb * C::HALF, &tmV, &kv_full[st], g * DH + hb * 64, ky, pol_kv);
           }
         }
         if (!ok) break;
@@ -464,6 +467,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const float sl2 = a.scale * 1.4426950408889634f;
     // causal output rows start on 32-byte boundaries: one 32-byte store per 16 columns
     const bool o32 = !GA && ((uintptr_t)a.o & 31) == 0 && a.o_ld % 16 == 0 && a.o_bstride % 16 == 0;
+    const uint64_t pol_out = policy_evict_first();  // output rows: written once, not read here
     int sit = 0;
     for (int rr = 0; rr * (int)gridDim.x < nwork; ++rr) {
       const int w = snake_item(rr, gridDim.x, blockIdx.x, nwork);
@@ -640,8 +644,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                                         __uint_as_float(ov[v >> 1][(v & 1) * 16 + 2 * e + 1]) * inv);
               wv[e] = *(uint32_t*)&hb;
             }
-            if (GA || o32) {
+            if (GA) {
               st_global_v8(orow + c + v * 16, wv);
+            } else if (o32) {
+              st_global_v8_hint(orow + c + v * 16, wv, pol_out);
             } else {
               *(uint4*)(orow + c + v * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
               *(uint4*)(orow + c + v * 16 + 8) = make_uint4(wv[4], wv[5], wv[6], wv[7]);
