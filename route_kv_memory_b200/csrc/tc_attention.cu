@@ -719,11 +719,12 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
   const int nqt = (a.S + tca::BQ - 1) / tca::BQ;
   const int nwork = a.B * a.Hq * ((nqt + 1) / 2);
   const int grid = ga ? sms : (nwork < sms ? nwork : sms);
-  // causal mode: streams per chunk of the work order.  When the K/V of all streams about fits in
-  // L2 (at most 1.5x its size), one chunk of all streams; otherwise the fewest streams for which
-  // one round of `grid` items spans at most an eighth of the pair lengths.  Measured at 1 x 131072
-  // (8 streams of 67 MB): 1 stream per chunk, 12 GB of DRAM reads per launch against 174 GB for a
-  // single chunk, and 4.7% less time; at 2 x 32768 (134 MB of K/V) the single chunk is 1% faster.
+  // causal mode: streams per chunk of the work order.  When the K/V of all streams fits in half of
+  // L2, one chunk of all streams; otherwise the fewest streams for which one round of `grid` items
+  // spans at most an eighth of the pair lengths.  Measured (with Q and O evict-first, K/V
+  // evict-last): at 1 x 131072 (8 streams of 67 MB) 1 stream per chunk reads 8.9 GB per launch
+  // from DRAM, where a single chunk read 174 GB; at 2 x 32768 (134 MB of K/V) chunks of 2 streams
+  // take 14.08 ms against 14.45 ms for a single chunk.
   AttnArgs c = a;
   if (!ga) {
     const int G = a.Hq / a.Hkv, NS = a.B * a.Hkv, npairs = (nqt + 1) / 2;
@@ -731,7 +732,7 @@ cudaError_t attention_prefill_tc(const AttnArgs& a, int* status, cudaStream_t s)
     cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
     const double kv_bytes = 2.0 * NS * (double)a.S * a.dh * 2;  // K and V, bf16
     const int want = (8 * grid + G * npairs - 1) / (G * npairs);
-    c.chunk = kv_bytes <= 1.5 * l2 ? NS : (want < 1 ? 1 : (want > NS ? NS : want));
+    c.chunk = kv_bytes <= 0.5 * l2 ? NS : (want < 1 ? 1 : (want > NS ? NS : want));
   }
   if (a.dh == 128)
     return ga ? launch_attn<128, 1>(tq, tk, tv, c, status, grid, s) : launch_attn<128, 0>(tq, tk, tv, c, status, grid, s);
