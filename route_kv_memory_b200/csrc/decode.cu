@@ -1,6 +1,7 @@
 // One FastMKA decode step (MKA paper, paper-notes page §1-§3: the cache holds
 // the fused routed K/V, so a step appends one fused row and runs one attention
-// path over the cache).  Four launches:
+// path over the cache).  bf16 layers run it as one cooperative launch (the fused
+// step below); float32 layers as four launches:
 //   1. gemv      y = x_new [W_q | W_k | W_v | W_q W_r1 | P]          (HBM: weights)
 //   2. token     router, L3 recall, fuse, K/V append, EMA / block update (one CTA per sequence)
 //   3. split-KV  attention partials over cache[0..pos]                 (HBM: cache)
@@ -756,20 +757,23 @@ __device__ void token_slice(const DecodeArgs& a, const int bi, const int pos, co
 
 // ---------------------------------------------------------------- fused decode step (bf16)
 // One cooperative launch, two CTAs per SM, NWD warps each:
-//   A  the projection row y = x_new [W_q | W_k | W_v | W_q W_r1 | P] for every sequence:
-//      each CTA streams its share of the packed weight rows (TMA bulk copies into a
-//      2-stage shared-memory ring) and forms the dot products from shared memory
+//   A  the projection row y = x_new [W_q | W_k | W_v | W_q W_r1 | P] for every sequence.
+//      Batch 1: every warp streams two packed weight rows at a time through registers, while
+//      the token CTAs copy their state slices into shared memory (cp.async); larger batches
+//      stream each CTA's rows through a 2-stage shared-memory ring of TMA bulk copies
 //   -- grid barrier --
-//   B  CTA b < B: the token update of sequence b (router, L3 recall, fuse, append the
-//      fused K/V row at position pos, EMA / block update, pos + 1); every other CTA:
-//      split-KV attention of the new queries over the old cache rows [0, pos)
-//   -- grid barrier --
-//   C  per (sequence, query head): merge the split partials and the new row's own
-//      term (its score against the appended K row, weight on the appended V row)
-// The two barriers share one arrival count in the decode state, each wait bounded by a
-// time limit that records MKA_ERR_DEVICE_TIMEOUT.  All CTAs are co-resident (cooperative
-// launch), so the barrier cannot deadlock on scheduling.  A CTA whose wait ran out leaves
-// the step.
+//   B  the first ntok CTAs: the token update of each sequence (router, L3 recall, fuse, append
+//      the fused K/V row at position pos, EMA / block update, pos + 1), split over their column
+//      slices; every CTA (from CTA ntok on): split-KV attention of the new queries over the old
+//      cache rows [0, pos).  Each attention unit and each token CTA then adds one to a
+//      completion count in the state (per (sequence, KV group) and per sequence)
+//   C  per (sequence, query head), on the CTAs that have one, once this step's counts are in:
+//      merge the split partials and the new row's own term (its score against the appended K
+//      row, weight on the appended V row); a block closed by this token gets its summary and
+//      code.  The other CTAs leave without waiting.
+// The grid barrier and the counts live in the decode state and only grow; every wait is bounded
+// by a time limit that records MKA_ERR_DEVICE_TIMEOUT.  All CTAs are co-resident (cooperative
+// launch), so no wait can deadlock on scheduling.  A CTA whose wait ran out leaves the step.
 // the token CTAs' prefetch area (batch 1): block codes, EMA and block-sum slices, d_model slices
 constexpr int kPfCodes = 2048, kPfCols = 256, kPfD = 128;
 constexpr size_t kPfBytes = (size_t)kPfCodes * 4 + 2 * kPfCols * 4 + kPfD * (8 + 2);
