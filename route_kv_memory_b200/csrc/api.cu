@@ -242,7 +242,7 @@ int decode_nsplit(const Dims& d, int Lmax) {
 
 struct DecodeWs {
   int nsplit;
-  size_t y, qf, part, total;
+  size_t y, y2, qf, part, total;
 };
 DecodeWs decode_ws(const Dims& d, int Lmax) {
   DecodeWs w;
@@ -250,6 +250,7 @@ DecodeWs decode_ws(const Dims& d, int Lmax) {
   w.nsplit = decode_nsplit(d, Lmax);
   size_t o = 0, B = d.B;
   w.y = o; o += al(B * p.Ntot * 4);
+  w.y2 = o; o += al(B * p.Ntot * 4);
   w.qf = o; o += al(B * d.dq * 4);
   w.part = o; o += al(B * d.Hq * (size_t)w.nsplit * (d.dh + 4) * 4);  // records of part_rec(dh) floats
   w.total = o;
@@ -997,7 +998,7 @@ int mka_decode_step(const mka_config* cfg, const void* packed, void* state, size
   a.pos = (int*)P(state, SL.pos); a.kcache = P(state, SL.kc); a.vcache = P(state, SL.vc);
   a.ema = (float*)P(state, SL.ema); a.blk_sum = (float*)P(state, SL.blk_sum); a.blk_x = (double*)P(state, SL.blk_x);
   a.summ = (float*)P(state, SL.summ); a.scode = (uint32_t*)P(state, SL.scode);
-  a.y = (float*)P(ws, W.y); a.qf = (float*)P(ws, W.qf); a.part = (float*)P(ws, W.part); a.nsplit = W.nsplit;
+  a.y = (float*)P(ws, W.y); a.y2 = (float*)P(ws, W.y2); a.qf = (float*)P(ws, W.qf); a.part = (float*)P(ws, W.part); a.nsplit = W.nsplit;
   a.sync = (unsigned long long*)P(state, SL.sync);
   a.status = status_ptr();
   prof_begin();

@@ -601,6 +601,20 @@ __global__ void decode_merge_kernel(DecodeArgs a) {
 // ---------------------------------------------------------------- token update, parallel form
 // Per-token decisions, recomputed by every CTA of the fused launch (deterministic, cheap):
 // lambda (router), the code of x_new (exact sign decisions), and the recalled blocks.
+// Batch-1 GEMV of the fused step: every warp of the grid (TW of them) takes the same number of
+// whole rows, q0 = Ntot / TW; the rem leftover rows at the end are split into halves of d / 2,
+// dealt one per warp round-robin over the CTAs, so every SM streams about the same bytes (a warp
+// with one more whole row than the others held its CTA's SM ~30% longer).  First halves go to y,
+// second halves to y2.  Only when the leftover rows lie past the query and K/V rows (the router
+// and hash rows, which only the token update reads and which it sums from both), when there are
+// enough warps, and when d / 2 is a whole number of 16-byte vectors per lane.  The returned first
+// split row is Ntot when rows are not split.
+__device__ __forceinline__ int gemv_split_row(const DecodeArgs& a, int TW) {
+  const int q0 = a.Ntot / TW, rem = a.Ntot - q0 * TW;
+  const bool on = a.B == 1 && a.y2 && rem > 0 && 2 * rem <= TW && q0 * TW >= a.dq + 2 * a.dkv && a.d % 512 == 0;
+  return on ? q0 * TW : a.Ntot;
+}
+
 struct TokenDecision {
   float lam[3];
   int cnt;
@@ -620,20 +634,22 @@ struct TokenPrefetch {
 
 template <typename T>
 __device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, TokenDecision* td,
-                             const TokenPrefetch* pf = nullptr) {
+                             const TokenPrefetch* pf, const int split_row) {
   __shared__ float s_red[32][3];
   __shared__ unsigned s_code;
   __shared__ int s_base[34], s_run[34];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   const float* y = a.y + (size_t)bi * a.Ntot;
-  const float* h = y + a.dq + 2 * a.dkv;
-  const float* p = h + a.rh * a.rh_segs;
+  const float* y2 = a.y2 + (size_t)bi * a.Ntot;
+  const int hrow = a.dq + 2 * a.dkv, prow = hrow + a.rh * a.rh_segs;
+  // row r of the projection: y[r], plus its second half for the rows the GEMV split
+  auto yr = [&](int r) { return r >= split_row ? y[r] + y2[r - split_row] : y[r]; };
   const T* xn = (const T*)a.x_new + (size_t)bi * a.d;
   float z0 = 0.f, z1 = 0.f, z2 = 0.f;
   for (int j = tid; j < a.rh; j += blockDim.x) {
     float hv;
-    if (a.r_inter) hv = h[(j >> 7) * 256 + (j & 127)] + h[(j >> 7) * 256 + 128 + (j & 127)];
-    else hv = a.rh_segs == 2 ? h[j] + h[a.rh + j] : h[j];
+    if (a.r_inter) hv = yr(hrow + (j >> 7) * 256 + (j & 127)) + yr(hrow + (j >> 7) * 256 + 128 + (j & 127));
+    else hv = a.rh_segs == 2 ? yr(hrow + j) + yr(hrow + a.rh + j) : yr(hrow + j);
     const float gv = gelu_erf(hv);
     z0 = fmaf(gv, a.w_r2[j * 3], z0);
     z1 = fmaf(gv, a.w_r2[j * 3 + 1], z1);
@@ -648,7 +664,7 @@ __device__ void token_decide(const DecodeArgs& a, const int bi, const int pos, T
     s_red[warp][2] = z2;
   }
   if (warp == 0) {  // code of x_new, same decision rule as the prefill path
-    const float pv = lane < a.nb ? p[lane] : 0.f;
+    const float pv = lane < a.nb ? yr(prow + lane) : 0.f;
     const float rms = sqrtf(warp_sum(pv * pv) / (float)a.nb);
     const float e = (float)a.d * 0x1p-21f * rms;
     bool bit = pv > 0.f;
@@ -991,6 +1007,8 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
   // batch 1 with d_model a multiple of 256 up to 4096: phase A streams the weight rows through
   // registers (no shared-memory ring, no set-up barrier)
   const bool reg_gemv = a.B == 1 && (a.d & 255) == 0 && a.d <= 4096;
+  // rows from split_row on go to the GEMV as halves (batch 1, see gemv_split_row)
+  const int split_row = reg_gemv ? gemv_split_row(a, (int)nblk * NW) : a.Ntot;
   if (!reg_gemv) {
     if (tid == 0) {
       sm100::mbar_init(&gbar[0], 1);
@@ -1042,9 +1060,9 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
     const size_t rowv = (size_t)a.d / 8;
     const uint4* xv = (const uint4*)a.x_new;  // read through L1: every warp reads the same 16 B pieces
     const uint64_t pol_w = dk::l2_evict_last();
-    for (int r = gw; r < a.Ntot; r += 2 * TW) {
+    for (int r = gw; r < split_row; r += 2 * TW) {
       const int r2 = r + TW;
-      const bool two = r2 < a.Ntot;
+      const bool two = r2 < split_row;
       uint4 w1[16], w2[16];
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
@@ -1080,6 +1098,38 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
       if (lane == 0) {
         a.y[r] = v1;
         if (two) a.y[r2] = v2;
+      }
+    }
+    // half-row hi of the split rows: warp (CTA c, warp wi) takes hi = wi * nblk + c
+    const int hi = warp * (int)nblk + (int)blockIdx.x;
+    if (hi < 2 * (a.Ntot - split_row)) {
+      const int row = split_row + (hi >> 1), half = hi & 1;
+      const int hv = a.d / 512;            // 16-byte vectors per lane in half a row
+      const size_t off = (size_t)half * (rowv / 2);
+      uint4 w1[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (k < hv) w1[k] = dk::ldg_nc_hint(W + (size_t)row * rowv + off + lane + 32 * k, pol_w);
+      float a1[2] = {0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < hv) {
+          const uint4 xu = __ldg(xv + off + lane + 32 * k);
+          const __nv_bfloat162* xh = (const __nv_bfloat162*)&xu;
+          const __nv_bfloat162* h1 = (const __nv_bfloat162*)&w1[k];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 xf = __bfloat1622float2(xh[e]);
+            const float2 f1 = __bfloat1622float2(h1[e]);
+            a1[k & 1] = fmaf(f1.x, xf.x, a1[k & 1]);
+            a1[k & 1] = fmaf(f1.y, xf.y, a1[k & 1]);
+          }
+        }
+      }
+      const float v1 = warp_sum(a1[0] + a1[1]);
+      if (lane == 0) {
+        if (half) a.y2[row - split_row] = v1;
+        else a.y[row] = v1;
       }
     }
   } else {
@@ -1187,7 +1237,7 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
         }
         const int c0 = min(width, (int)blockIdx.x * cpc), c1 = min(width, c0 + cpc);
         const int i0 = min(a.d, (int)blockIdx.x * dpc), i1 = min(a.d, i0 + dpc);
-        token_decide<bf16>(a, bi, pos, &td, tok_pf ? &pf : nullptr);
+        token_decide<bf16>(a, bi, pos, &td, tok_pf ? &pf : nullptr, split_row);
         token_slice<bf16>(a, bi, pos, &td, c0, c1, i0, i1, tok_pf ? &pf : nullptr);
         count_done(&tok_done[bi]);
       }

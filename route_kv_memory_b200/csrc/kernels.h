@@ -246,6 +246,7 @@ struct DecodeArgs {
   float* summ; uint32_t* scode;
   // scratch
   float* y;                      // [B, Ntot] projection row
+  float* y2 = nullptr;           // [B, Ntot] second halves of the rows the batch-1 GEMV splits (gemv_split_row on)
   float* qf;                     // [B, dq] float32 query
   float* part;                   // split-KV partials
   int nsplit;
