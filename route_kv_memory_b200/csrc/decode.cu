@@ -914,7 +914,11 @@ constexpr int kMergeBatch = 16;  // splits whose o a warp holds in registers at 
 // kMergeBatch splits' o); the splits are shared out over the warps (16-byte loads of o), then
 // summed over the warps in a fixed order: deterministic.
 template <int DH>
-__device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, const int pos_old) {
+// The split partials are final when this runs; the new row's own term (its K and V rows, written
+// by the token-update CTAs) is read only after *tok_count reaches tok_target, so the partials'
+// loads fly while the token update finishes.  False if that wait ran out.
+__device__ bool merge_unit(const DecodeArgs& a, const int bi, const int hq, const int pos_old,
+                           const unsigned long long* tok_count, unsigned long long tok_target) {
   __shared__ float s_w[kMaxSplits];
   __shared__ float red[32];
   __shared__ float2 red2[32];
@@ -927,10 +931,6 @@ __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, cons
   const bf16* kn = (const bf16*)a.kcache + ((size_t)bi * a.Lmax + pos_old) * a.dkv + (size_t)g * DH;
   const bf16* vn = (const bf16*)a.vcache + ((size_t)bi * a.Lmax + pos_old) * a.dkv + (size_t)g * DH;
   const float* q = a.y + (size_t)bi * a.Ntot + (size_t)hq * DH;
-  float s = 0.f;
-  if (has_new)
-    for (int c = tid; c < DH; c += blockDim.x)
-      s = fmaf(__bfloat162float(__float2bfloat16_rn(__ldcg(q + c))), __bfloat162float(kn[c]), s);
   float mloc = -INFINITY, lfirst = 0.f;
   for (int sp = tid; sp < a.nsplit; sp += blockDim.x) {
     const float m = __ldcg(pr + (size_t)sp * rec + DH);
@@ -945,6 +945,15 @@ __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, cons
     const int sp = warp + i * dk::NWD;
     ov[i] = olane && sp < a.nsplit ? __ldcg((const float4*)(pr + (size_t)sp * rec) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  if (!wait_count(tok_count, tok_target, a.status)) return false;
+  float s = 0.f;
+  if (has_new)
+    for (int c = tid; c < DH; c += blockDim.x)
+      s = fmaf(__bfloat162float(__float2bfloat16_rn(__ldcg(q + c))), __bfloat162float(__ldcg(kn + c)), s);
+  float vnew[4] = {0.f, 0.f, 0.f, 0.f};  // this thread's columns of the appended V row
+  if (has_new && tid < DH / 4)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) vnew[e] = __bfloat162float(__ldcg(vn + 4 * tid + e));
   const float2 sm = block_reduce_sum_max(s, mloc, red2);
   const float snew = sm.x * a.scale * 1.4426950408889634f;
   const float M = has_new ? fmaxf(sm.y, snew) : sm.y;
@@ -985,11 +994,12 @@ __device__ void merge_unit(const DecodeArgs& a, const int bi, const int hq, cons
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int c = 4 * tid + e;
-      if (has_new) o[e] = fmaf(wn, __bfloat162float(vn[c]), o[e]);
+      if (has_new) o[e] = fmaf(wn, vnew[e], o[e]);
       ((bf16*)a.out)[(size_t)bi * a.dq + (size_t)hq * DH + c] = __float2bfloat16_rn(o[e] * inv);
     }
   }
   __syncthreads();
+  return true;
 }
 
 template <int DH>
@@ -1254,9 +1264,8 @@ __device__ __forceinline__ void decode_fused_body(const DecodeArgs& a) {
   for (int u = blockIdx.x; u < a.B * a.Hq; u += nblk) {
     const int bi = u / a.Hq, hq = u % a.Hq, g = hq / (a.Hq / a.Hkv);
     if (!wait_count(&att_done[bi * a.Hkv + g], (step + 1) * (unsigned long long)a.nsplit, a.status) ||
-        !wait_count(&tok_done[bi], (step + 1) * (unsigned long long)ntok_run, a.status))
+        !merge_unit<DH>(a, bi, hq, s_pos[bi], &tok_done[bi], (step + 1) * (unsigned long long)ntok_run))
       return;
-    merge_unit<DH>(a, bi, hq, s_pos[bi]);
   }
   {
     const int width = 2 * a.dkv;
